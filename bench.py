@@ -1,0 +1,368 @@
+"""Benchmark of the MoE-layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--impl ours|reference]
+
+One step is one moe_forward over one batch of the workload (router GEMM,
+top-k + gates, dispatch layout with the deduplicated send layout, permute,
+grouped SwiGLU GEMMs, combine).  Default workload: configuration 2 of the
+MoE layer set (T=16384 tokens, d=256, E=64 SwiGLU experts of width 64,
+top-4, bf16, EP=8 contiguous), the fine-grained expert layer.
+
+Timing: inputs resident in HBM; L2 is flushed (a 256 MB write) before each
+step, outside the step's CUDA events; the K steps sit between a barrier and
+a device synchronisation on both sides; with N > 1 ranks (torchrun, one per
+GPU) each rank runs its own replica of the workload on its own tokens (the
+layer shards by tokens with no exchange), and the slowest rank's time
+counts.  Prints one JSON line on rank 0.
+
+`--impl reference` times the CPU oracle (the only reference this method
+has) on a bounded sample of the same workload, on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import routing_dispatch_experts_b200 as moe  # noqa: E402
+from routing_dispatch_experts_b200 import workloads as W  # noqa: E402
+
+METRIC = "MoE-layer fwd routed tokens/s"
+L2_FLUSH_BYTES = 256 << 20
+MEASURED_PEAKS = os.path.join(ROOT, "MEASURED_PEAKS.json")
+
+
+def peaks():
+    try:
+        p = json.load(open(MEASURED_PEAKS))
+        return dict(hbm=p["hbm_gbs"], bf16=p["bf16_tflops"], bf16_sus=p["bf16_tflops_sustained"],
+                    src="measured")
+    except Exception:
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+# ------------------------------------------------------------ algorithmic work
+def work(w: W.Workload, T: int):
+    """Algorithmic bytes / FLOPs of each call for T tokens (what the method
+    must move or compute, not what a particular kernel happens to move)."""
+    b = 2 if w.dtype == "bf16" else 4
+    R = T * w.k
+    return {
+        "route": dict(bytes=T * w.d * b + w.E * w.d * b + 2 * T * w.E * 4 + 2 * R * 4,
+                      flops=2 * T * w.d * w.E),
+        "layout": dict(bytes=2 * R * 4 + 4 * R * 4, flops=0),
+        "permute": dict(bytes=T * w.d * b + R * w.d * b + R * 4, flops=0),
+        "grouped_swiglu": dict(bytes=R * w.d * b + 3 * w.E * w.d * w.f * b + 2 * R * w.f * b
+                               + R * w.d * b, flops=6 * R * w.d * w.f),
+        "combine": dict(bytes=R * w.d * b + T * w.d * b + 2 * R * 4, flops=0),
+    }
+
+
+# ------------------------------------------------------------------- helpers
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled in the background."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.p = None
+        self.out = []
+
+    def start(self):
+        try:
+            self.p = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return None
+        self.p.terminate()
+        try:
+            out, _ = self.p.communicate(timeout=5)
+        except Exception:
+            self.p.kill()
+            out = ""
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [v.strip() for v in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(n_gpus):
+    if n_gpus <= 1 and "RANK" not in os.environ:
+        return 0, 1, 0
+    import datetime
+    import torch.distributed as dist
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    torch.cuda.set_device(local)
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                            device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local):
+    w = W.WORKLOADS[args.config]
+    T = w.T
+    ep = w.eps[0]
+    seed = args.seed + rank  # every replica works on its own tokens
+    dev = torch.device("cuda", local)
+    x = W.make_x(w, seed, T)
+    wr = W.make_router(w, args.seed)
+    bias = W.make_bias(w, args.seed)
+    wg, wu, wd = W.make_experts(w, args.seed)
+    shape = moe.Shape(T=T, d=w.d, E=w.E, k=w.k, f=w.f, ep=ep, dtype=w.torch_dtype)
+    dx = x.to(dev)
+    dbias = None if bias is None else bias.to(dev)
+    packed = moe.pack_weights(shape, wr.to(dev), wg.to(dev), wu.to(dev), wd.to(dev))
+    del wg, wu, wd
+    ws = moe.workspace(shape, forward=True, device=dev)
+    buf = moe.ForwardBuffers(shape, device=dev)
+    y = torch.empty((T, w.d), dtype=w.torch_dtype, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    rmap = None if (w.placements[0] == "contiguous") else W.permutation_placement(w.E, ep, args.seed)
+
+    def step():
+        moe.forward(shape, dx, packed, dbias, ws, expert_rank=rmap, y=y, buffers=buf)
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    # warm-up (at least W steps, and long enough for the clock sampler to see load)
+    t_end = time.time() + 1.0
+    i = 0
+    while i < args.warmup or time.time() < t_end:
+        flush.fill_(i & 0xFF)
+        step()
+        i += 1
+        if i % 64 == 0:
+            torch.cuda.synchronize(dev)
+    torch.cuda.synchronize(dev)
+    moe.check_device_status(ws)
+
+    # ---- timed region: K steps, L2 flushed before each
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    ms = max_over_ranks(sum(step_ms) / len(step_ms), world)
+    moe.check_device_status(ws)
+
+    # ---- per-call breakdown (same stream, same flushing) -> dominant call
+    calls = {}
+    lay_ws = ws  # the forward workspace starts with the scratch the calls need
+
+    def t_call(name, fn, reps):
+        e = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+             for _ in range(reps)]
+        for i in range(reps):
+            flush.fill_(i & 0xFF)
+            e[i][0].record(stream)
+            fn()
+            e[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        calls[name] = sum(a.elapsed_time(b) for a, b in e) / reps
+
+    reps = max(args.steps, 20)
+    lg = buf.logits
+    t_call("route", lambda: moe.route(shape, dx, packed, dbias, lay_ws), reps)
+    idx = buf.topk_idx
+    t_call("layout", lambda: moe.dispatch_layout(shape, idx, lay_ws, expert_rank=rmap), reps)
+    rt = buf.layout["row_token"]
+    t_call("permute", lambda: moe.permute(shape, dx, rt), reps)
+    off = buf.layout["expert_offsets"]
+    xp = buf.x_perm
+    t_call("grouped_swiglu", lambda: moe.grouped_swiglu(shape, xp, off, packed, lay_ws), reps)
+    t_call("combine", lambda: moe.combine(shape, buf.y_perm, buf.layout["slot_row"], buf.topk_gate), reps)
+    moe.check_device_status(ws)
+    clk = clocks.stop()
+
+    # ---- end to end through the public API with host buffers
+    x_host = x.pin_memory()
+    y_host = torch.empty((T, w.d), dtype=w.torch_dtype).pin_memory()
+    e2e_ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    for _ in range(3):
+        dx.copy_(x_host, non_blocking=True)
+        step()
+        y_host.copy_(y, non_blocking=True)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e2e_ev[0].record(stream)
+    for i in range(args.steps):
+        dx.copy_(x_host, non_blocking=True)
+        step()
+        y_host.copy_(y, non_blocking=True)
+    e2e_ev[1].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e2e_ms = max_over_ranks(e2e_ev[0].elapsed_time(e2e_ev[1]) / args.steps, world)
+
+    wk = work(w, T)
+    dom = max(calls, key=calls.get)
+    pk = peaks()
+    d = wk[dom]
+    if d["flops"] > 0 and d["flops"] / d["bytes"] > pk["bf16"] * 1e12 / (pk["hbm"] * 1e9):
+        bound, achieved, peak, unit = "tensor", d["flops"] / (calls[dom] * 1e-3) / 1e12, pk["bf16"], "TFLOP/s"
+    else:
+        bound, achieved, peak, unit = "hbm", d["bytes"] / (calls[dom] * 1e-3) / 1e9, pk["hbm"], "GB/s"
+    result = {
+        "metric": METRIC,
+        "value": T * world / (ms * 1e-3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "data": "synthetic",
+        "config": {"workload": f"MoE layer config {w.cfg} ({w.name}): {w.describe()}",
+                   "T": T, "d": w.d, "E": w.E, "f": w.f, "k": w.k, "ep": ep,
+                   "routed_rows_per_step": T * w.k,
+                   "l2": "flushed before every step (256 MB write, outside the step events)",
+                   "parallelism": f"replicas x{world} (tokens sharded, no exchange)"},
+        "e2e": {"value": T * world / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": x.numel() * x.element_size(),
+                "d2h_bytes_per_step": y.numel() * y.element_size()},
+        "gpu_launches": 8 * args.steps,
+        "breakdown_ms": {k: round(v, 5) for k, v in calls.items()},
+        "roofline": {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                     "frac": achieved / peak, "peak_source": pk["src"], "traffic": None,
+                     "algorithmic": d},
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(w, args)
+    return result
+
+
+# ------------------------------------------------- CPU oracle (reference arm)
+def cpu_baseline(w: W.Workload, args, budget_s: float = 12.0):
+    """The oracle, as it stands, on a bounded seeded sample of the workload's
+    tokens (routing, layout of the sample, experts, combine), scaled to
+    tokens/s.  Runs on the host cores."""
+    import oracle
+    oracle.build()
+    x = W.make_x(w, args.seed, w.T)
+    wr = W.make_router(w, args.seed)
+    bias = W.make_bias(w, args.seed)
+    wg, wu, wd = W.make_experts(w, args.seed)
+
+    def run(n):
+        toks = W.sample_tokens(w.T, n, seed=args.seed + 5)
+        t0 = time.perf_counter()
+        r = oracle.forward(x, wr, bias, wg, wu, wd, w.k, tokens=toks)
+        oracle.dispatch_layout(r["idx"], w.E, w.eps[0])
+        return time.perf_counter() - t0
+
+    n = 64
+    dt = run(n)
+    while dt < budget_s / 4 and n < w.T:
+        n = min(w.T, int(n * max(2.0, budget_s / 2 / max(dt, 1e-3))))
+        dt = run(n)
+    return {"value": n / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{n} of {w.T} tokens (seeded), full router + top-k + layout + experts + combine in float64"}
+
+
+def run_reference(args, rank, world):
+    w = W.WORKLOADS[args.config]
+    if rank != 0:
+        return None
+    cb = cpu_baseline(w, args, budget_s=max(5.0, 2.0 * args.steps))
+    return {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": w.T / cb["value"] * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"MoE layer config {w.cfg} ({w.name}): {w.describe()}"},
+            "cpu_baseline": cb,
+            "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", type=int, default=2, choices=sorted(W.WORKLOADS))
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", 0))
+        world = int(os.environ.get("WORLD_SIZE", 1))
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    rank, world, local = dist_setup(args.gpus)
+    res = run_ours(args, rank, world, local)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,321 @@
+/*
+ * moe.h - C ABI of the B200 (sm_100a) MoE-layer forward.
+ *
+ * One token-routed Mixture-of-Experts layer, forward only, on one GPU:
+ *
+ *   logits = x W_r (+ bias)                       router GEMM
+ *   idx, gate = top-k(logits), softmax over the k top-k with softmax gates
+ *   counts / offsets / permutation / send layout  expert-grouped dispatch
+ *   x_perm[r] = x[row_token[r]]                   permute
+ *   h = silu(x_perm W_g[e]) * (x_perm W_u[e])     grouped SwiGLU, gate/up
+ *   y_perm = h W_d[e]                             grouped SwiGLU, down
+ *   y[t] = sum_j gate[t,j] y_perm[slot_row[t*k+j]] combine
+ *
+ * Sources (page title, then section / table):
+ *  - "MoE Pretraining: Parallelism Layout Changes the Model, Not Quality",
+ *    Methodology / Models and Data: a router sends each token to a few of 16
+ *    SwiGLU experts (top-4); Finding 3: routing margin and near-ties.
+ *  - "Revisiting MoE and Dense Speed-Accuracy Comparisons for LLM Training",
+ *    2.1 Architecture (SwiGLU, Top-K routing) and Table 1 (weight layouts:
+ *    router "ME" = [d, E]; FFN1 "EMH" = [E, d, f]; FFN2 "EHM" = [E, f, d]).
+ *  - "Expert Coupling in MoE Pretraining: Reducing All-to-All Overhead with
+ *    Correlated Placement and Token Shuffling", Abstract (experts spread over
+ *    EP ranks; each token sent to each GPU once), Table I (distinct GPUs per
+ *    token, deduplicated rows, T/EP tokens per GPU), Table III (notation).
+ *
+ * Conventions for every call:
+ *  - All array arguments are DEVICE pointers owned by the caller, except
+ *    `expert_rank_host` (host memory, read during the call).  The library
+ *    never allocates, never frees, and never synchronises the stream except
+ *    in moe_get_device_status.
+ *  - Every call enqueues its kernels on `stream` (a cudaStream_t; NULL is the
+ *    legacy default stream) and returns without waiting.  The returned status
+ *    covers host-side argument checks and launch errors.  Errors detected on
+ *    the device (an expert index out of range, a bounded wait that gave up)
+ *    are recorded in the workspace's status word; read it with
+ *    moe_get_device_status.
+ *  - Row-major layouts throughout.  Floating-point tensors are bf16 (dtype
+ *    MOE_BF16, fp32 accumulation) or fp32 (MOE_F32) as the shape says;
+ *    router logits and gates are always fp32; indices are int32.
+ *  - Pointers to bf16/fp32 tensors must be 16-byte aligned; int32 arrays
+ *    4-byte aligned (MOE_ERR_ALIGNMENT otherwise).
+ *  - Results are deterministic: repeated calls with the same inputs give
+ *    bit-identical outputs (no floating-point atomics anywhere).
+ *  - The library holds no global mutable state; calls on different streams
+ *    with different workspaces may run concurrently.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* moe_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,    /* bad shape, NULL pointer, bad expert->rank map */
+  MOE_ERR_UNSUPPORTED = 2,    /* valid shape outside what the kernels cover */
+  MOE_ERR_ALIGNMENT = 3,      /* pointer not aligned as required */
+  MOE_ERR_WORKSPACE = 4,      /* workspace / packed buffer too small */
+  MOE_ERR_CUDA = 5,           /* a CUDA runtime call or launch failed */
+  MOE_ERR_DEVICE_TIMEOUT = 6, /* a bounded device-side wait gave up */
+  MOE_ERR_DEVICE_INDEX = 7    /* an expert index outside [0, E) reached a kernel */
+} moe_status;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+
+/*
+ * Problem statement, in the pages' notation (Expert Coupling, Table III):
+ * T tokens of width d, E experts of FFN width f, top-k routing, and the
+ * number of simulated expert-parallel ranks `ep` (P in Table III).
+ * Supported: 0 <= T, T*k < 2^31; 1 <= E <= 256; 1 <= k <= min(E, 16);
+ * 1 <= ep <= E with E % ep == 0; d % 64 == 0 and f % 64 == 0 with
+ * d * sizeof(dtype) <= 16384 (else MOE_ERR_UNSUPPORTED).
+ */
+typedef struct {
+  int64_t T;
+  int32_t d;
+  int32_t E;
+  int32_t k;
+  int32_t f;
+  int32_t ep;
+  int32_t dtype; /* moe_dtype */
+} moe_shape;
+
+/*
+ * Dispatch statistics, written to device memory by moe_dispatch_layout
+ * (Expert Coupling, Table I):
+ *  rows_sent          sum over tokens of the number of distinct ranks its k
+ *                     experts live on (one send row per token and rank);
+ *                     0 when ep == 1 (nothing is dispatched)
+ *  dup_removed        T*k - rows_sent: rows that a per-(token, expert)
+ *                     dispatch would send and the deduplicated one does not;
+ *                     0 when ep == 1
+ *  tokens_single_rank tokens whose k experts all live on one rank
+ *  home_rank_rows     assignments whose expert lives on the token's home
+ *                     rank floor(t * ep / T) (T/ep tokens per rank)
+ *  max/min_expert_rows largest / smallest per-expert row count
+ */
+typedef struct {
+  int64_t rows_sent;
+  int64_t dup_removed;
+  int64_t tokens_single_rank;
+  int64_t home_rank_rows;
+  int32_t max_expert_rows;
+  int32_t min_expert_rows;
+} moe_stats;
+
+/*
+ * Outputs of moe_dispatch_layout (all device memory, R = T*k):
+ *  expert_counts [E]      rows routed to each expert
+ *  expert_offsets[E+1]    exclusive prefix sum; expert e owns rows
+ *                         [expert_offsets[e], expert_offsets[e+1])
+ *  row_token     [R]      token of each expert-grouped row; inside an expert
+ *                         the rows follow the flat assignment index t*k+j
+ *                         (a stable counting sort)
+ *  slot_row      [R]      row of assignment t*k+j (inverse of row_token)
+ *  rank_counts   [ep]     send rows per rank (deduplicated)           (*)
+ *  rank_offsets  [ep+1]   exclusive prefix sum of rank_counts          (*)
+ *  send_token    [R]      token of each send row: grouped by rank, tokens
+ *                         ascending inside a rank; only the first
+ *                         rank_offsets[ep] entries are written          (*)
+ *  slot_send_row [R]      send row carrying assignment t*k+j            (*)
+ *  stats                  moe_stats (device), may be NULL
+ * (*) built only when ep > 1 (these may be NULL when ep == 1).
+ */
+typedef struct {
+  int32_t* expert_counts;
+  int32_t* expert_offsets;
+  int32_t* row_token;
+  int32_t* slot_row;
+  int32_t* rank_counts;
+  int32_t* rank_offsets;
+  int32_t* send_token;
+  int32_t* slot_send_row;
+  moe_stats* stats;
+} moe_layout;
+
+/* Human-readable name of a status code (static string). */
+MOE_API const char* moe_status_string(moe_status s);
+
+/*
+ * Scratch workspace for moe_route, moe_dispatch_layout and
+ * moe_grouped_swiglu (a few hundred KB): block histograms, the
+ * decoupled-lookback status words, and the device status word.
+ * The workspace must be zero-filled once before its first use (cudaMemset or
+ * moe_workspace_init); the library leaves it ready for the next call.
+ * One workspace serves one stream at a time.
+ */
+MOE_API moe_status moe_scratch_size(const moe_shape* shape, size_t* bytes);
+
+/*
+ * Workspace for moe_forward: the scratch above followed by every
+ * intermediate the forward needs and the caller did not pass in
+ * moe_forward_buffers (logits, routing, layout, x_perm, h, y_perm).
+ */
+MOE_API moe_status moe_forward_workspace_size(const moe_shape* shape, size_t* bytes);
+
+/* Zero-fill `bytes` of workspace on `stream` (a cudaMemsetAsync). */
+MOE_API moe_status moe_workspace_init(void* ws, size_t bytes, moe_stream_t stream);
+
+/*
+ * Size of the packed weight buffer for `shape`.
+ */
+MOE_API moe_status moe_packed_weights_size(const moe_shape* shape, size_t* bytes);
+
+/*
+ * Rearrange the layer's weights once into the kernels' operand layout
+ * (K-major, i.e. each output column's weights contiguous):
+ *   router  W_r [d, E] ("ME")   -> W_r^T [E16, d], E16 = E rounded up to 16,
+ *                                   extra rows zero
+ *   W_g, W_u [E, d, f] ("EMH")  -> per expert [2f, d]: blocks of B output
+ *                                   columns, gate rows then up rows
+ *                                   (B = 128 if f % 128 == 0 else 64)
+ *   W_d [E, f, d] ("EHM")       -> per expert W_d^T [d, f]
+ * All inputs in the shape's dtype, device memory, row-major.  The packed
+ * buffer is what moe_route, moe_grouped_swiglu and moe_forward read; it is
+ * only valid for the shape it was packed for.
+ */
+MOE_API moe_status moe_pack_weights(const moe_shape* shape, const void* w_router,
+                            const void* w_gate, const void* w_up,
+                            const void* w_down, void* packed,
+                            size_t packed_bytes, moe_stream_t stream);
+
+/*
+ * Router GEMM + top-k + gates.
+ *  x        [T, d] tokens (dtype), or NULL: then `logits` is an INPUT and only
+ *           the top-k step runs on it ("given logits" mode)
+ *  packed   packed weights (moe_pack_weights); unused when x == NULL
+ *  bias     [E] fp32 added to the logits before selection, or NULL
+ *  logits   [T, E] fp32: l[t,e] = sum_i x[t,i] W_r[i,e] + bias[e]
+ *  topk_idx [T, k] int32: the k experts with the largest logits, ordered
+ *           by (logit descending, expert index ascending); equal logits
+ *           (including -0.0 vs +0.0) resolve to the lower index
+ *  topk_gate[T, k] fp32: softmax of the k chosen logits
+ *           g_j = exp(l_j - l_0) / sum_i exp(l_i - l_0)
+ *  ws, ws_bytes scratch workspace (moe_scratch_size), for device errors
+ * Logits must be finite (NaN gives unspecified routing).
+ */
+MOE_API moe_status moe_route(const moe_shape* shape, const void* x, const void* packed,
+                     const float* bias, float* logits, int32_t* topk_idx,
+                     float* topk_gate, void* ws, size_t ws_bytes,
+                     moe_stream_t stream);
+
+/*
+ * Expert-grouped dispatch layout and the deduplicated per-rank send layout
+ * (see moe_layout).  Block-level histograms plus a decoupled-lookback scan
+ * across blocks, then a stable scatter.
+ *  topk_idx         [T, k] int32, device
+ *  expert_rank_host [E] int32 in HOST memory: rank owning each expert; NULL
+ *                   means contiguous placement e -> e / (E/ep).  Must be a
+ *                   partition: every rank owns exactly E/ep experts
+ *                   (MOE_ERR_INVALID_ARG otherwise).
+ *  ws, ws_bytes     scratch workspace (moe_scratch_size)
+ * An index outside [0, E) sets MOE_ERR_DEVICE_INDEX in the device status.
+ */
+MOE_API moe_status moe_dispatch_layout(const moe_shape* shape, const int32_t* topk_idx,
+                               const int32_t* expert_rank_host,
+                               const moe_layout* out, void* ws, size_t ws_bytes,
+                               moe_stream_t stream);
+
+/*
+ * Permute (gather): x_perm[r] = x[row_token[r]] for r < T*k, whole rows,
+ * moved by TMA bulk copies staged through shared memory.
+ *  x [T, d], x_perm [T*k, d] (dtype); row_token [T*k] int32.
+ */
+MOE_API moe_status moe_permute(const moe_shape* shape, const void* x,
+                       const int32_t* row_token, void* x_perm,
+                       moe_stream_t stream);
+
+/*
+ * Grouped SwiGLU experts over the expert-grouped rows:
+ *  h[r]      = silu(x_perm[r] W_g[e]) * (x_perm[r] W_u[e])   [T*k, f]
+ *  y_perm[r] = h[r] W_d[e]                                   [T*k, d]
+ * for expert e owning row r (expert_offsets [E+1], device, as produced by
+ * moe_dispatch_layout).  bf16: tcgen05 tensor cores, fp32 accumulation in
+ * tensor memory, h and y_perm rounded to bf16.  fp32: CUDA-core FMA.
+ *  ws, ws_bytes  scratch workspace (moe_scratch_size)
+ */
+MOE_API moe_status moe_grouped_swiglu(const moe_shape* shape, const void* x_perm,
+                              const int32_t* expert_offsets, const void* packed,
+                              void* h, void* y_perm, void* ws, size_t ws_bytes,
+                              moe_stream_t stream);
+
+/*
+ * Gate-weighted combine (un-permute):
+ *   y[t] = sum_{j<k} gate[t,j] * y_perm[slot_row[t*k+j]]
+ * summed in fp32 in ascending j, rounded once to the dtype.
+ *  y_perm [T*k, d]; slot_row [T*k] int32; topk_gate [T, k] fp32 or NULL for
+ *  unit gates; y [T, d].
+ */
+MOE_API moe_status moe_combine(const moe_shape* shape, const void* y_perm,
+                       const int32_t* slot_row, const float* topk_gate,
+                       void* y, moe_stream_t stream);
+
+/*
+ * Optional caller-owned buffers of moe_forward's intermediates (device).
+ * Any NULL member is placed in the workspace instead; pass NULL for the
+ * whole struct to keep everything in the workspace.
+ */
+typedef struct {
+  float* logits;      /* [T, E] */
+  int32_t* topk_idx;  /* [T, k] */
+  float* topk_gate;   /* [T, k] */
+  moe_layout layout;  /* as moe_dispatch_layout */
+  void* x_perm;       /* [T*k, d] */
+  void* h;            /* [T*k, f] */
+  void* y_perm;       /* [T*k, d] */
+} moe_forward_buffers;
+
+/*
+ * The whole layer: moe_route, moe_dispatch_layout, moe_permute,
+ * moe_grouped_swiglu and moe_combine enqueued back to back on `stream`,
+ * with no host synchronisation in between.
+ *  x [T, d]; packed weights; bias [E] or NULL; expert_rank_host as in
+ *  moe_dispatch_layout; y [T, d]; buffers may be NULL;
+ *  ws, ws_bytes  moe_forward_workspace_size bytes.
+ */
+MOE_API moe_status moe_forward(const moe_shape* shape, const void* x, const void* packed,
+                       const float* bias, const int32_t* expert_rank_host,
+                       void* y, const moe_forward_buffers* buffers, void* ws,
+                       size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Synchronise `stream`, read the device status word of workspace `ws`
+ * (MOE_OK, MOE_ERR_DEVICE_TIMEOUT or MOE_ERR_DEVICE_INDEX) into *out and
+ * reset it to MOE_OK.  Returns MOE_ERR_CUDA if the stream reports an error.
+ */
+MOE_API moe_status moe_get_device_status(void* ws, moe_stream_t stream, moe_status* out);
+
+/*
+ * Test hook for the bounded wait of moe_dispatch_layout's decoupled lookback:
+ * identical to moe_dispatch_layout, except that the block holding lookback
+ * ticket `stall_block` never publishes its histogram, and the waits give up
+ * after `wait_limit_ns` nanoseconds (production calls use one second).
+ * The call then reports MOE_ERR_DEVICE_TIMEOUT through the device status, the
+ * layout outputs are unspecified, and the context stays usable.
+ */
+MOE_API moe_status moe_debug_dispatch_layout_stall(const moe_shape* shape,
+                                           const int32_t* topk_idx,
+                                           const int32_t* expert_rank_host,
+                                           const moe_layout* out, void* ws,
+                                           size_t ws_bytes, int32_t stall_block,
+                                           int64_t wait_limit_ns,
+                                           moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

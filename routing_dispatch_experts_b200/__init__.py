@@ -1,0 +1,367 @@
+"""B200 (sm_100a) MoE-layer forward: Python binding of ``libmoe_b200.so``.
+
+The functions here carry the names of the C ABI in ``include/moe.h`` and only
+marshal arguments: they check tensor devices/dtypes/shapes, pass raw device
+pointers and the current CUDA stream, and raise :class:`MoeError` on a
+non-OK status.  Every step of the layer runs in the library's CUDA kernels;
+there is no CPU or PyTorch fallback.  Importing this package does not need a
+GPU, but it does need the built library (``python -m
+routing_dispatch_experts_b200.build``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = 1
+MOE_ERR_UNSUPPORTED = 2
+MOE_ERR_ALIGNMENT = 3
+MOE_ERR_WORKSPACE = 4
+MOE_ERR_CUDA = 5
+MOE_ERR_DEVICE_TIMEOUT = 6
+MOE_ERR_DEVICE_INDEX = 7
+STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
+                3: "MOE_ERR_ALIGNMENT", 4: "MOE_ERR_WORKSPACE", 5: "MOE_ERR_CUDA",
+                6: "MOE_ERR_DEVICE_TIMEOUT", 7: "MOE_ERR_DEVICE_INDEX"}
+MOE_F32, MOE_BF16 = 0, 1
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}")
+
+
+class moe_shape(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int64), ("d", ctypes.c_int32), ("E", ctypes.c_int32),
+                ("k", ctypes.c_int32), ("f", ctypes.c_int32), ("ep", ctypes.c_int32),
+                ("dtype", ctypes.c_int32)]
+
+
+class moe_stats(ctypes.Structure):
+    _fields_ = [("rows_sent", ctypes.c_int64), ("dup_removed", ctypes.c_int64),
+                ("tokens_single_rank", ctypes.c_int64), ("home_rank_rows", ctypes.c_int64),
+                ("max_expert_rows", ctypes.c_int32), ("min_expert_rows", ctypes.c_int32)]
+
+
+STATS_FIELDS = ("rows_sent", "dup_removed", "tokens_single_rank", "home_rank_rows",
+                "max_expert_rows", "min_expert_rows")
+
+
+class moe_layout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "expert_counts", "expert_offsets", "row_token", "slot_row", "rank_counts",
+        "rank_offsets", "send_token", "slot_send_row", "stats")]
+
+
+class moe_forward_buffers(ctypes.Structure):
+    _fields_ = [("logits", ctypes.c_void_p), ("topk_idx", ctypes.c_void_p),
+                ("topk_gate", ctypes.c_void_p), ("layout", moe_layout),
+                ("x_perm", ctypes.c_void_p), ("h", ctypes.c_void_p), ("y_perm", ctypes.c_void_p)]
+
+
+_lib = None
+
+# exported C symbols, in header order (checked against include/moe.h by the tests)
+SYMBOLS = ("moe_status_string", "moe_scratch_size", "moe_forward_workspace_size",
+           "moe_workspace_init", "moe_packed_weights_size", "moe_pack_weights", "moe_route",
+           "moe_dispatch_layout", "moe_permute", "moe_grouped_swiglu", "moe_combine",
+           "moe_forward", "moe_get_device_status", "moe_debug_dispatch_layout_stall")
+
+
+def lib() -> ctypes.CDLL:
+    """Load the CUDA library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m routing_dispatch_experts_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, S = ctypes.c_void_p, ctypes.POINTER(moe_shape)
+        sz = ctypes.POINTER(ctypes.c_size_t)
+        sig = {
+            "moe_status_string": ([ctypes.c_int], ctypes.c_char_p),
+            "moe_scratch_size": ([S, sz], ctypes.c_int),
+            "moe_forward_workspace_size": ([S, sz], ctypes.c_int),
+            "moe_workspace_init": ([P, ctypes.c_size_t, P], ctypes.c_int),
+            "moe_packed_weights_size": ([S, sz], ctypes.c_int),
+            "moe_pack_weights": ([S, P, P, P, P, P, ctypes.c_size_t, P], ctypes.c_int),
+            "moe_route": ([S, P, P, P, P, P, P, P, ctypes.c_size_t, P], ctypes.c_int),
+            "moe_dispatch_layout": ([S, P, P, ctypes.POINTER(moe_layout), P, ctypes.c_size_t, P],
+                                    ctypes.c_int),
+            "moe_permute": ([S, P, P, P, P], ctypes.c_int),
+            "moe_grouped_swiglu": ([S, P, P, P, P, P, P, ctypes.c_size_t, P], ctypes.c_int),
+            "moe_combine": ([S, P, P, P, P, P], ctypes.c_int),
+            "moe_forward": ([S, P, P, P, P, P, ctypes.POINTER(moe_forward_buffers), P,
+                             ctypes.c_size_t, P], ctypes.c_int),
+            "moe_get_device_status": ([P, P, ctypes.POINTER(ctypes.c_int)], ctypes.c_int),
+            "moe_debug_dispatch_layout_stall": ([S, P, P, ctypes.POINTER(moe_layout), P,
+                                                 ctypes.c_size_t, ctypes.c_int32, ctypes.c_int64, P],
+                                                ctypes.c_int),
+        }
+        for name, (args, res) in sig.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = L
+    return _lib
+
+
+def _check(status: int, where: str):
+    if status != MOE_OK:
+        raise MoeError(status, where)
+
+
+# ------------------------------------------------------------------ helpers
+@dataclass(frozen=True)
+class Shape:
+    T: int
+    d: int
+    E: int
+    k: int
+    f: int
+    ep: int = 1
+    dtype: torch.dtype = torch.bfloat16
+
+    @property
+    def c(self) -> moe_shape:
+        return moe_shape(self.T, self.d, self.E, self.k, self.f, self.ep,
+                         MOE_BF16 if self.dtype == torch.bfloat16 else MOE_F32)
+
+    @property
+    def R(self) -> int:
+        return self.T * self.k
+
+
+def _p(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t, dtype, shape, name):
+    if t.dtype != dtype or tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected {dtype} {tuple(shape)}, got {t.dtype} {tuple(t.shape)}")
+
+
+def scratch_size(shape: Shape) -> int:
+    n = ctypes.c_size_t()
+    s = shape.c
+    _check(lib().moe_scratch_size(ctypes.byref(s), ctypes.byref(n)), "moe_scratch_size")
+    return n.value
+
+
+def forward_workspace_size(shape: Shape) -> int:
+    n = ctypes.c_size_t()
+    s = shape.c
+    _check(lib().moe_forward_workspace_size(ctypes.byref(s), ctypes.byref(n)),
+           "moe_forward_workspace_size")
+    return n.value
+
+
+def packed_weights_size(shape: Shape) -> int:
+    n = ctypes.c_size_t()
+    s = shape.c
+    _check(lib().moe_packed_weights_size(ctypes.byref(s), ctypes.byref(n)),
+           "moe_packed_weights_size")
+    return n.value
+
+
+def workspace(shape: Shape, forward: bool = False, device="cuda") -> torch.Tensor:
+    """A zero-filled workspace (uint8) of the size the ABI asks for."""
+    n = forward_workspace_size(shape) if forward else scratch_size(shape)
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def workspace_init(ws: torch.Tensor, stream=None):
+    _check(lib().moe_workspace_init(_p(ws), ws.numel(), _stream(stream)), "moe_workspace_init")
+
+
+def pack_weights(shape: Shape, w_router, w_gate, w_up, w_down, stream=None) -> torch.Tensor:
+    """Pack W_r [d,E], W_g/W_u [E,d,f], W_d [E,f,d] into the kernels' layout."""
+    _need(w_router, shape.dtype, (shape.d, shape.E), "w_router")
+    _need(w_gate, shape.dtype, (shape.E, shape.d, shape.f), "w_gate")
+    _need(w_up, shape.dtype, (shape.E, shape.d, shape.f), "w_up")
+    _need(w_down, shape.dtype, (shape.E, shape.f, shape.d), "w_down")
+    n = packed_weights_size(shape)
+    packed = torch.empty(n, dtype=torch.uint8, device=w_gate.device)
+    s = shape.c
+    _check(lib().moe_pack_weights(ctypes.byref(s), _p(w_router), _p(w_gate), _p(w_up), _p(w_down),
+                                  _p(packed), n, _stream(stream)), "moe_pack_weights")
+    return packed
+
+
+def route(shape: Shape, x, packed, bias, ws, logits=None, stream=None):
+    """moe_route: returns (logits [T,E] f32, topk_idx [T,k] i32, topk_gate [T,k] f32).
+
+    x=None runs only the top-k step on the given `logits`."""
+    dev = ws.device
+    if x is not None:
+        _need(x, shape.dtype, (shape.T, shape.d), "x")
+        logits = torch.empty((shape.T, shape.E), dtype=torch.float32, device=dev)
+    else:
+        _need(logits, torch.float32, (shape.T, shape.E), "logits")
+    if bias is not None:
+        _need(bias, torch.float32, (shape.E,), "bias")
+    idx = torch.empty((shape.T, shape.k), dtype=torch.int32, device=dev)
+    gate = torch.empty((shape.T, shape.k), dtype=torch.float32, device=dev)
+    s = shape.c
+    _check(lib().moe_route(ctypes.byref(s), _p(x), _p(packed), _p(bias), _p(logits), _p(idx),
+                           _p(gate), _p(ws), ws.numel(), _stream(stream)), "moe_route")
+    return logits, idx, gate
+
+
+def _layout_tensors(shape: Shape, dev):
+    R = shape.R
+    i32 = dict(dtype=torch.int32, device=dev)
+    out = dict(expert_counts=torch.empty(shape.E, **i32),
+               expert_offsets=torch.empty(shape.E + 1, **i32),
+               row_token=torch.empty(R, **i32), slot_row=torch.empty(R, **i32),
+               stats=torch.zeros(6, dtype=torch.int64, device=dev))
+    if shape.ep > 1:
+        out.update(rank_counts=torch.empty(shape.ep, **i32),
+                   rank_offsets=torch.empty(shape.ep + 1, **i32),
+                   send_token=torch.full((R,), -1, **i32),
+                   slot_send_row=torch.empty(R, **i32))
+    return out
+
+
+def _c_layout(t: dict) -> moe_layout:
+    return moe_layout(*[_p(t.get(n)) for n in (
+        "expert_counts", "expert_offsets", "row_token", "slot_row", "rank_counts",
+        "rank_offsets", "send_token", "slot_send_row", "stats")])
+
+
+def _host_map(shape: Shape, expert_rank: Optional[Sequence[int]]):
+    if expert_rank is None:
+        return None
+    if len(expert_rank) != shape.E:
+        raise ValueError("expert_rank must have E entries")
+    return (ctypes.c_int32 * shape.E)(*[int(r) for r in expert_rank])
+
+
+def stats_dict(stats: torch.Tensor) -> dict:
+    """Decode the device moe_stats (6 int64 words as allocated here)."""
+    v = stats.cpu().tolist()
+    lo = v[4] & 0xFFFFFFFF
+    hi = (v[4] >> 32) & 0xFFFFFFFF
+    return dict(rows_sent=v[0], dup_removed=v[1], tokens_single_rank=v[2],
+                home_rank_rows=v[3], max_expert_rows=lo, min_expert_rows=hi)
+
+
+def dispatch_layout(shape: Shape, topk_idx, ws, expert_rank=None, stream=None) -> dict:
+    """moe_dispatch_layout: returns the layout tensors (see moe.h)."""
+    _need(topk_idx, torch.int32, (shape.T, shape.k), "topk_idx")
+    out = _layout_tensors(shape, ws.device)
+    lay = _c_layout(out)
+    s = shape.c
+    _check(lib().moe_dispatch_layout(ctypes.byref(s), _p(topk_idx), _host_map(shape, expert_rank),
+                                     ctypes.byref(lay), _p(ws), ws.numel(), _stream(stream)),
+           "moe_dispatch_layout")
+    return out
+
+
+def debug_dispatch_layout_stall(shape: Shape, topk_idx, ws, stall_block: int, wait_limit_ns: int,
+                                expert_rank=None, stream=None) -> dict:
+    out = _layout_tensors(shape, ws.device)
+    lay = _c_layout(out)
+    s = shape.c
+    _check(lib().moe_debug_dispatch_layout_stall(
+        ctypes.byref(s), _p(topk_idx), _host_map(shape, expert_rank), ctypes.byref(lay), _p(ws),
+        ws.numel(), stall_block, wait_limit_ns, _stream(stream)), "moe_debug_dispatch_layout_stall")
+    return out
+
+
+def permute(shape: Shape, x, row_token, stream=None):
+    _need(x, shape.dtype, (shape.T, shape.d), "x")
+    x_perm = torch.empty((shape.R, shape.d), dtype=shape.dtype, device=x.device)
+    s = shape.c
+    _check(lib().moe_permute(ctypes.byref(s), _p(x), _p(row_token), _p(x_perm), _stream(stream)),
+           "moe_permute")
+    return x_perm
+
+
+def grouped_swiglu(shape: Shape, x_perm, expert_offsets, packed, ws, stream=None):
+    """moe_grouped_swiglu: returns (h [R,f], y_perm [R,d])."""
+    _need(x_perm, shape.dtype, (shape.R, shape.d), "x_perm")
+    h = torch.empty((shape.R, shape.f), dtype=shape.dtype, device=x_perm.device)
+    y_perm = torch.empty((shape.R, shape.d), dtype=shape.dtype, device=x_perm.device)
+    s = shape.c
+    _check(lib().moe_grouped_swiglu(ctypes.byref(s), _p(x_perm), _p(expert_offsets), _p(packed),
+                                    _p(h), _p(y_perm), _p(ws), ws.numel(), _stream(stream)),
+           "moe_grouped_swiglu")
+    return h, y_perm
+
+
+def combine(shape: Shape, y_perm, slot_row, topk_gate=None, stream=None):
+    _need(y_perm, shape.dtype, (shape.R, shape.d), "y_perm")
+    y = torch.empty((shape.T, shape.d), dtype=shape.dtype, device=y_perm.device)
+    s = shape.c
+    _check(lib().moe_combine(ctypes.byref(s), _p(y_perm), _p(slot_row), _p(topk_gate), _p(y),
+                             _stream(stream)), "moe_combine")
+    return y
+
+
+class ForwardBuffers:
+    """Caller-owned intermediates of moe_forward, readable after the call."""
+
+    def __init__(self, shape: Shape, device="cuda"):
+        R = shape.R
+        self.logits = torch.empty((shape.T, shape.E), dtype=torch.float32, device=device)
+        self.topk_idx = torch.empty((shape.T, shape.k), dtype=torch.int32, device=device)
+        self.topk_gate = torch.empty((shape.T, shape.k), dtype=torch.float32, device=device)
+        self.layout = _layout_tensors(shape, device)
+        self.x_perm = torch.empty((R, shape.d), dtype=shape.dtype, device=device)
+        self.h = torch.empty((R, shape.f), dtype=shape.dtype, device=device)
+        self.y_perm = torch.empty((R, shape.d), dtype=shape.dtype, device=device)
+
+    @property
+    def c(self) -> moe_forward_buffers:
+        return moe_forward_buffers(_p(self.logits), _p(self.topk_idx), _p(self.topk_gate),
+                                   _c_layout(self.layout), _p(self.x_perm), _p(self.h),
+                                   _p(self.y_perm))
+
+
+def forward(shape: Shape, x, packed, bias, ws, expert_rank=None, y=None,
+            buffers: Optional[ForwardBuffers] = None, stream=None):
+    """moe_forward: the whole layer; returns y [T, d]."""
+    _need(x, shape.dtype, (shape.T, shape.d), "x")
+    if y is None:
+        y = torch.empty((shape.T, shape.d), dtype=shape.dtype, device=x.device)
+    s = shape.c
+    b = buffers.c if buffers is not None else None
+    _check(lib().moe_forward(ctypes.byref(s), _p(x), _p(packed), _p(bias),
+                             _host_map(shape, expert_rank), _p(y),
+                             ctypes.byref(b) if b is not None else None, _p(ws), ws.numel(),
+                             _stream(stream)), "moe_forward")
+    return y
+
+
+def get_device_status(ws, stream=None) -> int:
+    out = ctypes.c_int(0)
+    _check(lib().moe_get_device_status(_p(ws), _stream(stream), ctypes.byref(out)),
+           "moe_get_device_status")
+    return out.value
+
+
+def check_device_status(ws, stream=None):
+    st = get_device_status(ws, stream)
+    if st != MOE_OK:
+        raise MoeError(st, "device status")

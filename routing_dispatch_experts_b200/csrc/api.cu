@@ -1,0 +1,482 @@
+// api.cu - the C ABI: argument checks, workspace carving, kernel sequencing.
+//
+// Host code only; every step of the layer runs in the kernels of the other
+// files.  Nothing here allocates device memory or synchronises a stream
+// (except moe_get_device_status, whose job is to read the device status).
+#include <algorithm>
+#include <cstring>
+
+#include "kernels.cuh"
+
+using namespace moe;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+int esize(int dtype) { return dtype == MOE_BF16 ? 2 : 4; }
+
+int gu_block(int f) { return f % 128 == 0 ? 128 : 64; }
+
+int pad16(int E) { return (E + 15) / 16 * 16; }
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+moe_status check_shape(const moe_shape* s) {
+  if (!s) return MOE_ERR_INVALID_ARG;
+  if (s->dtype != MOE_F32 && s->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+  if (s->T < 0 || s->E < 1 || s->E > 256 || s->k < 1 || s->k > std::min(s->E, 16) || s->ep < 1 ||
+      s->ep > s->E || s->E % s->ep != 0 || s->d <= 0 || s->f <= 0)
+    return MOE_ERR_INVALID_ARG;
+  if (s->T * (int64_t)s->k >= (int64_t(1) << 31)) return MOE_ERR_INVALID_ARG;
+  if (s->d % 64 != 0 || s->f % 64 != 0 || (int64_t)s->d * esize(s->dtype) > 16384)
+    return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+// ---- scratch workspace: control block, lookback status words, prefixes
+struct Scratch {
+  Control* ctl;
+  uint64_t* status;
+  int32_t* prefix;
+  int32_t* totals;
+};
+
+size_t scratch_bytes(const moe_shape* s) {
+  const size_t nb = (size_t)layout_blocks(s->T), bins = (size_t)layout_bins(s->E, s->ep);
+  return align_up(sizeof(Control)) + align_up(nb * bins * 8) + align_up(nb * bins * 4) +
+         align_up(bins * 4);
+}
+
+Scratch carve_scratch(const moe_shape* s, void* ws) {
+  const size_t nb = (size_t)layout_blocks(s->T), bins = (size_t)layout_bins(s->E, s->ep);
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  Scratch sc;
+  sc.ctl = reinterpret_cast<Control*>(p);
+  p += align_up(sizeof(Control));
+  sc.status = reinterpret_cast<uint64_t*>(p);
+  p += align_up(nb * bins * 8);
+  sc.prefix = reinterpret_cast<int32_t*>(p);
+  p += align_up(nb * bins * 4);
+  sc.totals = reinterpret_cast<int32_t*>(p);
+  return sc;
+}
+
+// ---- packed weights
+struct Packed {
+  const void* wrT;
+  const void* wgu;
+  const void* wdT;
+};
+
+size_t packed_bytes(const moe_shape* s) {
+  const size_t es = esize(s->dtype);
+  return align_up((size_t)pad16(s->E) * s->d * es) + align_up((size_t)s->E * 2 * s->f * s->d * es) +
+         align_up((size_t)s->E * s->d * s->f * es);
+}
+
+Packed carve_packed(const moe_shape* s, const void* packed) {
+  const size_t es = esize(s->dtype);
+  const uint8_t* p = static_cast<const uint8_t*>(packed);
+  Packed pk;
+  pk.wrT = p;
+  p += align_up((size_t)pad16(s->E) * s->d * es);
+  pk.wgu = p;
+  p += align_up((size_t)s->E * 2 * s->f * s->d * es);
+  pk.wdT = p;
+  return pk;
+}
+
+// ---- forward intermediates placed after the scratch
+struct FwdBufs {
+  float* logits;
+  int32_t* idx;
+  float* gate;
+  moe_layout lay;
+  void* x_perm;
+  void* h;
+  void* y_perm;
+};
+
+size_t forward_bytes(const moe_shape* s) {
+  const size_t R = (size_t)s->T * s->k, es = esize(s->dtype);
+  size_t n = scratch_bytes(s);
+  n += align_up((size_t)s->T * s->E * 4);      // logits
+  n += 2 * align_up(R * 4);                     // idx, gate
+  n += align_up((size_t)s->E * 4) + align_up((size_t)(s->E + 1) * 4);
+  n += 2 * align_up(R * 4);                     // row_token, slot_row
+  n += align_up((size_t)s->ep * 4) + align_up((size_t)(s->ep + 1) * 4);
+  n += 2 * align_up(R * 4);                     // send_token, slot_send_row
+  n += align_up(sizeof(moe_stats));
+  n += align_up(R * s->d * es) + align_up(R * s->f * es) + align_up(R * s->d * es);
+  return n;
+}
+
+FwdBufs carve_forward(const moe_shape* s, void* ws, const moe_forward_buffers* b) {
+  const size_t R = (size_t)s->T * s->k, es = esize(s->dtype);
+  uint8_t* p = static_cast<uint8_t*>(ws) + scratch_bytes(s);
+  auto take = [&p](size_t bytes) {
+    void* q = p;
+    p += align_up(bytes);
+    return q;
+  };
+  FwdBufs f;
+  f.logits = static_cast<float*>(take((size_t)s->T * s->E * 4));
+  f.idx = static_cast<int32_t*>(take(R * 4));
+  f.gate = static_cast<float*>(take(R * 4));
+  f.lay.expert_counts = static_cast<int32_t*>(take((size_t)s->E * 4));
+  f.lay.expert_offsets = static_cast<int32_t*>(take((size_t)(s->E + 1) * 4));
+  f.lay.row_token = static_cast<int32_t*>(take(R * 4));
+  f.lay.slot_row = static_cast<int32_t*>(take(R * 4));
+  f.lay.rank_counts = static_cast<int32_t*>(take((size_t)s->ep * 4));
+  f.lay.rank_offsets = static_cast<int32_t*>(take((size_t)(s->ep + 1) * 4));
+  f.lay.send_token = static_cast<int32_t*>(take(R * 4));
+  f.lay.slot_send_row = static_cast<int32_t*>(take(R * 4));
+  f.lay.stats = static_cast<moe_stats*>(take(sizeof(moe_stats)));
+  f.x_perm = take(R * s->d * es);
+  f.h = take(R * s->f * es);
+  f.y_perm = take(R * s->d * es);
+  if (b) {
+    if (b->logits) f.logits = b->logits;
+    if (b->topk_idx) f.idx = b->topk_idx;
+    if (b->topk_gate) f.gate = b->topk_gate;
+    if (b->layout.expert_counts) f.lay.expert_counts = b->layout.expert_counts;
+    if (b->layout.expert_offsets) f.lay.expert_offsets = b->layout.expert_offsets;
+    if (b->layout.row_token) f.lay.row_token = b->layout.row_token;
+    if (b->layout.slot_row) f.lay.slot_row = b->layout.slot_row;
+    if (b->layout.rank_counts) f.lay.rank_counts = b->layout.rank_counts;
+    if (b->layout.rank_offsets) f.lay.rank_offsets = b->layout.rank_offsets;
+    if (b->layout.send_token) f.lay.send_token = b->layout.send_token;
+    if (b->layout.slot_send_row) f.lay.slot_send_row = b->layout.slot_send_row;
+    if (b->layout.stats) f.lay.stats = b->layout.stats;
+    if (b->x_perm) f.x_perm = b->x_perm;
+    if (b->h) f.h = b->h;
+    if (b->y_perm) f.y_perm = b->y_perm;
+  }
+  return f;
+}
+
+moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+moe_status build_map(const moe_shape* s, const int32_t* host_map, RankMap* m) {
+  std::memset(m, 0, sizeof(*m));
+  const int per = s->E / s->ep;
+  if (!host_map) {
+    for (int e = 0; e < s->E; ++e) m->r[e] = (uint8_t)(e / per);
+    return MOE_OK;
+  }
+  int count[256] = {0};
+  for (int e = 0; e < s->E; ++e) {
+    const int r = host_map[e];
+    if (r < 0 || r >= s->ep) return MOE_ERR_INVALID_ARG;
+    ++count[r];
+    m->r[e] = (uint8_t)r;
+  }
+  // a placement is a partition: every rank owns exactly E/ep experts
+  for (int r = 0; r < s->ep; ++r)
+    if (count[r] != per) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+// ---- the steps, after their arguments are checked
+moe_status do_route(const moe_shape* s, const void* x, const Packed* pk, const float* bias,
+                    float* logits, int32_t* idx, float* gate, Control* ctl, cudaStream_t st) {
+  if (x) {
+    cudaError_t e;
+    if (s->dtype == MOE_BF16) {
+      GemmArgs a{};
+      a.A = x;
+      a.rows = s->T;
+      a.B = pk->wrT;
+      a.offsets = nullptr;
+      a.G = 1;
+      a.K = s->d;
+      a.n_per_group = pad16(s->E);
+      a.n_out = s->E;
+      a.out = logits;
+      a.ld_out = s->E;
+      a.bias = bias;
+      a.ctl = ctl;
+      e = launch_gemm_tc(kEpiLogits, pad16(s->E), a, st);
+    } else {
+      e = launch_router_f32(static_cast<const float*>(x), static_cast<const float*>(pk->wrT), bias,
+                            s->T, s->d, s->E, logits, st);
+    }
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  return cuda_status(launch_topk(logits, s->T, s->E, s->k, idx, gate, st));
+}
+
+moe_status do_layout(const moe_shape* s, const int32_t* idx, const RankMap& map,
+                     const moe_layout* o, const Scratch& sc, int stall, int64_t limit,
+                     cudaStream_t st) {
+  LayoutOut lo;
+  lo.counts = o->expert_counts;
+  lo.offsets = o->expert_offsets;
+  lo.row_token = o->row_token;
+  lo.slot_row = o->slot_row;
+  lo.rank_counts = o->rank_counts;
+  lo.rank_offsets = o->rank_offsets;
+  lo.send_token = o->send_token;
+  lo.slot_send_row = o->slot_send_row;
+  lo.stats = o->stats;
+  return cuda_status(launch_layout(idx, s->T, s->k, s->E, s->ep, map, lo, sc.ctl, sc.status,
+                                   sc.prefix, sc.totals, stall, limit, st));
+}
+
+moe_status do_grouped(const moe_shape* s, const void* x_perm, const int32_t* offsets,
+                      const Packed* pk, void* h, void* y_perm, Control* ctl, cudaStream_t st) {
+  const int64_t R = s->T * (int64_t)s->k;
+  if (s->dtype == MOE_F32)
+    return cuda_status(launch_grouped_f32(static_cast<const float*>(x_perm), offsets, s->E, R, s->d,
+                                          s->f, gu_block(s->f), static_cast<const float*>(pk->wgu),
+                                          static_cast<const float*>(pk->wdT),
+                                          static_cast<float*>(h), static_cast<float*>(y_perm), st));
+  GemmArgs a{};
+  a.A = x_perm;
+  a.rows = R;
+  a.B = pk->wgu;
+  a.offsets = offsets;
+  a.G = s->E;
+  a.K = s->d;
+  a.n_per_group = 2 * s->f;
+  a.n_out = s->f;
+  a.out = h;
+  a.ld_out = s->f;
+  a.ctl = ctl;
+  cudaError_t e = launch_gemm_tc(kEpiSwiGLU, 2 * gu_block(s->f), a, st);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  GemmArgs b{};
+  b.A = h;
+  b.rows = R;
+  b.B = pk->wdT;
+  b.offsets = offsets;
+  b.G = s->E;
+  b.K = s->f;
+  b.n_per_group = s->d;
+  b.n_out = s->d;
+  b.out = y_perm;
+  b.ld_out = s->d;
+  b.ctl = ctl;
+  const int bn = s->d % 256 == 0 ? 256 : (s->d % 128 == 0 ? 128 : 64);
+  return cuda_status(launch_gemm_tc(kEpiBF16, bn, b, st));
+}
+
+moe_status check_layout_ptrs(const moe_shape* s, const moe_layout* o) {
+  if (!o || !o->expert_counts || !o->expert_offsets || !o->row_token || !o->slot_row)
+    return MOE_ERR_INVALID_ARG;
+  if (s->ep > 1 && (!o->rank_counts || !o->rank_offsets || !o->send_token || !o->slot_send_row))
+    return MOE_ERR_INVALID_ARG;
+  const void* ps[] = {o->expert_counts, o->expert_offsets, o->row_token, o->slot_row,
+                      o->rank_counts, o->rank_offsets, o->send_token, o->slot_send_row};
+  for (const void* p : ps)
+    if (p && !aligned(p, 4)) return MOE_ERR_ALIGNMENT;
+  if (o->stats && !aligned(o->stats, 8)) return MOE_ERR_ALIGNMENT;
+  return MOE_OK;
+}
+
+moe_status layout_entry(const moe_shape* s, const int32_t* idx, const int32_t* host_map,
+                        const moe_layout* o, void* ws, size_t ws_bytes, int stall, int64_t limit,
+                        cudaStream_t st) {
+  moe_status r = check_shape(s);
+  if (r != MOE_OK) return r;
+  if ((!idx && s->T > 0) || !ws) return MOE_ERR_INVALID_ARG;
+  if ((r = check_layout_ptrs(s, o)) != MOE_OK) return r;
+  if (!aligned(idx, 4) || !aligned(ws, kAlign)) return MOE_ERR_ALIGNMENT;
+  if (ws_bytes < scratch_bytes(s)) return MOE_ERR_WORKSPACE;
+  RankMap map;
+  if ((r = build_map(s, host_map, &map)) != MOE_OK) return r;
+  return do_layout(s, idx, map, o, carve_scratch(s, ws), stall, limit, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_ALIGNMENT: return "MOE_ERR_ALIGNMENT";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_DEVICE_TIMEOUT: return "MOE_ERR_DEVICE_TIMEOUT";
+    case MOE_ERR_DEVICE_INDEX: return "MOE_ERR_DEVICE_INDEX";
+  }
+  return "MOE_ERR_UNKNOWN";
+}
+
+moe_status moe_scratch_size(const moe_shape* s, size_t* bytes) {
+  moe_status r = check_shape(s);
+  if (r != MOE_OK) return r;
+  if (!bytes) return MOE_ERR_INVALID_ARG;
+  *bytes = scratch_bytes(s);
+  return MOE_OK;
+}
+
+moe_status moe_forward_workspace_size(const moe_shape* s, size_t* bytes) {
+  moe_status r = check_shape(s);
+  if (r != MOE_OK) return r;
+  if (!bytes) return MOE_ERR_INVALID_ARG;
+  *bytes = forward_bytes(s);
+  return MOE_OK;
+}
+
+moe_status moe_workspace_init(void* ws, size_t bytes, moe_stream_t stream) {
+  if (!ws) return MOE_ERR_INVALID_ARG;
+  return cuda_status(cudaMemsetAsync(ws, 0, bytes, (cudaStream_t)stream));
+}
+
+moe_status moe_packed_weights_size(const moe_shape* s, size_t* bytes) {
+  moe_status r = check_shape(s);
+  if (r != MOE_OK) return r;
+  if (!bytes) return MOE_ERR_INVALID_ARG;
+  *bytes = packed_bytes(s);
+  return MOE_OK;
+}
+
+moe_status moe_pack_weights(const moe_shape* s, const void* w_router, const void* w_gate,
+                            const void* w_up, const void* w_down, void* packed,
+                            size_t packed_bytes_, moe_stream_t stream) {
+  moe_status r = check_shape(s);
+  if (r != MOE_OK) return r;
+  if (!w_router || !w_gate || !w_up || !w_down || !packed) return MOE_ERR_INVALID_ARG;
+  const size_t es = esize(s->dtype);
+  for (const void* p : {w_router, w_gate, w_up, w_down})
+    if (!aligned(p, es)) return MOE_ERR_ALIGNMENT;
+  if (!aligned(packed, kAlign)) return MOE_ERR_ALIGNMENT;
+  if (packed_bytes_ < packed_bytes(s)) return MOE_ERR_WORKSPACE;
+  Packed pk = carve_packed(s, packed);
+  return cuda_status(launch_pack(s->dtype, s->d, s->E, s->f, gu_block(s->f), pad16(s->E), w_router,
+                                 w_gate, w_up, w_down, const_cast<void*>(pk.wrT),
+                                 const_cast<void*>(pk.wgu), const_cast<void*>(pk.wdT),
+                                 (cudaStream_t)stream));
+}
+
+moe_status moe_route(const moe_shape* s, const void* x, const void* packed, const float* bias,
+                     float* logits, int32_t* topk_idx, float* topk_gate, void* ws,
+                     size_t ws_bytes, moe_stream_t stream) {
+  moe_status r = check_shape(s);
+  if (r != MOE_OK) return r;
+  if (s->T > 0 && (!logits || !topk_idx || !topk_gate)) return MOE_ERR_INVALID_ARG;
+  if (x && (!packed || !ws)) return MOE_ERR_INVALID_ARG;
+  if ((x && !aligned(x, 16)) || (packed && !aligned(packed, kAlign)) || !aligned(logits, 4) ||
+      !aligned(topk_idx, 4) || !aligned(topk_gate, 4) || (bias && !aligned(bias, 4)) ||
+      (ws && !aligned(ws, kAlign)))
+    return MOE_ERR_ALIGNMENT;
+  if (ws && ws_bytes < scratch_bytes(s)) return MOE_ERR_WORKSPACE;
+  if (s->T == 0) return MOE_OK;
+  Packed pk{};
+  if (packed) pk = carve_packed(s, packed);
+  Control* ctl = ws ? carve_scratch(s, ws).ctl : nullptr;
+  return do_route(s, x, &pk, bias, logits, topk_idx, topk_gate, ctl, (cudaStream_t)stream);
+}
+
+moe_status moe_dispatch_layout(const moe_shape* s, const int32_t* topk_idx,
+                               const int32_t* expert_rank_host, const moe_layout* out, void* ws,
+                               size_t ws_bytes, moe_stream_t stream) {
+  return layout_entry(s, topk_idx, expert_rank_host, out, ws, ws_bytes, -1, kWaitLimitNs,
+                      (cudaStream_t)stream);
+}
+
+moe_status moe_debug_dispatch_layout_stall(const moe_shape* s, const int32_t* topk_idx,
+                                           const int32_t* expert_rank_host, const moe_layout* out,
+                                           void* ws, size_t ws_bytes, int32_t stall_block,
+                                           int64_t wait_limit_ns, moe_stream_t stream) {
+  if (wait_limit_ns <= 0 || wait_limit_ns > kWaitLimitNs) return MOE_ERR_INVALID_ARG;
+  return layout_entry(s, topk_idx, expert_rank_host, out, ws, ws_bytes, stall_block,
+                      wait_limit_ns, (cudaStream_t)stream);
+}
+
+moe_status moe_permute(const moe_shape* s, const void* x, const int32_t* row_token, void* x_perm,
+                       moe_stream_t stream) {
+  moe_status r = check_shape(s);
+  if (r != MOE_OK) return r;
+  if (s->T == 0) return MOE_OK;
+  if (!x || !row_token || !x_perm) return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(x_perm, 16) || !aligned(row_token, 4)) return MOE_ERR_ALIGNMENT;
+  return cuda_status(launch_permute(x, row_token, x_perm, s->T, s->T * (int64_t)s->k,
+                                    (uint32_t)(s->d * esize(s->dtype)), (cudaStream_t)stream));
+}
+
+moe_status moe_grouped_swiglu(const moe_shape* s, const void* x_perm, const int32_t* offsets,
+                              const void* packed, void* h, void* y_perm, void* ws, size_t ws_bytes,
+                              moe_stream_t stream) {
+  moe_status r = check_shape(s);
+  if (r != MOE_OK) return r;
+  if (s->T == 0) return MOE_OK;
+  if (!x_perm || !offsets || !packed || !h || !y_perm || !ws) return MOE_ERR_INVALID_ARG;
+  if (!aligned(x_perm, 16) || !aligned(h, 16) || !aligned(y_perm, 16) || !aligned(offsets, 4) ||
+      !aligned(packed, kAlign) || !aligned(ws, kAlign))
+    return MOE_ERR_ALIGNMENT;
+  if (ws_bytes < scratch_bytes(s)) return MOE_ERR_WORKSPACE;
+  Packed pk = carve_packed(s, packed);
+  return do_grouped(s, x_perm, offsets, &pk, h, y_perm, carve_scratch(s, ws).ctl,
+                    (cudaStream_t)stream);
+}
+
+moe_status moe_combine(const moe_shape* s, const void* y_perm, const int32_t* slot_row,
+                       const float* gate, void* y, moe_stream_t stream) {
+  moe_status r = check_shape(s);
+  if (r != MOE_OK) return r;
+  if (s->T == 0) return MOE_OK;
+  if (!y_perm || !slot_row || !y) return MOE_ERR_INVALID_ARG;
+  if (!aligned(y_perm, 16) || !aligned(y, 16) || !aligned(slot_row, 4) || (gate && !aligned(gate, 4)))
+    return MOE_ERR_ALIGNMENT;
+  return cuda_status(
+      launch_combine(s->dtype, y_perm, slot_row, gate, y, s->T, s->d, s->k, (cudaStream_t)stream));
+}
+
+moe_status moe_forward(const moe_shape* s, const void* x, const void* packed, const float* bias,
+                       const int32_t* expert_rank_host, void* y, const moe_forward_buffers* buffers,
+                       void* ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status r = check_shape(s);
+  if (r != MOE_OK) return r;
+  if (!ws) return MOE_ERR_INVALID_ARG;
+  if (!aligned(ws, kAlign)) return MOE_ERR_ALIGNMENT;
+  if (ws_bytes < forward_bytes(s)) return MOE_ERR_WORKSPACE;
+  RankMap map;
+  if ((r = build_map(s, expert_rank_host, &map)) != MOE_OK) return r;
+  if (s->T == 0) return MOE_OK;
+  if (!x || !packed || !y) return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(y, 16) || !aligned(packed, kAlign) || (bias && !aligned(bias, 4)))
+    return MOE_ERR_ALIGNMENT;
+  FwdBufs f = carve_forward(s, ws, buffers);
+  if ((r = check_layout_ptrs(s, &f.lay)) != MOE_OK) return r;
+  if (!aligned(f.logits, 4) || !aligned(f.idx, 4) || !aligned(f.gate, 4) || !aligned(f.x_perm, 16) ||
+      !aligned(f.h, 16) || !aligned(f.y_perm, 16))
+    return MOE_ERR_ALIGNMENT;
+  const Scratch sc = carve_scratch(s, ws);
+  const Packed pk = carve_packed(s, packed);
+  cudaStream_t st = (cudaStream_t)stream;
+  if ((r = do_route(s, x, &pk, bias, f.logits, f.idx, f.gate, sc.ctl, st)) != MOE_OK) return r;
+  if ((r = do_layout(s, f.idx, map, &f.lay, sc, -1, kWaitLimitNs, st)) != MOE_OK) return r;
+  if ((r = cuda_status(launch_permute(x, f.lay.row_token, f.x_perm, s->T, s->T * (int64_t)s->k,
+                                      (uint32_t)(s->d * esize(s->dtype)), st))) != MOE_OK)
+    return r;
+  if ((r = do_grouped(s, f.x_perm, f.lay.expert_offsets, &pk, f.h, f.y_perm, sc.ctl, st)) != MOE_OK)
+    return r;
+  return cuda_status(launch_combine(s->dtype, f.y_perm, f.lay.slot_row, f.gate, y, s->T, s->d, s->k, st));
+}
+
+moe_status moe_get_device_status(void* ws, moe_stream_t stream, moe_status* out) {
+  if (!ws || !out) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
+  uint32_t v = 0;
+  if (cudaMemcpy(&v, ws, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  *out = (moe_status)v;
+  if (v != MOE_OK) {
+    if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), st) != cudaSuccess) return MOE_ERR_CUDA;
+    // the detail word (offset 8) is informational; clear it with the status
+    if (cudaMemsetAsync(static_cast<uint8_t*>(ws) + 8, 0, sizeof(uint32_t), st) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,410 @@
+// gemm_tc.cu - grouped GEMM on the fifth-generation tensor cores (tcgen05).
+//
+// The only dense contraction of the layer.  For each group g (an expert, or
+// the whole batch for the router) and each row r in [offsets[g],
+// offsets[g+1]):  acc[r, n] = sum_k A[r, k] * B[g*n_per_group + n, k], with
+// one of three epilogues:
+//   kEpiSwiGLU  B holds, per block of BN/2 output columns, the gate rows then
+//               the up rows of W_g / W_u; out = silu(acc_gate) * acc_up in
+//               bf16 (SwiGLU: "Revisiting MoE and Dense Speed-Accuracy
+//               Comparisons", 2.1 Architecture)
+//   kEpiBF16    out = acc in bf16 (the down projection)
+//   kEpiLogits  out = acc + bias in fp32 (the router GEMM)
+//
+// Design (one CTA per SM, persistent, 6 warps):
+//   warp 0      TMA producer: 128 x 64 A tiles and BN x 64 B tiles, 128-byte
+//               swizzle, into a STAGES-deep shared-memory ring (full/empty
+//               mbarriers)
+//   warp 1      allocates tensor memory (two BN-column fp32 accumulators) and
+//               one lane issues tcgen05.mma (M=128, N=BN, K=16) from shared-
+//               memory descriptors; tcgen05.commit frees smem stages and
+//               hands finished accumulators to the epilogue
+//   warps 2-5   epilogue: tcgen05.ld of the warp's 32 TMEM lanes (= tile
+//               rows), activation, bf16/fp32 rows stored to global memory;
+//               predicated on the group's last row so a tile never writes
+//               rows of the next expert
+// The tile list is (group, 128-row tile, N tile), N fastest, walked with a
+// static stride of gridDim.x.  Group row counts come from device memory (no
+// host synchronisation); every CTA rebuilds the tile prefix in shared memory.
+// Every wait is bounded: a wait that gives up records MOE_ERR_DEVICE_TIMEOUT,
+// stops the other roles, drains in-flight copies and MMAs, and frees TMEM.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+
+#include "kernels.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int BM = 128, BK = 64;
+constexpr int kThreads = 192;
+
+struct Params {
+  const int32_t* offsets;  // NULL: a single group of `rows` rows
+  int64_t rows;
+  int G, K, n_per_group, n_out;
+  void* out;
+  int64_t ld_out;
+  const float* bias;
+  Control* ctl;
+};
+
+template <int BN>
+constexpr int stages_for() {
+  return (BN >= 256) ? 4 : (BN >= 128 ? 6 : 8);
+}
+
+template <int BN>
+constexpr uint32_t tmem_cols_for() {
+  return (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128 : (2 * BN <= 256) ? 256 : 512;
+}
+
+template <int BN>
+constexpr size_t smem_bytes_for() {
+  return (size_t)stages_for<BN>() * (BM * BK * 2 + BN * BK * 2) + 1024;
+}
+
+struct TileInfo {
+  int g, row0, rows, nt;
+};
+
+__device__ __forceinline__ TileInfo decode(int tile, int n_tiles, const int* tile_off,
+                                           const int* s_off, int G) {
+  TileInfo ti;
+  const int mt = tile / n_tiles;
+  ti.nt = tile - mt * n_tiles;
+  // first i in [1, G] with tile_off[i] > mt  ->  group i - 1
+  int lo = 1, hi = G;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (tile_off[mid] > mt) hi = mid; else lo = mid + 1;
+  }
+  ti.g = lo - 1;
+  ti.row0 = s_off[ti.g] + (mt - tile_off[ti.g]) * BM;
+  ti.rows = min(BM, s_off[ti.g + 1] - ti.row0);
+  return ti;
+}
+
+__device__ __forceinline__ float silu_mul(float g, float u) {
+  return __fdividef(g, 1.f + __expf(-g)) * u;
+}
+
+template <int BN, int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ Params p) {
+  constexpr int STAGES = stages_for<BN>();
+  constexpr uint32_t A_BYTES = BM * BK * 2;
+  constexpr uint32_t B_BYTES = BN * BK * 2;
+  constexpr uint32_t TMEM_COLS = tmem_cols_for<BN>();
+  constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
+  constexpr uint32_t ACC_STRIDE = TMEM_COLS / 2;  // column distance of the two accumulators
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * A_BYTES;
+
+  __shared__ __align__(8) uint64_t full[STAGES], empty[STAGES], tfull[2], tempty[2], done;
+  __shared__ uint32_t tmem_base_s;
+  __shared__ int tile_off[257];
+  __shared__ int s_off[257];
+  __shared__ volatile int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = p.G;
+
+  // group offsets and the prefix of 128-row tiles per group
+  // offsets clamped to [0, rows]: a malformed offset array can never make
+  // the epilogue store outside the output
+  for (int g = threadIdx.x; g <= G; g += kThreads)
+    s_off[g] = p.offsets ? min(max(__ldg(p.offsets + g), 0), (int)p.rows) : (g == 0 ? 0 : (int)p.rows);
+  if (threadIdx.x == 0) abort_flag = 0;
+  __syncthreads();
+  if (warp == 0) {
+    int carry = 0;
+    for (int g0 = 0; g0 < G; g0 += 32) {
+      const int g = g0 + lane;
+      const int v = g < G ? (max(s_off[g + 1] - s_off[g], 0) + BM - 1) / BM : 0;
+      int incl = v;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+      }
+      if (g < G) tile_off[g] = carry + incl - v;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) {
+      tile_off[G] = carry;
+      for (int s = 0; s < STAGES; ++s) {
+        mbar_init(&full[s], 1);
+        mbar_init(&empty[s], 1);
+      }
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(&tfull[b], 1);
+        mbar_init(&tempty[b], 4);
+      }
+      mbar_init(&done, 1);
+      fence_barrier_init();
+      tma_prefetch_desc(&tmA);
+      tma_prefetch_desc(&tmB);
+    }
+  } else if (warp == 1) {
+    tmem_alloc(&tmem_base_s, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_base_s;
+  const int n_tiles = p.n_per_group / BN;
+  const int total = tile_off[G] * n_tiles;
+  const int kblocks = p.K / BK;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        const TileInfo ti = decode(tile, n_tiles, tile_off, s_off, G);
+        const int brow = ti.g * p.n_per_group + ti.nt * BN;
+        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+          const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
+          if (!mbar_wait_bounded(&empty[s], ph ^ 1, &abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[s], A_BYTES + B_BYTES);
+          tma_load_2d(sA + s * A_BYTES, &tmA, &full[s], kb * BK, ti.row0);
+          tma_load_2d(sB + s * B_BYTES, &tmB, &full[s], kb * BK, brow);
+        }
+      }
+      if (!ok) {
+        abort_flag = 1;
+        record_error(p.ctl, MOE_ERR_DEVICE_TIMEOUT, 0x100u);
+      }
+      // drain: every issued stage completes before the CTA may exit
+      const uint32_t first = it > (uint32_t)STAGES ? it - STAGES : 0;
+      for (uint32_t q = first; q < it; ++q)
+        mbar_wait_bounded(&full[q % STAGES], (q / STAGES) & 1, nullptr);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      uint32_t it = 0, tc = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++tc) {
+        const uint32_t b = tc & 1, tph = (tc >> 1) & 1;
+        if (!mbar_wait_bounded(&tempty[b], tph ^ 1, &abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + b * ACC_STRIDE;
+        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+          const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
+          if (!mbar_wait_bounded(&full[s], ph, &abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + s * A_BYTES);
+          const uint32_t b0 = smem_u32(sB + s * B_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            tc_mma_f16(d_tmem, smem_desc_k128(a0 + kk * 32), smem_desc_k128(b0 + kk * 32), IDESC,
+                       (kb | kk) != 0);
+          tc_commit(&empty[s]);
+        }
+        if (!ok) break;
+        tc_commit(&tfull[b]);
+      }
+      if (!ok) {
+        abort_flag = 1;
+        record_error(p.ctl, MOE_ERR_DEVICE_TIMEOUT, 0x200u);
+      }
+      // all MMAs issued by this thread complete before TMEM is released
+      tc_commit(&done);
+      mbar_wait_bounded(&done, 0, nullptr);
+    }
+  } else {
+    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    const int rr = q * 32 + lane;
+    uint32_t tc = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tc) {
+      const TileInfo ti = decode(tile, n_tiles, tile_off, s_off, G);
+      const uint32_t b = tc & 1, tph = (tc >> 1) & 1;
+      if (!mbar_wait_bounded(&tfull[b], tph, &abort_flag)) {
+        abort_flag = 1;
+        record_error(p.ctl, MOE_ERR_DEVICE_TIMEOUT, 0x300u);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + b * ACC_STRIDE;
+      const bool valid = rr < ti.rows;
+      const int64_t grow = (int64_t)ti.row0 + rr;
+      if constexpr (EPI == kEpiSwiGLU) {
+        constexpr int HALF = BN / 2;
+        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + grow * p.ld_out + ti.nt * HALF;
+#pragma unroll 1
+        for (int c = 0; c < HALF; c += 16) {
+          uint32_t gr[16], ur[16];
+          tmem_ld16(taddr + c, gr);
+          tmem_ld16(taddr + HALF + c, ur);
+          tmem_ld_wait();
+          uint32_t pk[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            pk[i] = pack_bf16x2(silu_mul(__uint_as_float(gr[2 * i]), __uint_as_float(ur[2 * i])),
+                                silu_mul(__uint_as_float(gr[2 * i + 1]), __uint_as_float(ur[2 * i + 1])));
+          if (valid) {
+            uint4* o = reinterpret_cast<uint4*>(out + c);
+            o[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            o[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          }
+        }
+      } else if constexpr (EPI == kEpiBF16) {
+        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + grow * p.ld_out + ti.nt * BN;
+        const int ncols = min(BN, p.n_out - ti.nt * BN);
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 16) {
+          uint32_t r[16];
+          tmem_ld16(taddr + c, r);
+          tmem_ld_wait();
+          uint32_t pk[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+          if (valid && c < ncols) {
+            uint4* o = reinterpret_cast<uint4*>(out + c);
+            o[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            o[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          }
+        }
+      } else {
+        float* out = static_cast<float*>(p.out) + grow * p.ld_out;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 16) {
+          uint32_t r[16];
+          tmem_ld16(taddr + c, r);
+          tmem_ld_wait();
+          if (valid) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int col = c + i;
+              if (col < p.n_out) out[col] = __uint_as_float(r[i]) + (p.bias ? __ldg(p.bias + col) : 0.f);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[b]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// 2-D bf16 K-major operand [rows, K]: box of 64 K-elements (128 B) x box_rows
+bool make_map(CUtensorMap* m, const void* base, int64_t rows, int K, int box_rows) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+  cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int BN, int EPI>
+cudaError_t run(const GemmArgs& a, cudaStream_t s) {
+  static bool attr_set = false;
+  constexpr size_t smem = smem_bytes_for<BN>();
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  CUtensorMap mA, mB;
+  if (!make_map(&mA, a.A, a.rows, a.K, BM)) return cudaErrorInvalidValue;
+  if (!make_map(&mB, a.B, (int64_t)a.G * a.n_per_group, a.K, BN)) return cudaErrorInvalidValue;
+  Params p;
+  p.offsets = a.offsets;
+  p.rows = a.rows;
+  p.G = a.offsets ? a.G : 1;
+  p.K = a.K;
+  p.n_per_group = a.n_per_group;
+  p.n_out = a.n_out;
+  p.out = a.out;
+  p.ld_out = a.ld_out;
+  p.bias = a.bias;
+  p.ctl = a.ctl;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // upper bound of the tile count: every group adds at most one partial tile
+  const int64_t mt_max = (a.rows + BM - 1) / BM + a.G;
+  const int64_t tiles_max = mt_max * (a.n_per_group / BN);
+  const int grid = (int)std::min<int64_t>(tiles_max, sms);
+  if (grid <= 0) return cudaSuccess;
+  gemm_tc_kernel<BN, EPI><<<grid, kThreads, smem, s>>>(mA, mB, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_tc(int epi, int bn, const GemmArgs& a, cudaStream_t s) {
+  if (a.rows == 0) return cudaSuccess;
+#define MOE_GEMM_CASE(EPI, BN) \
+  if (epi == EPI && bn == BN) return run<BN, EPI>(a, s);
+  MOE_GEMM_CASE(kEpiSwiGLU, 256)
+  MOE_GEMM_CASE(kEpiSwiGLU, 128)
+  MOE_GEMM_CASE(kEpiBF16, 256)
+  MOE_GEMM_CASE(kEpiBF16, 128)
+  MOE_GEMM_CASE(kEpiBF16, 64)
+  MOE_GEMM_CASE(kEpiLogits, 16)
+  MOE_GEMM_CASE(kEpiLogits, 32)
+  MOE_GEMM_CASE(kEpiLogits, 48)
+  MOE_GEMM_CASE(kEpiLogits, 64)
+  MOE_GEMM_CASE(kEpiLogits, 80)
+  MOE_GEMM_CASE(kEpiLogits, 96)
+  MOE_GEMM_CASE(kEpiLogits, 112)
+  MOE_GEMM_CASE(kEpiLogits, 128)
+  MOE_GEMM_CASE(kEpiLogits, 144)
+  MOE_GEMM_CASE(kEpiLogits, 160)
+  MOE_GEMM_CASE(kEpiLogits, 176)
+  MOE_GEMM_CASE(kEpiLogits, 192)
+  MOE_GEMM_CASE(kEpiLogits, 208)
+  MOE_GEMM_CASE(kEpiLogits, 224)
+  MOE_GEMM_CASE(kEpiLogits, 240)
+  MOE_GEMM_CASE(kEpiLogits, 256)
+#undef MOE_GEMM_CASE
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace moe

@@ -1,0 +1,75 @@
+// kernels.cuh - launchers shared between the kernel files and the C ABI.
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+// expert -> rank map passed by value to the layout kernels (E <= 256,
+// ep <= 256, so a rank fits one byte)
+struct RankMap {
+  uint8_t r[256];
+};
+
+// ---- route.cu
+cudaError_t launch_topk(const float* logits, int64_t T, int E, int k, int32_t* idx, float* gate,
+                        cudaStream_t s);
+cudaError_t launch_router_f32(const float* x, const float* wrT, const float* bias, int64_t T,
+                              int d, int E, float* logits, cudaStream_t s);
+
+// ---- layout.cu
+constexpr int kTokPerBlock = 512;        // tokens per lookback block
+constexpr int kLayoutThreads = 256;
+constexpr int kMaxBins = 256 + 256 + 2;  // experts + ranks + two stat counters
+
+inline int layout_blocks(int64_t T) { return (int)((T + kTokPerBlock - 1) / kTokPerBlock); }
+inline int layout_bins(int E, int ep) { return E + (ep > 1 ? ep : 0) + 2; }
+
+struct LayoutOut {
+  int32_t *counts, *offsets, *row_token, *slot_row;
+  int32_t *rank_counts, *rank_offsets, *send_token, *slot_send_row;
+  moe_stats* stats;
+};
+
+cudaError_t launch_layout(const int32_t* idx, int64_t T, int k, int E, int ep, const RankMap& map,
+                          const LayoutOut& out, Control* ctl, uint64_t* status_words,
+                          int32_t* prefix, int32_t* totals, int stall_block, int64_t limit_ns,
+                          cudaStream_t s);
+
+// ---- permute_combine.cu
+cudaError_t launch_permute(const void* x, const int32_t* row_token, void* x_perm, int64_t T,
+                           int64_t R, uint32_t row_bytes, cudaStream_t s);
+cudaError_t launch_combine(int dtype, const void* y_perm, const int32_t* slot_row,
+                           const float* gate, void* y, int64_t T, int d, int k, cudaStream_t s);
+
+// ---- gemm_tc.cu (bf16, tcgen05)
+// Grouped GEMM  out[r, :] = epilogue(A[r, :] . B_g^T)  for rows r of group g
+// (rows [offsets[g], offsets[g+1])), with B_g rows [g*n_per_group, ...).
+enum Epilogue { kEpiSwiGLU = 0, kEpiBF16 = 1, kEpiLogits = 2 };
+struct GemmArgs {
+  const void* A;           // [rows, K] bf16 row-major
+  int64_t rows;            // rows of A (tensor-map extent)
+  const void* B;           // [G * n_per_group, K] bf16 row-major (K-major)
+  const int32_t* offsets;  // [G+1] device, or NULL: one group of all `rows`
+  int G;
+  int K;
+  int n_per_group;
+  int n_out;               // valid output columns
+  void* out;
+  int64_t ld_out;          // output row stride in elements
+  const float* bias;       // kEpiLogits only, may be NULL
+  Control* ctl;
+};
+cudaError_t launch_gemm_tc(int epi, int bn, const GemmArgs& a, cudaStream_t s);
+
+// ---- gemm_simt.cu (fp32, CUDA cores)
+cudaError_t launch_grouped_f32(const float* x_perm, const int32_t* offsets, int E, int64_t R,
+                               int d, int f, int blk, const float* wgu, const float* wdT, float* h,
+                               float* y_perm, cudaStream_t s);
+
+// ---- pack.cu
+cudaError_t launch_pack(int dtype, int d, int E, int f, int blk, int E16, const void* w_router,
+                        const void* w_gate, const void* w_up, const void* w_down, void* wrT,
+                        void* wgu, void* wdT, cudaStream_t s);
+
+}  // namespace moe

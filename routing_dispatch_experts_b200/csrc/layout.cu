@@ -1,0 +1,365 @@
+// layout.cu - expert-grouped dispatch layout and the deduplicated send layout.
+//
+// Two kernels over blocks of kTokPerBlock tokens (all k assignments of a
+// token stay in one block):
+//
+//  1. histogram + decoupled lookback: each block counts its assignments per
+//     expert, its distinct (token, rank) pairs per rank, and two statistics;
+//     it publishes its counts and walks back over its predecessors' published
+//     aggregates / inclusive prefixes to get its exclusive prefix in every bin
+//     (single pass, dynamic block ids from a ticket counter, so a block only
+//     ever waits on blocks that are already running).  Waits are bounded.
+//  2. stable scatter: expert offsets from the totals, then every warp places
+//     its contiguous run of assignments in flat-index order (match_any ranks
+//     equal experts inside a 32-wide step), giving rows ordered by
+//     (expert, t*k+j); send rows ordered by (rank, token) likewise, one per
+//     distinct rank of a token.
+//
+// Deduplicated send layout: "Expert Coupling in MoE Pretraining", Abstract
+// (each token is sent to each GPU once) and Table I (GPUs per token = distinct
+// destinations; deduplication = rows removed as duplicates; T/EP tokens per
+// GPU for the home rank).
+#include "kernels.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr uint32_t kFlagNone = 0, kFlagAgg = 1, kFlagIncl = 2, kFlagErr = 3;
+constexpr int kWarps = kLayoutThreads / 32;
+constexpr int kTokPerWarp = kTokPerBlock / kWarps;
+
+struct Params {
+  const int32_t* idx;
+  int64_t T;
+  int k, E, ep, nb, bins, stall_block;
+  int64_t limit_ns;
+  RankMap map;
+  Control* ctl;
+  uint64_t* status;  // [nb][bins]
+  int32_t* prefix;   // [nb][bins]
+  int32_t* totals;   // [bins]
+  LayoutOut out;
+};
+
+__device__ __forceinline__ void publish(uint64_t* w, uint32_t flag, uint32_t value) {
+  atomicExch(reinterpret_cast<unsigned long long*>(w),
+             ((unsigned long long)flag << 32) | (unsigned long long)value);
+}
+
+__device__ __forceinline__ uint64_t poll(const uint64_t* w) {
+  return *reinterpret_cast<const volatile unsigned long long*>(w);
+}
+
+__global__ void __launch_bounds__(kLayoutThreads) layout_hist_kernel(const __grid_constant__ Params p) {
+  __shared__ int hist[kMaxBins];
+  __shared__ int s_ticket;
+  const int tid = threadIdx.x;
+  for (int i = tid; i < p.bins; i += kLayoutThreads) hist[i] = 0;
+  if (tid == 0) s_ticket = (int)atomicAdd(&p.ctl->ticket, 1u);
+  __syncthreads();
+  const int b = s_ticket;
+  if (b >= p.nb) {  // the workspace was not zero-filled before first use
+    if (tid == 0) record_error(p.ctl, MOE_ERR_WORKSPACE, (uint32_t)b);
+    return;
+  }
+  const int64_t t0 = (int64_t)b * kTokPerBlock;
+  const int64_t t1 = min(p.T, t0 + kTokPerBlock);
+  const int ebin_r = p.E;                                // first rank bin
+  const int sbin = p.E + (p.ep > 1 ? p.ep : 0);          // the two stat bins
+  int single = 0, home = 0;
+  for (int64_t t = t0 + tid; t < t1; t += kLayoutThreads) {
+    const int home_r = (int)((t * p.ep) / p.T);
+    int rs[16];
+    int nr = 0;
+    for (int j = 0; j < p.k; ++j) {
+      const int e = __ldg(p.idx + t * p.k + j);
+      if ((unsigned)e >= (unsigned)p.E) {
+        record_error(p.ctl, MOE_ERR_DEVICE_INDEX, (uint32_t)(t * p.k + j));
+        continue;
+      }
+      atomicAdd(&hist[e], 1);
+      const int r = p.ep > 1 ? p.map.r[e] : 0;
+      home += r == home_r;
+      bool seen = false;
+      for (int q = 0; q < nr; ++q) seen |= rs[q] == r;
+      if (!seen) {
+        rs[nr++] = r;
+        if (p.ep > 1) atomicAdd(&hist[ebin_r + r], 1);
+      }
+    }
+    single += nr == 1;
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    single += __shfl_xor_sync(0xffffffffu, single, off);
+    home += __shfl_xor_sync(0xffffffffu, home, off);
+  }
+  if ((tid & 31) == 0) {
+    atomicAdd(&hist[sbin], single);
+    atomicAdd(&hist[sbin + 1], home);
+  }
+  __syncthreads();
+
+  // decoupled lookback, one bin per thread
+  const bool stalled = b == p.stall_block;
+  for (int bin = tid; bin < p.bins; bin += kLayoutThreads) {
+    const uint32_t agg = (uint32_t)hist[bin];
+    uint64_t* mine = p.status + (size_t)b * p.bins + bin;
+    uint32_t excl = 0;
+    if (b > 0) {
+      if (!stalled) publish(mine, kFlagAgg, agg);
+      bool ok = true;
+      for (int q = b - 1; q >= 0;) {
+        uint64_t w = poll(p.status + (size_t)q * p.bins + bin);
+        if ((uint32_t)(w >> 32) == kFlagNone) {
+          const uint64_t ts = globaltimer_ns();
+          do {
+            __nanosleep(64);
+            w = poll(p.status + (size_t)q * p.bins + bin);
+            if ((uint32_t)(w >> 32) != kFlagNone) break;
+          } while (globaltimer_ns() - ts <= (uint64_t)p.limit_ns);
+          if ((uint32_t)(w >> 32) == kFlagNone) {
+            ok = false;
+            break;
+          }
+        }
+        const uint32_t fl = (uint32_t)(w >> 32);
+        if (fl == kFlagErr) {
+          ok = false;
+          break;
+        }
+        excl += (uint32_t)w;
+        if (fl == kFlagIncl) break;
+        --q;
+      }
+      if (!ok) {
+        record_error(p.ctl, MOE_ERR_DEVICE_TIMEOUT, (uint32_t)b);
+        if (!stalled) publish(mine, kFlagErr, 0);
+        continue;
+      }
+    }
+    if (!stalled) publish(mine, kFlagIncl, excl + agg);
+    p.prefix[(size_t)b * p.bins + bin] = (int32_t)excl;
+    if (b == p.nb - 1) p.totals[bin] = (int32_t)(excl + agg);
+  }
+}
+
+__device__ __forceinline__ uint32_t lanemask_lt() {
+  uint32_t m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+__global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(const __grid_constant__ Params p) {
+  __shared__ int s_off[kMaxBins + 2];  // expert offsets [E+1], then rank offsets [ep+1]
+  __shared__ int wh[kWarps][kMaxBins];
+  __shared__ int s_ok;
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int b = blockIdx.x;
+  const int E = p.E, ep = p.ep, k = p.k;
+  const bool dedup = ep > 1;
+  const int sbin = E + (dedup ? ep : 0);
+
+  // leave the lookback state clean for the next call (stream order puts this
+  // after every block of the histogram kernel)
+  for (int i = tid; i < p.bins; i += kLayoutThreads) p.status[(size_t)b * p.bins + i] = 0;
+  if (b == 0 && tid == 0) p.ctl->ticket = 0;
+  if (tid == 0) s_ok = *reinterpret_cast<volatile uint32_t*>(&p.ctl->status) == MOE_OK;
+  __syncthreads();
+  if (!s_ok) return;
+
+  // exclusive scans of the expert totals and the rank totals (one warp each)
+  if (warp < 2) {
+    const int n = warp == 0 ? E : (dedup ? ep : 0);
+    const int base_bin = warp == 0 ? 0 : E;
+    int* dst = warp == 0 ? s_off : s_off + E + 1;
+    if (n > 0) {
+      int carry = 0;
+      for (int c0 = 0; c0 < n; c0 += 32) {
+        const int i = c0 + lane;
+        const int v = i < n ? p.totals[base_bin + i] : 0;
+        int incl = v;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const int o = __shfl_up_sync(0xffffffffu, incl, off);
+          if (lane >= off) incl += o;
+        }
+        if (i < n) dst[i] = carry + incl - v;
+        carry += __shfl_sync(0xffffffffu, incl, 31);
+      }
+      if (lane == 0) dst[n] = carry;
+    }
+  }
+  __syncthreads();
+
+  if (b == 0) {
+    for (int e = tid; e < E; e += kLayoutThreads) {
+      p.out.counts[e] = p.totals[e];
+      p.out.offsets[e] = s_off[e];
+    }
+    if (tid == 0) p.out.offsets[E] = s_off[E];
+    if (dedup) {
+      for (int r = tid; r < ep; r += kLayoutThreads) {
+        p.out.rank_counts[r] = p.totals[E + r];
+        p.out.rank_offsets[r] = s_off[E + 1 + r];
+      }
+      if (tid == 0) p.out.rank_offsets[ep] = s_off[E + 1 + ep];
+    }
+    if (p.out.stats && warp == 0) {
+      int mx = 0, mn = 0x7FFFFFFF;
+      for (int e = lane; e < E; e += 32) {
+        mx = max(mx, p.totals[e]);
+        mn = min(mn, p.totals[e]);
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+      }
+      if (lane == 0) {
+        moe_stats st;
+        st.rows_sent = dedup ? (int64_t)s_off[E + 1 + ep] : 0;
+        st.dup_removed = dedup ? p.T * k - st.rows_sent : 0;
+        st.tokens_single_rank = p.totals[sbin];
+        st.home_rank_rows = p.totals[sbin + 1];
+        st.max_expert_rows = mx;
+        st.min_expert_rows = E > 0 ? mn : 0;
+        *p.out.stats = st;
+      }
+    }
+  }
+
+  // per-warp histograms of this block's assignments / send rows
+  for (int i = tid; i < kWarps * kMaxBins; i += kLayoutThreads) (&wh[0][0])[i] = 0;
+  __syncthreads();
+  const int64_t tb0 = (int64_t)b * kTokPerBlock;
+  const int64_t tw0 = min(p.T, tb0 + (int64_t)warp * kTokPerWarp);
+  const int64_t tw1 = min(p.T, tw0 + kTokPerWarp);
+  const int64_t aw0 = tw0 * k, aw1 = tw1 * k;
+  for (int64_t a = aw0 + lane; a < aw1; a += 32) atomicAdd(&wh[warp][__ldg(p.idx + a)], 1);
+  if (dedup) {
+    for (int64_t t = tw0 + lane; t < tw1; t += 32) {
+      int rs[16];
+      int nr = 0;
+      for (int j = 0; j < k; ++j) {
+        const int r = p.map.r[__ldg(p.idx + t * k + j)];
+        bool seen = false;
+        for (int q = 0; q < nr; ++q) seen |= rs[q] == r;
+        if (!seen) {
+          rs[nr++] = r;
+          atomicAdd(&wh[warp][E + r], 1);
+        }
+      }
+    }
+  }
+  __syncthreads();
+  // warp-exclusive starting rows: global offset + this block's lookback
+  // prefix + the counts of the block's earlier warps
+  const int nbins_used = E + (dedup ? ep : 0);
+  for (int bin = tid; bin < nbins_used; bin += kLayoutThreads) {
+    int run = (bin < E ? s_off[bin] : s_off[E + 1 + (bin - E)]) +
+              p.prefix[(size_t)b * p.bins + bin];
+    for (int w = 0; w < kWarps; ++w) {
+      const int c = wh[w][bin];
+      wh[w][bin] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+
+  // stable scatter of the assignments, in flat-index order
+  const uint32_t lt = lanemask_lt();
+  for (int64_t a0 = aw0; a0 < aw1; a0 += 32) {
+    const int64_t a = a0 + lane;
+    const bool valid = a < aw1;
+    const int e = valid ? __ldg(p.idx + a) : -1;
+    const uint32_t peers = __match_any_sync(0xffffffffu, e);
+    if (valid) {
+      const int row = wh[warp][e] + __popc(peers & lt);
+      p.out.row_token[row] = (int32_t)(a / k);
+      p.out.slot_row[a] = row;
+    }
+    __syncwarp();
+    if (valid && lane == __ffs(peers) - 1) wh[warp][e] += __popc(peers);
+    __syncwarp();
+  }
+
+  // deduplicated send rows, tokens in order, one row per distinct rank
+  if (dedup) {
+    const int nw = (ep + 31) >> 5;
+    for (int64_t tt = tw0; tt < tw1; tt += 32) {
+      const int64_t t = tt + lane;
+      const bool valid = t < tw1;
+      uint32_t m[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) m[i] = 0;
+      if (valid)
+        for (int j = 0; j < k; ++j) {
+          const int r = p.map.r[__ldg(p.idx + t * k + j)];
+          m[r >> 5] |= 1u << (r & 31);
+        }
+      for (int i = 0; i < nw; ++i) {
+        uint32_t u = __reduce_or_sync(0xffffffffu, m[i]);
+        while (u) {
+          const int r = (i << 5) + __ffs(u) - 1;
+          u &= u - 1;
+          const bool has = (m[i] >> (r & 31)) & 1u;
+          const uint32_t bal = __ballot_sync(0xffffffffu, has);
+          if (has) {
+            const int srow = wh[warp][E + r] + __popc(bal & lt);
+            p.out.send_token[srow] = (int32_t)t;
+            for (int j = 0; j < k; ++j)
+              if (p.map.r[__ldg(p.idx + t * k + j)] == r) p.out.slot_send_row[t * k + j] = srow;
+          }
+          __syncwarp();
+          if (lane == 0) wh[warp][E + r] += __popc(bal);
+          __syncwarp();
+        }
+      }
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_layout(const int32_t* idx, int64_t T, int k, int E, int ep, const RankMap& map,
+                          const LayoutOut& out, Control* ctl, uint64_t* status_words,
+                          int32_t* prefix, int32_t* totals, int stall_block, int64_t limit_ns,
+                          cudaStream_t s) {
+  Params p;
+  p.idx = idx;
+  p.T = T;
+  p.k = k;
+  p.E = E;
+  p.ep = ep;
+  p.nb = layout_blocks(T);
+  p.bins = layout_bins(E, ep);
+  p.stall_block = stall_block;
+  p.limit_ns = limit_ns;
+  p.map = map;
+  p.ctl = ctl;
+  p.status = status_words;
+  p.prefix = prefix;
+  p.totals = totals;
+  p.out = out;
+  if (p.nb == 0) {
+    // no tokens: counts and offsets are all zero, no send rows
+    cudaError_t err = cudaMemsetAsync(out.counts, 0, sizeof(int32_t) * E, s);
+    if (err == cudaSuccess) err = cudaMemsetAsync(out.offsets, 0, sizeof(int32_t) * (E + 1), s);
+    if (err == cudaSuccess && ep > 1) {
+      err = cudaMemsetAsync(out.rank_counts, 0, sizeof(int32_t) * ep, s);
+      if (err == cudaSuccess) err = cudaMemsetAsync(out.rank_offsets, 0, sizeof(int32_t) * (ep + 1), s);
+    }
+    if (err == cudaSuccess && out.stats) err = cudaMemsetAsync(out.stats, 0, sizeof(moe_stats), s);
+    return err;
+  }
+  layout_hist_kernel<<<p.nb, kLayoutThreads, 0, s>>>(p);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  layout_scatter_kernel<<<p.nb, kLayoutThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,200 @@
+// permute_combine.cu - the two data-movement steps around the experts.
+//
+//  permute: x_perm[r] = x[row_token[r]]  (dispatch of token rows to their
+//           experts' contiguous row ranges; "Expert Coupling in MoE
+//           Pretraining", Abstract: dispatch tokens to their experts)
+//  combine: y[t] = sum_j gate[t,j] * y_perm[slot_row[t*k+j]]  (gather the
+//           expert outputs back and weight them by the gates)
+#include <algorithm>
+
+#include "kernels.cuh"
+
+namespace moe {
+
+namespace {
+
+// ---------------------------------------------------------------- permute
+// One warp per CTA.  Rows move in groups of `rps` rows (one group fills a
+// 16 KB shared-memory stage); lane i of the warp owns row i of every group.
+// Lane i issues a TMA bulk load of its source row into the stage (completing
+// on the stage's mbarrier), then, LOOKAHEAD groups later, a TMA bulk store of
+// the staged row to its destination.  A lane reuses a stage region only after
+// its own bulk store from that region has finished reading (bulk-group wait),
+// so loads of group g+LOOKAHEAD overlap the stores of group g.
+constexpr int kPermStages = 4;
+constexpr int kPermLookahead = 2;
+constexpr uint32_t kPermStageBytes = 16384;
+constexpr int kPermCtasPerSm = 3;
+
+__global__ void __launch_bounds__(32) permute_kernel(const uint8_t* __restrict__ x,
+                                                     const int32_t* __restrict__ row_token,
+                                                     uint8_t* __restrict__ x_perm, int64_t R,
+                                                     int64_t T, uint32_t row_bytes, int rps) {
+  extern __shared__ __align__(128) uint8_t stage[];
+  __shared__ __align__(8) uint64_t full[kPermStages];
+  const int lane = threadIdx.x;
+  if (lane == 0) {
+    for (int s = 0; s < kPermStages; ++s) mbar_init(&full[s], 1);
+    fence_barrier_init();
+  }
+  __syncwarp();
+  const int64_t ngroups = (R + rps - 1) / rps;
+  const int64_t nmine = ngroups > blockIdx.x ? (ngroups - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+  for (int64_t i = 0; i < nmine + kPermLookahead; ++i) {
+    if (i < nmine) {
+      const int s = (int)(i % kPermStages);
+      const int64_t g = blockIdx.x + i * gridDim.x;
+      const int64_t r0 = g * rps;
+      const int n = (int)(R - r0 < rps ? R - r0 : rps);
+      // this lane's store of group i - kPermStages read the same region
+      bulk_wait_read<kPermStages - kPermLookahead - 1>();
+      if (lane == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)n * row_bytes);
+      __syncwarp();
+      if (lane < n) {
+        // an out-of-range token (malformed input) reads row 0 instead of
+        // faulting; the result is then unspecified, as documented
+        int64_t src = __ldg(row_token + r0 + lane);
+        if (src < 0 || src >= T) src = 0;
+        bulk_load(stage + (size_t)s * kPermStageBytes + (size_t)lane * row_bytes,
+                  x + src * row_bytes, row_bytes, &full[s]);
+      }
+    }
+    const int64_t j = i - kPermLookahead;
+    if (j >= 0 && j < nmine) {
+      const int s = (int)(j % kPermStages);
+      const int64_t g = blockIdx.x + j * gridDim.x;
+      const int64_t r0 = g * rps;
+      const int n = (int)(R - r0 < rps ? R - r0 : rps);
+      // the loads of a group complete on the stage barrier; bounded wait
+      if (!mbar_wait_bounded(&full[s], (uint32_t)((j / kPermStages) & 1), nullptr)) {
+        // never expected: a bulk load did not land within the limit
+        break;
+      }
+      if (lane < n)
+        bulk_store(x_perm + (r0 + lane) * row_bytes,
+                   stage + (size_t)s * kPermStageBytes + (size_t)lane * row_bytes, row_bytes);
+      bulk_commit();
+    }
+  }
+  bulk_wait<0>();
+}
+
+// ---------------------------------------------------------------- combine
+// One thread per 16-byte output vector (8 bf16 or 4 fp32 of one token's
+// row): it reads the token's k slot rows and gates, loads the k matching
+// vectors of y_perm and sums gate * value in fp32 with j ascending, then
+// rounds once.  Consecutive threads cover consecutive vectors of a row.
+template <typename T>
+struct Vec;
+template <>
+struct Vec<__nv_bfloat16> {
+  static constexpr int N = 8;
+  __device__ static void acc(float* a, const uint4& q, float g) {
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      a[2 * i] = fmaf(g, bf16_lo(w[i]), a[2 * i]);
+      a[2 * i + 1] = fmaf(g, bf16_hi(w[i]), a[2 * i + 1]);
+    }
+  }
+  __device__ static uint4 pack(const float* a) {
+    return make_uint4(pack_bf16x2(a[0], a[1]), pack_bf16x2(a[2], a[3]), pack_bf16x2(a[4], a[5]),
+                      pack_bf16x2(a[6], a[7]));
+  }
+};
+template <>
+struct Vec<float> {
+  static constexpr int N = 4;
+  __device__ static void acc(float* a, const uint4& q, float g) {
+    a[0] = fmaf(g, __uint_as_float(q.x), a[0]);
+    a[1] = fmaf(g, __uint_as_float(q.y), a[1]);
+    a[2] = fmaf(g, __uint_as_float(q.z), a[2]);
+    a[3] = fmaf(g, __uint_as_float(q.w), a[3]);
+  }
+  __device__ static uint4 pack(const float* a) {
+    return make_uint4(__float_as_uint(a[0]), __float_as_uint(a[1]), __float_as_uint(a[2]),
+                      __float_as_uint(a[3]));
+  }
+};
+
+template <typename T>
+__global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ y_perm,
+                                                      const int32_t* __restrict__ slot_row,
+                                                      const float* __restrict__ gate,
+                                                      uint4* __restrict__ y, int64_t Tn, int V,
+                                                      int k) {
+  const int64_t n = Tn * V;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = i / V;
+    const int v = (int)(i - t * V);
+    float a[Vec<T>::N];
+#pragma unroll
+    for (int q = 0; q < Vec<T>::N; ++q) a[q] = 0.f;
+    int j = 0;
+    for (; j + 4 <= k; j += 4) {
+      uint4 q[4];
+      float g[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        int64_t row = __ldg(slot_row + t * k + j + u);
+        if (row < 0 || row >= Tn * k) row = 0;
+        g[u] = gate ? __ldg(gate + t * k + j + u) : 1.f;
+        q[u] = __ldg(y_perm + row * V + v);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) Vec<T>::acc(a, q[u], g[u]);
+    }
+    for (; j < k; ++j) {
+      int64_t row = __ldg(slot_row + t * k + j);
+      if (row < 0 || row >= Tn * k) row = 0;
+      const float g = gate ? __ldg(gate + t * k + j) : 1.f;
+      Vec<T>::acc(a, __ldg(y_perm + row * V + v), g);
+    }
+    y[i] = Vec<T>::pack(a);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_permute(const void* x, const int32_t* row_token, void* x_perm, int64_t T,
+                           int64_t R, uint32_t row_bytes, cudaStream_t s) {
+  if (R == 0) return cudaSuccess;
+  static bool attr_set = false;
+  const int smem = kPermStages * (int)kPermStageBytes;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int rps = (int)std::min<uint32_t>(32u, kPermStageBytes / row_bytes);
+  const int64_t ngroups = (R + rps - 1) / rps;
+  const int grid = (int)std::min<int64_t>(ngroups, (int64_t)sms * kPermCtasPerSm);
+  permute_kernel<<<grid, 32, smem, s>>>(static_cast<const uint8_t*>(x), row_token,
+                                        static_cast<uint8_t*>(x_perm), R, T, row_bytes, rps);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(int dtype, const void* y_perm, const int32_t* slot_row,
+                           const float* gate, void* y, int64_t T, int d, int k, cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  const int esz = dtype == MOE_BF16 ? 2 : 4;
+  const int V = d * esz / 16;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t n = T * V;
+  const int grid = (int)std::min<int64_t>((n + 255) / 256, (int64_t)sms * 8);
+  if (dtype == MOE_BF16)
+    combine_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(static_cast<const uint4*>(y_perm), slot_row,
+                                                       gate, static_cast<uint4*>(y), T, V, k);
+  else
+    combine_kernel<float><<<grid, 256, 0, s>>>(static_cast<const uint4*>(y_perm), slot_row, gate,
+                                               static_cast<uint4*>(y), T, V, k);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,136 @@
+// route.cu - top-k expert selection with softmax gates, and the fp32 router.
+//
+// Top-k routing with softmax gates renormalised over the k ("MoE Pretraining:
+// Parallelism Layout Changes the Model, Not Quality", Methodology / Models
+// and Data: top-4 routing; "Revisiting MoE and Dense Speed-Accuracy
+// Comparisons", 2.1 Architecture: Top-K routing).
+#include "kernels.cuh"
+
+namespace moe {
+
+// One warp per token.  Lane l holds logits e = l, l+32, ... (VPL of them) in
+// registers.  k rounds: every lane proposes its best remaining expert under
+// the key (logit desc, index asc); a butterfly of shuffles finds the warp's
+// best; its owner marks it taken.  The key is a total order, so every lane
+// ends each round with the same winner.  Equal logits (-0.0 == +0.0 too)
+// resolve to the lower index because the comparison is the IEEE one.
+// Gates: softmax of the chosen logits, exp(l_j - l_0) / sum_i exp(l_i - l_0),
+// the sum reduced by the same butterfly in every lane (deterministic).
+template <int VPL>
+__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int64_t T,
+                                                   int E, int k, int32_t* __restrict__ idx,
+                                                   float* __restrict__ gate) {
+  const int lane = threadIdx.x & 31;
+  const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;  // uniform per warp
+  const float* row = logits + t * E;
+  float v[VPL];
+#pragma unroll
+  for (int c = 0; c < VPL; ++c) {
+    const int e = lane + 32 * c;
+    v[c] = e < E ? __ldg(row + e) : 0.f;
+  }
+  uint32_t taken = 0;
+  float my_l = 0.f;
+  int my_e = 0;
+  for (int j = 0; j < k; ++j) {
+    float bv = -INFINITY;
+    int bi = 0x7FFFFFFF;
+#pragma unroll
+    for (int c = 0; c < VPL; ++c) {
+      const int e = lane + 32 * c;
+      if (e < E && !((taken >> c) & 1u)) {
+        if (bi == 0x7FFFFFFF || v[c] > bv) {  // e ascending: keep the first of equals
+          bv = v[c];
+          bi = e;
+        }
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+      if (ov > bv || (ov == bv && oi < bi)) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+    if (lane == j) {
+      my_l = bv;
+      my_e = bi;
+    }
+  }
+  const float l0 = __shfl_sync(0xffffffffu, my_l, 0);
+  float ex = lane < k ? expf(my_l - l0) : 0.f;
+  float z = ex;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
+  if (lane < k) {
+    idx[t * k + lane] = my_e;
+    gate[t * k + lane] = ex / z;
+  }
+}
+
+cudaError_t launch_topk(const float* logits, int64_t T, int E, int k, int32_t* idx, float* gate,
+                        cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  const int warps = 8;
+  const unsigned grid = (unsigned)((T + warps - 1) / warps);
+  const int vpl = (E + 31) / 32;
+  switch (vpl) {
+#define MOE_TOPK_CASE(N) \
+  case N:                \
+    topk_kernel<N><<<grid, warps * 32, 0, s>>>(logits, T, E, k, idx, gate); \
+    break;
+    MOE_TOPK_CASE(1)
+    MOE_TOPK_CASE(2)
+    MOE_TOPK_CASE(3)
+    MOE_TOPK_CASE(4)
+    MOE_TOPK_CASE(5)
+    MOE_TOPK_CASE(6)
+    MOE_TOPK_CASE(7)
+    MOE_TOPK_CASE(8)
+#undef MOE_TOPK_CASE
+    default:
+      return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+// fp32 router on CUDA cores: logits[t,e] = sum_i x[t,i] W_r^T[e,i] + bias[e],
+// one thread per (t, e), i ascending.  Threads of a warp share t (the x row is
+// a broadcast) and walk consecutive experts.
+__global__ void __launch_bounds__(256) router_f32_kernel(const float* __restrict__ x,
+                                                         const float* __restrict__ wrT,
+                                                         const float* __restrict__ bias,
+                                                         int64_t T, int d, int E,
+                                                         float* __restrict__ logits) {
+  const int64_t o = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (o >= T * E) return;
+  const int64_t t = o / E;
+  const int e = (int)(o % E);
+  const float4* xr = reinterpret_cast<const float4*>(x + t * d);
+  const float4* wr = reinterpret_cast<const float4*>(wrT + (int64_t)e * d);
+  float s = 0.f;
+  for (int i = 0; i < d / 4; ++i) {
+    const float4 a = __ldg(xr + i);
+    const float4 b = __ldg(wr + i);
+    s = fmaf(a.x, b.x, s);
+    s = fmaf(a.y, b.y, s);
+    s = fmaf(a.z, b.z, s);
+    s = fmaf(a.w, b.w, s);
+  }
+  if (bias) s += bias[e];
+  logits[o] = s;
+}
+
+cudaError_t launch_router_f32(const float* x, const float* wrT, const float* bias, int64_t T,
+                              int d, int E, float* logits, cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  const int64_t n = T * E;
+  router_f32_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(x, wrT, bias, T, d, E, logits);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

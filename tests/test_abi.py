@@ -1,0 +1,114 @@
+"""The C-ABI library builds, loads without a GPU, and exports every entry
+point that include/moe.h declares; host-side argument checks answer without
+launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import routing_dispatch_experts_b200 as moe
+from routing_dispatch_experts_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return re.findall(r"^\s*(?:MOE_API\s+)?(?:const\s+char\s*\*|moe_status)\s+(moe_\w+)\s*\(", src, flags=re.M)
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return moe.lib()
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for n in ("moe_route", "moe_dispatch_layout", "moe_permute", "moe_grouped_swiglu",
+              "moe_combine", "moe_forward"):
+        assert n in names
+    assert sorted(names) == sorted(moe.SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol(L):
+    for n in _declared():
+        assert hasattr(L, n), n
+
+
+def test_status_strings(L):
+    for code, name in moe.STATUS_NAMES.items():
+        assert L.moe_status_string(code).decode() == name
+
+
+def _size(fn, **kw):
+    s = moe.moe_shape(**{**dict(T=2048, d=256, E=16, k=4, f=256, ep=1, dtype=moe.MOE_F32), **kw})
+    n = ctypes.c_size_t(0)
+    return fn(ctypes.byref(s), ctypes.byref(n)), n.value
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(), moe.MOE_OK),
+    (dict(E=0), moe.MOE_ERR_INVALID_ARG),
+    (dict(E=257), moe.MOE_ERR_INVALID_ARG),
+    (dict(k=0), moe.MOE_ERR_INVALID_ARG),
+    (dict(k=17, E=64), moe.MOE_ERR_INVALID_ARG),
+    (dict(k=5, E=4), moe.MOE_ERR_INVALID_ARG),
+    (dict(ep=3), moe.MOE_ERR_INVALID_ARG),     # 16 % 3 != 0
+    (dict(ep=32), moe.MOE_ERR_INVALID_ARG),    # more ranks than experts
+    (dict(T=-1), moe.MOE_ERR_INVALID_ARG),
+    (dict(T=1 << 29, k=4), moe.MOE_ERR_INVALID_ARG),  # T*k >= 2^31
+    (dict(d=100), moe.MOE_ERR_UNSUPPORTED),
+    (dict(f=96), moe.MOE_ERR_UNSUPPORTED),
+    (dict(d=8192, dtype=moe.MOE_F32), moe.MOE_ERR_UNSUPPORTED),
+    (dict(d=8192, dtype=moe.MOE_BF16), moe.MOE_OK),
+    (dict(dtype=7), moe.MOE_ERR_INVALID_ARG),
+    (dict(T=0), moe.MOE_OK),
+])
+def test_shape_checks(L, kw, expect):
+    for fn in (L.moe_scratch_size, L.moe_forward_workspace_size, L.moe_packed_weights_size):
+        st, n = _size(fn, **kw)
+        assert st == expect
+        if st == moe.MOE_OK:
+            assert n > 0
+
+
+def test_workspace_sizes_grow_with_tokens(L):
+    _, a = _size(L.moe_forward_workspace_size, T=1024)
+    _, b = _size(L.moe_forward_workspace_size, T=4096)
+    assert b > a
+    _, p = _size(L.moe_packed_weights_size, d=256, E=16, f=256)
+    assert p >= 4 * (16 * 256 + 3 * 16 * 256 * 256)
+
+
+def test_bad_placement_rejected_before_any_launch(L):
+    s = moe.moe_shape(T=8, d=256, E=16, k=2, f=256, ep=4, dtype=moe.MOE_F32)
+    lay = moe.moe_layout(*([ctypes.c_void_p(256)] * 9))
+    ws = ctypes.c_void_p(1 << 20)
+    # rank 0 owns 5 experts, rank 3 owns 3: not a partition
+    bad = (ctypes.c_int32 * 16)(*([0] * 5 + [1] * 4 + [2] * 4 + [3] * 3))
+    assert L.moe_dispatch_layout(ctypes.byref(s), ctypes.c_void_p(256), bad, ctypes.byref(lay),
+                                 ws, 1 << 30, None) == moe.MOE_ERR_INVALID_ARG
+    out_of_range = (ctypes.c_int32 * 16)(*([0] * 4 + [1] * 4 + [2] * 4 + [4] * 4))
+    assert L.moe_dispatch_layout(ctypes.byref(s), ctypes.c_void_p(256), out_of_range,
+                                 ctypes.byref(lay), ws, 1 << 30, None) == moe.MOE_ERR_INVALID_ARG
+    # too small a workspace
+    assert L.moe_dispatch_layout(ctypes.byref(s), ctypes.c_void_p(256), None, ctypes.byref(lay),
+                                 ws, 16, None) == moe.MOE_ERR_WORKSPACE
+    # misaligned index pointer
+    assert L.moe_dispatch_layout(ctypes.byref(s), ctypes.c_void_p(258), None, ctypes.byref(lay),
+                                 ws, 1 << 30, None) == moe.MOE_ERR_ALIGNMENT
+    # missing send-layout outputs with ep > 1
+    lay2 = moe.moe_layout(*([ctypes.c_void_p(256)] * 4 + [None] * 5))
+    assert L.moe_dispatch_layout(ctypes.byref(s), ctypes.c_void_p(256), None, ctypes.byref(lay2),
+                                 ws, 1 << 30, None) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_misaligned_tensors_rejected(L):
+    s = moe.moe_shape(T=8, d=256, E=16, k=2, f=256, ep=1, dtype=moe.MOE_BF16)
+    P = ctypes.c_void_p
+    assert L.moe_permute(ctypes.byref(s), P(8), P(256), P(4096), None) == moe.MOE_ERR_ALIGNMENT
+    assert L.moe_combine(ctypes.byref(s), P(4096), P(256), None, P(4100), None) == moe.MOE_ERR_ALIGNMENT
+    assert L.moe_permute(ctypes.byref(s), None, P(256), P(4096), None) == moe.MOE_ERR_INVALID_ARG

@@ -1,0 +1,134 @@
+"""Shared helpers of the GPU parity tests: seeded inputs on both sides, the
+near-tie injection of the top-6 workload, and tolerance checks.
+
+Inputs are always drawn on the CPU (routing_dispatch_experts_b200.workloads)
+and copied to the GPU; expected values come only from the CPU oracle.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+import routing_dispatch_experts_b200 as moe
+from routing_dispatch_experts_b200 import workloads as W
+
+# max |y_gpu - y_oracle| <= TOL * max |y_oracle|: bf16 storage with fp32
+# accumulation (2e-2), and the fp32 workload (1e-5)
+TOL = {"bf16": 2e-2, "f32": 1e-5}
+# routing decisions whose margin is below this may legitimately differ
+NEAR_TIE = 1e-5
+
+
+def shape_of(w: W.Workload, T=None, ep=1) -> moe.Shape:
+    return moe.Shape(T=w.T if T is None else T, d=w.d, E=w.E, k=w.k, f=w.f, ep=ep,
+                     dtype=w.torch_dtype)
+
+
+class Case:
+    """One workload instance: CPU tensors, device tensors and packed weights."""
+
+    def __init__(self, cfg: int, T=None, seed=0, near_ties=None, experts=None):
+        self.w = W.WORKLOADS[cfg]
+        self.T = self.w.T if T is None else T
+        self.x = W.make_x(self.w, seed, self.T)
+        self.wr = W.make_router(self.w, seed)
+        self.bias = W.make_bias(self.w, seed)
+        self.wg, self.wu, self.wd = W.make_experts(self.w, seed)
+        inject = self.w.near_tie_frac > 0 if near_ties is None else near_ties
+        self.near_tie_tokens = inject_near_ties(self, seed) if inject else np.array([], np.int64)
+        self.shape = shape_of(self.w, self.T)
+        dev = "cuda"
+        self.dx = self.x.to(dev)
+        self.dbias = None if self.bias is None else self.bias.to(dev)
+        self.packed = moe.pack_weights(self.shape, self.wr.to(dev), self.wg.to(dev),
+                                       self.wu.to(dev), self.wd.to(dev))
+        torch.cuda.synchronize()
+
+    def shape_ep(self, ep):
+        return shape_of(self.w, self.T, ep)
+
+
+def _bf16_step(v: np.ndarray, up: bool) -> np.ndarray:
+    """Next bf16 value above / below (bit patterns as uint16)."""
+    neg = (v & 0x8000) != 0
+    mag = v & 0x7FFF
+    out = v.copy()
+    # moving away from zero increments the magnitude
+    away = ~neg if up else neg
+    out[away] = v[away] + 1
+    tow = ~away
+    zero = tow & (mag == 0)
+    out[tow & ~zero] = v[tow & ~zero] - 1
+    out[zero] = 0x0001 if up else 0x8001
+    return out
+
+
+def inject_near_ties(case: Case, seed: int, frac=None, target=5e-6, max_steps=4000):
+    """Nudge x of a seeded fraction of tokens, one bf16 ulp at a time, until
+    the gap between the k-th and (k+1)-th router logits (in double) is below
+    `target` times the token's logit spread.  Returns the tokens changed."""
+    w = case.w
+    frac = w.near_tie_frac if frac is None else frac
+    n = int(round(frac * case.T))
+    if n == 0:
+        return np.array([], np.int64)
+    toks = W.sample_tokens(case.T, n, seed + 101).numpy()
+    wr = case.wr.double().numpy()
+    b = 0.0 if case.bias is None else case.bias.double().numpy()
+    xb = case.x.view(torch.int16).numpy().view(np.uint16)
+    done = []
+    for t in toks:
+        row = xb[t].copy()
+        # coarse move: project x onto the tie plane of the k-th / (k+1)-th
+        # experts in double, then round back to bf16
+        xv = torch.from_numpy(row.view(np.int16).copy()).view(torch.bfloat16).double().numpy()
+        l = xv @ wr + b
+        o = np.argsort(-l, kind="stable")
+        v = wr[:, o[w.k - 1]] - wr[:, o[w.k]]
+        xv = xv - (l[o[w.k - 1]] - l[o[w.k]]) / (v @ v) * v
+        row = torch.from_numpy(xv).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16).copy()
+        for _ in range(max_steps):
+            xv = torch.from_numpy(row.view(np.int16).copy()).view(torch.bfloat16).double().numpy()
+            l = xv @ wr + b
+            o = np.argsort(-l, kind="stable")
+            a, c = o[w.k - 1], o[w.k]
+            spread = l.max() - l.min()
+            gap = l[a] - l[c]
+            if gap <= target * spread:
+                break
+            v = wr[:, a] - wr[:, c]
+            # every coordinate's one-ulp step up and down, pick the best
+            up = _bf16_step(row, True)
+            dn = _bf16_step(row, False)
+            xu = torch.from_numpy(up.view(np.int16).copy()).view(torch.bfloat16).double().numpy()
+            xd = torch.from_numpy(dn.view(np.int16).copy()).view(torch.bfloat16).double().numpy()
+            gu = gap + (xu - xv) * v
+            gd = gap + (xd - xv) * v
+            gu[~np.isfinite(gu)] = np.inf
+            gd[~np.isfinite(gd)] = np.inf
+            iu, idn = np.argmin(np.abs(gu)), np.argmin(np.abs(gd))
+            if abs(gu[iu]) <= abs(gd[idn]):
+                row[iu] = up[iu]
+            else:
+                row[idn] = dn[idn]
+        xb[t] = row
+        done.append(t)
+    return np.array(done, np.int64)
+
+
+def routing_mismatches(idx_gpu: np.ndarray, idx_ref: np.ndarray) -> np.ndarray:
+    """Tokens whose expert sets differ."""
+    return np.where((np.sort(idx_gpu, 1) != np.sort(idx_ref, 1)).any(1))[0]
+
+
+def check_output(y_gpu: torch.Tensor, y_ref: np.ndarray, dtype: str, rows=None):
+    yg = y_gpu.float().cpu().double().numpy()
+    if rows is not None:
+        yg, y_ref = yg[rows], y_ref[rows]
+    if yg.size == 0:
+        return 0.0
+    scale = np.abs(y_ref).max()
+    err = np.abs(yg - y_ref).max()
+    assert err <= TOL[dtype] * scale, f"max|dy| = {err:.3e} > {TOL[dtype]} * {scale:.3e}"
+    return err / scale
