@@ -39,6 +39,7 @@ from routing_dispatch_experts_b200 import workloads as W  # noqa: E402
 
 METRIC = "MoE-layer fwd routed tokens/s"
 L2_FLUSH_BYTES = 256 << 20
+SLEEP_CYCLES = 200_000  # ~0.1 ms of device-side sleep before each timed iteration
 MEASURED_PEAKS = os.path.join(ROOT, "MEASURED_PEAKS.json")
 
 
@@ -174,64 +175,77 @@ def run_ours(args, rank, world, local):
     def step():
         moe.forward(shape, dx, packed, dbias, ws, expert_rank=rmap, y=y, buffers=buf)
 
+    def graph_of(fn):
+        # the whole call sequence in one CUDA graph: one launch per step
+        fn()
+        torch.cuda.synchronize(dev)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            fn()
+        torch.cuda.synchronize(dev)
+        return g
+
+    side = torch.cuda.Stream(dev)
     clocks = ClockSampler(local)
     clocks.start()
+    step_graph = graph_of(step)
     # warm-up (at least W steps, and long enough for the clock sampler to see load)
-    t_end = time.time() + 1.0
+    t_end = time.time() + (0.0 if args.profile else 1.0)
     i = 0
     while i < args.warmup or time.time() < t_end:
         flush.fill_(i & 0xFF)
-        step()
+        step_graph.replay()
         i += 1
         if i % 64 == 0:
             torch.cuda.synchronize(dev)
     torch.cuda.synchronize(dev)
     moe.check_device_status(ws)
 
-    # ---- timed region: K steps, L2 flushed before each
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
-    barrier(world)
-    torch.cuda.synchronize(dev)
-    for i in range(args.steps):
-        flush.fill_(i & 0xFF)
-        ev[i][0].record(stream)
-        step()
-        ev[i][1].record(stream)
-    torch.cuda.synchronize(dev)
-    barrier(world)
-    step_ms = [a.elapsed_time(b) for a, b in ev]
-    ms = max_over_ranks(sum(step_ms) / len(step_ms), world)
-    moe.check_device_status(ws)
-
-    # ---- per-call breakdown (same stream, same flushing) -> dominant call
-    calls = {}
-    lay_ws = ws  # the forward workspace starts with the scratch the calls need
-
-    def t_call(name, fn, reps):
+    def timed(run, n, gap=True):
+        """Per-iteration CUDA-event durations of run(); before each, L2 is
+        flushed and a short device-side sleep lets the host queue the
+        iteration, so no host launch gap falls inside the events."""
         e = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-             for _ in range(reps)]
-        for i in range(reps):
+             for _ in range(n)]
+        for i in range(n):
             flush.fill_(i & 0xFF)
+            if gap:
+                torch.cuda._sleep(SLEEP_CYCLES)
             e[i][0].record(stream)
-            fn()
+            run()
             e[i][1].record(stream)
         torch.cuda.synchronize(dev)
-        calls[name] = sum(a.elapsed_time(b) for a, b in e) / reps
+        return [a.elapsed_time(b) for a, b in e]
 
+    # ---- timed region: K steps, L2 flushed before each
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    step_ms = timed(step_graph.replay, args.steps)
+    barrier(world)
+    ms = max_over_ranks(sum(step_ms) / len(step_ms), world)
+    moe.check_device_status(ws)
+    # the same steps issued eagerly (one moe_forward call each, no graph)
+    eager_ms = sum(timed(step, args.steps)) / args.steps
+
+    # ---- per-call breakdown (same stream, same flushing, each call replayed
+    # from its own CUDA graph) -> the dominant call
+    calls = {}
+    lay_ws = ws  # the forward workspace starts with the scratch the calls need
     reps = max(args.steps, 20)
-    lg = buf.logits
-    t_call("route", lambda: moe.route(shape, dx, packed, dbias, lay_ws), reps)
-    idx = buf.topk_idx
-    t_call("layout", lambda: moe.dispatch_layout(shape, idx, lay_ws, expert_rank=rmap), reps)
-    rt = buf.layout["row_token"]
-    t_call("permute", lambda: moe.permute(shape, dx, rt), reps)
-    off = buf.layout["expert_offsets"]
-    xp = buf.x_perm
-    t_call("grouped_swiglu", lambda: moe.grouped_swiglu(shape, xp, off, packed, lay_ws), reps)
-    t_call("combine", lambda: moe.combine(shape, buf.y_perm, buf.layout["slot_row"], buf.topk_gate), reps)
+    idx, rt = buf.topk_idx, buf.layout["row_token"]
+    off, xp = buf.layout["expert_offsets"], buf.x_perm
+    for name, fn in (
+            ("route", lambda: moe.route(shape, dx, packed, dbias, lay_ws)),
+            ("layout", lambda: moe.dispatch_layout(shape, idx, lay_ws, expert_rank=rmap)),
+            ("permute", lambda: moe.permute(shape, dx, rt)),
+            ("grouped_swiglu", lambda: moe.grouped_swiglu(shape, xp, off, packed, lay_ws)),
+            ("combine", lambda: moe.combine(shape, buf.y_perm, buf.layout["slot_row"], buf.topk_gate))):
+        g = graph_of(fn)
+        calls[name] = sum(timed(g.replay, reps)) / reps
     moe.check_device_status(ws)
     clk = clocks.stop()
+    if args.profile:
+        return {"profile": True, "ms_per_step": ms, "breakdown_ms": calls}
 
     # ---- end to end through the public API with host buffers
     x_host = x.pin_memory()
@@ -239,14 +253,14 @@ def run_ours(args, rank, world, local):
     e2e_ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
     for _ in range(3):
         dx.copy_(x_host, non_blocking=True)
-        step()
+        step_graph.replay()
         y_host.copy_(y, non_blocking=True)
     torch.cuda.synchronize(dev)
     barrier(world)
     e2e_ev[0].record(stream)
     for i in range(args.steps):
         dx.copy_(x_host, non_blocking=True)
-        step()
+        step_graph.replay()
         y_host.copy_(y, non_blocking=True)
     e2e_ev[1].record(stream)
     torch.cuda.synchronize(dev)
@@ -283,13 +297,15 @@ def run_ours(args, rank, world, local):
                 "h2d_bytes_per_step": x.numel() * x.element_size(),
                 "d2h_bytes_per_step": y.numel() * y.element_size()},
         "gpu_launches": 8 * args.steps,
+        "ms_per_step_eager": eager_ms,
+        "step": "one moe_forward (8 kernels) replayed from a CUDA graph",
         "breakdown_ms": {k: round(v, 5) for k, v in calls.items()},
         "roofline": {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
                      "frac": achieved / peak, "peak_source": pk["src"], "traffic": None,
                      "algorithmic": d},
         "clocks": clk,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.profile:
         result["cpu_baseline"] = cpu_baseline(w, args)
     return result
 
@@ -346,6 +362,8 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", action="store_true",
+                    help="short run for a profiler: no clock warm-up, e2e or CPU baseline")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.impl == "reference":

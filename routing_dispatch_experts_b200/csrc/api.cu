@@ -265,9 +265,12 @@ moe_status do_grouped(const moe_shape* s, const void* x_perm, const int32_t* off
 }
 
 moe_status check_layout_ptrs(const moe_shape* s, const moe_layout* o) {
-  if (!o || !o->expert_counts || !o->expert_offsets || !o->row_token || !o->slot_row)
+  // with T == 0 the per-assignment arrays are empty and may be NULL
+  const bool rows = s->T > 0;
+  if (!o || !o->expert_counts || !o->expert_offsets || (rows && (!o->row_token || !o->slot_row)))
     return MOE_ERR_INVALID_ARG;
-  if (s->ep > 1 && (!o->rank_counts || !o->rank_offsets || !o->send_token || !o->slot_send_row))
+  if (s->ep > 1 && (!o->rank_counts || !o->rank_offsets ||
+                    (rows && (!o->send_token || !o->slot_send_row))))
     return MOE_ERR_INVALID_ARG;
   const void* ps[] = {o->expert_counts, o->expert_offsets, o->row_token, o->slot_row,
                       o->rank_counts, o->rank_offsets, o->send_token, o->slot_send_row};
