@@ -314,6 +314,42 @@ MOE_API moe_status moe_debug_dispatch_layout_stall(const moe_shape* shape,
                                            int64_t wait_limit_ns,
                                            moe_stream_t stream);
 
+/*
+ * moe_dispatch_layout for callers that cannot allocate device memory.
+ * The source pages have no counterpart of this call; it exists for callers
+ * that may not call cudaMalloc or any other allocator where they call this
+ * library (an operator inside a framework whose device memory is planned
+ * ahead and which receives only its inputs and outputs, or a C caller with
+ * no device allocator), and therefore cannot pass the workspace that
+ * moe_dispatch_layout needs.
+ *
+ * Same inputs and outputs as moe_dispatch_layout, but no workspace: the
+ * scratch lives in a 1 MiB array inside this library, one per GPU, held
+ * from when the library's device code is loaded until the process exits.
+ * Nothing is allocated and nothing is freed by this call.
+ *  - Shapes whose scratch exceeds 1 MiB are rejected with MOE_ERR_WORKSPACE
+ *    (the scratch is 256 B + 12 B * ceil(T/512) * (E + (ep>1 ? ep : 0) + 2)
+ *    + 4 B * bins, each part rounded up to 256 B; e.g. E=64, ep=8 fits up
+ *    to about 600k tokens, E=256, ep=256 about 87k).
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before capturing any stream on that device.
+ *  - Every call on a device shares the one array, and it keeps the previous
+ *    call's contents: each call first clears the part that must start at
+ *    zero (on `stream`).  Calls whose work overlaps on the GPU (different
+ *    streams or threads at the same time on one device) race on the array
+ *    and give wrong layouts; order them on one stream.
+ *  - device_status: optional device int32 that receives this call's device
+ *    status (MOE_OK, MOE_ERR_DEVICE_INDEX or MOE_ERR_DEVICE_TIMEOUT) when
+ *    the layout kernels finish; NULL to skip.
+ */
+MOE_API moe_status moe_dispatch_layout_static(const moe_shape* shape,
+                                              const int32_t* topk_idx,
+                                              const int32_t* expert_rank_host,
+                                              const moe_layout* out,
+                                              int32_t* device_status,
+                                              moe_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -74,7 +74,8 @@ _lib = None
 SYMBOLS = ("moe_status_string", "moe_scratch_size", "moe_forward_workspace_size",
            "moe_workspace_init", "moe_packed_weights_size", "moe_pack_weights", "moe_route",
            "moe_dispatch_layout", "moe_permute", "moe_grouped_swiglu", "moe_combine",
-           "moe_forward", "moe_get_device_status", "moe_debug_dispatch_layout_stall")
+           "moe_forward", "moe_get_device_status", "moe_debug_dispatch_layout_stall",
+           "moe_dispatch_layout_static")
 
 
 def lib() -> ctypes.CDLL:
@@ -106,6 +107,7 @@ def lib() -> ctypes.CDLL:
             "moe_debug_dispatch_layout_stall": ([S, P, P, ctypes.POINTER(moe_layout), P,
                                                  ctypes.c_size_t, ctypes.c_int32, ctypes.c_int64, P],
                                                 ctypes.c_int),
+            "moe_dispatch_layout_static": ([S, P, P, ctypes.POINTER(moe_layout), P, P], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -287,6 +289,21 @@ def debug_dispatch_layout_stall(shape: Shape, topk_idx, ws, stall_block: int, wa
         ctypes.byref(s), _p(topk_idx), _host_map(shape, expert_rank), ctypes.byref(lay), _p(ws),
         ws.numel(), stall_block, wait_limit_ns, _stream(stream)), "moe_debug_dispatch_layout_stall")
     return out
+
+
+def dispatch_layout_static(shape: Shape, topk_idx, expert_rank=None, stream=None):
+    """moe_dispatch_layout_static: the layout with the library's own scratch
+    (no workspace).  Returns (layout tensors, device status tensor [1])."""
+    _need(topk_idx, torch.int32, (shape.T, shape.k), "topk_idx")
+    out = _layout_tensors(shape, topk_idx.device)
+    status = torch.full((1,), -1, dtype=torch.int32, device=topk_idx.device)
+    lay = _c_layout(out)
+    s = shape.c
+    _check(lib().moe_dispatch_layout_static(ctypes.byref(s), _p(topk_idx),
+                                            _host_map(shape, expert_rank), ctypes.byref(lay),
+                                            _p(status), _stream(stream)),
+           "moe_dispatch_layout_static")
+    return out, status
 
 
 def permute(shape: Shape, x, row_token, stream=None):
