@@ -40,6 +40,10 @@ from routing_dispatch_experts_b200 import workloads as W  # noqa: E402
 METRIC = "MoE-layer fwd routed tokens/s"
 L2_FLUSH_BYTES = 256 << 20
 SLEEP_CYCLES = 200_000  # ~0.1 ms of device-side sleep before each timed iteration
+# kernels of one moe_forward: bf16 = fused router, layout scatter, gate/up
+# GEMM (with the gather), down GEMM, combine; fp32 = router, top-k, layout
+# histogram, layout scatter, permute, gate/up, down, combine
+LAUNCHES_PER_STEP = {"bf16": 5, "f32": 8}
 MEASURED_PEAKS = os.path.join(ROOT, "MEASURED_PEAKS.json")
 
 
@@ -54,17 +58,26 @@ def peaks():
 
 # ------------------------------------------------------------ algorithmic work
 def work(w: W.Workload, T: int):
-    """Algorithmic bytes / FLOPs of each call for T tokens (what the method
-    must move or compute, not what a particular kernel happens to move)."""
+    """Algorithmic bytes / FLOPs of each forward stage for T tokens: what the
+    method must move or compute, not what a particular kernel happens to
+    move.  Stages as moe_forward_timed names them."""
     b = 2 if w.dtype == "bf16" else 4
     R = T * w.k
     return {
-        "route": dict(bytes=T * w.d * b + w.E * w.d * b + 2 * T * w.E * 4 + 2 * R * 4,
+        # x read, W_r read, logits + idx + gate written
+        "route": dict(bytes=T * w.d * b + w.E * w.d * b + T * w.E * 4 + 2 * R * 4,
                       flops=2 * T * w.d * w.E),
-        "layout": dict(bytes=2 * R * 4 + 4 * R * 4, flops=0),
-        "permute": dict(bytes=T * w.d * b + R * w.d * b + R * 4, flops=0),
-        "grouped_swiglu": dict(bytes=R * w.d * b + 3 * w.E * w.d * w.f * b + 2 * R * w.f * b
-                               + R * w.d * b, flops=6 * R * w.d * w.f),
+        # idx read; row_token, slot_row, send_token, slot_send_row written
+        "layout": dict(bytes=R * 4 + 4 * R * 4, flops=0),
+        # x rows read once per assignment, x_perm written
+        "permute": dict(bytes=R * w.d * b + R * w.d * b + R * 4, flops=0),
+        # rows of x (or x_perm) read, W_g / W_u read, h written
+        "gate_up": dict(bytes=R * w.d * b + 2 * w.E * w.d * w.f * b + R * w.f * b,
+                        flops=4 * R * w.d * w.f),
+        # h read, W_d read, y_perm written
+        "down": dict(bytes=R * w.f * b + w.E * w.f * w.d * b + R * w.d * b,
+                     flops=2 * R * w.d * w.f),
+        # y_perm read, gates / slot rows read, y written
         "combine": dict(bytes=R * w.d * b + T * w.d * b + 2 * R * 4, flops=0),
     }
 
@@ -227,25 +240,27 @@ def run_ours(args, rank, world, local):
     # the same steps issued eagerly (one moe_forward call each, no graph)
     eager_ms = sum(timed(step, args.steps)) / args.steps
 
-    # ---- per-call breakdown (same stream, same flushing, each call replayed
-    # from its own CUDA graph) -> the dominant call
-    calls = {}
-    lay_ws = ws  # the forward workspace starts with the scratch the calls need
+    # ---- per-stage device times inside the forward (moe_forward_timed:
+    # events recorded between the stages on the launching stream), same L2
+    # flush and host lead as the timed steps
+    nst = len(moe.FORWARD_STAGES)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)]
+    for e in evs:
+        e.record(stream)
     reps = max(args.steps, 20)
-    idx, rt = buf.topk_idx, buf.layout["row_token"]
-    off, xp = buf.layout["expert_offsets"], buf.x_perm
-    for name, fn in (
-            ("route", lambda: moe.route(shape, dx, packed, dbias, lay_ws)),
-            ("layout", lambda: moe.dispatch_layout(shape, idx, lay_ws, expert_rank=rmap)),
-            ("permute", lambda: moe.permute(shape, dx, rt)),
-            ("grouped_swiglu", lambda: moe.grouped_swiglu(shape, xp, off, packed, lay_ws)),
-            ("combine", lambda: moe.combine(shape, buf.y_perm, buf.layout["slot_row"], buf.topk_gate))):
-        g = graph_of(fn)
-        calls[name] = sum(timed(g.replay, reps)) / reps
+    acc = [0.0] * nst
+    for i in range(reps):
+        flush.fill_(i & 0xFF)
+        torch.cuda._sleep(SLEEP_CYCLES)
+        moe.forward_timed(shape, dx, packed, dbias, ws, evs, expert_rank=rmap, y=y, buffers=buf)
+        torch.cuda.synchronize(dev)
+        for j in range(nst):
+            acc[j] += evs[j].elapsed_time(evs[j + 1])
+    calls = {name: acc[j] / reps for j, name in enumerate(moe.FORWARD_STAGES)}
     moe.check_device_status(ws)
     clk = clocks.stop()
     if args.profile:
-        return {"profile": True, "ms_per_step": ms, "breakdown_ms": calls}
+        return {"profile": True, "ms_per_step": ms, "stage_ms": calls}
 
     # ---- end to end through the public API with host buffers
     x_host = x.pin_memory()
@@ -296,10 +311,10 @@ def run_ours(args, rank, world, local):
         "e2e": {"value": T * world / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": x.numel() * x.element_size(),
                 "d2h_bytes_per_step": y.numel() * y.element_size()},
-        "gpu_launches": 8 * args.steps,
+        "gpu_launches": LAUNCHES_PER_STEP[w.dtype] * args.steps,
         "ms_per_step_eager": eager_ms,
-        "step": "one moe_forward (8 kernels) replayed from a CUDA graph",
-        "breakdown_ms": {k: round(v, 5) for k, v in calls.items()},
+        "step": f"one moe_forward ({LAUNCHES_PER_STEP[w.dtype]} kernels) replayed from a CUDA graph",
+        "stage_ms": {k: round(v, 5) for k, v in calls.items()},
         "roofline": {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
                      "frac": achieved / peak, "peak_source": pk["src"], "traffic": None,
                      "algorithmic": d},

@@ -253,6 +253,21 @@ MOE_API moe_status moe_grouped_swiglu(const moe_shape* shape, const void* x_perm
                               moe_stream_t stream);
 
 /*
+ * The permute fused into the grouped SwiGLU experts (bf16 only): the same
+ * h and y_perm as moe_permute followed by moe_grouped_swiglu, but the
+ * gate/up GEMM fetches row r of its operand straight from x[row_token[r]]
+ * with TMA gather loads, so x_perm is never written or read.
+ *  x [T, d]; row_token [T*k] (moe_dispatch_layout); other arguments as in
+ *  moe_grouped_swiglu.  MOE_ERR_UNSUPPORTED for fp32.
+ */
+MOE_API moe_status moe_grouped_swiglu_gather(const moe_shape* shape, const void* x,
+                                             const int32_t* row_token,
+                                             const int32_t* expert_offsets,
+                                             const void* packed, void* h, void* y_perm,
+                                             void* ws, size_t ws_bytes,
+                                             moe_stream_t stream);
+
+/*
  * Gate-weighted combine (un-permute):
  *   y[t] = sum_{j<k} gate[t,j] * y_perm[slot_row[t*k+j]]
  * summed in fp32 in ascending j, rounded once to the dtype.
@@ -279,9 +294,13 @@ typedef struct {
 } moe_forward_buffers;
 
 /*
- * The whole layer: moe_route, moe_dispatch_layout, moe_permute,
- * moe_grouped_swiglu and moe_combine enqueued back to back on `stream`,
- * with no host synchronisation in between.
+ * The whole layer enqueued back to back on `stream`, with no host
+ * synchronisation in between.  bf16: one kernel for router GEMM + top-k +
+ * gates + the dispatch histogram and its lookback scan, the layout scatter,
+ * the gate/up GEMM reading rows of x through the permutation (as
+ * moe_grouped_swiglu_gather; x_perm is not written), the down GEMM and the
+ * combine.  fp32: moe_route, moe_dispatch_layout, moe_permute,
+ * moe_grouped_swiglu and moe_combine in turn.
  *  x [T, d]; packed weights; bias [E] or NULL; expert_rank_host as in
  *  moe_dispatch_layout; y [T, d]; buffers may be NULL;
  *  ws, ws_bytes  moe_forward_workspace_size bytes.
@@ -290,6 +309,24 @@ MOE_API moe_status moe_forward(const moe_shape* shape, const void* x, const void
                        const float* bias, const int32_t* expert_rank_host,
                        void* y, const moe_forward_buffers* buffers, void* ws,
                        size_t ws_bytes, moe_stream_t stream);
+
+typedef struct CUevent_st* moe_event_t; /* same type as cudaEvent_t */
+#define MOE_FORWARD_STAGES 6
+
+/*
+ * moe_forward that also records events[i] on `stream` just before stage i
+ * (0 route, 1 dispatch layout, 2 permute, 3 gate/up GEMM, 4 down GEMM,
+ * 5 combine) and events[6] after the last, so cudaEventElapsedTime between
+ * neighbours gives each stage's device time inside the forward.  A stage
+ * that a path fuses into another (the permute on bf16) has no work between
+ * its two events.  events: MOE_FORWARD_STAGES + 1 caller-created events.
+ */
+MOE_API moe_status moe_forward_timed(const moe_shape* shape, const void* x,
+                                     const void* packed, const float* bias,
+                                     const int32_t* expert_rank_host, void* y,
+                                     const moe_forward_buffers* buffers, void* ws,
+                                     size_t ws_bytes, moe_event_t* events,
+                                     moe_stream_t stream);
 
 /*
  * Synchronise `stream`, read the device status word of workspace `ws`
@@ -328,9 +365,9 @@ MOE_API moe_status moe_debug_dispatch_layout_stall(const moe_shape* shape,
  * from when the library's device code is loaded until the process exits.
  * Nothing is allocated and nothing is freed by this call.
  *  - Shapes whose scratch exceeds 1 MiB are rejected with MOE_ERR_WORKSPACE
- *    (the scratch is 256 B + 12 B * ceil(T/512) * (E + (ep>1 ? ep : 0) + 2)
- *    + 4 B * bins, each part rounded up to 256 B; e.g. E=64, ep=8 fits up
- *    to about 600k tokens, E=256, ep=256 about 87k).
+ *    (the scratch is 256 B + 12 B * ceil(T/128) * bins + 4 B * bins with
+ *    bins = E + (ep > 1 ? ep : 0) + 2, each part rounded up to 256 B; e.g.
+ *    E=64, ep=8 fits up to about 150k tokens, E=256, ep=256 about 21k).
  *  - The first call on each device looks up the array's device address
  *    (cudaGetSymbolAddress) with that device current; make that first call
  *    before capturing any stream on that device.

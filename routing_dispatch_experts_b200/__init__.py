@@ -73,9 +73,11 @@ _lib = None
 # exported C symbols, in header order (checked against include/moe.h by the tests)
 SYMBOLS = ("moe_status_string", "moe_scratch_size", "moe_forward_workspace_size",
            "moe_workspace_init", "moe_packed_weights_size", "moe_pack_weights", "moe_route",
-           "moe_dispatch_layout", "moe_permute", "moe_grouped_swiglu", "moe_combine",
-           "moe_forward", "moe_get_device_status", "moe_debug_dispatch_layout_stall",
+           "moe_dispatch_layout", "moe_permute", "moe_grouped_swiglu",
+           "moe_grouped_swiglu_gather", "moe_combine", "moe_forward", "moe_forward_timed",
+           "moe_get_device_status", "moe_debug_dispatch_layout_stall",
            "moe_dispatch_layout_static")
+FORWARD_STAGES = ("route", "layout", "permute", "gate_up", "down", "combine")
 
 
 def lib() -> ctypes.CDLL:
@@ -101,6 +103,10 @@ def lib() -> ctypes.CDLL:
             "moe_permute": ([S, P, P, P, P], ctypes.c_int),
             "moe_grouped_swiglu": ([S, P, P, P, P, P, P, ctypes.c_size_t, P], ctypes.c_int),
             "moe_combine": ([S, P, P, P, P, P], ctypes.c_int),
+            "moe_grouped_swiglu_gather": ([S, P, P, P, P, P, P, P, ctypes.c_size_t, P], ctypes.c_int),
+            "moe_forward_timed": ([S, P, P, P, P, P, ctypes.POINTER(moe_forward_buffers), P,
+                                   ctypes.c_size_t, ctypes.POINTER(ctypes.c_void_p), P],
+                                  ctypes.c_int),
             "moe_forward": ([S, P, P, P, P, P, ctypes.POINTER(moe_forward_buffers), P,
                              ctypes.c_size_t, P], ctypes.c_int),
             "moe_get_device_status": ([P, P, ctypes.POINTER(ctypes.c_int)], ctypes.c_int),
@@ -327,6 +333,19 @@ def grouped_swiglu(shape: Shape, x_perm, expert_offsets, packed, ws, stream=None
     return h, y_perm
 
 
+def grouped_swiglu_gather(shape: Shape, x, row_token, expert_offsets, packed, ws, stream=None):
+    """moe_grouped_swiglu_gather: (h, y_perm) with rows gathered from x."""
+    _need(x, shape.dtype, (shape.T, shape.d), "x")
+    h = torch.empty((shape.R, shape.f), dtype=shape.dtype, device=x.device)
+    y_perm = torch.empty((shape.R, shape.d), dtype=shape.dtype, device=x.device)
+    s = shape.c
+    _check(lib().moe_grouped_swiglu_gather(ctypes.byref(s), _p(x), _p(row_token),
+                                           _p(expert_offsets), _p(packed), _p(h), _p(y_perm),
+                                           _p(ws), ws.numel(), _stream(stream)),
+           "moe_grouped_swiglu_gather")
+    return h, y_perm
+
+
 def combine(shape: Shape, y_perm, slot_row, topk_gate=None, stream=None):
     _need(y_perm, shape.dtype, (shape.R, shape.d), "y_perm")
     y = torch.empty((shape.T, shape.d), dtype=shape.dtype, device=y_perm.device)
@@ -368,6 +387,25 @@ def forward(shape: Shape, x, packed, bias, ws, expert_rank=None, y=None,
                              _host_map(shape, expert_rank), _p(y),
                              ctypes.byref(b) if b is not None else None, _p(ws), ws.numel(),
                              _stream(stream)), "moe_forward")
+    return y
+
+
+def forward_timed(shape: Shape, x, packed, bias, ws, events, expert_rank=None, y=None,
+                  buffers: Optional[ForwardBuffers] = None, stream=None):
+    """moe_forward_timed: moe_forward recording `events` (7 torch.cuda.Event
+    with timing) around its stages (FORWARD_STAGES)."""
+    _need(x, shape.dtype, (shape.T, shape.d), "x")
+    if len(events) != len(FORWARD_STAGES) + 1:
+        raise ValueError("need one event per stage plus one")
+    if y is None:
+        y = torch.empty((shape.T, shape.d), dtype=shape.dtype, device=x.device)
+    ev = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+    s = shape.c
+    b = buffers.c if buffers is not None else None
+    _check(lib().moe_forward_timed(ctypes.byref(s), _p(x), _p(packed), _p(bias),
+                                   _host_map(shape, expert_rank), _p(y),
+                                   ctypes.byref(b) if b is not None else None, _p(ws), ws.numel(),
+                                   ev, _stream(stream)), "moe_forward_timed")
     return y
 
 

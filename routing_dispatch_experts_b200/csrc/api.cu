@@ -186,20 +186,22 @@ moe_status do_route(const moe_shape* s, const void* x, const Packed* pk, const f
   if (x) {
     cudaError_t e;
     if (s->dtype == MOE_BF16) {
-      GemmArgs a{};
-      a.A = x;
-      a.rows = s->T;
-      a.B = pk->wrT;
-      a.offsets = nullptr;
-      a.G = 1;
-      a.K = s->d;
-      a.n_per_group = pad16(s->E);
-      a.n_out = s->E;
-      a.out = logits;
-      a.ld_out = s->E;
+      // router GEMM, top-k and gates in one tcgen05 kernel
+      RouteArgs a{};
+      a.x = x;
+      a.wrT = pk->wrT;
       a.bias = bias;
+      a.T = s->T;
+      a.d = s->d;
+      a.E = s->E;
+      a.k = s->k;
+      a.logits = logits;
+      a.idx = idx;
+      a.gate = gate;
       a.ctl = ctl;
-      e = launch_gemm_tc(kEpiLogits, pad16(s->E), a, st);
+      a.hist = false;
+      a.ep = s->ep;
+      return cuda_status(launch_route_tc(a, st));
     } else {
       e = launch_router_f32(static_cast<const float*>(x), static_cast<const float*>(pk->wrT), bias,
                             s->T, s->d, s->E, logits, st);
@@ -226,42 +228,53 @@ moe_status do_layout(const moe_shape* s, const int32_t* idx, const RankMap& map,
                                    sc.prefix, sc.totals, stall, limit, st));
 }
 
-moe_status do_grouped(const moe_shape* s, const void* x_perm, const int32_t* offsets,
-                      const Packed* pk, void* h, void* y_perm, Control* ctl, cudaStream_t st) {
+// gate/up GEMM + SwiGLU (part 0) or down GEMM (part 1).  With `gather`
+// (bf16 only) the gate/up GEMM reads its rows straight from x through the
+// permutation instead of from x_perm.
+moe_status do_grouped_part(int part, const moe_shape* s, const void* a_rows,
+                           const int32_t* gather, const int32_t* offsets, const Packed* pk,
+                           void* h, void* y_perm, Control* ctl, cudaStream_t st) {
   const int64_t R = s->T * (int64_t)s->k;
   if (s->dtype == MOE_F32)
-    return cuda_status(launch_grouped_f32(static_cast<const float*>(x_perm), offsets, s->E, R, s->d,
-                                          s->f, gu_block(s->f), static_cast<const float*>(pk->wgu),
-                                          static_cast<const float*>(pk->wdT),
-                                          static_cast<float*>(h), static_cast<float*>(y_perm), st));
+    return cuda_status(launch_grouped_f32_part(part, static_cast<const float*>(a_rows), offsets,
+                                               s->E, R, s->d, s->f, gu_block(s->f),
+                                               static_cast<const float*>(pk->wgu),
+                                               static_cast<const float*>(pk->wdT),
+                                               static_cast<float*>(h), static_cast<float*>(y_perm),
+                                               st));
   GemmArgs a{};
-  a.A = x_perm;
-  a.rows = R;
-  a.B = pk->wgu;
   a.offsets = offsets;
   a.G = s->E;
-  a.K = s->d;
-  a.n_per_group = 2 * s->f;
-  a.n_out = s->f;
-  a.out = h;
-  a.ld_out = s->f;
+  a.rows = R;
   a.ctl = ctl;
-  cudaError_t e = launch_gemm_tc(kEpiSwiGLU, 2 * gu_block(s->f), a, st);
-  if (e != cudaSuccess) return MOE_ERR_CUDA;
-  GemmArgs b{};
-  b.A = h;
-  b.rows = R;
-  b.B = pk->wdT;
-  b.offsets = offsets;
-  b.G = s->E;
-  b.K = s->f;
-  b.n_per_group = s->d;
-  b.n_out = s->d;
-  b.out = y_perm;
-  b.ld_out = s->d;
-  b.ctl = ctl;
+  if (part == 0) {
+    a.A = a_rows;
+    a.gather = gather;
+    a.src_rows = s->T;
+    a.B = pk->wgu;
+    a.K = s->d;
+    a.n_per_group = 2 * s->f;
+    a.n_out = s->f;
+    a.out = h;
+    a.ld_out = s->f;
+    return cuda_status(launch_gemm_tc(kEpiSwiGLU, 2 * gu_block(s->f), a, st));
+  }
+  a.A = h;
+  a.B = pk->wdT;
+  a.K = s->f;
+  a.n_per_group = s->d;
+  a.n_out = s->d;
+  a.out = y_perm;
+  a.ld_out = s->d;
   const int bn = s->d % 256 == 0 ? 256 : (s->d % 128 == 0 ? 128 : 64);
-  return cuda_status(launch_gemm_tc(kEpiBF16, bn, b, st));
+  return cuda_status(launch_gemm_tc(kEpiBF16, bn, a, st));
+}
+
+moe_status do_grouped(const moe_shape* s, const void* x_perm, const int32_t* offsets,
+                      const Packed* pk, void* h, void* y_perm, Control* ctl, cudaStream_t st) {
+  moe_status r = do_grouped_part(0, s, x_perm, nullptr, offsets, pk, h, y_perm, ctl, st);
+  if (r != MOE_OK) return r;
+  return do_grouped_part(1, s, x_perm, nullptr, offsets, pk, h, y_perm, ctl, st);
 }
 
 moe_status check_layout_ptrs(const moe_shape* s, const moe_layout* o) {
@@ -292,6 +305,97 @@ moe_status layout_entry(const moe_shape* s, const int32_t* idx, const int32_t* h
   RankMap map;
   if ((r = build_map(s, host_map, &map)) != MOE_OK) return r;
   return do_layout(s, idx, map, o, carve_scratch(s, ws), stall, limit, st);
+}
+
+moe_status forward_impl(const moe_shape* s, const void* x, const void* packed, const float* bias,
+                        const int32_t* expert_rank_host, void* y, const moe_forward_buffers* buffers,
+                        void* ws, size_t ws_bytes, cudaStream_t st, cudaEvent_t* ev) {
+  moe_status r = check_shape(s);
+  if (r != MOE_OK) return r;
+  if (!ws) return MOE_ERR_INVALID_ARG;
+  if (!aligned(ws, kAlign)) return MOE_ERR_ALIGNMENT;
+  if (ws_bytes < forward_bytes(s)) return MOE_ERR_WORKSPACE;
+  RankMap map;
+  if ((r = build_map(s, expert_rank_host, &map)) != MOE_OK) return r;
+  if (s->T == 0) return MOE_OK;
+  if (!x || !packed || !y) return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(y, 16) || !aligned(packed, kAlign) || (bias && !aligned(bias, 4)))
+    return MOE_ERR_ALIGNMENT;
+  FwdBufs f = carve_forward(s, ws, buffers);
+  if ((r = check_layout_ptrs(s, &f.lay)) != MOE_OK) return r;
+  if (!aligned(f.logits, 4) || !aligned(f.idx, 4) || !aligned(f.gate, 4) || !aligned(f.x_perm, 16) ||
+      !aligned(f.h, 16) || !aligned(f.y_perm, 16))
+    return MOE_ERR_ALIGNMENT;
+  const Scratch sc = carve_scratch(s, ws);
+  const Packed pk = carve_packed(s, packed);
+  // stage markers for moe_forward_timed: 0 route, 1 layout, 2 permute,
+  // 3 gate/up GEMM, 4 down GEMM, 5 combine, 6 end
+  auto mark = [&](int i) { return ev ? cuda_status(cudaEventRecord(ev[i], st)) : MOE_OK; };
+  LayoutOut lo;
+  lo.counts = f.lay.expert_counts;
+  lo.offsets = f.lay.expert_offsets;
+  lo.row_token = f.lay.row_token;
+  lo.slot_row = f.lay.slot_row;
+  lo.rank_counts = f.lay.rank_counts;
+  lo.rank_offsets = f.lay.rank_offsets;
+  lo.send_token = f.lay.send_token;
+  lo.slot_send_row = f.lay.slot_send_row;
+  lo.stats = f.lay.stats;
+  const bool bf16 = s->dtype == MOE_BF16;
+  if ((r = mark(0)) != MOE_OK) return r;
+  if (bf16) {
+    // router + top-k + gates + dispatch histogram and lookback in one kernel
+    RouteArgs a{};
+    a.x = x;
+    a.wrT = pk.wrT;
+    a.bias = bias;
+    a.T = s->T;
+    a.d = s->d;
+    a.E = s->E;
+    a.k = s->k;
+    a.logits = f.logits;
+    a.idx = f.idx;
+    a.gate = f.gate;
+    a.ctl = sc.ctl;
+    a.hist = true;
+    a.ep = s->ep;
+    a.map = map;
+    a.status_words = sc.status;
+    a.prefix = sc.prefix;
+    a.totals = sc.totals;
+    if ((r = cuda_status(launch_route_tc(a, st))) != MOE_OK) return r;
+    if ((r = mark(1)) != MOE_OK) return r;
+    // the scatter half of the layout
+    if ((r = cuda_status(launch_layout_scatter(f.idx, s->T, s->k, s->E, s->ep, map, lo, sc.ctl,
+                                               sc.prefix, sc.totals, st))) != MOE_OK)
+      return r;
+    // no separate permute: the gate/up GEMM gathers its rows from x
+    if ((r = mark(2)) != MOE_OK || (r = mark(3)) != MOE_OK) return r;
+    if ((r = do_grouped_part(0, s, x, f.lay.row_token, f.lay.expert_offsets, &pk, f.h, f.y_perm,
+                             sc.ctl, st)) != MOE_OK)
+      return r;
+  } else {
+    if ((r = do_route(s, x, &pk, bias, f.logits, f.idx, f.gate, sc.ctl, st)) != MOE_OK) return r;
+    if ((r = mark(1)) != MOE_OK) return r;
+    if ((r = do_layout(s, f.idx, map, &f.lay, sc, -1, kWaitLimitNs, st)) != MOE_OK) return r;
+    if ((r = mark(2)) != MOE_OK) return r;
+    if ((r = cuda_status(launch_permute(x, f.lay.row_token, f.x_perm, s->T, s->T * (int64_t)s->k,
+                                        (uint32_t)(s->d * esize(s->dtype)), st))) != MOE_OK)
+      return r;
+    if ((r = mark(3)) != MOE_OK) return r;
+    if ((r = do_grouped_part(0, s, f.x_perm, nullptr, f.lay.expert_offsets, &pk, f.h, f.y_perm,
+                             sc.ctl, st)) != MOE_OK)
+      return r;
+  }
+  if ((r = mark(4)) != MOE_OK) return r;
+  if ((r = do_grouped_part(1, s, nullptr, nullptr, f.lay.expert_offsets, &pk, f.h, f.y_perm, sc.ctl,
+                           st)) != MOE_OK)
+    return r;
+  if ((r = mark(5)) != MOE_OK) return r;
+  if ((r = cuda_status(launch_combine(s->dtype, f.y_perm, f.lay.slot_row, f.gate, y, s->T, s->d,
+                                      s->k, st))) != MOE_OK)
+    return r;
+  return mark(6);
 }
 
 }  // namespace
@@ -436,33 +540,38 @@ moe_status moe_combine(const moe_shape* s, const void* y_perm, const int32_t* sl
 moe_status moe_forward(const moe_shape* s, const void* x, const void* packed, const float* bias,
                        const int32_t* expert_rank_host, void* y, const moe_forward_buffers* buffers,
                        void* ws, size_t ws_bytes, moe_stream_t stream) {
+  return forward_impl(s, x, packed, bias, expert_rank_host, y, buffers, ws, ws_bytes,
+                      (cudaStream_t)stream, nullptr);
+}
+
+moe_status moe_forward_timed(const moe_shape* s, const void* x, const void* packed,
+                             const float* bias, const int32_t* expert_rank_host, void* y,
+                             const moe_forward_buffers* buffers, void* ws, size_t ws_bytes,
+                             moe_event_t* events, moe_stream_t stream) {
+  if (!events) return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i <= MOE_FORWARD_STAGES; ++i)
+    if (!events[i]) return MOE_ERR_INVALID_ARG;
+  return forward_impl(s, x, packed, bias, expert_rank_host, y, buffers, ws, ws_bytes,
+                      (cudaStream_t)stream, reinterpret_cast<cudaEvent_t*>(events));
+}
+
+moe_status moe_grouped_swiglu_gather(const moe_shape* s, const void* x, const int32_t* row_token,
+                                     const int32_t* offsets, const void* packed, void* h,
+                                     void* y_perm, void* ws, size_t ws_bytes, moe_stream_t stream) {
   moe_status r = check_shape(s);
   if (r != MOE_OK) return r;
-  if (!ws) return MOE_ERR_INVALID_ARG;
-  if (!aligned(ws, kAlign)) return MOE_ERR_ALIGNMENT;
-  if (ws_bytes < forward_bytes(s)) return MOE_ERR_WORKSPACE;
-  RankMap map;
-  if ((r = build_map(s, expert_rank_host, &map)) != MOE_OK) return r;
+  if (s->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
   if (s->T == 0) return MOE_OK;
-  if (!x || !packed || !y) return MOE_ERR_INVALID_ARG;
-  if (!aligned(x, 16) || !aligned(y, 16) || !aligned(packed, kAlign) || (bias && !aligned(bias, 4)))
+  if (!x || !row_token || !offsets || !packed || !h || !y_perm || !ws) return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(h, 16) || !aligned(y_perm, 16) || !aligned(offsets, 4) ||
+      !aligned(row_token, 4) || !aligned(packed, kAlign) || !aligned(ws, kAlign))
     return MOE_ERR_ALIGNMENT;
-  FwdBufs f = carve_forward(s, ws, buffers);
-  if ((r = check_layout_ptrs(s, &f.lay)) != MOE_OK) return r;
-  if (!aligned(f.logits, 4) || !aligned(f.idx, 4) || !aligned(f.gate, 4) || !aligned(f.x_perm, 16) ||
-      !aligned(f.h, 16) || !aligned(f.y_perm, 16))
-    return MOE_ERR_ALIGNMENT;
-  const Scratch sc = carve_scratch(s, ws);
+  if (ws_bytes < scratch_bytes(s)) return MOE_ERR_WORKSPACE;
   const Packed pk = carve_packed(s, packed);
+  Control* ctl = carve_scratch(s, ws).ctl;
   cudaStream_t st = (cudaStream_t)stream;
-  if ((r = do_route(s, x, &pk, bias, f.logits, f.idx, f.gate, sc.ctl, st)) != MOE_OK) return r;
-  if ((r = do_layout(s, f.idx, map, &f.lay, sc, -1, kWaitLimitNs, st)) != MOE_OK) return r;
-  if ((r = cuda_status(launch_permute(x, f.lay.row_token, f.x_perm, s->T, s->T * (int64_t)s->k,
-                                      (uint32_t)(s->d * esize(s->dtype)), st))) != MOE_OK)
-    return r;
-  if ((r = do_grouped(s, f.x_perm, f.lay.expert_offsets, &pk, f.h, f.y_perm, sc.ctl, st)) != MOE_OK)
-    return r;
-  return cuda_status(launch_combine(s->dtype, f.y_perm, f.lay.slot_row, f.gate, y, s->T, s->d, s->k, st));
+  if ((r = do_grouped_part(0, s, x, row_token, offsets, &pk, h, y_perm, ctl, st)) != MOE_OK) return r;
+  return do_grouped_part(1, s, x, nullptr, offsets, &pk, h, y_perm, ctl, st);
 }
 
 moe_status moe_get_device_status(void* ws, moe_stream_t stream, moe_status* out) {
@@ -474,8 +583,8 @@ moe_status moe_get_device_status(void* ws, moe_stream_t stream, moe_status* out)
   *out = (moe_status)v;
   if (v != MOE_OK) {
     if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), st) != cudaSuccess) return MOE_ERR_CUDA;
-    // the detail word (offset 8) is informational; clear it with the status
-    if (cudaMemsetAsync(static_cast<uint8_t*>(ws) + 8, 0, sizeof(uint32_t), st) != cudaSuccess)
+    // the detail word (offset 4) is informational; clear it with the status
+    if (cudaMemsetAsync(static_cast<uint8_t*>(ws) + 4, 0, sizeof(uint32_t), st) != cudaSuccess)
       return MOE_ERR_CUDA;
     if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
   }

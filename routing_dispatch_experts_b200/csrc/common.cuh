@@ -22,8 +22,8 @@ namespace moe {
 // The scratch workspace starts with this control block.
 struct Control {
   uint32_t status;       // moe_status recorded by a kernel (first error wins)
-  uint32_t ticket;       // dynamic block id counter of the lookback scan
   uint32_t detail;       // kernel-specific detail of the first error
+  uint32_t ticket;       // dynamic block id counter of the lookback scan
   uint32_t pad[61];
 };
 static_assert(sizeof(Control) == 256, "control block is 256 bytes");
@@ -110,6 +110,17 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const void* tmap, ui
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
       "[%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(smem_dst)),
       "l"(tmap), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+// 2-D gather of four rows (one-row-high box): rows[0..3] at column c0, into
+// four consecutive box rows of shared memory, completing on `bar`.
+__device__ __forceinline__ void tma_gather4(void* smem_dst, const void* tmap, uint64_t* bar,
+                                            int32_t c0, const int32_t (&rows)[4]) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(smem_dst)),
+      "l"(tmap), "r"(smem_u32(bar)), "r"(c0), "r"(rows[0]), "r"(rows[1]), "r"(rows[2]), "r"(rows[3])
       : "memory");
 }
 

@@ -118,23 +118,32 @@ __global__ void __launch_bounds__(256) grouped_f32_kernel(const float* __restric
 
 }  // namespace
 
-cudaError_t launch_grouped_f32(const float* x_perm, const int32_t* offsets, int E, int64_t R,
-                               int d, int f, int blk, const float* wgu, const float* wdT, float* h,
-                               float* y_perm, cudaStream_t s) {
+cudaError_t launch_grouped_f32_part(int part, const float* x_perm, const int32_t* offsets, int E,
+                                    int64_t R, int d, int f, int blk, const float* wgu,
+                                    const float* wdT, float* h, float* y_perm, cudaStream_t s) {
   if (R == 0) return cudaSuccess;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t mt_max = (R + TM - 1) / TM + E;
-  const int grid1 = (int)std::min<int64_t>(mt_max * (f / TN), (int64_t)sms * 8);
-  grouped_f32_kernel<true><<<grid1, 256, 0, s>>>(x_perm, offsets, E, d, f, wgu, blk,
-                                                 (int64_t)2 * f * d, h);
-  cudaError_t err = cudaGetLastError();
-  if (err != cudaSuccess) return err;
-  const int grid2 = (int)std::min<int64_t>(mt_max * (d / TN), (int64_t)sms * 8);
-  grouped_f32_kernel<false><<<grid2, 256, 0, s>>>(h, offsets, E, f, d, wdT, blk,
-                                                  (int64_t)d * f, y_perm);
+  if (part == 0) {
+    const int grid1 = (int)std::min<int64_t>(mt_max * (f / TN), (int64_t)sms * 8);
+    grouped_f32_kernel<true><<<grid1, 256, 0, s>>>(x_perm, offsets, E, d, f, wgu, blk,
+                                                   (int64_t)2 * f * d, h);
+  } else {
+    const int grid2 = (int)std::min<int64_t>(mt_max * (d / TN), (int64_t)sms * 8);
+    grouped_f32_kernel<false><<<grid2, 256, 0, s>>>(h, offsets, E, f, d, wdT, blk,
+                                                    (int64_t)d * f, y_perm);
+  }
   return cudaGetLastError();
+}
+
+cudaError_t launch_grouped_f32(const float* x_perm, const int32_t* offsets, int E, int64_t R,
+                               int d, int f, int blk, const float* wgu, const float* wdT, float* h,
+                               float* y_perm, cudaStream_t s) {
+  cudaError_t err = launch_grouped_f32_part(0, x_perm, offsets, E, R, d, f, blk, wgu, wdT, h, y_perm, s);
+  if (err != cudaSuccess) return err;
+  return launch_grouped_f32_part(1, x_perm, offsets, E, R, d, f, blk, wgu, wdT, h, y_perm, s);
 }
 
 }  // namespace moe

@@ -43,6 +43,8 @@ constexpr int kThreads = 192;
 
 struct Params {
   const int32_t* offsets;  // NULL: a single group of `rows` rows
+  const int32_t* gather;   // gather mode: A row r is source row gather[r]
+  int64_t src_rows;        // gather mode: rows of the source matrix
   int64_t rows;
   int G, K, n_per_group, n_out;
   void* out;
@@ -91,7 +93,7 @@ __device__ __forceinline__ float silu_mul(float g, float u) {
   return __fdividef(g, 1.f + __expf(-g)) * u;
 }
 
-template <int BN, int EPI>
+template <int BN, int EPI, bool GATHER>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ Params p) {
@@ -165,7 +167,52 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int kblocks = p.K / BK;
 
   if (warp == 0) {
-    if (lane == 0) {
+    if constexpr (GATHER) {
+      // Permute fused into the operand load: the tile's 128 A rows are rows
+      // gather[row0 .. row0+127] of the source (x), fetched by TMA gather4,
+      // four rows per lane (lane i: tile rows 4i..4i+3), into the same
+      // swizzled layout a tiled load would produce.  Rows past the end of
+      // the gather list read source row 0; their results are never stored.
+      uint32_t it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        const TileInfo ti = decode(tile, n_tiles, tile_off, s_off, G);
+        const int brow = ti.g * p.n_per_group + ti.nt * BN;
+        int32_t src[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int64_t r = (int64_t)ti.row0 + 4 * lane + u;
+          int32_t v = r < p.rows ? __ldg(p.gather + r) : 0;
+          src[u] = (v >= 0 && v < p.src_rows) ? v : 0;
+        }
+        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+          const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
+          int good = 1;
+          if (lane == 0) {
+            good = mbar_wait_bounded(&empty[s], ph ^ 1, &abort_flag);
+            if (good) {
+              mbar_arrive_expect_tx(&full[s], A_BYTES + B_BYTES);
+              tma_load_2d(sB + s * B_BYTES, &tmB, &full[s], kb * BK, brow);
+            }
+          }
+          good = __shfl_sync(0xffffffffu, good, 0);
+          if (!good) {
+            ok = false;
+            break;
+          }
+          tma_gather4(sA + s * A_BYTES + lane * 4 * (BK * 2), &tmA, &full[s], kb * BK, src);
+        }
+      }
+      if (lane == 0) {
+        if (!ok) {
+          abort_flag = 1;
+          record_error(p.ctl, MOE_ERR_DEVICE_TIMEOUT, 0x100u);
+        }
+        const uint32_t first = it > (uint32_t)STAGES ? it - STAGES : 0;
+        for (uint32_t q = first; q < it; ++q)
+          mbar_wait_bounded(&full[q % STAGES], (q / STAGES) & 1, nullptr);
+      }
+    } else if (lane == 0) {
       uint32_t it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
@@ -313,7 +360,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+}  // namespace
+
 // ------------------------------------------------------------- host side
+namespace {
 PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (!fn) {
@@ -326,8 +376,11 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   return fn;
 }
 
-// 2-D bf16 K-major operand [rows, K]: box of 64 K-elements (128 B) x box_rows
-bool make_map(CUtensorMap* m, const void* base, int64_t rows, int K, int box_rows) {
+}  // namespace
+
+// 2-D bf16 K-major operand [rows, K]: box of 64 K-elements (128 B) x box_rows,
+// 128-byte swizzle, out-of-range rows read as zero
+bool make_kmajor_map(CUtensorMap* m, const void* base, int64_t rows, int K, int box_rows) {
   auto enc = get_encode();
   if (!enc) return false;
   cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
@@ -340,21 +393,28 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int K, int box_row
   return r == CUDA_SUCCESS;
 }
 
-template <int BN, int EPI>
+namespace {
+
+template <int BN, int EPI, bool GATHER>
 cudaError_t run(const GemmArgs& a, cudaStream_t s) {
   static bool attr_set = false;
   constexpr size_t smem = smem_bytes_for<BN>();
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI>,
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI, GATHER>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   CUtensorMap mA, mB;
-  if (!make_map(&mA, a.A, a.rows, a.K, BM)) return cudaErrorInvalidValue;
-  if (!make_map(&mB, a.B, (int64_t)a.G * a.n_per_group, a.K, BN)) return cudaErrorInvalidValue;
+  // gather mode: A is the source matrix read one row per gathered coordinate
+  if (GATHER ? !make_kmajor_map(&mA, a.A, a.src_rows, a.K, 1)
+             : !make_kmajor_map(&mA, a.A, a.rows, a.K, BM))
+    return cudaErrorInvalidValue;
+  if (!make_kmajor_map(&mB, a.B, (int64_t)a.G * a.n_per_group, a.K, BN)) return cudaErrorInvalidValue;
   Params p;
   p.offsets = a.offsets;
+  p.gather = a.gather;
+  p.src_rows = a.src_rows;
   p.rows = a.rows;
   p.G = a.offsets ? a.G : 1;
   p.K = a.K;
@@ -372,7 +432,7 @@ cudaError_t run(const GemmArgs& a, cudaStream_t s) {
   const int64_t tiles_max = mt_max * (a.n_per_group / BN);
   const int grid = (int)std::min<int64_t>(tiles_max, sms);
   if (grid <= 0) return cudaSuccess;
-  gemm_tc_kernel<BN, EPI><<<grid, kThreads, smem, s>>>(mA, mB, p);
+  gemm_tc_kernel<BN, EPI, GATHER><<<grid, kThreads, smem, s>>>(mA, mB, p);
   return cudaGetLastError();
 }
 
@@ -380,29 +440,18 @@ cudaError_t run(const GemmArgs& a, cudaStream_t s) {
 
 cudaError_t launch_gemm_tc(int epi, int bn, const GemmArgs& a, cudaStream_t s) {
   if (a.rows == 0) return cudaSuccess;
+  const bool g = a.gather != nullptr;
 #define MOE_GEMM_CASE(EPI, BN) \
-  if (epi == EPI && bn == BN) return run<BN, EPI>(a, s);
+  if (epi == EPI && bn == BN) return g ? run<BN, EPI, true>(a, s) : run<BN, EPI, false>(a, s);
   MOE_GEMM_CASE(kEpiSwiGLU, 256)
   MOE_GEMM_CASE(kEpiSwiGLU, 128)
+  if (g) return cudaErrorInvalidValue;  // gather is for the gate/up GEMM
+#undef MOE_GEMM_CASE
+#define MOE_GEMM_CASE(EPI, BN) \
+  if (epi == EPI && bn == BN) return run<BN, EPI, false>(a, s);
   MOE_GEMM_CASE(kEpiBF16, 256)
   MOE_GEMM_CASE(kEpiBF16, 128)
   MOE_GEMM_CASE(kEpiBF16, 64)
-  MOE_GEMM_CASE(kEpiLogits, 16)
-  MOE_GEMM_CASE(kEpiLogits, 32)
-  MOE_GEMM_CASE(kEpiLogits, 48)
-  MOE_GEMM_CASE(kEpiLogits, 64)
-  MOE_GEMM_CASE(kEpiLogits, 80)
-  MOE_GEMM_CASE(kEpiLogits, 96)
-  MOE_GEMM_CASE(kEpiLogits, 112)
-  MOE_GEMM_CASE(kEpiLogits, 128)
-  MOE_GEMM_CASE(kEpiLogits, 144)
-  MOE_GEMM_CASE(kEpiLogits, 160)
-  MOE_GEMM_CASE(kEpiLogits, 176)
-  MOE_GEMM_CASE(kEpiLogits, 192)
-  MOE_GEMM_CASE(kEpiLogits, 208)
-  MOE_GEMM_CASE(kEpiLogits, 224)
-  MOE_GEMM_CASE(kEpiLogits, 240)
-  MOE_GEMM_CASE(kEpiLogits, 256)
 #undef MOE_GEMM_CASE
   return cudaErrorInvalidValue;
 }

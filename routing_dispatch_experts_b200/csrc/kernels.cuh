@@ -18,7 +18,7 @@ cudaError_t launch_router_f32(const float* x, const float* wrT, const float* bia
                               int d, int E, float* logits, cudaStream_t s);
 
 // ---- layout.cu
-constexpr int kTokPerBlock = 512;        // tokens per lookback block
+constexpr int kTokPerBlock = 128;        // tokens per lookback block (= one router tile)
 constexpr int kLayoutThreads = 256;
 constexpr int kMaxBins = 256 + 256 + 2;  // experts + ranks + two stat counters
 
@@ -35,6 +35,14 @@ cudaError_t launch_layout(const int32_t* idx, int64_t T, int k, int E, int ep, c
                           const LayoutOut& out, Control* ctl, uint64_t* status_words,
                           int32_t* prefix, int32_t* totals, int stall_block, int64_t limit_ns,
                           cudaStream_t s);
+// zero the ticket counter and the lookback status words of a layout
+cudaError_t clear_lookback(Control* ctl, uint64_t* status_words, int64_t T, int E, int ep,
+                           cudaStream_t s);
+// the scatter half of the layout, after block prefixes and totals exist
+// (from the histogram kernel or the fused router)
+cudaError_t launch_layout_scatter(const int32_t* idx, int64_t T, int k, int E, int ep,
+                                  const RankMap& map, const LayoutOut& out, Control* ctl,
+                                  int32_t* prefix, int32_t* totals, cudaStream_t s);
 
 // ---- permute_combine.cu
 cudaError_t launch_permute(const void* x, const int32_t* row_token, void* x_perm, int64_t T,
@@ -59,13 +67,44 @@ struct GemmArgs {
   int64_t ld_out;          // output row stride in elements
   const float* bias;       // kEpiLogits only, may be NULL
   Control* ctl;
+  // gather mode (gate/up GEMM only): A row r is row gather[r] of A, which
+  // then has src_rows rows -- the permute fused into the operand load
+  const int32_t* gather = nullptr;
+  int64_t src_rows = 0;
 };
 cudaError_t launch_gemm_tc(int epi, int bn, const GemmArgs& a, cudaStream_t s);
+bool make_kmajor_map(CUtensorMap* m, const void* base, int64_t rows, int K, int box_rows);
+
+// ---- route_tc.cu (bf16, tcgen05): router GEMM + bias + top-k + gates in one
+// kernel, optionally with the layout histogram and its lookback scan
+struct RouteArgs {
+  const void* x;        // [T, d] bf16
+  const void* wrT;      // [E16, d] bf16 (packed router)
+  const float* bias;    // [E] or NULL
+  int64_t T;
+  int d, E, k;
+  float* logits;        // [T, E]
+  int32_t* idx;         // [T, k]
+  float* gate;          // [T, k]
+  Control* ctl;
+  // histogram + lookback for the dispatch layout (hist = false: skipped)
+  bool hist;
+  int ep;
+  RankMap map;
+  uint64_t* status_words;
+  int32_t* prefix;
+  int32_t* totals;
+};
+cudaError_t launch_route_tc(const RouteArgs& a, cudaStream_t s);
 
 // ---- gemm_simt.cu (fp32, CUDA cores)
 cudaError_t launch_grouped_f32(const float* x_perm, const int32_t* offsets, int E, int64_t R,
                                int d, int f, int blk, const float* wgu, const float* wdT, float* h,
                                float* y_perm, cudaStream_t s);
+// part 0: gate/up + SwiGLU into h; part 1: down into y_perm
+cudaError_t launch_grouped_f32_part(int part, const float* x_perm, const int32_t* offsets, int E,
+                                    int64_t R, int d, int f, int blk, const float* wgu,
+                                    const float* wdT, float* h, float* y_perm, cudaStream_t s);
 
 // ---- pack.cu
 cudaError_t launch_pack(int dtype, int d, int E, int f, int blk, int E16, const void* w_router,

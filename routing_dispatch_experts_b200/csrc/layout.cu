@@ -1,14 +1,13 @@
 // layout.cu - expert-grouped dispatch layout and the deduplicated send layout.
 //
-// Two kernels over blocks of kTokPerBlock tokens (all k assignments of a
-// token stay in one block):
+// Blocks of kTokPerBlock tokens (all k assignments of a token stay in one
+// block), two phases:
 //
-//  1. histogram + decoupled lookback: each block counts its assignments per
-//     expert, its distinct (token, rank) pairs per rank, and two statistics;
-//     it publishes its counts and walks back over its predecessors' published
-//     aggregates / inclusive prefixes to get its exclusive prefix in every bin
-//     (single pass, dynamic block ids from a ticket counter, so a block only
-//     ever waits on blocks that are already running).  Waits are bounded.
+//  1. histogram + decoupled lookback (lookback.cuh): each block counts its
+//     assignments per expert, its distinct (token, rank) pairs per rank, and
+//     two statistics, and obtains its exclusive prefix in every bin.  This
+//     phase is either layout_hist_kernel below or the epilogue of the fused
+//     router (route_tc.cu), which has the routing in registers already.
 //  2. stable scatter: expert offsets from the totals, then every warp places
 //     its contiguous run of assignments in flat-index order (match_any ranks
 //     equal experts inside a 32-wide step), giving rows ordered by
@@ -19,15 +18,15 @@
 // (each token is sent to each GPU once) and Table I (GPUs per token = distinct
 // destinations; deduplication = rows removed as duplicates; T/EP tokens per
 // GPU for the home rank).
-#include "kernels.cuh"
+#include "lookback.cuh"
 
 namespace moe {
 
 namespace {
 
-constexpr uint32_t kFlagNone = 0, kFlagAgg = 1, kFlagIncl = 2, kFlagErr = 3;
 constexpr int kWarps = kLayoutThreads / 32;
 constexpr int kTokPerWarp = kTokPerBlock / kWarps;
+constexpr int kMaxIdx = kTokPerBlock * 16;  // the block's routing, staged in smem
 
 struct Params {
   const int32_t* idx;
@@ -42,15 +41,6 @@ struct Params {
   LayoutOut out;
 };
 
-__device__ __forceinline__ void publish(uint64_t* w, uint32_t flag, uint32_t value) {
-  atomicExch(reinterpret_cast<unsigned long long*>(w),
-             ((unsigned long long)flag << 32) | (unsigned long long)value);
-}
-
-__device__ __forceinline__ uint64_t poll(const uint64_t* w) {
-  return *reinterpret_cast<const volatile unsigned long long*>(w);
-}
-
 __global__ void __launch_bounds__(kLayoutThreads) layout_hist_kernel(const __grid_constant__ Params p) {
   __shared__ int hist[kMaxBins];
   __shared__ int s_ticket;
@@ -59,36 +49,25 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_hist_kernel(const __gri
   if (tid == 0) s_ticket = (int)atomicAdd(&p.ctl->ticket, 1u);
   __syncthreads();
   const int b = s_ticket;
-  if (b >= p.nb) {  // the workspace was not zero-filled before first use
+  if (b >= p.nb) {  // only if two calls share one workspace at the same time
     if (tid == 0) record_error(p.ctl, MOE_ERR_WORKSPACE, (uint32_t)b);
     return;
   }
   const int64_t t0 = (int64_t)b * kTokPerBlock;
   const int64_t t1 = min(p.T, t0 + kTokPerBlock);
-  const int ebin_r = p.E;                                // first rank bin
-  const int sbin = p.E + (p.ep > 1 ? p.ep : 0);          // the two stat bins
+  const int sbin = p.E + (p.ep > 1 ? p.ep : 0);  // the two stat bins
   int single = 0, home = 0;
   for (int64_t t = t0 + tid; t < t1; t += kLayoutThreads) {
-    const int home_r = (int)((t * p.ep) / p.T);
-    int rs[16];
-    int nr = 0;
+    int e[16];
+    bool ok = true;
     for (int j = 0; j < p.k; ++j) {
-      const int e = __ldg(p.idx + t * p.k + j);
-      if ((unsigned)e >= (unsigned)p.E) {
+      e[j] = __ldg(p.idx + t * p.k + j);
+      if ((unsigned)e[j] >= (unsigned)p.E) {
         record_error(p.ctl, MOE_ERR_DEVICE_INDEX, (uint32_t)(t * p.k + j));
-        continue;
-      }
-      atomicAdd(&hist[e], 1);
-      const int r = p.ep > 1 ? p.map.r[e] : 0;
-      home += r == home_r;
-      bool seen = false;
-      for (int q = 0; q < nr; ++q) seen |= rs[q] == r;
-      if (!seen) {
-        rs[nr++] = r;
-        if (p.ep > 1) atomicAdd(&hist[ebin_r + r], 1);
+        ok = false;
       }
     }
-    single += nr == 1;
+    if (ok) count_token(e, p.k, t, p.T, p.E, p.ep, p.map, hist, &single, &home);
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) {
@@ -100,48 +79,15 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_hist_kernel(const __gri
     atomicAdd(&hist[sbin + 1], home);
   }
   __syncthreads();
-
-  // decoupled lookback, one bin per thread
-  const bool stalled = b == p.stall_block;
+  const bool publish = b != p.stall_block;
   for (int bin = tid; bin < p.bins; bin += kLayoutThreads) {
-    const uint32_t agg = (uint32_t)hist[bin];
-    uint64_t* mine = p.status + (size_t)b * p.bins + bin;
     uint32_t excl = 0;
-    if (b > 0) {
-      if (!stalled) publish(mine, kFlagAgg, agg);
-      bool ok = true;
-      for (int q = b - 1; q >= 0;) {
-        uint64_t w = poll(p.status + (size_t)q * p.bins + bin);
-        if ((uint32_t)(w >> 32) == kFlagNone) {
-          const uint64_t ts = globaltimer_ns();
-          do {
-            __nanosleep(64);
-            w = poll(p.status + (size_t)q * p.bins + bin);
-            if ((uint32_t)(w >> 32) != kFlagNone) break;
-          } while (globaltimer_ns() - ts <= (uint64_t)p.limit_ns);
-          if ((uint32_t)(w >> 32) == kFlagNone) {
-            ok = false;
-            break;
-          }
-        }
-        const uint32_t fl = (uint32_t)(w >> 32);
-        if (fl == kFlagErr) {
-          ok = false;
-          break;
-        }
-        excl += (uint32_t)w;
-        if (fl == kFlagIncl) break;
-        --q;
-      }
-      if (!ok) {
-        record_error(p.ctl, MOE_ERR_DEVICE_TIMEOUT, (uint32_t)b);
-        if (!stalled) publish(mine, kFlagErr, 0);
-        continue;
-      }
+    if (!lookback_bin(p.status, p.bins, b, bin, (uint32_t)hist[bin], publish, p.limit_ns, &excl)) {
+      record_error(p.ctl, MOE_ERR_DEVICE_TIMEOUT, (uint32_t)b);
+      continue;
     }
-    if (!stalled) publish(mine, kFlagIncl, excl + agg);
     p.prefix[(size_t)b * p.bins + bin] = (int32_t)excl;
-    if (b == p.nb - 1) p.totals[bin] = (int32_t)(excl + agg);
+    if (b == p.nb - 1) p.totals[bin] = (int32_t)(excl + (uint32_t)hist[bin]);
   }
 }
 
@@ -154,6 +100,7 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
 __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(const __grid_constant__ Params p) {
   __shared__ int s_off[kMaxBins + 2];  // expert offsets [E+1], then rank offsets [ep+1]
   __shared__ int wh[kWarps][kMaxBins];
+  __shared__ int s_idx[kMaxIdx];
   __shared__ int s_ok;
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -161,12 +108,13 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(const __
   const int E = p.E, ep = p.ep, k = p.k;
   const bool dedup = ep > 1;
   const int sbin = E + (dedup ? ep : 0);
+  const int64_t tb0 = (int64_t)b * kTokPerBlock;
+  const int ntok = (int)(p.T - tb0 < kTokPerBlock ? p.T - tb0 : kTokPerBlock);
 
-  // leave the lookback state clean for the next call (stream order puts this
-  // after every block of the histogram kernel)
-  for (int i = tid; i < p.bins; i += kLayoutThreads) p.status[(size_t)b * p.bins + i] = 0;
-  if (b == 0 && tid == 0) p.ctl->ticket = 0;
   if (tid == 0) s_ok = *reinterpret_cast<volatile uint32_t*>(&p.ctl->status) == MOE_OK;
+  // the block's routing, read once (coalesced) into shared memory
+  for (int i = tid; i < ntok * k; i += kLayoutThreads) s_idx[i] = __ldg(p.idx + tb0 * k + i);
+  for (int i = tid; i < kWarps * kMaxBins; i += kLayoutThreads) (&wh[0][0])[i] = 0;
   __syncthreads();
   if (!s_ok) return;
 
@@ -190,6 +138,21 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(const __
         carry += __shfl_sync(0xffffffffu, incl, 31);
       }
       if (lane == 0) dst[n] = carry;
+    }
+  }
+  // per-warp histograms of this block's assignments / send rows
+  const int tw0 = min(ntok, warp * kTokPerWarp), tw1 = min(ntok, tw0 + kTokPerWarp);
+  const int aw0 = tw0 * k, aw1 = tw1 * k;
+  for (int a = aw0 + lane; a < aw1; a += 32) atomicAdd(&wh[warp][s_idx[a]], 1);
+  if (dedup) {
+    for (int t = tw0 + lane; t < tw1; t += 32) {
+      uint32_t m[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      for (int j = 0; j < k; ++j) {
+        const int r = p.map.r[s_idx[t * k + j]];
+        m[r >> 5] |= 1u << (r & 31);
+      }
+      for (int i = 0; i < 8; ++i)
+        for (uint32_t u = m[i]; u; u &= u - 1) atomicAdd(&wh[warp][E + (i << 5) + __ffs(u) - 1], 1);
     }
   }
   __syncthreads();
@@ -231,30 +194,6 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(const __
     }
   }
 
-  // per-warp histograms of this block's assignments / send rows
-  for (int i = tid; i < kWarps * kMaxBins; i += kLayoutThreads) (&wh[0][0])[i] = 0;
-  __syncthreads();
-  const int64_t tb0 = (int64_t)b * kTokPerBlock;
-  const int64_t tw0 = min(p.T, tb0 + (int64_t)warp * kTokPerWarp);
-  const int64_t tw1 = min(p.T, tw0 + kTokPerWarp);
-  const int64_t aw0 = tw0 * k, aw1 = tw1 * k;
-  for (int64_t a = aw0 + lane; a < aw1; a += 32) atomicAdd(&wh[warp][__ldg(p.idx + a)], 1);
-  if (dedup) {
-    for (int64_t t = tw0 + lane; t < tw1; t += 32) {
-      int rs[16];
-      int nr = 0;
-      for (int j = 0; j < k; ++j) {
-        const int r = p.map.r[__ldg(p.idx + t * k + j)];
-        bool seen = false;
-        for (int q = 0; q < nr; ++q) seen |= rs[q] == r;
-        if (!seen) {
-          rs[nr++] = r;
-          atomicAdd(&wh[warp][E + r], 1);
-        }
-      }
-    }
-  }
-  __syncthreads();
   // warp-exclusive starting rows: global offset + this block's lookback
   // prefix + the counts of the block's earlier warps
   const int nbins_used = E + (dedup ? ep : 0);
@@ -271,15 +210,16 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(const __
 
   // stable scatter of the assignments, in flat-index order
   const uint32_t lt = lanemask_lt();
-  for (int64_t a0 = aw0; a0 < aw1; a0 += 32) {
-    const int64_t a = a0 + lane;
+  for (int a0 = aw0; a0 < aw1; a0 += 32) {
+    const int a = a0 + lane;
     const bool valid = a < aw1;
-    const int e = valid ? __ldg(p.idx + a) : -1;
+    const int e = valid ? s_idx[a] : -1;
     const uint32_t peers = __match_any_sync(0xffffffffu, e);
     if (valid) {
       const int row = wh[warp][e] + __popc(peers & lt);
-      p.out.row_token[row] = (int32_t)(a / k);
-      p.out.slot_row[a] = row;
+      const int64_t ga = tb0 * k + a;
+      p.out.row_token[row] = (int32_t)(ga / k);
+      p.out.slot_row[ga] = row;
     }
     __syncwarp();
     if (valid && lane == __ffs(peers) - 1) wh[warp][e] += __popc(peers);
@@ -289,16 +229,15 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(const __
   // deduplicated send rows, tokens in order, one row per distinct rank
   if (dedup) {
     const int nw = (ep + 31) >> 5;
-    for (int64_t tt = tw0; tt < tw1; tt += 32) {
-      const int64_t t = tt + lane;
+    for (int tt = tw0; tt < tw1; tt += 32) {
+      const int t = tt + lane;
       const bool valid = t < tw1;
-      uint32_t m[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) m[i] = 0;
+      uint32_t m[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      int rr[16];
       if (valid)
         for (int j = 0; j < k; ++j) {
-          const int r = p.map.r[__ldg(p.idx + t * k + j)];
-          m[r >> 5] |= 1u << (r & 31);
+          rr[j] = p.map.r[s_idx[t * k + j]];
+          m[rr[j] >> 5] |= 1u << (rr[j] & 31);
         }
       for (int i = 0; i < nw; ++i) {
         uint32_t u = __reduce_or_sync(0xffffffffu, m[i]);
@@ -309,9 +248,10 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(const __
           const uint32_t bal = __ballot_sync(0xffffffffu, has);
           if (has) {
             const int srow = wh[warp][E + r] + __popc(bal & lt);
-            p.out.send_token[srow] = (int32_t)t;
+            const int64_t gt = tb0 + t;
+            p.out.send_token[srow] = (int32_t)gt;
             for (int j = 0; j < k; ++j)
-              if (p.map.r[__ldg(p.idx + t * k + j)] == r) p.out.slot_send_row[t * k + j] = srow;
+              if (rr[j] == r) p.out.slot_send_row[gt * k + j] = srow;
           }
           __syncwarp();
           if (lane == 0) wh[warp][E + r] += __popc(bal);
@@ -322,12 +262,9 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(const __
   }
 }
 
-}  // namespace
-
-cudaError_t launch_layout(const int32_t* idx, int64_t T, int k, int E, int ep, const RankMap& map,
-                          const LayoutOut& out, Control* ctl, uint64_t* status_words,
-                          int32_t* prefix, int32_t* totals, int stall_block, int64_t limit_ns,
-                          cudaStream_t s) {
+Params make_params(const int32_t* idx, int64_t T, int k, int E, int ep, const RankMap& map,
+                   const LayoutOut& out, Control* ctl, uint64_t* status_words, int32_t* prefix,
+                   int32_t* totals, int stall_block, int64_t limit_ns) {
   Params p;
   p.idx = idx;
   p.T = T;
@@ -344,20 +281,58 @@ cudaError_t launch_layout(const int32_t* idx, int64_t T, int k, int E, int ep, c
   p.prefix = prefix;
   p.totals = totals;
   p.out = out;
-  if (p.nb == 0) {
-    // no tokens: counts and offsets are all zero, no send rows
-    cudaError_t err = cudaMemsetAsync(out.counts, 0, sizeof(int32_t) * E, s);
-    if (err == cudaSuccess) err = cudaMemsetAsync(out.offsets, 0, sizeof(int32_t) * (E + 1), s);
-    if (err == cudaSuccess && ep > 1) {
-      err = cudaMemsetAsync(out.rank_counts, 0, sizeof(int32_t) * ep, s);
-      if (err == cudaSuccess) err = cudaMemsetAsync(out.rank_offsets, 0, sizeof(int32_t) * (ep + 1), s);
-    }
-    if (err == cudaSuccess && out.stats) err = cudaMemsetAsync(out.stats, 0, sizeof(moe_stats), s);
-    return err;
+  return p;
+}
+
+cudaError_t empty_layout(int E, int ep, const LayoutOut& out, cudaStream_t s) {
+  // no tokens: counts and offsets are all zero, no send rows
+  cudaError_t err = cudaMemsetAsync(out.counts, 0, sizeof(int32_t) * E, s);
+  if (err == cudaSuccess) err = cudaMemsetAsync(out.offsets, 0, sizeof(int32_t) * (E + 1), s);
+  if (err == cudaSuccess && ep > 1) {
+    err = cudaMemsetAsync(out.rank_counts, 0, sizeof(int32_t) * ep, s);
+    if (err == cudaSuccess) err = cudaMemsetAsync(out.rank_offsets, 0, sizeof(int32_t) * (ep + 1), s);
   }
-  layout_hist_kernel<<<p.nb, kLayoutThreads, 0, s>>>(p);
-  cudaError_t err = cudaGetLastError();
+  if (err == cudaSuccess && out.stats) err = cudaMemsetAsync(out.stats, 0, sizeof(moe_stats), s);
+  return err;
+}
+
+}  // namespace
+
+cudaError_t clear_lookback(Control* ctl, uint64_t* status_words, int64_t T, int E, int ep,
+                           cudaStream_t s) {
+  // The ticket counter and the lookback status words start every call at
+  // zero, whatever an earlier call of another shape left in the workspace.
+  const size_t words = (size_t)layout_blocks(T) * layout_bins(E, ep) * sizeof(uint64_t);
+  uint8_t* tk = reinterpret_cast<uint8_t*>(&ctl->ticket);
+  uint8_t* sw = reinterpret_cast<uint8_t*>(status_words);
+  if (sw == reinterpret_cast<uint8_t*>(ctl) + sizeof(Control))
+    return cudaMemsetAsync(tk, 0, (size_t)(sw - tk) + words, s);
+  cudaError_t err = cudaMemsetAsync(tk, 0, sizeof(uint32_t), s);
+  if (err == cudaSuccess) err = cudaMemsetAsync(sw, 0, words, s);
+  return err;
+}
+
+cudaError_t launch_layout(const int32_t* idx, int64_t T, int k, int E, int ep, const RankMap& map,
+                          const LayoutOut& out, Control* ctl, uint64_t* status_words,
+                          int32_t* prefix, int32_t* totals, int stall_block, int64_t limit_ns,
+                          cudaStream_t s) {
+  if (T == 0) return empty_layout(E, ep, out, s);
+  Params p = make_params(idx, T, k, E, ep, map, out, ctl, status_words, prefix, totals,
+                         stall_block, limit_ns);
+  cudaError_t err = clear_lookback(ctl, status_words, T, E, ep, s);
   if (err != cudaSuccess) return err;
+  layout_hist_kernel<<<p.nb, kLayoutThreads, 0, s>>>(p);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  layout_scatter_kernel<<<p.nb, kLayoutThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_layout_scatter(const int32_t* idx, int64_t T, int k, int E, int ep,
+                                  const RankMap& map, const LayoutOut& out, Control* ctl,
+                                  int32_t* prefix, int32_t* totals, cudaStream_t s) {
+  if (T == 0) return empty_layout(E, ep, out, s);
+  Params p = make_params(idx, T, k, E, ep, map, out, ctl, nullptr, prefix, totals, -1, 0);
   layout_scatter_kernel<<<p.nb, kLayoutThreads, 0, s>>>(p);
   return cudaGetLastError();
 }

@@ -1,0 +1,308 @@
+// route_tc.cu - the router in one tcgen05 kernel: logits GEMM, bias, top-k
+// selection, softmax gates, and (for the forward) the dispatch histogram with
+// its decoupled-lookback scan.
+//
+// Top-k routing with softmax gates over the k ("MoE Pretraining: Parallelism
+// Layout Changes the Model, Not Quality", Methodology: top-4 routing;
+// "Revisiting MoE and Dense Speed-Accuracy Comparisons", 2.1: Top-K routing;
+// router weights "ME", Table 1).
+//
+// One CTA per 128-token tile (ids from a ticket counter, in start order):
+//   warp 0      TMA producer: x tile [128 x 64] and W_r^T tile [E16 x 64] per
+//               k-block, 128-byte swizzle, 3-stage ring
+//   warp 1      TMEM allocation; one lane issues tcgen05.mma 128 x E16 x 16
+//   warps 2-5   epilogue, one token row per thread: tcgen05.ld of the row's
+//               E16 fp32 logits, + bias, logits stored, and a running top-k
+//               kept sorted in registers (key: logit desc, index asc; equal
+//               logits keep the lower index because only a strictly larger
+//               logit moves an entry); gates exp(l_j - l_0) / sum_i.
+// With the histogram on, each thread adds its token's experts, distinct
+// ranks and two statistics to a shared histogram, and the CTA runs the
+// lookback scan (lookback.cuh) for its tile: the layout's scatter kernel
+// then needs no separate histogram pass.
+#include <algorithm>
+
+#include "lookback.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int BM = 128, BK = 64, kThreads = 192, kStages = 3;
+
+struct Params {
+  int64_t T;
+  int K, E, BN, k;
+  const float* bias;
+  float* logits;
+  int32_t* idx;
+  float* gate;
+  Control* ctl;
+  int hist, ep, nb, bins;
+  int64_t limit_ns;
+  RankMap map;
+  uint64_t* status;
+  int32_t* prefix;
+  int32_t* totals;
+};
+
+// insert (v, e) into the descending list (tv, ti); e arrives in increasing
+// order, so an equal logit never displaces an earlier (lower) index
+template <int KMAX>
+__device__ __forceinline__ void topk_insert(float (&tv)[KMAX], int (&ti)[KMAX], float v, int e) {
+#pragma unroll
+  for (int s = KMAX - 1; s > 0; --s) {
+    const bool above = v > tv[s - 1];
+    const bool here = v > tv[s];
+    tv[s] = above ? tv[s - 1] : (here ? v : tv[s]);
+    ti[s] = above ? ti[s - 1] : (here ? e : ti[s]);
+  }
+  if (v > tv[0]) {
+    tv[0] = v;
+    ti[0] = e;
+  }
+}
+
+template <int KMAX>
+__global__ void __launch_bounds__(kThreads)
+    route_fused_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                       const __grid_constant__ Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t A_BYTES = BM * BK * 2;
+  const uint32_t B_BYTES = (uint32_t)p.BN * BK * 2;
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kStages * A_BYTES;
+
+  __shared__ __align__(8) uint64_t full[kStages], empty[kStages], tfull;
+  __shared__ uint32_t tmem_base_s;
+  __shared__ int s_tile;
+  __shared__ int hist[kMaxBins];
+  __shared__ volatile int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t tmem_cols = p.BN <= 32 ? 32 : (p.BN <= 64 ? 64 : (p.BN <= 128 ? 128 : 256));
+
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(&tfull, 1);
+    fence_barrier_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  for (int i = threadIdx.x; i < p.bins; i += kThreads) hist[i] = 0;
+  if (warp == 1) {
+    tmem_alloc(&tmem_base_s, tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  // the tile id is taken only once this CTA holds its tensor memory, so a
+  // CTA waiting in the lookback never waits on one still waiting to allocate
+  if (threadIdx.x == 0) s_tile = p.hist ? (int)atomicAdd(&p.ctl->ticket, 1u) : (int)blockIdx.x;
+  __syncthreads();
+  const uint32_t tmem_base = tmem_base_s;
+  const int b = s_tile;
+  const bool tile_ok = b < p.nb;  // false only if two calls share a workspace at once
+  const int64_t row0 = (int64_t)b * BM;
+  const int kblocks = p.K / BK;
+
+  if (warp == 0) {
+    if (lane == 0 && tile_ok) {
+      int kb = 0;
+      for (; kb < kblocks; ++kb) {
+        const uint32_t s = kb % kStages, ph = (kb / kStages) & 1;
+        if (!mbar_wait_bounded(&empty[s], ph ^ 1, &abort_flag)) {
+          abort_flag = 1;
+          record_error(p.ctl, MOE_ERR_DEVICE_TIMEOUT, 0x400u);
+          break;
+        }
+        mbar_arrive_expect_tx(&full[s], A_BYTES + B_BYTES);
+        tma_load_2d(sA + s * A_BYTES, &tmA, &full[s], kb * BK, (int32_t)row0);
+        tma_load_2d(sB + s * B_BYTES, &tmB, &full[s], kb * BK, 0);
+      }
+      for (int q = kb > kStages ? kb - kStages : 0; q < kb; ++q)  // drain
+        mbar_wait_bounded(&full[q % kStages], (q / kStages) & 1, nullptr);
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && tile_ok) {
+      const uint32_t idesc = idesc_bf16_f32(BM, p.BN);
+      bool ok = true;
+      for (int kb = 0; kb < kblocks; ++kb) {
+        const uint32_t s = kb % kStages, ph = (kb / kStages) & 1;
+        if (!mbar_wait_bounded(&full[s], ph, &abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a0 = smem_u32(sA + s * A_BYTES);
+        const uint32_t b0 = smem_u32(sB + s * B_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk)
+          tc_mma_f16(tmem_base, smem_desc_k128(a0 + kk * 32), smem_desc_k128(b0 + kk * 32), idesc,
+                     (kb | kk) != 0);
+        tc_commit(&empty[s]);
+      }
+      if (!ok) {
+        abort_flag = 1;
+        record_error(p.ctl, MOE_ERR_DEVICE_TIMEOUT, 0x500u);
+      }
+      // arrives when every MMA above has completed (also on the error path)
+      tc_commit(&tfull);
+    }
+  } else if (tile_ok) {
+    const int q = warp & 3;
+    const int rr = q * 32 + lane;
+    const int64_t t = row0 + rr;
+    const bool valid = t < p.T;
+    float tv[KMAX];
+    int ti[KMAX];
+#pragma unroll
+    for (int s = 0; s < KMAX; ++s) {
+      tv[s] = -INFINITY;
+      ti[s] = 0x7FFFFFFF;
+    }
+    if (mbar_wait_bounded(&tfull, 0, &abort_flag) && !abort_flag) {
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16);
+      float* lrow = p.logits + t * p.E;
+      const bool vec = (p.E & 3) == 0 && (reinterpret_cast<uintptr_t>(p.logits) & 15) == 0;
+      for (int c = 0; c < p.BN; c += 16) {
+        uint32_t r[16];
+        tmem_ld16(taddr + c, r);
+        tmem_ld_wait();
+        float v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int col = c + i;
+          v[i] = __uint_as_float(r[i]) + ((p.bias && col < p.E) ? __ldg(p.bias + col) : 0.f);
+        }
+        if (valid) {
+          if (vec && c + 16 <= p.E) {
+#pragma unroll
+            for (int i = 0; i < 16; i += 4)
+              *reinterpret_cast<float4*>(lrow + c + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+          } else {
+            for (int i = 0; i < 16 && c + i < p.E; ++i) lrow[c + i] = v[i];
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          if (c + i < p.E) topk_insert<KMAX>(tv, ti, v[i], c + i);
+      }
+      if (valid) {
+        float ex[KMAX];
+        float z = 0.f;
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+          ex[j] = j < p.k ? expf(tv[j] - tv[0]) : 0.f;
+          z += ex[j];
+        }
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j)
+          if (j < p.k) {
+            p.idx[t * p.k + j] = ti[j];
+            p.gate[t * p.k + j] = ex[j] / z;
+          }
+      }
+    }
+    if (p.hist) {
+      int single = 0, home = 0;
+      if (valid && !abort_flag) {
+        int e[KMAX];  // a copy, so the running list above stays in registers
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) e[j] = ti[j];
+        count_token(e, p.k, t, p.T, p.E, p.ep, p.map, hist, &single, &home);
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        single += __shfl_xor_sync(0xffffffffu, single, off);
+        home += __shfl_xor_sync(0xffffffffu, home, off);
+      }
+      const int sbin = p.E + (p.ep > 1 ? p.ep : 0);
+      if (lane == 0) {
+        atomicAdd(&hist[sbin], single);
+        atomicAdd(&hist[sbin + 1], home);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, tmem_cols);
+  }
+  if (p.hist && tile_ok) {
+    for (int bin = threadIdx.x; bin < p.bins; bin += kThreads) {
+      uint32_t excl = 0;
+      if (abort_flag ||
+          !lookback_bin(p.status, p.bins, b, bin, (uint32_t)hist[bin], true, p.limit_ns, &excl)) {
+        record_error(p.ctl, MOE_ERR_DEVICE_TIMEOUT, (uint32_t)b);
+        if (abort_flag) lb_publish(p.status + (size_t)b * p.bins + bin, kFlagErr, 0);
+        continue;
+      }
+      p.prefix[(size_t)b * p.bins + bin] = (int32_t)excl;
+      if (b == p.nb - 1) p.totals[bin] = (int32_t)(excl + (uint32_t)hist[bin]);
+    }
+  }
+}
+
+template <int KMAX>
+cudaError_t run(const RouteArgs& a, const CUtensorMap& mA, const CUtensorMap& mB, const Params& p,
+                cudaStream_t s) {
+  // dynamic shared memory grows with E; raise the kernel's limit when needed
+  static size_t attr_bytes = 0;
+  const size_t smem = (size_t)kStages * (BM * BK * 2 + (size_t)p.BN * BK * 2) + 1024;
+  if (smem > attr_bytes) {
+    cudaError_t e = cudaFuncSetAttribute(route_fused_kernel<KMAX>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attr_bytes = smem;
+  }
+  route_fused_kernel<KMAX><<<p.nb, kThreads, smem, s>>>(mA, mB, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_route_tc(const RouteArgs& a, cudaStream_t s) {
+  if (a.T == 0) return cudaSuccess;
+  Params p;
+  p.T = a.T;
+  p.K = a.d;
+  p.E = a.E;
+  p.BN = (a.E + 15) / 16 * 16;
+  p.k = a.k;
+  p.bias = a.bias;
+  p.logits = a.logits;
+  p.idx = a.idx;
+  p.gate = a.gate;
+  p.ctl = a.ctl;
+  p.hist = a.hist ? 1 : 0;
+  p.ep = a.ep;
+  p.nb = layout_blocks(a.T);
+  p.bins = layout_bins(a.E, a.ep);
+  p.limit_ns = kWaitLimitNs;
+  p.map = a.map;
+  p.status = a.status_words;
+  p.prefix = a.prefix;
+  p.totals = a.totals;
+  CUtensorMap mA, mB;
+  if (!make_kmajor_map(&mA, a.x, a.T, a.d, BM)) return cudaErrorInvalidValue;
+  if (!make_kmajor_map(&mB, a.wrT, p.BN, a.d, p.BN)) return cudaErrorInvalidValue;
+  if (a.hist) {
+    cudaError_t e = clear_lookback(a.ctl, a.status_words, a.T, a.E, a.ep, s);
+    if (e != cudaSuccess) return e;
+  }
+  if (a.k <= 2) return run<2>(a, mA, mB, p, s);
+  if (a.k <= 4) return run<4>(a, mA, mB, p, s);
+  if (a.k <= 8) return run<8>(a, mA, mB, p, s);
+  return run<16>(a, mA, mB, p, s);
+}
+
+}  // namespace moe

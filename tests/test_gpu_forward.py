@@ -96,6 +96,23 @@ def test_forward_is_deterministic_and_placement_invariant():
                 assert moe.stats_dict(buf.layout["stats"]) == ref["stats"]
 
 
+def test_forward_timed_matches_forward_and_orders_events():
+    """moe_forward_timed computes the same output and its stage events are
+    ordered in time (each stage's elapsed time is >= 0)."""
+    c = Case(2, T=4000)
+    shape = c.shape_ep(8)
+    ws = moe.workspace(shape, forward=True)
+    y0 = moe.forward(shape, c.dx, c.packed, None, ws)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(moe.FORWARD_STAGES) + 1)]
+    for e in ev:
+        e.record()
+    y1 = moe.forward_timed(shape, c.dx, c.packed, None, ws, ev)
+    torch.cuda.synchronize()
+    assert torch.equal(y0, y1)
+    ms = [ev[i].elapsed_time(ev[i + 1]) for i in range(len(moe.FORWARD_STAGES))]
+    assert all(m >= 0 for m in ms) and sum(ms) > 0
+
+
 def test_forward_correlated_placement_reduces_send_rows():
     """Top-2 workload: the greedy correlated placement (fit on a separate
     calibration batch through the oracle) removes more duplicate rows than

@@ -99,3 +99,32 @@ def test_grouped_swiglu_deterministic():
     a = moe.grouped_swiglu(shape, x_perm, off, packed, ws)[1]
     b = moe.grouped_swiglu(shape, x_perm, off, packed, ws)[1]
     assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("cfg,T,skew", [(2, 3000, False), (2, 1000, True), (3, 777, False),
+                                        (4, 300, True), (5, 129, False)])
+def test_gather_fused_permute_matches(cfg, T, skew):
+    """The gate/up GEMM reading rows of x through row_token (TMA gather)
+    gives bit-for-bit the outputs of moe_permute + moe_grouped_swiglu, and
+    matches the oracle."""
+    w = W.WORKLOADS[cfg]
+    x = W.make_x(w, T=T)
+    idx = _rows(w, T, skew, seed=T + 2 * cfg)
+    lay = oracle.dispatch_layout(idx.numpy(), w.E, 1)
+    rt = torch.from_numpy(lay["row_token"])
+    wg, wu, wd = W.make_experts(w)
+    shape = moe.Shape(T=T, d=w.d, E=w.E, k=w.k, f=w.f, dtype=w.torch_dtype)
+    packed = moe.pack_weights(shape, W.make_router(w).cuda(), wg.cuda(), wu.cuda(), wd.cuda())
+    ws = moe.workspace(shape)
+    off = torch.from_numpy(lay["expert_offsets"]).cuda()
+    dx, drt = x.cuda(), rt.cuda()
+    h1, y1 = moe.grouped_swiglu_gather(shape, dx, drt, off, packed, ws)
+    h0, y0 = moe.grouped_swiglu(shape, moe.permute(shape, dx, drt), off, packed, ws)
+    moe.check_device_status(ws)
+    assert torch.equal(h1, h0)
+    assert torch.equal(y1, y0)
+    R = T * w.k
+    rows = np.arange(R) if R * w.d * w.f < 4e9 else np.unique(W.sample_tokens(R, 200, seed=2).numpy())
+    ref = oracle.grouped_swiglu(x[rt.long()], lay["expert_offsets"], wg, wu, wd, rows=rows)
+    err = np.abs(y1.cpu().double().numpy()[rows] - ref).max()
+    assert err <= TOL[w.dtype] * np.abs(ref).max()
