@@ -255,8 +255,9 @@ MOE_API moe_status moe_grouped_swiglu(const moe_shape* shape, const void* x_perm
 /*
  * The permute fused into the grouped SwiGLU experts (bf16 only): the same
  * h and y_perm as moe_permute followed by moe_grouped_swiglu, but the
- * gate/up GEMM fetches row r of its operand straight from x[row_token[r]]
- * with TMA gather loads, so x_perm is never written or read.
+ * gate/up GEMM copies row r of its operand straight from x[row_token[r]]
+ * into shared memory (cp.async, 16 bytes per lane), so x_perm is never
+ * written or read.
  *  x [T, d]; row_token [T*k] (moe_dispatch_layout); other arguments as in
  *  moe_grouped_swiglu.  MOE_ERR_UNSUPPORTED for fp32.
  */
@@ -297,9 +298,10 @@ typedef struct {
  * The whole layer enqueued back to back on `stream`, with no host
  * synchronisation in between.  bf16: one kernel for router GEMM + top-k +
  * gates + the dispatch histogram and its lookback scan, the layout scatter,
- * the gate/up GEMM reading rows of x through the permutation (as
- * moe_grouped_swiglu_gather; x_perm is not written), the down GEMM and the
- * combine.  fp32: moe_route, moe_dispatch_layout, moe_permute,
+ * the gate/up GEMM with SwiGLU, the down GEMM and the combine; the permute
+ * is fused into the gate/up GEMM (as moe_grouped_swiglu_gather, x_perm not
+ * written) while x is at most 96 MB, and a separate moe_permute kernel
+ * otherwise.  fp32: moe_route, moe_dispatch_layout, moe_permute,
  * moe_grouped_swiglu and moe_combine in turn.
  *  x [T, d]; packed weights; bias [E] or NULL; expert_rank_host as in
  *  moe_dispatch_layout; y [T, d]; buffers may be NULL;
@@ -318,8 +320,8 @@ typedef struct CUevent_st* moe_event_t; /* same type as cudaEvent_t */
  * (0 route, 1 dispatch layout, 2 permute, 3 gate/up GEMM, 4 down GEMM,
  * 5 combine) and events[6] after the last, so cudaEventElapsedTime between
  * neighbours gives each stage's device time inside the forward.  A stage
- * that a path fuses into another (the permute on bf16) has no work between
- * its two events.  events: MOE_FORWARD_STAGES + 1 caller-created events.
+ * that a path fuses into another has no work between its two events.
+ * events: MOE_FORWARD_STAGES + 1 caller-created events.
  */
 MOE_API moe_status moe_forward_timed(const moe_shape* shape, const void* x,
                                      const void* packed, const float* bias,

@@ -307,6 +307,15 @@ moe_status layout_entry(const moe_shape* s, const int32_t* idx, const int32_t* h
   return do_layout(s, idx, map, o, carve_scratch(s, ws), stall, limit, st);
 }
 
+// The gathered gate/up GEMM reads each row of x once per expert that picks
+// it, 128 bytes at a time; that pays while x stays in the 126 MB L2, and a
+// separate streaming permute wins once x is much larger (measured on B200:
+// faster at x = 8 and 67 MB, slower at 268 MB).
+constexpr int64_t kGatherMaxBytes = 96ll << 20;
+bool gather_fits(const moe_shape* s) {
+  return s->dtype == MOE_BF16 && s->T * (int64_t)s->d * 2 <= kGatherMaxBytes;
+}
+
 moe_status forward_impl(const moe_shape* s, const void* x, const void* packed, const float* bias,
                         const int32_t* expert_rank_host, void* y, const moe_forward_buffers* buffers,
                         void* ws, size_t ws_bytes, cudaStream_t st, cudaEvent_t* ev) {
@@ -369,11 +378,23 @@ moe_status forward_impl(const moe_shape* s, const void* x, const void* packed, c
     if ((r = cuda_status(launch_layout_scatter(f.idx, s->T, s->k, s->E, s->ep, map, lo, sc.ctl,
                                                sc.prefix, sc.totals, st))) != MOE_OK)
       return r;
-    // no separate permute: the gate/up GEMM gathers its rows from x
-    if ((r = mark(2)) != MOE_OK || (r = mark(3)) != MOE_OK) return r;
-    if ((r = do_grouped_part(0, s, x, f.lay.row_token, f.lay.expert_offsets, &pk, f.h, f.y_perm,
-                             sc.ctl, st)) != MOE_OK)
-      return r;
+    if ((r = mark(2)) != MOE_OK) return r;
+    if (gather_fits(s)) {
+      // the permute is fused into the gate/up GEMM's operand loads
+      if ((r = mark(3)) != MOE_OK) return r;
+      if ((r = do_grouped_part(0, s, x, f.lay.row_token, f.lay.expert_offsets, &pk, f.h, f.y_perm,
+                               sc.ctl, st)) != MOE_OK)
+        return r;
+    } else {
+      if ((r = cuda_status(launch_permute(x, f.lay.row_token, f.x_perm, s->T,
+                                          s->T * (int64_t)s->k,
+                                          (uint32_t)(s->d * esize(s->dtype)), st))) != MOE_OK)
+        return r;
+      if ((r = mark(3)) != MOE_OK) return r;
+      if ((r = do_grouped_part(0, s, f.x_perm, nullptr, f.lay.expert_offsets, &pk, f.h, f.y_perm,
+                               sc.ctl, st)) != MOE_OK)
+        return r;
+    }
   } else {
     if ((r = do_route(s, x, &pk, bias, f.logits, f.idx, f.gate, sc.ctl, st)) != MOE_OK) return r;
     if ((r = mark(1)) != MOE_OK) return r;

@@ -124,6 +124,17 @@ __device__ __forceinline__ void tma_gather4(void* smem_dst, const void* tmap, ui
       : "memory");
 }
 
+// 16-byte asynchronous copy global -> shared (L2 only), generic proxy
+__device__ __forceinline__ void cp_async_16(uint32_t smem_dst, const void* gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_dst), "l"(gsrc) : "memory");
+}
+
+// one arrival on `bar` once every cp.async issued so far by this thread has
+// landed (counted among the barrier's expected arrivals)
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 // Untiled bulk copy global -> shared, completing on `bar` (16-B aligned,
 // size a multiple of 16).
 __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes,
@@ -140,6 +151,12 @@ __device__ __forceinline__ void bulk_store(void* gdst, const void* smem_src, uin
   asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst),
                "r"(smem_u32(smem_src)), "r"(bytes)
                : "memory");
+}
+
+// order this thread's generic-proxy shared-memory writes before later
+// async-proxy (bulk copy / tensor core) reads of them
+__device__ __forceinline__ void fence_proxy_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 __device__ __forceinline__ void bulk_commit() {

@@ -1,28 +1,30 @@
 // gemm_tc.cu - grouped GEMM on the fifth-generation tensor cores (tcgen05).
 //
-// The only dense contraction of the layer.  For each group g (an expert, or
-// the whole batch for the router) and each row r in [offsets[g],
-// offsets[g+1]):  acc[r, n] = sum_k A[r, k] * B[g*n_per_group + n, k], with
-// one of three epilogues:
+// The only dense contraction of the layer.  For each group g (an expert)
+// and each row r in [offsets[g], offsets[g+1]):
+//   acc[r, n] = sum_k A[r, k] * B[g*n_per_group + n, k]
+// with one of two epilogues:
 //   kEpiSwiGLU  B holds, per block of BN/2 output columns, the gate rows then
 //               the up rows of W_g / W_u; out = silu(acc_gate) * acc_up in
 //               bf16 (SwiGLU: "Revisiting MoE and Dense Speed-Accuracy
 //               Comparisons", 2.1 Architecture)
 //   kEpiBF16    out = acc in bf16 (the down projection)
-//   kEpiLogits  out = acc + bias in fp32 (the router GEMM)
 //
 // Design (one CTA per SM, persistent, 6 warps):
 //   warp 0      TMA producer: 128 x 64 A tiles and BN x 64 B tiles, 128-byte
 //               swizzle, into a STAGES-deep shared-memory ring (full/empty
-//               mbarriers)
+//               mbarriers).  Gather mode: the A rows are rows of x picked by
+//               the permutation, copied by the whole warp with cp.async into
+//               the same swizzled layout
 //   warp 1      allocates tensor memory (two BN-column fp32 accumulators) and
 //               one lane issues tcgen05.mma (M=128, N=BN, K=16) from shared-
 //               memory descriptors; tcgen05.commit frees smem stages and
 //               hands finished accumulators to the epilogue
 //   warps 2-5   epilogue: tcgen05.ld of the warp's 32 TMEM lanes (= tile
-//               rows), activation, bf16/fp32 rows stored to global memory;
-//               predicated on the group's last row so a tile never writes
-//               rows of the next expert
+//               rows), activation, bf16 rows to global memory -- straight
+//               from registers, or (short K loops) through shared memory with
+//               one bulk copy per row; predicated on the group's last row so
+//               a tile never writes rows of the next expert
 // The tile list is (group, 128-row tile, N tile), N fastest, walked with a
 // static stride of gridDim.x.  Group row counts come from device memory (no
 // host synchronisation); every CTA rebuilds the tile prefix in shared memory.
@@ -43,6 +45,7 @@ constexpr int kThreads = 192;
 
 struct Params {
   const int32_t* offsets;  // NULL: a single group of `rows` rows
+  const void* A;           // gather mode: the source matrix [src_rows, K]
   const int32_t* gather;   // gather mode: A row r is source row gather[r]
   int64_t src_rows;        // gather mode: rows of the source matrix
   int64_t rows;
@@ -54,18 +57,34 @@ struct Params {
 };
 
 template <int BN>
-constexpr int stages_for() {
-  return (BN >= 256) ? 4 : (BN >= 128 ? 6 : 8);
-}
-
-template <int BN>
 constexpr uint32_t tmem_cols_for() {
   return (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128 : (2 * BN <= 256) ? 256 : 512;
 }
 
-template <int BN>
+// output columns of one tile, and the padded bytes of one staged output row
+template <int BN, int EPI>
+constexpr int out_cols() { return EPI == kEpiSwiGLU ? BN / 2 : BN; }
+template <int BN, int EPI>
+constexpr uint32_t staged_row_bytes() { return out_cols<BN, EPI>() * 2 + 16; }
+
+// Staged epilogue: each epilogue thread writes its output row into shared
+// memory and one bulk copy per row moves it to global memory (whole rows,
+// coalesced, asynchronous).  Used when the K loop is short and the epilogue
+// would otherwise dominate; it costs pipeline stages.
+template <int BN, int EPI, bool STAGED>
+constexpr uint32_t staging_bytes() { return STAGED ? 128u * staged_row_bytes<BN, EPI>() : 0u; }
+
+template <int BN, int EPI, bool STAGED>
+constexpr int stages_for() {
+  constexpr uint32_t stage = BM * BK * 2 + BN * BK * 2;
+  constexpr uint32_t n = (220u * 1024u - staging_bytes<BN, EPI, STAGED>()) / stage;
+  return n > 8 ? 8 : (int)n;
+}
+
+template <int BN, int EPI, bool STAGED>
 constexpr size_t smem_bytes_for() {
-  return (size_t)stages_for<BN>() * (BM * BK * 2 + BN * BK * 2) + 1024;
+  return (size_t)stages_for<BN, EPI, STAGED>() * (BM * BK * 2 + BN * BK * 2) +
+         staging_bytes<BN, EPI, STAGED>() + 1024;
 }
 
 struct TileInfo {
@@ -93,11 +112,11 @@ __device__ __forceinline__ float silu_mul(float g, float u) {
   return __fdividef(g, 1.f + __expf(-g)) * u;
 }
 
-template <int BN, int EPI, bool GATHER>
+template <int BN, int EPI, bool GATHER, bool STAGED>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ Params p) {
-  constexpr int STAGES = stages_for<BN>();
+  constexpr int STAGES = stages_for<BN, EPI, STAGED>();
   constexpr uint32_t A_BYTES = BM * BK * 2;
   constexpr uint32_t B_BYTES = BN * BK * 2;
   constexpr uint32_t TMEM_COLS = tmem_cols_for<BN>();
@@ -108,6 +127,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_BYTES;
+  uint8_t* sOut = smem + STAGES * (A_BYTES + B_BYTES);  // staged epilogue rows
 
   __shared__ __align__(8) uint64_t full[STAGES], empty[STAGES], tfull[2], tempty[2], done;
   __shared__ uint32_t tmem_base_s;
@@ -142,7 +162,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       tile_off[G] = carry;
       for (int s = 0; s < STAGES; ++s) {
-        mbar_init(&full[s], 1);
+        // gather mode: the TMA arrival plus one cp.async arrival per lane
+        mbar_init(&full[s], GATHER ? 33 : 1);
         mbar_init(&empty[s], 1);
       }
       for (int b = 0; b < 2; ++b) {
@@ -169,21 +190,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     if constexpr (GATHER) {
       // Permute fused into the operand load: the tile's 128 A rows are rows
-      // gather[row0 .. row0+127] of the source (x), fetched by TMA gather4,
-      // four rows per lane (lane i: tile rows 4i..4i+3), into the same
-      // swizzled layout a tiled load would produce.  Rows past the end of
-      // the gather list read source row 0; their results are never stored.
+      // gather[row0 .. row0+127] of the source (x).  The whole warp copies
+      // them with 16-byte cp.async (lane l: chunk l%8 of rows 4i + l/8),
+      // writing the 128-byte-swizzled layout a TMA tile load would produce
+      // (chunk c of row r at c ^ (r % 8)); each lane's copies arrive on the
+      // stage barrier when they land.  B still comes by TMA.  Rows past the
+      // end of the gather list read source row 0; their results are never
+      // stored.
+      const int ch = lane & 7, rsub = lane >> 3;
       uint32_t it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         const TileInfo ti = decode(tile, n_tiles, tile_off, s_off, G);
         const int brow = ti.g * p.n_per_group + ti.nt * BN;
-        int32_t src[4];
+        int32_t src[BM / 4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int64_t r = (int64_t)ti.row0 + 4 * lane + u;
-          int32_t v = r < p.rows ? __ldg(p.gather + r) : 0;
-          src[u] = (v >= 0 && v < p.src_rows) ? v : 0;
+        for (int i = 0; i < BM / 4; ++i) {
+          const int64_t r = (int64_t)ti.row0 + 4 * i + rsub;
+          const int32_t v = r < p.rows ? __ldg(p.gather + r) : 0;
+          src[i] = (v >= 0 && v < p.src_rows) ? v : 0;
         }
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
           const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
@@ -191,7 +216,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) {
             good = mbar_wait_bounded(&empty[s], ph ^ 1, &abort_flag);
             if (good) {
-              mbar_arrive_expect_tx(&full[s], A_BYTES + B_BYTES);
+              mbar_arrive_expect_tx(&full[s], B_BYTES);
               tma_load_2d(sB + s * B_BYTES, &tmB, &full[s], kb * BK, brow);
             }
           }
@@ -200,7 +225,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          tma_gather4(sA + s * A_BYTES + lane * 4 * (BK * 2), &tmA, &full[s], kb * BK, src);
+          const __nv_bfloat16* xa = static_cast<const __nv_bfloat16*>(p.A) + kb * BK + ch * 8;
+          const uint32_t sa = smem_u32(sA + s * A_BYTES);
+#pragma unroll
+          for (int i = 0; i < BM / 4; ++i) {
+            const int r = 4 * i + rsub;
+            cp_async_16(sa + r * 128 + ((ch ^ (r & 7)) << 4), xa + (int64_t)src[i] * p.K);
+          }
+          cp_async_arrive_noinc(&full[s]);
         }
       }
       if (lane == 0) {
@@ -208,10 +240,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           abort_flag = 1;
           record_error(p.ctl, MOE_ERR_DEVICE_TIMEOUT, 0x100u);
         }
-        const uint32_t first = it > (uint32_t)STAGES ? it - STAGES : 0;
-        for (uint32_t q = first; q < it; ++q)
-          mbar_wait_bounded(&full[q % STAGES], (q / STAGES) & 1, nullptr);
       }
+      // drain: every issued stage completes before the CTA may exit
+      const uint32_t first = it > (uint32_t)STAGES ? it - STAGES : 0;
+      for (uint32_t q = first; q < it; ++q)
+        mbar_wait_bounded(&full[q % STAGES], (q / STAGES) & 1, nullptr);
     } else if (lane == 0) {
       uint32_t it = 0;
       bool ok = true;
@@ -256,6 +289,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
+          // cp.async wrote A through the generic proxy; the MMA reads it
+          // through the async proxy
+          if constexpr (GATHER) fence_proxy_async_shared();
           tc_fence_after();
           const uint32_t a0 = smem_u32(sA + s * A_BYTES);
           const uint32_t b0 = smem_u32(sB + s * B_BYTES);
@@ -292,59 +328,49 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + b * ACC_STRIDE;
       const bool valid = rr < ti.rows;
       const int64_t grow = (int64_t)ti.row0 + rr;
-      if constexpr (EPI == kEpiSwiGLU) {
-        constexpr int HALF = BN / 2;
-        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + grow * p.ld_out + ti.nt * HALF;
+      constexpr int OC = out_cols<BN, EPI>();
+      __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + grow * p.ld_out + ti.nt * OC;
+      uint8_t* stg = sOut + (size_t)rr * staged_row_bytes<BN, EPI>();
+      if constexpr (STAGED) bulk_wait_read<0>();  // this row's previous bulk store has read smem
 #pragma unroll 1
-        for (int c = 0; c < HALF; c += 16) {
+      for (int c = 0; c < OC; c += 16) {
+        uint32_t pk[8];
+        if constexpr (EPI == kEpiSwiGLU) {
           uint32_t gr[16], ur[16];
           tmem_ld16(taddr + c, gr);
-          tmem_ld16(taddr + HALF + c, ur);
+          tmem_ld16(taddr + OC + c, ur);
           tmem_ld_wait();
-          uint32_t pk[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i)
             pk[i] = pack_bf16x2(silu_mul(__uint_as_float(gr[2 * i]), __uint_as_float(ur[2 * i])),
                                 silu_mul(__uint_as_float(gr[2 * i + 1]), __uint_as_float(ur[2 * i + 1])));
-          if (valid) {
-            uint4* o = reinterpret_cast<uint4*>(out + c);
-            o[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            o[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-          }
-        }
-      } else if constexpr (EPI == kEpiBF16) {
-        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + grow * p.ld_out + ti.nt * BN;
-        const int ncols = min(BN, p.n_out - ti.nt * BN);
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 16) {
+        } else {
           uint32_t r[16];
           tmem_ld16(taddr + c, r);
           tmem_ld_wait();
-          uint32_t pk[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i)
             pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-          if (valid && c < ncols) {
-            uint4* o = reinterpret_cast<uint4*>(out + c);
-            o[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            o[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-          }
         }
-      } else {
-        float* out = static_cast<float*>(p.out) + grow * p.ld_out;
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 16) {
-          uint32_t r[16];
-          tmem_ld16(taddr + c, r);
-          tmem_ld_wait();
-          if (valid) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int col = c + i;
-              if (col < p.n_out) out[col] = __uint_as_float(r[i]) + (p.bias ? __ldg(p.bias + col) : 0.f);
-            }
-          }
+        if constexpr (STAGED) {
+          uint4* o = reinterpret_cast<uint4*>(stg + c * 2);
+          o[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          o[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        } else if (valid) {
+          uint4* o = reinterpret_cast<uint4*>(out + c);
+          o[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          o[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         }
+      }
+      if constexpr (STAGED) {
+        // the accumulator is free once it is in shared memory
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[b]);
+        fence_proxy_async_shared();
+        if (valid) bulk_store(out, stg, OC * 2);
+        bulk_commit();
+        continue;
       }
       tc_fence_before();
       __syncwarp();
@@ -352,6 +378,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
+  if constexpr (STAGED) {
+    if (warp >= 2) bulk_wait<0>();  // staged rows written before the CTA exits
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -395,24 +424,23 @@ bool make_kmajor_map(CUtensorMap* m, const void* base, int64_t rows, int K, int 
 
 namespace {
 
-template <int BN, int EPI, bool GATHER>
+template <int BN, int EPI, bool GATHER, bool STAGED>
 cudaError_t run(const GemmArgs& a, cudaStream_t s) {
   static bool attr_set = false;
-  constexpr size_t smem = smem_bytes_for<BN>();
+  constexpr size_t smem = smem_bytes_for<BN, EPI, STAGED>();
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI, GATHER>,
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI, GATHER, STAGED>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   CUtensorMap mA, mB;
-  // gather mode: A is the source matrix read one row per gathered coordinate
-  if (GATHER ? !make_kmajor_map(&mA, a.A, a.src_rows, a.K, 1)
-             : !make_kmajor_map(&mA, a.A, a.rows, a.K, BM))
-    return cudaErrorInvalidValue;
+  // gather mode reads A with cp.async; its tensor map is built but unused
+  if (!make_kmajor_map(&mA, a.A, GATHER ? a.src_rows : a.rows, a.K, BM)) return cudaErrorInvalidValue;
   if (!make_kmajor_map(&mB, a.B, (int64_t)a.G * a.n_per_group, a.K, BN)) return cudaErrorInvalidValue;
   Params p;
   p.offsets = a.offsets;
+  p.A = a.A;
   p.gather = a.gather;
   p.src_rows = a.src_rows;
   p.rows = a.rows;
@@ -432,7 +460,7 @@ cudaError_t run(const GemmArgs& a, cudaStream_t s) {
   const int64_t tiles_max = mt_max * (a.n_per_group / BN);
   const int grid = (int)std::min<int64_t>(tiles_max, sms);
   if (grid <= 0) return cudaSuccess;
-  gemm_tc_kernel<BN, EPI, GATHER><<<grid, kThreads, smem, s>>>(mA, mB, p);
+  gemm_tc_kernel<BN, EPI, GATHER, STAGED><<<grid, kThreads, smem, s>>>(mA, mB, p);
   return cudaGetLastError();
 }
 
@@ -441,14 +469,18 @@ cudaError_t run(const GemmArgs& a, cudaStream_t s) {
 cudaError_t launch_gemm_tc(int epi, int bn, const GemmArgs& a, cudaStream_t s) {
   if (a.rows == 0) return cudaSuccess;
   const bool g = a.gather != nullptr;
-#define MOE_GEMM_CASE(EPI, BN) \
-  if (epi == EPI && bn == BN) return g ? run<BN, EPI, true>(a, s) : run<BN, EPI, false>(a, s);
+  // short K loops: stage the epilogue through shared memory (see above)
+  const bool st = a.K / BK <= 8;
+#define MOE_GEMM_CASE(EPI, BN)                                                         \
+  if (epi == EPI && bn == BN)                                                          \
+    return g ? (st ? run<BN, EPI, true, true>(a, s) : run<BN, EPI, true, false>(a, s)) \
+             : (st ? run<BN, EPI, false, true>(a, s) : run<BN, EPI, false, false>(a, s));
   MOE_GEMM_CASE(kEpiSwiGLU, 256)
   MOE_GEMM_CASE(kEpiSwiGLU, 128)
   if (g) return cudaErrorInvalidValue;  // gather is for the gate/up GEMM
 #undef MOE_GEMM_CASE
 #define MOE_GEMM_CASE(EPI, BN) \
-  if (epi == EPI && bn == BN) return run<BN, EPI, false>(a, s);
+  if (epi == EPI && bn == BN) return st ? run<BN, EPI, false, true>(a, s) : run<BN, EPI, false, false>(a, s);
   MOE_GEMM_CASE(kEpiBF16, 256)
   MOE_GEMM_CASE(kEpiBF16, 128)
   MOE_GEMM_CASE(kEpiBF16, 64)

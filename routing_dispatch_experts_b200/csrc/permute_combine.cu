@@ -14,17 +14,30 @@ namespace moe {
 namespace {
 
 // ---------------------------------------------------------------- permute
-// One warp per CTA.  Rows move in groups of `rps` rows (one group fills a
+// TMA-staged ring for rows longer than 1 KB.  One warp per CTA.  Rows move in groups of `rps` rows (one group fills a
 // 16 KB shared-memory stage); lane i of the warp owns row i of every group.
 // Lane i issues a TMA bulk load of its source row into the stage (completing
 // on the stage's mbarrier), then, LOOKAHEAD groups later, a TMA bulk store of
 // the staged row to its destination.  A lane reuses a stage region only after
 // its own bulk store from that region has finished reading (bulk-group wait),
 // so loads of group g+LOOKAHEAD overlap the stores of group g.
-constexpr int kPermStages = 4;
-constexpr int kPermLookahead = 2;
-constexpr uint32_t kPermStageBytes = 16384;
-constexpr int kPermCtasPerSm = 3;
+#ifndef MOE_PERM_STAGES
+#define MOE_PERM_STAGES 4
+#endif
+#ifndef MOE_PERM_LOOKAHEAD
+#define MOE_PERM_LOOKAHEAD 2
+#endif
+#ifndef MOE_PERM_STAGE_BYTES
+#define MOE_PERM_STAGE_BYTES 16384
+#endif
+#ifndef MOE_PERM_CTAS
+#define MOE_PERM_CTAS 3
+#endif
+constexpr int kPermStages = MOE_PERM_STAGES;
+constexpr int kPermLookahead = MOE_PERM_LOOKAHEAD;
+constexpr uint32_t kPermStageBytes = MOE_PERM_STAGE_BYTES;
+constexpr int kPermCtasPerSm = MOE_PERM_CTAS;
+static_assert(kPermLookahead < kPermStages, "lookahead must leave a stage to store from");
 
 __global__ void __launch_bounds__(32) permute_kernel(const uint8_t* __restrict__ x,
                                                      const int32_t* __restrict__ row_token,
@@ -77,6 +90,43 @@ __global__ void __launch_bounds__(32) permute_kernel(const uint8_t* __restrict__
     }
   }
   bulk_wait<0>();
+}
+
+// Register copy for short rows: each warp copies 32 16-byte vectors per
+// item (an item is a row, or a 512-byte piece of a longer row), U items in
+// flight per lane, loads all issued before the stores.
+template <int U>
+__global__ void __launch_bounds__(256) permute_vec_kernel(const uint4* __restrict__ x,
+                                                          const int32_t* __restrict__ row_token,
+                                                          uint4* __restrict__ x_perm, int64_t R,
+                                                          int64_t T, int V) {
+  const int lane = threadIdx.x & 31;
+  const int ipr = (V + 31) / 32;  // items per row
+  const int64_t items = R * ipr;
+  const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t it0 = warp0 * U; it0 < items; it0 += nwarps * U) {
+    uint4 v[U];
+    int64_t dst[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t it = it0 + u;
+      dst[u] = -1;
+      if (it < items) {
+        const int64_t r = it / ipr;
+        const int c = (int)(it - r * ipr) * 32 + lane;
+        if (c < V) {
+          int64_t src = __ldg(row_token + r);
+          if (src < 0 || src >= T) src = 0;
+          v[u] = __ldg(x + src * V + c);
+          dst[u] = r * V + c;
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      if (dst[u] >= 0) x_perm[dst[u]] = v[u];
+  }
 }
 
 // ---------------------------------------------------------------- combine
@@ -170,6 +220,18 @@ cudaError_t launch_permute(const void* x, const int32_t* row_token, void* x_perm
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // Short rows (<= 1 KB): the register copy keeps more rows in flight than
+  // the staged ring; longer rows go through the TMA-staged ring.
+  if (row_bytes <= 1024) {
+    constexpr int U = 4;
+    const int V = (int)(row_bytes / 16);
+    const int64_t items = R * ((V + 31) / 32);
+    const int64_t warps = (items + U - 1) / U;
+    const int grid = (int)std::min<int64_t>((warps + 7) / 8, (int64_t)sms * 8);
+    permute_vec_kernel<U><<<grid, 256, 0, s>>>(static_cast<const uint4*>(x), row_token,
+                                               static_cast<uint4*>(x_perm), R, T, V);
+    return cudaGetLastError();
+  }
   const int rps = (int)std::min<uint32_t>(32u, kPermStageBytes / row_bytes);
   const int64_t ngroups = (R + rps - 1) / rps;
   const int grid = (int)std::min<int64_t>(ngroups, (int64_t)sms * kPermCtasPerSm);
