@@ -151,11 +151,12 @@ MOE_API const char* moe_status_string(moe_status s);
 
 /*
  * Scratch workspace for moe_route, moe_dispatch_layout and
- * moe_grouped_swiglu (a few hundred KB): block histograms, the
- * decoupled-lookback status words, and the device status word.
+ * moe_grouped_swiglu (at most a few hundred KB): the device status word,
+ * per-bin totals, the decoupled-lookback status words and the fused
+ * router's per-tile histograms.
  * The workspace must be zero-filled once before its first use (cudaMemset or
- * moe_workspace_init); the library leaves it ready for the next call.
- * One workspace serves one stream at a time.
+ * moe_workspace_init); every call leaves it ready for the next call of any
+ * shape.  One workspace serves one stream at a time.
  */
 MOE_API moe_status moe_scratch_size(const moe_shape* shape, size_t* bytes);
 
@@ -367,9 +368,9 @@ MOE_API moe_status moe_debug_dispatch_layout_stall(const moe_shape* shape,
  * from when the library's device code is loaded until the process exits.
  * Nothing is allocated and nothing is freed by this call.
  *  - Shapes whose scratch exceeds 1 MiB are rejected with MOE_ERR_WORKSPACE
- *    (the scratch is 256 B + 12 B * ceil(T/128) * bins + 4 B * bins with
- *    bins = E + (ep > 1 ? ep : 0) + 2, each part rounded up to 256 B; e.g.
- *    E=64, ep=8 fits up to about 150k tokens, E=256, ep=256 about 21k).
+ *    (the scratch is 4352 B + 8 B * ceil(T/128) * bins, the second part
+ *    rounded up to 256 B, with bins = E + (ep > 1 ? ep : 0) + 2; e.g.
+ *    E=64, ep=8 fits up to about 225k tokens, E=256, ep=256 about 32k).
  *  - The first call on each device looks up the array's device address
  *    (cudaGetSymbolAddress) with that device current; make that first call
  *    before capturing any stream on that device.

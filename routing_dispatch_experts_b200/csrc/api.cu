@@ -36,18 +36,18 @@ moe_status check_shape(const moe_shape* s) {
   return MOE_OK;
 }
 
-// ---- scratch workspace: control block, lookback status words, prefixes
+// ---- scratch workspace: control block, per-bin totals, lookback words
 struct Scratch {
   Control* ctl;
-  uint64_t* status;
-  int32_t* prefix;
   int32_t* totals;
+  uint64_t* status;      // lookback words, zero between calls
+  int32_t* block_hist;   // per-block histogram rows of the fused router
 };
 
 size_t scratch_bytes(const moe_shape* s) {
   const size_t nb = (size_t)layout_blocks(s->T), bins = (size_t)layout_bins(s->E, s->ep);
-  return align_up(sizeof(Control)) + align_up(nb * bins * 8) + align_up(nb * bins * 4) +
-         align_up(bins * 4);
+  return align_up(sizeof(Control)) + kTotalsBytes + align_up(nb * bins * 8) +
+         align_up(nb * bins * 4);
 }
 
 Scratch carve_scratch(const moe_shape* s, void* ws) {
@@ -56,11 +56,11 @@ Scratch carve_scratch(const moe_shape* s, void* ws) {
   Scratch sc;
   sc.ctl = reinterpret_cast<Control*>(p);
   p += align_up(sizeof(Control));
+  sc.totals = reinterpret_cast<int32_t*>(p);
+  p += kTotalsBytes;
   sc.status = reinterpret_cast<uint64_t*>(p);
   p += align_up(nb * bins * 8);
-  sc.prefix = reinterpret_cast<int32_t*>(p);
-  p += align_up(nb * bins * 4);
-  sc.totals = reinterpret_cast<int32_t*>(p);
+  sc.block_hist = reinterpret_cast<int32_t*>(p);
   return sc;
 }
 
@@ -225,7 +225,7 @@ moe_status do_layout(const moe_shape* s, const int32_t* idx, const RankMap& map,
   lo.slot_send_row = o->slot_send_row;
   lo.stats = o->stats;
   return cuda_status(launch_layout(idx, s->T, s->k, s->E, s->ep, map, lo, sc.ctl, sc.status,
-                                   sc.prefix, sc.totals, stall, limit, st));
+                                   sc.totals, stall, limit, st));
 }
 
 // gate/up GEMM + SwiGLU (part 0) or down GEMM (part 1).  With `gather`
@@ -353,7 +353,7 @@ moe_status forward_impl(const moe_shape* s, const void* x, const void* packed, c
   const bool bf16 = s->dtype == MOE_BF16;
   if ((r = mark(0)) != MOE_OK) return r;
   if (bf16) {
-    // router + top-k + gates + dispatch histogram and lookback in one kernel
+    // router + top-k + gates + per-tile dispatch histogram in one kernel
     RouteArgs a{};
     a.x = x;
     a.wrT = pk.wrT;
@@ -369,14 +369,12 @@ moe_status forward_impl(const moe_shape* s, const void* x, const void* packed, c
     a.hist = true;
     a.ep = s->ep;
     a.map = map;
-    a.status_words = sc.status;
-    a.prefix = sc.prefix;
-    a.totals = sc.totals;
+    a.block_hist = sc.block_hist;
     if ((r = cuda_status(launch_route_tc(a, st))) != MOE_OK) return r;
     if ((r = mark(1)) != MOE_OK) return r;
     // the scatter half of the layout
     if ((r = cuda_status(launch_layout_scatter(f.idx, s->T, s->k, s->E, s->ep, map, lo, sc.ctl,
-                                               sc.prefix, sc.totals, st))) != MOE_OK)
+                                               sc.block_hist, st))) != MOE_OK)
       return r;
     if ((r = mark(2)) != MOE_OK) return r;
     if (gather_fits(s)) {

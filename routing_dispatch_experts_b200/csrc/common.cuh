@@ -48,6 +48,23 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
 
 __device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31; }
 
+// ------------------------------------------------ programmatic dependent launch
+// Kernels are launched with programmatic stream serialization (launch_pdl):
+// a kernel's CTAs may be scheduled while its predecessor in the stream is
+// still finishing (each predecessor CTA releases its successor when it
+// exits).  Each kernel runs its setup (barriers, tensor memory, descriptor
+// prefetch), then pdl_wait() -- which returns once the predecessor grid has
+// completed and its writes are visible -- before touching anything a
+// predecessor produced.  Without the launch attribute it is a no-op.
+// (Releasing successors earlier, at kernel start, measured slower on B200:
+// waiting successor CTAs then crowd the SMs the predecessor still uses.)
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// barrier among `count` threads (a multiple of 32) of the CTA, id 1..15
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // ------------------------------------------------------------------ mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));

@@ -34,6 +34,7 @@ __global__ void __launch_bounds__(256) grouped_f32_kernel(const float* __restric
   __shared__ float sG[TK][TN + 4];
   __shared__ float sU[SWIGLU ? TK : 1][TN + 4];
   const int tid = threadIdx.x;
+  pdl_wait();
   if (tid < 32) {
     int carry = 0;
     for (int g0 = 0; g0 < E; g0 += 32) {
@@ -128,14 +129,14 @@ cudaError_t launch_grouped_f32_part(int part, const float* x_perm, const int32_t
   const int64_t mt_max = (R + TM - 1) / TM + E;
   if (part == 0) {
     const int grid1 = (int)std::min<int64_t>(mt_max * (f / TN), (int64_t)sms * 8);
-    grouped_f32_kernel<true><<<grid1, 256, 0, s>>>(x_perm, offsets, E, d, f, wgu, blk,
-                                                   (int64_t)2 * f * d, h);
+    return launch_pdl(grouped_f32_kernel<true>, dim3(grid1), dim3(256), 0, s, x_perm, offsets, E,
+                      d, f, wgu, blk, (int64_t)2 * f * d, h);
   } else {
     const int grid2 = (int)std::min<int64_t>(mt_max * (d / TN), (int64_t)sms * 8);
-    grouped_f32_kernel<false><<<grid2, 256, 0, s>>>(h, offsets, E, f, d, wdT, blk,
-                                                    (int64_t)d * f, y_perm);
+    return launch_pdl(grouped_f32_kernel<false>, dim3(grid2), dim3(256), 0, s,
+                      static_cast<const float*>(h), offsets, E, f, d, wdT, blk, (int64_t)d * f,
+                      y_perm);
   }
-  return cudaGetLastError();
 }
 
 cudaError_t launch_grouped_f32(const float* x_perm, const int32_t* offsets, int E, int64_t R,

@@ -20,11 +20,12 @@
 //               one lane issues tcgen05.mma (M=128, N=BN, K=16) from shared-
 //               memory descriptors; tcgen05.commit frees smem stages and
 //               hands finished accumulators to the epilogue
-//   warps 2-5   epilogue: tcgen05.ld of the warp's 32 TMEM lanes (= tile
-//               rows), activation, bf16 rows to global memory -- straight
-//               from registers, or (short K loops) through shared memory with
-//               one bulk copy per row; predicated on the group's last row so
-//               a tile never writes rows of the next expert
+//   warps 2-9   epilogue, two warps per TMEM lane quadrant (each reads half
+//               of its 32 rows' columns): tcgen05.ld, activation, bf16 rows
+//               to global memory -- straight from registers, or (short K
+//               loops) through shared memory with one bulk copy per row;
+//               predicated on the group's last row so a tile never writes
+//               rows of the next expert
 // The tile list is (group, 128-row tile, N tile), N fastest, walked with a
 // static stride of gridDim.x.  Group row counts come from device memory (no
 // host synchronisation); every CTA rebuilds the tile prefix in shared memory.
@@ -41,7 +42,8 @@ namespace moe {
 namespace {
 
 constexpr int BM = 128, BK = 64;
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;                   // two per TMEM lane quadrant
+constexpr int kThreads = 64 + 32 * kEpiWarps;  // producer + MMA + epilogue
 
 struct Params {
   const int32_t* offsets;  // NULL: a single group of `rows` rows
@@ -138,6 +140,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.G;
 
+  // everything below reads what earlier kernels wrote (offsets, operands)
+  pdl_wait();
   // group offsets and the prefix of 128-row tiles per group
   // offsets clamped to [0, rows]: a malformed offset array can never make
   // the epilogue store outside the output
@@ -168,7 +172,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       for (int b = 0; b < 2; ++b) {
         mbar_init(&tfull[b], 1);
-        mbar_init(&tempty[b], 4);
+        mbar_init(&tempty[b], kEpiWarps);
       }
       mbar_init(&done, 1);
       fence_barrier_init();
@@ -313,8 +317,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait_bounded(&done, 0, nullptr);
     }
   } else {
-    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    // warps 2..9: quadrant q = warp % 4 (the TMEM lanes = tile rows this
+    // warp may read), half h of the tile's output columns
+    const int q = warp & 3;
+    const int h = (warp - 2) >> 2;
     const int rr = q * 32 + lane;
+    const int qbar = 1 + q;  // named barrier of the quadrant's two warps
     uint32_t tc = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tc) {
       const TileInfo ti = decode(tile, n_tiles, tile_off, s_off, G);
@@ -329,11 +337,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool valid = rr < ti.rows;
       const int64_t grow = (int64_t)ti.row0 + rr;
       constexpr int OC = out_cols<BN, EPI>();
+      constexpr int HC = OC / 2;
       __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + grow * p.ld_out + ti.nt * OC;
       uint8_t* stg = sOut + (size_t)rr * staged_row_bytes<BN, EPI>();
-      if constexpr (STAGED) bulk_wait_read<0>();  // this row's previous bulk store has read smem
+      if constexpr (STAGED) {
+        // the row's previous bulk store (issued by the h = 0 thread) has read
+        // the staging row before either half overwrites it
+        if (h == 0) bulk_wait_read<0>();
+        named_bar_sync(qbar, 64);
+      }
 #pragma unroll 1
-      for (int c = 0; c < OC; c += 16) {
+      for (int c = h * HC; c < (h + 1) * HC; c += 16) {
         uint32_t pk[8];
         if constexpr (EPI == kEpiSwiGLU) {
           uint32_t gr[16], ur[16];
@@ -368,8 +382,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[b]);
         fence_proxy_async_shared();
-        if (valid) bulk_store(out, stg, OC * 2);
-        bulk_commit();
+        named_bar_sync(qbar, 64);  // both halves of every row staged
+        if (h == 0) {
+          if (valid) bulk_store(out, stg, OC * 2);
+          bulk_commit();
+        }
         continue;
       }
       tc_fence_before();
@@ -379,7 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   if constexpr (STAGED) {
-    if (warp >= 2) bulk_wait<0>();  // staged rows written before the CTA exits
+    if (warp >= 2) bulk_wait<0>();  // staged rows written before the CTA exits (h = 0 owns them)
   }
   tc_fence_before();
   __syncthreads();
@@ -460,8 +477,8 @@ cudaError_t run(const GemmArgs& a, cudaStream_t s) {
   const int64_t tiles_max = mt_max * (a.n_per_group / BN);
   const int grid = (int)std::min<int64_t>(tiles_max, sms);
   if (grid <= 0) return cudaSuccess;
-  gemm_tc_kernel<BN, EPI, GATHER, STAGED><<<grid, kThreads, smem, s>>>(mA, mB, p);
-  return cudaGetLastError();
+  return launch_pdl(gemm_tc_kernel<BN, EPI, GATHER, STAGED>, dim3(grid), dim3(kThreads), smem, s,
+                    mA, mB, p);
 }
 
 }  // namespace

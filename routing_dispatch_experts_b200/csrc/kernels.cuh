@@ -5,6 +5,23 @@
 
 namespace moe {
 
+// Launch with programmatic stream serialization (see common.cuh).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // expert -> rank map passed by value to the layout kernels (E <= 256,
 // ep <= 256, so a rank fits one byte)
 struct RankMap {
@@ -31,18 +48,20 @@ struct LayoutOut {
   moe_stats* stats;
 };
 
+// Scratch layout shared by every layout path: the control block, then
+// kTotalsBytes for the per-bin totals, then the lookback status words
+// [nb][bins] (zero between calls).
+constexpr size_t kTotalsBytes = 4096;
+static_assert(kTotalsBytes >= kMaxBins * sizeof(int32_t), "totals fit");
+
 cudaError_t launch_layout(const int32_t* idx, int64_t T, int k, int E, int ep, const RankMap& map,
                           const LayoutOut& out, Control* ctl, uint64_t* status_words,
-                          int32_t* prefix, int32_t* totals, int stall_block, int64_t limit_ns,
-                          cudaStream_t s);
-// zero the ticket counter and the lookback status words of a layout
-cudaError_t clear_lookback(Control* ctl, uint64_t* status_words, int64_t T, int E, int ep,
-                           cudaStream_t s);
-// the scatter half of the layout, after block prefixes and totals exist
-// (from the histogram kernel or the fused router)
+                          int32_t* totals, int stall_block, int64_t limit_ns, cudaStream_t s);
+// the scatter half of the layout after the fused router, which left one
+// histogram column per 128-token block in block_hist [bins][nb]
 cudaError_t launch_layout_scatter(const int32_t* idx, int64_t T, int k, int E, int ep,
                                   const RankMap& map, const LayoutOut& out, Control* ctl,
-                                  int32_t* prefix, int32_t* totals, cudaStream_t s);
+                                  const int32_t* block_hist, cudaStream_t s);
 
 // ---- permute_combine.cu
 cudaError_t launch_permute(const void* x, const int32_t* row_token, void* x_perm, int64_t T,
@@ -87,13 +106,12 @@ struct RouteArgs {
   int32_t* idx;         // [T, k]
   float* gate;          // [T, k]
   Control* ctl;
-  // histogram + lookback for the dispatch layout (hist = false: skipped)
+  // per-block dispatch histogram for the layout scatter (hist = false:
+  // skipped): block_hist[bin][tile], layout_bins(E, ep) bins
   bool hist;
   int ep;
   RankMap map;
-  uint64_t* status_words;
-  int32_t* prefix;
-  int32_t* totals;
+  int32_t* block_hist;
 };
 cudaError_t launch_route_tc(const RouteArgs& a, cudaStream_t s);
 

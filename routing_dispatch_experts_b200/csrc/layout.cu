@@ -35,9 +35,9 @@ struct Params {
   int64_t limit_ns;
   RankMap map;
   Control* ctl;
-  uint64_t* status;  // [nb][bins]
-  int32_t* prefix;   // [nb][bins]
-  int32_t* totals;   // [bins]
+  uint64_t* status;  // [nb][bins] lookback words (histogram-kernel mode)
+  int32_t* totals;   // [bins]   (histogram-kernel mode)
+  const int32_t* block_hist;  // [bins][nb] per-block counts (fused-router mode)
   LayoutOut out;
 };
 
@@ -46,10 +46,11 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_hist_kernel(const __gri
   __shared__ int s_ticket;
   const int tid = threadIdx.x;
   for (int i = tid; i < p.bins; i += kLayoutThreads) hist[i] = 0;
+  pdl_wait();
   if (tid == 0) s_ticket = (int)atomicAdd(&p.ctl->ticket, 1u);
   __syncthreads();
   const int b = s_ticket;
-  if (b >= p.nb) {  // only if two calls share one workspace at the same time
+  if (b >= p.nb) {  // only if the workspace was not zeroed, or two calls share it at once
     if (tid == 0) record_error(p.ctl, MOE_ERR_WORKSPACE, (uint32_t)b);
     return;
   }
@@ -86,7 +87,6 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_hist_kernel(const __gri
       record_error(p.ctl, MOE_ERR_DEVICE_TIMEOUT, (uint32_t)b);
       continue;
     }
-    p.prefix[(size_t)b * p.bins + bin] = (int32_t)excl;
     if (b == p.nb - 1) p.totals[bin] = (int32_t)(excl + (uint32_t)hist[bin]);
   }
 }
@@ -101,6 +101,8 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(const __
   __shared__ int s_off[kMaxBins + 2];  // expert offsets [E+1], then rank offsets [ep+1]
   __shared__ int wh[kWarps][kMaxBins];
   __shared__ int s_idx[kMaxIdx];
+  __shared__ int s_pre[kMaxBins];  // this block's exclusive prefix per bin
+  __shared__ int s_tot[kMaxBins];  // totals per bin
   __shared__ int s_ok;
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -110,8 +112,52 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(const __
   const int sbin = E + (dedup ? ep : 0);
   const int64_t tb0 = (int64_t)b * kTokPerBlock;
   const int ntok = (int)(p.T - tb0 < kTokPerBlock ? p.T - tb0 : kTokPerBlock);
+  pdl_wait();
 
   if (tid == 0) s_ok = *reinterpret_cast<volatile uint32_t*>(&p.ctl->status) == MOE_OK;
+  if (p.block_hist) {
+    // fused-router mode: the kernel boundary already ordered every block's
+    // histogram, so sum them directly.  block_hist is [bins][nb]; warp w
+    // takes bins w, w+8, ..., its lanes read 32 consecutive blocks per load
+    // (independent loads, four bins at a time), and two warp reductions give
+    // the bin's total and this block's exclusive prefix (integer sums: exact)
+    for (int bin0 = warp * 4; bin0 < p.bins; bin0 += kWarps * 4) {
+      int pre[4] = {0, 0, 0, 0}, tot[4] = {0, 0, 0, 0};
+      for (int q0 = 0; q0 < p.nb; q0 += 32) {
+        const int q = q0 + lane;
+        int v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          v[u] = (q < p.nb && bin0 + u < p.bins) ? __ldg(p.block_hist + (size_t)(bin0 + u) * p.nb + q) : 0;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          tot[u] += v[u];
+          pre[u] += q < b ? v[u] : 0;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int t = __reduce_add_sync(0xffffffffu, tot[u]);
+        const int pr = __reduce_add_sync(0xffffffffu, pre[u]);
+        if (lane == 0 && bin0 + u < p.bins) {
+          s_tot[bin0 + u] = t;
+          s_pre[bin0 + u] = pr;
+        }
+      }
+    }
+  } else {
+    // histogram-kernel mode: this block's inclusive prefixes from its
+    // lookback words, which are then zeroed for the next call (nothing else
+    // reads them); block 0 resets the ticket counter.  The exclusive prefix
+    // is the inclusive one minus the block's own count (below).
+    uint64_t* words = p.status + (size_t)b * p.bins;
+    for (int i = tid; i < p.bins; i += kLayoutThreads) {
+      s_pre[i] = (int)(uint32_t)words[i];
+      s_tot[i] = p.totals[i];
+      words[i] = 0;
+    }
+    if (b == 0 && tid == 0) p.ctl->ticket = 0;
+  }
   // the block's routing, read once (coalesced) into shared memory
   for (int i = tid; i < ntok * k; i += kLayoutThreads) s_idx[i] = __ldg(p.idx + tb0 * k + i);
   for (int i = tid; i < kWarps * kMaxBins; i += kLayoutThreads) (&wh[0][0])[i] = 0;
@@ -127,7 +173,7 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(const __
       int carry = 0;
       for (int c0 = 0; c0 < n; c0 += 32) {
         const int i = c0 + lane;
-        const int v = i < n ? p.totals[base_bin + i] : 0;
+        const int v = i < n ? s_tot[base_bin + i] : 0;
         int incl = v;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
@@ -159,13 +205,13 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(const __
 
   if (b == 0) {
     for (int e = tid; e < E; e += kLayoutThreads) {
-      p.out.counts[e] = p.totals[e];
+      p.out.counts[e] = s_tot[e];
       p.out.offsets[e] = s_off[e];
     }
     if (tid == 0) p.out.offsets[E] = s_off[E];
     if (dedup) {
       for (int r = tid; r < ep; r += kLayoutThreads) {
-        p.out.rank_counts[r] = p.totals[E + r];
+        p.out.rank_counts[r] = s_tot[E + r];
         p.out.rank_offsets[r] = s_off[E + 1 + r];
       }
       if (tid == 0) p.out.rank_offsets[ep] = s_off[E + 1 + ep];
@@ -173,8 +219,8 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(const __
     if (p.out.stats && warp == 0) {
       int mx = 0, mn = 0x7FFFFFFF;
       for (int e = lane; e < E; e += 32) {
-        mx = max(mx, p.totals[e]);
-        mn = min(mn, p.totals[e]);
+        mx = max(mx, s_tot[e]);
+        mn = min(mn, s_tot[e]);
       }
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) {
@@ -185,8 +231,8 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(const __
         moe_stats st;
         st.rows_sent = dedup ? (int64_t)s_off[E + 1 + ep] : 0;
         st.dup_removed = dedup ? p.T * k - st.rows_sent : 0;
-        st.tokens_single_rank = p.totals[sbin];
-        st.home_rank_rows = p.totals[sbin + 1];
+        st.tokens_single_rank = s_tot[sbin];
+        st.home_rank_rows = s_tot[sbin + 1];
         st.max_expert_rows = mx;
         st.min_expert_rows = E > 0 ? mn : 0;
         *p.out.stats = st;
@@ -194,12 +240,14 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(const __
     }
   }
 
-  // warp-exclusive starting rows: global offset + this block's lookback
+  // warp-exclusive starting rows: global offset + this block's exclusive
   // prefix + the counts of the block's earlier warps
   const int nbins_used = E + (dedup ? ep : 0);
   for (int bin = tid; bin < nbins_used; bin += kLayoutThreads) {
-    int run = (bin < E ? s_off[bin] : s_off[E + 1 + (bin - E)]) +
-              p.prefix[(size_t)b * p.bins + bin];
+    int own = 0;
+    if (!p.block_hist)
+      for (int w = 0; w < kWarps; ++w) own += wh[w][bin];
+    int run = (bin < E ? s_off[bin] : s_off[E + 1 + (bin - E)]) + s_pre[bin] - own;
     for (int w = 0; w < kWarps; ++w) {
       const int c = wh[w][bin];
       wh[w][bin] = run;
@@ -263,8 +311,8 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(const __
 }
 
 Params make_params(const int32_t* idx, int64_t T, int k, int E, int ep, const RankMap& map,
-                   const LayoutOut& out, Control* ctl, uint64_t* status_words, int32_t* prefix,
-                   int32_t* totals, int stall_block, int64_t limit_ns) {
+                   const LayoutOut& out, Control* ctl, uint64_t* status_words, int32_t* totals,
+                   int stall_block, int64_t limit_ns) {
   Params p;
   p.idx = idx;
   p.T = T;
@@ -278,8 +326,8 @@ Params make_params(const int32_t* idx, int64_t T, int k, int E, int ep, const Ra
   p.map = map;
   p.ctl = ctl;
   p.status = status_words;
-  p.prefix = prefix;
   p.totals = totals;
+  p.block_hist = nullptr;
   p.out = out;
   return p;
 }
@@ -298,43 +346,24 @@ cudaError_t empty_layout(int E, int ep, const LayoutOut& out, cudaStream_t s) {
 
 }  // namespace
 
-cudaError_t clear_lookback(Control* ctl, uint64_t* status_words, int64_t T, int E, int ep,
-                           cudaStream_t s) {
-  // The ticket counter and the lookback status words start every call at
-  // zero, whatever an earlier call of another shape left in the workspace.
-  const size_t words = (size_t)layout_blocks(T) * layout_bins(E, ep) * sizeof(uint64_t);
-  uint8_t* tk = reinterpret_cast<uint8_t*>(&ctl->ticket);
-  uint8_t* sw = reinterpret_cast<uint8_t*>(status_words);
-  if (sw == reinterpret_cast<uint8_t*>(ctl) + sizeof(Control))
-    return cudaMemsetAsync(tk, 0, (size_t)(sw - tk) + words, s);
-  cudaError_t err = cudaMemsetAsync(tk, 0, sizeof(uint32_t), s);
-  if (err == cudaSuccess) err = cudaMemsetAsync(sw, 0, words, s);
-  return err;
-}
-
 cudaError_t launch_layout(const int32_t* idx, int64_t T, int k, int E, int ep, const RankMap& map,
                           const LayoutOut& out, Control* ctl, uint64_t* status_words,
-                          int32_t* prefix, int32_t* totals, int stall_block, int64_t limit_ns,
-                          cudaStream_t s) {
+                          int32_t* totals, int stall_block, int64_t limit_ns, cudaStream_t s) {
   if (T == 0) return empty_layout(E, ep, out, s);
-  Params p = make_params(idx, T, k, E, ep, map, out, ctl, status_words, prefix, totals,
-                         stall_block, limit_ns);
-  cudaError_t err = clear_lookback(ctl, status_words, T, E, ep, s);
+  Params p = make_params(idx, T, k, E, ep, map, out, ctl, status_words, totals, stall_block,
+                         limit_ns);
+  cudaError_t err = launch_pdl(layout_hist_kernel, dim3(p.nb), dim3(kLayoutThreads), 0, s, p);
   if (err != cudaSuccess) return err;
-  layout_hist_kernel<<<p.nb, kLayoutThreads, 0, s>>>(p);
-  err = cudaGetLastError();
-  if (err != cudaSuccess) return err;
-  layout_scatter_kernel<<<p.nb, kLayoutThreads, 0, s>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(layout_scatter_kernel, dim3(p.nb), dim3(kLayoutThreads), 0, s, p);
 }
 
 cudaError_t launch_layout_scatter(const int32_t* idx, int64_t T, int k, int E, int ep,
                                   const RankMap& map, const LayoutOut& out, Control* ctl,
-                                  int32_t* prefix, int32_t* totals, cudaStream_t s) {
+                                  const int32_t* block_hist, cudaStream_t s) {
   if (T == 0) return empty_layout(E, ep, out, s);
-  Params p = make_params(idx, T, k, E, ep, map, out, ctl, nullptr, prefix, totals, -1, 0);
-  layout_scatter_kernel<<<p.nb, kLayoutThreads, 0, s>>>(p);
-  return cudaGetLastError();
+  Params p = make_params(idx, T, k, E, ep, map, out, ctl, nullptr, nullptr, -1, 0);
+  p.block_hist = block_hist;
+  return launch_pdl(layout_scatter_kernel, dim3(p.nb), dim3(kLayoutThreads), 0, s, p);
 }
 
 }  // namespace moe

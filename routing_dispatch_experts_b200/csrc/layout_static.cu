@@ -9,8 +9,8 @@
 // allocator of its own.  cudaMalloc can also synchronise the whole device,
 // which latency-sensitive callers avoid.  Such a caller cannot provide the
 // workspace that moe_dispatch_layout takes, so this variant keeps the
-// layout's scratch (control word, decoupled-lookback status words, block
-// prefixes, totals) in `g_layout_scratch` below.
+// layout's scratch (control word, per-bin totals, decoupled-lookback status
+// words) in `g_layout_scratch` below.
 //
 // The array is a file-scope __device__ variable: every GPU that loads the
 // library holds its kStaticScratchBytes until the process exits.  Host code
@@ -76,10 +76,9 @@ extern "C" MOE_API moe_status moe_dispatch_layout_static(const moe_shape* s, con
 
   // the scratch this shape needs, laid out as in moe_dispatch_layout
   const size_t nb = (size_t)layout_blocks(s->T), bins = (size_t)layout_bins(s->E, s->ep);
-  const size_t off_status = round256(sizeof(Control));
-  const size_t off_prefix = off_status + round256(nb * bins * 8);
-  const size_t off_totals = off_prefix + round256(nb * bins * 4);
-  const size_t need = off_totals + round256(bins * 4);
+  const size_t off_totals = round256(sizeof(Control));
+  const size_t off_status = off_totals + kTotalsBytes;
+  const size_t need = off_status + round256(nb * bins * 8);
   if (need > kStaticScratchBytes) return MOE_ERR_WORKSPACE;
 
   // expert -> rank map: NULL = contiguous; otherwise a partition
@@ -100,7 +99,7 @@ extern "C" MOE_API moe_status moe_dispatch_layout_static(const moe_shape* s, con
   cudaStream_t st = (cudaStream_t)stream;
   // The array keeps whatever the previous call left; the control word, the
   // ticket counter and the lookback status words must start at zero.
-  if (cudaMemsetAsync(base, 0, off_prefix, st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemsetAsync(base, 0, need, st) != cudaSuccess) return MOE_ERR_CUDA;
   LayoutOut lo;
   lo.counts = o->expert_counts;
   lo.offsets = o->expert_offsets;
@@ -114,7 +113,6 @@ extern "C" MOE_API moe_status moe_dispatch_layout_static(const moe_shape* s, con
   Control* ctl = reinterpret_cast<Control*>(base);
   if (launch_layout(topk_idx, s->T, s->k, s->E, s->ep, map, lo, ctl,
                     reinterpret_cast<uint64_t*>(base + off_status),
-                    reinterpret_cast<int32_t*>(base + off_prefix),
                     reinterpret_cast<int32_t*>(base + off_totals), -1, kWaitLimitNs, st) != cudaSuccess)
     return MOE_ERR_CUDA;
   // the device-side status of this call (MOE_OK, MOE_ERR_DEVICE_INDEX or

@@ -8,7 +8,10 @@
 // inclusive prefix.  One 64-bit word per (block, bin) holds flag and value,
 // so a reader sees both together.  Waits give up after `limit_ns`; a block
 // that gives up records MOE_ERR_DEVICE_TIMEOUT and publishes an error flag so
-// its successors stop at once.  The words must be zero when the scan starts.
+// its successors stop at once.  The words must be zero when the scan starts;
+// the layout scatter kernel, the one reader of the results, zeroes each
+// block's words after reading them, so a workspace stays ready for the next
+// call of any shape.
 #pragma once
 
 #include "kernels.cuh"
@@ -28,6 +31,10 @@ __device__ __forceinline__ uint64_t lb_poll(const uint64_t* w) {
 
 // One bin of the scan for block b: returns false on time-out / error.
 // `publish_self` = false models a block that never publishes (test hook).
+// Predecessors are read kLookbackWindow at a time with independent loads,
+// so a block far from the last inclusive prefix needs few round trips.
+constexpr int kLookbackWindow = 8;
+
 __device__ __forceinline__ bool lookback_bin(uint64_t* status, int bins, int b, int bin,
                                              uint32_t agg, bool publish_self, int64_t limit_ns,
                                              uint32_t* excl_out) {
@@ -35,28 +42,40 @@ __device__ __forceinline__ bool lookback_bin(uint64_t* status, int bins, int b, 
   uint32_t excl = 0;
   if (b > 0) {
     if (publish_self) lb_publish(mine, kFlagAgg, agg);
-    for (int q = b - 1; q >= 0;) {
-      uint64_t w = lb_poll(status + (size_t)q * bins + bin);
-      if ((uint32_t)(w >> 32) == kFlagNone) {
-        const uint64_t ts = globaltimer_ns();
-        do {
-          __nanosleep(32);
-          w = lb_poll(status + (size_t)q * bins + bin);
-          if ((uint32_t)(w >> 32) != kFlagNone) break;
-        } while (globaltimer_ns() - ts <= (uint64_t)limit_ns);
-        if ((uint32_t)(w >> 32) == kFlagNone) {
+    int q = b - 1;
+    bool done = false;
+    while (!done && q >= 0) {
+      const int n = q + 1 < kLookbackWindow ? q + 1 : kLookbackWindow;
+      uint64_t w[kLookbackWindow];
+#pragma unroll
+      for (int i = 0; i < kLookbackWindow; ++i)
+        if (i < n) w[i] = lb_poll(status + (size_t)(q - i) * bins + bin);
+#pragma unroll
+      for (int i = 0; i < kLookbackWindow; ++i) {
+        if (i >= n || done) continue;
+        uint64_t v = w[i];
+        if ((uint32_t)(v >> 32) == kFlagNone) {
+          const uint64_t* src = status + (size_t)(q - i) * bins + bin;
+          const uint64_t ts = globaltimer_ns();
+          do {
+            __nanosleep(32);
+            v = lb_poll(src);
+            if ((uint32_t)(v >> 32) != kFlagNone) break;
+          } while (globaltimer_ns() - ts <= (uint64_t)limit_ns);
+          if ((uint32_t)(v >> 32) == kFlagNone) {
+            if (publish_self) lb_publish(mine, kFlagErr, 0);
+            return false;
+          }
+        }
+        const uint32_t fl = (uint32_t)(v >> 32);
+        if (fl == kFlagErr) {
           if (publish_self) lb_publish(mine, kFlagErr, 0);
           return false;
         }
+        excl += (uint32_t)v;
+        if (fl == kFlagIncl) done = true;
       }
-      const uint32_t fl = (uint32_t)(w >> 32);
-      if (fl == kFlagErr) {
-        if (publish_self) lb_publish(mine, kFlagErr, 0);
-        return false;
-      }
-      excl += (uint32_t)w;
-      if (fl == kFlagIncl) break;
-      --q;
+      q -= n;
     }
   }
   if (publish_self) lb_publish(mine, kFlagIncl, excl + agg);

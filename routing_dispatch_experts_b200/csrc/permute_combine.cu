@@ -51,6 +51,7 @@ __global__ void __launch_bounds__(32) permute_kernel(const uint8_t* __restrict__
     fence_barrier_init();
   }
   __syncwarp();
+  pdl_wait();
   const int64_t ngroups = (R + rps - 1) / rps;
   const int64_t nmine = ngroups > blockIdx.x ? (ngroups - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
   for (int64_t i = 0; i < nmine + kPermLookahead; ++i) {
@@ -101,6 +102,7 @@ __global__ void __launch_bounds__(256) permute_vec_kernel(const uint4* __restric
                                                           uint4* __restrict__ x_perm, int64_t R,
                                                           int64_t T, int V) {
   const int lane = threadIdx.x & 31;
+  pdl_wait();
   const int ipr = (V + 31) / 32;  // items per row
   const int64_t items = R * ipr;
   const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -173,6 +175,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ 
                                                       const float* __restrict__ gate,
                                                       uint4* __restrict__ y, int64_t Tn, int V,
                                                       int k) {
+  pdl_wait();
   const int64_t n = Tn * V;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
        i += (int64_t)gridDim.x * blockDim.x) {
@@ -228,16 +231,15 @@ cudaError_t launch_permute(const void* x, const int32_t* row_token, void* x_perm
     const int64_t items = R * ((V + 31) / 32);
     const int64_t warps = (items + U - 1) / U;
     const int grid = (int)std::min<int64_t>((warps + 7) / 8, (int64_t)sms * 8);
-    permute_vec_kernel<U><<<grid, 256, 0, s>>>(static_cast<const uint4*>(x), row_token,
-                                               static_cast<uint4*>(x_perm), R, T, V);
-    return cudaGetLastError();
+    return launch_pdl(permute_vec_kernel<U>, dim3(grid), dim3(256), 0, s,
+                      static_cast<const uint4*>(x), row_token, static_cast<uint4*>(x_perm), R, T, V);
   }
   const int rps = (int)std::min<uint32_t>(32u, kPermStageBytes / row_bytes);
   const int64_t ngroups = (R + rps - 1) / rps;
   const int grid = (int)std::min<int64_t>(ngroups, (int64_t)sms * kPermCtasPerSm);
-  permute_kernel<<<grid, 32, smem, s>>>(static_cast<const uint8_t*>(x), row_token,
-                                        static_cast<uint8_t*>(x_perm), R, T, row_bytes, rps);
-  return cudaGetLastError();
+  return launch_pdl(permute_kernel, dim3(grid), dim3(32), (size_t)smem, s,
+                    static_cast<const uint8_t*>(x), row_token, static_cast<uint8_t*>(x_perm), R, T,
+                    row_bytes, rps);
 }
 
 cudaError_t launch_combine(int dtype, const void* y_perm, const int32_t* slot_row,
@@ -251,12 +253,12 @@ cudaError_t launch_combine(int dtype, const void* y_perm, const int32_t* slot_ro
   const int64_t n = T * V;
   const int grid = (int)std::min<int64_t>((n + 255) / 256, (int64_t)sms * 8);
   if (dtype == MOE_BF16)
-    combine_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(static_cast<const uint4*>(y_perm), slot_row,
-                                                       gate, static_cast<uint4*>(y), T, V, k);
-  else
-    combine_kernel<float><<<grid, 256, 0, s>>>(static_cast<const uint4*>(y_perm), slot_row, gate,
-                                               static_cast<uint4*>(y), T, V, k);
-  return cudaGetLastError();
+    return launch_pdl(combine_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s,
+                      static_cast<const uint4*>(y_perm), slot_row, gate, static_cast<uint4*>(y), T,
+                      V, k);
+  return launch_pdl(combine_kernel<float>, dim3(grid), dim3(256), 0, s,
+                    static_cast<const uint4*>(y_perm), slot_row, gate, static_cast<uint4*>(y), T, V,
+                    k);
 }
 
 }  // namespace moe

@@ -22,6 +22,7 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
                                                    float* __restrict__ gate) {
   const int lane = threadIdx.x & 31;
   const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  pdl_wait();
   if (t >= T) return;  // uniform per warp
   const float* row = logits + t * E;
   float v[VPL];
@@ -81,8 +82,7 @@ cudaError_t launch_topk(const float* logits, int64_t T, int E, int k, int32_t* i
   switch (vpl) {
 #define MOE_TOPK_CASE(N) \
   case N:                \
-    topk_kernel<N><<<grid, warps * 32, 0, s>>>(logits, T, E, k, idx, gate); \
-    break;
+    return launch_pdl(topk_kernel<N>, dim3(grid), dim3(warps * 32), 0, s, logits, T, E, k, idx, gate);
     MOE_TOPK_CASE(1)
     MOE_TOPK_CASE(2)
     MOE_TOPK_CASE(3)
@@ -106,6 +106,7 @@ __global__ void __launch_bounds__(256) router_f32_kernel(const float* __restrict
                                                          const float* __restrict__ bias,
                                                          int64_t T, int d, int E,
                                                          float* __restrict__ logits) {
+  pdl_wait();
   const int64_t o = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (o >= T * E) return;
   const int64_t t = o / E;
@@ -129,8 +130,8 @@ cudaError_t launch_router_f32(const float* x, const float* wrT, const float* bia
                               int d, int E, float* logits, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
   const int64_t n = T * E;
-  router_f32_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(x, wrT, bias, T, d, E, logits);
-  return cudaGetLastError();
+  return launch_pdl(router_f32_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, x, wrT,
+                    bias, T, d, E, logits);
 }
 
 }  // namespace moe

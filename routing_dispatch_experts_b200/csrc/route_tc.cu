@@ -1,34 +1,38 @@
 // route_tc.cu - the router in one tcgen05 kernel: logits GEMM, bias, top-k
-// selection, softmax gates, and (for the forward) the dispatch histogram with
-// its decoupled-lookback scan.
+// selection, softmax gates, and (for the forward) the per-tile dispatch
+// histogram that the layout scatter turns into offsets.
 //
 // Top-k routing with softmax gates over the k ("MoE Pretraining: Parallelism
 // Layout Changes the Model, Not Quality", Methodology: top-4 routing;
 // "Revisiting MoE and Dense Speed-Accuracy Comparisons", 2.1: Top-K routing;
 // router weights "ME", Table 1).
 //
-// One CTA per 128-token tile (ids from a ticket counter, in start order):
+// One CTA per 128-token tile:
 //   warp 0      TMA producer: x tile [128 x 64] and W_r^T tile [E16 x 64] per
 //               k-block, 128-byte swizzle, 3-stage ring
 //   warp 1      TMEM allocation; one lane issues tcgen05.mma 128 x E16 x 16
-//   warps 2-5   epilogue, one token row per thread: tcgen05.ld of the row's
-//               E16 fp32 logits, + bias, logits stored, and a running top-k
-//               kept sorted in registers (key: logit desc, index asc; equal
-//               logits keep the lower index because only a strictly larger
-//               logit moves an entry); gates exp(l_j - l_0) / sum_i.
-// With the histogram on, each thread adds its token's experts, distinct
-// ranks and two statistics to a shared histogram, and the CTA runs the
-// lookback scan (lookback.cuh) for its tile: the layout's scatter kernel
-// then needs no separate histogram pass.
+//   warps 2-9   epilogue, two threads per token row (each reads half of the
+//               row's E16 fp32 logits with tcgen05.ld): + bias, logits
+//               stored, and a running top-k kept sorted in registers (key:
+//               logit desc, index asc; equal logits keep the lower index
+//               because only a strictly larger logit moves an entry); the
+//               second half's list is merged into the first through shared
+//               memory; gates exp(l_j - l_0) / sum_i.
+// With the histogram on, each token adds its experts, distinct ranks and two
+// statistics to a shared histogram that the CTA stores as its column of
+// block_hist [bins][nb]; the scatter kernel (after the kernel boundary, so every row is
+// complete) sums the rows into offsets and per-block prefixes.
 #include <algorithm>
 
-#include "lookback.cuh"
+#include "lookback.cuh"  // count_token
 
 namespace moe {
 
 namespace {
 
-constexpr int BM = 128, BK = 64, kThreads = 192, kStages = 3;
+constexpr int BM = 128, BK = 64, kStages = 3;
+constexpr int kEpiWarps = 8;                     // two per TMEM lane quadrant
+constexpr int kThreads = 64 + 32 * kEpiWarps;    // producer + MMA + epilogue
 
 struct Params {
   int64_t T;
@@ -39,11 +43,8 @@ struct Params {
   float* gate;
   Control* ctl;
   int hist, ep, nb, bins;
-  int64_t limit_ns;
   RankMap map;
-  uint64_t* status;
-  int32_t* prefix;
-  int32_t* totals;
+  int32_t* block_hist;
 };
 
 // insert (v, e) into the descending list (tv, ti); e arrives in increasing
@@ -64,7 +65,7 @@ __device__ __forceinline__ void topk_insert(float (&tv)[KMAX], int (&ti)[KMAX], 
 }
 
 template <int KMAX>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 2)
     route_fused_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                        const __grid_constant__ Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -76,9 +77,11 @@ __global__ void __launch_bounds__(kThreads)
 
   __shared__ __align__(8) uint64_t full[kStages], empty[kStages], tfull;
   __shared__ uint32_t tmem_base_s;
-  __shared__ int s_tile;
   __shared__ int hist[kMaxBins];
   __shared__ volatile int abort_flag;
+  // the second column half's partial top-k lists, merged by the first half
+  __shared__ float m_v[BM][KMAX];
+  __shared__ int m_i[BM][KMAX];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t tmem_cols = p.BN <= 32 ? 32 : (p.BN <= 64 ? 64 : (p.BN <= 128 ? 128 : 256));
@@ -102,13 +105,10 @@ __global__ void __launch_bounds__(kThreads)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  // the tile id is taken only once this CTA holds its tensor memory, so a
-  // CTA waiting in the lookback never waits on one still waiting to allocate
-  if (threadIdx.x == 0) s_tile = p.hist ? (int)atomicAdd(&p.ctl->ticket, 1u) : (int)blockIdx.x;
-  __syncthreads();
+  pdl_wait();
   const uint32_t tmem_base = tmem_base_s;
-  const int b = s_tile;
-  const bool tile_ok = b < p.nb;  // false only if two calls share a workspace at once
+  const int b = blockIdx.x;
+  const bool tile_ok = b < p.nb;
   const int64_t row0 = (int64_t)b * BM;
   const int kblocks = p.K / BK;
 
@@ -156,10 +156,16 @@ __global__ void __launch_bounds__(kThreads)
       tc_commit(&tfull);
     }
   } else if (tile_ok) {
+    // warps 2..9: quadrant q = warp % 4 (the TMEM lanes this warp may read),
+    // half h = which half of the 16-column chunks it scans
     const int q = warp & 3;
+    const int h = (warp - 2) >> 2;
     const int rr = q * 32 + lane;
     const int64_t t = row0 + rr;
     const bool valid = t < p.T;
+    const int nchunks = p.BN / 16;
+    const int c_lo = h == 0 ? 0 : (nchunks + 1) / 2;
+    const int c_hi = h == 0 ? (nchunks + 1) / 2 : nchunks;
     float tv[KMAX];
     int ti[KMAX];
 #pragma unroll
@@ -167,12 +173,14 @@ __global__ void __launch_bounds__(kThreads)
       tv[s] = -INFINITY;
       ti[s] = 0x7FFFFFFF;
     }
-    if (mbar_wait_bounded(&tfull, 0, &abort_flag) && !abort_flag) {
+    const bool have = mbar_wait_bounded(&tfull, 0, &abort_flag) && !abort_flag;
+    if (have) {
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16);
       float* lrow = p.logits + t * p.E;
       const bool vec = (p.E & 3) == 0 && (reinterpret_cast<uintptr_t>(p.logits) & 15) == 0;
-      for (int c = 0; c < p.BN; c += 16) {
+      for (int ch = c_lo; ch < c_hi; ++ch) {
+        const int c = ch * 16;
         uint32_t r[16];
         tmem_ld16(taddr + c, r);
         tmem_ld_wait();
@@ -195,7 +203,21 @@ __global__ void __launch_bounds__(kThreads)
         for (int i = 0; i < 16; ++i)
           if (c + i < p.E) topk_insert<KMAX>(tv, ti, v[i], c + i);
       }
-      if (valid) {
+    }
+    if (h == 1) {
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j) {
+        m_v[rr][j] = tv[j];
+        m_i[rr][j] = ti[j];
+      }
+    }
+    asm volatile("bar.sync 1, %0;" ::"r"(32 * kEpiWarps) : "memory");  // epilogue warps only
+    if (h == 0) {
+      // the second half's columns are all higher, so inserting its entries
+      // in order keeps lower indices first among equal logits
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j) topk_insert<KMAX>(tv, ti, m_v[rr][j], m_i[rr][j]);
+      if (have && valid) {
         float ex[KMAX];
         float z = 0.f;
 #pragma unroll
@@ -210,24 +232,24 @@ __global__ void __launch_bounds__(kThreads)
             p.gate[t * p.k + j] = ex[j] / z;
           }
       }
-    }
-    if (p.hist) {
-      int single = 0, home = 0;
-      if (valid && !abort_flag) {
-        int e[KMAX];  // a copy, so the running list above stays in registers
+      if (p.hist) {
+        int single = 0, home = 0;
+        if (have && valid) {
+          int e[KMAX];  // a copy, so the list above stays in registers
 #pragma unroll
-        for (int j = 0; j < KMAX; ++j) e[j] = ti[j];
-        count_token(e, p.k, t, p.T, p.E, p.ep, p.map, hist, &single, &home);
-      }
+          for (int j = 0; j < KMAX; ++j) e[j] = ti[j];
+          count_token(e, p.k, t, p.T, p.E, p.ep, p.map, hist, &single, &home);
+        }
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        single += __shfl_xor_sync(0xffffffffu, single, off);
-        home += __shfl_xor_sync(0xffffffffu, home, off);
-      }
-      const int sbin = p.E + (p.ep > 1 ? p.ep : 0);
-      if (lane == 0) {
-        atomicAdd(&hist[sbin], single);
-        atomicAdd(&hist[sbin + 1], home);
+        for (int off = 16; off > 0; off >>= 1) {
+          single += __shfl_xor_sync(0xffffffffu, single, off);
+          home += __shfl_xor_sync(0xffffffffu, home, off);
+        }
+        const int sbin = p.E + (p.ep > 1 ? p.ep : 0);
+        if (lane == 0) {
+          atomicAdd(&hist[sbin], single);
+          atomicAdd(&hist[sbin + 1], home);
+        }
       }
     }
   }
@@ -237,19 +259,9 @@ __global__ void __launch_bounds__(kThreads)
     tc_fence_after();
     tmem_dealloc(tmem_base, tmem_cols);
   }
-  if (p.hist && tile_ok) {
-    for (int bin = threadIdx.x; bin < p.bins; bin += kThreads) {
-      uint32_t excl = 0;
-      if (abort_flag ||
-          !lookback_bin(p.status, p.bins, b, bin, (uint32_t)hist[bin], true, p.limit_ns, &excl)) {
-        record_error(p.ctl, MOE_ERR_DEVICE_TIMEOUT, (uint32_t)b);
-        if (abort_flag) lb_publish(p.status + (size_t)b * p.bins + bin, kFlagErr, 0);
-        continue;
-      }
-      p.prefix[(size_t)b * p.bins + bin] = (int32_t)excl;
-      if (b == p.nb - 1) p.totals[bin] = (int32_t)(excl + (uint32_t)hist[bin]);
-    }
-  }
+  if (p.hist && tile_ok)  // bin-major [bins][nb], so the scatter reads rows of blocks
+    for (int bin = threadIdx.x; bin < p.bins; bin += kThreads)
+      p.block_hist[(size_t)bin * p.nb + b] = hist[bin];
 }
 
 template <int KMAX>
@@ -264,8 +276,7 @@ cudaError_t run(const RouteArgs& a, const CUtensorMap& mA, const CUtensorMap& mB
     if (e != cudaSuccess) return e;
     attr_bytes = smem;
   }
-  route_fused_kernel<KMAX><<<p.nb, kThreads, smem, s>>>(mA, mB, p);
-  return cudaGetLastError();
+  return launch_pdl(route_fused_kernel<KMAX>, dim3(p.nb), dim3(kThreads), smem, s, mA, mB, p);
 }
 
 }  // namespace
@@ -287,18 +298,11 @@ cudaError_t launch_route_tc(const RouteArgs& a, cudaStream_t s) {
   p.ep = a.ep;
   p.nb = layout_blocks(a.T);
   p.bins = layout_bins(a.E, a.ep);
-  p.limit_ns = kWaitLimitNs;
   p.map = a.map;
-  p.status = a.status_words;
-  p.prefix = a.prefix;
-  p.totals = a.totals;
+  p.block_hist = a.block_hist;
   CUtensorMap mA, mB;
   if (!make_kmajor_map(&mA, a.x, a.T, a.d, BM)) return cudaErrorInvalidValue;
   if (!make_kmajor_map(&mB, a.wrT, p.BN, a.d, p.BN)) return cudaErrorInvalidValue;
-  if (a.hist) {
-    cudaError_t e = clear_lookback(a.ctl, a.status_words, a.T, a.E, a.ep, s);
-    if (e != cudaSuccess) return e;
-  }
   if (a.k <= 2) return run<2>(a, mA, mB, p, s);
   if (a.k <= 4) return run<4>(a, mA, mB, p, s);
   if (a.k <= 8) return run<8>(a, mA, mB, p, s);

@@ -115,3 +115,23 @@ def test_lookback_wait_is_bounded():
     assert moe.get_device_status(ws) == moe.MOE_OK
     ref = oracle.dispatch_layout(idx.cpu().numpy(), E, 8)
     np.testing.assert_array_equal(out["slot_send_row"].cpu().numpy(), ref["slot_send_row"])
+
+
+def test_forward_and_standalone_layout_share_a_workspace():
+    """The forward's fused router writes per-tile histograms; a standalone
+    layout on the same workspace afterwards (and a forward after that) must
+    still find its lookback words zeroed."""
+    from util import Case
+    c = Case(2, T=3000)
+    shape = c.shape_ep(8)
+    ws = moe.workspace(shape, forward=True)
+    buf = moe.ForwardBuffers(shape)
+    y0 = moe.forward(shape, c.dx, c.packed, None, ws, buffers=buf)
+    idx = W.uniform_routing(3000, 64, 4, seed=21)
+    out = moe.dispatch_layout(shape, idx.cuda(), ws)
+    ref = oracle.dispatch_layout(idx.numpy(), 64, 8)
+    np.testing.assert_array_equal(out["slot_send_row"].cpu().numpy(), ref["slot_send_row"])
+    np.testing.assert_array_equal(out["row_token"].cpu().numpy(), ref["row_token"])
+    y1 = moe.forward(shape, c.dx, c.packed, None, ws)
+    assert torch.equal(y0, y1)
+    assert moe.get_device_status(ws) == moe.MOE_OK
