@@ -240,6 +240,17 @@ MOE_API moe_status moe_permute(const moe_shape* shape, const void* x,
                        moe_stream_t stream);
 
 /*
+ * The same permute done in token order: x row t is read once and written to
+ * its k rows x_perm[slot_row[t*k + j]] (slot_row [T*k] from
+ * moe_dispatch_layout).  Equal output to moe_permute; it moves |x| + |x_perm|
+ * bytes through DRAM even when x is much larger than L2, where the gather
+ * re-reads each row of x once per expert that picks it.
+ */
+MOE_API moe_status moe_permute_by_token(const moe_shape* shape, const void* x,
+                                        const int32_t* slot_row, void* x_perm,
+                                        moe_stream_t stream);
+
+/*
  * Grouped SwiGLU experts over the expert-grouped rows:
  *  h[r]      = silu(x_perm[r] W_g[e]) * (x_perm[r] W_u[e])   [T*k, f]
  *  y_perm[r] = h[r] W_d[e]                                   [T*k, d]
@@ -301,8 +312,8 @@ typedef struct {
  * gates + the dispatch histogram and its lookback scan, the layout scatter,
  * the gate/up GEMM with SwiGLU, the down GEMM and the combine; the permute
  * is fused into the gate/up GEMM (as moe_grouped_swiglu_gather, x_perm not
- * written) while x is at most 96 MB, and a separate moe_permute kernel
- * otherwise.  fp32: moe_route, moe_dispatch_layout, moe_permute,
+ * written) while x is at most 96 MB, and a separate token-order permute
+ * (moe_permute_by_token) otherwise.  fp32: moe_route, moe_dispatch_layout, moe_permute,
  * moe_grouped_swiglu and moe_combine in turn.
  *  x [T, d]; packed weights; bias [E] or NULL; expert_rank_host as in
  *  moe_dispatch_layout; y [T, d]; buffers may be NULL;

@@ -73,7 +73,7 @@ _lib = None
 # exported C symbols, in header order (checked against include/moe.h by the tests)
 SYMBOLS = ("moe_status_string", "moe_scratch_size", "moe_forward_workspace_size",
            "moe_workspace_init", "moe_packed_weights_size", "moe_pack_weights", "moe_route",
-           "moe_dispatch_layout", "moe_permute", "moe_grouped_swiglu",
+           "moe_dispatch_layout", "moe_permute", "moe_permute_by_token", "moe_grouped_swiglu",
            "moe_grouped_swiglu_gather", "moe_combine", "moe_forward", "moe_forward_timed",
            "moe_get_device_status", "moe_debug_dispatch_layout_stall",
            "moe_dispatch_layout_static")
@@ -101,6 +101,7 @@ def lib() -> ctypes.CDLL:
             "moe_dispatch_layout": ([S, P, P, ctypes.POINTER(moe_layout), P, ctypes.c_size_t, P],
                                     ctypes.c_int),
             "moe_permute": ([S, P, P, P, P], ctypes.c_int),
+            "moe_permute_by_token": ([S, P, P, P, P], ctypes.c_int),
             "moe_grouped_swiglu": ([S, P, P, P, P, P, P, ctypes.c_size_t, P], ctypes.c_int),
             "moe_combine": ([S, P, P, P, P, P], ctypes.c_int),
             "moe_grouped_swiglu_gather": ([S, P, P, P, P, P, P, P, ctypes.c_size_t, P], ctypes.c_int),
@@ -318,6 +319,16 @@ def permute(shape: Shape, x, row_token, stream=None):
     s = shape.c
     _check(lib().moe_permute(ctypes.byref(s), _p(x), _p(row_token), _p(x_perm), _stream(stream)),
            "moe_permute")
+    return x_perm
+
+
+def permute_by_token(shape: Shape, x, slot_row, stream=None):
+    """moe_permute_by_token: x_perm via a token-order copy (x read once)."""
+    _need(x, shape.dtype, (shape.T, shape.d), "x")
+    x_perm = torch.empty((shape.R, shape.d), dtype=shape.dtype, device=x.device)
+    s = shape.c
+    _check(lib().moe_permute_by_token(ctypes.byref(s), _p(x), _p(slot_row), _p(x_perm),
+                                      _stream(stream)), "moe_permute_by_token")
     return x_perm
 
 

@@ -266,7 +266,8 @@ moe_status do_grouped_part(int part, const moe_shape* s, const void* a_rows,
   a.n_out = s->d;
   a.out = y_perm;
   a.ld_out = s->d;
-  const int bn = s->d % 256 == 0 ? 256 : (s->d % 128 == 0 ? 128 : 64);
+  // short K (f <= 512): 128-column tiles, so two CTAs fit per SM
+  const int bn = (s->d % 256 == 0 && s->f > 512) ? 256 : (s->d % 128 == 0 ? 128 : 64);
   return cuda_status(launch_gemm_tc(kEpiBF16, bn, a, st));
 }
 
@@ -384,9 +385,9 @@ moe_status forward_impl(const moe_shape* s, const void* x, const void* packed, c
                                sc.ctl, st)) != MOE_OK)
         return r;
     } else {
-      if ((r = cuda_status(launch_permute(x, f.lay.row_token, f.x_perm, s->T,
-                                          s->T * (int64_t)s->k,
-                                          (uint32_t)(s->d * esize(s->dtype)), st))) != MOE_OK)
+      // x larger than L2: copy in token order, reading each row of x once
+      if ((r = cuda_status(launch_permute(x, f.lay.row_token, f.lay.slot_row, f.x_perm, s->T,
+                                          s->k, (uint32_t)(s->d * esize(s->dtype)), st))) != MOE_OK)
         return r;
       if ((r = mark(3)) != MOE_OK) return r;
       if ((r = do_grouped_part(0, s, f.x_perm, nullptr, f.lay.expert_offsets, &pk, f.h, f.y_perm,
@@ -398,7 +399,7 @@ moe_status forward_impl(const moe_shape* s, const void* x, const void* packed, c
     if ((r = mark(1)) != MOE_OK) return r;
     if ((r = do_layout(s, f.idx, map, &f.lay, sc, -1, kWaitLimitNs, st)) != MOE_OK) return r;
     if ((r = mark(2)) != MOE_OK) return r;
-    if ((r = cuda_status(launch_permute(x, f.lay.row_token, f.x_perm, s->T, s->T * (int64_t)s->k,
+    if ((r = cuda_status(launch_permute(x, f.lay.row_token, nullptr, f.x_perm, s->T, s->k,
                                         (uint32_t)(s->d * esize(s->dtype)), st))) != MOE_OK)
       return r;
     if ((r = mark(3)) != MOE_OK) return r;
@@ -524,7 +525,18 @@ moe_status moe_permute(const moe_shape* s, const void* x, const int32_t* row_tok
   if (s->T == 0) return MOE_OK;
   if (!x || !row_token || !x_perm) return MOE_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(x_perm, 16) || !aligned(row_token, 4)) return MOE_ERR_ALIGNMENT;
-  return cuda_status(launch_permute(x, row_token, x_perm, s->T, s->T * (int64_t)s->k,
+  return cuda_status(launch_permute(x, row_token, nullptr, x_perm, s->T, s->k,
+                                    (uint32_t)(s->d * esize(s->dtype)), (cudaStream_t)stream));
+}
+
+moe_status moe_permute_by_token(const moe_shape* s, const void* x, const int32_t* slot_row,
+                                void* x_perm, moe_stream_t stream) {
+  moe_status r = check_shape(s);
+  if (r != MOE_OK) return r;
+  if (s->T == 0) return MOE_OK;
+  if (!x || !slot_row || !x_perm) return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(x_perm, 16) || !aligned(slot_row, 4)) return MOE_ERR_ALIGNMENT;
+  return cuda_status(launch_permute(x, nullptr, slot_row, x_perm, s->T, s->k,
                                     (uint32_t)(s->d * esize(s->dtype)), (cudaStream_t)stream));
 }
 

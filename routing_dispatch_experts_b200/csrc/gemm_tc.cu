@@ -76,16 +76,23 @@ constexpr uint32_t staged_row_bytes() { return out_cols<BN, EPI>() * 2 + 16; }
 template <int BN, int EPI, bool STAGED>
 constexpr uint32_t staging_bytes() { return STAGED ? 128u * staged_row_bytes<BN, EPI>() : 0u; }
 
-template <int BN, int EPI, bool STAGED>
+// Short K loops also run two CTAs per SM (when both fit in tensor memory and
+// the producer needs no per-tile register state), so one CTA's load latency
+// overlaps the other's tiles.
+template <int BN, bool STAGED, bool GATHER>
+constexpr int ctas_per_sm() { return (STAGED && !GATHER && tmem_cols_for<BN>() <= 256) ? 2 : 1; }
+
+template <int BN, int EPI, bool STAGED, bool GATHER>
 constexpr int stages_for() {
   constexpr uint32_t stage = BM * BK * 2 + BN * BK * 2;
-  constexpr uint32_t n = (220u * 1024u - staging_bytes<BN, EPI, STAGED>()) / stage;
-  return n > 8 ? 8 : (int)n;
+  constexpr uint32_t budget = (ctas_per_sm<BN, STAGED, GATHER>() == 2 ? 104u : 220u) * 1024u;
+  constexpr uint32_t n = (budget - staging_bytes<BN, EPI, STAGED>()) / stage;
+  return n > 8 ? 8 : (n < 2 ? 2 : (int)n);
 }
 
-template <int BN, int EPI, bool STAGED>
+template <int BN, int EPI, bool STAGED, bool GATHER>
 constexpr size_t smem_bytes_for() {
-  return (size_t)stages_for<BN, EPI, STAGED>() * (BM * BK * 2 + BN * BK * 2) +
+  return (size_t)stages_for<BN, EPI, STAGED, GATHER>() * (BM * BK * 2 + BN * BK * 2) +
          staging_bytes<BN, EPI, STAGED>() + 1024;
 }
 
@@ -115,10 +122,10 @@ __device__ __forceinline__ float silu_mul(float g, float u) {
 }
 
 template <int BN, int EPI, bool GATHER, bool STAGED>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, (ctas_per_sm<BN, STAGED, GATHER>()))
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ Params p) {
-  constexpr int STAGES = stages_for<BN, EPI, STAGED>();
+  constexpr int STAGES = stages_for<BN, EPI, STAGED, GATHER>();
   constexpr uint32_t A_BYTES = BM * BK * 2;
   constexpr uint32_t B_BYTES = BN * BK * 2;
   constexpr uint32_t TMEM_COLS = tmem_cols_for<BN>();
@@ -338,6 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t grow = (int64_t)ti.row0 + rr;
       constexpr int OC = out_cols<BN, EPI>();
       constexpr int HC = OC / 2;
+      static_assert(HC % 32 == 0, "each epilogue half covers whole 32-column groups");
       __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + grow * p.ld_out + ti.nt * OC;
       uint8_t* stg = sOut + (size_t)rr * staged_row_bytes<BN, EPI>();
       if constexpr (STAGED) {
@@ -346,34 +354,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (h == 0) bulk_wait_read<0>();
         named_bar_sync(qbar, 64);
       }
+      // 32 output columns per TMEM round trip: issue all loads, then wait once
 #pragma unroll 1
-      for (int c = h * HC; c < (h + 1) * HC; c += 16) {
-        uint32_t pk[8];
+      for (int c = h * HC; c < (h + 1) * HC; c += 32) {
+        uint32_t pk[16];
         if constexpr (EPI == kEpiSwiGLU) {
-          uint32_t gr[16], ur[16];
-          tmem_ld16(taddr + c, gr);
-          tmem_ld16(taddr + OC + c, ur);
+          uint32_t g0[16], g1[16], u0[16], u1[16];
+          tmem_ld16(taddr + c, g0);
+          tmem_ld16(taddr + c + 16, g1);
+          tmem_ld16(taddr + OC + c, u0);
+          tmem_ld16(taddr + OC + c + 16, u1);
           tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            pk[i] = pack_bf16x2(silu_mul(__uint_as_float(gr[2 * i]), __uint_as_float(ur[2 * i])),
-                                silu_mul(__uint_as_float(gr[2 * i + 1]), __uint_as_float(ur[2 * i + 1])));
+          for (int i = 0; i < 8; ++i) {
+            pk[i] = pack_bf16x2(silu_mul(__uint_as_float(g0[2 * i]), __uint_as_float(u0[2 * i])),
+                                silu_mul(__uint_as_float(g0[2 * i + 1]), __uint_as_float(u0[2 * i + 1])));
+            pk[8 + i] = pack_bf16x2(silu_mul(__uint_as_float(g1[2 * i]), __uint_as_float(u1[2 * i])),
+                                    silu_mul(__uint_as_float(g1[2 * i + 1]), __uint_as_float(u1[2 * i + 1])));
+          }
         } else {
-          uint32_t r[16];
-          tmem_ld16(taddr + c, r);
+          uint32_t r0[16], r1[16];
+          tmem_ld16(taddr + c, r0);
+          tmem_ld16(taddr + c + 16, r1);
           tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+          for (int i = 0; i < 8; ++i) {
+            pk[i] = pack_bf16x2(__uint_as_float(r0[2 * i]), __uint_as_float(r0[2 * i + 1]));
+            pk[8 + i] = pack_bf16x2(__uint_as_float(r1[2 * i]), __uint_as_float(r1[2 * i + 1]));
+          }
         }
-        if constexpr (STAGED) {
-          uint4* o = reinterpret_cast<uint4*>(stg + c * 2);
-          o[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          o[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-        } else if (valid) {
-          uint4* o = reinterpret_cast<uint4*>(out + c);
-          o[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          o[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        uint4* o = reinterpret_cast<uint4*>(STAGED ? static_cast<void*>(stg + c * 2)
+                                                   : static_cast<void*>(out + c));
+        if (STAGED || valid) {
+#pragma unroll
+          for (int v = 0; v < 4; ++v) o[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
         }
       }
       if constexpr (STAGED) {
@@ -444,7 +458,7 @@ namespace {
 template <int BN, int EPI, bool GATHER, bool STAGED>
 cudaError_t run(const GemmArgs& a, cudaStream_t s) {
   static bool attr_set = false;
-  constexpr size_t smem = smem_bytes_for<BN, EPI, STAGED>();
+  constexpr size_t smem = smem_bytes_for<BN, EPI, STAGED, GATHER>();
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI, GATHER, STAGED>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -475,7 +489,7 @@ cudaError_t run(const GemmArgs& a, cudaStream_t s) {
   // upper bound of the tile count: every group adds at most one partial tile
   const int64_t mt_max = (a.rows + BM - 1) / BM + a.G;
   const int64_t tiles_max = mt_max * (a.n_per_group / BN);
-  const int grid = (int)std::min<int64_t>(tiles_max, sms);
+  const int grid = (int)std::min<int64_t>(tiles_max, (int64_t)sms * ctas_per_sm<BN, STAGED, GATHER>());
   if (grid <= 0) return cudaSuccess;
   return launch_pdl(gemm_tc_kernel<BN, EPI, GATHER, STAGED>, dim3(grid), dim3(kThreads), smem, s,
                     mA, mB, p);

@@ -64,8 +64,10 @@ cudaError_t launch_layout_scatter(const int32_t* idx, int64_t T, int k, int E, i
                                   const int32_t* block_hist, cudaStream_t s);
 
 // ---- permute_combine.cu
-cudaError_t launch_permute(const void* x, const int32_t* row_token, void* x_perm, int64_t T,
-                           int64_t R, uint32_t row_bytes, cudaStream_t s);
+// x_perm[r] = x[row_token[r]].  With slot_row non-NULL the copy runs in
+// token order instead (x row t to rows slot_row[t*k + j]), same result.
+cudaError_t launch_permute(const void* x, const int32_t* row_token, const int32_t* slot_row,
+                           void* x_perm, int64_t T, int k, uint32_t row_bytes, cudaStream_t s);
 cudaError_t launch_combine(int dtype, const void* y_perm, const int32_t* slot_row,
                            const float* gate, void* y, int64_t T, int d, int k, cudaStream_t s);
 

@@ -14,7 +14,8 @@ namespace moe {
 namespace {
 
 // ---------------------------------------------------------------- permute
-// TMA-staged ring for rows longer than 1 KB.  One warp per CTA.  Rows move in groups of `rps` rows (one group fills a
+// TMA-staged ring for rows longer than 1 KB (and for the token-order
+// variant).  One warp per CTA.  Rows move in groups of `rps` rows (one group fills a
 // 16 KB shared-memory stage); lane i of the warp owns row i of every group.
 // Lane i issues a TMA bulk load of its source row into the stage (completing
 // on the stage's mbarrier), then, LOOKAHEAD groups later, a TMA bulk store of
@@ -39,12 +40,18 @@ constexpr uint32_t kPermStageBytes = MOE_PERM_STAGE_BYTES;
 constexpr int kPermCtasPerSm = MOE_PERM_CTAS;
 static_assert(kPermLookahead < kPermStages, "lookahead must leave a stage to store from");
 
+// BY_TOKEN = false: item r is x_perm row r, read from x[row_token[r]].
+// BY_TOKEN = true:  item t is x row t, read once and written to its k rows
+// x_perm[slot_row[t*k + j]] -- x streams through once, which keeps DRAM
+// traffic at |x| + |x_perm| when x does not fit in L2.
+template <bool BY_TOKEN>
 __global__ void __launch_bounds__(32) permute_kernel(const uint8_t* __restrict__ x,
-                                                     const int32_t* __restrict__ row_token,
+                                                     const int32_t* __restrict__ index,
                                                      uint8_t* __restrict__ x_perm, int64_t R,
-                                                     int64_t T, uint32_t row_bytes, int rps) {
+                                                     int64_t T, int k, uint32_t row_bytes, int rps) {
   extern __shared__ __align__(128) uint8_t stage[];
   __shared__ __align__(8) uint64_t full[kPermStages];
+  __shared__ int dst_rows[BY_TOKEN ? kPermStages : 1][BY_TOKEN ? 32 * 16 : 1];
   const int lane = threadIdx.x;
   if (lane == 0) {
     for (int s = 0; s < kPermStages; ++s) mbar_init(&full[s], 1);
@@ -52,23 +59,34 @@ __global__ void __launch_bounds__(32) permute_kernel(const uint8_t* __restrict__
   }
   __syncwarp();
   pdl_wait();
-  const int64_t ngroups = (R + rps - 1) / rps;
+  const int64_t items = BY_TOKEN ? T : R;
+  const int64_t ngroups = (items + rps - 1) / rps;
   const int64_t nmine = ngroups > blockIdx.x ? (ngroups - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
   for (int64_t i = 0; i < nmine + kPermLookahead; ++i) {
     if (i < nmine) {
       const int s = (int)(i % kPermStages);
       const int64_t g = blockIdx.x + i * gridDim.x;
       const int64_t r0 = g * rps;
-      const int n = (int)(R - r0 < rps ? R - r0 : rps);
-      // this lane's store of group i - kPermStages read the same region
+      const int n = (int)(items - r0 < rps ? items - r0 : rps);
+      // this lane's stores of group i - kPermStages read the same region
       bulk_wait_read<kPermStages - kPermLookahead - 1>();
       if (lane == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)n * row_bytes);
       __syncwarp();
       if (lane < n) {
-        // an out-of-range token (malformed input) reads row 0 instead of
-        // faulting; the result is then unspecified, as documented
-        int64_t src = __ldg(row_token + r0 + lane);
-        if (src < 0 || src >= T) src = 0;
+        int64_t src;
+        if constexpr (BY_TOKEN) {
+          src = r0 + lane;
+          for (int j = 0; j < k; ++j) {
+            // an out-of-range row (malformed input) is skipped
+            const int32_t d = __ldg(index + src * k + j);
+            dst_rows[s][lane * 16 + j] = (d >= 0 && d < R) ? d : -1;
+          }
+        } else {
+          // an out-of-range token (malformed input) reads row 0 instead of
+          // faulting; the result is then unspecified, as documented
+          src = __ldg(index + r0 + lane);
+          if (src < 0 || src >= T) src = 0;
+        }
         bulk_load(stage + (size_t)s * kPermStageBytes + (size_t)lane * row_bytes,
                   x + src * row_bytes, row_bytes, &full[s]);
       }
@@ -78,15 +96,23 @@ __global__ void __launch_bounds__(32) permute_kernel(const uint8_t* __restrict__
       const int s = (int)(j % kPermStages);
       const int64_t g = blockIdx.x + j * gridDim.x;
       const int64_t r0 = g * rps;
-      const int n = (int)(R - r0 < rps ? R - r0 : rps);
+      const int n = (int)(items - r0 < rps ? items - r0 : rps);
       // the loads of a group complete on the stage barrier; bounded wait
       if (!mbar_wait_bounded(&full[s], (uint32_t)((j / kPermStages) & 1), nullptr)) {
         // never expected: a bulk load did not land within the limit
         break;
       }
-      if (lane < n)
-        bulk_store(x_perm + (r0 + lane) * row_bytes,
-                   stage + (size_t)s * kPermStageBytes + (size_t)lane * row_bytes, row_bytes);
+      if (lane < n) {
+        const uint8_t* src = stage + (size_t)s * kPermStageBytes + (size_t)lane * row_bytes;
+        if constexpr (BY_TOKEN) {
+          for (int q = 0; q < k; ++q) {
+            const int d = dst_rows[s][lane * 16 + q];
+            if (d >= 0) bulk_store(x_perm + (int64_t)d * row_bytes, src, row_bytes);
+          }
+        } else {
+          bulk_store(x_perm + (r0 + lane) * row_bytes, src, row_bytes);
+        }
+      }
       bulk_commit();
     }
   }
@@ -210,22 +236,16 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ 
 
 }  // namespace
 
-cudaError_t launch_permute(const void* x, const int32_t* row_token, void* x_perm, int64_t T,
-                           int64_t R, uint32_t row_bytes, cudaStream_t s) {
+cudaError_t launch_permute(const void* x, const int32_t* row_token, const int32_t* slot_row,
+                           void* x_perm, int64_t T, int k, uint32_t row_bytes, cudaStream_t s) {
+  const int64_t R = T * k;
   if (R == 0) return cudaSuccess;
-  static bool attr_set = false;
-  const int smem = kPermStages * (int)kPermStageBytes;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   // Short rows (<= 1 KB): the register copy keeps more rows in flight than
   // the staged ring; longer rows go through the TMA-staged ring.
-  if (row_bytes <= 1024) {
+  if (!slot_row && row_bytes <= 1024) {
     constexpr int U = 4;
     const int V = (int)(row_bytes / 16);
     const int64_t items = R * ((V + 31) / 32);
@@ -234,11 +254,26 @@ cudaError_t launch_permute(const void* x, const int32_t* row_token, void* x_perm
     return launch_pdl(permute_vec_kernel<U>, dim3(grid), dim3(256), 0, s,
                       static_cast<const uint4*>(x), row_token, static_cast<uint4*>(x_perm), R, T, V);
   }
+  const int smem = kPermStages * (int)kPermStageBytes;
+  static bool attr_set[2] = {false, false};
+  const bool by_token = slot_row != nullptr;
+  if (!attr_set[by_token]) {
+    cudaError_t e = by_token ? cudaFuncSetAttribute(permute_kernel<true>,
+                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, smem)
+                             : cudaFuncSetAttribute(permute_kernel<false>,
+                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    attr_set[by_token] = true;
+  }
   const int rps = (int)std::min<uint32_t>(32u, kPermStageBytes / row_bytes);
-  const int64_t ngroups = (R + rps - 1) / rps;
+  const int64_t ngroups = ((by_token ? T : R) + rps - 1) / rps;
   const int grid = (int)std::min<int64_t>(ngroups, (int64_t)sms * kPermCtasPerSm);
-  return launch_pdl(permute_kernel, dim3(grid), dim3(32), (size_t)smem, s,
-                    static_cast<const uint8_t*>(x), row_token, static_cast<uint8_t*>(x_perm), R, T,
+  if (by_token)
+    return launch_pdl(permute_kernel<true>, dim3(grid), dim3(32), (size_t)smem, s,
+                      static_cast<const uint8_t*>(x), slot_row, static_cast<uint8_t*>(x_perm), R,
+                      T, k, row_bytes, rps);
+  return launch_pdl(permute_kernel<false>, dim3(grid), dim3(32), (size_t)smem, s,
+                    static_cast<const uint8_t*>(x), row_token, static_cast<uint8_t*>(x_perm), R, T, k,
                     row_bytes, rps);
 }
 

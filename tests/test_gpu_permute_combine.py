@@ -23,6 +23,18 @@ def test_permute_bit_exact(cfg, T):
     assert torch.equal(x_perm.cpu(), x[rt.long()])
 
 
+@pytest.mark.parametrize("cfg,T", [(1, 2048), (2, 1000), (3, 1025), (4, 77), (5, 301), (5, 1)])
+def test_permute_by_token_bit_exact(cfg, T):
+    """The token-order copy writes the same x_perm as the gather."""
+    w = W.WORKLOADS[cfg]
+    x = W.make_x(w, T=T)
+    idx = W.uniform_routing(T, w.E, w.k, seed=T + 3)
+    lay = oracle.dispatch_layout(idx.numpy(), w.E, 1)
+    shape = moe.Shape(T=T, d=w.d, E=w.E, k=w.k, f=w.f, dtype=w.torch_dtype)
+    x_perm = moe.permute_by_token(shape, x.cuda(), torch.from_numpy(lay["slot_row"]).cuda())
+    assert torch.equal(x_perm.cpu(), x[torch.from_numpy(lay["row_token"]).long()])
+
+
 @pytest.mark.parametrize("cfg,T", [(1, 2048), (2, 4099), (3, 513), (4, 300), (5, 129)])
 def test_identity_experts_unit_gates_give_k_x(cfg, T):
     """Permute, then combine with the experts replaced by the identity and
