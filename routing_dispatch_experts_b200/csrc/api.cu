@@ -46,8 +46,9 @@ struct Scratch {
 
 size_t scratch_bytes(const moe_shape* s) {
   const size_t nb = (size_t)layout_blocks(s->T), bins = (size_t)layout_bins(s->E, s->ep);
+  const size_t hs = (size_t)layout_hist_stride((int)nb);
   return align_up(sizeof(Control)) + kTotalsBytes + align_up(nb * bins * 8) +
-         align_up(nb * bins * 4);
+         align_up(hs * bins * 4);
 }
 
 Scratch carve_scratch(const moe_shape* s, void* ws) {

@@ -56,9 +56,15 @@ __device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31; }
 // prefetch), then pdl_wait() -- which returns once the predecessor grid has
 // completed and its writes are visible -- before touching anything a
 // predecessor produced.  Without the launch attribute it is a no-op.
-// (Releasing successors earlier, at kernel start, measured slower on B200:
-// waiting successor CTAs then crowd the SMs the predecessor still uses.)
+// A kernel may also release its successor explicitly with pdl_trigger()
+// once a CTA's remaining work is short (the successor grid is scheduled when
+// every CTA has triggered or exited); the successor's pdl_wait() still waits
+// for this grid's completion.  Releasing at kernel start measured slower on
+// B200: waiting successor CTAs then crowd the SMs the predecessor still uses.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 
 // barrier among `count` threads (a multiple of 32) of the CTA, id 1..15
 __device__ __forceinline__ void named_bar_sync(int id, int count) {
@@ -151,6 +157,9 @@ __device__ __forceinline__ void cp_async_16(uint32_t smem_dst, const void* gsrc)
 __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
+
+// wait until every cp.async issued by this thread has landed
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 // Untiled bulk copy global -> shared, completing on `bar` (16-B aligned,
 // size a multiple of 16).

@@ -10,12 +10,13 @@
 //               Comparisons", 2.1 Architecture)
 //   kEpiBF16    out = acc in bf16 (the down projection)
 //
-// Design (one CTA per SM, persistent, 6 warps):
+// Design (persistent: one CTA per SM, two for short K loops; 10 warps, 13
+// in gather mode):
 //   warp 0      TMA producer: 128 x 64 A tiles and BN x 64 B tiles, 128-byte
 //               swizzle, into a STAGES-deep shared-memory ring (full/empty
 //               mbarriers).  Gather mode: the A rows are rows of x picked by
-//               the permutation, copied by the whole warp with cp.async into
-//               the same swizzled layout
+//               the permutation, copied with cp.async into the same swizzled
+//               layout by warp 0 and warps 10-12, 32 rows each
 //   warp 1      allocates tensor memory (two BN-column fp32 accumulators) and
 //               one lane issues tcgen05.mma (M=128, N=BN, K=16) from shared-
 //               memory descriptors; tcgen05.commit frees smem stages and
@@ -42,8 +43,13 @@ namespace moe {
 namespace {
 
 constexpr int BM = 128, BK = 64;
-constexpr int kEpiWarps = 8;                   // two per TMEM lane quadrant
-constexpr int kThreads = 64 + 32 * kEpiWarps;  // producer + MMA + epilogue
+constexpr int kEpiWarps = 8;  // two per TMEM lane quadrant
+// gather mode: the A rows of a stage are copied by this many warps (warp 0
+// and the warps after the epilogue), 32 rows each
+constexpr int kGatherWarps = 4;
+// producer + MMA + epilogue (+ the extra gather warps)
+template <bool GATHER>
+constexpr int threads_for() { return 64 + 32 * kEpiWarps + (GATHER ? 32 * (kGatherWarps - 1) : 0); }
 
 struct Params {
   const int32_t* offsets;  // NULL: a single group of `rows` rows
@@ -122,7 +128,7 @@ __device__ __forceinline__ float silu_mul(float g, float u) {
 }
 
 template <int BN, int EPI, bool GATHER, bool STAGED>
-__global__ void __launch_bounds__(kThreads, (ctas_per_sm<BN, STAGED, GATHER>()))
+__global__ void __launch_bounds__(threads_for<GATHER>(), (ctas_per_sm<BN, STAGED, GATHER>()))
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ Params p) {
   constexpr int STAGES = stages_for<BN, EPI, STAGED, GATHER>();
@@ -131,6 +137,7 @@ __global__ void __launch_bounds__(kThreads, (ctas_per_sm<BN, STAGED, GATHER>()))
   constexpr uint32_t TMEM_COLS = tmem_cols_for<BN>();
   constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
   constexpr uint32_t ACC_STRIDE = TMEM_COLS / 2;  // column distance of the two accumulators
+  constexpr int NT = threads_for<GATHER>();
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -152,7 +159,7 @@ __global__ void __launch_bounds__(kThreads, (ctas_per_sm<BN, STAGED, GATHER>()))
   // group offsets and the prefix of 128-row tiles per group
   // offsets clamped to [0, rows]: a malformed offset array can never make
   // the epilogue store outside the output
-  for (int g = threadIdx.x; g <= G; g += kThreads)
+  for (int g = threadIdx.x; g <= G; g += NT)
     s_off[g] = p.offsets ? min(max(__ldg(p.offsets + g), 0), (int)p.rows) : (g == 0 ? 0 : (int)p.rows);
   if (threadIdx.x == 0) abort_flag = 0;
   __syncthreads();
@@ -174,7 +181,8 @@ __global__ void __launch_bounds__(kThreads, (ctas_per_sm<BN, STAGED, GATHER>()))
       tile_off[G] = carry;
       for (int s = 0; s < STAGES; ++s) {
         // gather mode: the TMA arrival plus one cp.async arrival per lane
-        mbar_init(&full[s], GATHER ? 33 : 1);
+        // of every gather warp
+        mbar_init(&full[s], GATHER ? 32 * kGatherWarps + 1 : 1);
         mbar_init(&empty[s], 1);
       }
       for (int b = 0; b < 2; ++b) {
@@ -198,26 +206,29 @@ __global__ void __launch_bounds__(kThreads, (ctas_per_sm<BN, STAGED, GATHER>()))
   const int total = tile_off[G] * n_tiles;
   const int kblocks = p.K / BK;
 
-  if (warp == 0) {
+  const bool gather_warp = GATHER && (warp == 0 || warp >= 2 + kEpiWarps);
+  if (warp == 0 || gather_warp) {
     if constexpr (GATHER) {
       // Permute fused into the operand load: the tile's 128 A rows are rows
-      // gather[row0 .. row0+127] of the source (x).  The whole warp copies
-      // them with 16-byte cp.async (lane l: chunk l%8 of rows 4i + l/8),
-      // writing the 128-byte-swizzled layout a TMA tile load would produce
-      // (chunk c of row r at c ^ (r % 8)); each lane's copies arrive on the
-      // stage barrier when they land.  B still comes by TMA.  Rows past the
-      // end of the gather list read source row 0; their results are never
-      // stored.
+      // gather[row0 .. row0+127] of the source (x).  Gather warp gw copies
+      // rows 32*gw .. 32*gw+31 with 16-byte cp.async (lane l: chunk l%8 of
+      // rows 32*gw + 4i + l/8), writing the 128-byte-swizzled layout a TMA
+      // tile load would produce (chunk c of row r at c ^ (r % 8)); each
+      // lane's copies arrive on the stage barrier when they land.  Warp 0
+      // also loads B by TMA.  Rows past the end of the gather list read
+      // source row 0; their results are never stored.
+      constexpr int RPW = BM / kGatherWarps;  // rows per gather warp
+      const int gw = warp == 0 ? 0 : warp - (1 + kEpiWarps);
       const int ch = lane & 7, rsub = lane >> 3;
       uint32_t it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         const TileInfo ti = decode(tile, n_tiles, tile_off, s_off, G);
         const int brow = ti.g * p.n_per_group + ti.nt * BN;
-        int32_t src[BM / 4];
+        int32_t src[RPW / 4];
 #pragma unroll
-        for (int i = 0; i < BM / 4; ++i) {
-          const int64_t r = (int64_t)ti.row0 + 4 * i + rsub;
+        for (int i = 0; i < RPW / 4; ++i) {
+          const int64_t r = (int64_t)ti.row0 + gw * RPW + 4 * i + rsub;
           const int32_t v = r < p.rows ? __ldg(p.gather + r) : 0;
           src[i] = (v >= 0 && v < p.src_rows) ? v : 0;
         }
@@ -226,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, (ctas_per_sm<BN, STAGED, GATHER>()))
           int good = 1;
           if (lane == 0) {
             good = mbar_wait_bounded(&empty[s], ph ^ 1, &abort_flag);
-            if (good) {
+            if (good && gw == 0) {
               mbar_arrive_expect_tx(&full[s], B_BYTES);
               tma_load_2d(sB + s * B_BYTES, &tmB, &full[s], kb * BK, brow);
             }
@@ -239,8 +250,8 @@ __global__ void __launch_bounds__(kThreads, (ctas_per_sm<BN, STAGED, GATHER>()))
           const __nv_bfloat16* xa = static_cast<const __nv_bfloat16*>(p.A) + kb * BK + ch * 8;
           const uint32_t sa = smem_u32(sA + s * A_BYTES);
 #pragma unroll
-          for (int i = 0; i < BM / 4; ++i) {
-            const int r = 4 * i + rsub;
+          for (int i = 0; i < RPW / 4; ++i) {
+            const int r = gw * RPW + 4 * i + rsub;
             cp_async_16(sa + r * 128 + ((ch ^ (r & 7)) << 4), xa + (int64_t)src[i] * p.K);
           }
           cp_async_arrive_noinc(&full[s]);
@@ -252,10 +263,14 @@ __global__ void __launch_bounds__(kThreads, (ctas_per_sm<BN, STAGED, GATHER>()))
           record_error(p.ctl, MOE_ERR_DEVICE_TIMEOUT, 0x100u);
         }
       }
-      // drain: every issued stage completes before the CTA may exit
-      const uint32_t first = it > (uint32_t)STAGES ? it - STAGES : 0;
-      for (uint32_t q = first; q < it; ++q)
-        mbar_wait_bounded(&full[q % STAGES], (q / STAGES) & 1, nullptr);
+      cp_async_wait_all();
+      // drain: every issued stage (the B loads too) completes before the CTA
+      // may exit
+      if (gw == 0) {
+        const uint32_t first = it > (uint32_t)STAGES ? it - STAGES : 0;
+        for (uint32_t q = first; q < it; ++q)
+          mbar_wait_bounded(&full[q % STAGES], (q / STAGES) & 1, nullptr);
+      }
     } else if (lane == 0) {
       uint32_t it = 0;
       bool ok = true;
@@ -319,6 +334,9 @@ __global__ void __launch_bounds__(kThreads, (ctas_per_sm<BN, STAGED, GATHER>()))
         abort_flag = 1;
         record_error(p.ctl, MOE_ERR_DEVICE_TIMEOUT, 0x200u);
       }
+      // every MMA of this CTA is issued: let the next kernel's CTAs be
+      // scheduled (they still wait for this grid to complete)
+      pdl_trigger();
       // all MMAs issued by this thread complete before TMEM is released
       tc_commit(&done);
       mbar_wait_bounded(&done, 0, nullptr);
@@ -491,7 +509,7 @@ cudaError_t run(const GemmArgs& a, cudaStream_t s) {
   const int64_t tiles_max = mt_max * (a.n_per_group / BN);
   const int grid = (int)std::min<int64_t>(tiles_max, (int64_t)sms * ctas_per_sm<BN, STAGED, GATHER>());
   if (grid <= 0) return cudaSuccess;
-  return launch_pdl(gemm_tc_kernel<BN, EPI, GATHER, STAGED>, dim3(grid), dim3(kThreads), smem, s,
+  return launch_pdl(gemm_tc_kernel<BN, EPI, GATHER, STAGED>, dim3(grid), dim3(threads_for<GATHER>()), smem, s,
                     mA, mB, p);
 }
 

@@ -41,6 +41,9 @@ constexpr int kMaxBins = 256 + 256 + 2;  // experts + ranks + two stat counters
 
 inline int layout_blocks(int64_t T) { return (int)((T + kTokPerBlock - 1) / kTokPerBlock); }
 inline int layout_bins(int E, int ep) { return E + (ep > 1 ? ep : 0) + 2; }
+// row stride (ints) of block_hist [bins][stride]: nb rounded up to a multiple
+// of 4 so every row starts 16-byte aligned
+inline int layout_hist_stride(int nb) { return (nb + 3) & ~3; }
 
 struct LayoutOut {
   int32_t *counts, *offsets, *row_token, *slot_row;
@@ -58,7 +61,8 @@ cudaError_t launch_layout(const int32_t* idx, int64_t T, int k, int E, int ep, c
                           const LayoutOut& out, Control* ctl, uint64_t* status_words,
                           int32_t* totals, int stall_block, int64_t limit_ns, cudaStream_t s);
 // the scatter half of the layout after the fused router, which left one
-// histogram column per 128-token block in block_hist [bins][nb]
+// histogram column per 128-token block in block_hist [bins][stride]
+// (stride = layout_hist_stride(nb))
 cudaError_t launch_layout_scatter(const int32_t* idx, int64_t T, int k, int E, int ep,
                                   const RankMap& map, const LayoutOut& out, Control* ctl,
                                   const int32_t* block_hist, cudaStream_t s);

@@ -37,15 +37,20 @@ struct Params {
   Control* ctl;
   uint64_t* status;  // [nb][bins] lookback words (histogram-kernel mode)
   int32_t* totals;   // [bins]   (histogram-kernel mode)
-  const int32_t* block_hist;  // [bins][nb] per-block counts (fused-router mode)
+  const int32_t* block_hist;  // [bins][hist_stride] per-block counts (fused-router mode)
+  int hist_stride;
   LayoutOut out;
 };
+
+constexpr int kMaxK = 16;
 
 __global__ void __launch_bounds__(kLayoutThreads) layout_hist_kernel(const __grid_constant__ Params p) {
   __shared__ int hist[kMaxBins];
   __shared__ int s_ticket;
+  __shared__ uint8_t s_map[256];
   const int tid = threadIdx.x;
   for (int i = tid; i < p.bins; i += kLayoutThreads) hist[i] = 0;
+  for (int i = tid; i < p.E; i += kLayoutThreads) s_map[i] = p.map.r[i];
   pdl_wait();
   if (tid == 0) s_ticket = (int)atomicAdd(&p.ctl->ticket, 1u);
   __syncthreads();
@@ -59,16 +64,17 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_hist_kernel(const __gri
   const int sbin = p.E + (p.ep > 1 ? p.ep : 0);  // the two stat bins
   int single = 0, home = 0;
   for (int64_t t = t0 + tid; t < t1; t += kLayoutThreads) {
-    int e[16];
+    int e[kMaxK];
     bool ok = true;
-    for (int j = 0; j < p.k; ++j) {
-      e[j] = __ldg(p.idx + t * p.k + j);
-      if ((unsigned)e[j] >= (unsigned)p.E) {
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) {
+      e[j] = j < p.k ? __ldg(p.idx + t * p.k + j) : 0;
+      if (j < p.k && (unsigned)e[j] >= (unsigned)p.E) {
         record_error(p.ctl, MOE_ERR_DEVICE_INDEX, (uint32_t)(t * p.k + j));
         ok = false;
       }
     }
-    if (ok) count_token(e, p.k, t, p.T, p.E, p.ep, p.map, hist, &single, &home);
+    if (ok) count_token<kMaxK>(e, p.k, t, p.T, p.E, p.ep, s_map, hist, &single, &home);
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) {
@@ -104,6 +110,7 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(const __
   __shared__ int s_pre[kMaxBins];  // this block's exclusive prefix per bin
   __shared__ int s_tot[kMaxBins];  // totals per bin
   __shared__ int s_ok;
+  __shared__ uint8_t s_map[256];
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int b = blockIdx.x;
@@ -117,33 +124,33 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(const __
   if (tid == 0) s_ok = *reinterpret_cast<volatile uint32_t*>(&p.ctl->status) == MOE_OK;
   if (p.block_hist) {
     // fused-router mode: the kernel boundary already ordered every block's
-    // histogram, so sum them directly.  block_hist is [bins][nb]; warp w
-    // takes bins w, w+8, ..., its lanes read 32 consecutive blocks per load
-    // (independent loads, four bins at a time), and two warp reductions give
-    // the bin's total and this block's exclusive prefix (integer sums: exact)
-    for (int bin0 = warp * 4; bin0 < p.bins; bin0 += kWarps * 4) {
-      int pre[4] = {0, 0, 0, 0}, tot[4] = {0, 0, 0, 0};
-      for (int q0 = 0; q0 < p.nb; q0 += 32) {
-        const int q = q0 + lane;
-        int v[4];
+    // histogram, so sum them directly.  block_hist is [bins][stride]; one
+    // thread per bin reads its row with 16-byte loads, 16 in flight at a
+    // time, and keeps the total and this block's exclusive prefix (integer
+    // sums: exact)
+    const int hs = p.hist_stride;
+    for (int bin = tid; bin < p.bins; bin += kLayoutThreads) {
+      const int4* row = reinterpret_cast<const int4*>(p.block_hist + (size_t)bin * hs);
+      int tot = 0, pre = 0;
+      for (int q4 = 0; q4 * 4 < p.nb; q4 += 16) {
+        int4 v[16];
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-          v[u] = (q < p.nb && bin0 + u < p.bins) ? __ldg(p.block_hist + (size_t)(bin0 + u) * p.nb + q) : 0;
+        for (int u = 0; u < 16; ++u)
+          v[u] = (q4 + u) * 4 < p.nb ? __ldg(row + q4 + u) : make_int4(0, 0, 0, 0);
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          tot[u] += v[u];
-          pre[u] += q < b ? v[u] : 0;
+        for (int u = 0; u < 16; ++u) {
+          const int q = (q4 + u) * 4;
+          const int a[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const int x = q + c < p.nb ? a[c] : 0;  // entries past nb are padding
+            tot += x;
+            pre += q + c < b ? x : 0;
+          }
         }
       }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int t = __reduce_add_sync(0xffffffffu, tot[u]);
-        const int pr = __reduce_add_sync(0xffffffffu, pre[u]);
-        if (lane == 0 && bin0 + u < p.bins) {
-          s_tot[bin0 + u] = t;
-          s_pre[bin0 + u] = pr;
-        }
-      }
+      s_tot[bin] = tot;
+      s_pre[bin] = pre;
     }
   } else {
     // histogram-kernel mode: this block's inclusive prefixes from its
@@ -158,10 +165,15 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(const __
     }
     if (b == 0 && tid == 0) p.ctl->ticket = 0;
   }
-  // the block's routing, read once (coalesced) into shared memory
+  // the block's routing, read once (coalesced) into shared memory, and the
+  // expert -> rank map
   for (int i = tid; i < ntok * k; i += kLayoutThreads) s_idx[i] = __ldg(p.idx + tb0 * k + i);
+  if (dedup)
+    for (int i = tid; i < E; i += kLayoutThreads) s_map[i] = p.map.r[i];
   for (int i = tid; i < kWarps * kMaxBins; i += kLayoutThreads) (&wh[0][0])[i] = 0;
   __syncthreads();
+  // what is left is short: let the next kernel's CTAs be scheduled
+  pdl_trigger();
   if (!s_ok) return;
 
   // exclusive scans of the expert totals and the rank totals (one warp each)
@@ -191,14 +203,20 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(const __
   const int aw0 = tw0 * k, aw1 = tw1 * k;
   for (int a = aw0 + lane; a < aw1; a += 32) atomicAdd(&wh[warp][s_idx[a]], 1);
   if (dedup) {
+    // one count per distinct rank of the token (ranks compared against the
+    // token's earlier slots, in registers)
     for (int t = tw0 + lane; t < tw1; t += 32) {
-      uint32_t m[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-      for (int j = 0; j < k; ++j) {
-        const int r = p.map.r[s_idx[t * k + j]];
-        m[r >> 5] |= 1u << (r & 31);
+      int rr[kMaxK];
+#pragma unroll
+      for (int j = 0; j < kMaxK; ++j) {
+        if (j < k) {
+          rr[j] = s_map[s_idx[t * k + j]];
+          bool seen = false;
+#pragma unroll
+          for (int q = 0; q < j; ++q) seen |= rr[q] == rr[j];
+          if (!seen) atomicAdd(&wh[warp][E + rr[j]], 1);
+        }
       }
-      for (int i = 0; i < 8; ++i)
-        for (uint32_t u = m[i]; u; u &= u - 1) atomicAdd(&wh[warp][E + (i << 5) + __ffs(u) - 1], 1);
     }
   }
   __syncthreads();
@@ -280,25 +298,28 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(const __
     for (int tt = tw0; tt < tw1; tt += 32) {
       const int t = tt + lane;
       const bool valid = t < tw1;
-      uint32_t m[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-      int rr[16];
-      if (valid)
-        for (int j = 0; j < k; ++j) {
-          rr[j] = p.map.r[s_idx[t * k + j]];
-          m[rr[j] >> 5] |= 1u << (rr[j] & 31);
-        }
+      int rr[kMaxK];
+#pragma unroll
+      for (int j = 0; j < kMaxK; ++j) rr[j] = (valid && j < k) ? (int)s_map[s_idx[t * k + j]] : -1;
+      const int64_t gt = tb0 + t;
       for (int i = 0; i < nw; ++i) {
-        uint32_t u = __reduce_or_sync(0xffffffffu, m[i]);
+        // this lane's ranks in [32i, 32i + 32), then the warp's union
+        uint32_t mi = 0;
+#pragma unroll
+        for (int j = 0; j < kMaxK; ++j)
+          if (rr[j] >= 0 && (rr[j] >> 5) == i) mi |= 1u << (rr[j] & 31);
+        uint32_t u = __reduce_or_sync(0xffffffffu, mi);
         while (u) {
-          const int r = (i << 5) + __ffs(u) - 1;
+          const int rb = __ffs(u) - 1;
           u &= u - 1;
-          const bool has = (m[i] >> (r & 31)) & 1u;
+          const int r = (i << 5) + rb;
+          const bool has = (mi >> rb) & 1u;
           const uint32_t bal = __ballot_sync(0xffffffffu, has);
           if (has) {
             const int srow = wh[warp][E + r] + __popc(bal & lt);
-            const int64_t gt = tb0 + t;
             p.out.send_token[srow] = (int32_t)gt;
-            for (int j = 0; j < k; ++j)
+#pragma unroll
+            for (int j = 0; j < kMaxK; ++j)
               if (rr[j] == r) p.out.slot_send_row[gt * k + j] = srow;
           }
           __syncwarp();
@@ -328,6 +349,7 @@ Params make_params(const int32_t* idx, int64_t T, int k, int E, int ep, const Ra
   p.status = status_words;
   p.totals = totals;
   p.block_hist = nullptr;
+  p.hist_stride = 0;
   p.out = out;
   return p;
 }
@@ -363,6 +385,7 @@ cudaError_t launch_layout_scatter(const int32_t* idx, int64_t T, int k, int E, i
   if (T == 0) return empty_layout(E, ep, out, s);
   Params p = make_params(idx, T, k, E, ep, map, out, ctl, nullptr, nullptr, -1, 0);
   p.block_hist = block_hist;
+  p.hist_stride = layout_hist_stride(p.nb);
   return launch_pdl(layout_scatter_kernel, dim3(p.nb), dim3(kLayoutThreads), 0, s, p);
 }
 

@@ -83,23 +83,31 @@ __device__ __forceinline__ bool lookback_bin(uint64_t* status, int bins, int b, 
   return true;
 }
 
-// Statistic bins at the end of the histogram: tokens whose experts sit on one
-// rank, and assignments on the token's home rank floor(t * ep / T).
-__device__ __forceinline__ void count_token(const int* e, int k, int64_t t, int64_t T, int E,
-                                            int ep, const RankMap& map, int* hist,
-                                            int* single, int* home) {
+// Count one token into a shared histogram: its k experts, its distinct
+// ranks, and the two statistic bins at the end (tokens whose experts sit on
+// one rank; assignments on the token's home rank floor(t * ep / T)).
+// Registers only: the distinct-rank test compares against the token's
+// earlier slots.  s_map is the expert -> rank map in shared memory.
+template <int KMAX>
+__device__ __forceinline__ void count_token(const int (&e)[KMAX], int k, int64_t t, int64_t T, int E,
+                                            int ep, const uint8_t* s_map, int* hist, int* single,
+                                            int* home) {
   const int home_r = (int)((t * ep) / T);
-  int rs[16];
+  int r[KMAX];
   int nr = 0;
-  for (int j = 0; j < k; ++j) {
-    atomicAdd(&hist[e[j]], 1);
-    const int r = ep > 1 ? map.r[e[j]] : 0;
-    *home += r == home_r;
-    bool seen = false;
-    for (int q = 0; q < nr; ++q) seen |= rs[q] == r;
-    if (!seen) {
-      rs[nr++] = r;
-      if (ep > 1) atomicAdd(&hist[E + r], 1);
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j) {
+    if (j < k) {
+      atomicAdd(&hist[e[j]], 1);
+      r[j] = ep > 1 ? (int)s_map[e[j]] : 0;
+      *home += r[j] == home_r;
+      bool seen = false;
+#pragma unroll
+      for (int q = 0; q < j; ++q) seen |= r[q] == r[j];
+      if (!seen) {
+        ++nr;
+        if (ep > 1) atomicAdd(&hist[E + r[j]], 1);
+      }
     }
   }
   *single += nr == 1;

@@ -12,12 +12,14 @@
 //               k-block, 128-byte swizzle, 3-stage ring
 //   warp 1      TMEM allocation; one lane issues tcgen05.mma 128 x E16 x 16
 //   warps 2-9   epilogue, two threads per token row (each reads half of the
-//               row's E16 fp32 logits with tcgen05.ld): + bias, logits
-//               stored, and a running top-k kept sorted in registers (key:
-//               logit desc, index asc; equal logits keep the lower index
-//               because only a strictly larger logit moves an entry); the
-//               second half's list is merged into the first through shared
-//               memory; gates exp(l_j - l_0) / sum_i.
+//               row's E16 fp32 logits with tcgen05.ld): + bias, and a
+//               running top-k kept sorted in registers (key: logit desc,
+//               index asc; equal logits keep the lower index because only a
+//               strictly larger logit moves an entry); the second half's
+//               list is merged into the first through shared memory; gates
+//               exp(l_j - l_0) / sum_i.  The logits rows are staged in the
+//               operand ring (idle once the accumulator is complete) and
+//               leave with one bulk copy per row.
 // With the histogram on, each token adds its experts, distinct ranks and two
 // statistics to a shared histogram that the CTA stores as its column of
 // block_hist [bins][nb]; the scatter kernel (after the kernel boundary, so every row is
@@ -42,7 +44,7 @@ struct Params {
   int32_t* idx;
   float* gate;
   Control* ctl;
-  int hist, ep, nb, bins;
+  int hist, ep, nb, bins, hist_stride;
   RankMap map;
   int32_t* block_hist;
 };
@@ -78,6 +80,8 @@ __global__ void __launch_bounds__(kThreads, 2)
   __shared__ __align__(8) uint64_t full[kStages], empty[kStages], tfull;
   __shared__ uint32_t tmem_base_s;
   __shared__ int hist[kMaxBins];
+  __shared__ float s_bias[256];
+  __shared__ uint8_t s_map[256];
   __shared__ volatile int abort_flag;
   // the second column half's partial top-k lists, merged by the first half
   __shared__ float m_v[BM][KMAX];
@@ -166,6 +170,13 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int nchunks = p.BN / 16;
     const int c_lo = h == 0 ? 0 : (nchunks + 1) / 2;
     const int c_hi = h == 0 ? (nchunks + 1) / 2 : nchunks;
+    // bias and expert -> rank map in shared memory (read after the
+    // predecessor's completion, like every input)
+    for (int i = threadIdx.x - 64; i < p.E; i += 32 * kEpiWarps) {
+      s_bias[i] = p.bias ? __ldg(p.bias + i) : 0.f;
+      s_map[i] = p.map.r[i];
+    }
+    named_bar_sync(1, 32 * kEpiWarps);
     float tv[KMAX];
     int ti[KMAX];
 #pragma unroll
@@ -174,11 +185,17 @@ __global__ void __launch_bounds__(kThreads, 2)
       ti[s] = 0x7FFFFFFF;
     }
     const bool have = mbar_wait_bounded(&tfull, 0, &abort_flag) && !abort_flag;
+    // the rest of this CTA is short: let the next kernel's CTAs be scheduled
+    pdl_trigger();
+    // logits rows staged in the operand ring (row stride 4E + 16 bytes):
+    // every MMA has completed, so nothing reads the ring any more
+    const bool staged = (p.E & 3) == 0 && (reinterpret_cast<uintptr_t>(p.logits) & 15) == 0;
+    const uint32_t lstride = (uint32_t)p.E * 4 + 16;
+    float* srow = reinterpret_cast<float*>(smem + (size_t)rr * lstride);
+    float* lrow = p.logits + t * p.E;
     if (have) {
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16);
-      float* lrow = p.logits + t * p.E;
-      const bool vec = (p.E & 3) == 0 && (reinterpret_cast<uintptr_t>(p.logits) & 15) == 0;
       for (int ch = c_lo; ch < c_hi; ++ch) {
         const int c = ch * 16;
         uint32_t r[16];
@@ -186,18 +203,21 @@ __global__ void __launch_bounds__(kThreads, 2)
         tmem_ld_wait();
         float v[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int col = c + i;
-          v[i] = __uint_as_float(r[i]) + ((p.bias && col < p.E) ? __ldg(p.bias + col) : 0.f);
-        }
-        if (valid) {
-          if (vec && c + 16 <= p.E) {
+        for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]) + (c + i < p.E ? s_bias[c + i] : 0.f);
+        if (staged) {
+          if (c + 16 <= p.E) {
 #pragma unroll
             for (int i = 0; i < 16; i += 4)
-              *reinterpret_cast<float4*>(lrow + c + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+              *reinterpret_cast<float4*>(srow + c + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
           } else {
-            for (int i = 0; i < 16 && c + i < p.E; ++i) lrow[c + i] = v[i];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              if (c + i < p.E) srow[c + i] = v[i];
           }
+        } else if (valid) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            if (c + i < p.E) lrow[c + i] = v[i];
         }
 #pragma unroll
         for (int i = 0; i < 16; ++i)
@@ -211,8 +231,13 @@ __global__ void __launch_bounds__(kThreads, 2)
         m_i[rr][j] = ti[j];
       }
     }
-    asm volatile("bar.sync 1, %0;" ::"r"(32 * kEpiWarps) : "memory");  // epilogue warps only
+    if (staged) fence_proxy_async_shared();  // staged rows -> bulk copy
+    named_bar_sync(1, 32 * kEpiWarps);       // epilogue warps only
     if (h == 0) {
+      if (have && valid && staged) {
+        bulk_store(lrow, srow, (uint32_t)p.E * 4);
+        bulk_commit();
+      }
       // the second half's columns are all higher, so inserting its entries
       // in order keeps lower indices first among equal logits
 #pragma unroll
@@ -234,12 +259,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       if (p.hist) {
         int single = 0, home = 0;
-        if (have && valid) {
-          int e[KMAX];  // a copy, so the list above stays in registers
-#pragma unroll
-          for (int j = 0; j < KMAX; ++j) e[j] = ti[j];
-          count_token(e, p.k, t, p.T, p.E, p.ep, p.map, hist, &single, &home);
-        }
+        if (have && valid) count_token<KMAX>(ti, p.k, t, p.T, p.E, p.ep, s_map, hist, &single, &home);
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) {
           single += __shfl_xor_sync(0xffffffffu, single, off);
@@ -251,6 +271,8 @@ __global__ void __launch_bounds__(kThreads, 2)
           atomicAdd(&hist[sbin + 1], home);
         }
       }
+      // the staged rows are read before the CTA exits
+      if (have && valid && staged) bulk_wait<0>();
     }
   }
   tc_fence_before();
@@ -259,9 +281,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     tc_fence_after();
     tmem_dealloc(tmem_base, tmem_cols);
   }
-  if (p.hist && tile_ok)  // bin-major [bins][nb], so the scatter reads rows of blocks
+  if (p.hist && tile_ok)  // bin-major [bins][stride], so the scatter reads rows of blocks
     for (int bin = threadIdx.x; bin < p.bins; bin += kThreads)
-      p.block_hist[(size_t)bin * p.nb + b] = hist[bin];
+      p.block_hist[(size_t)bin * p.hist_stride + b] = hist[bin];
 }
 
 template <int KMAX>
@@ -298,6 +320,7 @@ cudaError_t launch_route_tc(const RouteArgs& a, cudaStream_t s) {
   p.ep = a.ep;
   p.nb = layout_blocks(a.T);
   p.bins = layout_bins(a.E, a.ep);
+  p.hist_stride = layout_hist_stride(p.nb);
   p.map = a.map;
   p.block_hist = a.block_hist;
   CUtensorMap mA, mB;
