@@ -46,10 +46,17 @@ SLEEP_CYCLES = 200_000  # ~0.1 ms of device-side sleep before each timed iterati
 # combine
 
 
+def fused_ffn(w: W.Workload) -> bool:
+    """moe_forward runs the expert FFN as one kernel (H on chip) for these."""
+    return w.dtype == "bf16" and w.f in (64, 128) and w.d in (128, 256)
+
+
 def launches_per_step(w: W.Workload) -> int:
     if w.dtype != "bf16":
         return 8
-    return 5 + (1 if w.T * w.d * 2 > (96 << 20) else 0)
+    permute = 1 if w.T * w.d * 2 > (96 << 20) else 0
+    # route, scatter, [permute], gate/up [+ down], combine
+    return (4 if fused_ffn(w) else 5) + permute
 MEASURED_PEAKS = os.path.join(ROOT, "MEASURED_PEAKS.json")
 
 
@@ -69,7 +76,7 @@ def work(w: W.Workload, T: int):
     move.  Stages as moe_forward_timed names them."""
     b = 2 if w.dtype == "bf16" else 4
     R = T * w.k
-    return {
+    out = {
         # x read, W_r read, logits + idx + gate written
         "route": dict(bytes=T * w.d * b + w.E * w.d * b + T * w.E * 4 + 2 * R * 4,
                       flops=2 * T * w.d * w.E),
@@ -86,6 +93,13 @@ def work(w: W.Workload, T: int):
         # y_perm read, gates / slot rows read, y written
         "combine": dict(bytes=R * w.d * b + T * w.d * b + 2 * R * 4, flops=0),
     }
+    if fused_ffn(w):
+        # one kernel for the whole expert FFN, timed as the gate/up stage:
+        # rows of x read, W_g / W_u / W_d read, y_perm written (h stays on chip)
+        out["gate_up"] = dict(bytes=R * w.d * b + 3 * w.E * w.d * w.f * b + R * w.d * b,
+                              flops=6 * R * w.d * w.f)
+        out["down"] = dict(bytes=0, flops=0)
+    return out
 
 
 # ------------------------------------------------------------------- helpers
@@ -292,10 +306,16 @@ def run_ours(args, rank, world, local):
     dom = max(calls, key=calls.get)
     pk = peaks()
     d = wk[dom]
-    if d["flops"] > 0 and d["flops"] / d["bytes"] > pk["bf16"] * 1e12 / (pk["hbm"] * 1e9):
-        bound, achieved, peak, unit = "tensor", d["flops"] / (calls[dom] * 1e-3) / 1e12, pk["bf16"], "TFLOP/s"
+    # a step of a millisecond or more runs at the power-capped clock: the
+    # sustained GEMM peak is its denominator, the burst one otherwise
+    sustained = ms >= 1.0
+    tpeak = pk["bf16_sus"] if sustained else pk["bf16"]
+    if d["flops"] > 0 and d["flops"] / d["bytes"] > tpeak * 1e12 / (pk["hbm"] * 1e9):
+        bound, achieved, peak, unit = "tensor", d["flops"] / (calls[dom] * 1e-3) / 1e12, tpeak, "TFLOP/s"
+        psrc = pk["src"] + (" bf16 sustained" if sustained else " bf16 burst")
     else:
         bound, achieved, peak, unit = "hbm", d["bytes"] / (calls[dom] * 1e-3) / 1e9, pk["hbm"], "GB/s"
+        psrc = pk["src"] + " hbm copy"
     result = {
         "metric": METRIC,
         "value": T * world / (ms * 1e-3),
@@ -322,7 +342,7 @@ def run_ours(args, rank, world, local):
         "step": f"one moe_forward ({launches_per_step(w)} kernels) replayed from a CUDA graph",
         "stage_ms": {k: round(v, 5) for k, v in calls.items()},
         "roofline": {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-                     "frac": achieved / peak, "peak_source": pk["src"], "traffic": None,
+                     "frac": achieved / peak, "peak_source": psrc, "traffic": None,
                      "algorithmic": d},
         "clocks": clk,
     }

@@ -294,7 +294,10 @@ MOE_API moe_status moe_combine(const moe_shape* shape, const void* y_perm,
 /*
  * Optional caller-owned buffers of moe_forward's intermediates (device).
  * Any NULL member is placed in the workspace instead; pass NULL for the
- * whole struct to keep everything in the workspace.
+ * whole struct to keep everything in the workspace.  After the call logits,
+ * routing, layout and y_perm hold their values; x_perm and h are written
+ * only by the paths that materialise them (x_perm: x above 96 MB or fp32;
+ * h: the unfused expert GEMMs) and are otherwise left untouched.
  */
 typedef struct {
   float* logits;      /* [T, E] */
@@ -309,12 +312,16 @@ typedef struct {
 /*
  * The whole layer enqueued back to back on `stream`, with no host
  * synchronisation in between.  bf16: one kernel for router GEMM + top-k +
- * gates + the dispatch histogram and its lookback scan, the layout scatter,
- * the gate/up GEMM with SwiGLU, the down GEMM and the combine; the permute
- * is fused into the gate/up GEMM (as moe_grouped_swiglu_gather, x_perm not
- * written) while x is at most 96 MB, and a separate token-order permute
- * (moe_permute_by_token) otherwise.  fp32: moe_route, moe_dispatch_layout, moe_permute,
- * moe_grouped_swiglu and moe_combine in turn.
+ * gates + the per-tile dispatch histogram, the layout scatter, then the
+ * expert FFN: for f in {64, 128} and d in {128, 256} one kernel for the
+ * gate/up GEMM, SwiGLU (H kept on chip) and down GEMM (same arithmetic as
+ * the separate GEMMs, so the same y_perm), otherwise the gate/up GEMM with
+ * SwiGLU and the down GEMM; then the combine.  The permute is
+ * fused into the gate/up operand load (as moe_grouped_swiglu_gather, x_perm
+ * not written) while x is at most 96 MB, and a separate token-order permute
+ * (moe_permute_by_token) runs otherwise.  fp32: moe_route,
+ * moe_dispatch_layout, moe_permute, moe_grouped_swiglu and moe_combine in
+ * turn.
  *  x [T, d]; packed weights; bias [E] or NULL; expert_rank_host as in
  *  moe_dispatch_layout; y [T, d]; buffers may be NULL;
  *  ws, ws_bytes  moe_forward_workspace_size bytes.

@@ -353,6 +353,8 @@ moe_status forward_impl(const moe_shape* s, const void* x, const void* packed, c
   lo.slot_send_row = f.lay.slot_send_row;
   lo.stats = f.lay.stats;
   const bool bf16 = s->dtype == MOE_BF16;
+  // small f: the whole expert FFN and the combine in one kernel
+  const bool fused = bf16 && ffn_fused_supported(s->d, s->f);
   if ((r = mark(0)) != MOE_OK) return r;
   if (bf16) {
     // router + top-k + gates + per-tile dispatch histogram in one kernel
@@ -379,7 +381,28 @@ moe_status forward_impl(const moe_shape* s, const void* x, const void* packed, c
                                                sc.block_hist, st))) != MOE_OK)
       return r;
     if ((r = mark(2)) != MOE_OK) return r;
-    if (gather_fits(s)) {
+    if (fused) {
+      FfnArgs fa{};
+      const bool g = gather_fits(s);
+      if (!g && (r = cuda_status(launch_permute(x, f.lay.row_token, f.lay.slot_row, f.x_perm, s->T,
+                                                s->k, (uint32_t)(s->d * 2), st))) != MOE_OK)
+        return r;
+      if ((r = mark(3)) != MOE_OK) return r;
+      fa.A = g ? x : f.x_perm;
+      fa.gather = g ? f.lay.row_token : nullptr;
+      fa.src_rows = s->T;
+      fa.rows = s->T * (int64_t)s->k;
+      fa.offsets = f.lay.expert_offsets;
+      fa.G = s->E;
+      fa.d = s->d;
+      fa.f = s->f;
+      fa.wgu = pk.wgu;
+      fa.wdT = pk.wdT;
+      fa.y_perm = f.y_perm;
+      fa.ctl = sc.ctl;
+      if ((r = cuda_status(launch_ffn_fused(fa, st))) != MOE_OK) return r;
+      if ((r = mark(4)) != MOE_OK) return r;
+    } else if (gather_fits(s)) {
       // the permute is fused into the gate/up GEMM's operand loads
       if ((r = mark(3)) != MOE_OK) return r;
       if ((r = do_grouped_part(0, s, x, f.lay.row_token, f.lay.expert_offsets, &pk, f.h, f.y_perm,
@@ -408,10 +431,12 @@ moe_status forward_impl(const moe_shape* s, const void* x, const void* packed, c
                              sc.ctl, st)) != MOE_OK)
       return r;
   }
-  if ((r = mark(4)) != MOE_OK) return r;
-  if ((r = do_grouped_part(1, s, nullptr, nullptr, f.lay.expert_offsets, &pk, f.h, f.y_perm, sc.ctl,
-                           st)) != MOE_OK)
-    return r;
+  if (!fused) {
+    if ((r = mark(4)) != MOE_OK) return r;
+    if ((r = do_grouped_part(1, s, nullptr, nullptr, f.lay.expert_offsets, &pk, f.h, f.y_perm,
+                             sc.ctl, st)) != MOE_OK)
+      return r;
+  }
   if ((r = mark(5)) != MOE_OK) return r;
   if ((r = cuda_status(launch_combine(s->dtype, f.y_perm, f.lay.slot_row, f.gate, y, s->T, s->d,
                                       s->k, st))) != MOE_OK)

@@ -24,7 +24,8 @@
 //   warps 2-9   epilogue, two warps per TMEM lane quadrant (each reads half
 //               of its 32 rows' columns): tcgen05.ld, activation, bf16 rows
 //               to global memory -- straight from registers, or (short K
-//               loops) through shared memory with one bulk copy per row;
+//               loops) staged in shared memory and copied out by whole rows
+//               per warp instruction;
 //               predicated on the group's last row so a tile never writes
 //               rows of the next expert
 // The tile list is (group, 128-row tile, N tile), N fastest, walked with a
@@ -76,9 +77,11 @@ template <int BN, int EPI>
 constexpr uint32_t staged_row_bytes() { return out_cols<BN, EPI>() * 2 + 16; }
 
 // Staged epilogue: each epilogue thread writes its output row into shared
-// memory and one bulk copy per row moves it to global memory (whole rows,
-// coalesced, asynchronous).  Used when the K loop is short and the epilogue
-// would otherwise dominate; it costs pipeline stages.
+// memory, then the quadrant's two warps copy the rows out with every store
+// instruction covering whole contiguous row segments (one small bulk copy
+// per row measured slower: the copy engine's issue rate bound the tile).
+// Used when the K loop is short and the epilogue would otherwise dominate;
+// it costs pipeline stages.
 template <int BN, int EPI, bool STAGED>
 constexpr uint32_t staging_bytes() { return STAGED ? 128u * staged_row_bytes<BN, EPI>() : 0u; }
 
@@ -222,16 +225,24 @@ __global__ void __launch_bounds__(threads_for<GATHER>(), (ctas_per_sm<BN, STAGED
       const int ch = lane & 7, rsub = lane >> 3;
       uint32_t it = 0;
       bool ok = true;
+      // this warp's source rows of a tile; the next tile's are loaded while
+      // the current one is copied, so their latency stays off the critical path
+      auto load_src = [&](int tile, int32_t (&dst)[RPW / 4]) {
+        const TileInfo t2 = decode(tile, n_tiles, tile_off, s_off, G);
+#pragma unroll
+        for (int i = 0; i < RPW / 4; ++i) {
+          const int64_t r = (int64_t)t2.row0 + gw * RPW + 4 * i + rsub;
+          dst[i] = r < p.rows ? __ldg(p.gather + r) : 0;
+        }
+      };
+      int32_t src[RPW / 4], nxt[RPW / 4];
+      if (blockIdx.x < total) load_src(blockIdx.x, nxt);
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         const TileInfo ti = decode(tile, n_tiles, tile_off, s_off, G);
         const int brow = ti.g * p.n_per_group + ti.nt * BN;
-        int32_t src[RPW / 4];
 #pragma unroll
-        for (int i = 0; i < RPW / 4; ++i) {
-          const int64_t r = (int64_t)ti.row0 + gw * RPW + 4 * i + rsub;
-          const int32_t v = r < p.rows ? __ldg(p.gather + r) : 0;
-          src[i] = (v >= 0 && v < p.src_rows) ? v : 0;
-        }
+        for (int i = 0; i < RPW / 4; ++i) src[i] = (nxt[i] >= 0 && nxt[i] < p.src_rows) ? nxt[i] : 0;
+        if (tile + (int)gridDim.x < total) load_src(tile + gridDim.x, nxt);
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
           const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
           int good = 1;
@@ -352,7 +363,12 @@ __global__ void __launch_bounds__(threads_for<GATHER>(), (ctas_per_sm<BN, STAGED
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tc) {
       const TileInfo ti = decode(tile, n_tiles, tile_off, s_off, G);
       const uint32_t b = tc & 1, tph = (tc >> 1) & 1;
-      if (!mbar_wait_bounded(&tfull[b], tph, &abort_flag)) {
+      bool got = mbar_wait_bounded(&tfull[b], tph, &abort_flag);
+      // staged: the quadrant's two warps meet at named barriers below, so
+      // they stop together (and this barrier also orders the previous
+      // tile's copy-out before the staging rows are rewritten)
+      if constexpr (STAGED) got = named_bar_and(qbar, 64, got);
+      if (!got) {
         abort_flag = 1;
         record_error(p.ctl, MOE_ERR_DEVICE_TIMEOUT, 0x300u);
         break;
@@ -366,12 +382,6 @@ __global__ void __launch_bounds__(threads_for<GATHER>(), (ctas_per_sm<BN, STAGED
       static_assert(HC % 32 == 0, "each epilogue half covers whole 32-column groups");
       __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + grow * p.ld_out + ti.nt * OC;
       uint8_t* stg = sOut + (size_t)rr * staged_row_bytes<BN, EPI>();
-      if constexpr (STAGED) {
-        // the row's previous bulk store (issued by the h = 0 thread) has read
-        // the staging row before either half overwrites it
-        if (h == 0) bulk_wait_read<0>();
-        named_bar_sync(qbar, 64);
-      }
       // 32 output columns per TMEM round trip: issue all loads, then wait once
 #pragma unroll 1
       for (int c = h * HC; c < (h + 1) * HC; c += 32) {
@@ -413,11 +423,21 @@ __global__ void __launch_bounds__(threads_for<GATHER>(), (ctas_per_sm<BN, STAGED
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[b]);
-        fence_proxy_async_shared();
         named_bar_sync(qbar, 64);  // both halves of every row staged
-        if (h == 0) {
-          if (valid) bulk_store(out, stg, OC * 2);
-          bulk_commit();
+        // copy-out: warp h writes rows [16h, 16h + 16) of the quadrant, whole
+        // rows per instruction (16 bytes a lane), so every store covers full
+        // contiguous row segments
+        constexpr int RB = OC * 2;    // bytes of one output row of the tile
+        constexpr int CPR = RB / 16;  // 16-byte chunks per row
+        constexpr int RPI = 32 / CPR; // rows per warp instruction
+        static_assert(CPR <= 32 && 32 % CPR == 0, "row chunks tile a warp");
+        const int ch = lane % CPR;
+#pragma unroll
+        for (int r = q * 32 + h * 16 + lane / CPR; r < q * 32 + h * 16 + 16; r += RPI) {
+          const uint4 v = *reinterpret_cast<const uint4*>(sOut + (size_t)r * staged_row_bytes<BN, EPI>() + ch * 16);
+          if (r < ti.rows)
+            *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) +
+                                      ((int64_t)ti.row0 + r) * p.ld_out + ti.nt * OC + ch * 8) = v;
         }
         continue;
       }
@@ -427,9 +447,6 @@ __global__ void __launch_bounds__(threads_for<GATHER>(), (ctas_per_sm<BN, STAGED
     }
   }
 
-  if constexpr (STAGED) {
-    if (warp >= 2) bulk_wait<0>();  // staged rows written before the CTA exits (h = 0 owns them)
-  }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

@@ -121,6 +121,24 @@ struct RouteArgs {
 };
 cudaError_t launch_route_tc(const RouteArgs& a, cudaStream_t s);
 
+// ---- ffn_fused.cu (bf16, tcgen05): gate/up GEMM + SwiGLU + down GEMM in
+// one kernel for small f (H stays on chip); y_perm as moe_grouped_swiglu
+struct FfnArgs {
+  const void* A;             // gather: x [T, d]; else x_perm [rows, d]
+  const int32_t* gather;     // row_token for gather mode, else NULL
+  int64_t src_rows;          // T (gather mode)
+  int64_t rows;              // T * k
+  const int32_t* offsets;    // [E + 1]
+  int G;                     // E
+  int d, f;
+  const void* wgu;           // packed [E * 2f, d] (gate rows then up rows per expert)
+  const void* wdT;           // packed [E * d, f]
+  void* y_perm;              // [rows, d]
+  Control* ctl;
+};
+bool ffn_fused_supported(int d, int f);
+cudaError_t launch_ffn_fused(const FfnArgs& a, cudaStream_t s);
+
 // ---- gemm_simt.cu (fp32, CUDA cores)
 cudaError_t launch_grouped_f32(const float* x_perm, const int32_t* offsets, int E, int64_t R,
                                int d, int f, int blk, const float* wgu, const float* wdT, float* h,

@@ -19,7 +19,7 @@
 //               list is merged into the first through shared memory; gates
 //               exp(l_j - l_0) / sum_i.  The logits rows are staged in the
 //               operand ring (idle once the accumulator is complete) and
-//               leave with one bulk copy per row.
+//               copied out by all epilogue warps in coalesced chunks.
 // With the histogram on, each token adds its experts, distinct ranks and two
 // statistics to a shared histogram that the CTA stores as its column of
 // block_hist [bins][nb]; the scatter kernel (after the kernel boundary, so every row is
@@ -231,13 +231,19 @@ __global__ void __launch_bounds__(kThreads, 2)
         m_i[rr][j] = ti[j];
       }
     }
-    if (staged) fence_proxy_async_shared();  // staged rows -> bulk copy
-    named_bar_sync(1, 32 * kEpiWarps);       // epilogue warps only
-    if (h == 0) {
-      if (have && valid && staged) {
-        bulk_store(lrow, srow, (uint32_t)p.E * 4);
-        bulk_commit();
+    named_bar_sync(1, 32 * kEpiWarps);  // epilogue warps only
+    if (have && staged) {
+      // the tile's valid logits rows are contiguous in global memory: the
+      // eight warps copy them out in 16-byte chunks, fully coalesced
+      const int cpr = p.E / 4;  // chunks per row
+      const int nvalid = (int)(p.T - row0 < BM ? p.T - row0 : BM);
+      float4* dst = reinterpret_cast<float4*>(p.logits + row0 * p.E);
+      for (int c = threadIdx.x - 64; c < nvalid * cpr; c += 32 * kEpiWarps) {
+        const int r = c / cpr, cc = c - r * cpr;
+        dst[c] = *reinterpret_cast<const float4*>(smem + (size_t)r * lstride + cc * 16);
       }
+    }
+    if (h == 0) {
       // the second half's columns are all higher, so inserting its entries
       // in order keeps lower indices first among equal logits
 #pragma unroll
@@ -271,8 +277,6 @@ __global__ void __launch_bounds__(kThreads, 2)
           atomicAdd(&hist[sbin + 1], home);
         }
       }
-      // the staged rows are read before the CTA exits
-      if (have && valid && staged) bulk_wait<0>();
     }
   }
   tc_fence_before();
