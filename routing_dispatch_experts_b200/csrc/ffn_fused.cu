@@ -12,18 +12,21 @@
 // When f is small the whole H tile of 128 rows fits in tensor memory and
 // shared memory, so H never travels to global memory and the three stages
 // of a tile overlap inside one persistent CTA per SM:
-//   warp 0 (+ warps 14-16 in gather mode)  producer: the 128 x 64 A blocks
+//   warp 0 (+ warps 15-17 in gather mode)  producer: the 128 x 64 A blocks
 //           (rows of x through the permutation, by cp.async in gather mode,
 //           else TMA tiles of x_perm) with the matching W_g/W_u block into a
-//           ring; the tile's W_d [d x f] into a double buffer (issued first:
-//           it is needed last, after the gate/up GEMM and the SwiGLU)
-//   warp 1  MMA: acc1 = A W_gu^T (M 128, N 2f) into one of two TMEM
-//           accumulators; acc2 = H W_d^T (M 128, N d) from the H tile in
-//           shared memory.  Issue order MMA1(i), MMA2(i-1), so the SwiGLU of
-//           tile i overlaps the down GEMM of tile i-1
-//   warps 2-5   SwiGLU: acc1 -> bf16 H rows written in the 128-byte-swizzled
+//           ring
+//   warp 1  MMA1: acc1 = A W_gu^T (M 128, N 2f) into one of two TMEM
+//           accumulators (allocates TMEM)
+//   warp 2  MMA2: acc2 = H W_d^T (M 128, N d) from the H tile in shared
+//           memory; it also loads each tile's W_d [d x f] by TMA into one
+//           buffer, the next tile's as soon as the down GEMM has read it.
+//           Separate issuing threads, so neither GEMM's waits hold up the
+//           other (one thread issuing both measured a bubble: each down GEMM
+//           waited for the next tile's rows)
+//   warps 3-6   SwiGLU: acc1 -> bf16 H rows written in the 128-byte-swizzled
 //               K-major layout the down GEMM reads (double-buffered)
-//   warps 6-13  down epilogue: acc2 -> bf16 Y_perm rows (staged per warp,
+//   warps 7-14  down epilogue: acc2 -> bf16 Y_perm rows (staged per warp,
 //               stored in whole 64-byte row segments)
 // The gate-weighted combine stays a separate kernel: folding it in (per-token
 // arrival counters, the last arrival summing the k rows) measured slower on
@@ -44,7 +47,8 @@ constexpr int BM = 128, BK = 64;
 constexpr int kGatherWarps = 4;
 constexpr int kEpi1Warps = 4;
 constexpr int kEpi2Warps = 8;
-constexpr int kEpi1First = 2, kEpi2First = 6, kGatherFirst = 14;
+constexpr int kMma1Warp = 1, kMma2Warp = 2;
+constexpr int kEpi1First = 3, kEpi2First = 7, kGatherFirst = 15;
 
 template <bool GATHER>
 constexpr int ffn_threads() { return 32 * (kGatherFirst + (GATHER ? kGatherWarps - 1 : 0)); }
@@ -66,13 +70,10 @@ struct Cfg {
   static constexpr uint32_t STG_WARP = 32 * STG_ROW;
   static constexpr uint32_t STG_BYTES = kEpi2Warps * STG_WARP;
   static constexpr uint32_t BUDGET = 222u * 1024u;  // of the 227 KB a CTA may use
-  static constexpr int NWD = (2 * (WD_BYTES + H_BYTES) + 2 * STAGE + STG_BYTES <= BUDGET) ? 2 : 1;
-  static constexpr int NHB = NWD;
-  static constexpr int STAGES_RAW =
-      (int)((BUDGET - NWD * WD_BYTES - NHB * H_BYTES - STG_BYTES) / STAGE);
+  static constexpr int NHB = (2 * H_BYTES + WD_BYTES + 3 * STAGE + STG_BYTES <= BUDGET) ? 2 : 1;
+  static constexpr int STAGES_RAW = (int)((BUDGET - WD_BYTES - NHB * H_BYTES - STG_BYTES) / STAGE);
   static constexpr int STAGES = STAGES_RAW > 6 ? 6 : (STAGES_RAW < 2 ? 2 : STAGES_RAW);
-  static constexpr size_t SMEM =
-      (size_t)STAGES * STAGE + NWD * WD_BYTES + NHB * H_BYTES + STG_BYTES + 1024;
+  static constexpr size_t SMEM = (size_t)STAGES * STAGE + WD_BYTES + NHB * H_BYTES + STG_BYTES + 1024;
   static constexpr int KB1 = D / BK;
   static constexpr int KB2 = F / BK;
   static constexpr uint32_t IDESC1 = idesc_bf16_f32(BM, 2 * F);
@@ -115,17 +116,17 @@ __global__ void __launch_bounds__(ffn_threads<GATHER>(), 1)
     ffn_fused_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB1,
                      const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ Params p) {
   using C = Cfg<F, D>;
-  constexpr int STAGES = C::STAGES, NA1 = C::NA1, NWD = C::NWD, NHB = C::NHB;
+  constexpr int STAGES = C::STAGES, NA1 = C::NA1, NHB = C::NHB;
   constexpr int NT = ffn_threads<GATHER>();
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sRing = smem;                                // STAGES x (A | B1)
-  uint8_t* sWd = sRing + STAGES * C::STAGE;             // NWD x W_d tile
-  uint8_t* sH = sWd + NWD * C::WD_BYTES;                // NHB x H tile
+  uint8_t* sWd = sRing + STAGES * C::STAGE;             // W_d tile
+  uint8_t* sH = sWd + C::WD_BYTES;                      // NHB x H tile
   uint8_t* sStg = sH + NHB * C::H_BYTES;                // per-warp staging (down epilogue)
 
-  __shared__ __align__(8) uint64_t full[STAGES], empty[STAGES], wfull[NWD], wempty[NWD];
+  __shared__ __align__(8) uint64_t full[STAGES], empty[STAGES], wfull, wempty;
   __shared__ __align__(8) uint64_t a1full[NA1], a1empty[NA1], hfull[NHB], hempty[NHB];
   __shared__ __align__(8) uint64_t a2full, a2empty, done;
   __shared__ uint32_t tmem_base_s;
@@ -161,10 +162,8 @@ __global__ void __launch_bounds__(ffn_threads<GATHER>(), 1)
         mbar_init(&full[s], GATHER ? 32 * kGatherWarps + 1 : 1);
         mbar_init(&empty[s], 1);
       }
-      for (int b = 0; b < NWD; ++b) {
-        mbar_init(&wfull[b], 1);
-        mbar_init(&wempty[b], 1);
-      }
+      mbar_init(&wfull, 1);
+      mbar_init(&wempty, 1);
       for (int b = 0; b < NA1; ++b) {
         mbar_init(&a1full[b], 1);
         mbar_init(&a1empty[b], kEpi1Warps);
@@ -175,13 +174,13 @@ __global__ void __launch_bounds__(ffn_threads<GATHER>(), 1)
       }
       mbar_init(&a2full, 1);
       mbar_init(&a2empty, kEpi2Warps);
-      mbar_init(&done, 1);
+      mbar_init(&done, 2);  // one commit per MMA-issuing thread
       fence_barrier_init();
       if (!GATHER) tma_prefetch_desc(&tmA);
       tma_prefetch_desc(&tmB1);
       tma_prefetch_desc(&tmB2);
     }
-  } else if (warp == 1) {
+  } else if (warp == kMma1Warp) {
     tmem_alloc(&tmem_base_s, C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -197,7 +196,7 @@ __global__ void __launch_bounds__(ffn_threads<GATHER>(), 1)
     constexpr int RPW = BM / kGatherWarps;
     const int gw = warp == 0 ? 0 : warp - (kGatherFirst - 1);
     const int ch = lane & 7, rsub = lane >> 3;
-    uint32_t it = 0, tl = 0;
+    uint32_t it = 0;
     bool ok = true;
     int32_t src[RPW / 4], nxt[RPW / 4];
     auto load_src = [&](int tile, int32_t (&dst)[RPW / 4]) {
@@ -209,34 +208,12 @@ __global__ void __launch_bounds__(ffn_threads<GATHER>(), 1)
       }
     };
     if (GATHER && blockIdx.x < total) load_src(blockIdx.x, nxt);
-    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++tl) {
+    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
       const TileInfo ti = decode(tile, tile_off, s_off, G);
       if constexpr (GATHER) {
 #pragma unroll
         for (int i = 0; i < RPW / 4; ++i) src[i] = (nxt[i] >= 0 && nxt[i] < p.src_rows) ? nxt[i] : 0;
         if (tile + (int)gridDim.x < total) load_src(tile + gridDim.x, nxt);
-      }
-      // the tile's W_d [D x F]: F / 64 blocks of D rows x 64.  Double-
-      // buffered, it goes first (its buffer was freed by MMA2 two tiles back,
-      // which the MMA warp issues before this tile's MMA1); single-buffered,
-      // after the A blocks, since its buffer frees only after MMA2 of the
-      // previous tile, which follows this tile's MMA1.
-      auto issue_wd = [&]() {
-        if (gw == 0 && lane == 0) {
-          const uint32_t wb = tl % NWD, wph = (tl / NWD) & 1;
-          if (!mbar_wait_bounded(&wempty[wb], wph ^ 1, &abort_flag)) {
-            ok = false;
-          } else {
-            mbar_arrive_expect_tx(&wfull[wb], C::WD_BYTES);
-            for (int kb = 0; kb < C::KB2; ++kb)
-              tma_load_2d(sWd + wb * C::WD_BYTES + kb * C::WD_KBLK, &tmB2, &wfull[wb], kb * BK, ti.g * D);
-          }
-        }
-        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-      };
-      if (NWD == 2) {
-        issue_wd();
-        if (!ok) break;
       }
       for (int kb = 0; kb < C::KB1; ++kb, ++it) {
         const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
@@ -266,7 +243,6 @@ __global__ void __launch_bounds__(ffn_threads<GATHER>(), 1)
           cp_async_arrive_noinc(&full[s]);
         }
       }
-      if (NWD == 1 && ok) issue_wd();
     }
     if (lane == 0 && !ok) {
       abort_flag = 1;
@@ -277,76 +253,106 @@ __global__ void __launch_bounds__(ffn_threads<GATHER>(), 1)
     if (gw == 0 && lane == 0) {
       const uint32_t first = it > (uint32_t)STAGES ? it - STAGES : 0;
       for (uint32_t q = first; q < it; ++q) mbar_wait_bounded(&full[q % STAGES], (q / STAGES) & 1, nullptr);
-      const uint32_t wfirst = tl > (uint32_t)NWD ? tl - NWD : 0;
-      for (uint32_t q = wfirst; q < tl; ++q) mbar_wait_bounded(&wfull[q % NWD], (q / NWD) & 1, nullptr);
     }
-  } else if (warp == 1) {
-    // ----------------------------------------------------------------- MMA
+  } else if (warp == kMma1Warp) {
+    // ---------------------------------------------------------------- MMA1
     if (lane == 0) {
-      int n = 0;
-      for (int tile = blockIdx.x; tile < total; tile += gridDim.x) ++n;
-      uint32_t it = 0;
+      uint32_t it = 0, i = 0;
       bool ok = true;
-      for (int i = 0; i <= n && ok; ++i) {
-        if (i < n) {
-          // MMA1(i): acc1[i % NA1] = A W_gu^T over D
-          const uint32_t ab = i % NA1, aph = (i / NA1) & 1;
-          if (!mbar_wait_bounded(&a1empty[ab], aph ^ 1, &abort_flag)) {
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++i) {
+        // acc1[i % NA1] = A W_gu^T over D
+        const uint32_t ab = i % NA1, aph = (i / NA1) & 1;
+        if (!mbar_wait_bounded(&a1empty[ab], aph ^ 1, &abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d1 = tmem_base + ab * 2 * F;
+        for (int kb = 0; kb < C::KB1; ++kb, ++it) {
+          const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
+          if (!mbar_wait_bounded(&full[s], ph, &abort_flag)) {
             ok = false;
             break;
           }
+          if constexpr (GATHER) fence_proxy_async_shared();  // cp.async rows -> tensor core
           tc_fence_after();
-          const uint32_t d1 = tmem_base + ab * 2 * F;
-          for (int kb = 0; kb < C::KB1; ++kb, ++it) {
-            const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
-            if (!mbar_wait_bounded(&full[s], ph, &abort_flag)) {
-              ok = false;
-              break;
-            }
-            if constexpr (GATHER) fence_proxy_async_shared();  // cp.async rows -> tensor core
-            tc_fence_after();
-            const uint32_t a0 = smem_u32(sRing + s * C::STAGE);
-            const uint32_t b0 = a0 + C::A_BYTES;
+          const uint32_t a0 = smem_u32(sRing + s * C::STAGE);
+          const uint32_t b0 = a0 + C::A_BYTES;
 #pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk)
-              tc_mma_f16(d1, smem_desc_k128(a0 + kk * 32), smem_desc_k128(b0 + kk * 32), C::IDESC1,
-                         (kb | kk) != 0);
-            tc_commit(&empty[s]);
-          }
-          if (!ok) break;
-          tc_commit(&a1full[ab]);
+          for (int kk = 0; kk < BK / 16; ++kk)
+            tc_mma_f16(d1, smem_desc_k128(a0 + kk * 32), smem_desc_k128(b0 + kk * 32), C::IDESC1,
+                       (kb | kk) != 0);
+          tc_commit(&empty[s]);
         }
-        if (i >= 1) {
-          // MMA2(i-1): acc2 = H W_d^T over F
-          const int j = i - 1;
-          const uint32_t hb = j % NHB, wb = j % NWD;
-          if (!mbar_wait_bounded(&hfull[hb], (j / NHB) & 1, &abort_flag) ||
-              !mbar_wait_bounded(&wfull[wb], (j / NWD) & 1, &abort_flag) ||
-              !mbar_wait_bounded(&a2empty, (j & 1) ^ 1, &abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t d2 = tmem_base + C::A2_COL;
-#pragma unroll
-          for (int kb = 0; kb < C::KB2; ++kb) {
-            const uint32_t h0 = smem_u32(sH + hb * C::H_BYTES + kb * C::H_KBLK);
-            const uint32_t w0 = smem_u32(sWd + wb * C::WD_BYTES + kb * C::WD_KBLK);
-#pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk)
-              tc_mma_f16(d2, smem_desc_k128(h0 + kk * 32), smem_desc_k128(w0 + kk * 32), C::IDESC2,
-                         (kb | kk) != 0);
-          }
-          tc_commit(&hempty[hb]);
-          tc_commit(&wempty[wb]);
-          tc_commit(&a2full);
-        }
+        if (!ok) break;
+        tc_commit(&a1full[ab]);
       }
       if (!ok) {
         abort_flag = 1;
         record_error(p.ctl, MOE_ERR_DEVICE_TIMEOUT, 0x700u);
       }
+      // this thread's MMAs complete before TMEM is released
+      tc_commit(&done);
+      mbar_wait_bounded(&done, 0, nullptr);
+    }
+  } else if (warp == kMma2Warp) {
+    // ---------------------------------------------------------------- MMA2
+    // This warp also loads each tile's W_d [D x F] (F / 64 blocks of D rows
+    // x 64) into the single W_d buffer: the next tile's as soon as this
+    // tile's down GEMM has completed, while the SwiGLU of the next tile is
+    // still running.
+    if (lane == 0) {
+      uint32_t j = 0;
+      bool ok = true;
+      auto load_wd = [&](int tile) {
+        const TileInfo ti = decode(tile, tile_off, s_off, G);
+        mbar_arrive_expect_tx(&wfull, C::WD_BYTES);
+        for (int kb = 0; kb < C::KB2; ++kb)
+          tma_load_2d(sWd + kb * C::WD_KBLK, &tmB2, &wfull, kb * BK, ti.g * D);
+      };
+      if (blockIdx.x < total) load_wd(blockIdx.x);
+      for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++j) {
+        // acc2 = H W_d^T over F
+        const uint32_t hb = j % NHB;
+        if (!mbar_wait_bounded(&hfull[hb], (j / NHB) & 1, &abort_flag) ||
+            !mbar_wait_bounded(&wfull, j & 1, &abort_flag) ||
+            !mbar_wait_bounded(&a2empty, (j & 1) ^ 1, &abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d2 = tmem_base + C::A2_COL;
+#pragma unroll
+        for (int kb = 0; kb < C::KB2; ++kb) {
+          const uint32_t h0 = smem_u32(sH + hb * C::H_BYTES + kb * C::H_KBLK);
+          const uint32_t w0 = smem_u32(sWd + kb * C::WD_KBLK);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            tc_mma_f16(d2, smem_desc_k128(h0 + kk * 32), smem_desc_k128(w0 + kk * 32), C::IDESC2,
+                       (kb | kk) != 0);
+        }
+        tc_commit(&hempty[hb]);
+        tc_commit(&wempty);
+        tc_commit(&a2full);
+        if (tile + (int)gridDim.x < total) {
+          // W_d of the next tile once this down GEMM has read the buffer
+          if (!mbar_wait_bounded(&wempty, j & 1, &abort_flag)) {
+            ok = false;
+            break;
+          }
+          load_wd(tile + gridDim.x);
+        }
+      }
+      if (!ok) {
+        abort_flag = 1;
+        record_error(p.ctl, MOE_ERR_DEVICE_TIMEOUT, 0x780u);
+      }
+      // every MMA of this CTA is issued: let the next kernel's CTAs be
+      // scheduled (they still wait for this grid to complete)
       pdl_trigger();
+      // a W_d load issued for a tile that was not reached (error path) lands
+      // before the CTA may exit
+      if (!ok) mbar_wait_bounded(&wfull, j & 1, nullptr);
       tc_commit(&done);
       mbar_wait_bounded(&done, 0, nullptr);
     }
@@ -449,7 +455,7 @@ __global__ void __launch_bounds__(ffn_threads<GATHER>(), 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kMma1Warp) {
     tc_fence_after();
     tmem_dealloc(tmem_base, C::TMEM_COLS);
   }

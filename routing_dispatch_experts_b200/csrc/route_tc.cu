@@ -9,7 +9,7 @@
 //
 // One CTA per 128-token tile:
 //   warp 0      TMA producer: x tile [128 x 64] and W_r^T tile [E16 x 64] per
-//               k-block, 128-byte swizzle, 3-stage ring
+//               k-block, 128-byte swizzle, 4-stage ring
 //   warp 1      TMEM allocation; one lane issues tcgen05.mma 128 x E16 x 16
 //   warps 2-9   epilogue, two threads per token row (each reads half of the
 //               row's E16 fp32 logits with tcgen05.ld): + bias, and a
@@ -32,7 +32,7 @@ namespace moe {
 
 namespace {
 
-constexpr int BM = 128, BK = 64, kStages = 3;
+constexpr int BM = 128, BK = 64, kStages = 4;  // d = 256: every k-block in flight at once
 constexpr int kEpiWarps = 8;                     // two per TMEM lane quadrant
 constexpr int kThreads = 64 + 32 * kEpiWarps;    // producer + MMA + epilogue
 
