@@ -64,9 +64,17 @@ def peaks():
     try:
         p = json.load(open(MEASURED_PEAKS))
         return dict(hbm=p["hbm_gbs"], bf16=p["bf16_tflops"], bf16_sus=p["bf16_tflops_sustained"],
-                    src="measured")
+                    sm_max_mhz=p.get("sm_max_mhz", 1965.0), src="measured")
     except Exception:
-        return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, sm_max_mhz=1965.0, src="fallback")
+
+
+# DRAM bytes (read + write) per launch of the dominant kernel, from one ncu
+# capture of that kernel as committed (cold cache, the profiles directory
+# holds the summary); None where no capture of the current kernel exists
+NCU_TRAFFIC = {
+    (2, "gate_up"): 14_990_592 + 11_776,  # ffn_fused_kernel<64, 256, gather>
+}
 
 
 # ------------------------------------------------------------ algorithmic work
@@ -310,7 +318,15 @@ def run_ours(args, rank, world, local):
     # sustained GEMM peak is its denominator, the burst one otherwise
     sustained = ms >= 1.0
     tpeak = pk["bf16_sus"] if sustained else pk["bf16"]
-    if d["flops"] > 0 and d["flops"] / d["bytes"] > tpeak * 1e12 / (pk["hbm"] * 1e9):
+    if w.dtype != "bf16" and d["flops"] > 0:
+        # fp32 expert GEMMs run on the CUDA cores' FMA pipes: SMs x 128 fp32
+        # lanes x 2 FLOP per clock at the maximum SM clock
+        props = torch.cuda.get_device_properties(dev)
+        fma_peak = props.multi_processor_count * 128 * 2 * pk["sm_max_mhz"] * 1e6 / 1e12
+        bound, achieved, peak, unit = "alu", d["flops"] / (calls[dom] * 1e-3) / 1e12, fma_peak, "TFLOP/s"
+        psrc = (f"derived: {props.multi_processor_count} SMs x 128 fp32 lanes x 2 FLOP x "
+                f"{pk['sm_max_mhz']:.0f} MHz")
+    elif d["flops"] > 0 and d["flops"] / d["bytes"] > tpeak * 1e12 / (pk["hbm"] * 1e9):
         bound, achieved, peak, unit = "tensor", d["flops"] / (calls[dom] * 1e-3) / 1e12, tpeak, "TFLOP/s"
         psrc = pk["src"] + (" bf16 sustained" if sustained else " bf16 burst")
     else:
@@ -342,7 +358,8 @@ def run_ours(args, rank, world, local):
         "step": f"one moe_forward ({launches_per_step(w)} kernels) replayed from a CUDA graph",
         "stage_ms": {k: round(v, 5) for k, v in calls.items()},
         "roofline": {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-                     "frac": achieved / peak, "peak_source": psrc, "traffic": None,
+                     "frac": achieved / peak, "peak_source": psrc,
+                     "traffic": NCU_TRAFFIC.get((args.config, dom)),
                      "algorithmic": d},
         "clocks": clk,
     }
