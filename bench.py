@@ -90,8 +90,8 @@ def work(w: W.Workload, T: int):
                       flops=2 * T * w.d * w.E),
         # idx read; row_token, slot_row, send_token, slot_send_row written
         "layout": dict(bytes=R * 4 + 4 * R * 4, flops=0),
-        # x rows read once per assignment, x_perm written
-        "permute": dict(bytes=R * w.d * b + R * w.d * b + R * 4, flops=0),
+        # x read once, x_perm written, row indices read
+        "permute": dict(bytes=T * w.d * b + R * w.d * b + R * 4, flops=0),
         # rows of x (or x_perm) read, W_g / W_u read, h written
         "gate_up": dict(bytes=R * w.d * b + 2 * w.E * w.d * w.f * b + R * w.f * b,
                         flops=4 * R * w.d * w.f),
