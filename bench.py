@@ -314,9 +314,10 @@ def run_ours(args, rank, world, local):
     dom = max(calls, key=calls.get)
     pk = peaks()
     d = wk[dom]
-    # a step of a millisecond or more runs at the power-capped clock: the
-    # sustained GEMM peak is its denominator, the burst one otherwise
-    sustained = ms >= 1.0
+    # steps that ran at the power-capped clock (the sampler saw sw_power_cap
+    # during the timed region, or the step is a millisecond or more) take the
+    # sustained GEMM peak as denominator, the others the burst one
+    sustained = ms >= 1.0 or bool(clk and "sw_power_cap" in clk.get("reasons", []))
     tpeak = pk["bf16_sus"] if sustained else pk["bf16"]
     if w.dtype != "bf16" and d["flops"] > 0:
         # fp32 expert GEMMs run on the CUDA cores' FMA pipes: SMs x 128 fp32

@@ -137,10 +137,39 @@ __global__ void __launch_bounds__(ffn_threads<GATHER>(), 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.G;
 
+  // setup that reads nothing the previous kernel writes runs before the
+  // dependency wait: barriers, tensor memory, descriptor prefetch
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], GATHER ? 32 * kGatherWarps + 1 : 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(&wfull, 1);
+    mbar_init(&wempty, 1);
+    for (int b = 0; b < NA1; ++b) {
+      mbar_init(&a1full[b], 1);
+      mbar_init(&a1empty[b], kEpi1Warps);
+    }
+    for (int b = 0; b < NHB; ++b) {
+      mbar_init(&hfull[b], kEpi1Warps);
+      mbar_init(&hempty[b], 1);
+    }
+    mbar_init(&a2full, 1);
+    mbar_init(&a2empty, kEpi2Warps);
+    mbar_init(&done, 2);  // one commit per MMA-issuing thread
+    fence_barrier_init();
+    if (!GATHER) tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB1);
+    tma_prefetch_desc(&tmB2);
+  } else if (warp == kMma1Warp) {
+    tmem_alloc(&tmem_base_s, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  __syncwarp();
   pdl_wait();
   for (int g = threadIdx.x; g <= G; g += NT)
     s_off[g] = min(max(__ldg(p.offsets + g), 0), (int)p.rows);
-  if (threadIdx.x == 0) abort_flag = 0;
   __syncthreads();
   if (warp == 0) {
     int carry = 0;
@@ -156,35 +185,10 @@ __global__ void __launch_bounds__(ffn_threads<GATHER>(), 1)
       if (g < G) tile_off[g] = carry + incl - v;
       carry += __shfl_sync(0xffffffffu, incl, 31);
     }
-    if (lane == 0) {
-      tile_off[G] = carry;
-      for (int s = 0; s < STAGES; ++s) {
-        mbar_init(&full[s], GATHER ? 32 * kGatherWarps + 1 : 1);
-        mbar_init(&empty[s], 1);
-      }
-      mbar_init(&wfull, 1);
-      mbar_init(&wempty, 1);
-      for (int b = 0; b < NA1; ++b) {
-        mbar_init(&a1full[b], 1);
-        mbar_init(&a1empty[b], kEpi1Warps);
-      }
-      for (int b = 0; b < NHB; ++b) {
-        mbar_init(&hfull[b], kEpi1Warps);
-        mbar_init(&hempty[b], 1);
-      }
-      mbar_init(&a2full, 1);
-      mbar_init(&a2empty, kEpi2Warps);
-      mbar_init(&done, 2);  // one commit per MMA-issuing thread
-      fence_barrier_init();
-      if (!GATHER) tma_prefetch_desc(&tmA);
-      tma_prefetch_desc(&tmB1);
-      tma_prefetch_desc(&tmB2);
-    }
-  } else if (warp == kMma1Warp) {
-    tmem_alloc(&tmem_base_s, C::TMEM_COLS);
-    tmem_relinquish();
+    if (lane == 0) tile_off[G] = carry;
   }
   tc_fence_before();
+  __syncwarp();  // role branches diverged single lanes: reconverge before the CTA barrier
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = tmem_base_s;
@@ -454,6 +458,7 @@ __global__ void __launch_bounds__(ffn_threads<GATHER>(), 1)
   }
 
   tc_fence_before();
+  __syncwarp();  // role branches diverged single lanes: reconverge before the CTA barrier
   __syncthreads();
   if (warp == kMma1Warp) {
     tc_fence_after();

@@ -157,14 +157,36 @@ __global__ void __launch_bounds__(threads_for<GATHER>(), (ctas_per_sm<BN, STAGED
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.G;
 
+  // setup that reads nothing an earlier kernel writes runs before the
+  // dependency wait: barriers, tensor memory, descriptor prefetch
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    for (int s = 0; s < STAGES; ++s) {
+      // gather mode: the TMA arrival plus one cp.async arrival per lane of
+      // every gather warp
+      mbar_init(&full[s], GATHER ? 32 * kGatherWarps + 1 : 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], kEpiWarps);
+    }
+    mbar_init(&done, 1);
+    fence_barrier_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  } else if (warp == 1) {
+    tmem_alloc(&tmem_base_s, TMEM_COLS);
+    tmem_relinquish();
+  }
+  __syncwarp();
   // everything below reads what earlier kernels wrote (offsets, operands)
   pdl_wait();
-  // group offsets and the prefix of 128-row tiles per group
-  // offsets clamped to [0, rows]: a malformed offset array can never make
-  // the epilogue store outside the output
+  // group offsets and the prefix of 128-row tiles per group; offsets clamped
+  // to [0, rows]: a malformed offset array can never make the epilogue store
+  // outside the output
   for (int g = threadIdx.x; g <= G; g += NT)
     s_off[g] = p.offsets ? min(max(__ldg(p.offsets + g), 0), (int)p.rows) : (g == 0 ? 0 : (int)p.rows);
-  if (threadIdx.x == 0) abort_flag = 0;
   __syncthreads();
   if (warp == 0) {
     int carry = 0;
@@ -180,28 +202,10 @@ __global__ void __launch_bounds__(threads_for<GATHER>(), (ctas_per_sm<BN, STAGED
       if (g < G) tile_off[g] = carry + incl - v;
       carry += __shfl_sync(0xffffffffu, incl, 31);
     }
-    if (lane == 0) {
-      tile_off[G] = carry;
-      for (int s = 0; s < STAGES; ++s) {
-        // gather mode: the TMA arrival plus one cp.async arrival per lane
-        // of every gather warp
-        mbar_init(&full[s], GATHER ? 32 * kGatherWarps + 1 : 1);
-        mbar_init(&empty[s], 1);
-      }
-      for (int b = 0; b < 2; ++b) {
-        mbar_init(&tfull[b], 1);
-        mbar_init(&tempty[b], kEpiWarps);
-      }
-      mbar_init(&done, 1);
-      fence_barrier_init();
-      tma_prefetch_desc(&tmA);
-      tma_prefetch_desc(&tmB);
-    }
-  } else if (warp == 1) {
-    tmem_alloc(&tmem_base_s, TMEM_COLS);
-    tmem_relinquish();
+    if (lane == 0) tile_off[G] = carry;
   }
   tc_fence_before();
+  __syncwarp();  // role branches diverged single lanes: reconverge before the CTA barrier
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = tmem_base_s;
@@ -448,6 +452,7 @@ __global__ void __launch_bounds__(threads_for<GATHER>(), (ctas_per_sm<BN, STAGED
   }
 
   tc_fence_before();
+  __syncwarp();  // role branches diverged single lanes: reconverge before the CTA barrier
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
@@ -485,6 +490,19 @@ bool make_kmajor_map(CUtensorMap* m, const void* base, int64_t rows, int K, int 
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool make_f32_map(CUtensorMap* m, const void* base, int64_t rows, int cols, int box_rows) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * 4};
+  cuuint32_t box[2] = {32, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 

@@ -99,6 +99,9 @@ struct GemmArgs {
 };
 cudaError_t launch_gemm_tc(int epi, int bn, const GemmArgs& a, cudaStream_t s);
 bool make_kmajor_map(CUtensorMap* m, const void* base, int64_t rows, int K, int box_rows);
+// 2-D fp32 [rows, cols] row-major, box of 32 columns (128 B) x box_rows,
+// 128-byte swizzle (for tiled stores of swizzled shared-memory tiles)
+bool make_f32_map(CUtensorMap* m, const void* base, int64_t rows, int cols, int box_rows);
 
 // ---- route_tc.cu (bf16, tcgen05): router GEMM + bias + top-k + gates in one
 // kernel, optionally with the layout histogram and its lookback scan

@@ -9,17 +9,18 @@
 //
 // One CTA per 128-token tile:
 //   warp 0      TMA producer: x tile [128 x 64] and W_r^T tile [E16 x 64] per
-//               k-block, 128-byte swizzle, 4-stage ring
+//               k-block, 128-byte swizzle, a ring as deep as fits (all
+//               k-blocks of d = 256 in flight)
 //   warp 1      TMEM allocation; one lane issues tcgen05.mma 128 x E16 x 16
-//   warps 2-9   epilogue, two threads per token row (each reads half of the
-//               row's E16 fp32 logits with tcgen05.ld): + bias, and a
+//   warps 2-9   epilogue, two threads per token row (each reads a half of
+//               the row's E16 fp32 logits with tcgen05.ld): + bias, and a
 //               running top-k kept sorted in registers (key: logit desc,
 //               index asc; equal logits keep the lower index because only a
-//               strictly larger logit moves an entry); the second half's
-//               list is merged into the first through shared memory; gates
-//               exp(l_j - l_0) / sum_i.  The logits rows are staged in the
-//               operand ring (idle once the accumulator is complete) and
-//               copied out by all epilogue warps in coalesced chunks.
+//               strictly larger logit moves an entry); the other half's
+//               list is merged into the first's through shared memory;
+//               gates exp(l_j - l_0) / sum_i.  The logits tile is staged in
+//               the operand ring (idle once the accumulator is complete) and
+//               leaves by TMA tiled stores (E % 32 == 0) or a coalesced copy.
 // With the histogram on, each token adds its experts, distinct ranks and two
 // statistics to a shared histogram that the CTA stores as its column of
 // block_hist [bins][nb]; the scatter kernel (after the kernel boundary, so every row is
@@ -32,8 +33,13 @@ namespace moe {
 
 namespace {
 
-constexpr int BM = 128, BK = 64, kStages = 4;  // d = 256: every k-block in flight at once
-constexpr int kEpiWarps = 8;                     // two per TMEM lane quadrant
+constexpr int BM = 128, BK = 64;
+// operand ring depth: as many k-blocks in flight as fit (all of them for
+// d = 256), so a CTA streaming a tall x tile keeps enough bytes in flight
+constexpr int kMaxStages = 8;
+constexpr size_t kRingBudget = 200u * 1024u;
+constexpr int kEpiWarps = 8;                     // kParts per TMEM lane quadrant (16 measured slower)
+constexpr int kParts = kEpiWarps / 4;            // threads per token row
 constexpr int kThreads = 64 + 32 * kEpiWarps;    // producer + MMA + epilogue
 
 struct Params {
@@ -45,6 +51,11 @@ struct Params {
   float* gate;
   Control* ctl;
   int hist, ep, nb, bins, hist_stride;
+  int stages;
+  // logits out of the staged tile: 2 = TMA tiled stores of 128-byte-swizzled
+  // 32-column blocks, 1 = coalesced copy of padded rows, 0 = direct stores
+  int logits_mode;
+  uint32_t merge_off;  // shared-memory offset of the partial top-k lists
   RankMap map;
   int32_t* block_hist;
 };
@@ -67,25 +78,23 @@ __device__ __forceinline__ void topk_insert(float (&tv)[KMAX], int (&ti)[KMAX], 
 }
 
 template <int KMAX>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 1)
     route_fused_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                       const __grid_constant__ Params p) {
+                       const __grid_constant__ CUtensorMap tmL, const __grid_constant__ Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t A_BYTES = BM * BK * 2;
   const uint32_t B_BYTES = (uint32_t)p.BN * BK * 2;
   uint8_t* sA = smem;
+  const int kStages = p.stages;
   uint8_t* sB = smem + kStages * A_BYTES;
 
-  __shared__ __align__(8) uint64_t full[kStages], empty[kStages], tfull;
+  __shared__ __align__(8) uint64_t full[kMaxStages], empty[kMaxStages], tfull;
   __shared__ uint32_t tmem_base_s;
   __shared__ int hist[kMaxBins];
   __shared__ float s_bias[256];
   __shared__ uint8_t s_map[256];
   __shared__ volatile int abort_flag;
-  // the second column half's partial top-k lists, merged by the first half
-  __shared__ float m_v[BM][KMAX];
-  __shared__ int m_i[BM][KMAX];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t tmem_cols = p.BN <= 32 ? 32 : (p.BN <= 64 ? 64 : (p.BN <= 128 ? 128 : 256));
@@ -100,6 +109,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     fence_barrier_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if (p.logits_mode == 2) tma_prefetch_desc(&tmL);
   }
   for (int i = threadIdx.x; i < p.bins; i += kThreads) hist[i] = 0;
   if (warp == 1) {
@@ -107,6 +117,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     tmem_relinquish();
   }
   tc_fence_before();
+  __syncwarp();  // role branches diverged single lanes: reconverge before the CTA barrier
   __syncthreads();
   tc_fence_after();
   pdl_wait();
@@ -160,16 +171,17 @@ __global__ void __launch_bounds__(kThreads, 2)
       tc_commit(&tfull);
     }
   } else if (tile_ok) {
-    // warps 2..9: quadrant q = warp % 4 (the TMEM lanes this warp may read),
-    // half h = which half of the 16-column chunks it scans
+    // warps 2..: quadrant q = warp % 4 (the TMEM lanes this warp may read),
+    // part = which share of the row's 16-column chunks it scans
     const int q = warp & 3;
-    const int h = (warp - 2) >> 2;
+    const int part = (warp - 2) >> 2;  // 0 .. kParts-1
     const int rr = q * 32 + lane;
     const int64_t t = row0 + rr;
     const bool valid = t < p.T;
     const int nchunks = p.BN / 16;
-    const int c_lo = h == 0 ? 0 : (nchunks + 1) / 2;
-    const int c_hi = h == 0 ? (nchunks + 1) / 2 : nchunks;
+    const int per = (nchunks + kParts - 1) / kParts;
+    const int c_lo = min(part * per, nchunks);
+    const int c_hi = min(c_lo + per, nchunks);
     // bias and expert -> rank map in shared memory (read after the
     // predecessor's completion, like every input)
     for (int i = threadIdx.x - 64; i < p.E; i += 32 * kEpiWarps) {
@@ -187,11 +199,12 @@ __global__ void __launch_bounds__(kThreads, 2)
     const bool have = mbar_wait_bounded(&tfull, 0, &abort_flag) && !abort_flag;
     // the rest of this CTA is short: let the next kernel's CTAs be scheduled
     pdl_trigger();
-    // logits rows staged in the operand ring (row stride 4E + 16 bytes):
-    // every MMA has completed, so nothing reads the ring any more
-    const bool staged = (p.E & 3) == 0 && (reinterpret_cast<uintptr_t>(p.logits) & 15) == 0;
+    // The logits tile is staged in the operand ring (every MMA has completed,
+    // so nothing reads it any more).  Mode 2: 32-column blocks of 128 rows x
+    // 128 B, 16-byte chunk x of row r at chunk x ^ (r % 8) (the 128-byte
+    // swizzle the tensor map undoes); mode 1: rows of 4E + 16 bytes.
+    const int mode = p.logits_mode;
     const uint32_t lstride = (uint32_t)p.E * 4 + 16;
-    float* srow = reinterpret_cast<float*>(smem + (size_t)rr * lstride);
     float* lrow = p.logits + t * p.E;
     if (have) {
       tc_fence_after();
@@ -204,7 +217,16 @@ __global__ void __launch_bounds__(kThreads, 2)
         float v[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]) + (c + i < p.E ? s_bias[c + i] : 0.f);
-        if (staged) {
+        if (mode == 2) {
+          // E % 32 == 0: the chunk's 16 columns are 4 whole 16-byte chunks
+          uint8_t* blk = smem + (size_t)(c >> 5) * (BM * 128) + rr * 128;
+          const int x0 = (c & 31) >> 2;
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            *reinterpret_cast<float4*>(blk + (((x0 + u) ^ (rr & 7)) << 4)) =
+                make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+        } else if (mode == 1) {
+          float* srow = reinterpret_cast<float*>(smem + (size_t)rr * lstride);
           if (c + 16 <= p.E) {
 #pragma unroll
             for (int i = 0; i < 16; i += 4)
@@ -224,17 +246,28 @@ __global__ void __launch_bounds__(kThreads, 2)
           if (c + i < p.E) topk_insert<KMAX>(tv, ti, v[i], c + i);
       }
     }
-    if (h == 1) {
+    // parts 1.. leave their lists for part 0 in shared memory
+    float* m_v = reinterpret_cast<float*>(smem + p.merge_off);  // [kParts-1][BM][KMAX]
+    int* m_i = reinterpret_cast<int*>(smem + p.merge_off) + (kParts - 1) * BM * KMAX;
+    if (part > 0) {
 #pragma unroll
       for (int j = 0; j < KMAX; ++j) {
-        m_v[rr][j] = tv[j];
-        m_i[rr][j] = ti[j];
+        m_v[((part - 1) * BM + rr) * KMAX + j] = tv[j];
+        m_i[((part - 1) * BM + rr) * KMAX + j] = ti[j];
       }
     }
-    named_bar_sync(1, 32 * kEpiWarps);  // epilogue warps only
-    if (have && staged) {
+    if (mode == 2) fence_proxy_async_shared();  // staged tile -> TMA store
+    named_bar_sync(1, 32 * kEpiWarps);          // epilogue warps only
+    if (have && mode == 2) {
+      if (threadIdx.x == 64) {
+        // rows past T are outside the tensor map and are not written
+        for (int b = 0; b < p.E / 32; ++b)
+          tma_store_2d(&tmL, smem + (size_t)b * (BM * 128), b * 32, (int32_t)row0);
+        bulk_commit();
+      }
+    } else if (have && mode == 1) {
       // the tile's valid logits rows are contiguous in global memory: the
-      // eight warps copy them out in 16-byte chunks, fully coalesced
+      // epilogue warps copy them out in 16-byte chunks, fully coalesced
       const int cpr = p.E / 4;  // chunks per row
       const int nvalid = (int)(p.T - row0 < BM ? p.T - row0 : BM);
       float4* dst = reinterpret_cast<float4*>(p.logits + row0 * p.E);
@@ -243,11 +276,14 @@ __global__ void __launch_bounds__(kThreads, 2)
         dst[c] = *reinterpret_cast<const float4*>(smem + (size_t)r * lstride + cc * 16);
       }
     }
-    if (h == 0) {
-      // the second half's columns are all higher, so inserting its entries
-      // in order keeps lower indices first among equal logits
+    if (part == 0) {
+      // later parts' columns are all higher, so inserting their entries part
+      // by part, in list order, keeps lower indices first among equal logits
+#pragma unroll 1
+      for (int pp = 0; pp < kParts - 1; ++pp)
 #pragma unroll
-      for (int j = 0; j < KMAX; ++j) topk_insert<KMAX>(tv, ti, m_v[rr][j], m_i[rr][j]);
+        for (int j = 0; j < KMAX; ++j)
+          topk_insert<KMAX>(tv, ti, m_v[(pp * BM + rr) * KMAX + j], m_i[(pp * BM + rr) * KMAX + j]);
       if (have && valid) {
         float ex[KMAX];
         float z = 0.f;
@@ -278,8 +314,11 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
       }
     }
+    // the staged tile has been read by the TMA stores before the CTA exits
+    if (have && mode == 2 && threadIdx.x == 64) bulk_wait_read<0>();
   }
   tc_fence_before();
+  __syncwarp();  // role branches diverged single lanes: reconverge before the CTA barrier
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
@@ -291,18 +330,27 @@ __global__ void __launch_bounds__(kThreads, 2)
 }
 
 template <int KMAX>
-cudaError_t run(const RouteArgs& a, const CUtensorMap& mA, const CUtensorMap& mB, const Params& p,
-                cudaStream_t s) {
+cudaError_t run(const RouteArgs& a, const CUtensorMap& mA, const CUtensorMap& mB,
+                const CUtensorMap& mL, Params p, cudaStream_t s) {
+  // the ring also holds, after the GEMM, the staged logits tile and the
+  // partial top-k lists of parts 1-3: grow it when they need more room
+  const size_t stage = (size_t)BM * BK * 2 + (size_t)p.BN * BK * 2;
+  const size_t staged = p.logits_mode == 2 ? (size_t)p.E * 512
+                        : p.logits_mode == 1 ? (size_t)BM * (p.E * 4 + 16) : 0;
+  p.merge_off = (uint32_t)((staged + 15) & ~size_t(15));
+  const size_t need = p.merge_off + (size_t)(kParts - 1) * BM * KMAX * 8;
+  while ((size_t)p.stages * stage < need) ++p.stages;
+  if (p.stages > kMaxStages) return cudaErrorInvalidValue;
   // dynamic shared memory grows with E; raise the kernel's limit when needed
   static size_t attr_bytes = 0;
-  const size_t smem = (size_t)kStages * (BM * BK * 2 + (size_t)p.BN * BK * 2) + 1024;
+  const size_t smem = (size_t)p.stages * stage + 1024;
   if (smem > attr_bytes) {
     cudaError_t e = cudaFuncSetAttribute(route_fused_kernel<KMAX>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     attr_bytes = smem;
   }
-  return launch_pdl(route_fused_kernel<KMAX>, dim3(p.nb), dim3(kThreads), smem, s, mA, mB, p);
+  return launch_pdl(route_fused_kernel<KMAX>, dim3(p.nb), dim3(kThreads), smem, s, mA, mB, mL, p);
 }
 
 }  // namespace
@@ -325,15 +373,27 @@ cudaError_t launch_route_tc(const RouteArgs& a, cudaStream_t s) {
   p.nb = layout_blocks(a.T);
   p.bins = layout_bins(a.E, a.ep);
   p.hist_stride = layout_hist_stride(p.nb);
+  {
+    const size_t stage = (size_t)BM * BK * 2 + (size_t)p.BN * BK * 2;
+    const int kblocks = a.d / BK;
+    int st = (int)(kRingBudget / stage);
+    st = st > kMaxStages ? kMaxStages : st;
+    st = st > kblocks ? kblocks : st;
+    p.stages = st < 1 ? 1 : st;
+  }
   p.map = a.map;
   p.block_hist = a.block_hist;
-  CUtensorMap mA, mB;
+  CUtensorMap mA, mB, mL;
   if (!make_kmajor_map(&mA, a.x, a.T, a.d, BM)) return cudaErrorInvalidValue;
   if (!make_kmajor_map(&mB, a.wrT, p.BN, a.d, p.BN)) return cudaErrorInvalidValue;
-  if (a.k <= 2) return run<2>(a, mA, mB, p, s);
-  if (a.k <= 4) return run<4>(a, mA, mB, p, s);
-  if (a.k <= 8) return run<8>(a, mA, mB, p, s);
-  return run<16>(a, mA, mB, p, s);
+  const bool al16 = (reinterpret_cast<uintptr_t>(a.logits) & 15) == 0;
+  p.logits_mode = (al16 && a.E % 32 == 0) ? 2 : (al16 && a.E % 4 == 0) ? 1 : 0;
+  if (p.logits_mode == 2 && !make_f32_map(&mL, a.logits, a.T, a.E, BM)) p.logits_mode = 1;
+  if (p.logits_mode != 2) mL = mA;  // unused
+  if (a.k <= 2) return run<2>(a, mA, mB, mL, p, s);
+  if (a.k <= 4) return run<4>(a, mA, mB, mL, p, s);
+  if (a.k <= 8) return run<8>(a, mA, mB, mL, p, s);
+  return run<16>(a, mA, mB, mL, p, s);
 }
 
 }  // namespace moe
