@@ -421,25 +421,33 @@ __global__ void __launch_bounds__(ffn_threads<GATHER>(), 1)
       }
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + C::A2_COL + h * HALF;
+      // rounds of 32 columns; the next round's TMEM loads are in flight while
+      // this round is staged and stored, and the accumulator is released as
+      // soon as its last columns are in registers
+      uint32_t r0[16], r1[16];
+      tmem_ld16(taddr, r0);
+      tmem_ld16(taddr + 16, r1);
+      tmem_ld_wait();
 #pragma unroll 1
       for (int c = 0; c < HALF; c += 32) {
-        uint32_t r0[16], r1[16];
-        tmem_ld16(taddr + c, r0);
-        tmem_ld16(taddr + c + 16, r1);
-        tmem_ld_wait();
+        uint32_t pk[16];
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          pk[v] = pack_bf16x2(__uint_as_float(r0[2 * v]), __uint_as_float(r0[2 * v + 1]));
+          pk[8 + v] = pack_bf16x2(__uint_as_float(r1[2 * v]), __uint_as_float(r1[2 * v + 1]));
+        }
+        if (c + 32 < HALF) {
+          tmem_ld16(taddr + c + 32, r0);
+          tmem_ld16(taddr + c + 48, r1);
+        } else {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&a2empty);
+        }
         // this lane's 32 columns -> its staging row (64 bytes)
         uint4* srow = reinterpret_cast<uint4*>(stg + lane * C::STG_ROW);
 #pragma unroll
-        for (int v = 0; v < 2; ++v) {
-          srow[v] = make_uint4(pack_bf16x2(__uint_as_float(r0[8 * v]), __uint_as_float(r0[8 * v + 1])),
-                               pack_bf16x2(__uint_as_float(r0[8 * v + 2]), __uint_as_float(r0[8 * v + 3])),
-                               pack_bf16x2(__uint_as_float(r0[8 * v + 4]), __uint_as_float(r0[8 * v + 5])),
-                               pack_bf16x2(__uint_as_float(r0[8 * v + 6]), __uint_as_float(r0[8 * v + 7])));
-          srow[2 + v] = make_uint4(pack_bf16x2(__uint_as_float(r1[8 * v]), __uint_as_float(r1[8 * v + 1])),
-                                   pack_bf16x2(__uint_as_float(r1[8 * v + 2]), __uint_as_float(r1[8 * v + 3])),
-                                   pack_bf16x2(__uint_as_float(r1[8 * v + 4]), __uint_as_float(r1[8 * v + 5])),
-                                   pack_bf16x2(__uint_as_float(r1[8 * v + 6]), __uint_as_float(r1[8 * v + 7])));
-        }
+        for (int v = 0; v < 4; ++v) srow[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
         __syncwarp();
         // copy-out: 8 rows x 64 bytes per instruction (4 lanes a row)
 #pragma unroll
@@ -450,10 +458,8 @@ __global__ void __launch_bounds__(ffn_threads<GATHER>(), 1)
             *reinterpret_cast<uint4*>(p.y_perm + ((int64_t)ti.row0 + q * 32 + r) * D + h * HALF + c + cc * 8) = v;
         }
         __syncwarp();
+        if (c + 32 < HALF) tmem_ld_wait();
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&a2empty);
     }
   }
 
