@@ -182,12 +182,25 @@ def barrier(world):
 
 
 def max_over_ranks(v: float, world: int) -> float:
+    """The largest of every rank's v (a timing is the slowest rank's)."""
     if world == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_seed(base: int, rank: int) -> int:
+    """Every replica draws its own tokens (the layer shards by tokens)."""
+    return base + rank
+
+
+def job_value(T: int, world: int, ms: float) -> float:
+    """Whole-job routed tokens/s: all ranks' tokens over the slowest rank's
+    step time (weak scaling: T tokens per rank)."""
+    return T * world / (ms * 1e-3)
 
 
 # ----------------------------------------------------------------- our arm
@@ -195,7 +208,7 @@ def run_ours(args, rank, world, local):
     w = W.WORKLOADS[args.config]
     T = w.T
     ep = w.eps[0]
-    seed = args.seed + rank  # every replica works on its own tokens
+    seed = replica_seed(args.seed, rank)
     dev = torch.device("cuda", local)
     x = W.make_x(w, seed, T)
     wr = W.make_router(w, args.seed)
@@ -335,7 +348,7 @@ def run_ours(args, rank, world, local):
         psrc = pk["src"] + " hbm copy"
     result = {
         "metric": METRIC,
-        "value": T * world / (ms * 1e-3),
+        "value": job_value(T, world, ms),
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": args.steps,
@@ -351,7 +364,7 @@ def run_ours(args, rank, world, local):
                    "routed_rows_per_step": T * w.k,
                    "l2": "flushed before every step (256 MB write, outside the step events)",
                    "parallelism": f"replicas x{world} (tokens sharded, no exchange)"},
-        "e2e": {"value": T * world / (e2e_ms * 1e-3), "unit": "tokens/s",
+        "e2e": {"value": job_value(T, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": x.numel() * x.element_size(),
                 "d2h_bytes_per_step": y.numel() * y.element_size()},
         "gpu_launches": launches_per_step(w) * args.steps,
