@@ -195,42 +195,56 @@ struct Vec<float> {
   }
 };
 
-template <typename T>
+template <typename T, int VPT>
 __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ y_perm,
                                                       const int32_t* __restrict__ slot_row,
                                                       const float* __restrict__ gate,
                                                       uint4* __restrict__ y, int64_t Tn, int V,
                                                       int k) {
   pdl_wait();
-  const int64_t n = Tn * V;
+  // thread item i: vectors [i*VPT, i*VPT + VPT) of the flattened [T, V]
+  // output (V % VPT == 0, so they belong to one token); the token's slot
+  // rows and gates are loaded once and every vector load is issued before
+  // any is used
+  const int64_t n = Tn * V / VPT;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
        i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t t = i / V;
-    const int v = (int)(i - t * V);
-    float a[Vec<T>::N];
+    const int64_t t = i * VPT / V;
+    const int v = (int)(i * VPT - t * V);
+    float a[VPT][Vec<T>::N];
 #pragma unroll
-    for (int q = 0; q < Vec<T>::N; ++q) a[q] = 0.f;
+    for (int u = 0; u < VPT; ++u)
+#pragma unroll
+      for (int q = 0; q < Vec<T>::N; ++q) a[u][q] = 0.f;
     int j = 0;
     for (; j + 4 <= k; j += 4) {
-      uint4 q[4];
+      uint4 q[4][VPT];
       float g[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        int64_t row = __ldg(slot_row + t * k + j + u);
+      for (int w = 0; w < 4; ++w) {
+        int64_t row = __ldg(slot_row + t * k + j + w);
         if (row < 0 || row >= Tn * k) row = 0;
-        g[u] = gate ? __ldg(gate + t * k + j + u) : 1.f;
-        q[u] = __ldg(y_perm + row * V + v);
+        g[w] = gate ? __ldg(gate + t * k + j + w) : 1.f;
+#pragma unroll
+        for (int u = 0; u < VPT; ++u) q[w][u] = __ldg(y_perm + row * V + v + u);
       }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) Vec<T>::acc(a, q[u], g[u]);
+      for (int w = 0; w < 4; ++w)
+#pragma unroll
+        for (int u = 0; u < VPT; ++u) Vec<T>::acc(a[u], q[w][u], g[w]);
     }
     for (; j < k; ++j) {
       int64_t row = __ldg(slot_row + t * k + j);
       if (row < 0 || row >= Tn * k) row = 0;
       const float g = gate ? __ldg(gate + t * k + j) : 1.f;
-      Vec<T>::acc(a, __ldg(y_perm + row * V + v), g);
+      uint4 q[VPT];
+#pragma unroll
+      for (int u = 0; u < VPT; ++u) q[u] = __ldg(y_perm + row * V + v + u);
+#pragma unroll
+      for (int u = 0; u < VPT; ++u) Vec<T>::acc(a[u], q[u], g);
     }
-    y[i] = Vec<T>::pack(a);
+#pragma unroll
+    for (int u = 0; u < VPT; ++u) y[i * VPT + u] = Vec<T>::pack(a[u]);
   }
 }
 
@@ -285,15 +299,22 @@ cudaError_t launch_combine(int dtype, const void* y_perm, const int32_t* slot_ro
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t n = T * V;
+  // two vectors per thread when the row allows it: the grid of a
+  // fine-grained batch then fits one wave and no thread waits for a second
+  // round of loads
+  const int vpt = V % 2 == 0 ? 2 : 1;
+  const int64_t n = T * V / vpt;
   const int grid = (int)std::min<int64_t>((n + 255) / 256, (int64_t)sms * 8);
-  if (dtype == MOE_BF16)
-    return launch_pdl(combine_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s,
-                      static_cast<const uint4*>(y_perm), slot_row, gate, static_cast<uint4*>(y), T,
-                      V, k);
-  return launch_pdl(combine_kernel<float>, dim3(grid), dim3(256), 0, s,
-                    static_cast<const uint4*>(y_perm), slot_row, gate, static_cast<uint4*>(y), T, V,
-                    k);
+#define MOE_COMBINE(TY, VP)                                                                           \
+  return launch_pdl(combine_kernel<TY, VP>, dim3(grid), dim3(256), 0, s,                              \
+                    static_cast<const uint4*>(y_perm), slot_row, gate, static_cast<uint4*>(y), T, V, k);
+  if (dtype == MOE_BF16) {
+    if (vpt == 2) { MOE_COMBINE(__nv_bfloat16, 2) }
+    MOE_COMBINE(__nv_bfloat16, 1)
+  }
+  if (vpt == 2) { MOE_COMBINE(float, 2) }
+  MOE_COMBINE(float, 1)
+#undef MOE_COMBINE
 }
 
 }  // namespace moe
