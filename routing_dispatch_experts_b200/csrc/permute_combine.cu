@@ -299,22 +299,19 @@ cudaError_t launch_combine(int dtype, const void* y_perm, const int32_t* slot_ro
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // two vectors per thread when the row allows it: the grid of a
-  // fine-grained batch then fits one wave and no thread waits for a second
-  // round of loads
-  const int vpt = V % 2 == 0 ? 2 : 1;
-  const int64_t n = T * V / vpt;
+  // two vectors per thread (d % 64 == 0, so every row has an even number of
+  // 16-byte vectors): more loads in flight per thread and, for a
+  // fine-grained batch, a grid that fits one wave
+  if (V % 2 != 0) return cudaErrorInvalidValue;
+  const int64_t n = T * V / 2;
   const int grid = (int)std::min<int64_t>((n + 255) / 256, (int64_t)sms * 8);
-#define MOE_COMBINE(TY, VP)                                                                           \
-  return launch_pdl(combine_kernel<TY, VP>, dim3(grid), dim3(256), 0, s,                              \
-                    static_cast<const uint4*>(y_perm), slot_row, gate, static_cast<uint4*>(y), T, V, k);
-  if (dtype == MOE_BF16) {
-    if (vpt == 2) { MOE_COMBINE(__nv_bfloat16, 2) }
-    MOE_COMBINE(__nv_bfloat16, 1)
-  }
-  if (vpt == 2) { MOE_COMBINE(float, 2) }
-  MOE_COMBINE(float, 1)
-#undef MOE_COMBINE
+  if (dtype == MOE_BF16)
+    return launch_pdl(combine_kernel<__nv_bfloat16, 2>, dim3(grid), dim3(256), 0, s,
+                      static_cast<const uint4*>(y_perm), slot_row, gate, static_cast<uint4*>(y), T,
+                      V, k);
+  return launch_pdl(combine_kernel<float, 2>, dim3(grid), dim3(256), 0, s,
+                    static_cast<const uint4*>(y_perm), slot_row, gate, static_cast<uint4*>(y), T, V,
+                    k);
 }
 
 }  // namespace moe
