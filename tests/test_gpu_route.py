@@ -83,3 +83,58 @@ def test_route_zero_tokens():
     l = torch.empty(0, 16, device="cuda")
     _, idx, gate = moe.route(shape, None, None, None, moe.workspace(shape), logits=l)
     assert idx.numel() == 0
+
+
+def _bf16_router_case(T, d, E, k, seed):
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn(T, d, generator=g).bfloat16()
+    wr = (torch.randn(d, E, generator=g) * 0.05).bfloat16()
+    f = 64
+    wg = (torch.randn(E, d, f, generator=g) * 0.02).bfloat16()
+    shape = moe.Shape(T=T, d=d, E=E, k=k, f=f)
+    packed = moe.pack_weights(shape, wr.cuda(), wg.cuda(), wg.cuda(), wg.transpose(1, 2).contiguous().cuda())
+    return x, wr, shape, packed
+
+
+@pytest.mark.parametrize("T,d,E,k", [(1000, 64, 12, 3), (777, 256, 16, 4), (333, 128, 33, 5),
+                                     (1500, 512, 96, 6), (900, 256, 256, 16), (129, 64, 64, 2)])
+def test_bf16_router_logit_layouts_and_ragged_tiles(T, d, E, k):
+    """The tensor-core router for every way its logits tile leaves the SM
+    (TMA tiled stores for E % 32 == 0 -- 2 to 8 boxes --, a coalesced copy
+    for E % 4 == 0, per-thread stores otherwise) and a ragged last tile: the
+    logits match the oracle's double router within the fp32 accumulation
+    bound, and its top-k is bit-exact against the oracle's top-k of the
+    same fp32 logits."""
+    x, wr, shape, packed = _bf16_router_case(T, d, E, k, seed=T + E)
+    ws = moe.workspace(shape)
+    logits, idx, gate = moe.route(shape, x.cuda(), packed, None, ws)
+    moe.check_device_status(ws)
+    ref = oracle.router_logits(x, wr)
+    mag = (x.double().abs() @ wr.double().abs()).numpy()
+    err = np.abs(logits.cpu().double().numpy() - ref)
+    assert (err <= 1e-5 * mag + 1e-6).all()
+    ref_idx, ref_gate = oracle.topk(logits.cpu().double().numpy(), k)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ref_idx)
+    np.testing.assert_allclose(gate.cpu().double().numpy(), ref_gate, rtol=0, atol=1e-6)
+
+
+def test_bf16_router_unaligned_logits_buffer():
+    """A logits buffer that is only 4-byte aligned takes the per-thread
+    store path and gives the same bits as an aligned one."""
+    import ctypes
+    T, d, E, k = 700, 256, 64, 4
+    x, wr, shape, packed = _bf16_router_case(T, d, E, k, seed=5)
+    ws = moe.workspace(shape)
+    dx = x.cuda()
+    l0, i0, g0 = moe.route(shape, dx, packed, None, ws)
+    base = torch.empty(T * E + 4, dtype=torch.float32, device="cuda")
+    l1 = base[1:1 + T * E].view(T, E)
+    i1 = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    g1 = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    s = shape.c
+    p = lambda t: ctypes.c_void_p(t.data_ptr())
+    st = moe.lib().moe_route(ctypes.byref(s), p(dx), p(packed), None, p(l1), p(i1), p(g1), p(ws),
+                             ws.numel(), None)
+    assert st == moe.MOE_OK
+    moe.check_device_status(ws)
+    assert torch.equal(l1, l0) and torch.equal(i1, i0) and torch.equal(g1, g0)
