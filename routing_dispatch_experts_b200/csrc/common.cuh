@@ -152,17 +152,6 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const void* tmap, ui
       : "memory");
 }
 
-// 2-D gather of four rows (one-row-high box): rows[0..3] at column c0, into
-// four consecutive box rows of shared memory, completing on `bar`.
-__device__ __forceinline__ void tma_gather4(void* smem_dst, const void* tmap, uint64_t* bar,
-                                            int32_t c0, const int32_t (&rows)[4]) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes "
-      "[%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(smem_dst)),
-      "l"(tmap), "r"(smem_u32(bar)), "r"(c0), "r"(rows[0]), "r"(rows[1]), "r"(rows[2]), "r"(rows[3])
-      : "memory");
-}
-
 // 2-D tiled store shared -> global (no multicast), tracked by bulk groups;
 // elements of the box outside the tensor are not written
 __device__ __forceinline__ void tma_store_2d(const void* tmap, const void* smem_src, int32_t c0,

@@ -139,12 +139,4 @@ cudaError_t launch_grouped_f32_part(int part, const float* x_perm, const int32_t
   }
 }
 
-cudaError_t launch_grouped_f32(const float* x_perm, const int32_t* offsets, int E, int64_t R,
-                               int d, int f, int blk, const float* wgu, const float* wdT, float* h,
-                               float* y_perm, cudaStream_t s) {
-  cudaError_t err = launch_grouped_f32_part(0, x_perm, offsets, E, R, d, f, blk, wgu, wdT, h, y_perm, s);
-  if (err != cudaSuccess) return err;
-  return launch_grouped_f32_part(1, x_perm, offsets, E, R, d, f, blk, wgu, wdT, h, y_perm, s);
-}
-
 }  // namespace moe

@@ -61,7 +61,6 @@ struct Params {
   int G, K, n_per_group, n_out;
   void* out;
   int64_t ld_out;
-  const float* bias;
   Control* ctl;
 };
 
@@ -534,7 +533,6 @@ cudaError_t run(const GemmArgs& a, cudaStream_t s) {
   p.n_out = a.n_out;
   p.out = a.out;
   p.ld_out = a.ld_out;
-  p.bias = a.bias;
   p.ctl = a.ctl;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);

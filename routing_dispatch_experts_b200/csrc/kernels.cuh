@@ -78,7 +78,7 @@ cudaError_t launch_combine(int dtype, const void* y_perm, const int32_t* slot_ro
 // ---- gemm_tc.cu (bf16, tcgen05)
 // Grouped GEMM  out[r, :] = epilogue(A[r, :] . B_g^T)  for rows r of group g
 // (rows [offsets[g], offsets[g+1])), with B_g rows [g*n_per_group, ...).
-enum Epilogue { kEpiSwiGLU = 0, kEpiBF16 = 1, kEpiLogits = 2 };
+enum Epilogue { kEpiSwiGLU = 0, kEpiBF16 = 1 };
 struct GemmArgs {
   const void* A;           // [rows, K] bf16 row-major
   int64_t rows;            // rows of A (tensor-map extent)
@@ -90,7 +90,6 @@ struct GemmArgs {
   int n_out;               // valid output columns
   void* out;
   int64_t ld_out;          // output row stride in elements
-  const float* bias;       // kEpiLogits only, may be NULL
   Control* ctl;
   // gather mode (gate/up GEMM only): A row r is row gather[r] of A, which
   // then has src_rows rows -- the permute fused into the operand load
@@ -143,9 +142,6 @@ bool ffn_fused_supported(int d, int f);
 cudaError_t launch_ffn_fused(const FfnArgs& a, cudaStream_t s);
 
 // ---- gemm_simt.cu (fp32, CUDA cores)
-cudaError_t launch_grouped_f32(const float* x_perm, const int32_t* offsets, int E, int64_t R,
-                               int d, int f, int blk, const float* wgu, const float* wdT, float* h,
-                               float* y_perm, cudaStream_t s);
 // part 0: gate/up + SwiGLU into h; part 1: down into y_perm
 cudaError_t launch_grouped_f32_part(int part, const float* x_perm, const int32_t* offsets, int E,
                                     int64_t R, int d, int f, int blk, const float* wgu,
