@@ -41,14 +41,14 @@ struct Scratch {
   Control* ctl;
   int32_t* totals;
   uint64_t* status;      // lookback words, zero between calls
-  int32_t* block_hist;   // per-block histogram rows of the fused router
+  uint16_t* block_hist;  // per-block histogram rows of the fused router (16-bit counts)
 };
 
 size_t scratch_bytes(const moe_shape* s) {
   const size_t nb = (size_t)layout_blocks(s->T), bins = (size_t)layout_bins(s->E, s->ep);
   const size_t hs = (size_t)layout_hist_stride((int)nb);
   return align_up(sizeof(Control)) + kTotalsBytes + align_up(nb * bins * 8) +
-         align_up(hs * bins * 4);
+         align_up(hs * bins * 2);
 }
 
 Scratch carve_scratch(const moe_shape* s, void* ws) {
@@ -61,7 +61,7 @@ Scratch carve_scratch(const moe_shape* s, void* ws) {
   p += kTotalsBytes;
   sc.status = reinterpret_cast<uint64_t*>(p);
   p += align_up(nb * bins * 8);
-  sc.block_hist = reinterpret_cast<int32_t*>(p);
+  sc.block_hist = reinterpret_cast<uint16_t*>(p);
   return sc;
 }
 

@@ -41,9 +41,10 @@ constexpr int kMaxBins = 256 + 256 + 2;  // experts + ranks + two stat counters
 
 inline int layout_blocks(int64_t T) { return (int)((T + kTokPerBlock - 1) / kTokPerBlock); }
 inline int layout_bins(int E, int ep) { return E + (ep > 1 ? ep : 0) + 2; }
-// row stride (ints) of block_hist [bins][stride]: nb rounded up to a multiple
-// of 4 so every row starts 16-byte aligned
-inline int layout_hist_stride(int nb) { return (nb + 3) & ~3; }
+// Per-tile histogram counts are 16-bit (at most 128 tokens x k <= 16 per
+// tile and bin).  Row stride (entries) of block_hist [bins][stride]: nb
+// rounded up to a multiple of 8 so every row starts 16-byte aligned.
+inline int layout_hist_stride(int nb) { return (nb + 7) & ~7; }
 
 struct LayoutOut {
   int32_t *counts, *offsets, *row_token, *slot_row;
@@ -65,7 +66,7 @@ cudaError_t launch_layout(const int32_t* idx, int64_t T, int k, int E, int ep, c
 // (stride = layout_hist_stride(nb))
 cudaError_t launch_layout_scatter(const int32_t* idx, int64_t T, int k, int E, int ep,
                                   const RankMap& map, const LayoutOut& out, Control* ctl,
-                                  const int32_t* block_hist, cudaStream_t s);
+                                  const uint16_t* block_hist, cudaStream_t s);
 
 // ---- permute_combine.cu
 // x_perm[r] = x[row_token[r]].  With slot_row non-NULL the copy runs in
@@ -119,7 +120,7 @@ struct RouteArgs {
   bool hist;
   int ep;
   RankMap map;
-  int32_t* block_hist;
+  uint16_t* block_hist;
 };
 cudaError_t launch_route_tc(const RouteArgs& a, cudaStream_t s);
 

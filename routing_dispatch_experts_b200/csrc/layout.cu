@@ -37,7 +37,7 @@ struct Params {
   Control* ctl;
   uint64_t* status;  // [nb][bins] lookback words (histogram-kernel mode)
   int32_t* totals;   // [bins]   (histogram-kernel mode)
-  const int32_t* block_hist;  // [bins][hist_stride] per-block counts (fused-router mode)
+  const uint16_t* block_hist;  // [bins][hist_stride] per-block counts (fused-router mode)
   int hist_stride;
   LayoutOut out;
 };
@@ -124,26 +124,28 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(const __
   if (tid == 0) s_ok = *reinterpret_cast<volatile uint32_t*>(&p.ctl->status) == MOE_OK;
   if (p.block_hist) {
     // fused-router mode: the kernel boundary already ordered every block's
-    // histogram, so sum them directly.  block_hist is [bins][stride]; one
-    // thread per bin reads its row with 16-byte loads, 16 in flight at a
-    // time, and keeps the total and this block's exclusive prefix (integer
-    // sums: exact)
+    // histogram, so sum them directly.  block_hist is [bins][stride] of
+    // 16-bit counts; one thread per bin reads its row with 16-byte loads (8
+    // blocks each), 16 in flight at a time -- one round for up to 128
+    // blocks -- and keeps the total and this block's exclusive prefix
+    // (integer sums: exact)
     const int hs = p.hist_stride;
     for (int bin = tid; bin < p.bins; bin += kLayoutThreads) {
       const int4* row = reinterpret_cast<const int4*>(p.block_hist + (size_t)bin * hs);
       int tot = 0, pre = 0;
-      for (int q4 = 0; q4 * 4 < p.nb; q4 += 16) {
+      for (int q8 = 0; q8 * 8 < p.nb; q8 += 16) {
         int4 v[16];
 #pragma unroll
         for (int u = 0; u < 16; ++u)
-          v[u] = (q4 + u) * 4 < p.nb ? __ldg(row + q4 + u) : make_int4(0, 0, 0, 0);
+          v[u] = (q8 + u) * 8 < p.nb ? __ldg(row + q8 + u) : make_int4(0, 0, 0, 0);
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
-          const int q = (q4 + u) * 4;
-          const int a[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+          const int q = (q8 + u) * 8;
+          const uint32_t w[4] = {(uint32_t)v[u].x, (uint32_t)v[u].y, (uint32_t)v[u].z, (uint32_t)v[u].w};
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const int x = q + c < p.nb ? a[c] : 0;  // entries past nb are padding
+          for (int c = 0; c < 8; ++c) {
+            const int cnt = (int)((w[c >> 1] >> (16 * (c & 1))) & 0xFFFFu);
+            const int x = q + c < p.nb ? cnt : 0;  // entries past nb are padding
             tot += x;
             pre += q + c < b ? x : 0;
           }
@@ -381,7 +383,7 @@ cudaError_t launch_layout(const int32_t* idx, int64_t T, int k, int E, int ep, c
 
 cudaError_t launch_layout_scatter(const int32_t* idx, int64_t T, int k, int E, int ep,
                                   const RankMap& map, const LayoutOut& out, Control* ctl,
-                                  const int32_t* block_hist, cudaStream_t s) {
+                                  const uint16_t* block_hist, cudaStream_t s) {
   if (T == 0) return empty_layout(E, ep, out, s);
   Params p = make_params(idx, T, k, E, ep, map, out, ctl, nullptr, nullptr, -1, 0);
   p.block_hist = block_hist;

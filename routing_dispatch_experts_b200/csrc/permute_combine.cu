@@ -196,7 +196,7 @@ struct Vec<float> {
 };
 
 template <typename T, int VPT>
-__global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ y_perm,
+__global__ void __launch_bounds__(128) combine_kernel(const uint4* __restrict__ y_perm,
                                                       const int32_t* __restrict__ slot_row,
                                                       const float* __restrict__ gate,
                                                       uint4* __restrict__ y, int64_t Tn, int V,
@@ -302,14 +302,17 @@ cudaError_t launch_combine(int dtype, const void* y_perm, const int32_t* slot_ro
   // two vectors per thread (d % 64 == 0, so every row has an even number of
   // 16-byte vectors): more loads in flight per thread and, for a
   // fine-grained batch, a grid that fits one wave
+  // 128-thread CTAs (one warp per SM sub-partition): launched early, they fit
+  // beside the preceding expert-FFN CTA, whose warps leave about one warp's
+  // worth of registers free on each sub-partition
   if (V % 2 != 0) return cudaErrorInvalidValue;
   const int64_t n = T * V / 2;
-  const int grid = (int)std::min<int64_t>((n + 255) / 256, (int64_t)sms * 8);
+  const int grid = (int)std::min<int64_t>((n + 127) / 128, (int64_t)sms * 16);
   if (dtype == MOE_BF16)
-    return launch_pdl(combine_kernel<__nv_bfloat16, 2>, dim3(grid), dim3(256), 0, s,
+    return launch_pdl(combine_kernel<__nv_bfloat16, 2>, dim3(grid), dim3(128), 0, s,
                       static_cast<const uint4*>(y_perm), slot_row, gate, static_cast<uint4*>(y), T,
                       V, k);
-  return launch_pdl(combine_kernel<float, 2>, dim3(grid), dim3(256), 0, s,
+  return launch_pdl(combine_kernel<float, 2>, dim3(grid), dim3(128), 0, s,
                     static_cast<const uint4*>(y_perm), slot_row, gate, static_cast<uint4*>(y), T, V,
                     k);
 }

@@ -57,7 +57,7 @@ struct Params {
   int logits_mode;
   uint32_t merge_off;  // shared-memory offset of the partial top-k lists
   RankMap map;
-  int32_t* block_hist;
+  uint16_t* block_hist;
 };
 
 // insert (v, e) into the descending list (tv, ti); e arrives in increasing
@@ -77,8 +77,12 @@ __device__ __forceinline__ void topk_insert(float (&tv)[KMAX], int (&ti)[KMAX], 
   }
 }
 
+// At most 102 registers a thread (two CTAs' worth): the layout scatter that
+// follows is launched early and must fit on the SM beside this kernel's CTA
+// (registers are split per SM sub-partition); when it could not, the forward
+// measured 4.5 us slower.
 template <int KMAX>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     route_fused_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                        const __grid_constant__ CUtensorMap tmL, const __grid_constant__ Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -326,7 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (p.hist && tile_ok)  // bin-major [bins][stride], so the scatter reads rows of blocks
     for (int bin = threadIdx.x; bin < p.bins; bin += kThreads)
-      p.block_hist[(size_t)bin * p.hist_stride + b] = hist[bin];
+      p.block_hist[(size_t)bin * p.hist_stride + b] = (uint16_t)hist[bin];
 }
 
 template <int KMAX>
