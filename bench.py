@@ -192,6 +192,15 @@ def max_over_ranks(v: float, world: int) -> float:
     return float(t.item())
 
 
+def config_of(w: W.Workload, world: int) -> dict:
+    """The workload a bench line measures (the same for both arms)."""
+    return {"workload": f"MoE layer config {w.cfg} ({w.name}): {w.describe()}",
+            "T": w.T, "d": w.d, "E": w.E, "f": w.f, "k": w.k, "ep": w.eps[0],
+            "routed_rows_per_step": w.T * w.k,
+            "l2": "flushed before every step (256 MB write, outside the step events)",
+            "parallelism": f"replicas x{world} (tokens sharded, no exchange)"}
+
+
 def replica_seed(base: int, rank: int) -> int:
     """Every replica draws its own tokens (the layer shards by tokens)."""
     return base + rank
@@ -393,11 +402,7 @@ def run_ours(args, rank, world, local):
         "vs_baseline": None,
         "dtype": "bf16" if w.dtype == "bf16" else "f32",
         "data": "synthetic",
-        "config": {"workload": f"MoE layer config {w.cfg} ({w.name}): {w.describe()}",
-                   "T": T, "d": w.d, "E": w.E, "f": w.f, "k": w.k, "ep": ep,
-                   "routed_rows_per_step": T * w.k,
-                   "l2": "flushed before every step (256 MB write, outside the step events)",
-                   "parallelism": f"replicas x{world} (tokens sharded, no exchange)"},
+        "config": config_of(w, world),
         "e2e": {"value": job_value(T, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": x.numel() * x.element_size(),
                 "d2h_bytes_per_step": y.numel() * y.element_size(),
@@ -455,7 +460,7 @@ def run_reference(args, rank, world):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": w.T / cb["value"] * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": f"MoE layer config {w.cfg} ({w.name}): {w.describe()}"},
+            "config": config_of(w, world),
             "cpu_baseline": cb,
             "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
