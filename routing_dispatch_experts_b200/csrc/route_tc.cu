@@ -35,7 +35,8 @@ namespace {
 
 constexpr int BM = 128, BK = 64;
 // operand ring depth: as many k-blocks in flight as fit (all of them for
-// d = 256), so a CTA streaming a tall x tile keeps enough bytes in flight
+// d = 256), so a CTA streaming a tall x tile keeps enough bytes in flight;
+// half of it when two CTAs share an SM
 constexpr int kMaxStages = 8;
 constexpr size_t kRingBudget = 200u * 1024u;
 constexpr int kEpiWarps = 8;                     // kParts per TMEM lane quadrant (16 measured slower)
@@ -378,9 +379,17 @@ cudaError_t launch_route_tc(const RouteArgs& a, cudaStream_t s) {
   p.bins = layout_bins(a.E, a.ep);
   p.hist_stride = layout_hist_stride(p.nb);
   {
+    // More tiles than SMs: a half-size ring lets two CTAs share an SM, so
+    // every tile is resident at once instead of a second wave of tiles
+    // starting when the first has finished (T = 32768, d = 4096, E = 128:
+    // 74 us instead of 86 us; the bytes in flight per SM are unchanged).
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const size_t budget = p.nb > sms ? kRingBudget / 2 : kRingBudget;
     const size_t stage = (size_t)BM * BK * 2 + (size_t)p.BN * BK * 2;
     const int kblocks = a.d / BK;
-    int st = (int)(kRingBudget / stage);
+    int st = (int)(budget / stage);
     st = st > kMaxStages ? kMaxStages : st;
     st = st > kblocks ? kblocks : st;
     p.stages = st < 1 ? 1 : st;
