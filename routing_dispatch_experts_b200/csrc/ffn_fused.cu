@@ -475,13 +475,8 @@ __global__ void __launch_bounds__(ffn_threads<GATHER>(), 1)
 template <int F, int D, bool GATHER>
 cudaError_t run(const FfnArgs& a, cudaStream_t s) {
   using C = Cfg<F, D>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(ffn_fused_kernel<F, D, GATHER>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  cudaError_t e = set_smem_limit((const void*)ffn_fused_kernel<F, D, GATHER>, C::SMEM);
+  if (e != cudaSuccess) return e;
   CUtensorMap mA, mB1, mB2;
   // gather mode reads A with cp.async; its tensor map is built but unused
   if (!make_kmajor_map(&mA, a.A, GATHER ? a.src_rows : a.rows, D, BM)) return cudaErrorInvalidValue;

@@ -509,14 +509,9 @@ namespace {
 
 template <int BN, int EPI, bool GATHER, bool STAGED>
 cudaError_t run(const GemmArgs& a, cudaStream_t s) {
-  static bool attr_set = false;
   constexpr size_t smem = smem_bytes_for<BN, EPI, STAGED, GATHER>();
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI, GATHER, STAGED>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  cudaError_t e = set_smem_limit((const void*)gemm_tc_kernel<BN, EPI, GATHER, STAGED>, smem);
+  if (e != cudaSuccess) return e;
   CUtensorMap mA, mB;
   // gather mode reads A with cp.async; its tensor map is built but unused
   if (!make_kmajor_map(&mA, a.A, GATHER ? a.src_rows : a.rows, a.K, BM)) return cudaErrorInvalidValue;

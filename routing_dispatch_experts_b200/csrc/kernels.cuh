@@ -1,9 +1,41 @@
 // kernels.cuh - launchers shared between the kernel files and the C ABI.
 #pragma once
 
+#include <mutex>
+#include <vector>
+
 #include "common.cuh"
 
 namespace moe {
+
+// Raise `kernel`'s dynamic shared-memory limit to at least `bytes` on the
+// current device.  The limit belongs to each device's context, so it is
+// recorded per (kernel, device); calls from several host threads are
+// serialised.
+inline cudaError_t set_smem_limit(const void* kernel, size_t bytes) {
+  struct Done {
+    const void* fn;
+    int dev;
+    size_t bytes;
+  };
+  static std::mutex mu;
+  static std::vector<Done> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  Done* rec = nullptr;
+  for (Done& d : done)
+    if (d.fn == kernel && d.dev == dev) rec = &d;
+  if (rec && rec->bytes >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e != cudaSuccess) return e;
+  if (rec)
+    rec->bytes = bytes;
+  else
+    done.push_back({kernel, dev, bytes});
+  return cudaSuccess;
+}
 
 // Launch with programmatic stream serialization (see common.cuh).
 template <typename... KArgs, typename... Args>

@@ -269,15 +269,12 @@ cudaError_t launch_permute(const void* x, const int32_t* row_token, const int32_
                       static_cast<const uint4*>(x), row_token, static_cast<uint4*>(x_perm), R, T, V);
   }
   const int smem = kPermStages * (int)kPermStageBytes;
-  static bool attr_set[2] = {false, false};
   const bool by_token = slot_row != nullptr;
-  if (!attr_set[by_token]) {
-    cudaError_t e = by_token ? cudaFuncSetAttribute(permute_kernel<true>,
-                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, smem)
-                             : cudaFuncSetAttribute(permute_kernel<false>,
-                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  {
+    cudaError_t e = set_smem_limit(by_token ? (const void*)permute_kernel<true>
+                                            : (const void*)permute_kernel<false>,
+                                   (size_t)smem);
     if (e != cudaSuccess) return e;
-    attr_set[by_token] = true;
   }
   const int rps = (int)std::min<uint32_t>(32u, kPermStageBytes / row_bytes);
   const int64_t ngroups = ((by_token ? T : R) + rps - 1) / rps;

@@ -347,14 +347,9 @@ cudaError_t run(const RouteArgs& a, const CUtensorMap& mA, const CUtensorMap& mB
   while ((size_t)p.stages * stage < need) ++p.stages;
   if (p.stages > kMaxStages) return cudaErrorInvalidValue;
   // dynamic shared memory grows with E; raise the kernel's limit when needed
-  static size_t attr_bytes = 0;
   const size_t smem = (size_t)p.stages * stage + 1024;
-  if (smem > attr_bytes) {
-    cudaError_t e = cudaFuncSetAttribute(route_fused_kernel<KMAX>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    attr_bytes = smem;
-  }
+  cudaError_t e = set_smem_limit((const void*)route_fused_kernel<KMAX>, smem);
+  if (e != cudaSuccess) return e;
   return launch_pdl(route_fused_kernel<KMAX>, dim3(p.nb), dim3(kThreads), smem, s, mA, mB, mL, p);
 }
 
