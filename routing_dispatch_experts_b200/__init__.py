@@ -166,8 +166,32 @@ def _stream(stream=None):
 
 
 def _need(t, dtype, shape, name):
+    if t is None:
+        raise ValueError(f"{name}: required")
     if t.dtype != dtype or tuple(t.shape) != tuple(shape):
         raise ValueError(f"{name}: expected {dtype} {tuple(shape)}, got {t.dtype} {tuple(t.shape)}")
+
+
+def _need_n(t, dtype, n, name):
+    """dtype and element count of an index or gate array (any shape)."""
+    if t is None:
+        raise ValueError(f"{name}: required")
+    if t.dtype != dtype or t.numel() != n:
+        raise ValueError(f"{name}: expected {dtype} with {n} elements, "
+                         f"got {t.dtype} {tuple(t.shape)}")
+
+
+def _need_packed(shape: "Shape", packed):
+    """The packed weights buffer: uint8, at least the size pack_weights makes."""
+    n = packed_weights_size(shape)
+    if packed is None or packed.dtype != torch.uint8 or packed.numel() < n:
+        got = "None" if packed is None else f"{packed.dtype} x {packed.numel()}"
+        raise ValueError(f"packed: expected uint8 of at least {n} bytes (pack_weights), got {got}")
+
+
+def _need_bias(shape: "Shape", bias):
+    if bias is not None:
+        _need(bias, torch.float32, (shape.E,), "bias")
 
 
 def scratch_size(shape: Shape) -> int:
@@ -224,11 +248,11 @@ def route(shape: Shape, x, packed, bias, ws, logits=None, stream=None):
     dev = ws.device
     if x is not None:
         _need(x, shape.dtype, (shape.T, shape.d), "x")
+        _need_packed(shape, packed)
         logits = torch.empty((shape.T, shape.E), dtype=torch.float32, device=dev)
     else:
         _need(logits, torch.float32, (shape.T, shape.E), "logits")
-    if bias is not None:
-        _need(bias, torch.float32, (shape.E,), "bias")
+    _need_bias(shape, bias)
     idx = torch.empty((shape.T, shape.k), dtype=torch.int32, device=dev)
     gate = torch.empty((shape.T, shape.k), dtype=torch.float32, device=dev)
     s = shape.c
@@ -289,6 +313,7 @@ def dispatch_layout(shape: Shape, topk_idx, ws, expert_rank=None, stream=None) -
 
 def debug_dispatch_layout_stall(shape: Shape, topk_idx, ws, stall_block: int, wait_limit_ns: int,
                                 expert_rank=None, stream=None) -> dict:
+    _need(topk_idx, torch.int32, (shape.T, shape.k), "topk_idx")
     out = _layout_tensors(shape, ws.device)
     lay = _c_layout(out)
     s = shape.c
@@ -315,6 +340,7 @@ def dispatch_layout_static(shape: Shape, topk_idx, expert_rank=None, stream=None
 
 def permute(shape: Shape, x, row_token, stream=None):
     _need(x, shape.dtype, (shape.T, shape.d), "x")
+    _need_n(row_token, torch.int32, shape.R, "row_token")
     x_perm = torch.empty((shape.R, shape.d), dtype=shape.dtype, device=x.device)
     s = shape.c
     _check(lib().moe_permute(ctypes.byref(s), _p(x), _p(row_token), _p(x_perm), _stream(stream)),
@@ -325,6 +351,7 @@ def permute(shape: Shape, x, row_token, stream=None):
 def permute_by_token(shape: Shape, x, slot_row, stream=None):
     """moe_permute_by_token: x_perm via a token-order copy (x read once)."""
     _need(x, shape.dtype, (shape.T, shape.d), "x")
+    _need_n(slot_row, torch.int32, shape.R, "slot_row")
     x_perm = torch.empty((shape.R, shape.d), dtype=shape.dtype, device=x.device)
     s = shape.c
     _check(lib().moe_permute_by_token(ctypes.byref(s), _p(x), _p(slot_row), _p(x_perm),
@@ -335,6 +362,8 @@ def permute_by_token(shape: Shape, x, slot_row, stream=None):
 def grouped_swiglu(shape: Shape, x_perm, expert_offsets, packed, ws, stream=None):
     """moe_grouped_swiglu: returns (h [R,f], y_perm [R,d])."""
     _need(x_perm, shape.dtype, (shape.R, shape.d), "x_perm")
+    _need_n(expert_offsets, torch.int32, shape.E + 1, "expert_offsets")
+    _need_packed(shape, packed)
     h = torch.empty((shape.R, shape.f), dtype=shape.dtype, device=x_perm.device)
     y_perm = torch.empty((shape.R, shape.d), dtype=shape.dtype, device=x_perm.device)
     s = shape.c
@@ -347,6 +376,9 @@ def grouped_swiglu(shape: Shape, x_perm, expert_offsets, packed, ws, stream=None
 def grouped_swiglu_gather(shape: Shape, x, row_token, expert_offsets, packed, ws, stream=None):
     """moe_grouped_swiglu_gather: (h, y_perm) with rows gathered from x."""
     _need(x, shape.dtype, (shape.T, shape.d), "x")
+    _need_n(row_token, torch.int32, shape.R, "row_token")
+    _need_n(expert_offsets, torch.int32, shape.E + 1, "expert_offsets")
+    _need_packed(shape, packed)
     h = torch.empty((shape.R, shape.f), dtype=shape.dtype, device=x.device)
     y_perm = torch.empty((shape.R, shape.d), dtype=shape.dtype, device=x.device)
     s = shape.c
@@ -359,6 +391,9 @@ def grouped_swiglu_gather(shape: Shape, x, row_token, expert_offsets, packed, ws
 
 def combine(shape: Shape, y_perm, slot_row, topk_gate=None, stream=None):
     _need(y_perm, shape.dtype, (shape.R, shape.d), "y_perm")
+    _need_n(slot_row, torch.int32, shape.R, "slot_row")
+    if topk_gate is not None:
+        _need_n(topk_gate, torch.float32, shape.R, "topk_gate")
     y = torch.empty((shape.T, shape.d), dtype=shape.dtype, device=y_perm.device)
     s = shape.c
     _check(lib().moe_combine(ctypes.byref(s), _p(y_perm), _p(slot_row), _p(topk_gate), _p(y),
@@ -370,6 +405,7 @@ class ForwardBuffers:
     """Caller-owned intermediates of moe_forward, readable after the call."""
 
     def __init__(self, shape: Shape, device="cuda"):
+        self.shape = shape
         R = shape.R
         self.logits = torch.empty((shape.T, shape.E), dtype=torch.float32, device=device)
         self.topk_idx = torch.empty((shape.T, shape.k), dtype=torch.int32, device=device)
@@ -386,10 +422,20 @@ class ForwardBuffers:
                                    _p(self.y_perm))
 
 
+def _forward_args(shape: Shape, x, packed, bias, y, buffers):
+    _need(x, shape.dtype, (shape.T, shape.d), "x")
+    _need_packed(shape, packed)
+    _need_bias(shape, bias)
+    if y is not None:
+        _need(y, shape.dtype, (shape.T, shape.d), "y")
+    if buffers is not None and buffers.shape != shape:
+        raise ValueError(f"buffers: made for {buffers.shape}, not {shape}")
+
+
 def forward(shape: Shape, x, packed, bias, ws, expert_rank=None, y=None,
             buffers: Optional[ForwardBuffers] = None, stream=None):
     """moe_forward: the whole layer; returns y [T, d]."""
-    _need(x, shape.dtype, (shape.T, shape.d), "x")
+    _forward_args(shape, x, packed, bias, y, buffers)
     if y is None:
         y = torch.empty((shape.T, shape.d), dtype=shape.dtype, device=x.device)
     s = shape.c
@@ -405,7 +451,7 @@ def forward_timed(shape: Shape, x, packed, bias, ws, events, expert_rank=None, y
                   buffers: Optional[ForwardBuffers] = None, stream=None):
     """moe_forward_timed: moe_forward recording `events` (7 torch.cuda.Event
     with timing) around its stages (FORWARD_STAGES)."""
-    _need(x, shape.dtype, (shape.T, shape.d), "x")
+    _forward_args(shape, x, packed, bias, y, buffers)
     if len(events) != len(FORWARD_STAGES) + 1:
         raise ValueError("need one event per stage plus one")
     if y is None:
