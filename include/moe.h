@@ -234,6 +234,8 @@ MOE_API moe_status moe_dispatch_layout(const moe_shape* shape, const int32_t* to
  * Permute (gather): x_perm[r] = x[row_token[r]] for r < T*k, whole rows,
  * moved by TMA bulk copies staged through shared memory.
  *  x [T, d], x_perm [T*k, d] (dtype); row_token [T*k] int32.
+ * A row_token entry outside [0, T) is read as 0 (wrong values, no access
+ * outside x); moe_dispatch_layout never produces one.
  */
 MOE_API moe_status moe_permute(const moe_shape* shape, const void* x,
                        const int32_t* row_token, void* x_perm,
@@ -245,6 +247,7 @@ MOE_API moe_status moe_permute(const moe_shape* shape, const void* x,
  * moe_dispatch_layout).  Equal output to moe_permute; it moves |x| + |x_perm|
  * bytes through DRAM even when x is much larger than L2, where the gather
  * re-reads each row of x once per expert that picks it.
+ * A slot_row entry outside [0, T*k) is read as 0 (no access outside x_perm).
  */
 MOE_API moe_status moe_permute_by_token(const moe_shape* shape, const void* x,
                                         const int32_t* slot_row, void* x_perm,
@@ -257,6 +260,9 @@ MOE_API moe_status moe_permute_by_token(const moe_shape* shape, const void* x,
  * for expert e owning row r (expert_offsets [E+1], device, as produced by
  * moe_dispatch_layout).  bf16: tcgen05 tensor cores, fp32 accumulation in
  * tensor memory, h and y_perm rounded to bf16.  fp32: CUDA-core FMA.
+ * Offsets are clamped to [0, T*k] and a negative group size counts as
+ * empty, so a malformed offset array gives wrong rows but no access outside
+ * x_perm, h or y_perm.
  *  ws, ws_bytes  scratch workspace (moe_scratch_size)
  */
 MOE_API moe_status moe_grouped_swiglu(const moe_shape* shape, const void* x_perm,
@@ -271,7 +277,8 @@ MOE_API moe_status moe_grouped_swiglu(const moe_shape* shape, const void* x_perm
  * into shared memory (cp.async, 16 bytes per lane), so x_perm is never
  * written or read.
  *  x [T, d]; row_token [T*k] (moe_dispatch_layout); other arguments as in
- *  moe_grouped_swiglu.  MOE_ERR_UNSUPPORTED for fp32.
+ *  moe_grouped_swiglu.  MOE_ERR_UNSUPPORTED for fp32.  A row_token entry
+ *  outside [0, T) is read as 0.
  */
 MOE_API moe_status moe_grouped_swiglu_gather(const moe_shape* shape, const void* x,
                                              const int32_t* row_token,
@@ -285,7 +292,7 @@ MOE_API moe_status moe_grouped_swiglu_gather(const moe_shape* shape, const void*
  *   y[t] = sum_{j<k} gate[t,j] * y_perm[slot_row[t*k+j]]
  * summed in fp32 in ascending j, rounded once to the dtype.
  *  y_perm [T*k, d]; slot_row [T*k] int32; topk_gate [T, k] fp32 or NULL for
- *  unit gates; y [T, d].
+ *  unit gates; y [T, d].  A slot_row entry outside [0, T*k) is read as 0.
  */
 MOE_API moe_status moe_combine(const moe_shape* shape, const void* y_perm,
                        const int32_t* slot_row, const float* topk_gate,

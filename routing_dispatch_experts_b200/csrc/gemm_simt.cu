@@ -25,21 +25,26 @@ constexpr int TM = 64, TN = 64, TK = 16;
 template <bool SWIGLU>
 __global__ void __launch_bounds__(256) grouped_f32_kernel(const float* __restrict__ A,
                                                           const int32_t* __restrict__ offsets,
-                                                          int E, int K, int N,
+                                                          int E, int rows, int K, int N,
                                                           const float* __restrict__ W, int blk,
                                                           int64_t w_group_stride,
                                                           float* __restrict__ out) {
   __shared__ int tile_off[257];
+  __shared__ int s_off[257];
   __shared__ float sA[TK][TM + 4];
   __shared__ float sG[TK][TN + 4];
   __shared__ float sU[SWIGLU ? TK : 1][TN + 4];
   const int tid = threadIdx.x;
   pdl_wait();
+  // offsets clamped to [0, rows] and a negative group size read as empty: a
+  // malformed offset array can never move a load or a store outside A / out
+  for (int g = tid; g <= E; g += 256) s_off[g] = min(max(__ldg(offsets + g), 0), rows);
+  __syncthreads();
   if (tid < 32) {
     int carry = 0;
     for (int g0 = 0; g0 < E; g0 += 32) {
       const int g = g0 + tid;
-      const int v = g < E ? (__ldg(offsets + g + 1) - __ldg(offsets + g) + TM - 1) / TM : 0;
+      const int v = g < E ? (max(s_off[g + 1] - s_off[g], 0) + TM - 1) / TM : 0;
       int incl = v;
       for (int off = 1; off < 32; off <<= 1) {
         const int o = __shfl_up_sync(0xffffffffu, incl, off);
@@ -61,8 +66,8 @@ __global__ void __launch_bounds__(256) grouped_f32_kernel(const float* __restric
       if (tile_off[mid] > mt) hi = mid; else lo = mid + 1;
     }
     const int e = lo - 1;
-    const int row0 = __ldg(offsets + e) + (mt - tile_off[e]) * TM;
-    const int row_end = __ldg(offsets + e + 1);
+    const int row0 = s_off[e] + (mt - tile_off[e]) * TM;
+    const int row_end = s_off[e + 1];
     const float* We = W + (int64_t)e * w_group_stride;
     const int tx = tid & 15, ty = tid >> 4;  // 16 x 16 threads, 4 x 4 outputs each
     float accg[4][4] = {}, accu[4][4] = {};
@@ -130,12 +135,12 @@ cudaError_t launch_grouped_f32_part(int part, const float* x_perm, const int32_t
   if (part == 0) {
     const int grid1 = (int)std::min<int64_t>(mt_max * (f / TN), (int64_t)sms * 8);
     return launch_pdl(grouped_f32_kernel<true>, dim3(grid1), dim3(256), 0, s, x_perm, offsets, E,
-                      d, f, wgu, blk, (int64_t)2 * f * d, h);
+                      (int)R, d, f, wgu, blk, (int64_t)2 * f * d, h);
   } else {
     const int grid2 = (int)std::min<int64_t>(mt_max * (d / TN), (int64_t)sms * 8);
     return launch_pdl(grouped_f32_kernel<false>, dim3(grid2), dim3(256), 0, s,
-                      static_cast<const float*>(h), offsets, E, f, d, wdT, blk, (int64_t)d * f,
-                      y_perm);
+                      static_cast<const float*>(h), offsets, E, (int)R, f, d, wdT, blk,
+                      (int64_t)d * f, y_perm);
   }
 }
 
