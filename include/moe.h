@@ -357,6 +357,29 @@ MOE_API moe_status moe_forward_timed(const moe_shape* shape, const void* x,
                                      moe_stream_t stream);
 
 /*
+ * The layer below the router on a routing the caller supplies: the
+ * dispatch layout of topk_idx, then permute, expert FFN and combine with
+ * topk_gate, as in moe_forward (same kernels, same results for the same
+ * routing).  It replays a recorded routing table, which applications that
+ * depend on specific experts need once routing is not reproducible ("MoE
+ * Pretraining: Parallelism Layout Changes the Model, Not Quality",
+ * Practical Implications: routing replay).  No logits are computed and the
+ * router block of `packed` is not read.
+ *  topk_idx [T, k] int32 (device): experts in [0, E); an entry outside
+ *    that range sets MOE_ERR_DEVICE_INDEX in the device status word, as in
+ *    moe_dispatch_layout.
+ *  topk_gate [T, k] fp32 (device) or NULL for unit gates.
+ *  Other arguments as in moe_forward; the logits, topk_idx and topk_gate
+ *  members of `buffers` are not used.
+ */
+MOE_API moe_status moe_forward_routed(const moe_shape* shape, const void* x,
+                                      const void* packed, const int32_t* topk_idx,
+                                      const float* topk_gate,
+                                      const int32_t* expert_rank_host, void* y,
+                                      const moe_forward_buffers* buffers, void* ws,
+                                      size_t ws_bytes, moe_stream_t stream);
+
+/*
  * Synchronise `stream`, read the device status word of workspace `ws`
  * (MOE_OK, MOE_ERR_DEVICE_TIMEOUT or MOE_ERR_DEVICE_INDEX) into *out and
  * reset it to MOE_OK.  Returns MOE_ERR_CUDA if the stream reports an error.

@@ -75,7 +75,7 @@ SYMBOLS = ("moe_status_string", "moe_scratch_size", "moe_forward_workspace_size"
            "moe_workspace_init", "moe_packed_weights_size", "moe_pack_weights", "moe_route",
            "moe_dispatch_layout", "moe_permute", "moe_permute_by_token", "moe_grouped_swiglu",
            "moe_grouped_swiglu_gather", "moe_combine", "moe_forward", "moe_forward_timed",
-           "moe_get_device_status", "moe_debug_dispatch_layout_stall",
+           "moe_forward_routed", "moe_get_device_status", "moe_debug_dispatch_layout_stall",
            "moe_dispatch_layout_static")
 FORWARD_STAGES = ("route", "layout", "permute", "gate_up", "down", "combine")
 
@@ -110,6 +110,8 @@ def lib() -> ctypes.CDLL:
                                   ctypes.c_int),
             "moe_forward": ([S, P, P, P, P, P, ctypes.POINTER(moe_forward_buffers), P,
                              ctypes.c_size_t, P], ctypes.c_int),
+            "moe_forward_routed": ([S, P, P, P, P, P, P, ctypes.POINTER(moe_forward_buffers), P,
+                                    ctypes.c_size_t, P], ctypes.c_int),
             "moe_get_device_status": ([P, P, ctypes.POINTER(ctypes.c_int)], ctypes.c_int),
             "moe_debug_dispatch_layout_stall": ([S, P, P, ctypes.POINTER(moe_layout), P,
                                                  ctypes.c_size_t, ctypes.c_int32, ctypes.c_int64, P],
@@ -463,6 +465,26 @@ def forward_timed(shape: Shape, x, packed, bias, ws, events, expert_rank=None, y
                                    _host_map(shape, expert_rank), _p(y),
                                    ctypes.byref(b) if b is not None else None, _p(ws), ws.numel(),
                                    ev, _stream(stream)), "moe_forward_timed")
+    return y
+
+
+def forward_routed(shape: Shape, x, packed, topk_idx, topk_gate, ws, expert_rank=None, y=None,
+                   buffers: Optional[ForwardBuffers] = None, stream=None):
+    """moe_forward_routed: the layer below the router on a given routing
+    (topk_idx [T,k] int32, topk_gate [T,k] fp32 or None for unit gates);
+    returns y [T, d]."""
+    _forward_args(shape, x, packed, None, y, buffers)
+    _need(topk_idx, torch.int32, (shape.T, shape.k), "topk_idx")
+    if topk_gate is not None:
+        _need(topk_gate, torch.float32, (shape.T, shape.k), "topk_gate")
+    if y is None:
+        y = torch.empty((shape.T, shape.d), dtype=shape.dtype, device=x.device)
+    s = shape.c
+    b = buffers.c if buffers is not None else None
+    _check(lib().moe_forward_routed(ctypes.byref(s), _p(x), _p(packed), _p(topk_idx),
+                                    _p(topk_gate), _host_map(shape, expert_rank), _p(y),
+                                    ctypes.byref(b) if b is not None else None, _p(ws),
+                                    ws.numel(), _stream(stream)), "moe_forward_routed")
     return y
 
 

@@ -318,9 +318,13 @@ bool gather_fits(const moe_shape* s) {
   return s->dtype == MOE_BF16 && s->T * (int64_t)s->d * 2 <= kGatherMaxBytes;
 }
 
+// The forward; with `routed` the caller's (r_idx, r_gate) replace the router
+// (no logits, no router kernel) and the standalone dispatch layout runs.
 moe_status forward_impl(const moe_shape* s, const void* x, const void* packed, const float* bias,
                         const int32_t* expert_rank_host, void* y, const moe_forward_buffers* buffers,
-                        void* ws, size_t ws_bytes, cudaStream_t st, cudaEvent_t* ev) {
+                        void* ws, size_t ws_bytes, cudaStream_t st, cudaEvent_t* ev,
+                        bool routed = false, const int32_t* r_idx = nullptr,
+                        const float* r_gate = nullptr) {
   moe_status r = check_shape(s);
   if (r != MOE_OK) return r;
   if (!ws) return MOE_ERR_INVALID_ARG;
@@ -329,9 +333,10 @@ moe_status forward_impl(const moe_shape* s, const void* x, const void* packed, c
   RankMap map;
   if ((r = build_map(s, expert_rank_host, &map)) != MOE_OK) return r;
   if (s->T == 0) return MOE_OK;
-  if (!x || !packed || !y) return MOE_ERR_INVALID_ARG;
+  if (!x || !packed || !y || (routed && !r_idx)) return MOE_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(y, 16) || !aligned(packed, kAlign) || (bias && !aligned(bias, 4)))
     return MOE_ERR_ALIGNMENT;
+  if (routed && (!aligned(r_idx, 4) || (r_gate && !aligned(r_gate, 4)))) return MOE_ERR_ALIGNMENT;
   FwdBufs f = carve_forward(s, ws, buffers);
   if ((r = check_layout_ptrs(s, &f.lay)) != MOE_OK) return r;
   if (!aligned(f.logits, 4) || !aligned(f.idx, 4) || !aligned(f.gate, 4) || !aligned(f.x_perm, 16) ||
@@ -356,7 +361,12 @@ moe_status forward_impl(const moe_shape* s, const void* x, const void* packed, c
   // small f: the whole expert FFN and the combine in one kernel
   const bool fused = bf16 && ffn_fused_supported(s->d, s->f);
   if ((r = mark(0)) != MOE_OK) return r;
-  if (bf16) {
+  // routing and dispatch layout
+  if (routed) {
+    if ((r = mark(1)) != MOE_OK) return r;
+    if ((r = do_layout(s, r_idx, map, &f.lay, sc, -1, kWaitLimitNs, st)) != MOE_OK) return r;
+    if ((r = mark(2)) != MOE_OK) return r;
+  } else if (bf16) {
     // router + top-k + gates + per-tile dispatch histogram in one kernel
     RouteArgs a{};
     a.x = x;
@@ -381,6 +391,14 @@ moe_status forward_impl(const moe_shape* s, const void* x, const void* packed, c
                                                sc.block_hist, st))) != MOE_OK)
       return r;
     if ((r = mark(2)) != MOE_OK) return r;
+  } else {
+    if ((r = do_route(s, x, &pk, bias, f.logits, f.idx, f.gate, sc.ctl, st)) != MOE_OK) return r;
+    if ((r = mark(1)) != MOE_OK) return r;
+    if ((r = do_layout(s, f.idx, map, &f.lay, sc, -1, kWaitLimitNs, st)) != MOE_OK) return r;
+    if ((r = mark(2)) != MOE_OK) return r;
+  }
+  // expert FFN
+  if (bf16) {
     if (fused) {
       FfnArgs fa{};
       const bool g = gather_fits(s);
@@ -419,10 +437,6 @@ moe_status forward_impl(const moe_shape* s, const void* x, const void* packed, c
         return r;
     }
   } else {
-    if ((r = do_route(s, x, &pk, bias, f.logits, f.idx, f.gate, sc.ctl, st)) != MOE_OK) return r;
-    if ((r = mark(1)) != MOE_OK) return r;
-    if ((r = do_layout(s, f.idx, map, &f.lay, sc, -1, kWaitLimitNs, st)) != MOE_OK) return r;
-    if ((r = mark(2)) != MOE_OK) return r;
     if ((r = cuda_status(launch_permute(x, f.lay.row_token, nullptr, f.x_perm, s->T, s->k,
                                         (uint32_t)(s->d * esize(s->dtype)), st))) != MOE_OK)
       return r;
@@ -438,8 +452,8 @@ moe_status forward_impl(const moe_shape* s, const void* x, const void* packed, c
       return r;
   }
   if ((r = mark(5)) != MOE_OK) return r;
-  if ((r = cuda_status(launch_combine(s->dtype, f.y_perm, f.lay.slot_row, f.gate, y, s->T, s->d,
-                                      s->k, st))) != MOE_OK)
+  if ((r = cuda_status(launch_combine(s->dtype, f.y_perm, f.lay.slot_row, routed ? r_gate : f.gate,
+                                      y, s->T, s->d, s->k, st))) != MOE_OK)
     return r;
   return mark(6);
 }
@@ -599,6 +613,15 @@ moe_status moe_forward(const moe_shape* s, const void* x, const void* packed, co
                        void* ws, size_t ws_bytes, moe_stream_t stream) {
   return forward_impl(s, x, packed, bias, expert_rank_host, y, buffers, ws, ws_bytes,
                       (cudaStream_t)stream, nullptr);
+}
+
+moe_status moe_forward_routed(const moe_shape* s, const void* x, const void* packed,
+                              const int32_t* topk_idx, const float* topk_gate,
+                              const int32_t* expert_rank_host, void* y,
+                              const moe_forward_buffers* buffers, void* ws, size_t ws_bytes,
+                              moe_stream_t stream) {
+  return forward_impl(s, x, packed, nullptr, expert_rank_host, y, buffers, ws, ws_bytes,
+                      (cudaStream_t)stream, nullptr, true, topk_idx, topk_gate);
 }
 
 moe_status moe_forward_timed(const moe_shape* s, const void* x, const void* packed,

@@ -111,3 +111,18 @@ def test_matching_buffers_pass_the_checks():
     with pytest.raises(ValueError, match="CUDA"):
         moe.combine(S, torch.zeros(R, S.d, dtype=S.dtype), torch.zeros(S.T, S.k, **i32),
                     torch.zeros(S.T, S.k))
+
+
+def test_forward_routed_routing_arrays():
+    x, p = _x(), _packed()
+    with pytest.raises(ValueError, match="^topk_idx:"):
+        moe.forward_routed(S, x, p, torch.zeros(S.T, S.k, dtype=torch.int64), None, _ws())
+    with pytest.raises(ValueError, match="^topk_idx:"):
+        moe.forward_routed(S, x, p, torch.zeros(R, **i32), None, _ws())
+    with pytest.raises(ValueError, match="^topk_gate:"):
+        moe.forward_routed(S, x, p, torch.zeros(S.T, S.k, **i32),
+                           torch.zeros(S.T, S.k, dtype=torch.float64), _ws())
+    with pytest.raises(ValueError, match="^packed:"):
+        moe.forward_routed(S, x, _packed(short=1), torch.zeros(S.T, S.k, **i32), None, _ws())
+    with pytest.raises(ValueError, match="CUDA"):
+        moe.forward_routed(S, x, p, torch.zeros(S.T, S.k, **i32), torch.zeros(S.T, S.k), _ws())
