@@ -1,6 +1,7 @@
 """The C-ABI library builds, loads without a GPU, and exports every entry
-point that include/moe.h declares; host-side argument checks answer without
-launching anything."""
+point that include/moe.h declares; the binding's ctypes prototypes take the
+declared number and kinds of arguments; host-side argument checks answer
+without launching anything."""
 import ctypes
 import os
 import re
@@ -112,3 +113,63 @@ def test_misaligned_tensors_rejected(L):
     assert L.moe_permute(ctypes.byref(s), P(8), P(256), P(4096), None) == moe.MOE_ERR_ALIGNMENT
     assert L.moe_combine(ctypes.byref(s), P(4096), P(256), None, P(4100), None) == moe.MOE_ERR_ALIGNMENT
     assert L.moe_permute(ctypes.byref(s), None, P(256), P(4096), None) == moe.MOE_ERR_INVALID_ARG
+
+
+def _declared_params():
+    """Entry point -> its parameter count, from include/moe.h."""
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    out = {}
+    for m in re.finditer(r"(?:MOE_API\s+)?(?:const\s+char\s*\*|moe_status)\s+(moe_\w+)\s*\(([^)]*)\)\s*;",
+                         src):
+        params = [p.strip() for p in m.group(2).split(",") if p.strip()]
+        out[m.group(1)] = 0 if params == ["void"] else len(params)
+    return out
+
+
+def test_binding_argument_counts_match_the_header(L):
+    """Each ctypes prototype takes as many arguments as the C declaration,
+    so no call can shift or drop an argument."""
+    decl = _declared_params()
+    assert sorted(decl) == sorted(moe.SYMBOLS)
+    for name, n in decl.items():
+        fn = getattr(L, name)
+        assert fn.argtypes is not None, name
+        assert len(fn.argtypes) == n, (name, len(fn.argtypes), n)
+
+
+def _c_kind(param: str) -> str:
+    p = " ".join(param.split())
+    if "*" in p or p.startswith(("moe_stream_t", "moe_event_t")):
+        return "ptr"
+    if p.startswith(("size_t", "const size_t")):
+        return "size"
+    if "int64_t" in p:
+        return "i64"
+    if p.startswith(("int32_t", "int ", "const int32_t", "moe_status", "moe_dtype")):
+        return "i32"
+    raise AssertionError(f"unclassified parameter {param!r}")
+
+
+def _py_kind(t) -> str:
+    if t is ctypes.c_void_p or t is ctypes.c_char_p or isinstance(t, type(ctypes.POINTER(ctypes.c_int))):
+        return "ptr"
+    if t is ctypes.c_size_t:
+        return "size"
+    if ctypes.sizeof(t) == 8:
+        return "i64"
+    if ctypes.sizeof(t) == 4:
+        return "i32"
+    raise AssertionError(f"unclassified ctypes type {t!r}")
+
+
+def test_binding_argument_kinds_match_the_header(L):
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    for m in re.finditer(r"(?:MOE_API\s+)?(?:const\s+char\s*\*|moe_status)\s+(moe_\w+)\s*\(([^)]*)\)\s*;",
+                         src):
+        params = [p.strip() for p in m.group(2).split(",") if p.strip()]
+        fn = getattr(L, m.group(1))
+        kinds_c = [_c_kind(p) for p in params]
+        kinds_py = [_py_kind(t) for t in fn.argtypes]
+        assert kinds_py == kinds_c, (m.group(1), kinds_py, kinds_c)
