@@ -173,3 +173,44 @@ def test_binding_argument_kinds_match_the_header(L):
         kinds_c = [_c_kind(p) for p in params]
         kinds_py = [_py_kind(t) for t in fn.argtypes]
         assert kinds_py == kinds_c, (m.group(1), kinds_py, kinds_c)
+
+
+def test_struct_layouts_match_the_header(tmp_path):
+    """sizeof / offsetof of the ABI structs as a C compiler lays them out
+    from include/moe.h, against the binding's ctypes structures (and the
+    device-resident moe_stats words that stats_dict decodes)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    structs = {
+        "moe_shape": [f for f, _ in moe.moe_shape._fields_],
+        "moe_layout": [f for f, _ in moe.moe_layout._fields_],
+        "moe_forward_buffers": [f for f, _ in moe.moe_forward_buffers._fields_],
+        "moe_stats": ["rows_sent", "dup_removed", "tokens_single_rank", "home_rank_rows",
+                      "max_expert_rows", "min_expert_rows"],
+    }
+    lines = ['#include <stdio.h>', '#include "moe.h"', "int main(void) {"]
+    for s, fields in structs.items():
+        lines.append(f'  printf("{s} size %zu\\n", sizeof({s}));')
+        for f in fields:
+            lines.append(f'  printf("{s} {f} %zu\\n", offsetof({s}, {f}));')
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.check_call([cc, "-std=c99", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)])
+    got = {}
+    for line in subprocess.check_output([str(exe)], text=True).splitlines():
+        s, f, v = line.split()
+        got[(s, f)] = int(v)
+    for s, cls in (("moe_shape", moe.moe_shape), ("moe_layout", moe.moe_layout),
+                   ("moe_forward_buffers", moe.moe_forward_buffers)):
+        assert got[(s, "size")] == ctypes.sizeof(cls), s
+        for f in structs[s]:
+            assert got[(s, f)] == getattr(cls, f).offset, (s, f)
+    # stats_dict reads six int64 words: the four counters, then max (low half)
+    # and min (high half) of word 4
+    assert [got[("moe_stats", f)] for f in structs["moe_stats"]] == [0, 8, 16, 24, 32, 36]
+    assert got[("moe_stats", "size")] <= 6 * 8
