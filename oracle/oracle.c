@@ -19,7 +19,8 @@
  *  [Coupling]     "Expert Coupling in MoE Pretraining: Reducing All-to-All
  *                 Overhead with Correlated Placement and Token Shuffling":
  *                 Abstract (each token sent to each GPU once), Table I
- *                 (GPUs per token, deduplication, T/EP tokens per GPU),
+ *                 (GPUs per token, deduplication; tokens split evenly
+ *                 over the GPUs),
  *                 Table III (notation S_l(t), W[e,e']).
  *  [Revisiting]   "Revisiting MoE and Dense Speed-Accuracy Comparisons for
  *                 LLM Training": 2.1 Architecture (SwiGLU; Top-K routing),
