@@ -21,7 +21,8 @@
  *  - "Expert Coupling in MoE Pretraining: Reducing All-to-All Overhead with
  *    Correlated Placement and Token Shuffling", Abstract (experts spread over
  *    EP ranks; each token sent to each GPU once), Table I (distinct GPUs per
- *    token, deduplicated rows, T/EP tokens per GPU), Table III (notation).
+ *    token, deduplicated rows; tokens split evenly over the GPUs), Table III
+ *    (notation).
  *
  * Conventions for every call:
  *  - All array arguments are DEVICE pointers owned by the caller, except

@@ -153,7 +153,7 @@ void oracle_margin(int64_t n, int32_t E, int32_t k, const double* logits, double
  * stats[2] tokens_single_rank = #t with |R(t)| == 1
  * stats[3] home_rank_rows     = #a with map[idx[a]] == home(t),
  *                               home(t) = floor(t*ep/T) ([Coupling] Table I:
- *                               T/EP tokens per GPU)
+ *                               tokens split evenly over the GPUs)
  * stats[4] max expert count, stats[5] min expert count.
  *
  * Returns 0, or -1 if an index is out of range.

@@ -16,8 +16,8 @@
 //
 // Deduplicated send layout: "Expert Coupling in MoE Pretraining", Abstract
 // (each token is sent to each GPU once) and Table I (GPUs per token = distinct
-// destinations; deduplication = rows removed as duplicates; T/EP tokens per
-// GPU for the home rank).
+// destinations; deduplication = rows removed as duplicates; the tokens split
+// evenly over the GPUs give the home rank).
 #include "lookback.cuh"
 
 namespace moe {
