@@ -16,6 +16,7 @@ rounds them to the compared precision itself.
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 import subprocess
 
@@ -260,3 +261,80 @@ def fit_correlated_placement(idx, E: int, ep: int) -> list:
         for e in members:
             rank_of[e] = r
     return rank_of
+
+
+# ----------------------------------------------------------------------------
+# Routing variants and router observability.  Oracle side only so far: the
+# CUDA path does not implement these yet.
+
+def near_tie_share(logits, k: int, threshold: float = 1e-5) -> float:
+    """Share of tokens whose routing margin is below `threshold`: the router
+    statistic that "MoE Pretraining: Parallelism Layout Changes the Model,
+    Not Quality" (Practical Implications: monitor the router) recommends
+    logging next to the loss.  Margin as in margin(); k = E has no margin
+    and counts as no tie."""
+    m = margin(logits, k)
+    return float(np.mean(m < threshold)) if len(m) else 0.0
+
+
+def routing_changes(idx_a, idx_b) -> dict:
+    """How two routings of the same tokens differ (a run against a recorded
+    routing table, same page, Practical Implications):
+      tokens   tokens whose set of k experts differs
+      experts  sum over tokens of |A(t) minus B(t)|, the experts swapped
+      slots    (t, j) whose expert differs, slot order included."""
+    a = _np(idx_a, np.int64)
+    b = _np(idx_b, np.int64)
+    assert a.shape == b.shape
+    swapped = np.array([len(set(ra) - set(rb)) for ra, rb in zip(a.tolist(), b.tolist())],
+                       np.int64)
+    return dict(tokens=int((swapped > 0).sum()), experts=int(swapped.sum()),
+                slots=int((a != b).sum()))
+
+
+def topk_selection_bias(logits, bias, k: int):
+    """Top-k with a selection-only expert bias (the auxiliary-loss-free
+    router named in "Expert Coupling in MoE Pretraining", Fig. 11; the
+    loss-free balancing counts of "MoE Pretraining: Parallelism Layout
+    Changes the Model, Not Quality", introduction): the experts are chosen
+    on logits + bias under the usual key (value desc, index asc), and the
+    gates are the softmax of the chosen experts' logits without the bias,
+    in the chosen order.  The sum logits + bias is taken in float32, the
+    precision a kernel adding two float32 vectors decides in.
+    Returns (idx int32 [n, k], gate float64 [n, k])."""
+    l = _np(logits, np.float64)
+    b = _np(bias, np.float64)
+    key = (l.astype(np.float32) + b.astype(np.float32)[None, :]).astype(np.float64)
+    idx, _ = topk(key, k)
+    chosen = np.take_along_axis(l, idx.astype(np.int64), 1)
+    e = np.exp(chosen - chosen.max(1, keepdims=True))
+    return idx, e / e.sum(1, keepdims=True)
+
+
+def expert_capacity(T: int, k: int, E: int, capacity_factor: float) -> int:
+    """Rows an expert may take: ceil(capacity_factor * T * k / E), the factor
+    times an expert's mean load ("Revisiting MoE and Dense Speed-Accuracy
+    Comparisons", 2.1: expert capacity factor 2 with top-2 routing; the
+    formula is the reading taken where the page names only the factor)."""
+    return int(math.ceil(capacity_factor * T * k / E))
+
+
+def capacity_keep(idx, E: int, capacity_factor: float) -> np.ndarray:
+    """Which assignments an expert of limited capacity keeps (bool [T, k]).
+    Reading taken: every token's first choice is served before any token's
+    second choice, and so on (choice rank j ascending), tokens in order
+    inside a rank; an assignment is kept while its expert has taken fewer
+    than expert_capacity() rows.  A dropped assignment contributes nothing
+    to the token's output (its gate is not redistributed)."""
+    ix = _np(idx, np.int64)
+    T, k = ix.shape
+    cap = expert_capacity(T, k, E, capacity_factor)
+    taken = [0] * E
+    keep = np.zeros((T, k), bool)
+    for j in range(k):
+        for t in range(T):
+            e = int(ix[t, j])
+            if taken[e] < cap:
+                taken[e] += 1
+                keep[t, j] = True
+    return keep
