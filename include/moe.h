@@ -4,21 +4,21 @@
  * One token-routed Mixture-of-Experts layer, forward only, on one GPU:
  *
  *   logits = x W_r (+ bias)                       router GEMM
- *   idx, gate = top-k(logits), softmax over the k top-k with softmax gates
+ *   idx = top-k(logits), gate = softmax over k    top-k routing
  *   counts / offsets / permutation / send layout  expert-grouped dispatch
  *   x_perm[r] = x[row_token[r]]                   permute
  *   h = silu(x_perm W_g[e]) * (x_perm W_u[e])     grouped SwiGLU, gate/up
  *   y_perm = h W_d[e]                             grouped SwiGLU, down
  *   y[t] = sum_j gate[t,j] y_perm[slot_row[t*k+j]] combine
  *
- * Sources (page title, then section / table):
- *  - "MoE Pretraining: Parallelism Layout Changes the Model, Not Quality",
+ * Sources (page title, then section / table; the tags are used below):
+ *  - [Layout] "MoE Pretraining: Parallelism Layout Changes the Model, Not Quality",
  *    Methodology / Models and Data: a router sends each token to a few of 16
  *    SwiGLU experts (top-4); Finding 3: routing margin and near-ties.
- *  - "Revisiting MoE and Dense Speed-Accuracy Comparisons for LLM Training",
+ *  - [Revisiting] "Revisiting MoE and Dense Speed-Accuracy Comparisons for LLM Training",
  *    2.1 Architecture (SwiGLU, Top-K routing) and Table 1 (weight layouts:
  *    router "ME" = [d, E]; FFN1 "EMH" = [E, d, f]; FFN2 "EHM" = [E, f, d]).
- *  - "Expert Coupling in MoE Pretraining: Reducing All-to-All Overhead with
+ *  - [Coupling] "Expert Coupling in MoE Pretraining: Reducing All-to-All Overhead with
  *    Correlated Placement and Token Shuffling", Abstract (experts spread over
  *    EP ranks; each token sent to each GPU once), Table I (distinct GPUs per
  *    token, deduplicated rows; tokens split evenly over the GPUs), Table III
@@ -42,8 +42,10 @@
  *    4-byte aligned (MOE_ERR_ALIGNMENT otherwise).
  *  - Results are deterministic: repeated calls with the same inputs give
  *    bit-identical outputs (no floating-point atomics anywhere).
- *  - The library holds no global mutable state; calls on different streams
- *    with different workspaces may run concurrently.
+ *  - Calls on different streams with different workspaces may run
+ *    concurrently.  The library's only global state is the scratch of
+ *    moe_dispatch_layout_static (see there) and a per-device record of the
+ *    kernels' shared-memory limits, kept under a lock.
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H
@@ -195,7 +197,9 @@ MOE_API moe_status moe_pack_weights(const moe_shape* shape, const void* w_router
                             size_t packed_bytes, moe_stream_t stream);
 
 /*
- * Router GEMM + top-k + gates.
+ * Router GEMM + top-k + gates.  Defined by: [Layout] Methodology / Models and
+ * Data (a router picks the top-4 of the experts per token); [Revisiting] 2.1
+ * (Top-K routing) and Table 1 (router "ME" = [d, E]).
  *  x        [T, d] tokens (dtype), or NULL: then `logits` is an INPUT and only
  *           the top-k step runs on it ("given logits" mode)
  *  packed   packed weights (moe_pack_weights); unused when x == NULL
@@ -216,7 +220,9 @@ MOE_API moe_status moe_route(const moe_shape* shape, const void* x, const void* 
 
 /*
  * Expert-grouped dispatch layout and the deduplicated per-rank send layout
- * (see moe_layout).  Block-level histograms plus a decoupled-lookback scan
+ * (see moe_layout).  Defined by: [Coupling] Abstract (each token is sent to
+ * each GPU that holds one of its experts once), Table I (GPUs per token,
+ * deduplicated rows), Table III (expert -> GPU placement).  Block-level histograms plus a decoupled-lookback scan
  * across blocks, then a stable scatter.
  *  topk_idx         [T, k] int32, device
  *  expert_rank_host [E] int32 in HOST memory: rank owning each expert; NULL
@@ -232,8 +238,10 @@ MOE_API moe_status moe_dispatch_layout(const moe_shape* shape, const int32_t* to
                                moe_stream_t stream);
 
 /*
- * Permute (gather): x_perm[r] = x[row_token[r]] for r < T*k, whole rows,
- * moved by TMA bulk copies staged through shared memory.
+ * Permute (gather): x_perm[r] = x[row_token[r]] for r < T*k, whole rows
+ * (the dispatch of token rows to their experts, [Coupling] Abstract),
+ * moved by TMA bulk copies staged through shared memory (rows over 1 KB) or
+ * by register copies (shorter rows).
  *  x [T, d], x_perm [T*k, d] (dtype); row_token [T*k] int32.
  * A row_token entry outside [0, T) is read as 0 (wrong values, no access
  * outside x); moe_dispatch_layout never produces one.
@@ -255,7 +263,8 @@ MOE_API moe_status moe_permute_by_token(const moe_shape* shape, const void* x,
                                         moe_stream_t stream);
 
 /*
- * Grouped SwiGLU experts over the expert-grouped rows:
+ * Grouped SwiGLU experts over the expert-grouped rows ([Revisiting] 2.1
+ * Architecture: SwiGLU experts; Table 1: FFN1 "EMH", FFN2 "EHM" layouts):
  *  h[r]      = silu(x_perm[r] W_g[e]) * (x_perm[r] W_u[e])   [T*k, f]
  *  y_perm[r] = h[r] W_d[e]                                   [T*k, d]
  * for expert e owning row r (expert_offsets [E+1], device, as produced by
@@ -289,7 +298,9 @@ MOE_API moe_status moe_grouped_swiglu_gather(const moe_shape* shape, const void*
                                              moe_stream_t stream);
 
 /*
- * Gate-weighted combine (un-permute):
+ * Gate-weighted combine (un-permute): each token's output is its k experts'
+ * outputs weighted by its gates ([Revisiting] 2.1: Top-K routing;
+ * [Layout] Models and Data):
  *   y[t] = sum_{j<k} gate[t,j] * y_perm[slot_row[t*k+j]]
  * summed in fp32 in ascending j, rounded once to the dtype.
  *  y_perm [T*k, d]; slot_row [T*k] int32; topk_gate [T, k] fp32 or NULL for
