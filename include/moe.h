@@ -330,7 +330,9 @@ typedef struct {
 
 /*
  * The whole layer enqueued back to back on `stream`, with no host
- * synchronisation in between.  bf16: one kernel for router GEMM + top-k +
+ * synchronisation in between (the steps and their sources as in the entry
+ * points above: [Layout] Models and Data, [Revisiting] 2.1, [Coupling]
+ * Abstract).  bf16: one kernel for router GEMM + top-k +
  * gates + the per-tile dispatch histogram, the layout scatter, then the
  * expert FFN: for f in {64, 128} and d in {128, 256} one kernel for the
  * gate/up GEMM, SwiGLU (H kept on chip) and down GEMM (same arithmetic as
