@@ -4,9 +4,10 @@
 
 One step is one moe_forward over one batch of the workload (router GEMM,
 top-k + gates, dispatch layout with the deduplicated send layout, permute,
-grouped SwiGLU GEMMs, combine).  Default workload: configuration 2 of the
-MoE layer set (T=16384 tokens, d=256, E=64 SwiGLU experts of width 64,
-top-4, bf16, EP=8 contiguous), the fine-grained expert layer.
+grouped SwiGLU GEMMs, combine).  Default workload: configuration 5 of the
+MoE layer set, the largest that fits one GPU (T=32768 tokens, d=4096,
+E=128 SwiGLU experts of width 1536, top-8, bf16, Zipf(1.1) logit bias,
+EP=16 contiguous); `--config N` selects the others.
 
 Timing: inputs resident in HBM; L2 is flushed (a 256 MB write) before each
 step, outside the step's CUDA events; the K steps sit between a barrier and
@@ -17,10 +18,14 @@ counts.  Prints one JSON line on rank 0.
 
 `--impl reference` times the CPU oracle (the only reference this method
 has) on a bounded sample of the same workload, on the host cores.
+
+`--kernel NAME` runs one entry point alone (see run_kernel) for profiler
+captures and per-kernel timing.
 """
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -38,6 +43,8 @@ import routing_dispatch_experts_b200 as moe  # noqa: E402
 from routing_dispatch_experts_b200 import workloads as W  # noqa: E402
 
 METRIC = "MoE-layer fwd routed tokens/s"
+# the largest workload that fits one GPU (T=32768, d=4096, E=128, f=1536, top-8)
+DEFAULT_CONFIG = 5
 L2_FLUSH_BYTES = 256 << 20
 SLEEP_CYCLES = 200_000  # ~0.1 ms of device-side sleep before each timed iteration
 # kernels of one moe_forward: bf16 = fused router, layout scatter, (permute
@@ -227,6 +234,10 @@ def run_ours(args, rank, world, local):
     dx = x.to(dev)
     dbias = None if bias is None else bias.to(dev)
     packed = moe.pack_weights(shape, wr.to(dev), wg.to(dev), wu.to(dev), wd.to(dev))
+    cpu_leg = rank == 0 and world == 1 and not args.no_cpu_baseline and not args.profile
+    # the CPU baseline reuses the host copies of the inputs (drawing the large
+    # workload's experts again would take minutes)
+    host_inputs = (x, wr, bias, wg, wu, wd) if cpu_leg else None
     del wg, wu, wd
     ws = moe.workspace(shape, forward=True, device=dev)
     buf = moe.ForwardBuffers(shape, device=dev)
@@ -370,11 +381,10 @@ def run_ours(args, rank, world, local):
     dom = max(calls, key=calls.get)
     pk = peaks()
     d = wk[dom]
-    # steps that ran at the power-capped clock (the sampler saw sw_power_cap
-    # during the timed region, or the step is a millisecond or more) take the
-    # sustained GEMM peak as denominator, the others the burst one
-    sustained = ms >= 1.0 or bool(clk and "sw_power_cap" in clk.get("reasons", []))
-    tpeak = pk["bf16_sus"] if sustained else pk["bf16"]
+    # the stage is timed inside a step of milliseconds, not a seconds-long
+    # loop, so the burst GEMM peak is the denominator; the fraction of the
+    # sustained (power-capped) peak is printed beside it
+    tpeak = pk["bf16"]
     if w.dtype != "bf16" and d["flops"] > 0:
         # fp32 expert GEMMs run on the CUDA cores' FMA pipes: SMs x 128 fp32
         # lanes x 2 FLOP per clock at the maximum SM clock
@@ -385,7 +395,7 @@ def run_ours(args, rank, world, local):
                 f"{pk['sm_max_mhz']:.0f} MHz")
     elif d["flops"] > 0 and d["flops"] / d["bytes"] > tpeak * 1e12 / (pk["hbm"] * 1e9):
         bound, achieved, peak, unit = "tensor", d["flops"] / (calls[dom] * 1e-3) / 1e12, tpeak, "TFLOP/s"
-        psrc = pk["src"] + (" bf16 sustained" if sustained else " bf16 burst")
+        psrc = pk["src"] + " bf16 burst"
     else:
         bound, achieved, peak, unit = "hbm", d["bytes"] / (calls[dom] * 1e-3) / 1e9, pk["hbm"], "GB/s"
         psrc = pk["src"] + " hbm copy"
@@ -418,37 +428,84 @@ def run_ours(args, rank, world, local):
                      "algorithmic": d},
         "clocks": clk,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.profile:
-        result["cpu_baseline"] = cpu_baseline(w, args)
+    if bound == "tensor":
+        result["roofline"]["frac_of_sustained"] = achieved / pk["bf16_sus"]
+    result["stage_roofline"] = stage_rooflines(wk, calls, pk)
+    if cpu_leg:
+        result["cpu_baseline"] = cpu_baseline(w, args, inputs=host_inputs,
+                                              gpu_idx=buf.topk_idx.cpu().numpy())
+        result["routing_check"] = result["cpu_baseline"].pop("routing_check")
     return result
 
 
+def stage_rooflines(wk, calls, pk):
+    """Every stage's fraction of its own roofline: HBM copy bandwidth for the
+    data-movement stages, the burst bf16 GEMM peak (and the sustained one)
+    for the expert GEMMs; stages that a path fuses into another are left
+    out."""
+    out = {}
+    for name, ms in calls.items():
+        d = wk[name]
+        if ms <= 0 or (d["bytes"] == 0 and d["flops"] == 0):
+            continue
+        gbs = d["bytes"] / (ms * 1e-3) / 1e9
+        e = {"ms": round(ms, 5), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / pk["hbm"], 4)}
+        if d["flops"] and d["flops"] / d["bytes"] > pk["bf16"] * 1e12 / (pk["hbm"] * 1e9):
+            tf = d["flops"] / (ms * 1e-3) / 1e12
+            e.update({"TFLOP/s": round(tf, 1), "frac_bf16_burst": round(tf / pk["bf16"], 4),
+                      "frac_bf16_sustained": round(tf / pk["bf16_sus"], 4)})
+        out[name] = e
+    return out
+
+
 # ------------------------------------------------- CPU oracle (reference arm)
-def cpu_baseline(w: W.Workload, args, budget_s: float = 12.0):
+def cpu_baseline(w: W.Workload, args, budget_s: float = 12.0, inputs=None, gpu_idx=None):
     """The oracle, as it stands, on a bounded seeded sample of the workload's
-    tokens (routing, layout of the sample, experts, combine), scaled to
-    tokens/s.  Runs on the host cores."""
+    tokens (router, top-k and gates of the sample, its dispatch layout, its
+    experts and combine, all in float64), with the sample's rate taken as
+    the batch's tokens/s: tokens are independent once routed, so the
+    sample's rate extrapolates to the whole batch.  Runs on the host cores.
+    With `gpu_idx` (the GPU's routing of the whole batch) it also counts the
+    sampled tokens whose expert sets differ from the oracle's, and how many
+    of those are not near-ties (margin below 1e-5)."""
     import oracle
     oracle.build()
-    x = W.make_x(w, args.seed, w.T)
-    wr = W.make_router(w, args.seed)
-    bias = W.make_bias(w, args.seed)
-    wg, wu, wd = W.make_experts(w, args.seed)
+    if inputs is None:
+        x = W.make_x(w, args.seed, w.T)
+        wr = W.make_router(w, args.seed)
+        bias = W.make_bias(w, args.seed)
+        wg, wu, wd = W.make_experts(w, args.seed)
+    else:
+        x, wr, bias, wg, wu, wd = inputs
 
     def run(n):
         toks = W.sample_tokens(w.T, n, seed=args.seed + 5)
         t0 = time.perf_counter()
         r = oracle.forward(x, wr, bias, wg, wu, wd, w.k, tokens=toks)
         oracle.dispatch_layout(r["idx"], w.E, w.eps[0])
-        return time.perf_counter() - t0
+        return time.perf_counter() - t0, toks, r
 
     n = 64
-    dt = run(n)
+    dt, toks, r = run(n)
     while dt < budget_s / 4 and n < w.T:
         n = min(w.T, int(n * max(2.0, budget_s / 2 / max(dt, 1e-3))))
-        dt = run(n)
-    return {"value": n / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"{n} of {w.T} tokens (seeded), full router + top-k + layout + experts + combine in float64"}
+        dt, toks, r = run(n)
+    what = "router, top-k, layout, experts and combine in float64"
+    sample = (f"all {w.T} tokens: {what}" if n == w.T else
+              f"{n} of {w.T} tokens (seeded): {what}; tokens/s of the sample, extrapolated "
+              f"to the batch (tokens are independent once routed)")
+    out = {"value": n / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+           "sample": sample, "extrapolated": n < w.T}
+    if gpu_idx is not None:
+        import numpy as np
+        gi = gpu_idx[toks.numpy()]
+        bad = np.where((np.sort(gi, 1) != np.sort(r["idx"], 1)).any(1))[0]
+        m = oracle.margin(r["logits"], w.k)
+        out["routing_check"] = {"tokens": n, "mismatches": int(len(bad)),
+                                "mismatches_not_near_tie": int((m[bad] >= 1e-5).sum()),
+                                "near_tie_threshold": 1e-5,
+                                "oracle_near_ties_in_sample": int((m < 1e-5).sum())}
+    return out
 
 
 def run_reference(args, rank, world):
@@ -466,19 +523,165 @@ def run_reference(args, rank, world):
                     "d2h_bytes_per_step": 0}}
 
 
+# ------------------------------------------------- one kernel, for profilers
+KERNELS = ("route", "topk", "layout", "permute", "permute_by_token", "grouped",
+           "grouped_gather", "combine", "forward")
+
+
+def run_kernel(args):
+    """One entry point of the library alone on a workload's seeded inputs,
+    for profiler captures and per-kernel timing:
+
+      route            moe_route (bf16: the fused router; fp32: router + top-k)
+      topk             moe_route in given-logits mode (top-k + gates only)
+      layout           moe_dispatch_layout (histogram + lookback, scatter)
+      permute          moe_permute (row order)
+      permute_by_token moe_permute_by_token (token order)
+      grouped          moe_grouped_swiglu (gate/up GEMM + SwiGLU, down GEMM)
+      grouped_gather   moe_grouped_swiglu_gather
+      combine          moe_combine
+      forward          moe_forward
+
+    Routing comes from the workload's own router on its own x; expert
+    weights are seeded N(0, 1/d) stand-ins drawn on the device (values do
+    not change what the kernels move or compute), and kernels that never
+    read them get f = 64 stand-ins.  `--tokens` / `--experts` shrink the
+    case for captures (fewer tokens; fewer experts with the same EP degree).
+    `--launches N` makes N launches and synchronises (a profiler picks
+    among them); `--time REPS` times CUDA graphs of 10 x (256 MB L2 flush +
+    launch) minus graphs of the 10 flushes alone and prints the median
+    microseconds per launch."""
+    import ctypes
+    w = W.WORKLOADS[args.config]
+    T = args.tokens or w.T
+    E = args.experts or w.E
+    ep = min(w.eps[0], E)
+    dev = torch.device("cuda", 0)
+    needs_experts = args.kernel in ("grouped", "grouped_gather", "forward")
+    f = w.f if needs_experts else 64
+    shape = moe.Shape(T=T, d=w.d, E=E, k=w.k, f=f, ep=ep, dtype=w.torch_dtype)
+    wc = dataclasses.replace(w, E=E) if E != w.E else w
+    x = W.make_x(w, args.seed, T).to(dev)
+    bias = W.make_bias(wc, args.seed)
+    bias = None if bias is None else bias.to(dev)
+    g = torch.Generator(device=dev).manual_seed(args.seed + 1)
+    std = 1.0 / math.sqrt(w.d)
+
+    def stand_in(*sz):
+        return (torch.randn(*sz, generator=g, device=dev) * std).to(w.torch_dtype)
+
+    packed = moe.pack_weights(shape, W.make_router(wc, args.seed).to(dev), stand_in(E, w.d, f),
+                              stand_in(E, w.d, f), stand_in(E, f, w.d))
+    ws = moe.workspace(shape, forward=args.kernel == "forward", device=dev)
+    logits, idx, gate = moe.route(shape, x, packed, bias, ws)
+    lay = moe.dispatch_layout(shape, idx, ws)
+    torch.cuda.synchronize()
+    moe.check_device_status(ws)
+    R = shape.R
+    L, sc, P = moe.lib(), shape.c, moe._p
+    x_perm = moe.permute(shape, x, lay["row_token"]) if args.kernel.startswith("grouped") \
+        or args.kernel == "combine" else None
+    h = torch.empty((R, f), dtype=w.torch_dtype, device=dev) if needs_experts else None
+    y_perm = torch.empty((R, w.d), dtype=w.torch_dtype, device=dev) if needs_experts else x_perm
+    out = torch.empty((R, w.d), dtype=w.torch_dtype, device=dev) if "permute" in args.kernel \
+        else torch.empty((T, w.d), dtype=w.torch_dtype, device=dev)
+    idx2 = torch.empty_like(idx)
+    gate2 = torch.empty_like(gate)
+    clay = moe._c_layout(moe._layout_tensors(shape, dev))
+    rmap = None
+
+    def launch(stream=None):
+        st = moe._stream(stream)
+        k = args.kernel
+        if k == "route":
+            r = L.moe_route(ctypes.byref(sc), P(x), P(packed), P(bias), P(logits), P(idx2),
+                            P(gate2), P(ws), ws.numel(), st)
+        elif k == "topk":
+            r = L.moe_route(ctypes.byref(sc), None, None, P(bias), P(logits), P(idx2), P(gate2),
+                            P(ws), ws.numel(), st)
+        elif k == "layout":
+            r = L.moe_dispatch_layout(ctypes.byref(sc), P(idx), rmap, ctypes.byref(clay), P(ws),
+                                      ws.numel(), st)
+        elif k == "permute":
+            r = L.moe_permute(ctypes.byref(sc), P(x), P(lay["row_token"]), P(out), st)
+        elif k == "permute_by_token":
+            r = L.moe_permute_by_token(ctypes.byref(sc), P(x), P(lay["slot_row"]), P(out), st)
+        elif k == "grouped":
+            r = L.moe_grouped_swiglu(ctypes.byref(sc), P(x_perm), P(lay["expert_offsets"]),
+                                     P(packed), P(h), P(y_perm), P(ws), ws.numel(), st)
+        elif k == "grouped_gather":
+            r = L.moe_grouped_swiglu_gather(ctypes.byref(sc), P(x), P(lay["row_token"]),
+                                            P(lay["expert_offsets"]), P(packed), P(h),
+                                            P(y_perm), P(ws), ws.numel(), st)
+        elif k == "combine":
+            r = L.moe_combine(ctypes.byref(sc), P(y_perm), P(lay["slot_row"]), P(gate), P(out), st)
+        else:
+            r = L.moe_forward(ctypes.byref(sc), P(x), P(packed), P(bias), rmap, P(out), None,
+                              P(ws), ws.numel(), st)
+        moe._check(r, k)
+
+    for _ in range(args.launches):
+        launch()
+    torch.cuda.synchronize()
+    moe.check_device_status(ws)
+    print(f"config {args.config} {args.kernel}: T={T} E={E} f={f} ep={ep}, "
+          f"{args.launches} launches ok", flush=True)
+    if not args.time:
+        return
+    reps = 10
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    side = torch.cuda.Stream(dev)
+
+    def capture(with_kernel):
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=side):
+            for i in range(reps):
+                flush.fill_(i & 255)
+                if with_kernel:
+                    launch(side)
+        return gr
+
+    g1, g0 = capture(True), capture(False)
+
+    def run(gr):
+        gr.replay()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        gr.replay()
+        e1.record()
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) * 1e3
+
+    d = [(run(g1) - run(g0)) / reps for _ in range(args.time)]
+    moe.check_device_status(ws)
+    us = statistics.median(d)
+    print(json.dumps({"kernel": args.kernel, "config": args.config, "T": T, "E": E,
+                      "us_median": us, "us_min": min(d), "us_max": max(d), "reps": args.time}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", type=int, default=2, choices=sorted(W.WORKLOADS))
+    ap.add_argument("--config", type=int, default=DEFAULT_CONFIG, choices=sorted(W.WORKLOADS))
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", action="store_true",
                     help="short run for a profiler: no clock warm-up, e2e or CPU baseline")
+    ap.add_argument("--kernel", choices=KERNELS,
+                    help="run one entry point alone (profiler captures, per-kernel timing)")
+    ap.add_argument("--tokens", type=int, default=0, help="--kernel: token count (default: the workload's)")
+    ap.add_argument("--experts", type=int, default=0, help="--kernel: expert count (default: the workload's)")
+    ap.add_argument("--launches", type=int, default=5, help="--kernel: launches before exit")
+    ap.add_argument("--time", type=int, default=0, metavar="REPS", help="--kernel: timing repetitions")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.kernel:
+        run_kernel(args)
+        return
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", 0))
         world = int(os.environ.get("WORLD_SIZE", 1))

@@ -6,7 +6,7 @@
 #include <algorithm>
 #include <cstring>
 
-#include "kernels.cuh"
+#include "checks.cuh"
 
 using namespace moe;
 
@@ -16,25 +16,9 @@ constexpr size_t kAlign = 256;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
-int esize(int dtype) { return dtype == MOE_BF16 ? 2 : 4; }
-
 int gu_block(int f) { return f % 128 == 0 ? 128 : 64; }
 
 int pad16(int E) { return (E + 15) / 16 * 16; }
-
-bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
-
-moe_status check_shape(const moe_shape* s) {
-  if (!s) return MOE_ERR_INVALID_ARG;
-  if (s->dtype != MOE_F32 && s->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
-  if (s->T < 0 || s->E < 1 || s->E > 256 || s->k < 1 || s->k > std::min(s->E, 16) || s->ep < 1 ||
-      s->ep > s->E || s->E % s->ep != 0 || s->d <= 0 || s->f <= 0)
-    return MOE_ERR_INVALID_ARG;
-  if (s->T * (int64_t)s->k >= (int64_t(1) << 31)) return MOE_ERR_INVALID_ARG;
-  if (s->d % 64 != 0 || s->f % 64 != 0 || (int64_t)s->d * esize(s->dtype) > 16384)
-    return MOE_ERR_UNSUPPORTED;
-  return MOE_OK;
-}
 
 // ---- scratch workspace: control block, per-bin totals, lookback words
 struct Scratch {
@@ -161,26 +145,6 @@ FwdBufs carve_forward(const moe_shape* s, void* ws, const moe_forward_buffers* b
 
 moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
-moe_status build_map(const moe_shape* s, const int32_t* host_map, RankMap* m) {
-  std::memset(m, 0, sizeof(*m));
-  const int per = s->E / s->ep;
-  if (!host_map) {
-    for (int e = 0; e < s->E; ++e) m->r[e] = (uint8_t)(e / per);
-    return MOE_OK;
-  }
-  int count[256] = {0};
-  for (int e = 0; e < s->E; ++e) {
-    const int r = host_map[e];
-    if (r < 0 || r >= s->ep) return MOE_ERR_INVALID_ARG;
-    ++count[r];
-    m->r[e] = (uint8_t)r;
-  }
-  // a placement is a partition: every rank owns exactly E/ep experts
-  for (int r = 0; r < s->ep; ++r)
-    if (count[r] != per) return MOE_ERR_INVALID_ARG;
-  return MOE_OK;
-}
-
 // ---- the steps, after their arguments are checked
 moe_status do_route(const moe_shape* s, const void* x, const Packed* pk, const float* bias,
                     float* logits, int32_t* idx, float* gate, Control* ctl, cudaStream_t st) {
@@ -277,22 +241,6 @@ moe_status do_grouped(const moe_shape* s, const void* x_perm, const int32_t* off
   moe_status r = do_grouped_part(0, s, x_perm, nullptr, offsets, pk, h, y_perm, ctl, st);
   if (r != MOE_OK) return r;
   return do_grouped_part(1, s, x_perm, nullptr, offsets, pk, h, y_perm, ctl, st);
-}
-
-moe_status check_layout_ptrs(const moe_shape* s, const moe_layout* o) {
-  // with T == 0 the per-assignment arrays are empty and may be NULL
-  const bool rows = s->T > 0;
-  if (!o || !o->expert_counts || !o->expert_offsets || (rows && (!o->row_token || !o->slot_row)))
-    return MOE_ERR_INVALID_ARG;
-  if (s->ep > 1 && (!o->rank_counts || !o->rank_offsets ||
-                    (rows && (!o->send_token || !o->slot_send_row))))
-    return MOE_ERR_INVALID_ARG;
-  const void* ps[] = {o->expert_counts, o->expert_offsets, o->row_token, o->slot_row,
-                      o->rank_counts, o->rank_offsets, o->send_token, o->slot_send_row};
-  for (const void* p : ps)
-    if (p && !aligned(p, 4)) return MOE_ERR_ALIGNMENT;
-  if (o->stats && !aligned(o->stats, 8)) return MOE_ERR_ALIGNMENT;
-  return MOE_OK;
 }
 
 moe_status layout_entry(const moe_shape* s, const int32_t* idx, const int32_t* host_map,

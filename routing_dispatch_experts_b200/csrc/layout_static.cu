@@ -20,7 +20,7 @@
 // and later calls reuse the address.
 #include <mutex>
 
-#include "kernels.cuh"
+#include "checks.cuh"
 
 namespace {
 
@@ -49,8 +49,6 @@ void* scratch_address() {
   return g_scratch_ptr[dev];
 }
 
-bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3) == 0; }
-
 }  // namespace
 
 extern "C" MOE_API moe_status moe_dispatch_layout_static(const moe_shape* s, const int32_t* topk_idx,
@@ -58,21 +56,12 @@ extern "C" MOE_API moe_status moe_dispatch_layout_static(const moe_shape* s, con
                                                          const moe_layout* o, int32_t* device_status,
                                                          moe_stream_t stream) {
   using namespace moe;
-  if (!s || (s->dtype != MOE_F32 && s->dtype != MOE_BF16)) return MOE_ERR_INVALID_ARG;
-  if (s->T < 0 || s->E < 1 || s->E > 256 || s->k < 1 || s->k > (s->E < 16 ? s->E : 16) ||
-      s->ep < 1 || s->ep > s->E || s->E % s->ep != 0 || s->d <= 0 || s->f <= 0 ||
-      s->T * (int64_t)s->k >= (int64_t(1) << 31))
-    return MOE_ERR_INVALID_ARG;
-  const bool rows = s->T > 0;
-  if (!o || !o->expert_counts || !o->expert_offsets || (rows && (!topk_idx || !o->row_token || !o->slot_row)))
-    return MOE_ERR_INVALID_ARG;
-  if (s->ep > 1 && (!o->rank_counts || !o->rank_offsets || (rows && (!o->send_token || !o->slot_send_row))))
-    return MOE_ERR_INVALID_ARG;
-  const void* ps[] = {topk_idx, o->expert_counts, o->expert_offsets, o->row_token, o->slot_row,
-                      o->rank_counts, o->rank_offsets, o->send_token, o->slot_send_row, device_status};
-  for (const void* p : ps)
-    if (p && !aligned4(p)) return MOE_ERR_ALIGNMENT;
-  if (o->stats && (reinterpret_cast<uintptr_t>(o->stats) & 7)) return MOE_ERR_ALIGNMENT;
+  // the same checks, in the same order, as moe_dispatch_layout
+  moe_status r = check_shape(s);
+  if (r != MOE_OK) return r;
+  if (!topk_idx && s->T > 0) return MOE_ERR_INVALID_ARG;
+  if ((r = check_layout_ptrs(s, o)) != MOE_OK) return r;
+  if (!aligned(topk_idx, 4) || (device_status && !aligned(device_status, 4))) return MOE_ERR_ALIGNMENT;
 
   // the scratch this shape needs, laid out as in moe_dispatch_layout
   const size_t nb = (size_t)layout_blocks(s->T), bins = (size_t)layout_bins(s->E, s->ep);
@@ -81,18 +70,8 @@ extern "C" MOE_API moe_status moe_dispatch_layout_static(const moe_shape* s, con
   const size_t need = off_status + round256(nb * bins * 8);
   if (need > kStaticScratchBytes) return MOE_ERR_WORKSPACE;
 
-  // expert -> rank map: NULL = contiguous; otherwise a partition
-  RankMap map = {};
-  const int per = s->E / s->ep;
-  int count[256] = {0};
-  for (int e = 0; e < s->E; ++e) {
-    const int r = expert_rank_host ? expert_rank_host[e] : e / per;
-    if (r < 0 || r >= s->ep) return MOE_ERR_INVALID_ARG;
-    ++count[r];
-    map.r[e] = (uint8_t)r;
-  }
-  for (int r = 0; r < s->ep; ++r)
-    if (count[r] != per) return MOE_ERR_INVALID_ARG;
+  RankMap map;
+  if ((r = build_map(s, expert_rank_host, &map)) != MOE_OK) return r;
 
   uint8_t* base = static_cast<uint8_t*>(scratch_address());
   if (!base) return MOE_ERR_CUDA;

@@ -107,6 +107,36 @@ def test_bad_placement_rejected_before_any_launch(L):
                                  ws, 1 << 30, None) == moe.MOE_ERR_INVALID_ARG
 
 
+@pytest.mark.parametrize("kw", [
+    dict(E=0), dict(E=257), dict(k=0), dict(k=17, E=64), dict(ep=3), dict(T=-1),
+    dict(T=1 << 29, k=4), dict(d=100), dict(f=96), dict(d=8192, dtype=moe.MOE_F32), dict(dtype=7),
+])
+def test_static_layout_validates_like_the_workspace_layout(L, kw):
+    """moe_dispatch_layout_static takes the same inputs as
+    moe_dispatch_layout and rejects the same shapes with the same status,
+    before any launch (so no GPU is needed)."""
+    s = moe.moe_shape(**{**dict(T=2048, d=256, E=16, k=4, f=256, ep=1, dtype=moe.MOE_F32), **kw})
+    lay = moe.moe_layout(*([ctypes.c_void_p(256)] * 9))
+    a = L.moe_dispatch_layout(ctypes.byref(s), ctypes.c_void_p(256), None, ctypes.byref(lay),
+                              ctypes.c_void_p(1 << 20), 1 << 30, None)
+    b = L.moe_dispatch_layout_static(ctypes.byref(s), ctypes.c_void_p(256), None,
+                                     ctypes.byref(lay), None, None)
+    assert a == b != moe.MOE_OK
+
+
+def test_static_layout_rejects_bad_placements_and_pointers(L):
+    s = moe.moe_shape(T=8, d=256, E=16, k=2, f=256, ep=4, dtype=moe.MOE_F32)
+    lay = moe.moe_layout(*([ctypes.c_void_p(256)] * 9))
+    bad = (ctypes.c_int32 * 16)(*([0] * 5 + [1] * 4 + [2] * 4 + [3] * 3))
+    assert L.moe_dispatch_layout_static(ctypes.byref(s), ctypes.c_void_p(256), bad,
+                                        ctypes.byref(lay), None, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_dispatch_layout_static(ctypes.byref(s), ctypes.c_void_p(258), None,
+                                        ctypes.byref(lay), None, None) == moe.MOE_ERR_ALIGNMENT
+    lay2 = moe.moe_layout(*([ctypes.c_void_p(256)] * 4 + [None] * 5))
+    assert L.moe_dispatch_layout_static(ctypes.byref(s), ctypes.c_void_p(256), None,
+                                        ctypes.byref(lay2), None, None) == moe.MOE_ERR_INVALID_ARG
+
+
 def test_misaligned_tensors_rejected(L):
     s = moe.moe_shape(T=8, d=256, E=16, k=2, f=256, ep=1, dtype=moe.MOE_BF16)
     P = ctypes.c_void_p

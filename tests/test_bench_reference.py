@@ -9,10 +9,21 @@ import sys
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
+def test_default_workload_is_the_largest():
+    """With no flags the benchmark measures the largest single-GPU workload."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from routing_dispatch_experts_b200 import workloads as W
+    big = max(W.WORKLOADS.values(), key=lambda w: 6 * w.T * w.k * w.d * w.f)
+    assert bench.DEFAULT_CONFIG == big.cfg == 5
+
+
 def test_reference_arm_json_line():
+    # the fine-grained workload keeps this CPU test short (its expert weights
+    # are small); the arm runs the same code for every workload
     out = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1",
-                          "--warmup", "3"], cwd=ROOT, capture_output=True, text=True,
-                         timeout=600)
+                          "--warmup", "3", "--config", "2"], cwd=ROOT, capture_output=True,
+                         text=True, timeout=600)
     assert out.returncode == 0, out.stderr[-2000:]
     lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
     assert len(lines) == 1

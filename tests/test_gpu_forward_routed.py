@@ -17,6 +17,9 @@ from routing_dispatch_experts_b200 import workloads as W
 
 from util import TOL, Case
 
+LAYOUT_KEYS = ("expert_counts", "expert_offsets", "row_token", "slot_row", "rank_counts",
+               "rank_offsets", "slot_send_row")
+
 pytestmark = pytest.mark.gpu
 
 
@@ -67,3 +70,41 @@ def test_null_gates_are_unit_gates():
     y1 = moe.forward_routed(c.shape, c.dx, c.packed, idx, ones, ws)
     moe.check_device_status(ws)
     assert torch.equal(y0, y1)
+
+
+@pytest.mark.parametrize("cfg,T,ep", [(1, 300, 1), (2, 1500, 8), (3, 257, 16)])
+def test_repeated_expert_within_a_token(cfg, T, ep):
+    """A recorded routing may name one expert twice for a token (top-k never
+    does).  Each assignment is its own expert-grouped row, the token still
+    goes to that expert's rank once, and the output sums both gated copies:
+    layout bit-exact against the oracle's, output within the tolerance of
+    the oracle's per-token definition."""
+    c = Case(cfg, T=T, near_ties=False)
+    w = c.w
+    idx = W.uniform_routing(T, w.E, w.k, seed=T + 11)
+    g = torch.Generator().manual_seed(T + 1)
+    rep = torch.randperm(T, generator=g)[: T // 3]
+    idx[rep, 1] = idx[rep, 0]                  # slot 1 repeats slot 0
+    if w.k > 2:
+        idx[rep[: len(rep) // 2], w.k - 1] = idx[rep[: len(rep) // 2], 0]  # three copies
+    gate = torch.softmax(torch.randn((T, w.k), generator=g), 1)
+    shape = c.shape_ep(ep)
+    rmap = W.permutation_placement(w.E, ep, 5)
+    ws = moe.workspace(shape, forward=True)
+    buf = moe.ForwardBuffers(shape)
+    y = moe.forward_routed(shape, c.dx, c.packed, idx.cuda(), gate.cuda(), ws,
+                           expert_rank=rmap, buffers=buf)
+    moe.check_device_status(ws)
+    lay = oracle.dispatch_layout(idx.numpy(), w.E, ep, rmap)
+    for key in LAYOUT_KEYS:
+        if ep == 1 and (key.startswith("rank") or key == "slot_send_row"):
+            continue
+        np.testing.assert_array_equal(buf.layout[key].cpu().numpy(), lay[key], err_msg=key)
+    if ep > 1:
+        n = lay["stats"]["rows_sent"]
+        np.testing.assert_array_equal(buf.layout["send_token"][:n].cpu().numpy(), lay["send_token"])
+    assert moe.stats_dict(buf.layout["stats"]) == lay["stats"]
+    ref = oracle.moe_output(c.x, idx.numpy(), gate.double().numpy(), c.wg, c.wu, c.wd,
+                            tokens=np.arange(T))
+    err = np.abs(y.cpu().double().numpy() - ref).max()
+    assert err <= TOL[w.dtype] * np.abs(ref).max()

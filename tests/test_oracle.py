@@ -282,6 +282,42 @@ def test_identity_experts_unit_gates_give_k_times_x(oracle_mod, cfg):
     np.testing.assert_array_equal(y, w.k * x.double().numpy())
 
 
+def test_combine_weights_each_slot_by_its_own_gate_by_hand(oracle_mod):
+    """Non-unit gates worked by hand: two tokens, k = 2, slot rows out of
+    order.  y[0] = 0.25 * row 2 + 0.75 * row 0 = [1.75, 0];
+    y[1] = 0.5 * row 3 + 0.125 * row 1 = [0, 4.125]."""
+    y_perm = np.array([[1.0, 0.0], [0.0, 1.0], [4.0, 0.0], [0.0, 8.0]])
+    slot_row = np.array([2, 0, 3, 1], np.int32)
+    gate = np.array([[0.25, 0.75], [0.5, 0.125]])
+    y = oracle_mod.combine(y_perm, slot_row, gate)
+    np.testing.assert_array_equal(y, [[1.75, 0.0], [0.0, 4.125]])
+
+
+def test_layer_output_weights_experts_by_gates_by_hand(oracle_mod):
+    """moe_output with non-unit gates on experts whose outputs are known
+    exactly: d = f = 1, W_g = 64 for every expert, so for x in {1, 2} the
+    gate projection is 64x and silu(64x) = 64x in double (exp(-64) is below
+    half an ulp of 1).  Expert e then gives 64x * (b_e x) * c_e:
+    e0 (b=1, c=1), e1 (b=2, c=2), e2 (b=0.5, c=-1).
+    Token 0 (x=1), experts (1, 0), gates (0.75, 0.25): 0.75*256 + 0.25*64 = 208.
+    Token 1 (x=2), experts (2, 1), gates (0.625, 0.375):
+    0.625*(-128) + 0.375*1024 = 304."""
+    x = torch.tensor([[1.0], [2.0]])
+    wg = torch.full((3, 1, 1), 64.0)
+    wu = torch.tensor([1.0, 2.0, 0.5]).reshape(3, 1, 1)
+    wd = torch.tensor([1.0, 2.0, -1.0]).reshape(3, 1, 1)
+    idx = np.array([[1, 0], [2, 1]], np.int32)
+    gate = np.array([[0.75, 0.25], [0.625, 0.375]])
+    y = oracle_mod.moe_output(x, idx, gate, wg, wu, wd)
+    np.testing.assert_array_equal(y, [[208.0], [304.0]])
+    # and the same through the permuted path (layout, grouped experts, combine)
+    lay = oracle_mod.dispatch_layout(idx, 3, 1)
+    x_perm = x[torch.from_numpy(lay["row_token"]).long()]
+    y_perm = oracle_mod.grouped_swiglu(x_perm, lay["expert_offsets"], wg, wu, wd)
+    np.testing.assert_array_equal(oracle_mod.combine(y_perm, lay["slot_row"], gate),
+                                  [[208.0], [304.0]])
+
+
 def test_permuted_pipeline_equals_per_token_definition(oracle_mod):
     """layout -> permute -> grouped experts -> combine equals the per-token
     sum of gated expert outputs (same double arithmetic, bit-identical)."""

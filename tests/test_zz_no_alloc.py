@@ -80,3 +80,24 @@ def test_static_layout_rejects_shapes_beyond_its_scratch():
     rc = L.moe_dispatch_layout_static(ctypes.byref(s), ctypes.c_void_p(256), None,
                                       ctypes.byref(lay), None, None)
     assert rc == moe.MOE_ERR_WORKSPACE
+
+
+def test_static_layout_status_does_not_leak_into_the_next_call():
+    """The shared array keeps the previous call's contents, status word
+    included.  A call that meets an expert index outside [0, E) reports
+    MOE_ERR_DEVICE_INDEX; the next, valid call clears that word first and
+    reports MOE_OK with the same layout as the workspace entry point."""
+    T, E, k, ep = 3000, 64, 4, 8
+    shape = moe.Shape(T=T, d=256, E=E, k=k, f=64, ep=ep)
+    good = W.uniform_routing(T, E, k, seed=17).cuda()
+    bad = good.clone()
+    bad[T // 2, 1] = E
+    _, status = _static_call(shape, bad, None)
+    torch.cuda.synchronize()
+    assert int(status.item()) == moe.MOE_ERR_DEVICE_INDEX
+    ref = _workspace_call(shape, good, None)
+    for _ in range(2):
+        got, status = _static_call(shape, good, None)
+        torch.cuda.synchronize()
+        assert int(status.item()) == moe.MOE_OK
+        _compare(shape, got, ref)
