@@ -320,6 +320,10 @@ def run_ours(args, rank, world, local):
     calls = {name: acc[j] / reps for j, name in enumerate(moe.FORWARD_STAGES)}
     moe.check_device_status(ws)
     clk = clocks.stop()
+    # router observability of the measured batch (outside the timed region):
+    # tokens whose top-k margin is below the near-tie bound, where routing
+    # may flip between runs or implementations
+    rstats, _ = moe.router_stats(shape, buf.logits, buf.topk_idx, threshold=1e-5)
     if args.profile:
         return {"profile": True, "ms_per_step": ms, "stage_ms": calls}
 
@@ -430,6 +434,10 @@ def run_ours(args, rank, world, local):
     }
     if bound == "tensor":
         result["roofline"]["frac_of_sustained"] = achieved / pk["bf16_sus"]
+    result["routing"] = {"near_tie_tokens": rstats["near_tie_tokens"],
+                         "near_tie_share": rstats["near_tie_tokens"] / max(T, 1),
+                         "near_tie_threshold": 1e-5,
+                         "computed_by": "moe_router_stats on the timed forward's logits"}
     result["stage_roofline"] = stage_rooflines(wk, calls, pk)
     if cpu_leg:
         result["cpu_baseline"] = cpu_baseline(w, args, inputs=host_inputs,

@@ -219,6 +219,100 @@ MOE_API moe_status moe_route(const moe_shape* shape, const void* x, const void* 
                      moe_stream_t stream);
 
 /*
+ * moe_route with a selection-only expert bias: the experts are chosen on the
+ * fp32 sum logits + selection_bias (same key and tie-break as moe_route),
+ * and the gates are the softmax of the chosen experts' logits WITHOUT the
+ * selection bias, in the chosen order.  This is the auxiliary-loss-free
+ * router: a per-expert bias that steers which experts are picked for load
+ * balance without changing how their outputs are weighted ("Expert Coupling
+ * in MoE Pretraining", Fig. 11: the auxiliary-loss-free router; "MoE
+ * Pretraining: Parallelism Layout Changes the Model, Not Quality",
+ * introduction: loss-free balancing counts).
+ *  selection_bias [E] fp32, device (required; MOE_ERR_INVALID_ARG if NULL).
+ *  Every other argument as in moe_route; `logits` holds x W_r + bias (the
+ *  selection bias is not added to it).
+ */
+MOE_API moe_status moe_route_selection_bias(const moe_shape* shape, const void* x,
+                                            const void* packed, const float* bias,
+                                            const float* selection_bias, float* logits,
+                                            int32_t* topk_idx, float* topk_gate, void* ws,
+                                            size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Router statistics (moe_router_counts), written to device memory by
+ * moe_router_stats.  They
+ * are the quantities "MoE Pretraining: Parallelism Layout Changes the Model,
+ * Not Quality" recommends monitoring (Practical Implications: the near-tie
+ * share of the router, and how a run's routing differs from a recorded
+ * routing table; Finding 3: routing flips happen at near-ties).
+ *  tokens           T
+ *  near_tie_tokens  tokens whose routing margin is below the threshold
+ *  changed_tokens   tokens with at least one expert not in the recorded row
+ *  changed_experts  sum over tokens of the number of distinct experts of
+ *                   topk_idx[t] missing from recorded[t]
+ *  changed_slots    entries (t, j) with topk_idx[t,j] != recorded[t,j]
+ * (the last three are 0 when no recorded routing is given)
+ */
+typedef struct {
+  int64_t tokens;
+  int64_t near_tie_tokens;
+  int64_t changed_tokens;
+  int64_t changed_experts;
+  int64_t changed_slots;
+} moe_router_counts;
+
+/*
+ * Routing margin and router statistics ("MoE Pretraining: Parallelism
+ * Layout Changes the Model, Not Quality", Finding 3 and Practical
+ * Implications).  For each token, with s = its logits (+ selection_bias, the
+ * fp32 sum moe_route_selection_bias selects on):
+ *   margin[t] = (s_(k) - s_(k+1)) / (max_e s - min_e s)
+ * where s_(r) is the r-th largest value, computed in double from the fp32
+ * values; +inf when k == E, 0 when every value is equal.  A token is a
+ * near-tie when margin[t] < threshold.
+ *  logits         [T, E] fp32 (device), as moe_route writes it
+ *  selection_bias [E] fp32 or NULL
+ *  topk_idx       [T, k] int32, the routing to compare (may be NULL when
+ *                 recorded_idx is NULL)
+ *  recorded_idx   [T, k] int32 recorded routing table, or NULL
+ *  threshold      >= 0 (1e-5 is the near-tie bound of the parity tests)
+ *  margin         [T] double output, or NULL
+ *  stats          one moe_router_counts in device memory (8-byte aligned),
+ *                 overwritten
+ */
+MOE_API moe_status moe_router_stats(const moe_shape* shape, const float* logits,
+                                    const float* selection_bias, const int32_t* topk_idx,
+                                    const int32_t* recorded_idx, double threshold, double* margin,
+                                    moe_router_counts* stats, moe_stream_t stream);
+
+/*
+ * Expert capacity ("Revisiting MoE and Dense Speed-Accuracy Comparisons for
+ * LLM Training", 2.1: top-2 routing with an expert capacity factor).  Each
+ * expert takes at most
+ *   capacity = ceil(capacity_factor * T * k / E)
+ * assignments (the factor times an expert's mean load).  The page gives no
+ * drop order; the one taken here: every token's first choice is served
+ * before any token's second choice, and so on (choice rank ascending),
+ * tokens in index order within a rank; an assignment is kept while its
+ * expert has taken fewer than `capacity`.
+ *  topk_idx   [T, k] int32 (device)
+ *  topk_gate  [T, k] fp32 or NULL (unit gates)
+ *  keep       [T, k] int32 output: 1 kept, 0 dropped
+ *  kept_gate  [T, k] fp32 output or NULL: the gate where kept, 0 where
+ *             dropped; moe_forward_routed with these gates gives the layer
+ *             output with the dropped assignments removed (a dropped
+ *             assignment adds nothing and its gate is not redistributed)
+ *  capacity   host int64 output or NULL: the per-expert capacity
+ *  ws         scratch workspace (moe_scratch_size), for device errors
+ * capacity_factor must be > 0.  An index outside [0, E) sets
+ * MOE_ERR_DEVICE_INDEX; its keep / kept_gate entries read 0.
+ */
+MOE_API moe_status moe_capacity_keep(const moe_shape* shape, const int32_t* topk_idx,
+                                     const float* topk_gate, double capacity_factor,
+                                     int32_t* keep, float* kept_gate, int64_t* capacity,
+                                     void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
  * Expert-grouped dispatch layout and the deduplicated per-rank send layout
  * (see moe_layout).  Defined by: [Coupling] Abstract (each token is sent to
  * each GPU that holds one of its experts once), Table I (GPUs per token,
@@ -351,6 +445,20 @@ MOE_API moe_status moe_forward(const moe_shape* shape, const void* x, const void
                        const float* bias, const int32_t* expert_rank_host,
                        void* y, const moe_forward_buffers* buffers, void* ws,
                        size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * moe_forward with the router of moe_route_selection_bias: experts chosen on
+ * logits + selection_bias, gates from the logits alone; the dispatch layout,
+ * experts and combine follow that routing.  Same kernels as moe_forward.
+ *  selection_bias [E] fp32, device (required).  Other arguments as in
+ *  moe_forward.
+ */
+MOE_API moe_status moe_forward_selection_bias(const moe_shape* shape, const void* x,
+                                              const void* packed, const float* bias,
+                                              const float* selection_bias,
+                                              const int32_t* expert_rank_host, void* y,
+                                              const moe_forward_buffers* buffers, void* ws,
+                                              size_t ws_bytes, moe_stream_t stream);
 
 typedef struct CUevent_st* moe_event_t; /* same type as cudaEvent_t */
 #define MOE_FORWARD_STAGES 6

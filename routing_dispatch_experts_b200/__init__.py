@@ -56,6 +56,16 @@ STATS_FIELDS = ("rows_sent", "dup_removed", "tokens_single_rank", "home_rank_row
                 "max_expert_rows", "min_expert_rows")
 
 
+class moe_router_counts(ctypes.Structure):
+    _fields_ = [("tokens", ctypes.c_int64), ("near_tie_tokens", ctypes.c_int64),
+                ("changed_tokens", ctypes.c_int64), ("changed_experts", ctypes.c_int64),
+                ("changed_slots", ctypes.c_int64)]
+
+
+ROUTER_COUNT_FIELDS = ("tokens", "near_tie_tokens", "changed_tokens", "changed_experts",
+                       "changed_slots")
+
+
 class moe_layout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in (
         "expert_counts", "expert_offsets", "row_token", "slot_row", "rank_counts",
@@ -73,8 +83,9 @@ _lib = None
 # exported C symbols, in header order (checked against include/moe.h by the tests)
 SYMBOLS = ("moe_status_string", "moe_scratch_size", "moe_forward_workspace_size",
            "moe_workspace_init", "moe_packed_weights_size", "moe_pack_weights", "moe_route",
+           "moe_route_selection_bias", "moe_router_stats", "moe_capacity_keep",
            "moe_dispatch_layout", "moe_permute", "moe_permute_by_token", "moe_grouped_swiglu",
-           "moe_grouped_swiglu_gather", "moe_combine", "moe_forward", "moe_forward_timed",
+           "moe_grouped_swiglu_gather", "moe_combine", "moe_forward", "moe_forward_selection_bias", "moe_forward_timed",
            "moe_forward_routed", "moe_get_device_status", "moe_debug_dispatch_layout_stall",
            "moe_dispatch_layout_static")
 FORWARD_STAGES = ("route", "layout", "permute", "gate_up", "down", "combine")
@@ -98,6 +109,11 @@ def lib() -> ctypes.CDLL:
             "moe_packed_weights_size": ([S, sz], ctypes.c_int),
             "moe_pack_weights": ([S, P, P, P, P, P, ctypes.c_size_t, P], ctypes.c_int),
             "moe_route": ([S, P, P, P, P, P, P, P, ctypes.c_size_t, P], ctypes.c_int),
+            "moe_route_selection_bias": ([S, P, P, P, P, P, P, P, P, ctypes.c_size_t, P],
+                                         ctypes.c_int),
+            "moe_router_stats": ([S, P, P, P, P, ctypes.c_double, P, P, P], ctypes.c_int),
+            "moe_capacity_keep": ([S, P, P, ctypes.c_double, P, P, ctypes.POINTER(ctypes.c_int64),
+                                   P, ctypes.c_size_t, P], ctypes.c_int),
             "moe_dispatch_layout": ([S, P, P, ctypes.POINTER(moe_layout), P, ctypes.c_size_t, P],
                                     ctypes.c_int),
             "moe_permute": ([S, P, P, P, P], ctypes.c_int),
@@ -112,6 +128,9 @@ def lib() -> ctypes.CDLL:
                              ctypes.c_size_t, P], ctypes.c_int),
             "moe_forward_routed": ([S, P, P, P, P, P, P, ctypes.POINTER(moe_forward_buffers), P,
                                     ctypes.c_size_t, P], ctypes.c_int),
+            "moe_forward_selection_bias": ([S, P, P, P, P, P, P,
+                                            ctypes.POINTER(moe_forward_buffers), P,
+                                            ctypes.c_size_t, P], ctypes.c_int),
             "moe_get_device_status": ([P, P, ctypes.POINTER(ctypes.c_int)], ctypes.c_int),
             "moe_debug_dispatch_layout_stall": ([S, P, P, ctypes.POINTER(moe_layout), P,
                                                  ctypes.c_size_t, ctypes.c_int32, ctypes.c_int64, P],
@@ -261,6 +280,67 @@ def route(shape: Shape, x, packed, bias, ws, logits=None, stream=None):
     _check(lib().moe_route(ctypes.byref(s), _p(x), _p(packed), _p(bias), _p(logits), _p(idx),
                            _p(gate), _p(ws), ws.numel(), _stream(stream)), "moe_route")
     return logits, idx, gate
+
+
+def route_selection_bias(shape: Shape, x, packed, bias, selection_bias, ws, logits=None,
+                         stream=None):
+    """moe_route_selection_bias: experts chosen on logits + selection_bias,
+    gates from the logits alone.  Returns (logits, topk_idx, topk_gate);
+    x=None runs only the selection on the given `logits`."""
+    dev = ws.device
+    if x is not None:
+        _need(x, shape.dtype, (shape.T, shape.d), "x")
+        _need_packed(shape, packed)
+        logits = torch.empty((shape.T, shape.E), dtype=torch.float32, device=dev)
+    else:
+        _need(logits, torch.float32, (shape.T, shape.E), "logits")
+    _need_bias(shape, bias)
+    _need(selection_bias, torch.float32, (shape.E,), "selection_bias")
+    idx = torch.empty((shape.T, shape.k), dtype=torch.int32, device=dev)
+    gate = torch.empty((shape.T, shape.k), dtype=torch.float32, device=dev)
+    s = shape.c
+    _check(lib().moe_route_selection_bias(ctypes.byref(s), _p(x), _p(packed), _p(bias),
+                                          _p(selection_bias), _p(logits), _p(idx), _p(gate),
+                                          _p(ws), ws.numel(), _stream(stream)),
+           "moe_route_selection_bias")
+    return logits, idx, gate
+
+
+def router_stats(shape: Shape, logits, topk_idx=None, recorded_idx=None, threshold=1e-5,
+                 selection_bias=None, want_margin=False, stream=None):
+    """moe_router_stats: (dict of the counters, margin [T] float64 or None).
+    The counters are read back to the host (a synchronisation)."""
+    _need(logits, torch.float32, (shape.T, shape.E), "logits")
+    if topk_idx is not None:
+        _need(topk_idx, torch.int32, (shape.T, shape.k), "topk_idx")
+    if recorded_idx is not None:
+        _need(recorded_idx, torch.int32, (shape.T, shape.k), "recorded_idx")
+    if selection_bias is not None:
+        _need(selection_bias, torch.float32, (shape.E,), "selection_bias")
+    dev = logits.device
+    counts = torch.zeros(len(ROUTER_COUNT_FIELDS), dtype=torch.int64, device=dev)
+    margin = torch.empty(shape.T, dtype=torch.float64, device=dev) if want_margin else None
+    s = shape.c
+    _check(lib().moe_router_stats(ctypes.byref(s), _p(logits), _p(selection_bias), _p(topk_idx),
+                                  _p(recorded_idx), float(threshold), _p(margin), _p(counts),
+                                  _stream(stream)), "moe_router_stats")
+    return dict(zip(ROUTER_COUNT_FIELDS, counts.cpu().tolist())), margin
+
+
+def capacity_keep(shape: Shape, topk_idx, topk_gate, capacity_factor: float, ws, stream=None):
+    """moe_capacity_keep: (keep [T,k] int32, kept_gate [T,k] fp32, capacity)."""
+    _need(topk_idx, torch.int32, (shape.T, shape.k), "topk_idx")
+    if topk_gate is not None:
+        _need(topk_gate, torch.float32, (shape.T, shape.k), "topk_gate")
+    dev = topk_idx.device
+    keep = torch.empty((shape.T, shape.k), dtype=torch.int32, device=dev)
+    kept = torch.empty((shape.T, shape.k), dtype=torch.float32, device=dev)
+    cap = ctypes.c_int64(0)
+    s = shape.c
+    _check(lib().moe_capacity_keep(ctypes.byref(s), _p(topk_idx), _p(topk_gate),
+                                   float(capacity_factor), _p(keep), _p(kept), ctypes.byref(cap),
+                                   _p(ws), ws.numel(), _stream(stream)), "moe_capacity_keep")
+    return keep, kept, cap.value
 
 
 def _layout_tensors(shape: Shape, dev):
@@ -446,6 +526,24 @@ def forward(shape: Shape, x, packed, bias, ws, expert_rank=None, y=None,
                              _host_map(shape, expert_rank), _p(y),
                              ctypes.byref(b) if b is not None else None, _p(ws), ws.numel(),
                              _stream(stream)), "moe_forward")
+    return y
+
+
+def forward_selection_bias(shape: Shape, x, packed, bias, selection_bias, ws, expert_rank=None,
+                           y=None, buffers: Optional[ForwardBuffers] = None, stream=None):
+    """moe_forward_selection_bias: the layer with a selection-only expert
+    bias in the router; returns y [T, d]."""
+    _forward_args(shape, x, packed, bias, y, buffers)
+    _need(selection_bias, torch.float32, (shape.E,), "selection_bias")
+    if y is None:
+        y = torch.empty((shape.T, shape.d), dtype=shape.dtype, device=x.device)
+    s = shape.c
+    b = buffers.c if buffers is not None else None
+    _check(lib().moe_forward_selection_bias(ctypes.byref(s), _p(x), _p(packed), _p(bias),
+                                            _p(selection_bias), _host_map(shape, expert_rank),
+                                            _p(y), ctypes.byref(b) if b is not None else None,
+                                            _p(ws), ws.numel(), _stream(stream)),
+           "moe_forward_selection_bias")
     return y
 
 

@@ -4,6 +4,7 @@
 // files.  Nothing here allocates device memory or synchronises a stream
 // (except moe_get_device_status, whose job is to read the device status).
 #include <algorithm>
+#include <cmath>
 #include <cstring>
 
 #include "checks.cuh"
@@ -147,7 +148,8 @@ moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_E
 
 // ---- the steps, after their arguments are checked
 moe_status do_route(const moe_shape* s, const void* x, const Packed* pk, const float* bias,
-                    float* logits, int32_t* idx, float* gate, Control* ctl, cudaStream_t st) {
+                    const float* sel_bias, float* logits, int32_t* idx, float* gate, Control* ctl,
+                    cudaStream_t st) {
   if (x) {
     cudaError_t e;
     if (s->dtype == MOE_BF16) {
@@ -156,6 +158,7 @@ moe_status do_route(const moe_shape* s, const void* x, const Packed* pk, const f
       a.x = x;
       a.wrT = pk->wrT;
       a.bias = bias;
+      a.sel_bias = sel_bias;
       a.T = s->T;
       a.d = s->d;
       a.E = s->E;
@@ -173,7 +176,7 @@ moe_status do_route(const moe_shape* s, const void* x, const Packed* pk, const f
     }
     if (e != cudaSuccess) return MOE_ERR_CUDA;
   }
-  return cuda_status(launch_topk(logits, s->T, s->E, s->k, idx, gate, st));
+  return cuda_status(launch_topk(logits, sel_bias, s->T, s->E, s->k, idx, gate, st));
 }
 
 moe_status do_layout(const moe_shape* s, const int32_t* idx, const RankMap& map,
@@ -272,7 +275,7 @@ moe_status forward_impl(const moe_shape* s, const void* x, const void* packed, c
                         const int32_t* expert_rank_host, void* y, const moe_forward_buffers* buffers,
                         void* ws, size_t ws_bytes, cudaStream_t st, cudaEvent_t* ev,
                         bool routed = false, const int32_t* r_idx = nullptr,
-                        const float* r_gate = nullptr) {
+                        const float* r_gate = nullptr, const float* sel_bias = nullptr) {
   moe_status r = check_shape(s);
   if (r != MOE_OK) return r;
   if (!ws) return MOE_ERR_INVALID_ARG;
@@ -282,7 +285,8 @@ moe_status forward_impl(const moe_shape* s, const void* x, const void* packed, c
   if ((r = build_map(s, expert_rank_host, &map)) != MOE_OK) return r;
   if (s->T == 0) return MOE_OK;
   if (!x || !packed || !y || (routed && !r_idx)) return MOE_ERR_INVALID_ARG;
-  if (!aligned(x, 16) || !aligned(y, 16) || !aligned(packed, kAlign) || (bias && !aligned(bias, 4)))
+  if (!aligned(x, 16) || !aligned(y, 16) || !aligned(packed, kAlign) || (bias && !aligned(bias, 4)) ||
+      (sel_bias && !aligned(sel_bias, 4)))
     return MOE_ERR_ALIGNMENT;
   if (routed && (!aligned(r_idx, 4) || (r_gate && !aligned(r_gate, 4)))) return MOE_ERR_ALIGNMENT;
   FwdBufs f = carve_forward(s, ws, buffers);
@@ -320,6 +324,7 @@ moe_status forward_impl(const moe_shape* s, const void* x, const void* packed, c
     a.x = x;
     a.wrT = pk.wrT;
     a.bias = bias;
+    a.sel_bias = sel_bias;
     a.T = s->T;
     a.d = s->d;
     a.E = s->E;
@@ -340,7 +345,8 @@ moe_status forward_impl(const moe_shape* s, const void* x, const void* packed, c
       return r;
     if ((r = mark(2)) != MOE_OK) return r;
   } else {
-    if ((r = do_route(s, x, &pk, bias, f.logits, f.idx, f.gate, sc.ctl, st)) != MOE_OK) return r;
+    if ((r = do_route(s, x, &pk, bias, sel_bias, f.logits, f.idx, f.gate, sc.ctl, st)) != MOE_OK)
+      return r;
     if ((r = mark(1)) != MOE_OK) return r;
     if ((r = do_layout(s, f.idx, map, &f.lay, sc, -1, kWaitLimitNs, st)) != MOE_OK) return r;
     if ((r = mark(2)) != MOE_OK) return r;
@@ -404,6 +410,25 @@ moe_status forward_impl(const moe_shape* s, const void* x, const void* packed, c
                                       y, s->T, s->d, s->k, st))) != MOE_OK)
     return r;
   return mark(6);
+}
+
+moe_status route_impl(const moe_shape* s, const void* x, const void* packed, const float* bias,
+                      const float* sel_bias, float* logits, int32_t* topk_idx, float* topk_gate,
+                      void* ws, size_t ws_bytes, cudaStream_t st) {
+  moe_status r = check_shape(s);
+  if (r != MOE_OK) return r;
+  if (s->T > 0 && (!logits || !topk_idx || !topk_gate)) return MOE_ERR_INVALID_ARG;
+  if (x && (!packed || !ws)) return MOE_ERR_INVALID_ARG;
+  if ((x && !aligned(x, 16)) || (packed && !aligned(packed, kAlign)) || !aligned(logits, 4) ||
+      !aligned(topk_idx, 4) || !aligned(topk_gate, 4) || (bias && !aligned(bias, 4)) ||
+      (sel_bias && !aligned(sel_bias, 4)) || (ws && !aligned(ws, kAlign)))
+    return MOE_ERR_ALIGNMENT;
+  if (ws && ws_bytes < scratch_bytes(s)) return MOE_ERR_WORKSPACE;
+  if (s->T == 0) return MOE_OK;
+  Packed pk{};
+  if (packed) pk = carve_packed(s, packed);
+  Control* ctl = ws ? carve_scratch(s, ws).ctl : nullptr;
+  return do_route(s, x, &pk, bias, sel_bias, logits, topk_idx, topk_gate, ctl, st);
 }
 
 }  // namespace
@@ -474,20 +499,61 @@ moe_status moe_pack_weights(const moe_shape* s, const void* w_router, const void
 moe_status moe_route(const moe_shape* s, const void* x, const void* packed, const float* bias,
                      float* logits, int32_t* topk_idx, float* topk_gate, void* ws,
                      size_t ws_bytes, moe_stream_t stream) {
+  return route_impl(s, x, packed, bias, nullptr, logits, topk_idx, topk_gate, ws, ws_bytes,
+                    (cudaStream_t)stream);
+}
+
+moe_status moe_route_selection_bias(const moe_shape* s, const void* x, const void* packed,
+                                    const float* bias, const float* selection_bias, float* logits,
+                                    int32_t* topk_idx, float* topk_gate, void* ws, size_t ws_bytes,
+                                    moe_stream_t stream) {
+  if (!selection_bias) return MOE_ERR_INVALID_ARG;
+  return route_impl(s, x, packed, bias, selection_bias, logits, topk_idx, topk_gate, ws, ws_bytes,
+                    (cudaStream_t)stream);
+}
+
+moe_status moe_router_stats(const moe_shape* s, const float* logits, const float* selection_bias,
+                            const int32_t* topk_idx, const int32_t* recorded_idx, double threshold,
+                            double* margin, moe_router_counts* stats, moe_stream_t stream) {
   moe_status r = check_shape(s);
   if (r != MOE_OK) return r;
-  if (s->T > 0 && (!logits || !topk_idx || !topk_gate)) return MOE_ERR_INVALID_ARG;
-  if (x && (!packed || !ws)) return MOE_ERR_INVALID_ARG;
-  if ((x && !aligned(x, 16)) || (packed && !aligned(packed, kAlign)) || !aligned(logits, 4) ||
-      !aligned(topk_idx, 4) || !aligned(topk_gate, 4) || (bias && !aligned(bias, 4)) ||
-      (ws && !aligned(ws, kAlign)))
+  if (!stats || (s->T > 0 && !logits) || (recorded_idx && !topk_idx)) return MOE_ERR_INVALID_ARG;
+  if (!(threshold >= 0.0)) return MOE_ERR_INVALID_ARG;
+  if (!aligned(stats, 8) || (logits && !aligned(logits, 4)) || (margin && !aligned(margin, 8)) ||
+      (selection_bias && !aligned(selection_bias, 4)) || (topk_idx && !aligned(topk_idx, 4)) ||
+      (recorded_idx && !aligned(recorded_idx, 4)))
     return MOE_ERR_ALIGNMENT;
-  if (ws && ws_bytes < scratch_bytes(s)) return MOE_ERR_WORKSPACE;
+  cudaStream_t st = (cudaStream_t)stream;
+  // the kernel writes the token count and adds to the other counters
+  static_assert(sizeof(moe_router_counts) == 5 * sizeof(unsigned long long), "five counters");
+  if (cudaMemsetAsync(stats, 0, sizeof(moe_router_counts), st) != cudaSuccess) return MOE_ERR_CUDA;
+  return cuda_status(launch_router_stats(logits, selection_bias, s->T, s->E, s->k, topk_idx,
+                                         recorded_idx, threshold, margin,
+                                         reinterpret_cast<unsigned long long*>(stats), st));
+}
+
+moe_status moe_capacity_keep(const moe_shape* s, const int32_t* topk_idx, const float* topk_gate,
+                             double capacity_factor, int32_t* keep, float* kept_gate,
+                             int64_t* capacity, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status r = check_shape(s);
+  if (r != MOE_OK) return r;
+  if (!(capacity_factor > 0.0) || !(capacity_factor < 1e9) || !ws) return MOE_ERR_INVALID_ARG;
+  // the factor times an expert's mean load, rounded up
+  const int64_t cap = (int64_t)std::ceil(capacity_factor * (double)s->T * s->k / s->E);
+  if (capacity) *capacity = cap;
   if (s->T == 0) return MOE_OK;
-  Packed pk{};
-  if (packed) pk = carve_packed(s, packed);
-  Control* ctl = ws ? carve_scratch(s, ws).ctl : nullptr;
-  return do_route(s, x, &pk, bias, logits, topk_idx, topk_gate, ctl, (cudaStream_t)stream);
+  if (!topk_idx || !keep) return MOE_ERR_INVALID_ARG;
+  if (!aligned(topk_idx, 4) || !aligned(keep, 4) || (topk_gate && !aligned(topk_gate, 4)) ||
+      (kept_gate && !aligned(kept_gate, 4)) || !aligned(ws, kAlign))
+    return MOE_ERR_ALIGNMENT;
+  if (ws_bytes < scratch_bytes(s)) return MOE_ERR_WORKSPACE;
+  cudaStream_t st = (cudaStream_t)stream;
+  const size_t R = (size_t)s->T * s->k;
+  // entries with an out-of-range expert are written by no block: they read 0
+  if (cudaMemsetAsync(keep, 0, R * 4, st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (kept_gate && cudaMemsetAsync(kept_gate, 0, R * 4, st) != cudaSuccess) return MOE_ERR_CUDA;
+  return cuda_status(launch_capacity_keep(topk_idx, s->T, s->k, s->E, cap, topk_gate, keep,
+                                          kept_gate, carve_scratch(s, ws).ctl, st));
 }
 
 moe_status moe_dispatch_layout(const moe_shape* s, const int32_t* topk_idx,
@@ -561,6 +627,16 @@ moe_status moe_forward(const moe_shape* s, const void* x, const void* packed, co
                        void* ws, size_t ws_bytes, moe_stream_t stream) {
   return forward_impl(s, x, packed, bias, expert_rank_host, y, buffers, ws, ws_bytes,
                       (cudaStream_t)stream, nullptr);
+}
+
+moe_status moe_forward_selection_bias(const moe_shape* s, const void* x, const void* packed,
+                                      const float* bias, const float* selection_bias,
+                                      const int32_t* expert_rank_host, void* y,
+                                      const moe_forward_buffers* buffers, void* ws,
+                                      size_t ws_bytes, moe_stream_t stream) {
+  if (!selection_bias) return MOE_ERR_INVALID_ARG;
+  return forward_impl(s, x, packed, bias, expert_rank_host, y, buffers, ws, ws_bytes,
+                      (cudaStream_t)stream, nullptr, false, nullptr, nullptr, selection_bias);
 }
 
 moe_status moe_forward_routed(const moe_shape* s, const void* x, const void* packed,

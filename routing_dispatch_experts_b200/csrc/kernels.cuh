@@ -61,8 +61,9 @@ struct RankMap {
 };
 
 // ---- route.cu
-cudaError_t launch_topk(const float* logits, int64_t T, int E, int k, int32_t* idx, float* gate,
-                        cudaStream_t s);
+// sel_bias [E] or NULL: added to the logits for the choice of experts only
+cudaError_t launch_topk(const float* logits, const float* sel_bias, int64_t T, int E, int k,
+                        int32_t* idx, float* gate, cudaStream_t s);
 cudaError_t launch_router_f32(const float* x, const float* wrT, const float* bias, int64_t T,
                               int d, int E, float* logits, cudaStream_t s);
 
@@ -141,6 +142,7 @@ struct RouteArgs {
   const void* x;        // [T, d] bf16
   const void* wrT;      // [E16, d] bf16 (packed router)
   const float* bias;    // [E] or NULL
+  const float* sel_bias = nullptr;  // [E] or NULL: added for the choice of experts only
   int64_t T;
   int d, E, k;
   float* logits;        // [T, E]
@@ -179,6 +181,24 @@ cudaError_t launch_ffn_fused(const FfnArgs& a, cudaStream_t s);
 cudaError_t launch_grouped_f32_part(int part, const float* x_perm, const int32_t* offsets, int E,
                                     int64_t R, int d, int f, int blk, const float* wgu,
                                     const float* wdT, float* h, float* y_perm, cudaStream_t s);
+
+// ---- route_stats.cu
+// Router statistics of a routing: margin [T] (double, may be NULL); counts[0]
+// = T, and four counters added to counts[1..4] (zeroed by the caller):
+// tokens with margin below `threshold`; against `recorded` (may be NULL) the
+// tokens whose expert set changed, the experts swapped and the slots that
+// differ.
+cudaError_t launch_router_stats(const float* logits, const float* sel_bias, int64_t T, int E,
+                                int k, const int32_t* idx, const int32_t* recorded,
+                                double threshold, double* margin, unsigned long long* counts,
+                                cudaStream_t s);
+// Expert capacity: keep[a] = 1 for the first `cap` assignments of each
+// expert in (choice rank, token) order, else 0; kept_gate[a] = gate[a] (1
+// when gate is NULL) where kept, 0 where dropped (may be NULL).  Entries of
+// out-of-range indices are not written (MOE_ERR_DEVICE_INDEX in ctl).
+cudaError_t launch_capacity_keep(const int32_t* idx, int64_t T, int k, int E, int64_t cap,
+                                 const float* gate, int32_t* keep, float* kept_gate, Control* ctl,
+                                 cudaStream_t s);
 
 // ---- pack.cu
 cudaError_t launch_pack(int dtype, int d, int E, int f, int blk, int E16, const void* w_router,

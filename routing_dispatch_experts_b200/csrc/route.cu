@@ -16,8 +16,13 @@ namespace moe {
 // resolve to the lower index because the comparison is the IEEE one.
 // Gates: softmax of the chosen logits, exp(l_j - l_0) / sum_i exp(l_i - l_0),
 // the sum reduced by the same butterfly in every lane (deterministic).
+// With a selection bias b[E] the experts are chosen on the fp32 sum l + b
+// and the gates still come from the chosen experts' l (the auxiliary-loss-
+// free router of "Expert Coupling in MoE Pretraining", Fig. 11: a per-expert
+// bias steers which experts are picked, not how their outputs are weighted).
 template <int VPL>
-__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int64_t T,
+__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits,
+                                                   const float* __restrict__ sel_bias, int64_t T,
                                                    int E, int k, int32_t* __restrict__ idx,
                                                    float* __restrict__ gate) {
   const int lane = threadIdx.x & 31;
@@ -25,11 +30,12 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
   pdl_wait();
   if (t >= T) return;  // uniform per warp
   const float* row = logits + t * E;
-  float v[VPL];
+  float v[VPL], key[VPL];
 #pragma unroll
   for (int c = 0; c < VPL; ++c) {
     const int e = lane + 32 * c;
     v[c] = e < E ? __ldg(row + e) : 0.f;
+    key[c] = (sel_bias && e < E) ? v[c] + __ldg(sel_bias + e) : v[c];
   }
   uint32_t taken = 0;
   float my_l = 0.f;
@@ -41,8 +47,8 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
     for (int c = 0; c < VPL; ++c) {
       const int e = lane + 32 * c;
       if (e < E && !((taken >> c) & 1u)) {
-        if (bi == 0x7FFFFFFF || v[c] > bv) {  // e ascending: keep the first of equals
-          bv = v[c];
+        if (bi == 0x7FFFFFFF || key[c] > bv) {  // e ascending: keep the first of equals
+          bv = key[c];
           bi = e;
         }
       }
@@ -57,8 +63,15 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
       }
     }
     if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+    // the winner's own logit (equal to its key without a selection bias),
+    // from the lane that holds it
+    float mine = 0.f;
+#pragma unroll
+    for (int c = 0; c < VPL; ++c)
+      if (c == (bi >> 5)) mine = v[c];
+    const float raw = __shfl_sync(0xffffffffu, mine, bi & 31);
     if (lane == j) {
-      my_l = bv;
+      my_l = raw;
       my_e = bi;
     }
   }
@@ -73,16 +86,17 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
   }
 }
 
-cudaError_t launch_topk(const float* logits, int64_t T, int E, int k, int32_t* idx, float* gate,
-                        cudaStream_t s) {
+cudaError_t launch_topk(const float* logits, const float* sel_bias, int64_t T, int E, int k,
+                        int32_t* idx, float* gate, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
   const int warps = 8;
   const unsigned grid = (unsigned)((T + warps - 1) / warps);
   const int vpl = (E + 31) / 32;
   switch (vpl) {
-#define MOE_TOPK_CASE(N) \
-  case N:                \
-    return launch_pdl(topk_kernel<N>, dim3(grid), dim3(warps * 32), 0, s, logits, T, E, k, idx, gate);
+#define MOE_TOPK_CASE(N)                                                                    \
+  case N:                                                                                   \
+    return launch_pdl(topk_kernel<N>, dim3(grid), dim3(warps * 32), 0, s, logits, sel_bias, \
+                      T, E, k, idx, gate);
     MOE_TOPK_CASE(1)
     MOE_TOPK_CASE(2)
     MOE_TOPK_CASE(3)

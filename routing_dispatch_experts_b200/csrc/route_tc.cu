@@ -47,6 +47,7 @@ struct Params {
   int64_t T;
   int K, E, BN, k;
   const float* bias;
+  const float* sel_bias;  // [E] or NULL: added for the choice of experts only
   float* logits;
   int32_t* idx;
   float* gate;
@@ -98,6 +99,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   __shared__ uint32_t tmem_base_s;
   __shared__ int hist[kMaxBins];
   __shared__ float s_bias[256];
+  __shared__ float s_sbias[256];
   __shared__ uint8_t s_map[256];
   __shared__ volatile int abort_flag;
 
@@ -191,8 +193,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     // predecessor's completion, like every input)
     for (int i = threadIdx.x - 64; i < p.E; i += 32 * kEpiWarps) {
       s_bias[i] = p.bias ? __ldg(p.bias + i) : 0.f;
+      s_sbias[i] = p.sel_bias ? __ldg(p.sel_bias + i) : 0.f;
       s_map[i] = p.map.r[i];
     }
+    const bool sel = p.sel_bias != nullptr;
     named_bar_sync(1, 32 * kEpiWarps);
     float tv[KMAX];
     int ti[KMAX];
@@ -246,9 +250,10 @@ __global__ void __launch_bounds__(kThreads, 2)
           for (int i = 0; i < 16; ++i)
             if (c + i < p.E) lrow[c + i] = v[i];
         }
+        // the key: the logit, plus the selection bias when there is one
 #pragma unroll
         for (int i = 0; i < 16; ++i)
-          if (c + i < p.E) topk_insert<KMAX>(tv, ti, v[i], c + i);
+          if (c + i < p.E) topk_insert<KMAX>(tv, ti, sel ? v[i] + s_sbias[c + i] : v[i], c + i);
       }
     }
     // parts 1.. leave their lists for part 0 in shared memory
@@ -290,6 +295,24 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int j = 0; j < KMAX; ++j)
           topk_insert<KMAX>(tv, ti, m_v[(pp * BM + rr) * KMAX + j], m_i[(pp * BM + rr) * KMAX + j]);
       if (have && valid) {
+        if (sel) {
+          // gates from the chosen experts' own logits, read back from the
+          // staged tile (or, in mode 0, from this CTA's global stores; the
+          // barrier above ordered them) in place of the biased keys
+#pragma unroll
+          for (int j = 0; j < KMAX; ++j)
+            if (j < p.k) {
+              const int col = ti[j];
+              if (mode == 2)
+                tv[j] = *reinterpret_cast<const float*>(
+                    smem + (size_t)(col >> 5) * (BM * 128) + rr * 128 +
+                    (((((col & 31) >> 2) ^ (rr & 7))) << 4) + (col & 3) * 4);
+              else if (mode == 1)
+                tv[j] = *reinterpret_cast<const float*>(smem + (size_t)rr * lstride + col * 4);
+              else
+                tv[j] = lrow[col];
+            }
+        }
         float ex[KMAX];
         float z = 0.f;
 #pragma unroll
@@ -364,6 +387,7 @@ cudaError_t launch_route_tc(const RouteArgs& a, cudaStream_t s) {
   p.BN = (a.E + 15) / 16 * 16;
   p.k = a.k;
   p.bias = a.bias;
+  p.sel_bias = a.sel_bias;
   p.logits = a.logits;
   p.idx = a.idx;
   p.gate = a.gate;

@@ -174,6 +174,8 @@ def _c_kind(param: str) -> str:
         return "ptr"
     if p.startswith(("size_t", "const size_t")):
         return "size"
+    if p.startswith(("double", "const double")):
+        return "f64"
     if "int64_t" in p:
         return "i64"
     if p.startswith(("int32_t", "int ", "const int32_t", "moe_status", "moe_dtype")):
@@ -186,6 +188,8 @@ def _py_kind(t) -> str:
         return "ptr"
     if t is ctypes.c_size_t:
         return "size"
+    if t is ctypes.c_double:
+        return "f64"
     if ctypes.sizeof(t) == 8:
         return "i64"
     if ctypes.sizeof(t) == 4:
@@ -218,6 +222,7 @@ def test_struct_layouts_match_the_header(tmp_path):
         "moe_shape": [f for f, _ in moe.moe_shape._fields_],
         "moe_layout": [f for f, _ in moe.moe_layout._fields_],
         "moe_forward_buffers": [f for f, _ in moe.moe_forward_buffers._fields_],
+        "moe_router_counts": [f for f, _ in moe.moe_router_counts._fields_],
         "moe_stats": ["rows_sent", "dup_removed", "tokens_single_rank", "home_rank_rows",
                       "max_expert_rows", "min_expert_rows"],
     }
@@ -236,7 +241,8 @@ def test_struct_layouts_match_the_header(tmp_path):
         s, f, v = line.split()
         got[(s, f)] = int(v)
     for s, cls in (("moe_shape", moe.moe_shape), ("moe_layout", moe.moe_layout),
-                   ("moe_forward_buffers", moe.moe_forward_buffers)):
+                   ("moe_forward_buffers", moe.moe_forward_buffers),
+                   ("moe_router_counts", moe.moe_router_counts)):
         assert got[(s, "size")] == ctypes.sizeof(cls), s
         for f in structs[s]:
             assert got[(s, f)] == getattr(cls, f).offset, (s, f)
