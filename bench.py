@@ -533,7 +533,7 @@ def run_reference(args, rank, world):
 
 # ------------------------------------------------- one kernel, for profilers
 KERNELS = ("route", "topk", "layout", "permute", "permute_by_token", "grouped",
-           "grouped_gather", "combine", "forward")
+           "grouped_gather", "combine", "forward", "stats", "capacity")
 
 
 def run_kernel(args):
@@ -549,6 +549,8 @@ def run_kernel(args):
       grouped_gather   moe_grouped_swiglu_gather
       combine          moe_combine
       forward          moe_forward
+      stats            moe_router_stats (margin, near-tie count)
+      capacity         moe_capacity_keep (capacity factor 1.25)
 
     Routing comes from the workload's own router on its own x; expert
     weights are seeded N(0, 1/d) stand-ins drawn on the device (values do
@@ -595,6 +597,7 @@ def run_kernel(args):
         else torch.empty((T, w.d), dtype=w.torch_dtype, device=dev)
     idx2 = torch.empty_like(idx)
     gate2 = torch.empty_like(gate)
+    counts = torch.zeros(5, dtype=torch.int64, device=dev)
     clay = moe._c_layout(moe._layout_tensors(shape, dev))
     rmap = None
 
@@ -623,6 +626,12 @@ def run_kernel(args):
                                             P(y_perm), P(ws), ws.numel(), st)
         elif k == "combine":
             r = L.moe_combine(ctypes.byref(sc), P(y_perm), P(lay["slot_row"]), P(gate), P(out), st)
+        elif k == "stats":
+            r = L.moe_router_stats(ctypes.byref(sc), P(logits), None, P(idx), None, 1e-5, None,
+                                   P(counts), st)
+        elif k == "capacity":
+            r = L.moe_capacity_keep(ctypes.byref(sc), P(idx), P(gate), 1.25, P(idx2), P(gate2),
+                                    None, P(ws), ws.numel(), st)
         else:
             r = L.moe_forward(ctypes.byref(sc), P(x), P(packed), P(bias), rmap, P(out), None,
                               P(ws), ws.numel(), st)
