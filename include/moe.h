@@ -219,6 +219,42 @@ MOE_API moe_status moe_route(const moe_shape* shape, const void* x, const void* 
                      moe_stream_t stream);
 
 /*
+ * The router and the expert FFN on weights in the pages' own layouts, for
+ * callers that keep the weights as [d, E] ("ME") for the router and
+ * [E, d, f] ("EMH") / [E, f, d] ("EHM") for the experts ("Revisiting MoE and
+ * Dense Speed-Accuracy Comparisons", Table 1).  Each call first packs the
+ * weights it reads into the workspace (the transposes moe_pack_weights does
+ * once), then runs the packed path, so its results are bit-identical to
+ * moe_route / moe_grouped_swiglu on moe_pack_weights output.  Packing on
+ * every call moves every weight byte twice more: pack once with
+ * moe_pack_weights where the weights do not change between calls.
+ *  ws, ws_bytes  at least moe_unpacked_workspace_size bytes (the scratch
+ *                workspace followed by room for the packed weights),
+ *                zero-filled once before first use like the scratch
+ */
+MOE_API moe_status moe_unpacked_workspace_size(const moe_shape* shape, size_t* bytes);
+
+/*
+ * moe_route with W_r [d, E] ("ME") in the shape's dtype (device) in place of
+ * the packed buffer; x must not be NULL.  Other arguments as in moe_route.
+ */
+MOE_API moe_status moe_route_unpacked(const moe_shape* shape, const void* x,
+                                      const void* w_router, const float* bias, float* logits,
+                                      int32_t* topk_idx, float* topk_gate, void* ws,
+                                      size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * moe_grouped_swiglu with W_g, W_u [E, d, f] ("EMH") and W_d [E, f, d]
+ * ("EHM") in the shape's dtype (device) in place of the packed buffer.
+ * Other arguments as in moe_grouped_swiglu.
+ */
+MOE_API moe_status moe_grouped_swiglu_unpacked(const moe_shape* shape, const void* x_perm,
+                                               const int32_t* expert_offsets,
+                                               const void* w_gate, const void* w_up,
+                                               const void* w_down, void* h, void* y_perm,
+                                               void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
  * moe_route with a selection-only expert bias: the experts are chosen on the
  * fp32 sum logits + selection_bias (same key and tie-break as moe_route),
  * and the gates are the softmax of the chosen experts' logits WITHOUT the
@@ -330,6 +366,38 @@ MOE_API moe_status moe_dispatch_layout(const moe_shape* shape, const int32_t* to
                                const int32_t* expert_rank_host,
                                const moe_layout* out, void* ws, size_t ws_bytes,
                                moe_stream_t stream);
+
+/*
+ * Co-selection counts of a routing ("Expert Coupling in MoE Pretraining",
+ * Table III: W[e,e'], how often experts e and e' are selected by the same
+ * token; the statistic its correlated placement is fit on):
+ *   counts[e * E + e'] = number of ordered slot pairs (j, j'), j != j', of a
+ *                        token with topk_idx[t,j] = e and topk_idx[t,j'] = e'
+ * which, for a routing of distinct experts, is the number of tokens that
+ * select both.  Integer counts, identical on every run.
+ *  topk_idx [T, k] int32 (device); counts [E * E] uint64 (device, 8-byte
+ *  aligned, overwritten); ws scratch workspace (moe_scratch_size).  A token
+ *  with an index outside [0, E) adds nothing and sets MOE_ERR_DEVICE_INDEX.
+ */
+MOE_API moe_status moe_coselection_counts(const moe_shape* shape, const int32_t* topk_idx,
+                                          uint64_t* counts, void* ws, size_t ws_bytes,
+                                          moe_stream_t stream);
+
+/*
+ * Correlated expert placement fit on co-selection counts ("Expert Coupling
+ * in MoE Pretraining", Abstract: experts often selected together are placed
+ * on the same GPU; Table I caption: fit on other iterations than those it is
+ * measured on).  Host code, no GPU: rank r = 0, 1, ... in turn takes the
+ * unassigned expert with the largest row sum of counts, then, until it holds
+ * E/ep experts, the unassigned expert with the largest total count with the
+ * experts the rank already holds (ties: the lowest expert index).
+ *  counts_host      [E * E] uint64 in HOST memory (moe_coselection_counts,
+ *                   copied back)
+ *  expert_rank_host [E] int32 HOST output: a partition with E/ep experts per
+ *                   rank, ready for moe_dispatch_layout / moe_forward
+ */
+MOE_API moe_status moe_fit_placement(int32_t E, int32_t ep, const uint64_t* counts_host,
+                                     int32_t* expert_rank_host);
 
 /*
  * Permute (gather): x_perm[r] = x[row_token[r]] for r < T*k, whole rows
@@ -523,6 +591,22 @@ MOE_API moe_status moe_debug_dispatch_layout_stall(const moe_shape* shape,
                                            size_t ws_bytes, int32_t stall_block,
                                            int64_t wait_limit_ns,
                                            moe_stream_t stream);
+
+/*
+ * Test and measurement hook of moe_grouped_swiglu: the same call with the
+ * tensor-core GEMM engine chosen by the caller.
+ *  engine 0  the library's choice (what moe_grouped_swiglu runs)
+ *         1  one CTA per 128-row tile
+ *         2  CTA pairs on 256-row tiles (tcgen05 cta_group::2) where the
+ *            shape allows it (bf16, 256-column tiles), else as 1
+ * All engines sum every output in the same order, so h and y_perm are
+ * bit-identical across engines.  MOE_ERR_INVALID_ARG for another engine.
+ */
+MOE_API moe_status moe_debug_grouped_swiglu_engine(const moe_shape* shape, const void* x_perm,
+                                                   const int32_t* expert_offsets,
+                                                   const void* packed, void* h, void* y_perm,
+                                                   void* ws, size_t ws_bytes, int32_t engine,
+                                                   moe_stream_t stream);
 
 /*
  * moe_dispatch_layout for callers that cannot allocate device memory.

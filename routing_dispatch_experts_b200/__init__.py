@@ -83,11 +83,12 @@ _lib = None
 # exported C symbols, in header order (checked against include/moe.h by the tests)
 SYMBOLS = ("moe_status_string", "moe_scratch_size", "moe_forward_workspace_size",
            "moe_workspace_init", "moe_packed_weights_size", "moe_pack_weights", "moe_route",
+           "moe_unpacked_workspace_size", "moe_route_unpacked", "moe_grouped_swiglu_unpacked",
            "moe_route_selection_bias", "moe_router_stats", "moe_capacity_keep",
-           "moe_dispatch_layout", "moe_permute", "moe_permute_by_token", "moe_grouped_swiglu",
+           "moe_dispatch_layout", "moe_coselection_counts", "moe_fit_placement", "moe_permute", "moe_permute_by_token", "moe_grouped_swiglu",
            "moe_grouped_swiglu_gather", "moe_combine", "moe_forward", "moe_forward_selection_bias", "moe_forward_timed",
            "moe_forward_routed", "moe_get_device_status", "moe_debug_dispatch_layout_stall",
-           "moe_dispatch_layout_static")
+           "moe_debug_grouped_swiglu_engine", "moe_dispatch_layout_static")
 FORWARD_STAGES = ("route", "layout", "permute", "gate_up", "down", "combine")
 
 
@@ -109,6 +110,10 @@ def lib() -> ctypes.CDLL:
             "moe_packed_weights_size": ([S, sz], ctypes.c_int),
             "moe_pack_weights": ([S, P, P, P, P, P, ctypes.c_size_t, P], ctypes.c_int),
             "moe_route": ([S, P, P, P, P, P, P, P, ctypes.c_size_t, P], ctypes.c_int),
+            "moe_unpacked_workspace_size": ([S, sz], ctypes.c_int),
+            "moe_route_unpacked": ([S, P, P, P, P, P, P, P, ctypes.c_size_t, P], ctypes.c_int),
+            "moe_grouped_swiglu_unpacked": ([S, P, P, P, P, P, P, P, P, ctypes.c_size_t, P],
+                                            ctypes.c_int),
             "moe_route_selection_bias": ([S, P, P, P, P, P, P, P, P, ctypes.c_size_t, P],
                                          ctypes.c_int),
             "moe_router_stats": ([S, P, P, P, P, ctypes.c_double, P, P, P], ctypes.c_int),
@@ -116,6 +121,8 @@ def lib() -> ctypes.CDLL:
                                    P, ctypes.c_size_t, P], ctypes.c_int),
             "moe_dispatch_layout": ([S, P, P, ctypes.POINTER(moe_layout), P, ctypes.c_size_t, P],
                                     ctypes.c_int),
+            "moe_coselection_counts": ([S, P, P, P, ctypes.c_size_t, P], ctypes.c_int),
+            "moe_fit_placement": ([ctypes.c_int32, ctypes.c_int32, P, P], ctypes.c_int),
             "moe_permute": ([S, P, P, P, P], ctypes.c_int),
             "moe_permute_by_token": ([S, P, P, P, P], ctypes.c_int),
             "moe_grouped_swiglu": ([S, P, P, P, P, P, P, ctypes.c_size_t, P], ctypes.c_int),
@@ -136,6 +143,8 @@ def lib() -> ctypes.CDLL:
                                                  ctypes.c_size_t, ctypes.c_int32, ctypes.c_int64, P],
                                                 ctypes.c_int),
             "moe_dispatch_layout_static": ([S, P, P, ctypes.POINTER(moe_layout), P, P], ctypes.c_int),
+            "moe_debug_grouped_swiglu_engine": ([S, P, P, P, P, P, P, ctypes.c_size_t,
+                                                 ctypes.c_int32, P], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -282,6 +291,49 @@ def route(shape: Shape, x, packed, bias, ws, logits=None, stream=None):
     return logits, idx, gate
 
 
+def unpacked_workspace(shape: Shape, device="cuda") -> torch.Tensor:
+    """A zero-filled workspace for the *_unpacked calls."""
+    n = ctypes.c_size_t()
+    s = shape.c
+    _check(lib().moe_unpacked_workspace_size(ctypes.byref(s), ctypes.byref(n)),
+           "moe_unpacked_workspace_size")
+    return torch.zeros(n.value, dtype=torch.uint8, device=device)
+
+
+def route_unpacked(shape: Shape, x, w_router, bias, ws, stream=None):
+    """moe_route_unpacked: the router on W_r [d, E]; (logits, idx, gate)."""
+    _need(x, shape.dtype, (shape.T, shape.d), "x")
+    _need(w_router, shape.dtype, (shape.d, shape.E), "w_router")
+    _need_bias(shape, bias)
+    dev = ws.device
+    logits = torch.empty((shape.T, shape.E), dtype=torch.float32, device=dev)
+    idx = torch.empty((shape.T, shape.k), dtype=torch.int32, device=dev)
+    gate = torch.empty((shape.T, shape.k), dtype=torch.float32, device=dev)
+    s = shape.c
+    _check(lib().moe_route_unpacked(ctypes.byref(s), _p(x), _p(w_router), _p(bias), _p(logits),
+                                    _p(idx), _p(gate), _p(ws), ws.numel(), _stream(stream)),
+           "moe_route_unpacked")
+    return logits, idx, gate
+
+
+def grouped_swiglu_unpacked(shape: Shape, x_perm, expert_offsets, w_gate, w_up, w_down, ws,
+                            stream=None):
+    """moe_grouped_swiglu_unpacked: (h, y_perm) from W_g/W_u [E,d,f], W_d [E,f,d]."""
+    _need(x_perm, shape.dtype, (shape.R, shape.d), "x_perm")
+    _need_n(expert_offsets, torch.int32, shape.E + 1, "expert_offsets")
+    _need(w_gate, shape.dtype, (shape.E, shape.d, shape.f), "w_gate")
+    _need(w_up, shape.dtype, (shape.E, shape.d, shape.f), "w_up")
+    _need(w_down, shape.dtype, (shape.E, shape.f, shape.d), "w_down")
+    h = torch.empty((shape.R, shape.f), dtype=shape.dtype, device=x_perm.device)
+    y_perm = torch.empty((shape.R, shape.d), dtype=shape.dtype, device=x_perm.device)
+    s = shape.c
+    _check(lib().moe_grouped_swiglu_unpacked(ctypes.byref(s), _p(x_perm), _p(expert_offsets),
+                                             _p(w_gate), _p(w_up), _p(w_down), _p(h), _p(y_perm),
+                                             _p(ws), ws.numel(), _stream(stream)),
+           "moe_grouped_swiglu_unpacked")
+    return h, y_perm
+
+
 def route_selection_bias(shape: Shape, x, packed, bias, selection_bias, ws, logits=None,
                          stream=None):
     """moe_route_selection_bias: experts chosen on logits + selection_bias,
@@ -420,6 +472,31 @@ def dispatch_layout_static(shape: Shape, topk_idx, expert_rank=None, stream=None
     return out, status
 
 
+def coselection_counts(shape: Shape, topk_idx, ws, stream=None) -> torch.Tensor:
+    """moe_coselection_counts: W [E, E] (uint64 counts held in an int64
+    tensor on the device)."""
+    _need(topk_idx, torch.int32, (shape.T, shape.k), "topk_idx")
+    W = torch.empty((shape.E, shape.E), dtype=torch.int64, device=topk_idx.device)
+    s = shape.c
+    _check(lib().moe_coselection_counts(ctypes.byref(s), _p(topk_idx), _p(W), _p(ws), ws.numel(),
+                                        _stream(stream)), "moe_coselection_counts")
+    return W
+
+
+def fit_placement(E: int, ep: int, counts) -> list:
+    """moe_fit_placement on counts [E, E] (any int64 tensor or array; copied
+    to the host): returns the expert -> rank map as a list."""
+    import numpy as np
+    c = np.ascontiguousarray(counts.cpu().numpy() if isinstance(counts, torch.Tensor) else counts,
+                             dtype=np.uint64)
+    if c.shape != (E, E):
+        raise ValueError(f"counts: expected ({E}, {E}), got {c.shape}")
+    out = (ctypes.c_int32 * E)()
+    _check(lib().moe_fit_placement(E, ep, c.ctypes.data_as(ctypes.c_void_p), out),
+           "moe_fit_placement")
+    return list(out)
+
+
 def permute(shape: Shape, x, row_token, stream=None):
     _need(x, shape.dtype, (shape.T, shape.d), "x")
     _need_n(row_token, torch.int32, shape.R, "row_token")
@@ -441,17 +518,26 @@ def permute_by_token(shape: Shape, x, slot_row, stream=None):
     return x_perm
 
 
-def grouped_swiglu(shape: Shape, x_perm, expert_offsets, packed, ws, stream=None):
-    """moe_grouped_swiglu: returns (h [R,f], y_perm [R,d])."""
+def grouped_swiglu(shape: Shape, x_perm, expert_offsets, packed, ws, stream=None, engine=None):
+    """moe_grouped_swiglu: returns (h [R,f], y_perm [R,d]).  engine (test
+    hook, moe_debug_grouped_swiglu_engine): 1 = one CTA per tile, 2 = CTA
+    pairs."""
     _need(x_perm, shape.dtype, (shape.R, shape.d), "x_perm")
     _need_n(expert_offsets, torch.int32, shape.E + 1, "expert_offsets")
     _need_packed(shape, packed)
     h = torch.empty((shape.R, shape.f), dtype=shape.dtype, device=x_perm.device)
     y_perm = torch.empty((shape.R, shape.d), dtype=shape.dtype, device=x_perm.device)
     s = shape.c
-    _check(lib().moe_grouped_swiglu(ctypes.byref(s), _p(x_perm), _p(expert_offsets), _p(packed),
-                                    _p(h), _p(y_perm), _p(ws), ws.numel(), _stream(stream)),
-           "moe_grouped_swiglu")
+    if engine is None:
+        _check(lib().moe_grouped_swiglu(ctypes.byref(s), _p(x_perm), _p(expert_offsets),
+                                        _p(packed), _p(h), _p(y_perm), _p(ws), ws.numel(),
+                                        _stream(stream)), "moe_grouped_swiglu")
+    else:
+        _check(lib().moe_debug_grouped_swiglu_engine(ctypes.byref(s), _p(x_perm),
+                                                     _p(expert_offsets), _p(packed), _p(h),
+                                                     _p(y_perm), _p(ws), ws.numel(), int(engine),
+                                                     _stream(stream)),
+               "moe_debug_grouped_swiglu_engine")
     return h, y_perm
 
 

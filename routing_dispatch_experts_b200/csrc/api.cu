@@ -199,9 +199,19 @@ moe_status do_layout(const moe_shape* s, const int32_t* idx, const RankMap& map,
 // gate/up GEMM + SwiGLU (part 0) or down GEMM (part 1).  With `gather`
 // (bf16 only) the gate/up GEMM reads its rows straight from x through the
 // permutation instead of from x_perm.
+// Which tensor-core GEMM engine runs a grouped GEMM: the CTA-pair kernel
+// (256-row tiles, gemm_pair.cu) where it applies, else one CTA per tile.
+enum Engine { kEngineAuto = 0, kEngineSingle = 1, kEnginePair = 2 };
+
+cudaError_t launch_gemm(int epi, int bn, const GemmArgs& a, int engine, cudaStream_t st) {
+  if (engine != kEngineSingle && gemm_pair_supported(epi, bn, a)) return launch_gemm_pair(epi, bn, a, st);
+  return launch_gemm_tc(epi, bn, a, st);
+}
+
 moe_status do_grouped_part(int part, const moe_shape* s, const void* a_rows,
                            const int32_t* gather, const int32_t* offsets, const Packed* pk,
-                           void* h, void* y_perm, Control* ctl, cudaStream_t st) {
+                           void* h, void* y_perm, Control* ctl, cudaStream_t st,
+                           int engine = kEngineAuto) {
   const int64_t R = s->T * (int64_t)s->k;
   if (s->dtype == MOE_F32)
     return cuda_status(launch_grouped_f32_part(part, static_cast<const float*>(a_rows), offsets,
@@ -225,7 +235,7 @@ moe_status do_grouped_part(int part, const moe_shape* s, const void* a_rows,
     a.n_out = s->f;
     a.out = h;
     a.ld_out = s->f;
-    return cuda_status(launch_gemm_tc(kEpiSwiGLU, 2 * gu_block(s->f), a, st));
+    return cuda_status(launch_gemm(kEpiSwiGLU, 2 * gu_block(s->f), a, engine, st));
   }
   a.A = h;
   a.B = pk->wdT;
@@ -236,14 +246,15 @@ moe_status do_grouped_part(int part, const moe_shape* s, const void* a_rows,
   a.ld_out = s->d;
   // short K (f <= 512): 128-column tiles, so two CTAs fit per SM
   const int bn = (s->d % 256 == 0 && s->f > 512) ? 256 : (s->d % 128 == 0 ? 128 : 64);
-  return cuda_status(launch_gemm_tc(kEpiBF16, bn, a, st));
+  return cuda_status(launch_gemm(kEpiBF16, bn, a, engine, st));
 }
 
 moe_status do_grouped(const moe_shape* s, const void* x_perm, const int32_t* offsets,
-                      const Packed* pk, void* h, void* y_perm, Control* ctl, cudaStream_t st) {
-  moe_status r = do_grouped_part(0, s, x_perm, nullptr, offsets, pk, h, y_perm, ctl, st);
+                      const Packed* pk, void* h, void* y_perm, Control* ctl, cudaStream_t st,
+                      int engine = kEngineAuto) {
+  moe_status r = do_grouped_part(0, s, x_perm, nullptr, offsets, pk, h, y_perm, ctl, st, engine);
   if (r != MOE_OK) return r;
-  return do_grouped_part(1, s, x_perm, nullptr, offsets, pk, h, y_perm, ctl, st);
+  return do_grouped_part(1, s, x_perm, nullptr, offsets, pk, h, y_perm, ctl, st, engine);
 }
 
 moe_status layout_entry(const moe_shape* s, const int32_t* idx, const int32_t* host_map,
@@ -496,6 +507,60 @@ moe_status moe_pack_weights(const moe_shape* s, const void* w_router, const void
                                  (cudaStream_t)stream));
 }
 
+moe_status moe_unpacked_workspace_size(const moe_shape* s, size_t* bytes) {
+  moe_status r = check_shape(s);
+  if (r != MOE_OK) return r;
+  if (!bytes) return MOE_ERR_INVALID_ARG;
+  *bytes = scratch_bytes(s) + packed_bytes(s);
+  return MOE_OK;
+}
+
+moe_status moe_route_unpacked(const moe_shape* s, const void* x, const void* w_router,
+                              const float* bias, float* logits, int32_t* topk_idx,
+                              float* topk_gate, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status r = check_shape(s);
+  if (r != MOE_OK) return r;
+  if (!x || !w_router || !ws) return MOE_ERR_INVALID_ARG;
+  if (!aligned(w_router, esize(s->dtype)) || !aligned(ws, kAlign)) return MOE_ERR_ALIGNMENT;
+  if (ws_bytes < scratch_bytes(s) + packed_bytes(s)) return MOE_ERR_WORKSPACE;
+  if (s->T == 0) return MOE_OK;
+  // the router block of a packed buffer, built in the workspace after the
+  // scratch, then the packed path
+  void* packed = static_cast<uint8_t*>(ws) + scratch_bytes(s);
+  const Packed pk = carve_packed(s, packed);
+  cudaStream_t st = (cudaStream_t)stream;
+  if ((r = cuda_status(launch_pack(s->dtype, s->d, s->E, s->f, gu_block(s->f), pad16(s->E),
+                                   w_router, nullptr, nullptr, nullptr, const_cast<void*>(pk.wrT),
+                                   nullptr, nullptr, st))) != MOE_OK)
+    return r;
+  return route_impl(s, x, packed, bias, nullptr, logits, topk_idx, topk_gate, ws,
+                    scratch_bytes(s), st);
+}
+
+moe_status moe_grouped_swiglu_unpacked(const moe_shape* s, const void* x_perm,
+                                       const int32_t* offsets, const void* w_gate,
+                                       const void* w_up, const void* w_down, void* h,
+                                       void* y_perm, void* ws, size_t ws_bytes,
+                                       moe_stream_t stream) {
+  moe_status r = check_shape(s);
+  if (r != MOE_OK) return r;
+  if (!w_gate || !w_up || !w_down || !ws) return MOE_ERR_INVALID_ARG;
+  const int es = esize(s->dtype);
+  if (!aligned(w_gate, es) || !aligned(w_up, es) || !aligned(w_down, es) || !aligned(ws, kAlign))
+    return MOE_ERR_ALIGNMENT;
+  if (ws_bytes < scratch_bytes(s) + packed_bytes(s)) return MOE_ERR_WORKSPACE;
+  if (s->T == 0) return MOE_OK;
+  void* packed = static_cast<uint8_t*>(ws) + scratch_bytes(s);
+  const Packed pk = carve_packed(s, packed);
+  cudaStream_t st = (cudaStream_t)stream;
+  if ((r = cuda_status(launch_pack(s->dtype, s->d, s->E, s->f, gu_block(s->f), pad16(s->E),
+                                   nullptr, w_gate, w_up, w_down, nullptr,
+                                   const_cast<void*>(pk.wgu), const_cast<void*>(pk.wdT), st))) !=
+      MOE_OK)
+    return r;
+  return moe_grouped_swiglu(s, x_perm, offsets, packed, h, y_perm, ws, scratch_bytes(s), stream);
+}
+
 moe_status moe_route(const moe_shape* s, const void* x, const void* packed, const float* bias,
                      float* logits, int32_t* topk_idx, float* topk_gate, void* ws,
                      size_t ws_bytes, moe_stream_t stream) {
@@ -556,6 +621,26 @@ moe_status moe_capacity_keep(const moe_shape* s, const int32_t* topk_idx, const 
                                           kept_gate, carve_scratch(s, ws).ctl, st));
 }
 
+moe_status moe_coselection_counts(const moe_shape* s, const int32_t* topk_idx, uint64_t* counts,
+                                  void* ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status r = check_shape(s);
+  if (r != MOE_OK) return r;
+  if (!counts || !ws || (s->T > 0 && !topk_idx)) return MOE_ERR_INVALID_ARG;
+  if (!aligned(counts, 8) || (topk_idx && !aligned(topk_idx, 4)) || !aligned(ws, kAlign))
+    return MOE_ERR_ALIGNMENT;
+  if (ws_bytes < scratch_bytes(s)) return MOE_ERR_WORKSPACE;
+  return cuda_status(launch_coselection(topk_idx, s->T, s->k, s->E, counts,
+                                        carve_scratch(s, ws).ctl, (cudaStream_t)stream));
+}
+
+moe_status moe_fit_placement(int32_t E, int32_t ep, const uint64_t* counts_host,
+                             int32_t* expert_rank_host) {
+  if (E < 1 || E > 256 || ep < 1 || ep > E || E % ep != 0 || !counts_host || !expert_rank_host)
+    return MOE_ERR_INVALID_ARG;
+  fit_correlated_placement(counts_host, E, ep, expert_rank_host);
+  return MOE_OK;
+}
+
 moe_status moe_dispatch_layout(const moe_shape* s, const int32_t* topk_idx,
                                const int32_t* expert_rank_host, const moe_layout* out, void* ws,
                                size_t ws_bytes, moe_stream_t stream) {
@@ -597,6 +682,15 @@ moe_status moe_permute_by_token(const moe_shape* s, const void* x, const int32_t
 moe_status moe_grouped_swiglu(const moe_shape* s, const void* x_perm, const int32_t* offsets,
                               const void* packed, void* h, void* y_perm, void* ws, size_t ws_bytes,
                               moe_stream_t stream) {
+  return moe_debug_grouped_swiglu_engine(s, x_perm, offsets, packed, h, y_perm, ws, ws_bytes,
+                                         kEngineAuto, stream);
+}
+
+moe_status moe_debug_grouped_swiglu_engine(const moe_shape* s, const void* x_perm,
+                                           const int32_t* offsets, const void* packed, void* h,
+                                           void* y_perm, void* ws, size_t ws_bytes, int32_t engine,
+                                           moe_stream_t stream) {
+  if (engine < kEngineAuto || engine > kEnginePair) return MOE_ERR_INVALID_ARG;
   moe_status r = check_shape(s);
   if (r != MOE_OK) return r;
   if (s->T == 0) return MOE_OK;
@@ -607,7 +701,7 @@ moe_status moe_grouped_swiglu(const moe_shape* s, const void* x_perm, const int3
   if (ws_bytes < scratch_bytes(s)) return MOE_ERR_WORKSPACE;
   Packed pk = carve_packed(s, packed);
   return do_grouped(s, x_perm, offsets, &pk, h, y_perm, carve_scratch(s, ws).ctl,
-                    (cudaStream_t)stream);
+                    (cudaStream_t)stream, engine);
 }
 
 moe_status moe_combine(const moe_shape* s, const void* y_perm, const int32_t* slot_row,

@@ -131,6 +131,10 @@ struct GemmArgs {
   int64_t src_rows = 0;
 };
 cudaError_t launch_gemm_tc(int epi, int bn, const GemmArgs& a, cudaStream_t s);
+// ---- gemm_pair.cu: the same GEMM on CTA pairs (256-row tiles, tcgen05
+// cta_group::2), bit-identical results; BN = 256, no gather
+bool gemm_pair_supported(int epi, int bn, const GemmArgs& a);
+cudaError_t launch_gemm_pair(int epi, int bn, const GemmArgs& a, cudaStream_t s);
 bool make_kmajor_map(CUtensorMap* m, const void* base, int64_t rows, int K, int box_rows);
 // 2-D fp32 [rows, cols] row-major, box of 32 columns (128 B) x box_rows,
 // 128-byte swizzle (for tiled stores of swizzled shared-memory tiles)
@@ -200,7 +204,17 @@ cudaError_t launch_capacity_keep(const int32_t* idx, int64_t T, int k, int E, in
                                  const float* gate, int32_t* keep, float* kept_gate, Control* ctl,
                                  cudaStream_t s);
 
+// ---- placement.cu
+// W[e * E + e'] = ordered slot pairs (a != b) of a token with experts
+// (e, e') (zeroed here first); tokens with an index outside [0, E) add
+// nothing and set MOE_ERR_DEVICE_INDEX.
+cudaError_t launch_coselection(const int32_t* idx, int64_t T, int k, int E, uint64_t* W,
+                               Control* ctl, cudaStream_t s);
+// Greedy correlated placement from host counts W [E * E] (see placement.cu).
+void fit_correlated_placement(const uint64_t* W, int E, int ep, int32_t* rank_of);
+
 // ---- pack.cu
+// w_router NULL: only the experts; w_gate NULL: only the router
 cudaError_t launch_pack(int dtype, int d, int E, int f, int blk, int E16, const void* w_router,
                         const void* w_gate, const void* w_up, const void* w_down, void* wrT,
                         void* wgu, void* wdT, cudaStream_t s);

@@ -56,11 +56,15 @@ template <typename T>
 cudaError_t pack_all(int d, int E, int f, int blk, int E16, const void* w_router,
                      const void* w_gate, const void* w_up, const void* w_down, void* wrT, void* wgu,
                      void* wdT, cudaStream_t s) {
-  cudaError_t err = cudaMemsetAsync(wrT, 0, sizeof(T) * (size_t)E16 * d, s);
-  if (err != cudaSuccess) return err;
-  // router [d, E] -> [E, d]
-  err = transpose<T>(w_router, wrT, 1, d, E, 0, 0, E, 0, 0, s);
-  if (err != cudaSuccess) return err;
+  cudaError_t err = cudaSuccess;
+  if (w_router) {
+    err = cudaMemsetAsync(wrT, 0, sizeof(T) * (size_t)E16 * d, s);
+    if (err != cudaSuccess) return err;
+    // router [d, E] -> [E, d]
+    err = transpose<T>(w_router, wrT, 1, d, E, 0, 0, E, 0, 0, s);
+    if (err != cudaSuccess) return err;
+  }
+  if (!w_gate) return cudaSuccess;  // the router alone
   // gate / up [E][d, f] -> [E][2f, d], blocks of blk rows interleaved
   const int64_t gu_stride = (int64_t)2 * f * d;
   err = transpose<T>(w_gate, wgu, E, d, f, (int64_t)d * f, gu_stride, blk, 2 * blk, 0, s);
