@@ -189,7 +189,11 @@ MOE_API moe_status moe_packed_weights_size(const moe_shape* shape, size_t* bytes
  *   W_d [E, f, d] ("EHM")       -> per expert W_d^T [d, f]
  * All inputs in the shape's dtype, device memory, row-major.  The packed
  * buffer is what moe_route, moe_grouped_swiglu and moe_forward read; it is
- * only valid for the shape it was packed for.
+ * only valid for the shape it was packed for.  Either part may be left out:
+ * w_router NULL packs the experts alone, w_gate, w_up and w_down all NULL
+ * the router alone (the part left out is not written and must not be read:
+ * an expert-parallel rank routes with the whole router and holds only its
+ * own experts).
  */
 MOE_API moe_status moe_pack_weights(const moe_shape* shape, const void* w_router,
                             const void* w_gate, const void* w_up,
@@ -568,6 +572,80 @@ MOE_API moe_status moe_forward_routed(const moe_shape* shape, const void* x,
                                       const int32_t* expert_rank_host, void* y,
                                       const moe_forward_buffers* buffers, void* ws,
                                       size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Expert parallelism: the layer over P = shape->ep ranks (GPUs), tokens split
+ * over the ranks and the E experts placed on them by the expert -> rank map,
+ * with the deduplicated dispatch of "Expert Coupling in MoE Pretraining"
+ * (Abstract: each token is sent to each GPU that holds one of its experts
+ * once; Table I: GPUs per token and the rows deduplication removes; Fig. 7:
+ * baseline vs deduplicated dispatch).  One rank's forward:
+ *   moe_route, moe_dispatch_layout (ep = P)   the send plan of its tokens
+ *   moe_ep_pack                                its send rows
+ *   (exchange: rank_counts of every rank, then the send rows all-to-all;
+ *    the rows for rank r are rows [rank_offsets[r], rank_offsets[r+1]))
+ *   moe_ep_expert_forward                      one return row per received row
+ *   (reverse exchange of the return rows)
+ *   moe_ep_home_combine                        y of its tokens
+ * The exchange is the caller's (NCCL all-to-all, peer copies, ...): the
+ * library moves no bytes between GPUs.
+ */
+
+/*
+ * Send rows of one rank, grouped by destination rank (send row s goes to
+ * the rank r with rank_offsets[r] <= s < rank_offsets[r+1]):
+ *   send_x   [send_rows, d]  x[send_token[s]]
+ *   send_idx [send_rows, k]  the token's k experts as the destination's
+ *                            local expert ids (the expert's position among
+ *                            that rank's experts, ascending), or E/P for an
+ *                            expert another rank holds
+ *   send_gate[send_rows, k]  the token's k gates (1 when topk_gate is NULL)
+ *  shape: T local tokens, ep = P >= 2; topk_idx / topk_gate [T, k] (device);
+ *  expert_rank_host as in moe_dispatch_layout; layout: the send_token and
+ *  rank_offsets of moe_dispatch_layout on the same routing and map;
+ *  send_rows: rows the send buffers hold (rank_offsets[P], read back, or
+ *  any bound; rows past rank_offsets[P] are not written).
+ */
+MOE_API moe_status moe_ep_pack(const moe_shape* shape, const void* x, const int32_t* topk_idx,
+                               const float* topk_gate, const int32_t* expert_rank_host,
+                               const moe_layout* layout, void* send_x, int32_t* send_idx,
+                               float* send_gate, int64_t send_rows, moe_stream_t stream);
+
+/*
+ * Workspace of moe_ep_expert_forward for shape (T = rows this rank
+ * received, ep = P): layout scratch and the expert-grouped intermediates.
+ */
+MOE_API moe_status moe_ep_expert_workspace_size(const moe_shape* shape, size_t* bytes);
+
+/*
+ * The receiving rank's experts: the received rows' assignments to its E/P
+ * experts are laid out by local expert (a stable counting sort, the slots
+ * of other ranks' experts set aside), run through the grouped SwiGLU
+ * experts, and each received row's return row is the gated sum of its
+ * local experts' outputs:
+ *   y_ret[i] = sum_{j : recv_idx[i,j] < E/P} recv_gate[i,j] * expert_{recv_idx[i,j]}(recv_x[i])
+ * summed in fp32 in ascending j, rounded once to the dtype.
+ *  shape: T = received rows, E = all experts, ep = P; recv_x [T, d],
+ *  recv_idx [T, k], recv_gate [T, k] (the moe_ep_pack rows of every source
+ *  rank, in any order); packed_local: moe_pack_weights output for a shape
+ *  with E/P experts (this rank's experts, ascending); y_ret [T, d];
+ *  ws, ws_bytes: moe_ep_expert_workspace_size bytes, zero-filled once (its
+ *  device status word is read with moe_get_device_status).
+ */
+MOE_API moe_status moe_ep_expert_forward(const moe_shape* shape, const void* recv_x,
+                                         const int32_t* recv_idx, const float* recv_gate,
+                                         const void* packed_local, void* y_ret, void* ws,
+                                         size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * The home rank's output: y[t] = sum over the distinct send rows of token t
+ * (one per destination rank, taken in slot order) of y_back[row], in fp32,
+ * rounded once; y_back [send_rows, d] holds the return rows in send-row
+ * order, slot_send_row [T, k] is moe_dispatch_layout's.
+ */
+MOE_API moe_status moe_ep_home_combine(const moe_shape* shape, const void* y_back,
+                                       const int32_t* slot_send_row, int64_t send_rows, void* y,
+                                       moe_stream_t stream);
 
 /*
  * Synchronise `stream`, read the device status word of workspace `ws`

@@ -87,7 +87,8 @@ SYMBOLS = ("moe_status_string", "moe_scratch_size", "moe_forward_workspace_size"
            "moe_route_selection_bias", "moe_router_stats", "moe_capacity_keep",
            "moe_dispatch_layout", "moe_coselection_counts", "moe_fit_placement", "moe_permute", "moe_permute_by_token", "moe_grouped_swiglu",
            "moe_grouped_swiglu_gather", "moe_combine", "moe_forward", "moe_forward_selection_bias", "moe_forward_timed",
-           "moe_forward_routed", "moe_get_device_status", "moe_debug_dispatch_layout_stall",
+           "moe_forward_routed", "moe_ep_pack", "moe_ep_expert_workspace_size",
+           "moe_ep_expert_forward", "moe_ep_home_combine", "moe_get_device_status", "moe_debug_dispatch_layout_stall",
            "moe_debug_grouped_swiglu_engine", "moe_dispatch_layout_static")
 FORWARD_STAGES = ("route", "layout", "permute", "gate_up", "down", "combine")
 
@@ -138,6 +139,11 @@ def lib() -> ctypes.CDLL:
             "moe_forward_selection_bias": ([S, P, P, P, P, P, P,
                                             ctypes.POINTER(moe_forward_buffers), P,
                                             ctypes.c_size_t, P], ctypes.c_int),
+            "moe_ep_pack": ([S, P, P, P, P, ctypes.POINTER(moe_layout), P, P, P, ctypes.c_int64, P],
+                            ctypes.c_int),
+            "moe_ep_expert_workspace_size": ([S, sz], ctypes.c_int),
+            "moe_ep_expert_forward": ([S, P, P, P, P, P, P, ctypes.c_size_t, P], ctypes.c_int),
+            "moe_ep_home_combine": ([S, P, P, ctypes.c_int64, P, P], ctypes.c_int),
             "moe_get_device_status": ([P, P, ctypes.POINTER(ctypes.c_int)], ctypes.c_int),
             "moe_debug_dispatch_layout_stall": ([S, P, P, ctypes.POINTER(moe_layout), P,
                                                  ctypes.c_size_t, ctypes.c_int32, ctypes.c_int64, P],
@@ -258,13 +264,18 @@ def workspace_init(ws: torch.Tensor, stream=None):
 
 
 def pack_weights(shape: Shape, w_router, w_gate, w_up, w_down, stream=None) -> torch.Tensor:
-    """Pack W_r [d,E], W_g/W_u [E,d,f], W_d [E,f,d] into the kernels' layout."""
-    _need(w_router, shape.dtype, (shape.d, shape.E), "w_router")
-    _need(w_gate, shape.dtype, (shape.E, shape.d, shape.f), "w_gate")
-    _need(w_up, shape.dtype, (shape.E, shape.d, shape.f), "w_up")
-    _need(w_down, shape.dtype, (shape.E, shape.f, shape.d), "w_down")
+    """Pack W_r [d,E], W_g/W_u [E,d,f], W_d [E,f,d] into the kernels' layout.
+    w_router=None packs the experts alone; w_gate=w_up=w_down=None the
+    router alone."""
+    if w_router is not None:
+        _need(w_router, shape.dtype, (shape.d, shape.E), "w_router")
+    if w_gate is not None or w_up is not None or w_down is not None:
+        _need(w_gate, shape.dtype, (shape.E, shape.d, shape.f), "w_gate")
+        _need(w_up, shape.dtype, (shape.E, shape.d, shape.f), "w_up")
+        _need(w_down, shape.dtype, (shape.E, shape.f, shape.d), "w_down")
+    dev = (w_router if w_router is not None else w_gate).device
     n = packed_weights_size(shape)
-    packed = torch.empty(n, dtype=torch.uint8, device=w_gate.device)
+    packed = torch.zeros(n, dtype=torch.uint8, device=dev)
     s = shape.c
     _check(lib().moe_pack_weights(ctypes.byref(s), _p(w_router), _p(w_gate), _p(w_up), _p(w_down),
                                   _p(packed), n, _stream(stream)), "moe_pack_weights")
@@ -669,6 +680,62 @@ def forward_routed(shape: Shape, x, packed, topk_idx, topk_gate, ws, expert_rank
                                     _p(topk_gate), _host_map(shape, expert_rank), _p(y),
                                     ctypes.byref(b) if b is not None else None, _p(ws),
                                     ws.numel(), _stream(stream)), "moe_forward_routed")
+    return y
+
+
+def ep_pack(shape: Shape, x, topk_idx, topk_gate, layout: dict, send_rows: int,
+            expert_rank=None, stream=None):
+    """moe_ep_pack: (send_x [send_rows, d], send_idx [send_rows, k] int32,
+    send_gate [send_rows, k] fp32) for this rank's send plan."""
+    _need(x, shape.dtype, (shape.T, shape.d), "x")
+    _need(topk_idx, torch.int32, (shape.T, shape.k), "topk_idx")
+    if topk_gate is not None:
+        _need(topk_gate, torch.float32, (shape.T, shape.k), "topk_gate")
+    _need_n(layout["rank_offsets"], torch.int32, shape.ep + 1, "rank_offsets")
+    dev = x.device
+    send_x = torch.empty((send_rows, shape.d), dtype=shape.dtype, device=dev)
+    send_idx = torch.empty((send_rows, shape.k), dtype=torch.int32, device=dev)
+    send_gate = torch.empty((send_rows, shape.k), dtype=torch.float32, device=dev)
+    lay = _c_layout(layout)
+    s = shape.c
+    _check(lib().moe_ep_pack(ctypes.byref(s), _p(x), _p(topk_idx), _p(topk_gate),
+                             _host_map(shape, expert_rank), ctypes.byref(lay), _p(send_x),
+                             _p(send_idx), _p(send_gate), int(send_rows), _stream(stream)),
+           "moe_ep_pack")
+    return send_x, send_idx, send_gate
+
+
+def ep_expert_workspace(shape: Shape, device="cuda") -> torch.Tensor:
+    n = ctypes.c_size_t()
+    s = shape.c
+    _check(lib().moe_ep_expert_workspace_size(ctypes.byref(s), ctypes.byref(n)),
+           "moe_ep_expert_workspace_size")
+    return torch.zeros(n.value, dtype=torch.uint8, device=device)
+
+
+def ep_expert_forward(shape: Shape, recv_x, recv_idx, recv_gate, packed_local, ws, stream=None):
+    """moe_ep_expert_forward over shape.T received rows: y_ret [T, d]."""
+    _need(recv_x, shape.dtype, (shape.T, shape.d), "recv_x")
+    _need(recv_idx, torch.int32, (shape.T, shape.k), "recv_idx")
+    _need(recv_gate, torch.float32, (shape.T, shape.k), "recv_gate")
+    y_ret = torch.empty((shape.T, shape.d), dtype=shape.dtype, device=recv_x.device)
+    s = shape.c
+    _check(lib().moe_ep_expert_forward(ctypes.byref(s), _p(recv_x), _p(recv_idx), _p(recv_gate),
+                                       _p(packed_local), _p(y_ret), _p(ws), ws.numel(),
+                                       _stream(stream)), "moe_ep_expert_forward")
+    return y_ret
+
+
+def ep_home_combine(shape: Shape, y_back, slot_send_row, stream=None):
+    """moe_ep_home_combine: y [T, d] from the returned rows."""
+    _need_n(slot_send_row, torch.int32, shape.R, "slot_send_row")
+    if y_back.dtype != shape.dtype or y_back.dim() != 2 or y_back.shape[1] != shape.d:
+        raise ValueError(f"y_back: expected {shape.dtype} [rows, {shape.d}]")
+    y = torch.empty((shape.T, shape.d), dtype=shape.dtype, device=y_back.device)
+    s = shape.c
+    _check(lib().moe_ep_home_combine(ctypes.byref(s), _p(y_back), _p(slot_send_row),
+                                     int(y_back.shape[0]), _p(y), _stream(stream)),
+           "moe_ep_home_combine")
     return y
 
 

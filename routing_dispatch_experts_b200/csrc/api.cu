@@ -423,6 +423,55 @@ moe_status forward_impl(const moe_shape* s, const void* x, const void* packed, c
   return mark(6);
 }
 
+// ---- expert parallelism: the receiving rank's workspace
+// Received rows are routed over E_loc = E/ep local experts plus one group
+// (index E_loc) that collects the slots whose expert another rank holds.
+struct EpRecv {
+  Scratch sc;
+  LayoutOut lo;
+  void* x_perm;
+  void* h;
+  void* y_perm;
+};
+
+size_t ep_recv_bytes(const moe_shape* s) {
+  const int El = s->E / s->ep + 1;
+  const size_t R = (size_t)s->T * s->k, es = esize(s->dtype);
+  const size_t nb = (size_t)layout_blocks(s->T), bins = (size_t)layout_bins(El, 1);
+  size_t n = align_up(sizeof(Control)) + kTotalsBytes + align_up(nb * bins * 8);
+  n += align_up((size_t)El * 4) + align_up((size_t)(El + 1) * 4) + 2 * align_up(R * 4);
+  n += align_up(R * s->d * es) + align_up(R * s->f * es) + align_up(R * s->d * es);
+  return n;
+}
+
+EpRecv carve_ep_recv(const moe_shape* s, void* ws) {
+  const int El = s->E / s->ep + 1;
+  const size_t R = (size_t)s->T * s->k, es = esize(s->dtype);
+  const size_t nb = (size_t)layout_blocks(s->T), bins = (size_t)layout_bins(El, 1);
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  auto take = [&p](size_t bytes) {
+    void* q = p;
+    p += align_up(bytes);
+    return q;
+  };
+  EpRecv r{};
+  r.sc.ctl = static_cast<Control*>(take(sizeof(Control)));
+  r.sc.totals = static_cast<int32_t*>(static_cast<void*>(p));
+  p += kTotalsBytes;
+  r.sc.status = static_cast<uint64_t*>(take(nb * bins * 8));
+  r.sc.block_hist = nullptr;
+  r.lo.counts = static_cast<int32_t*>(take((size_t)El * 4));
+  r.lo.offsets = static_cast<int32_t*>(take((size_t)(El + 1) * 4));
+  r.lo.row_token = static_cast<int32_t*>(take(R * 4));
+  r.lo.slot_row = static_cast<int32_t*>(take(R * 4));
+  r.lo.rank_counts = r.lo.rank_offsets = r.lo.send_token = r.lo.slot_send_row = nullptr;
+  r.lo.stats = nullptr;
+  r.x_perm = take(R * s->d * es);
+  r.h = take(R * s->f * es);
+  r.y_perm = take(R * s->d * es);
+  return r;
+}
+
 moe_status route_impl(const moe_shape* s, const void* x, const void* packed, const float* bias,
                       const float* sel_bias, float* logits, int32_t* topk_idx, float* topk_gate,
                       void* ws, size_t ws_bytes, cudaStream_t st) {
@@ -494,10 +543,13 @@ moe_status moe_pack_weights(const moe_shape* s, const void* w_router, const void
                             size_t packed_bytes_, moe_stream_t stream) {
   moe_status r = check_shape(s);
   if (r != MOE_OK) return r;
-  if (!w_router || !w_gate || !w_up || !w_down || !packed) return MOE_ERR_INVALID_ARG;
+  // the router alone (no expert weights), the experts alone (no router), or both
+  const bool experts = w_gate || w_up || w_down;
+  if (experts && (!w_gate || !w_up || !w_down)) return MOE_ERR_INVALID_ARG;
+  if ((!w_router && !experts) || !packed) return MOE_ERR_INVALID_ARG;
   const size_t es = esize(s->dtype);
   for (const void* p : {w_router, w_gate, w_up, w_down})
-    if (!aligned(p, es)) return MOE_ERR_ALIGNMENT;
+    if (p && !aligned(p, es)) return MOE_ERR_ALIGNMENT;
   if (!aligned(packed, kAlign)) return MOE_ERR_ALIGNMENT;
   if (packed_bytes_ < packed_bytes(s)) return MOE_ERR_WORKSPACE;
   Packed pk = carve_packed(s, packed);
@@ -639,6 +691,121 @@ moe_status moe_fit_placement(int32_t E, int32_t ep, const uint64_t* counts_host,
     return MOE_ERR_INVALID_ARG;
   fit_correlated_placement(counts_host, E, ep, expert_rank_host);
   return MOE_OK;
+}
+
+moe_status moe_ep_pack(const moe_shape* s, const void* x, const int32_t* topk_idx,
+                       const float* topk_gate, const int32_t* expert_rank_host,
+                       const moe_layout* layout, void* send_x, int32_t* send_idx,
+                       float* send_gate, int64_t send_rows, moe_stream_t stream) {
+  moe_status r = check_shape(s);
+  if (r != MOE_OK) return r;
+  if (s->ep < 2) return MOE_ERR_INVALID_ARG;
+  if (send_rows < 0) return MOE_ERR_INVALID_ARG;
+  if (s->T == 0 || send_rows == 0) return MOE_OK;
+  if (!x || !topk_idx || !layout || !layout->send_token || !layout->rank_offsets || !send_x ||
+      !send_idx || !send_gate)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(send_x, 16) || !aligned(topk_idx, 4) ||
+      !aligned(layout->send_token, 4) || !aligned(layout->rank_offsets, 4) ||
+      !aligned(send_idx, 4) || !aligned(send_gate, 4) || (topk_gate && !aligned(topk_gate, 4)))
+    return MOE_ERR_ALIGNMENT;
+  RankMap map;
+  if ((r = build_map(s, expert_rank_host, &map)) != MOE_OK) return r;
+  EpMaps m{};
+  int next[256] = {0};
+  for (int e = 0; e < s->E; ++e) {
+    m.rank[e] = map.r[e];
+    m.local[e] = (uint8_t)next[map.r[e]]++;
+  }
+  return cuda_status(launch_ep_pack(s->dtype, x, s->T, s->d, s->k, topk_idx, topk_gate,
+                                    layout->send_token, layout->rank_offsets, s->ep, m, s->E,
+                                    send_x, send_idx, send_gate, send_rows, (cudaStream_t)stream));
+}
+
+moe_status moe_ep_expert_workspace_size(const moe_shape* s, size_t* bytes) {
+  moe_status r = check_shape(s);
+  if (r != MOE_OK) return r;
+  if (!bytes || s->ep < 2) return MOE_ERR_INVALID_ARG;
+  *bytes = ep_recv_bytes(s);
+  return MOE_OK;
+}
+
+moe_status moe_ep_expert_forward(const moe_shape* s, const void* recv_x, const int32_t* recv_idx,
+                                 const float* recv_gate, const void* packed_local, void* y_ret,
+                                 void* ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status r = check_shape(s);
+  if (r != MOE_OK) return r;
+  if (s->ep < 2 || !ws) return MOE_ERR_INVALID_ARG;
+  if (!aligned(ws, kAlign)) return MOE_ERR_ALIGNMENT;
+  if (ws_bytes < ep_recv_bytes(s)) return MOE_ERR_WORKSPACE;
+  if (s->T == 0) return MOE_OK;
+  if (!recv_x || !recv_idx || !recv_gate || !packed_local || !y_ret) return MOE_ERR_INVALID_ARG;
+  if (!aligned(recv_x, 16) || !aligned(y_ret, 16) || !aligned(recv_idx, 4) ||
+      !aligned(recv_gate, 4) || !aligned(packed_local, kAlign))
+    return MOE_ERR_ALIGNMENT;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int El = s->E / s->ep;
+  const EpRecv rv = carve_ep_recv(s, ws);
+  // the local experts' packed weights: a packed buffer of E/ep experts
+  moe_shape loc = *s;
+  loc.E = El;
+  loc.ep = 1;
+  loc.k = std::min(s->k, El);  // only E, d, f and dtype shape the packed buffer
+  const Packed pk = carve_packed(&loc, packed_local);
+  // layout of the received rows over the local experts plus the
+  // "held elsewhere" group El (no rank dispatch: ep = 1)
+  RankMap one;
+  std::memset(&one, 0, sizeof(one));
+  if ((r = cuda_status(launch_layout(recv_idx, s->T, s->k, El + 1, 1, one, rv.lo, rv.sc.ctl,
+                                     rv.sc.status, rv.sc.totals, -1, kWaitLimitNs, st))) != MOE_OK)
+    return r;
+  // expert FFN over groups 0..El-1: their rows are [offsets[0], offsets[El])
+  const int64_t R = s->T * (int64_t)s->k;
+  if (s->dtype == MOE_BF16 && ffn_fused_supported(s->d, s->f)) {
+    FfnArgs fa{};
+    fa.A = recv_x;
+    fa.gather = rv.lo.row_token;
+    fa.src_rows = s->T;
+    fa.rows = R;
+    fa.offsets = rv.lo.offsets;
+    fa.G = El;
+    fa.d = s->d;
+    fa.f = s->f;
+    fa.wgu = pk.wgu;
+    fa.wdT = pk.wdT;
+    fa.y_perm = rv.y_perm;
+    fa.ctl = rv.sc.ctl;
+    if ((r = cuda_status(launch_ffn_fused(fa, st))) != MOE_OK) return r;
+  } else {
+    loc.T = s->T;
+    loc.k = s->k;
+    const bool g = s->dtype == MOE_BF16;
+    if (!g && (r = cuda_status(launch_permute(recv_x, rv.lo.row_token, nullptr, rv.x_perm, s->T,
+                                              s->k, (uint32_t)(s->d * esize(s->dtype)), st))) !=
+                  MOE_OK)
+      return r;
+    if ((r = do_grouped_part(0, &loc, g ? recv_x : rv.x_perm, g ? rv.lo.row_token : nullptr,
+                             rv.lo.offsets, &pk, rv.h, rv.y_perm, rv.sc.ctl, st)) != MOE_OK)
+      return r;
+    if ((r = do_grouped_part(1, &loc, nullptr, nullptr, rv.lo.offsets, &pk, rv.h, rv.y_perm,
+                             rv.sc.ctl, st)) != MOE_OK)
+      return r;
+  }
+  return cuda_status(launch_ep_partial_combine(s->dtype, rv.y_perm, rv.lo.slot_row, recv_idx,
+                                               recv_gate, El, y_ret, s->T, s->d, s->k, st));
+}
+
+moe_status moe_ep_home_combine(const moe_shape* s, const void* y_back, const int32_t* slot_send_row,
+                               int64_t send_rows, void* y, moe_stream_t stream) {
+  moe_status r = check_shape(s);
+  if (r != MOE_OK) return r;
+  if (s->ep < 2 || send_rows < 0) return MOE_ERR_INVALID_ARG;
+  if (s->T == 0) return MOE_OK;
+  if (!y_back || !slot_send_row || !y || send_rows == 0) return MOE_ERR_INVALID_ARG;
+  if (!aligned(y_back, 16) || !aligned(y, 16) || !aligned(slot_send_row, 4))
+    return MOE_ERR_ALIGNMENT;
+  return cuda_status(launch_ep_home_combine(s->dtype, y_back, slot_send_row, y, s->T, s->d, s->k,
+                                            send_rows, (cudaStream_t)stream));
 }
 
 moe_status moe_dispatch_layout(const moe_shape* s, const int32_t* topk_idx,

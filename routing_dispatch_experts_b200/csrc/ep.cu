@@ -1,0 +1,208 @@
+// ep.cu - expert parallelism: the deduplicated dispatch of "Expert Coupling
+// in MoE Pretraining" (Abstract: each token is sent to each GPU that holds
+// one of its experts once, not once per expert; Table I: the rows removed;
+// Fig. 7: baseline vs deduplicated dispatch) and its combine return path.
+//
+// One rank's forward over P ranks (tokens split over ranks, experts placed
+// by the expert -> rank map):
+//   1. router + dispatch layout with ep = P: the send plan (rank_counts,
+//      send_token: one send row per (token, destination rank)),
+//   2. ep_pack_kernel: the send rows, grouped by destination, each carrying
+//      the token's row of x, its k gates and its k experts as the
+//      destination's local expert ids (E/P for an expert held elsewhere),
+//   3. the exchange (all-to-all of the send rows; outside this file),
+//   4. on each rank, the expert FFN over the received rows' local experts
+//      (layout over E/P + 1 groups, the last one collecting the "held
+//      elsewhere" slots, which no GEMM reads), then
+//      ep_partial_combine_kernel: one return row per received row, the
+//      gated sum of that rank's experts for the token,
+//   5. the reverse exchange, and ep_home_combine_kernel: each token's output
+//      is the sum of its returned rows (one per distinct destination rank).
+#include "kernels.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kPackWarps = 8;
+
+// one warp per send row s: destination r from rank_offsets (binary search in
+// shared memory), token t = send_token[s]
+__global__ void __launch_bounds__(32 * kPackWarps)
+    ep_pack_kernel(const uint4* __restrict__ x, int64_t T, int V, int k,
+                   const int32_t* __restrict__ idx, const float* __restrict__ gate,
+                   const int32_t* __restrict__ send_token, const int32_t* __restrict__ rank_offsets,
+                   int P, EpMaps maps, int E, int E_loc, uint4* __restrict__ send_x,
+                   int32_t* __restrict__ send_idx, float* __restrict__ send_gate, int64_t cap) {
+  __shared__ int s_off[257];
+  pdl_wait();
+  for (int i = threadIdx.x; i <= P; i += blockDim.x) s_off[i] = __ldg(rank_offsets + i);
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int64_t rows = min((int64_t)s_off[P], cap);
+  for (int64_t s = (int64_t)blockIdx.x * kPackWarps + (threadIdx.x >> 5); s < rows;
+       s += (int64_t)gridDim.x * kPackWarps) {
+    // last r with s_off[r] <= s
+    int lo = 0, hi = P - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_off[mid] <= s) lo = mid; else hi = mid - 1;
+    }
+    const int r = lo;
+    int64_t t = __ldg(send_token + s);
+    if (t < 0 || t >= T) t = 0;
+    const uint4* src = x + t * V;
+    uint4* dst = send_x + s * V;
+    for (int v = lane; v < V; v += 32) dst[v] = __ldg(src + v);
+    if (lane < k) {
+      const int e = __ldg(idx + t * k + lane);
+      const bool here = e >= 0 && e < E && maps.rank[e] == r;
+      send_idx[s * k + lane] = here ? (int)maps.local[e] : E_loc;
+      send_gate[s * k + lane] = gate ? __ldg(gate + t * k + lane) : 1.f;
+    }
+  }
+}
+
+template <typename T>
+struct Acc;
+template <>
+struct Acc<__nv_bfloat16> {
+  static constexpr int N = 8;
+  __device__ static void add(float* a, const uint4& q, float g) {
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      a[2 * i] = fmaf(g, bf16_lo(w[i]), a[2 * i]);
+      a[2 * i + 1] = fmaf(g, bf16_hi(w[i]), a[2 * i + 1]);
+    }
+  }
+  __device__ static uint4 pack(const float* a) {
+    return make_uint4(pack_bf16x2(a[0], a[1]), pack_bf16x2(a[2], a[3]), pack_bf16x2(a[4], a[5]),
+                      pack_bf16x2(a[6], a[7]));
+  }
+};
+template <>
+struct Acc<float> {
+  static constexpr int N = 4;
+  __device__ static void add(float* a, const uint4& q, float g) {
+    a[0] = fmaf(g, __uint_as_float(q.x), a[0]);
+    a[1] = fmaf(g, __uint_as_float(q.y), a[1]);
+    a[2] = fmaf(g, __uint_as_float(q.z), a[2]);
+    a[3] = fmaf(g, __uint_as_float(q.w), a[3]);
+  }
+  __device__ static uint4 pack(const float* a) {
+    return make_uint4(__float_as_uint(a[0]), __float_as_uint(a[1]), __float_as_uint(a[2]),
+                      __float_as_uint(a[3]));
+  }
+};
+
+// y_ret[i] = sum over slots j (ascending) of received row i whose expert is
+// held here (local id < E_loc) of gate[i,j] * y_perm[slot_row[i*k + j]], in
+// fp32, rounded once.  One thread per 16-byte vector of an output row.
+template <typename T>
+__global__ void __launch_bounds__(256)
+    ep_partial_combine_kernel(const uint4* __restrict__ y_perm, const int32_t* __restrict__ slot_row,
+                              const int32_t* __restrict__ recv_idx, const float* __restrict__ recv_gate,
+                              int E_loc, uint4* __restrict__ y_ret, int64_t Tr, int V, int k) {
+  pdl_wait();
+  const int64_t n = Tr * V;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = i / V;
+    const int v = (int)(i - t * V);
+    float a[Acc<T>::N];
+#pragma unroll
+    for (int q = 0; q < Acc<T>::N; ++q) a[q] = 0.f;
+    for (int j = 0; j < k; ++j) {
+      const int e = __ldg(recv_idx + t * k + j);
+      if (e < 0 || e >= E_loc) continue;  // held by another rank
+      int64_t row = __ldg(slot_row + t * k + j);
+      if (row < 0 || row >= Tr * k) row = 0;
+      Acc<T>::add(a, __ldg(y_perm + row * V + v), __ldg(recv_gate + t * k + j));
+    }
+    y_ret[i] = Acc<T>::pack(a);
+  }
+}
+
+// y[t] = sum, over the distinct send rows of token t in slot order (each
+// destination rank's row counted once), of y_back[row], in fp32, rounded
+// once.  One thread per 16-byte vector of an output row.
+template <typename T>
+__global__ void __launch_bounds__(256)
+    ep_home_combine_kernel(const uint4* __restrict__ y_back, const int32_t* __restrict__ slot_send_row,
+                           uint4* __restrict__ y, int64_t Tn, int V, int k, int64_t rows) {
+  pdl_wait();
+  const int64_t n = Tn * V;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = i / V;
+    const int v = (int)(i - t * V);
+    float a[Acc<T>::N];
+#pragma unroll
+    for (int q = 0; q < Acc<T>::N; ++q) a[q] = 0.f;
+    int seen[16];
+    for (int j = 0; j < k; ++j) {
+      int row = __ldg(slot_send_row + t * k + j);
+      bool dup = false;
+      for (int q = 0; q < j; ++q) dup |= seen[q] == row;
+      seen[j] = row;
+      if (dup) continue;
+      if (row < 0 || row >= rows) row = 0;
+      Acc<T>::add(a, __ldg(y_back + (int64_t)row * V + v), 1.f);
+    }
+    y[i] = Acc<T>::pack(a);
+  }
+}
+
+int grid_for(int64_t items, int per_block) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return (int)std::min<int64_t>((items + per_block - 1) / per_block, (int64_t)sms * 8);
+}
+
+}  // namespace
+
+cudaError_t launch_ep_pack(int dtype, const void* x, int64_t T, int d, int k, const int32_t* idx,
+                           const float* gate, const int32_t* send_token,
+                           const int32_t* rank_offsets, int P, const EpMaps& maps, int E,
+                           void* send_x, int32_t* send_idx, float* send_gate, int64_t cap,
+                           cudaStream_t s) {
+  if (T == 0 || cap == 0) return cudaSuccess;
+  const int V = d * (dtype == MOE_BF16 ? 2 : 4) / 16;
+  const int grid = std::max(1, grid_for(cap, kPackWarps));
+  return launch_pdl(ep_pack_kernel, dim3(grid), dim3(32 * kPackWarps), 0, s,
+                    static_cast<const uint4*>(x), T, V, k, idx, gate, send_token, rank_offsets, P,
+                    maps, E, E / P, static_cast<uint4*>(send_x), send_idx, send_gate, cap);
+}
+
+cudaError_t launch_ep_partial_combine(int dtype, const void* y_perm, const int32_t* slot_row,
+                                      const int32_t* recv_idx, const float* recv_gate, int E_loc,
+                                      void* y_ret, int64_t Tr, int d, int k, cudaStream_t s) {
+  if (Tr == 0) return cudaSuccess;
+  const int V = d * (dtype == MOE_BF16 ? 2 : 4) / 16;
+  const int grid = grid_for(Tr * V, 256);
+  if (dtype == MOE_BF16)
+    return launch_pdl(ep_partial_combine_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s,
+                      static_cast<const uint4*>(y_perm), slot_row, recv_idx, recv_gate, E_loc,
+                      static_cast<uint4*>(y_ret), Tr, V, k);
+  return launch_pdl(ep_partial_combine_kernel<float>, dim3(grid), dim3(256), 0, s,
+                    static_cast<const uint4*>(y_perm), slot_row, recv_idx, recv_gate, E_loc,
+                    static_cast<uint4*>(y_ret), Tr, V, k);
+}
+
+cudaError_t launch_ep_home_combine(int dtype, const void* y_back, const int32_t* slot_send_row,
+                                   void* y, int64_t T, int d, int k, int64_t rows, cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  const int V = d * (dtype == MOE_BF16 ? 2 : 4) / 16;
+  const int grid = grid_for(T * V, 256);
+  if (dtype == MOE_BF16)
+    return launch_pdl(ep_home_combine_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s,
+                      static_cast<const uint4*>(y_back), slot_send_row, static_cast<uint4*>(y), T, V,
+                      k, rows);
+  return launch_pdl(ep_home_combine_kernel<float>, dim3(grid), dim3(256), 0, s,
+                    static_cast<const uint4*>(y_back), slot_send_row, static_cast<uint4*>(y), T, V, k,
+                    rows);
+}
+
+}  // namespace moe

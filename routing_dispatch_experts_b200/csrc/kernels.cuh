@@ -213,6 +213,23 @@ cudaError_t launch_coselection(const int32_t* idx, int64_t T, int k, int E, uint
 // Greedy correlated placement from host counts W [E * E] (see placement.cu).
 void fit_correlated_placement(const uint64_t* W, int E, int ep, int32_t* rank_of);
 
+// ---- ep.cu (expert parallelism)
+// expert -> owning rank and -> index among that rank's experts (ascending)
+struct EpMaps {
+  uint8_t rank[256];
+  uint8_t local[256];
+};
+cudaError_t launch_ep_pack(int dtype, const void* x, int64_t T, int d, int k, const int32_t* idx,
+                           const float* gate, const int32_t* send_token,
+                           const int32_t* rank_offsets, int P, const EpMaps& maps, int E,
+                           void* send_x, int32_t* send_idx, float* send_gate, int64_t cap,
+                           cudaStream_t s);
+cudaError_t launch_ep_partial_combine(int dtype, const void* y_perm, const int32_t* slot_row,
+                                      const int32_t* recv_idx, const float* recv_gate, int E_loc,
+                                      void* y_ret, int64_t Tr, int d, int k, cudaStream_t s);
+cudaError_t launch_ep_home_combine(int dtype, const void* y_back, const int32_t* slot_send_row,
+                                   void* y, int64_t T, int d, int k, int64_t rows, cudaStream_t s);
+
 // ---- pack.cu
 // w_router NULL: only the experts; w_gate NULL: only the router
 cudaError_t launch_pack(int dtype, int d, int E, int f, int blk, int E16, const void* w_router,

@@ -1,0 +1,191 @@
+"""Expert-parallel MoE layer: one rank's forward over P ranks, around an
+exchange of rows between the ranks.
+
+The deduplicated dispatch of "Expert Coupling in MoE Pretraining"
+(Abstract: each token is sent to each GPU that holds one of its experts
+once; Fig. 7: baseline dispatch B vs deduplicated D, with or without
+correlated placement P): tokens are split over the ranks, experts are
+placed by an expert -> rank map, and every rank
+
+  1. routes its tokens and builds the send plan (moe_route,
+     moe_dispatch_layout with ep = P),
+  2. learns how many rows every rank sends every rank (exchange of the
+     rank_counts),
+  3. packs and sends its rows (moe_ep_pack, all-to-all),
+  4. runs its experts over the rows it received (moe_ep_expert_forward),
+  5. returns one row per received row (reverse all-to-all),
+  6. sums each token's returned rows (moe_ep_home_combine).
+
+Steps 1, 3, 4 and 6 are the library's CUDA kernels; this module only
+sequences them and moves rows through an Exchange:
+
+  TorchExchange  torch.distributed collectives (NCCL between GPUs, gloo on
+                 CPU tensors), one process per rank;
+  LocalExchange  P ranks emulated in one process (their buffers on one
+                 device), for single-GPU tests of the whole path.
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import List, Optional, Sequence
+
+import torch
+
+from . import Shape, dispatch_layout, ep_expert_forward, ep_expert_workspace, ep_home_combine, \
+    ep_pack, route, workspace
+
+# ------------------------------------------------------------------ exchange
+
+
+def splits(counts: Sequence[Sequence[int]], rank: int):
+    """(send splits, receive splits) of `rank` from the count matrix
+    counts[src][dst] = rows src sends dst: it sends row block dst of its
+    send rows to dst, and receives from every src in rank order."""
+    P = len(counts)
+    return [int(counts[rank][d]) for d in range(P)], [int(counts[s][rank]) for s in range(P)]
+
+
+class TorchExchange:
+    """Rows between ranks with torch.distributed (one process per rank)."""
+
+    def __init__(self, group=None):
+        import torch.distributed as dist
+        self.dist = dist
+        self.group = group
+        self.rank = dist.get_rank(group)
+        self.world = dist.get_world_size(group)
+
+    def counts(self, rank_counts: torch.Tensor) -> List[List[int]]:
+        """Every rank's rank_counts, as the host matrix counts[src][dst]."""
+        mine = rank_counts.to(torch.int64).reshape(-1)
+        allc = torch.empty(self.world * self.world, dtype=torch.int64, device=mine.device)
+        self.dist.all_gather_into_tensor(allc, mine, group=self.group)
+        return allc.reshape(self.world, self.world).tolist()
+
+    def rows(self, send: torch.Tensor, send_splits: List[int], recv_splits: List[int]) -> torch.Tensor:
+        """all-to-all-v of the rows of `send` (blocks of send_splits rows to
+        ranks 0..P-1), received in source-rank order."""
+        out = torch.empty((sum(recv_splits),) + tuple(send.shape[1:]), dtype=send.dtype,
+                          device=send.device)
+        self.dist.all_to_all_single(out, send.contiguous(), output_split_sizes=recv_splits,
+                                    input_split_sizes=send_splits, group=self.group)
+        return out
+
+
+class LocalExchange:
+    """P ranks in one process: each collective takes every rank's input at
+    once and returns every rank's output (plain block copies)."""
+
+    def __init__(self, world: int):
+        self.world = world
+
+    def counts(self, rank_counts: Sequence[torch.Tensor]) -> List[List[int]]:
+        return [[int(v) for v in rc.tolist()] for rc in rank_counts]
+
+    def rows(self, sends: Sequence[torch.Tensor], counts: List[List[int]]) -> List[torch.Tensor]:
+        P = self.world
+        blocks = [torch.split(sends[s], counts[s]) for s in range(P)]
+        return [torch.cat([blocks[s][r] for s in range(P)]) for r in range(P)]
+
+    def rows_back(self, rets: Sequence[torch.Tensor], counts: List[List[int]]) -> List[torch.Tensor]:
+        P = self.world
+        blocks = [torch.split(rets[r], [counts[s][r] for s in range(P)]) for r in range(P)]
+        return [torch.cat([blocks[r][s] for r in range(P)]) for s in range(P)]
+
+
+# ----------------------------------------------------------------- one rank
+
+
+@dataclasses.dataclass
+class Plan:
+    """What a rank keeps between the phases of its forward."""
+    idx: torch.Tensor
+    gate: torch.Tensor
+    layout: dict
+    counts: Optional[List[List[int]]] = None
+
+
+class EPRank:
+    """One rank of the expert-parallel layer.
+
+    shape          T = this rank's tokens, E = all experts, ep = P ranks
+    rank           this rank's index in [0, P)
+    expert_rank    expert -> rank map (a partition with E/P experts per
+                   rank), or None for contiguous placement
+    packed_router  moe_pack_weights output holding the router (all ranks
+                   route with the same router)
+    packed_local   moe_pack_weights output for this rank's E/P experts, in
+                   ascending expert order
+    """
+
+    def __init__(self, shape: Shape, rank: int, expert_rank, packed_router, packed_local,
+                 bias=None):
+        if shape.ep < 2:
+            raise ValueError("expert parallelism needs ep >= 2 ranks")
+        self.shape = shape
+        self.rank = rank
+        self.expert_rank = None if expert_rank is None else list(expert_rank)
+        self.packed_router = packed_router
+        self.packed_local = packed_local
+        self.bias = bias
+        self.ws = workspace(shape, device=packed_router.device)
+
+    # phase 1: routing and the send plan
+    def plan(self, x) -> Plan:
+        _, idx, gate = route(self.shape, x, self.packed_router, self.bias, self.ws)
+        lay = dispatch_layout(self.shape, idx, self.ws, expert_rank=self.expert_rank)
+        return Plan(idx=idx, gate=gate, layout=lay)
+
+    # phase 2: the send rows (after the count exchange)
+    def send(self, x, plan: Plan, counts: List[List[int]]):
+        plan.counts = counts
+        n = sum(counts[self.rank])
+        return ep_pack(self.shape, x, plan.idx, plan.gate, plan.layout, n,
+                       expert_rank=self.expert_rank)
+
+    # phase 3: this rank's experts over the rows it received
+    def experts(self, recv_x, recv_idx, recv_gate, ws=None):
+        rs = dataclasses.replace(self.shape, T=int(recv_x.shape[0]))
+        if ws is None:
+            ws = ep_expert_workspace(rs, device=recv_x.device)
+        return ep_expert_forward(rs, recv_x, recv_idx, recv_gate, self.packed_local, ws)
+
+    # phase 4: this rank's outputs from the returned rows
+    def finish(self, plan: Plan, y_back):
+        return ep_home_combine(self.shape, y_back, plan.layout["slot_send_row"])
+
+    def forward(self, x, ex: TorchExchange):
+        """The whole forward of this rank, exchanging through `ex` (every
+        rank calls it with its own tokens)."""
+        plan = self.plan(x)
+        counts = ex.counts(plan.layout["rank_counts"])
+        send_x, send_idx, send_gate = self.send(x, plan, counts)
+        s_sp, r_sp = splits(counts, self.rank)
+        recv_x = ex.rows(send_x, s_sp, r_sp)
+        recv_idx = ex.rows(send_idx, s_sp, r_sp)
+        recv_gate = ex.rows(send_gate, s_sp, r_sp)
+        y_ret = self.experts(recv_x, recv_idx, recv_gate)
+        y_back = ex.rows(y_ret, r_sp, s_sp)
+        return self.finish(plan, y_back), counts
+
+
+def forward_emulated(ranks: Sequence[EPRank], xs: Sequence[torch.Tensor]):
+    """Every rank's forward with the ranks emulated in one process (one
+    device): the same phases as EPRank.forward, the exchanges done by
+    LocalExchange.  Returns (per-rank outputs, count matrix)."""
+    P = len(ranks)
+    ex = LocalExchange(P)
+    plans = [r.plan(x) for r, x in zip(ranks, xs)]
+    counts = ex.counts([p.layout["rank_counts"] for p in plans])
+    sends = [r.send(x, p, counts) for r, x, p in zip(ranks, xs, plans)]
+    recv_x = ex.rows([s[0] for s in sends], counts)
+    recv_idx = ex.rows([s[1] for s in sends], counts)
+    recv_gate = ex.rows([s[2] for s in sends], counts)
+    rets = [r.experts(recv_x[i], recv_idx[i], recv_gate[i]) for i, r in enumerate(ranks)]
+    backs = ex.rows_back(rets, counts)
+    return [r.finish(p, b) for r, p, b in zip(ranks, plans, backs)], counts
+
+
+def local_experts(expert_rank: Sequence[int], rank: int) -> List[int]:
+    """The experts a rank holds, ascending (the order of their local ids)."""
+    return [e for e, r in enumerate(expert_rank) if r == rank]
