@@ -324,6 +324,9 @@ def run_ours(args, rank, world, local):
     # tokens whose top-k margin is below the near-tie bound, where routing
     # may flip between runs or implementations
     rstats, _ = moe.router_stats(shape, buf.logits, buf.topk_idx, threshold=1e-5)
+    # the deduplicated send plan of the measured batch ('Expert Coupling',
+    # Table I: GPUs per token, rows removed by deduplication)
+    dstats = moe.stats_dict(buf.layout["stats"])
     if args.profile:
         return {"profile": True, "ms_per_step": ms, "stage_ms": calls}
 
@@ -434,6 +437,16 @@ def run_ours(args, rank, world, local):
     }
     if bound == "tensor":
         result["roofline"]["frac_of_sustained"] = achieved / pk["bf16_sus"]
+    if ep > 1:
+        R = T * w.k
+        result["dispatch"] = {
+            "ep": ep, "placement": w.placements[0],
+            "rows_per_expert_dispatch": R, "rows_deduplicated": dstats["rows_sent"],
+            "rows_removed": dstats["dup_removed"], "rows_removed_frac": dstats["dup_removed"] / R,
+            "gpus_per_token": dstats["rows_sent"] / T,
+            "tokens_on_one_rank": dstats["tokens_single_rank"],
+            "home_rank_assignment_frac": dstats["home_rank_rows"] / R,
+            "computed_by": "moe_forward's dispatch layout (device statistics)"}
     result["routing"] = {"near_tie_tokens": rstats["near_tie_tokens"],
                          "near_tie_share": rstats["near_tie_tokens"] / max(T, 1),
                          "near_tie_threshold": 1e-5,
