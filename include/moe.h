@@ -671,16 +671,19 @@ MOE_API moe_status moe_debug_dispatch_layout_stall(const moe_shape* shape,
                                            moe_stream_t stream);
 
 /*
- * Test and measurement hook of moe_grouped_swiglu: the same call with the
- * tensor-core GEMM engine chosen by the caller.
- *  engine 0  the library's choice (what moe_grouped_swiglu runs)
- *         1  one CTA per 128-row tile
- *         2  CTA pairs on 256-row tiles (tcgen05 cta_group::2) where the
- *            shape allows it (bf16, 256-column tiles), else as 1
+ * Test and measurement hook of moe_grouped_swiglu (row_token NULL: a_rows
+ * is x_perm) and moe_grouped_swiglu_gather (row_token given: a_rows is x):
+ * the same call with the tensor-core GEMM engine chosen by the caller.
+ *  engine 0  the library's choice (what those calls run)
+ *         1  one CTA per 128-row tile (the gather by cp.async)
+ *         2  CTA pairs on 256-row tiles (tcgen05 cta_group::2; the gather
+ *            by TMA gather4) where the shape allows it (bf16, 256-column
+ *            tiles), else as 1
  * All engines sum every output in the same order, so h and y_perm are
  * bit-identical across engines.  MOE_ERR_INVALID_ARG for another engine.
  */
-MOE_API moe_status moe_debug_grouped_swiglu_engine(const moe_shape* shape, const void* x_perm,
+MOE_API moe_status moe_debug_grouped_swiglu_engine(const moe_shape* shape, const void* a_rows,
+                                                   const int32_t* row_token,
                                                    const int32_t* expert_offsets,
                                                    const void* packed, void* h, void* y_perm,
                                                    void* ws, size_t ws_bytes, int32_t engine,

@@ -149,7 +149,7 @@ def lib() -> ctypes.CDLL:
                                                  ctypes.c_size_t, ctypes.c_int32, ctypes.c_int64, P],
                                                 ctypes.c_int),
             "moe_dispatch_layout_static": ([S, P, P, ctypes.POINTER(moe_layout), P, P], ctypes.c_int),
-            "moe_debug_grouped_swiglu_engine": ([S, P, P, P, P, P, P, ctypes.c_size_t,
+            "moe_debug_grouped_swiglu_engine": ([S, P, P, P, P, P, P, P, ctypes.c_size_t,
                                                  ctypes.c_int32, P], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
@@ -544,7 +544,7 @@ def grouped_swiglu(shape: Shape, x_perm, expert_offsets, packed, ws, stream=None
                                         _p(packed), _p(h), _p(y_perm), _p(ws), ws.numel(),
                                         _stream(stream)), "moe_grouped_swiglu")
     else:
-        _check(lib().moe_debug_grouped_swiglu_engine(ctypes.byref(s), _p(x_perm),
+        _check(lib().moe_debug_grouped_swiglu_engine(ctypes.byref(s), _p(x_perm), None,
                                                      _p(expert_offsets), _p(packed), _p(h),
                                                      _p(y_perm), _p(ws), ws.numel(), int(engine),
                                                      _stream(stream)),
@@ -552,8 +552,10 @@ def grouped_swiglu(shape: Shape, x_perm, expert_offsets, packed, ws, stream=None
     return h, y_perm
 
 
-def grouped_swiglu_gather(shape: Shape, x, row_token, expert_offsets, packed, ws, stream=None):
-    """moe_grouped_swiglu_gather: (h, y_perm) with rows gathered from x."""
+def grouped_swiglu_gather(shape: Shape, x, row_token, expert_offsets, packed, ws, stream=None,
+                          engine=None):
+    """moe_grouped_swiglu_gather: (h, y_perm) with rows gathered from x.
+    engine: as in grouped_swiglu (test hook)."""
     _need(x, shape.dtype, (shape.T, shape.d), "x")
     _need_n(row_token, torch.int32, shape.R, "row_token")
     _need_n(expert_offsets, torch.int32, shape.E + 1, "expert_offsets")
@@ -561,10 +563,17 @@ def grouped_swiglu_gather(shape: Shape, x, row_token, expert_offsets, packed, ws
     h = torch.empty((shape.R, shape.f), dtype=shape.dtype, device=x.device)
     y_perm = torch.empty((shape.R, shape.d), dtype=shape.dtype, device=x.device)
     s = shape.c
-    _check(lib().moe_grouped_swiglu_gather(ctypes.byref(s), _p(x), _p(row_token),
-                                           _p(expert_offsets), _p(packed), _p(h), _p(y_perm),
-                                           _p(ws), ws.numel(), _stream(stream)),
-           "moe_grouped_swiglu_gather")
+    if engine is None:
+        _check(lib().moe_grouped_swiglu_gather(ctypes.byref(s), _p(x), _p(row_token),
+                                               _p(expert_offsets), _p(packed), _p(h), _p(y_perm),
+                                               _p(ws), ws.numel(), _stream(stream)),
+               "moe_grouped_swiglu_gather")
+    else:
+        _check(lib().moe_debug_grouped_swiglu_engine(ctypes.byref(s), _p(x), _p(row_token),
+                                                     _p(expert_offsets), _p(packed), _p(h),
+                                                     _p(y_perm), _p(ws), ws.numel(), int(engine),
+                                                     _stream(stream)),
+               "moe_debug_grouped_swiglu_engine")
     return h, y_perm
 
 

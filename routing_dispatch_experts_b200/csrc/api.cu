@@ -491,6 +491,25 @@ moe_status route_impl(const moe_shape* s, const void* x, const void* packed, con
   return do_route(s, x, &pk, bias, sel_bias, logits, topk_idx, topk_gate, ctl, st);
 }
 
+moe_status gather_impl(const moe_shape* s, const void* x, const int32_t* row_token,
+                       const int32_t* offsets, const void* packed, void* h, void* y_perm, void* ws,
+                       size_t ws_bytes, int engine, cudaStream_t st) {
+  moe_status r = check_shape(s);
+  if (r != MOE_OK) return r;
+  if (s->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (s->T == 0) return MOE_OK;
+  if (!x || !row_token || !offsets || !packed || !h || !y_perm || !ws) return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(h, 16) || !aligned(y_perm, 16) || !aligned(offsets, 4) ||
+      !aligned(row_token, 4) || !aligned(packed, kAlign) || !aligned(ws, kAlign))
+    return MOE_ERR_ALIGNMENT;
+  if (ws_bytes < scratch_bytes(s)) return MOE_ERR_WORKSPACE;
+  const Packed pk = carve_packed(s, packed);
+  Control* ctl = carve_scratch(s, ws).ctl;
+  if ((r = do_grouped_part(0, s, x, row_token, offsets, &pk, h, y_perm, ctl, st, engine)) != MOE_OK)
+    return r;
+  return do_grouped_part(1, s, x, nullptr, offsets, &pk, h, y_perm, ctl, st, engine);
+}
+
 }  // namespace
 
 extern "C" {
@@ -849,15 +868,19 @@ moe_status moe_permute_by_token(const moe_shape* s, const void* x, const int32_t
 moe_status moe_grouped_swiglu(const moe_shape* s, const void* x_perm, const int32_t* offsets,
                               const void* packed, void* h, void* y_perm, void* ws, size_t ws_bytes,
                               moe_stream_t stream) {
-  return moe_debug_grouped_swiglu_engine(s, x_perm, offsets, packed, h, y_perm, ws, ws_bytes,
-                                         kEngineAuto, stream);
+  return moe_debug_grouped_swiglu_engine(s, x_perm, nullptr, offsets, packed, h, y_perm, ws,
+                                         ws_bytes, kEngineAuto, stream);
 }
 
-moe_status moe_debug_grouped_swiglu_engine(const moe_shape* s, const void* x_perm,
-                                           const int32_t* offsets, const void* packed, void* h,
-                                           void* y_perm, void* ws, size_t ws_bytes, int32_t engine,
-                                           moe_stream_t stream) {
+moe_status moe_debug_grouped_swiglu_engine(const moe_shape* s, const void* a_rows,
+                                           const int32_t* row_token, const int32_t* offsets,
+                                           const void* packed, void* h, void* y_perm, void* ws,
+                                           size_t ws_bytes, int32_t engine, moe_stream_t stream) {
   if (engine < kEngineAuto || engine > kEnginePair) return MOE_ERR_INVALID_ARG;
+  if (row_token)
+    return gather_impl(s, a_rows, row_token, offsets, packed, h, y_perm, ws, ws_bytes, engine,
+                       (cudaStream_t)stream);
+  const void* x_perm = a_rows;
   moe_status r = check_shape(s);
   if (r != MOE_OK) return r;
   if (s->T == 0) return MOE_OK;
@@ -923,20 +946,8 @@ moe_status moe_forward_timed(const moe_shape* s, const void* x, const void* pack
 moe_status moe_grouped_swiglu_gather(const moe_shape* s, const void* x, const int32_t* row_token,
                                      const int32_t* offsets, const void* packed, void* h,
                                      void* y_perm, void* ws, size_t ws_bytes, moe_stream_t stream) {
-  moe_status r = check_shape(s);
-  if (r != MOE_OK) return r;
-  if (s->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
-  if (s->T == 0) return MOE_OK;
-  if (!x || !row_token || !offsets || !packed || !h || !y_perm || !ws) return MOE_ERR_INVALID_ARG;
-  if (!aligned(x, 16) || !aligned(h, 16) || !aligned(y_perm, 16) || !aligned(offsets, 4) ||
-      !aligned(row_token, 4) || !aligned(packed, kAlign) || !aligned(ws, kAlign))
-    return MOE_ERR_ALIGNMENT;
-  if (ws_bytes < scratch_bytes(s)) return MOE_ERR_WORKSPACE;
-  const Packed pk = carve_packed(s, packed);
-  Control* ctl = carve_scratch(s, ws).ctl;
-  cudaStream_t st = (cudaStream_t)stream;
-  if ((r = do_grouped_part(0, s, x, row_token, offsets, &pk, h, y_perm, ctl, st)) != MOE_OK) return r;
-  return do_grouped_part(1, s, x, nullptr, offsets, &pk, h, y_perm, ctl, st);
+  return gather_impl(s, x, row_token, offsets, packed, h, y_perm, ws, ws_bytes, kEngineAuto,
+                     (cudaStream_t)stream);
 }
 
 moe_status moe_get_device_status(void* ws, moe_stream_t stream, moe_status* out) {

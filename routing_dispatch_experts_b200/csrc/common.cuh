@@ -380,6 +380,21 @@ __device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const void* tma
       : "memory");
 }
 
+// Four rows of a 2-D bf16 tensor picked by index (rows r0..r3, columns
+// [c, c + box width)), in a CTA pair: into THIS CTA's shared memory as four
+// consecutive rows of the box width (the swizzled layout of a tile load),
+// counted on an mbarrier in either CTA of the pair.  The tensor map's box is
+// one row high.  Not a multicast.
+__device__ __forceinline__ void tma_gather4_pair(void* smem_dst, const void* tmap,
+                                                 uint32_t bar_cluster, int32_t c, int32_t r0,
+                                                 int32_t r1, int32_t r2, int32_t r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4.mbarrier::"
+      "complete_tx::bytes [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(smem_dst)),
+      "l"(tmap), "r"(bar_cluster), "r"(c), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+      : "memory");
+}
+
 // TMEM allocation for a CTA pair: one warp of EACH CTA executes it; each
 // gets the same column range in its own tensor memory
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst, uint32_t ncols) {

@@ -21,6 +21,12 @@
 // instead of the whole B tile, so more stages fit and each SM pulls half
 // the B bytes through L2 per FLOP.
 //
+// Gather mode (the gate/up GEMM): the permute fused into the operand load.
+// A row r of the tile is row gather[r] of the source (x), so x_perm is never
+// written; each lane of the producer warp loads four of the CTA's 128 rows
+// per k block with one TMA gather4 (rows picked by index, one-row box) into
+// the same swizzled layout a tile load writes, counted on CTA 0's barrier.
+//
 // Every mbarrier wait is bounded (one second); a role that gives up records
 // MOE_ERR_DEVICE_TIMEOUT and raises the abort flag in both CTAs.  The final
 // cluster barrier cannot time out, so every path of every role reaches it.
@@ -41,6 +47,8 @@ constexpr int kThreads = 64 + 32 * kEpiWarps;
 
 struct Params {
   const int32_t* offsets;  // NULL: one group of `rows` rows
+  const int32_t* gather;   // gather mode: A row r is source row gather[r]
+  int64_t src_rows;        // gather mode: rows of the source
   int64_t rows;
   int G, K, n_per_group;
   void* out;
@@ -93,7 +101,7 @@ __device__ __forceinline__ float silu_mul(float g, float u) {
   return __fdividef(g, 1.f + __expf(-g)) * u;
 }
 
-template <int BN, int EPI, bool STAGED>
+template <int BN, int EPI, bool STAGED, bool GATHER>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ Params p) {
@@ -181,7 +189,54 @@ __global__ void __launch_bounds__(kThreads, 1)
     record_error(p.ctl, MOE_ERR_DEVICE_TIMEOUT, detail);
   };
 
-  if (warp == 0) {
+  if (warp == 0 && GATHER) {
+    // the source rows of this lane's four A rows of a tile (rows past the
+    // end of the gather list read row 0; they are never stored)
+    auto rows_of = [&](int tile, int32_t (&src)[4]) {
+      const TileInfo t2 = decode(tile, n_tiles, tile_off, s_off, G);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int64_t r = (int64_t)t2.row0 + (int)rank * BM + 4 * lane + q;
+        const int32_t v = r < p.rows ? __ldg(p.gather + r) : 0;
+        src[q] = (v >= 0 && v < p.src_rows) ? v : 0;
+      }
+    };
+    uint32_t it = 0;
+    bool ok = true;
+    int32_t src[4], nxt[4];
+    if (cluster < total) rows_of(cluster, nxt);
+    for (int tile = cluster; tile < total && ok; tile += nclusters) {
+      const TileInfo ti = decode(tile, n_tiles, tile_off, s_off, G);
+      const int brow = ti.g * p.n_per_group + ti.nt * BN + (int)rank * (BN / 2);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) src[q] = nxt[q];
+      // the next tile's indices load while this tile's rows stream
+      if (tile + nclusters < total) rows_of(tile + nclusters, nxt);
+      for (int kb = 0; kb < kblocks; ++kb, ++it) {
+        const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
+        int good = 1;
+        if (lane == 0) good = mbar_wait_bounded_cluster(&empty[s], ph ^ 1, &abort_flag);
+        good = __shfl_sync(0xffffffffu, good, 0);
+        if (!good) {
+          ok = false;
+          break;
+        }
+        const uint32_t fbar = mapa_shared(&full[s], 0);
+        if (lane == 0) {
+          if (leader) mbar_arrive_expect_tx(&full[s], PAIR_TX);
+          tma_load_2d_pair(sB + s * B_BYTES, &tmB, fbar, kb * BK, brow);
+        }
+        tma_gather4_pair(sA + s * A_BYTES + lane * 4 * (BK * 2), &tmA, fbar, kb * BK, src[0], src[1],
+                         src[2], src[3]);
+      }
+    }
+    if (lane == 0) {
+      if (!ok) abort_pair(0x1100u);
+      const uint32_t first = it > (uint32_t)STAGES ? it - STAGES : 0;
+      for (uint32_t q = first; q < it; ++q)
+        mbar_wait_bounded(&empty[q % STAGES], (q / STAGES) & 1, &abort_flag);
+    }
+  } else if (warp == 0) {
     if (lane == 0) {
       uint32_t it = 0;
       bool ok = true;
@@ -346,17 +401,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int BN, int EPI, bool STAGED>
+template <int BN, int EPI, bool STAGED, bool GATHER>
 cudaError_t run(const GemmArgs& a, cudaStream_t s) {
-  auto kernel = gemm_pair_kernel<BN, EPI, STAGED>;
+  auto kernel = gemm_pair_kernel<BN, EPI, STAGED, GATHER>;
   constexpr size_t smem = smem_bytes_for<BN, EPI, STAGED>();
   cudaError_t e = set_smem_limit((const void*)kernel, smem);
   if (e != cudaSuccess) return e;
   CUtensorMap mA, mB;
-  if (!make_kmajor_map(&mA, a.A, a.rows, a.K, BM)) return cudaErrorInvalidValue;
+  // gather mode: the source rows one at a time (gather4 boxes are one row high)
+  if (!make_kmajor_map(&mA, a.A, GATHER ? a.src_rows : a.rows, a.K, GATHER ? 1 : BM))
+    return cudaErrorInvalidValue;
   if (!make_kmajor_map(&mB, a.B, (int64_t)a.G * a.n_per_group, a.K, BN / 2)) return cudaErrorInvalidValue;
   Params p;
   p.offsets = a.offsets;
+  p.gather = a.gather;
+  p.src_rows = a.src_rows;
   p.rows = a.rows;
   p.G = a.offsets ? a.G : 1;
   p.K = a.K;
@@ -410,8 +469,9 @@ cudaError_t run(const GemmArgs& a, cudaStream_t s) {
 }  // namespace
 
 bool gemm_pair_supported(int epi, int bn, const GemmArgs& a) {
-  return bn == 256 && a.gather == nullptr && (epi == kEpiSwiGLU || epi == kEpiBF16) &&
-         a.n_per_group % bn == 0;
+  // the row gather is the gate/up GEMM's (SwiGLU epilogue)
+  return bn == 256 && (epi == kEpiSwiGLU || (epi == kEpiBF16 && a.gather == nullptr)) &&
+         a.n_per_group % bn == 0 && (a.gather == nullptr || a.src_rows > 0);
 }
 
 cudaError_t launch_gemm_pair(int epi, int bn, const GemmArgs& a, cudaStream_t s) {
@@ -419,8 +479,11 @@ cudaError_t launch_gemm_pair(int epi, int bn, const GemmArgs& a, cudaStream_t s)
   if (!gemm_pair_supported(epi, bn, a)) return cudaErrorInvalidValue;
   // short K loops stage the epilogue (as in gemm_tc.cu)
   const bool st = a.K / BK <= (epi == kEpiBF16 ? 24 : 8);
-  if (epi == kEpiSwiGLU) return st ? run<256, kEpiSwiGLU, true>(a, s) : run<256, kEpiSwiGLU, false>(a, s);
-  return st ? run<256, kEpiBF16, true>(a, s) : run<256, kEpiBF16, false>(a, s);
+  const bool g = a.gather != nullptr;
+  if (epi == kEpiSwiGLU)
+    return g ? (st ? run<256, kEpiSwiGLU, true, true>(a, s) : run<256, kEpiSwiGLU, false, true>(a, s))
+             : (st ? run<256, kEpiSwiGLU, true, false>(a, s) : run<256, kEpiSwiGLU, false, false>(a, s));
+  return st ? run<256, kEpiBF16, true, false>(a, s) : run<256, kEpiBF16, false, false>(a, s);
 }
 
 }  // namespace moe

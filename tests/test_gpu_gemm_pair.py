@@ -62,3 +62,22 @@ def test_pair_engine_bit_identical_on_workload_routing(cfg, T):
     a, b, d = _both(c.shape, x_perm, lay["expert_offsets"], c.packed)
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
     assert torch.equal(b[1], d[1])
+
+
+@pytest.mark.parametrize("cfg,T", [(3, 3000), (5, 1500)])
+def test_pair_gather_equals_permute_then_grouped(cfg, T):
+    """The permute fused into the gate/up operand load: the pair engine's
+    TMA gather4 of x rows, the one-CTA engine's cp.async gather, and the
+    separate permute + grouped GEMM give the same h and y_perm bit for bit,
+    with some rows of x picked by no expert group's tail (ragged groups)."""
+    c = Case(cfg, T=T, near_ties=False)
+    ws = moe.workspace(c.shape)
+    _, idx, _ = moe.route(c.shape, c.dx, c.packed, c.dbias, ws)
+    lay = moe.dispatch_layout(c.shape, idx, ws)
+    x_perm = moe.permute(c.shape, c.dx, lay["row_token"])
+    h0, y0 = moe.grouped_swiglu(c.shape, x_perm, lay["expert_offsets"], c.packed, ws, engine=2)
+    outs = [moe.grouped_swiglu_gather(c.shape, c.dx, lay["row_token"], lay["expert_offsets"],
+                                      c.packed, ws, engine=e) for e in (1, 2, None)]
+    moe.check_device_status(ws)
+    for h, y in outs:
+        assert torch.equal(h, h0) and torch.equal(y, y0)
