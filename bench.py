@@ -634,12 +634,13 @@ def run_kernel(args):
         elif k == "permute_by_token":
             r = L.moe_permute_by_token(ctypes.byref(sc), P(x), P(lay["slot_row"]), P(out), st)
         elif k == "grouped":
-            r = L.moe_grouped_swiglu(ctypes.byref(sc), P(x_perm), P(lay["expert_offsets"]),
-                                     P(packed), P(h), P(y_perm), P(ws), ws.numel(), st)
+            r = L.moe_debug_grouped_swiglu_engine(ctypes.byref(sc), P(x_perm), None,
+                                                  P(lay["expert_offsets"]), P(packed), P(h),
+                                                  P(y_perm), P(ws), ws.numel(), args.engine, st)
         elif k == "grouped_gather":
-            r = L.moe_grouped_swiglu_gather(ctypes.byref(sc), P(x), P(lay["row_token"]),
-                                            P(lay["expert_offsets"]), P(packed), P(h),
-                                            P(y_perm), P(ws), ws.numel(), st)
+            r = L.moe_debug_grouped_swiglu_engine(ctypes.byref(sc), P(x), P(lay["row_token"]),
+                                                  P(lay["expert_offsets"]), P(packed), P(h),
+                                                  P(y_perm), P(ws), ws.numel(), args.engine, st)
         elif k == "combine":
             r = L.moe_combine(ctypes.byref(sc), P(y_perm), P(lay["slot_row"]), P(gate), P(out), st)
         elif k == "stats":
@@ -689,7 +690,7 @@ def run_kernel(args):
     d = [(run(g1) - run(g0)) / reps for _ in range(args.time)]
     moe.check_device_status(ws)
     us = statistics.median(d)
-    print(json.dumps({"kernel": args.kernel, "config": args.config, "T": T, "E": E,
+    print(json.dumps({"kernel": args.kernel, "engine": args.engine, "config": args.config, "T": T, "E": E,
                       "us_median": us, "us_min": min(d), "us_max": max(d), "reps": args.time}))
 
 
@@ -710,6 +711,9 @@ def main():
     ap.add_argument("--experts", type=int, default=0, help="--kernel: expert count (default: the workload's)")
     ap.add_argument("--launches", type=int, default=5, help="--kernel: launches before exit")
     ap.add_argument("--time", type=int, default=0, metavar="REPS", help="--kernel: timing repetitions")
+    ap.add_argument("--engine", type=int, default=0, choices=(0, 1, 2),
+                    help="--kernel grouped*: GEMM engine (0 library's choice, 1 one CTA per "
+                         "tile, 2 CTA pairs)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.kernel:
