@@ -112,40 +112,65 @@ cudaError_t launch_topk(const float* logits, const float* sel_bias, int64_t T, i
   return cudaGetLastError();
 }
 
-// fp32 router on CUDA cores: logits[t,e] = sum_i x[t,i] W_r^T[e,i] + bias[e],
-// one thread per (t, e), i ascending.  Threads of a warp share t (the x row is
-// a broadcast) and walk consecutive experts.
-__global__ void __launch_bounds__(256) router_f32_kernel(const float* __restrict__ x,
-                                                         const float* __restrict__ wrT,
-                                                         const float* __restrict__ bias,
-                                                         int64_t T, int d, int E,
-                                                         float* __restrict__ logits) {
+// fp32 router on CUDA cores: logits[t,e] = sum_i x[t,i] W_r^T[e,i] + bias[e].
+// One warp per token, experts in groups of 16: lane l accumulates, for each
+// expert of the group, the products of the elements i = 4l .. 4l+3 of every
+// 128-element chunk of d (chunks ascending), then a butterfly over the 32
+// lanes sums the partials; lane j < 16 holds expert j's logit.  The x row is
+// read through L1 once per expert group; W_r^T rows are read by every warp
+// of the block from L1/L2.  The summation order is fixed, so the logits are
+// identical on every run.
+constexpr int kRouterWarps = 8;
+
+__global__ void __launch_bounds__(32 * kRouterWarps)
+    router_f32_kernel(const float* __restrict__ x, const float* __restrict__ wrT,
+                      const float* __restrict__ bias, int64_t T, int d, int E,
+                      float* __restrict__ logits) {
   pdl_wait();
-  const int64_t o = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (o >= T * E) return;
-  const int64_t t = o / E;
-  const int e = (int)(o % E);
+  const int lane = threadIdx.x & 31;
+  const int64_t t = (int64_t)blockIdx.x * kRouterWarps + (threadIdx.x >> 5);
+  if (t >= T) return;  // uniform per warp
   const float4* xr = reinterpret_cast<const float4*>(x + t * d);
-  const float4* wr = reinterpret_cast<const float4*>(wrT + (int64_t)e * d);
-  float s = 0.f;
-  for (int i = 0; i < d / 4; ++i) {
-    const float4 a = __ldg(xr + i);
-    const float4 b = __ldg(wr + i);
-    s = fmaf(a.x, b.x, s);
-    s = fmaf(a.y, b.y, s);
-    s = fmaf(a.z, b.z, s);
-    s = fmaf(a.w, b.w, s);
+  const int nch = d / 128;  // d % 64 == 0: the last chunk may be half
+  const int tail = (d % 128) / 4;  // float4s in a half chunk (0 or 16)
+  for (int e0 = 0; e0 < E; e0 += 16) {
+    float acc[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) acc[j] = 0.f;
+    for (int c = 0; c <= nch; ++c) {
+      const int v = c * 32 + lane;  // float4 index in the row
+      if (c == nch && lane >= tail) break;
+      const float4 a = __ldg(xr + v);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        if (e0 + j < E) {
+          const float4 w = __ldg(reinterpret_cast<const float4*>(wrT + (int64_t)(e0 + j) * d) + v);
+          acc[j] = fmaf(a.x, w.x, acc[j]);
+          acc[j] = fmaf(a.y, w.y, acc[j]);
+          acc[j] = fmaf(a.z, w.z, acc[j]);
+          acc[j] = fmaf(a.w, w.w, acc[j]);
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], off);
+    float mine = 0.f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (lane == j) mine = acc[j];
+    const int e = e0 + lane;
+    if (lane < 16 && e < E) logits[t * E + e] = bias ? mine + __ldg(bias + e) : mine;
   }
-  if (bias) s += bias[e];
-  logits[o] = s;
 }
 
 cudaError_t launch_router_f32(const float* x, const float* wrT, const float* bias, int64_t T,
                               int d, int E, float* logits, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
-  const int64_t n = T * E;
-  return launch_pdl(router_f32_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, x, wrT,
-                    bias, T, d, E, logits);
+  const unsigned grid = (unsigned)((T + kRouterWarps - 1) / kRouterWarps);
+  return launch_pdl(router_f32_kernel, dim3(grid), dim3(32 * kRouterWarps), 0, s, x, wrT, bias,
+                    T, d, E, logits);
 }
 
 }  // namespace moe
