@@ -711,9 +711,9 @@ def main():
     ap.add_argument("--experts", type=int, default=0, help="--kernel: expert count (default: the workload's)")
     ap.add_argument("--launches", type=int, default=5, help="--kernel: launches before exit")
     ap.add_argument("--time", type=int, default=0, metavar="REPS", help="--kernel: timing repetitions")
-    ap.add_argument("--engine", type=int, default=0, choices=(0, 1, 2),
+    ap.add_argument("--engine", type=int, default=0, choices=(0, 1, 2, 3, 4),
                     help="--kernel grouped*: GEMM engine (0 library's choice, 1 one CTA per "
-                         "tile, 2 CTA pairs)")
+                         "tile, 2 CTA pairs, 3 pairs for the down GEMM, 4 for gate/up)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.kernel:

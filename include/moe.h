@@ -675,10 +675,13 @@ MOE_API moe_status moe_debug_dispatch_layout_stall(const moe_shape* shape,
  * is x_perm) and moe_grouped_swiglu_gather (row_token given: a_rows is x):
  * the same call with the tensor-core GEMM engine chosen by the caller.
  *  engine 0  the library's choice (what those calls run)
- *         1  one CTA per 128-row tile (the gather by cp.async)
+ *         1  one CTA per 128-row tile for both GEMMs (the gather by
+ *            cp.async)
  *         2  CTA pairs on 256-row tiles (tcgen05 cta_group::2; the gather
- *            by TMA gather4) where the shape allows it (bf16, 256-column
- *            tiles), else as 1
+ *            by TMA gather4) for both GEMMs where the shape allows it (bf16,
+ *            256-column tiles), else as 1
+ *         3  CTA pairs for the down GEMM only
+ *         4  CTA pairs for the gate/up GEMM only
  * All engines sum every output in the same order, so h and y_perm are
  * bit-identical across engines.  MOE_ERR_INVALID_ARG for another engine.
  */

@@ -199,12 +199,38 @@ moe_status do_layout(const moe_shape* s, const int32_t* idx, const RankMap& map,
 // gate/up GEMM + SwiGLU (part 0) or down GEMM (part 1).  With `gather`
 // (bf16 only) the gate/up GEMM reads its rows straight from x through the
 // permutation instead of from x_perm.
-// Which tensor-core GEMM engine runs a grouped GEMM: the CTA-pair kernel
-// (256-row tiles, gemm_pair.cu) where it applies, else one CTA per tile.
-enum Engine { kEngineAuto = 0, kEngineSingle = 1, kEnginePair = 2 };
+// Which tensor-core GEMM engine runs a grouped GEMM: one CTA per 128-row
+// tile (gemm_tc.cu) or CTA pairs on 256-row tiles (gemm_pair.cu).
+enum Engine {
+  kEngineAuto = 0,       // the library's choice (below)
+  kEngineSingle = 1,     // one CTA per tile for both GEMMs
+  kEnginePair = 2,       // CTA pairs for both GEMMs where they apply
+  kEnginePairDown = 3,   // CTA pairs for the down GEMM only
+  kEnginePairGateUp = 4  // CTA pairs for the gate/up GEMM only
+};
+
+// The library's choice, from full-size measurements on B200 (one flushed
+// call of both GEMMs): CTA pairs pay for the down GEMM with a long K loop
+// (the large workload's f = 1536: -10% per clock; its staged epilogue leaves
+// the one-CTA ring three stages deep), not for the gate/up GEMM (more DRAM
+// re-reads of its operands: 9.06 vs 7.0 GB per large-workload launch) nor
+// for the top-2 workload's GEMMs; the pair's TMA gather4 row gather issues
+// 32 row loads per stage and measured twice as slow as the one-CTA cp.async
+// gather.
+bool pair_chosen(int epi, const GemmArgs& a) {
+  return epi == kEpiBF16 && a.gather == nullptr && a.K >= 24 * 64;
+}
 
 cudaError_t launch_gemm(int epi, int bn, const GemmArgs& a, int engine, cudaStream_t st) {
-  if (engine != kEngineSingle && gemm_pair_supported(epi, bn, a)) return launch_gemm_pair(epi, bn, a, st);
+  bool pair = false;
+  switch (engine) {
+    case kEnginePair: pair = true; break;
+    case kEnginePairDown: pair = epi == kEpiBF16; break;
+    case kEnginePairGateUp: pair = epi == kEpiSwiGLU; break;
+    case kEngineAuto: pair = pair_chosen(epi, a); break;
+    default: break;
+  }
+  if (pair && gemm_pair_supported(epi, bn, a)) return launch_gemm_pair(epi, bn, a, st);
   return launch_gemm_tc(epi, bn, a, st);
 }
 
@@ -876,7 +902,7 @@ moe_status moe_debug_grouped_swiglu_engine(const moe_shape* s, const void* a_row
                                            const int32_t* row_token, const int32_t* offsets,
                                            const void* packed, void* h, void* y_perm, void* ws,
                                            size_t ws_bytes, int32_t engine, moe_stream_t stream) {
-  if (engine < kEngineAuto || engine > kEnginePair) return MOE_ERR_INVALID_ARG;
+  if (engine < kEngineAuto || engine > kEnginePairGateUp) return MOE_ERR_INVALID_ARG;
   if (row_token)
     return gather_impl(s, a_rows, row_token, offsets, packed, h, y_perm, ws, ws_bytes, engine,
                        (cudaStream_t)stream);
