@@ -97,6 +97,19 @@ def test_forward_matches_oracle(cfg, T, ep, placement):
     _check_layout(buf, c.w.E, ep, rmap)
 
 
+def test_forward_two_router_tiles_per_cta():
+    """The fine-grained workload at 19205 tokens (151 router tiles, more than
+    the SMs): the router's per-tile histograms come from CTAs holding two
+    tiles (the last one a single tile); the whole layout is bit-exact against
+    the oracle's layout of the GPU's routing, and the output matches."""
+    c = Case(2, T=19205)
+    y, buf, shape = _run(c, ep=8)
+    _check_layout(buf, c.w.E, 8, None)
+    toks = np.unique(np.concatenate([[0, c.T - 1], W.sample_tokens(c.T, 64, seed=9).numpy()]))
+    bad, _, _ = _compare(c, y, buf, tokens=toks)
+    assert len(bad) <= 2
+
+
 @pytest.mark.parametrize("cfg", [5, 4, 3, 2])
 def test_forward_full_size_sampled(cfg):
     """The benchmarked launch configuration at the workload's full size (its

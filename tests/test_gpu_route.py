@@ -118,6 +118,27 @@ def test_bf16_router_logit_layouts_and_ragged_tiles(T, d, E, k):
     np.testing.assert_allclose(gate.cpu().double().numpy(), ref_gate, rtol=0, atol=1e-6)
 
 
+@pytest.mark.parametrize("T,d,E,k", [(19205, 256, 64, 4), (19205, 128, 36, 5), (19205, 64, 12, 3),
+                                     (20000, 256, 128, 8), (19205, 128, 64, 16),
+                                     (19205, 64, 256, 6)])
+def test_bf16_router_two_tiles_per_cta(T, d, E, k):
+    """More 128-token tiles than SMs (151 or 157 tiles): each CTA routes two
+    tiles that share every W_r block of its ring (the last CTA one when the
+    count is odd).  Same checks as above for every way the logits leave the
+    SM and for k up to 16."""
+    x, wr, shape, packed = _bf16_router_case(T, d, E, k, seed=T + 3 * E)
+    ws = moe.workspace(shape)
+    logits, idx, gate = moe.route(shape, x.cuda(), packed, None, ws)
+    moe.check_device_status(ws)
+    ref = oracle.router_logits(x, wr)
+    mag = (x.double().abs() @ wr.double().abs()).numpy()
+    err = np.abs(logits.cpu().double().numpy() - ref)
+    assert (err <= 1e-5 * mag + 1e-6).all()
+    ref_idx, ref_gate = oracle.topk(logits.cpu().double().numpy(), k)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ref_idx)
+    np.testing.assert_allclose(gate.cpu().double().numpy(), ref_gate, rtol=0, atol=1e-6)
+
+
 def test_bf16_router_unaligned_logits_buffer():
     """A logits buffer that is only 4-byte aligned takes the per-thread
     store path and gives the same bits as an aligned one."""

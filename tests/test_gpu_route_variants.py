@@ -64,7 +64,7 @@ def test_selection_bias_given_logits(T, E, k):
     assert torch.equal(i0, i1) and torch.equal(g0, g1)
 
 
-@pytest.mark.parametrize("cfg,T", [(2, 1000), (3, 300), (5, 257)])
+@pytest.mark.parametrize("cfg,T", [(2, 1000), (3, 300), (5, 257), (2, 19205)])
 def test_selection_bias_fused_router(cfg, T):
     """bf16: the fused router picks on logits + bias and weights by logits;
     its logits equal moe_route's bit for bit (the bias is not added)."""
