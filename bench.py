@@ -81,9 +81,10 @@ def peaks():
 # holds the summary); None where no capture of the current kernel exists
 NCU_TRAFFIC = {
     (2, "gate_up"): 14_992_128 + 89_088,  # ffn_fused_kernel<64, 256, gather>
-    # gemm_pair_kernel<256, SwiGLU>: a quarter-size capture (32 of 128
-    # experts, same rows per expert) scaled by 4
-    (5, "gate_up"): 4 * (2_064_719_000 + 199_382_016),
+    # gemm_tc_kernel<256, SwiGLU> (one CTA per tile, the forward's gate/up
+    # engine on this workload): a quarter-size capture (32 of 128 experts,
+    # same rows per expert) scaled by 4
+    (5, "gate_up"): 4 * (1_551_803_136 + 197_091_072),
 }
 
 
