@@ -550,7 +550,8 @@ def run_reference(args, rank, world):
 
 # ------------------------------------------------- one kernel, for profilers
 KERNELS = ("route", "topk", "layout", "permute", "permute_by_token", "grouped",
-           "grouped_gather", "combine", "forward", "stats", "capacity")
+           "grouped_gather", "combine", "forward", "stats", "capacity", "coselection", "ep_pack",
+           "ep_home")
 
 
 def run_kernel(args):
@@ -568,6 +569,10 @@ def run_kernel(args):
       forward          moe_forward
       stats            moe_router_stats (margin, near-tie count)
       capacity         moe_capacity_keep (capacity factor 1.25)
+      coselection      moe_coselection_counts (W[e,e'])
+      ep_pack          moe_ep_pack (this rank's deduplicated send rows, ep = the
+                       workload's EP degree)
+      ep_home          moe_ep_home_combine (one returned row per send row)
 
     Routing comes from the workload's own router on its own x; expert
     weights are seeded N(0, 1/d) stand-ins drawn on the device (values do
@@ -615,7 +620,13 @@ def run_kernel(args):
     idx2 = torch.empty_like(idx)
     gate2 = torch.empty_like(gate)
     counts = torch.zeros(5, dtype=torch.int64, device=dev)
+    cosel = torch.empty((E, E), dtype=torch.int64, device=dev)
+    send_rows = int(lay["rank_offsets"][-1]) if ep > 1 else 0
+    if args.kernel in ("ep_pack", "ep_home"):
+        send = moe.ep_pack(shape, x, idx, gate, lay, send_rows) if ep > 1 else None
+        y_back = send[0] if send is not None else None
     clay = moe._c_layout(moe._layout_tensors(shape, dev))
+    clay_ep = moe._c_layout(lay)
     rmap = None
 
     def launch(stream=None):
@@ -647,6 +658,14 @@ def run_kernel(args):
         elif k == "stats":
             r = L.moe_router_stats(ctypes.byref(sc), P(logits), None, P(idx), None, 1e-5, None,
                                    P(counts), st)
+        elif k == "coselection":
+            r = L.moe_coselection_counts(ctypes.byref(sc), P(idx), P(cosel), P(ws), ws.numel(), st)
+        elif k == "ep_pack":
+            r = L.moe_ep_pack(ctypes.byref(sc), P(x), P(idx), P(gate), None, ctypes.byref(clay_ep),
+                              P(send[0]), P(send[1]), P(send[2]), send_rows, st)
+        elif k == "ep_home":
+            r = L.moe_ep_home_combine(ctypes.byref(sc), P(y_back), P(lay["slot_send_row"]),
+                                      send_rows, P(out), st)
         elif k == "capacity":
             r = L.moe_capacity_keep(ctypes.byref(sc), P(idx), P(gate), 1.25, P(idx2), P(gate2),
                                     None, P(ws), ws.numel(), st)
