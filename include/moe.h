@@ -651,6 +651,92 @@ MOE_API moe_status moe_ep_home_combine(const moe_shape* shape, const void* y_bac
                                        moe_stream_t stream);
 
 /*
+ * Peer-memory exchange: the pack fused with the dispatch all-to-all, and the
+ * experts' return rows fused with the reverse one.  Each kernel stores its
+ * rows straight into the other ranks' buffers, which the caller has mapped
+ * into this process (this GPU's own memory, or another GPU's over NVLink
+ * through a peer mapping: CUDA IPC, a symmetric-memory allocation, a
+ * cudaDeviceEnablePeerAccess'd allocation).  Plain 16-byte stores only:
+ * nothing reads a peer's memory.  The rows, their order within each block
+ * and every value are those of moe_ep_pack + all-to-all and
+ * moe_ep_expert_forward + reverse all-to-all; only where the bytes are
+ * written changes.  Rank order of the blocks: source rank s's rows at rank
+ * r start at row sum_{s' < s} counts[s'][r] of r's receive buffers (counts
+ * = every rank's rank_counts, exchanged first), and return rows go back to
+ * the send-row position they left from.
+ * Between the phases every rank must have finished storing before any
+ * rank reads: moe_ep_signal_wait on each rank (or a host barrier after a
+ * stream synchronisation).
+ */
+typedef struct moe_ep_peer_dest {
+  void* recv_x;       /* rank r's receive rows [.., d] (dtype) */
+  int32_t* recv_idx;  /* rank r's receive local expert ids [.., k] */
+  float* recv_gate;   /* rank r's receive gates [.., k] */
+  int64_t row0;       /* first row of this rank's block there */
+  int64_t rows;       /* rows of the block: rank_counts[r] of this rank */
+} moe_ep_peer_dest;
+
+/*
+ * moe_ep_pack whose send rows for rank r (rows rank_offsets[r] ..
+ * rank_offsets[r+1] of the send plan) are stored at rows dests_host[r].row0 ..
+ * of rank r's receive buffers.  dests_host: P entries (host); a block of 0
+ * rows needs no buffers.  Send rows past dests_host[r].rows are not stored
+ * (size rows from the exchanged counts).  Other arguments as moe_ep_pack.
+ */
+MOE_API moe_status moe_ep_dispatch_peer(const moe_shape* shape, const void* x,
+                                        const int32_t* topk_idx, const float* topk_gate,
+                                        const int32_t* expert_rank_host,
+                                        const moe_layout* layout,
+                                        const moe_ep_peer_dest* dests_host, moe_stream_t stream);
+
+typedef struct moe_ep_peer_return {
+  void* y_back;  /* source rank s's return rows [.., d] (its send-row order) */
+  int64_t row0;  /* where this rank's rows start there: rank_offsets[me] of s */
+  int64_t rows;  /* rows this rank received from s: counts[s][me] */
+} moe_ep_peer_return;
+
+/*
+ * moe_ep_expert_forward whose return rows go straight back: the received
+ * rows are the blocks of the source ranks in rank order (rets_host[s].rows
+ * rows each, summing to shape->T), and return row i of source s's block is
+ * stored at row rets_host[s].row0 + i of s's y_back.  Invalid argument when
+ * the blocks do not sum to shape->T.  Other arguments as
+ * moe_ep_expert_forward.
+ */
+MOE_API moe_status moe_ep_expert_forward_peer(const moe_shape* shape, const void* recv_x,
+                                              const int32_t* recv_idx, const float* recv_gate,
+                                              const void* packed_local,
+                                              const moe_ep_peer_return* rets_host, void* ws,
+                                              size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * The ranks' rendezvous on device: one kernel stores `epoch` into slot
+ * `rank` of every rank's flag array (a system-scope release after all
+ * earlier work of `stream`, so this rank's stores into peers' buffers are
+ * visible first) and waits until every slot of its own array holds at least
+ * `epoch` (system-scope acquire).  flags_host: P device pointers (host
+ * array), each rank's array of P uint64 slots, zero-filled before the first
+ * epoch; epochs start at 1 and grow by one per rendezvous.  The wait gives
+ * up after one second and records MOE_ERR_DEVICE_TIMEOUT (detail: the first
+ * rank missing) in the control block of `ws` (any workspace of this
+ * library; read with moe_get_device_status).  Every rank must call it once
+ * per epoch on its own GPU: kernels that wait for one another must run on
+ * different GPUs at the same time.
+ * No counterpart in the pages, which leave the exchange to the library
+ * they run on.
+ */
+MOE_API moe_status moe_ep_signal_wait(uint64_t* const* flags_host, int32_t rank, int32_t P,
+                                      uint64_t epoch, void* ws, moe_stream_t stream);
+
+/*
+ * Test hook: moe_ep_signal_wait with the wait limited to wait_limit_ns
+ * (0 < wait_limit_ns <= one second).
+ */
+MOE_API moe_status moe_debug_ep_signal_wait(uint64_t* const* flags_host, int32_t rank,
+                                            int32_t P, uint64_t epoch, void* ws,
+                                            int64_t wait_limit_ns, moe_stream_t stream);
+
+/*
  * Synchronise `stream`, read the device status word of workspace `ws`
  * (MOE_OK, MOE_ERR_DEVICE_TIMEOUT or MOE_ERR_DEVICE_INDEX) into *out and
  * reset it to MOE_OK.  Returns MOE_ERR_CUDA if the stream reports an error.

@@ -72,6 +72,15 @@ class moe_layout(ctypes.Structure):
         "rank_offsets", "send_token", "slot_send_row", "stats")]
 
 
+class moe_ep_peer_dest(ctypes.Structure):
+    _fields_ = [("recv_x", ctypes.c_void_p), ("recv_idx", ctypes.c_void_p),
+                ("recv_gate", ctypes.c_void_p), ("row0", ctypes.c_int64), ("rows", ctypes.c_int64)]
+
+
+class moe_ep_peer_return(ctypes.Structure):
+    _fields_ = [("y_back", ctypes.c_void_p), ("row0", ctypes.c_int64), ("rows", ctypes.c_int64)]
+
+
 class moe_forward_buffers(ctypes.Structure):
     _fields_ = [("logits", ctypes.c_void_p), ("topk_idx", ctypes.c_void_p),
                 ("topk_gate", ctypes.c_void_p), ("layout", moe_layout),
@@ -88,7 +97,9 @@ SYMBOLS = ("moe_status_string", "moe_scratch_size", "moe_forward_workspace_size"
            "moe_dispatch_layout", "moe_coselection_counts", "moe_fit_placement", "moe_permute", "moe_permute_by_token", "moe_grouped_swiglu",
            "moe_grouped_swiglu_gather", "moe_combine", "moe_forward", "moe_forward_selection_bias", "moe_forward_timed",
            "moe_forward_routed", "moe_ep_pack", "moe_ep_expert_workspace_size",
-           "moe_ep_expert_forward", "moe_ep_home_combine", "moe_get_device_status", "moe_debug_dispatch_layout_stall",
+           "moe_ep_expert_forward", "moe_ep_home_combine", "moe_ep_dispatch_peer",
+           "moe_ep_expert_forward_peer", "moe_ep_signal_wait", "moe_debug_ep_signal_wait",
+           "moe_get_device_status", "moe_debug_dispatch_layout_stall",
            "moe_debug_grouped_swiglu_engine", "moe_dispatch_layout_static")
 FORWARD_STAGES = ("route", "layout", "permute", "gate_up", "down", "combine")
 
@@ -144,6 +155,15 @@ def lib() -> ctypes.CDLL:
             "moe_ep_expert_workspace_size": ([S, sz], ctypes.c_int),
             "moe_ep_expert_forward": ([S, P, P, P, P, P, P, ctypes.c_size_t, P], ctypes.c_int),
             "moe_ep_home_combine": ([S, P, P, ctypes.c_int64, P, P], ctypes.c_int),
+            "moe_ep_dispatch_peer": ([S, P, P, P, P, ctypes.POINTER(moe_layout),
+                                      ctypes.POINTER(moe_ep_peer_dest), P], ctypes.c_int),
+            "moe_ep_expert_forward_peer": ([S, P, P, P, P, ctypes.POINTER(moe_ep_peer_return), P,
+                                            ctypes.c_size_t, P], ctypes.c_int),
+            "moe_ep_signal_wait": ([ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32,
+                                    ctypes.c_int32, ctypes.c_uint64, P, P], ctypes.c_int),
+            "moe_debug_ep_signal_wait": ([ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32,
+                                          ctypes.c_int32, ctypes.c_uint64, P, ctypes.c_int64, P],
+                                         ctypes.c_int),
             "moe_get_device_status": ([P, P, ctypes.POINTER(ctypes.c_int)], ctypes.c_int),
             "moe_debug_dispatch_layout_stall": ([S, P, P, ctypes.POINTER(moe_layout), P,
                                                  ctypes.c_size_t, ctypes.c_int32, ctypes.c_int64, P],
@@ -746,6 +766,79 @@ def ep_home_combine(shape: Shape, y_back, slot_send_row, stream=None):
                                      int(y_back.shape[0]), _p(y), _stream(stream)),
            "moe_ep_home_combine")
     return y
+
+
+def ep_dispatch_peer(shape: Shape, x, topk_idx, topk_gate, layout: dict, dests,
+                     expert_rank=None, stream=None):
+    """moe_ep_dispatch_peer: this rank's send rows stored straight into the
+    destination ranks' receive buffers.  dests: P tuples (recv_x, recv_idx,
+    recv_gate, row0, rows), the buffers as tensors (or None for rows == 0)
+    addressable from this process."""
+    _need(x, shape.dtype, (shape.T, shape.d), "x")
+    _need(topk_idx, torch.int32, (shape.T, shape.k), "topk_idx")
+    if topk_gate is not None:
+        _need(topk_gate, torch.float32, (shape.T, shape.k), "topk_gate")
+    _need_n(layout["rank_offsets"], torch.int32, shape.ep + 1, "rank_offsets")
+    if len(dests) != shape.ep:
+        raise ValueError(f"dests: expected {shape.ep} entries")
+    arr = (moe_ep_peer_dest * shape.ep)()
+    for r, (rx, ri, rg, row0, rows) in enumerate(dests):
+        if rows > 0:
+            for t, dt, w, nm in ((rx, shape.dtype, shape.d, "recv_x"),
+                                 (ri, torch.int32, shape.k, "recv_idx"),
+                                 (rg, torch.float32, shape.k, "recv_gate")):
+                if (t.dtype != dt or t.dim() != 2 or t.shape[1] != w or not t.is_contiguous()
+                        or row0 + rows > t.shape[0]):
+                    raise ValueError(f"{nm} of rank {r}: expected contiguous {dt} "
+                                     f"[>= {row0 + rows}, {w}]")
+        arr[r] = moe_ep_peer_dest(_p(rx), _p(ri), _p(rg), int(row0), int(rows))
+    lay = _c_layout(layout)
+    s = shape.c
+    _check(lib().moe_ep_dispatch_peer(ctypes.byref(s), _p(x), _p(topk_idx), _p(topk_gate),
+                                      _host_map(shape, expert_rank), ctypes.byref(lay), arr,
+                                      _stream(stream)), "moe_ep_dispatch_peer")
+
+
+def ep_expert_forward_peer(shape: Shape, recv_x, recv_idx, recv_gate, packed_local, rets, ws,
+                           stream=None):
+    """moe_ep_expert_forward_peer over shape.T received rows: the return rows
+    stored straight into the source ranks' buffers.  rets: P tuples (y_back,
+    row0, rows), y_back a tensor (or None for rows == 0) addressable from
+    this process."""
+    _need(recv_x, shape.dtype, (shape.T, shape.d), "recv_x")
+    _need(recv_idx, torch.int32, (shape.T, shape.k), "recv_idx")
+    _need(recv_gate, torch.float32, (shape.T, shape.k), "recv_gate")
+    if len(rets) != shape.ep:
+        raise ValueError(f"rets: expected {shape.ep} entries")
+    arr = (moe_ep_peer_return * shape.ep)()
+    for r, (yb, row0, rows) in enumerate(rets):
+        if rows > 0 and (yb.dtype != shape.dtype or yb.dim() != 2 or yb.shape[1] != shape.d
+                         or not yb.is_contiguous() or row0 + rows > yb.shape[0]):
+            raise ValueError(f"y_back of rank {r}: expected contiguous {shape.dtype} "
+                             f"[>= {row0 + rows}, {shape.d}]")
+        arr[r] = moe_ep_peer_return(_p(yb), int(row0), int(rows))
+    s = shape.c
+    _check(lib().moe_ep_expert_forward_peer(ctypes.byref(s), _p(recv_x), _p(recv_idx),
+                                            _p(recv_gate), _p(packed_local), arr, _p(ws),
+                                            ws.numel(), _stream(stream)),
+           "moe_ep_expert_forward_peer")
+
+
+def ep_signal_wait(flags, rank: int, epoch: int, ws, wait_limit_ns=None, stream=None):
+    """moe_ep_signal_wait (or its test hook with wait_limit_ns): flags = every
+    rank's flag array (uint64 [P] tensors, stored as int64), addressable
+    from this process."""
+    P = len(flags)
+    arr = (ctypes.c_void_p * P)(*[_p(f) for f in flags])
+    for f in flags:
+        if f.dtype != torch.int64 or f.numel() < P:
+            raise ValueError(f"flags: expected int64 tensors of >= {P} slots")
+    if wait_limit_ns is None:
+        _check(lib().moe_ep_signal_wait(arr, rank, P, epoch, _p(ws), _stream(stream)),
+               "moe_ep_signal_wait")
+    else:
+        _check(lib().moe_debug_ep_signal_wait(arr, rank, P, epoch, _p(ws), int(wait_limit_ns),
+                                              _stream(stream)), "moe_debug_ep_signal_wait")
 
 
 def get_device_status(ws, stream=None) -> int:

@@ -812,7 +812,51 @@ moe_status moe_ep_pack(const moe_shape* s, const void* x, const int32_t* topk_id
   }
   return cuda_status(launch_ep_pack(s->dtype, x, s->T, s->d, s->k, topk_idx, topk_gate,
                                     layout->send_token, layout->rank_offsets, s->ep, m, s->E,
-                                    send_x, send_idx, send_gate, send_rows, (cudaStream_t)stream));
+                                    send_x, send_idx, send_gate, send_rows, nullptr,
+                                    (cudaStream_t)stream));
+}
+
+moe_status moe_ep_dispatch_peer(const moe_shape* s, const void* x, const int32_t* topk_idx,
+                                const float* topk_gate, const int32_t* expert_rank_host,
+                                const moe_layout* layout, const moe_ep_peer_dest* dests_host,
+                                moe_stream_t stream) {
+  moe_status r = check_shape(s);
+  if (r != MOE_OK) return r;
+  if (s->ep < 2 || !dests_host) return MOE_ERR_INVALID_ARG;
+  EpDests dd{};
+  int64_t cap = 0;
+  for (int q = 0; q < s->ep; ++q) {
+    const moe_ep_peer_dest& d = dests_host[q];
+    if (d.rows < 0 || d.row0 < 0) return MOE_ERR_INVALID_ARG;
+    if (d.rows > 0) {
+      if (!d.recv_x || !d.recv_idx || !d.recv_gate) return MOE_ERR_INVALID_ARG;
+      if (!aligned(d.recv_x, 16) || !aligned(d.recv_idx, 4) || !aligned(d.recv_gate, 4))
+        return MOE_ERR_ALIGNMENT;
+    }
+    dd.d[q].recv_x = d.recv_x;
+    dd.d[q].recv_idx = d.recv_idx;
+    dd.d[q].recv_gate = d.recv_gate;
+    dd.d[q].row0 = d.row0;
+    dd.d[q].rows = d.rows;
+    cap += d.rows;
+  }
+  if (s->T == 0 || cap == 0) return MOE_OK;
+  if (!x || !topk_idx || !layout || !layout->send_token || !layout->rank_offsets)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(topk_idx, 4) || !aligned(layout->send_token, 4) ||
+      !aligned(layout->rank_offsets, 4) || (topk_gate && !aligned(topk_gate, 4)))
+    return MOE_ERR_ALIGNMENT;
+  RankMap map;
+  if ((r = build_map(s, expert_rank_host, &map)) != MOE_OK) return r;
+  EpMaps m{};
+  int next[256] = {0};
+  for (int e = 0; e < s->E; ++e) {
+    m.rank[e] = map.r[e];
+    m.local[e] = (uint8_t)next[map.r[e]]++;
+  }
+  return cuda_status(launch_ep_pack(s->dtype, x, s->T, s->d, s->k, topk_idx, topk_gate,
+                                    layout->send_token, layout->rank_offsets, s->ep, m, s->E,
+                                    nullptr, nullptr, nullptr, cap, &dd, (cudaStream_t)stream));
 }
 
 moe_status moe_ep_expert_workspace_size(const moe_shape* s, size_t* bytes) {
@@ -823,20 +867,22 @@ moe_status moe_ep_expert_workspace_size(const moe_shape* s, size_t* bytes) {
   return MOE_OK;
 }
 
-moe_status moe_ep_expert_forward(const moe_shape* s, const void* recv_x, const int32_t* recv_idx,
-                                 const float* recv_gate, const void* packed_local, void* y_ret,
-                                 void* ws, size_t ws_bytes, moe_stream_t stream) {
+// the receiving rank's experts; the return rows go to y_ret, or with
+// `rets` straight to their source ranks' buffers
+static moe_status ep_expert_impl(const moe_shape* s, const void* recv_x, const int32_t* recv_idx,
+                          const float* recv_gate, const void* packed_local, void* y_ret,
+                          const EpReturns* rets, void* ws, size_t ws_bytes, cudaStream_t st) {
   moe_status r = check_shape(s);
   if (r != MOE_OK) return r;
   if (s->ep < 2 || !ws) return MOE_ERR_INVALID_ARG;
   if (!aligned(ws, kAlign)) return MOE_ERR_ALIGNMENT;
   if (ws_bytes < ep_recv_bytes(s)) return MOE_ERR_WORKSPACE;
   if (s->T == 0) return MOE_OK;
-  if (!recv_x || !recv_idx || !recv_gate || !packed_local || !y_ret) return MOE_ERR_INVALID_ARG;
-  if (!aligned(recv_x, 16) || !aligned(y_ret, 16) || !aligned(recv_idx, 4) ||
+  if (!recv_x || !recv_idx || !recv_gate || !packed_local || (!y_ret && !rets))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(recv_x, 16) || (y_ret && !aligned(y_ret, 16)) || !aligned(recv_idx, 4) ||
       !aligned(recv_gate, 4) || !aligned(packed_local, kAlign))
     return MOE_ERR_ALIGNMENT;
-  cudaStream_t st = (cudaStream_t)stream;
   const int El = s->E / s->ep;
   const EpRecv rv = carve_ep_recv(s, ws);
   // the local experts' packed weights: a packed buffer of E/ep experts
@@ -885,7 +931,68 @@ moe_status moe_ep_expert_forward(const moe_shape* s, const void* recv_x, const i
       return r;
   }
   return cuda_status(launch_ep_partial_combine(s->dtype, rv.y_perm, rv.lo.slot_row, recv_idx,
-                                               recv_gate, El, y_ret, s->T, s->d, s->k, st));
+                                               recv_gate, El, y_ret, s->T, s->d, s->k, rets, st));
+}
+
+moe_status moe_ep_expert_forward(const moe_shape* s, const void* recv_x, const int32_t* recv_idx,
+                                 const float* recv_gate, const void* packed_local, void* y_ret,
+                                 void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (s && s->T > 0 && !y_ret) return MOE_ERR_INVALID_ARG;
+  return ep_expert_impl(s, recv_x, recv_idx, recv_gate, packed_local, y_ret, nullptr, ws,
+                        ws_bytes, (cudaStream_t)stream);
+}
+
+moe_status moe_ep_expert_forward_peer(const moe_shape* s, const void* recv_x,
+                                      const int32_t* recv_idx, const float* recv_gate,
+                                      const void* packed_local, const moe_ep_peer_return* rets_host,
+                                      void* ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status r = check_shape(s);
+  if (r != MOE_OK) return r;
+  if (s->ep < 2 || !rets_host) return MOE_ERR_INVALID_ARG;
+  EpReturns rr{};
+  rr.P = s->ep;
+  int64_t base = 0;
+  for (int q = 0; q < s->ep; ++q) {
+    const moe_ep_peer_return& b = rets_host[q];
+    if (b.rows < 0 || b.row0 < 0) return MOE_ERR_INVALID_ARG;
+    if (b.rows > 0 && !b.y_back) return MOE_ERR_INVALID_ARG;
+    if (b.rows > 0 && !aligned(b.y_back, 16)) return MOE_ERR_ALIGNMENT;
+    rr.d[q].y_back = b.y_back;
+    rr.d[q].row0 = b.row0;
+    rr.base[q] = base;
+    base += b.rows;
+  }
+  rr.base[s->ep] = base;
+  if (base != s->T) return MOE_ERR_INVALID_ARG;  // the blocks tile the received rows
+  return ep_expert_impl(s, recv_x, recv_idx, recv_gate, packed_local, nullptr, &rr, ws, ws_bytes,
+                        (cudaStream_t)stream);
+}
+
+static moe_status ep_signal_impl(uint64_t* const* flags_host, int32_t rank, int32_t P, uint64_t epoch,
+                          void* ws, int64_t wait_ns, cudaStream_t st) {
+  if (P < 1 || P > 256 || rank < 0 || rank >= P || !flags_host || !ws || epoch == 0)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(ws, kAlign)) return MOE_ERR_ALIGNMENT;
+  EpFlags fl{};
+  for (int q = 0; q < P; ++q) {
+    if (!flags_host[q]) return MOE_ERR_INVALID_ARG;
+    if (!aligned(flags_host[q], 8)) return MOE_ERR_ALIGNMENT;
+    fl.flags[q] = flags_host[q];
+  }
+  return cuda_status(
+      launch_ep_signal_wait(fl, rank, P, epoch, wait_ns, static_cast<Control*>(ws), st));
+}
+
+moe_status moe_ep_signal_wait(uint64_t* const* flags_host, int32_t rank, int32_t P,
+                              uint64_t epoch, void* ws, moe_stream_t stream) {
+  return ep_signal_impl(flags_host, rank, P, epoch, ws, kWaitLimitNs, (cudaStream_t)stream);
+}
+
+moe_status moe_debug_ep_signal_wait(uint64_t* const* flags_host, int32_t rank, int32_t P,
+                                    uint64_t epoch, void* ws, int64_t wait_limit_ns,
+                                    moe_stream_t stream) {
+  if (wait_limit_ns <= 0 || wait_limit_ns > kWaitLimitNs) return MOE_ERR_INVALID_ARG;
+  return ep_signal_impl(flags_host, rank, P, epoch, ws, wait_limit_ns, (cudaStream_t)stream);
 }
 
 moe_status moe_ep_home_combine(const moe_shape* s, const void* y_back, const int32_t* slot_send_row,

@@ -27,13 +27,18 @@ namespace {
 constexpr int kPackWarps = 8;
 
 // one warp per send row s: destination r from rank_offsets (binary search in
-// shared memory), token t = send_token[s]
+// shared memory), token t = send_token[s].  Row s lands at row s of the send
+// buffers, or, with `dests`, at row dests.d[r].row0 + s - rank_offsets[r] of
+// rank r's receive buffers (the pack and the all-to-all in one pass: plain
+// stores, to another GPU's memory through its peer mapping); rows past
+// dests.d[r].rows are not stored.
 __global__ void __launch_bounds__(32 * kPackWarps)
     ep_pack_kernel(const uint4* __restrict__ x, int64_t T, int V, int k,
                    const int32_t* __restrict__ idx, const float* __restrict__ gate,
                    const int32_t* __restrict__ send_token, const int32_t* __restrict__ rank_offsets,
                    int P, EpMaps maps, int E, int E_loc, uint4* __restrict__ send_x,
-                   int32_t* __restrict__ send_idx, float* __restrict__ send_gate, int64_t cap) {
+                   int32_t* __restrict__ send_idx, float* __restrict__ send_gate, int64_t cap,
+                   const __grid_constant__ EpDests dests, int use_dests) {
   __shared__ int s_off[257];
   pdl_wait();
   for (int i = threadIdx.x; i <= P; i += blockDim.x) s_off[i] = __ldg(rank_offsets + i);
@@ -52,13 +57,24 @@ __global__ void __launch_bounds__(32 * kPackWarps)
     int64_t t = __ldg(send_token + s);
     if (t < 0 || t >= T) t = 0;
     const uint4* src = x + t * V;
-    uint4* dst = send_x + s * V;
+    uint4* dx = send_x;
+    int32_t* di = send_idx;
+    float* dg = send_gate;
+    int64_t row = s;
+    if (use_dests) {
+      if (s - s_off[r] >= dests.d[r].rows) continue;  // warp-uniform
+      dx = static_cast<uint4*>(dests.d[r].recv_x);
+      di = dests.d[r].recv_idx;
+      dg = dests.d[r].recv_gate;
+      row = dests.d[r].row0 + (s - s_off[r]);
+    }
+    uint4* dst = dx + row * V;
     for (int v = lane; v < V; v += 32) dst[v] = __ldg(src + v);
     if (lane < k) {
       const int e = __ldg(idx + t * k + lane);
       const bool here = e >= 0 && e < E && maps.rank[e] == r;
-      send_idx[s * k + lane] = here ? (int)maps.local[e] : E_loc;
-      send_gate[s * k + lane] = gate ? __ldg(gate + t * k + lane) : 1.f;
+      di[row * k + lane] = here ? (int)maps.local[e] : E_loc;
+      dg[row * k + lane] = gate ? __ldg(gate + t * k + lane) : 1.f;
     }
   }
 }
@@ -99,17 +115,31 @@ struct Acc<float> {
 // y_ret[i] = sum over slots j (ascending) of received row i whose expert is
 // held here (local id < E_loc) of gate[i,j] * y_perm[slot_row[i*k + j]], in
 // fp32, rounded once.  One thread per 16-byte vector of an output row.
+// With `rets`, received row t (from source rank s: rets.base[s] <= t <
+// rets.base[s+1]) is stored at row rets.d[s].row0 + t - rets.base[s] of that
+// source's return buffer instead of row t of y_ret.
 template <typename T>
 __global__ void __launch_bounds__(256)
     ep_partial_combine_kernel(const uint4* __restrict__ y_perm, const int32_t* __restrict__ slot_row,
                               const int32_t* __restrict__ recv_idx, const float* __restrict__ recv_gate,
-                              int E_loc, uint4* __restrict__ y_ret, int64_t Tr, int V, int k) {
+                              int E_loc, uint4* __restrict__ y_ret, int64_t Tr, int V, int k,
+                              const __grid_constant__ EpReturns rets, int use_rets) {
   pdl_wait();
   const int64_t n = Tr * V;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
        i += (int64_t)gridDim.x * blockDim.x) {
     const int64_t t = i / V;
     const int v = (int)(i - t * V);
+    uint4* out = y_ret + i;
+    if (use_rets) {
+      // the source rank of received row t: last s with base[s] <= t
+      int lo = 0, hi = rets.P - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (rets.base[mid] <= t) lo = mid; else hi = mid - 1;
+      }
+      out = static_cast<uint4*>(rets.d[lo].y_back) + (rets.d[lo].row0 + (t - rets.base[lo])) * V + v;
+    }
     float a[Acc<T>::N];
 #pragma unroll
     for (int q = 0; q < Acc<T>::N; ++q) a[q] = 0.f;
@@ -120,7 +150,7 @@ __global__ void __launch_bounds__(256)
       if (row < 0 || row >= Tr * k) row = 0;
       Acc<T>::add(a, __ldg(y_perm + row * V + v), __ldg(recv_gate + t * k + j));
     }
-    y_ret[i] = Acc<T>::pack(a);
+    *out = Acc<T>::pack(a);
   }
 }
 
@@ -161,34 +191,73 @@ int grid_for(int64_t items, int per_block) {
   return (int)std::min<int64_t>((items + per_block - 1) / per_block, (int64_t)sms * 8);
 }
 
+// The ranks' rendezvous around a peer-memory exchange: rank `me` stores
+// `epoch` into slot `me` of every rank's flag array (a release at system
+// scope, after everything earlier in this stream, so the rows this rank
+// stored into peers' buffers are visible before the flag is), then waits
+// until every slot of its own array holds at least `epoch` (an acquire at
+// system scope), giving up after wait_ns and recording
+// MOE_ERR_DEVICE_TIMEOUT with detail = the first missing rank.
+__global__ void ep_signal_wait_kernel(const __grid_constant__ EpFlags fl, int me, int P,
+                                      uint64_t epoch, int64_t wait_ns, Control* ctl) {
+  pdl_wait();
+  const int r = threadIdx.x;
+  if (r < P) {
+    uint64_t* slot = fl.flags[r] + me;
+    asm volatile("fence.acq_rel.sys;" ::: "memory");
+    asm volatile("st.release.sys.global.u64 [%0], %1;" ::"l"(slot), "l"(epoch) : "memory");
+  }
+  __syncthreads();
+  if (r < P) {
+    const uint64_t* mine = fl.flags[me] + r;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+      uint64_t v;
+      asm volatile("ld.acquire.sys.global.u64 %0, [%1];" : "=l"(v) : "l"(mine) : "memory");
+      if (v >= epoch) break;
+      if (globaltimer_ns() - t0 > (uint64_t)wait_ns) {
+        record_error(ctl, MOE_ERR_DEVICE_TIMEOUT, (uint32_t)r);
+        break;
+      }
+    }
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_ep_pack(int dtype, const void* x, int64_t T, int d, int k, const int32_t* idx,
                            const float* gate, const int32_t* send_token,
                            const int32_t* rank_offsets, int P, const EpMaps& maps, int E,
                            void* send_x, int32_t* send_idx, float* send_gate, int64_t cap,
-                           cudaStream_t s) {
+                           const EpDests* dests, cudaStream_t s) {
   if (T == 0 || cap == 0) return cudaSuccess;
   const int V = d * (dtype == MOE_BF16 ? 2 : 4) / 16;
   const int grid = std::max(1, grid_for(cap, kPackWarps));
+  EpDests dd{};
+  if (dests) dd = *dests;
   return launch_pdl(ep_pack_kernel, dim3(grid), dim3(32 * kPackWarps), 0, s,
                     static_cast<const uint4*>(x), T, V, k, idx, gate, send_token, rank_offsets, P,
-                    maps, E, E / P, static_cast<uint4*>(send_x), send_idx, send_gate, cap);
+                    maps, E, E / P, static_cast<uint4*>(send_x), send_idx, send_gate, cap, dd,
+                    dests ? 1 : 0);
 }
 
 cudaError_t launch_ep_partial_combine(int dtype, const void* y_perm, const int32_t* slot_row,
                                       const int32_t* recv_idx, const float* recv_gate, int E_loc,
-                                      void* y_ret, int64_t Tr, int d, int k, cudaStream_t s) {
+                                      void* y_ret, int64_t Tr, int d, int k, const EpReturns* rets,
+                                      cudaStream_t s) {
   if (Tr == 0) return cudaSuccess;
   const int V = d * (dtype == MOE_BF16 ? 2 : 4) / 16;
   const int grid = grid_for(Tr * V, 256);
+  EpReturns rr{};
+  if (rets) rr = *rets;
+  const int use = rets ? 1 : 0;
   if (dtype == MOE_BF16)
     return launch_pdl(ep_partial_combine_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s,
                       static_cast<const uint4*>(y_perm), slot_row, recv_idx, recv_gate, E_loc,
-                      static_cast<uint4*>(y_ret), Tr, V, k);
+                      static_cast<uint4*>(y_ret), Tr, V, k, rr, use);
   return launch_pdl(ep_partial_combine_kernel<float>, dim3(grid), dim3(256), 0, s,
                     static_cast<const uint4*>(y_perm), slot_row, recv_idx, recv_gate, E_loc,
-                    static_cast<uint4*>(y_ret), Tr, V, k);
+                    static_cast<uint4*>(y_ret), Tr, V, k, rr, use);
 }
 
 cudaError_t launch_ep_home_combine(int dtype, const void* y_back, const int32_t* slot_send_row,
@@ -203,6 +272,12 @@ cudaError_t launch_ep_home_combine(int dtype, const void* y_back, const int32_t*
   return launch_pdl(ep_home_combine_kernel<float>, dim3(grid), dim3(256), 0, s,
                     static_cast<const uint4*>(y_back), slot_send_row, static_cast<uint4*>(y), T, V, k,
                     rows);
+}
+
+cudaError_t launch_ep_signal_wait(const EpFlags& fl, int me, int P, uint64_t epoch,
+                                  int64_t wait_ns, Control* ctl, cudaStream_t s) {
+  return launch_pdl(ep_signal_wait_kernel, dim3(1), dim3(256), 0, s, fl, me, P, epoch, wait_ns,
+                    ctl);
 }
 
 }  // namespace moe

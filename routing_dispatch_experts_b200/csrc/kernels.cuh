@@ -231,14 +231,46 @@ struct EpMaps {
   uint8_t rank[256];
   uint8_t local[256];
 };
+// where each destination rank's rows go when the pack stores them straight
+// into the ranks' receive buffers (a kernel parameter: up to 256 ranks)
+struct EpDest {
+  void* recv_x;
+  int32_t* recv_idx;
+  float* recv_gate;
+  int64_t row0;  // first row of this source's block there
+  int64_t rows;  // rows of the block (send rows past it are not stored)
+};
+struct EpDests {
+  EpDest d[256];
+};
+// where the return rows of each source rank go, and the received-row range
+// of each source (base[s] .. base[s+1])
+struct EpReturn {
+  void* y_back;
+  int64_t row0;
+};
+struct EpReturns {
+  EpReturn d[256];
+  int64_t base[257];
+  int P;
+};
+// dests NULL: rows into send_x / send_idx / send_gate
 cudaError_t launch_ep_pack(int dtype, const void* x, int64_t T, int d, int k, const int32_t* idx,
                            const float* gate, const int32_t* send_token,
                            const int32_t* rank_offsets, int P, const EpMaps& maps, int E,
                            void* send_x, int32_t* send_idx, float* send_gate, int64_t cap,
-                           cudaStream_t s);
+                           const EpDests* dests, cudaStream_t s);
+// every rank's flag array (P uint64 slots each), as this process maps them
+struct EpFlags {
+  uint64_t* flags[256];
+};
+cudaError_t launch_ep_signal_wait(const EpFlags& fl, int me, int P, uint64_t epoch,
+                                  int64_t wait_ns, Control* ctl, cudaStream_t s);
+// rets NULL: rows into y_ret
 cudaError_t launch_ep_partial_combine(int dtype, const void* y_perm, const int32_t* slot_row,
                                       const int32_t* recv_idx, const float* recv_gate, int E_loc,
-                                      void* y_ret, int64_t Tr, int d, int k, cudaStream_t s);
+                                      void* y_ret, int64_t Tr, int d, int k, const EpReturns* rets,
+                                      cudaStream_t s);
 cudaError_t launch_ep_home_combine(int dtype, const void* y_back, const int32_t* slot_send_row,
                                    void* y, int64_t T, int d, int k, int64_t rows, cudaStream_t s);
 

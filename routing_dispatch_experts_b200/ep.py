@@ -23,6 +23,13 @@ sequences them and moves rows through an Exchange:
                  CPU tensors), one process per rank;
   LocalExchange  P ranks emulated in one process (their buffers on one
                  device), for single-GPU tests of the whole path.
+
+or, with peer memory, without a separate exchange: moe_ep_dispatch_peer
+stores each send row straight into its destination's receive buffer and
+moe_ep_expert_forward_peer each return row straight into its source's
+buffer (peer_blocks gives where; PeerEPRank runs it over a symmetric-memory
+allocation with moe_ep_signal_wait between the phases; forward_peer_emulated
+runs the same kernels with the ranks' buffers on one device).
 """
 from __future__ import annotations
 
@@ -31,8 +38,9 @@ from typing import List, Optional, Sequence
 
 import torch
 
-from . import Shape, dispatch_layout, ep_expert_forward, ep_expert_workspace, ep_home_combine, \
-    ep_pack, route, workspace
+from . import Shape, check_device_status, dispatch_layout, ep_dispatch_peer, ep_expert_forward, \
+    ep_expert_forward_peer, ep_expert_workspace, ep_home_combine, ep_pack, ep_signal_wait, route, \
+    workspace
 
 # ------------------------------------------------------------------ exchange
 
@@ -43,6 +51,22 @@ def splits(counts: Sequence[Sequence[int]], rank: int):
     send rows to dst, and receives from every src in rank order."""
     P = len(counts)
     return [int(counts[rank][d]) for d in range(P)], [int(counts[s][rank]) for s in range(P)]
+
+
+def peer_blocks(counts: Sequence[Sequence[int]], rank: int):
+    """Where `rank`'s rows go in a peer-memory exchange, from the count
+    matrix counts[src][dst]:
+      dests[r] = (row0, rows) of its block in rank r's receive rows: after
+                 the blocks of the ranks below it (row0 = sum_{s < rank}
+                 counts[s][r]), rows = counts[rank][r];
+      rets[s]  = (row0, rows) of the block it received from rank s, in s's
+                 send-row order (row0 = sum_{r < rank} counts[s][r], s's
+                 rank_offsets[rank]), rows = counts[s][rank].
+    The same positions as the all-to-all of TorchExchange.rows."""
+    P = len(counts)
+    dests = [(sum(int(counts[q][r]) for q in range(rank)), int(counts[rank][r])) for r in range(P)]
+    rets = [(sum(int(counts[q][r]) for r in range(rank)), int(counts[q][rank])) for q in range(P)]
+    return dests, rets
 
 
 class TorchExchange:
@@ -184,6 +208,115 @@ def forward_emulated(ranks: Sequence[EPRank], xs: Sequence[torch.Tensor]):
     rets = [r.experts(recv_x[i], recv_idx[i], recv_gate[i]) for i, r in enumerate(ranks)]
     backs = ex.rows_back(rets, counts)
     return [r.finish(p, b) for r, p, b in zip(ranks, plans, backs)], counts
+
+
+def forward_peer_emulated(ranks: Sequence[EPRank], xs: Sequence[torch.Tensor]):
+    """forward_emulated through the peer-memory kernels: every rank's send
+    rows stored straight into the receiving ranks' buffers, every return row
+    straight into its source's buffer (the ranks' buffers on one device, the
+    phases in order on one stream, so no rendezvous is needed).  Returns
+    (per-rank outputs, count matrix)."""
+    P = len(ranks)
+    sh = ranks[0].shape
+    dev = xs[0].device
+    plans = [r.plan(x) for r, x in zip(ranks, xs)]
+    counts = LocalExchange(P).counts([p.layout["rank_counts"] for p in plans])
+    n_recv = [sum(counts[q][r] for q in range(P)) for r in range(P)]
+    n_send = [sum(counts[q]) for q in range(P)]
+    recv = [(torch.empty((n, sh.d), dtype=sh.dtype, device=dev),
+             torch.empty((n, sh.k), dtype=torch.int32, device=dev),
+             torch.empty((n, sh.k), dtype=torch.float32, device=dev)) for n in n_recv]
+    backs = [torch.empty((n, sh.d), dtype=sh.dtype, device=dev) for n in n_send]
+    for q, (rk, x, p) in enumerate(zip(ranks, xs, plans)):
+        p.counts = counts
+        dests, _ = peer_blocks(counts, q)
+        ep_dispatch_peer(rk.shape, x, p.idx, p.gate, p.layout,
+                         [recv[r] + dests[r] for r in range(P)], expert_rank=rk.expert_rank)
+    for r, rk in enumerate(ranks):
+        _, rets = peer_blocks(counts, r)
+        rs = dataclasses.replace(rk.shape, T=n_recv[r])
+        ws = ep_expert_workspace(rs, device=dev)
+        ep_expert_forward_peer(rs, *recv[r], rk.packed_local,
+                               [(backs[q],) + rets[q] for q in range(P)], ws)
+    return [rk.finish(p, b) for rk, p, b in zip(ranks, plans, backs)], counts
+
+
+class PeerEPRank(EPRank):
+    """One rank of the expert-parallel layer over peer memory (one process
+    per GPU, the ranks' GPUs peer-connected): the receive rows, the return
+    rows and the rendezvous flags of every rank live in one symmetric-memory
+    allocation per rank (torch.distributed._symmetric_memory), sized for at
+    most `max_tokens` tokens per rank; every forward takes two rendezvous
+    epochs (after the dispatch stores, after the return stores), which also
+    keep the next forward's stores out of buffers still being read."""
+
+    def __init__(self, shape: Shape, rank: int, expert_rank, packed_router, packed_local,
+                 group=None, max_tokens=None, bias=None):
+        super().__init__(shape, rank, expert_rank, packed_router, packed_local, bias)
+        import torch.distributed as dist
+        import torch.distributed._symmetric_memory as symm
+        self.ex = TorchExchange(group)
+        P, d, k = shape.ep, shape.d, shape.k
+        Tm = shape.T if max_tokens is None else int(max_tokens)
+        self.cap_recv = P * Tm            # rows from every source, at most one per token
+        self.cap_send = Tm * min(k, P)    # send rows of this rank's tokens
+        es = torch.tensor([], dtype=shape.dtype).element_size()
+        parts = [("flags", 8 * P), ("recv_x", es * d * self.cap_recv),
+                 ("recv_idx", 4 * k * self.cap_recv), ("recv_gate", 4 * k * self.cap_recv),
+                 ("y_back", es * d * self.cap_send)]
+        self.off, n = {}, 0
+        for name, b in parts:
+            self.off[name] = n
+            n += (b + 255) // 256 * 256
+        self.buf = symm.empty(n, dtype=torch.uint8, device=packed_router.device)
+        self.buf.zero_()
+        self.hdl = symm.rendezvous(self.buf, group if group is not None else dist.group.WORLD)
+        self.views = [self._views(self.hdl.get_buffer(q, (n,), torch.uint8)) for q in range(P)]
+        self.epoch = 0
+
+    def _views(self, b):
+        sh, o = self.shape, self.off
+        cr, cs = self.cap_recv, self.cap_send
+
+        def at(name, dt, shape):
+            nb = torch.tensor([], dtype=dt).element_size()
+            for s_ in shape:
+                nb *= s_
+            return b[o[name]:o[name] + nb].view(dt).view(shape)
+        return {"flags": at("flags", torch.int64, (sh.ep,)),
+                "recv_x": at("recv_x", sh.dtype, (cr, sh.d)),
+                "recv_idx": at("recv_idx", torch.int32, (cr, sh.k)),
+                "recv_gate": at("recv_gate", torch.float32, (cr, sh.k)),
+                "y_back": at("y_back", sh.dtype, (cs, sh.d))}
+
+    def _rendezvous(self):
+        self.epoch += 1
+        ep_signal_wait([v["flags"] for v in self.views], self.rank, self.epoch, self.ws)
+
+    def forward(self, x, ex=None):
+        """The whole forward of this rank (every rank calls it with its own
+        tokens); raises if a rendezvous timed out."""
+        P = self.shape.ep
+        plan = self.plan(x)
+        counts = self.ex.counts(plan.layout["rank_counts"])
+        plan.counts = counts
+        dests, rets = peer_blocks(counts, self.rank)
+        V = self.views
+        ep_dispatch_peer(self.shape, x, plan.idx, plan.gate, plan.layout,
+                         [(V[r]["recv_x"], V[r]["recv_idx"], V[r]["recv_gate"]) + dests[r]
+                          for r in range(P)], expert_rank=self.expert_rank)
+        self._rendezvous()
+        n_recv = sum(rows for _, rows in rets)
+        me = V[self.rank]
+        rs = dataclasses.replace(self.shape, T=n_recv)
+        ws = ep_expert_workspace(rs, device=x.device)
+        ep_expert_forward_peer(rs, me["recv_x"][:n_recv], me["recv_idx"][:n_recv],
+                               me["recv_gate"][:n_recv], self.packed_local,
+                               [(V[q]["y_back"],) + rets[q] for q in range(P)], ws)
+        self._rendezvous()
+        check_device_status(self.ws)
+        n_send = sum(counts[self.rank])
+        return self.finish(plan, me["y_back"][:n_send]), counts
 
 
 def local_experts(expert_rank: Sequence[int], rank: int) -> List[int]:

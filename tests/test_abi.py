@@ -172,8 +172,8 @@ def _c_kind(param: str) -> str:
     p = " ".join(param.split())
     if "*" in p or p.startswith(("moe_stream_t", "moe_event_t")):
         return "ptr"
-    if p.startswith(("size_t", "const size_t")):
-        return "size"
+    if p.startswith(("size_t", "const size_t", "uint64_t")):
+        return "size"  # unsigned 64-bit: ctypes' c_size_t is c_uint64
     if p.startswith(("double", "const double")):
         return "f64"
     if "int64_t" in p:
@@ -223,6 +223,8 @@ def test_struct_layouts_match_the_header(tmp_path):
         "moe_layout": [f for f, _ in moe.moe_layout._fields_],
         "moe_forward_buffers": [f for f, _ in moe.moe_forward_buffers._fields_],
         "moe_router_counts": [f for f, _ in moe.moe_router_counts._fields_],
+        "moe_ep_peer_dest": [f for f, _ in moe.moe_ep_peer_dest._fields_],
+        "moe_ep_peer_return": [f for f, _ in moe.moe_ep_peer_return._fields_],
         "moe_stats": ["rows_sent", "dup_removed", "tokens_single_rank", "home_rank_rows",
                       "max_expert_rows", "min_expert_rows"],
     }
@@ -242,7 +244,9 @@ def test_struct_layouts_match_the_header(tmp_path):
         got[(s, f)] = int(v)
     for s, cls in (("moe_shape", moe.moe_shape), ("moe_layout", moe.moe_layout),
                    ("moe_forward_buffers", moe.moe_forward_buffers),
-                   ("moe_router_counts", moe.moe_router_counts)):
+                   ("moe_router_counts", moe.moe_router_counts),
+                   ("moe_ep_peer_dest", moe.moe_ep_peer_dest),
+                   ("moe_ep_peer_return", moe.moe_ep_peer_return)):
         assert got[(s, "size")] == ctypes.sizeof(cls), s
         for f in structs[s]:
             assert got[(s, f)] == getattr(cls, f).offset, (s, f)
@@ -250,3 +254,51 @@ def test_struct_layouts_match_the_header(tmp_path):
     # and min (high half) of word 4
     assert [got[("moe_stats", f)] for f in structs["moe_stats"]] == [0, 8, 16, 24, 32, 36]
     assert got[("moe_stats", "size")] <= 6 * 8
+
+
+def test_peer_entry_points_reject_bad_arguments(L):
+    """Argument checks of the peer-memory exchange, all before any launch."""
+    s = moe.Shape(T=64, d=128, E=8, k=2, f=128, ep=2).c
+    lay = moe.moe_layout()
+    dests = (moe.moe_ep_peer_dest * 2)()
+    dests[0] = moe.moe_ep_peer_dest(None, None, None, 0, -1)
+    assert L.moe_ep_dispatch_peer(ctypes.byref(s), None, None, None, None, ctypes.byref(lay),
+                                  dests, None) == moe.MOE_ERR_INVALID_ARG
+    dests[0] = moe.moe_ep_peer_dest(None, None, None, 0, 3)  # rows but no buffers
+    assert L.moe_ep_dispatch_peer(ctypes.byref(s), None, None, None, None, ctypes.byref(lay),
+                                  dests, None) == moe.MOE_ERR_INVALID_ARG
+    dests[0] = moe.moe_ep_peer_dest(8, 16, 16, 0, 3)  # recv_x not 16-byte aligned
+    assert L.moe_ep_dispatch_peer(ctypes.byref(s), None, None, None, None, ctypes.byref(lay),
+                                  dests, None) == moe.MOE_ERR_ALIGNMENT
+    assert L.moe_ep_dispatch_peer(ctypes.byref(s), None, None, None, None, ctypes.byref(lay),
+                                  None, None) == moe.MOE_ERR_INVALID_ARG
+    one = moe.Shape(T=64, d=128, E=8, k=2, f=128, ep=1).c
+    dests[0] = moe.moe_ep_peer_dest(None, None, None, 0, 0)
+    assert L.moe_ep_dispatch_peer(ctypes.byref(one), None, None, None, None, ctypes.byref(lay),
+                                  dests, None) == moe.MOE_ERR_INVALID_ARG
+    # returns: blocks must tile the received rows
+    rets = (moe.moe_ep_peer_return * 2)()
+    rets[0] = moe.moe_ep_peer_return(256, 0, 30)
+    rets[1] = moe.moe_ep_peer_return(256, 0, 30)
+    assert L.moe_ep_expert_forward_peer(ctypes.byref(s), 256, 256, 256, 256, rets, 256, 1 << 30,
+                                        None) == moe.MOE_ERR_INVALID_ARG
+    rets[1] = moe.moe_ep_peer_return(8, 0, 34)
+    assert L.moe_ep_expert_forward_peer(ctypes.byref(s), 256, 256, 256, 256, rets, 256, 1 << 30,
+                                        None) == moe.MOE_ERR_ALIGNMENT
+    rets[1] = moe.moe_ep_peer_return(256, -1, 34)
+    assert L.moe_ep_expert_forward_peer(ctypes.byref(s), 256, 256, 256, 256, rets, 256, 1 << 30,
+                                        None) == moe.MOE_ERR_INVALID_ARG
+    # rendezvous
+    flags = (ctypes.c_void_p * 2)(256, 256)
+    assert L.moe_ep_signal_wait(flags, 0, 2, 0, 256, None) == moe.MOE_ERR_INVALID_ARG  # epoch 0
+    assert L.moe_ep_signal_wait(flags, 2, 2, 1, 256, None) == moe.MOE_ERR_INVALID_ARG  # rank
+    assert L.moe_ep_signal_wait(flags, 0, 0, 1, 256, None) == moe.MOE_ERR_INVALID_ARG  # P
+    assert L.moe_ep_signal_wait(flags, 0, 2, 1, None, None) == moe.MOE_ERR_INVALID_ARG  # ws
+    assert L.moe_ep_signal_wait(flags, 0, 2, 1, 260, None) == moe.MOE_ERR_ALIGNMENT
+    bad = (ctypes.c_void_p * 2)(256, 260)
+    assert L.moe_ep_signal_wait(bad, 0, 2, 1, 256, None) == moe.MOE_ERR_ALIGNMENT
+    nul = (ctypes.c_void_p * 2)(256, None)
+    assert L.moe_ep_signal_wait(nul, 0, 2, 1, 256, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_debug_ep_signal_wait(flags, 0, 2, 1, 256, 0, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_debug_ep_signal_wait(flags, 0, 2, 1, 256, 2_000_000_000,
+                                      None) == moe.MOE_ERR_INVALID_ARG

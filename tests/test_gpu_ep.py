@@ -111,3 +111,86 @@ def test_ep_dedup_and_correlated_placement_cut_rows():
     own = np.array(fit)[idx]
     dp_rows = sum(len(set(own[t]) - {home[t]}) for t in range(T))
     assert dp_rows < d_rows
+
+
+@pytest.mark.parametrize("cfg,T,P,placement", [
+    (3, 4096, 8, "contiguous"), (2, 4096, 8, "permutation"), (1, 1024, 4, "contiguous"),
+    (5, 1024, 16, "contiguous"),
+])
+def test_peer_exchange_equals_the_collective_exchange(cfg, T, P, placement):
+    """moe_ep_dispatch_peer + moe_ep_expert_forward_peer store the same rows
+    at the same positions as pack + all-to-all and experts + reverse
+    all-to-all: every rank's output bit-identical."""
+    *_, ranks, xs, shape = _setup(cfg, T, P, placement)
+    ys, counts = EP.forward_emulated(ranks, xs)
+    yp, counts_p = EP.forward_peer_emulated(ranks, xs)
+    torch.cuda.synchronize()
+    assert counts_p == counts
+    for r in range(P):
+        assert torch.equal(yp[r], ys[r]), r
+
+
+def test_peer_dispatch_stores_no_row_past_its_block():
+    """A destination block smaller than the rows the plan sends there: the
+    rows past it are not stored (the rows around the block keep their
+    sentinel), the rows inside it equal the pack's."""
+    cfg, T, P = 3, 2048, 4
+    *_, ranks, xs, shape = _setup(cfg, T, P, "contiguous")
+    rk, x = ranks[1], xs[1]
+    plan = rk.plan(x)
+    n = [int(v) for v in plan.layout["rank_counts"].tolist()]
+    send_x, send_idx, send_gate = moe.ep_pack(shape, x, plan.idx, plan.gate, plan.layout, sum(n),
+                                              expert_rank=rk.expert_rank)
+    off = np.concatenate([[0], np.cumsum(n)])
+    pad = 7
+    bufs = []
+    dests = []
+    for r in range(P):
+        rows = max(n[r] - 5, 0) if r == 2 else n[r]
+        bx = torch.full((pad + n[r] + pad, shape.d), 3.0, dtype=shape.dtype, device="cuda")
+        bi = torch.full((pad + n[r] + pad, shape.k), -9, dtype=torch.int32, device="cuda")
+        bg = torch.full((pad + n[r] + pad, shape.k), -2.0, dtype=torch.float32, device="cuda")
+        bufs.append((bx, bi, bg, rows))
+        dests.append((bx, bi, bg, pad, rows))
+    moe.ep_dispatch_peer(shape, x, plan.idx, plan.gate, plan.layout, dests,
+                         expert_rank=rk.expert_rank)
+    torch.cuda.synchronize()
+    for r, (bx, bi, bg, rows) in enumerate(bufs):
+        lo, hi = int(off[r]), int(off[r]) + rows
+        assert torch.equal(bx[pad:pad + rows], send_x[lo:hi])
+        assert torch.equal(bi[pad:pad + rows], send_idx[lo:hi])
+        assert torch.equal(bg[pad:pad + rows], send_gate[lo:hi])
+        assert (bx[:pad] == 3.0).all() and (bx[pad + rows:] == 3.0).all()
+        assert (bi[:pad] == -9).all() and (bi[pad + rows:] == -9).all()
+        assert (bg[:pad] == -2.0).all() and (bg[pad + rows:] == -2.0).all()
+
+
+def test_signal_wait_passes_when_every_slot_is_set():
+    """One kernel: rank 0 of 3 stores its epoch into slot 0 of each array
+    and finds slots 1 and 2 of its own array already at the epoch (set
+    beforehand, as ranks 1 and 2 would)."""
+    P = 3
+    flags = [torch.zeros(P, dtype=torch.int64, device="cuda") for _ in range(P)]
+    ws = moe.workspace(moe.Shape(T=1, d=64, E=4, k=1, f=64))
+    flags[0][1:] = 5
+    moe.ep_signal_wait(flags, 0, 5, ws)
+    assert moe.get_device_status(ws) == moe.MOE_OK
+    assert [int(f[0]) for f in flags] == [5, 5, 5]
+    # a single rank meets only itself
+    one = [torch.zeros(1, dtype=torch.int64, device="cuda")]
+    moe.ep_signal_wait(one, 0, 1, ws)
+    assert moe.get_device_status(ws) == moe.MOE_OK and int(one[0][0]) == 1
+
+
+def test_signal_wait_gives_up_on_a_flag_nothing_sets():
+    """Rank 0 of 2 with rank 1's slot never set: the bounded wait ends after
+    its limit with MOE_ERR_DEVICE_TIMEOUT (detail: rank 1), and the context
+    stays usable (a following rendezvous that finds its slots passes)."""
+    P = 2
+    flags = [torch.zeros(P, dtype=torch.int64, device="cuda") for _ in range(P)]
+    ws = moe.workspace(moe.Shape(T=1, d=64, E=4, k=1, f=64))
+    moe.ep_signal_wait(flags, 0, 1, ws, wait_limit_ns=2_000_000)
+    assert moe.get_device_status(ws) == moe.MOE_ERR_DEVICE_TIMEOUT
+    flags[0][1] = 2
+    moe.ep_signal_wait(flags, 0, 2, ws)
+    assert moe.get_device_status(ws) == moe.MOE_OK
