@@ -44,7 +44,9 @@ __global__ void __launch_bounds__(32 * kPackWarps)
   for (int i = threadIdx.x; i <= P; i += blockDim.x) s_off[i] = __ldg(rank_offsets + i);
   __syncthreads();
   const int lane = threadIdx.x & 31;
-  const int64_t rows = min((int64_t)s_off[P], cap);
+  // into send buffers: the first `cap` send rows; into receive buffers: every
+  // send row (the per-destination block bounds apply)
+  const int64_t rows = use_dests ? (int64_t)s_off[P] : min((int64_t)s_off[P], cap);
   for (int64_t s = (int64_t)blockIdx.x * kPackWarps + (threadIdx.x >> 5); s < rows;
        s += (int64_t)gridDim.x * kPackWarps) {
     // last r with s_off[r] <= s

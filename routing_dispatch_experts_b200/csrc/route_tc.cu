@@ -447,26 +447,54 @@ __global__ void __launch_bounds__(route_threads<MT>(), (MT == 1 ? 2 : 1))
         p.block_hist[(size_t)bin * p.hist_stride + b0 + mm] = (uint16_t)hist[mm][bin];
 }
 
+// shared-memory bytes the epilogue of MT tiles needs after the GEMM: the
+// staged logits tiles and the partial top-k lists of the other parts
 template <int KMAX, int MT>
-cudaError_t run(const RouteArgs& a, const CUtensorMap& mA, const CUtensorMap& mB,
-                const CUtensorMap& mL, Params p, cudaStream_t s) {
+size_t epilogue_bytes(const Params& p, uint32_t* staged_bytes) {
+  const size_t staged = p.logits_mode == 2 ? (size_t)p.E * 512
+                        : p.logits_mode == 1 ? (size_t)BM * (p.E * 4 + 16) : 0;
+  const size_t sb = (staged + 1023) & ~size_t(1023);
+  if (staged_bytes) *staged_bytes = (uint32_t)sb;
+  return (size_t)MT * sb + (size_t)MT * (kParts - 1) * BM * KMAX * 8;
+}
+
+// The ring's stages for MT tiles per CTA and the dynamic shared memory they
+// take; false when they do not fit next to the kernel's static arrays.
+template <int KMAX, int MT>
+bool plan_ring(Params& p, size_t* smem) {
   // the ring also holds, after the GEMM, the staged logits tiles and the
   // partial top-k lists of the other parts: grow it when they need more room
   const size_t stage = (size_t)MT * BM * BK * 2 + (size_t)p.BN * BK * 2;
-  const size_t staged = p.logits_mode == 2 ? (size_t)p.E * 512
-                        : p.logits_mode == 1 ? (size_t)BM * (p.E * 4 + 16) : 0;
-  p.staged_bytes = (uint32_t)((staged + 1023) & ~size_t(1023));
+  const size_t need = epilogue_bytes<KMAX, MT>(p, &p.staged_bytes);
   p.merge_off = (uint32_t)MT * p.staged_bytes;
-  const size_t need = p.merge_off + (size_t)MT * (kParts - 1) * BM * KMAX * 8;
   const size_t budget = MT == 1 && p.nb > p.sms ? kRingBudget / 2 : kRingBudget;
   int st = (int)(budget / stage);
   st = st > kMaxStages ? kMaxStages : st;
   st = st > p.K / BK ? p.K / BK : st;
   p.stages = st < 1 ? 1 : st;
   while ((size_t)p.stages * stage < need) ++p.stages;
-  if (p.stages > kMaxStages) return cudaErrorInvalidValue;
+  if (p.stages > kMaxStages) return false;
+  *smem = (size_t)p.stages * stage + 1024;
+  static size_t static_bytes = 0, optin = 0;
+  if (optin == 0) {
+    cudaFuncAttributes fa;
+    int dev = 0, v = 0;
+    cudaGetDevice(&dev);
+    if (cudaFuncGetAttributes(&fa, (const void*)route_fused_kernel<KMAX, MT>) != cudaSuccess ||
+        cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+      return false;
+    static_bytes = fa.sharedSizeBytes;
+    optin = (size_t)v;
+  }
+  return *smem + static_bytes <= optin;
+}
+
+template <int KMAX, int MT>
+cudaError_t run(const RouteArgs& a, const CUtensorMap& mA, const CUtensorMap& mB,
+                const CUtensorMap& mL, Params p, cudaStream_t s) {
+  size_t smem = 0;
+  if (!plan_ring<KMAX, MT>(p, &smem)) return cudaErrorInvalidValue;
   // dynamic shared memory grows with E; raise the kernel's limit when needed
-  const size_t smem = (size_t)p.stages * stage + 1024;
   cudaError_t e = set_smem_limit((const void*)route_fused_kernel<KMAX, MT>, smem);
   if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)((p.nb + MT - 1) / MT);
@@ -478,8 +506,13 @@ template <int KMAX>
 cudaError_t run_mt(const RouteArgs& a, const CUtensorMap& mA, const CUtensorMap& mB,
                    const CUtensorMap& mL, Params p, cudaStream_t s) {
   // two tiles per CTA when there are more tiles than SMs and both tiles'
-  // accumulators fit in tensor memory
-  if (p.nb > p.sms && 2 * p.BN <= 512) return run<KMAX, 2>(a, mA, mB, mL, p, s);
+  // accumulators fit in tensor memory, their epilogue in the ring budget and
+  // the ring in shared memory
+  if (p.nb > p.sms && 2 * p.BN <= 512 && epilogue_bytes<KMAX, 2>(p, nullptr) <= kRingBudget) {
+    Params q = p;
+    size_t smem = 0;
+    if (plan_ring<KMAX, 2>(q, &smem)) return run<KMAX, 2>(a, mA, mB, mL, p, s);
+  }
   return run<KMAX, 1>(a, mA, mB, mL, p, s);
 }
 

@@ -120,12 +120,14 @@ def test_bf16_router_logit_layouts_and_ragged_tiles(T, d, E, k):
 
 @pytest.mark.parametrize("T,d,E,k", [(19205, 256, 64, 4), (19205, 128, 36, 5), (19205, 64, 12, 3),
                                      (20000, 256, 128, 8), (19205, 128, 64, 16),
-                                     (19205, 64, 256, 6)])
+                                     (19205, 64, 256, 6), (19205, 64, 192, 2), (19205, 128, 192, 4),
+                                     (19205, 64, 224, 8)])
 def test_bf16_router_two_tiles_per_cta(T, d, E, k):
     """More 128-token tiles than SMs (151 or 157 tiles): each CTA routes two
     tiles that share every W_r block of its ring (the last CTA one when the
-    count is odd).  Same checks as above for every way the logits leave the
-    SM and for k up to 16."""
+    count is odd), or one tile where two tiles' staged logits do not fit in
+    shared memory (E >= 192).  Same checks as above for every way the logits
+    leave the SM and for k up to 16."""
     x, wr, shape, packed = _bf16_router_case(T, d, E, k, seed=T + 3 * E)
     ws = moe.workspace(shape)
     logits, idx, gate = moe.route(shape, x.cuda(), packed, None, ws)
