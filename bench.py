@@ -562,7 +562,7 @@ def run_reference(args, rank, world):
 # ------------------------------------------------- one kernel, for profilers
 KERNELS = ("route", "topk", "layout", "permute", "permute_by_token", "grouped",
            "grouped_gather", "combine", "forward", "stats", "capacity", "coselection", "ep_pack",
-           "ep_home")
+           "ep_dispatch_peer", "ep_home")
 
 
 def run_kernel(args):
@@ -583,6 +583,9 @@ def run_kernel(args):
       coselection      moe_coselection_counts (W[e,e'])
       ep_pack          moe_ep_pack (this rank's deduplicated send rows, ep = the
                        workload's EP degree)
+      ep_dispatch_peer moe_ep_dispatch_peer (the same rows stored into one
+                       receive buffer per destination rank, here all on this
+                       GPU: the pack's stores where NVLink would carry them)
       ep_home          moe_ep_home_combine (one returned row per send row)
 
     Routing comes from the workload's own router on its own x; expert
@@ -633,9 +636,18 @@ def run_kernel(args):
     counts = torch.zeros(5, dtype=torch.int64, device=dev)
     cosel = torch.empty((E, E), dtype=torch.int64, device=dev)
     send_rows = int(lay["rank_offsets"][-1]) if ep > 1 else 0
-    if args.kernel in ("ep_pack", "ep_home"):
+    if args.kernel in ("ep_pack", "ep_home", "ep_dispatch_peer"):
         send = moe.ep_pack(shape, x, idx, gate, lay, send_rows) if ep > 1 else None
         y_back = send[0] if send is not None else None
+    if args.kernel == "ep_dispatch_peer":
+        if ep < 2:
+            raise SystemExit("ep_dispatch_peer needs a workload with EP >= 2")
+        rc = [int(v) for v in lay["rank_counts"].tolist()]
+        recv = [(torch.empty((n, w.d), dtype=w.torch_dtype, device=dev),
+                 torch.empty((n, w.k), dtype=torch.int32, device=dev),
+                 torch.empty((n, w.k), dtype=torch.float32, device=dev)) for n in rc]
+        dests = (moe.moe_ep_peer_dest * ep)(*[moe.moe_ep_peer_dest(P(a), P(b), P(c), 0, n)
+                                              for (a, b, c), n in zip(recv, rc)])
     clay = moe._c_layout(moe._layout_tensors(shape, dev))
     clay_ep = moe._c_layout(lay)
     rmap = None
@@ -674,6 +686,9 @@ def run_kernel(args):
         elif k == "ep_pack":
             r = L.moe_ep_pack(ctypes.byref(sc), P(x), P(idx), P(gate), None, ctypes.byref(clay_ep),
                               P(send[0]), P(send[1]), P(send[2]), send_rows, st)
+        elif k == "ep_dispatch_peer":
+            r = L.moe_ep_dispatch_peer(ctypes.byref(sc), P(x), P(idx), P(gate), None,
+                                       ctypes.byref(clay_ep), dests, st)
         elif k == "ep_home":
             r = L.moe_ep_home_combine(ctypes.byref(sc), P(y_back), P(lay["slot_send_row"]),
                                       send_rows, P(out), st)
