@@ -58,18 +58,12 @@ def fused_ffn(w: W.Workload) -> bool:
     return w.dtype == "bf16" and w.f in (64, 128) and w.d in (128, 256)
 
 
-def fused_combine(w: W.Workload) -> bool:
-    """moe_forward sums the combine in the down GEMM's epilogue (CTA pairs,
-    f >= 1536) for these."""
-    return w.dtype == "bf16" and not fused_ffn(w) and w.d % 256 == 0 and w.f >= 1536
-
-
 def launches_per_step(w: W.Workload) -> int:
     if w.dtype != "bf16":
         return 8
     permute = 1 if w.T * w.d * 2 > (96 << 20) else 0
-    # route, scatter, [permute], gate/up [+ down], [combine]
-    return (4 if fused_ffn(w) else 5) + permute - (1 if fused_combine(w) else 0)
+    # route, scatter, [permute], gate/up [+ down], combine
+    return (4 if fused_ffn(w) else 5) + permute
 MEASURED_PEAKS = os.path.join(ROOT, "MEASURED_PEAKS.json")
 
 
@@ -124,11 +118,6 @@ def work(w: W.Workload, T: int):
         out["gate_up"] = dict(bytes=R * w.d * b + 3 * w.E * w.d * w.f * b + R * w.d * b,
                               flops=6 * R * w.d * w.f)
         out["down"] = dict(bytes=0, flops=0)
-    if fused_combine(w):
-        # the down GEMM's epilogue does the combine: its stage moves the
-        # combine's bytes too (y_perm read back, y written)
-        out["down"]["bytes"] += out["combine"]["bytes"]
-        out["combine"] = dict(bytes=0, flops=0)
     return out
 
 

@@ -503,10 +503,7 @@ typedef struct {
  * expert FFN: for f in {64, 128} and d in {128, 256} one kernel for the
  * gate/up GEMM, SwiGLU (H kept on chip) and down GEMM (same arithmetic as
  * the separate GEMMs, so the same y_perm), otherwise the gate/up GEMM with
- * SwiGLU and the down GEMM (on CTA pairs for f >= 1536, where the
- * combine is summed in the down GEMM's epilogue: the last of a token's k
- * rows written for a column tile adds them in slot order, the combine
- * kernel's arithmetic); then the combine.  The permute is
+ * SwiGLU and the down GEMM; then the combine.  The permute is
  * fused into the gate/up operand load (as moe_grouped_swiglu_gather, x_perm
  * not written) while x is at most 96 MB, and a separate token-order permute
  * (moe_permute_by_token) runs otherwise.  fp32: moe_route,

@@ -97,26 +97,6 @@ def test_forward_matches_oracle(cfg, T, ep, placement):
     _check_layout(buf, c.w.E, ep, rmap)
 
 
-def test_fused_combine_equals_the_combine_kernel():
-    """The large workload's forward sums the combine in the down GEMM's
-    epilogue (CTA pairs): its y equals the combine kernel run on the same
-    y_perm, slot rows and gates bit for bit (same fp32 sums in slot order),
-    on two calls in a row (the arrival counters start from zero each call)."""
-    c = Case(5, T=2051)
-    shape = c.shape_ep(16)
-    ws = moe.workspace(shape, forward=True)
-    for _ in range(2):
-        buf = moe.ForwardBuffers(shape)
-        y = moe.forward(shape, c.dx, c.packed, c.dbias, ws, buffers=buf)
-        moe.check_device_status(ws)
-        y2 = moe.combine(shape, buf.y_perm, buf.layout["slot_row"], buf.topk_gate)
-        assert torch.equal(y, y2)
-    # and through the routed forward with unit gates
-    y3 = moe.forward_routed(shape, c.dx, c.packed, buf.topk_idx, None, ws, buffers=buf)
-    moe.check_device_status(ws)
-    assert torch.equal(y3, moe.combine(shape, buf.y_perm, buf.layout["slot_row"], None))
-
-
 def test_forward_two_router_tiles_per_cta():
     """The fine-grained workload at 19205 tokens (151 router tiles, more than
     the SMs): the router's per-tile histograms come from CTAs holding two
