@@ -601,10 +601,11 @@ MOE_API moe_status moe_forward_routed(const moe_shape* shape, const void* x,
  *                            expert another rank holds
  *   send_gate[send_rows, k]  the token's k gates (1 when topk_gate is NULL)
  *  shape: T local tokens, ep = P >= 2; topk_idx / topk_gate [T, k] (device);
- *  expert_rank_host as in moe_dispatch_layout; layout: the send_token and
- *  rank_offsets of moe_dispatch_layout on the same routing and map;
+ *  expert_rank_host as in moe_dispatch_layout; layout: the slot_send_row
+ *  and rank_offsets of moe_dispatch_layout on the same routing and map;
  *  send_rows: rows the send buffers hold (rank_offsets[P], read back, or
- *  any bound; rows past rank_offsets[P] are not written).
+ *  any bound; rows s >= send_rows are not written).  Each token's x row is
+ *  read once and stored into each of its send rows.
  */
 MOE_API moe_status moe_ep_pack(const moe_shape* shape, const void* x, const int32_t* topk_idx,
                                const float* topk_gate, const int32_t* expert_rank_host,

@@ -29,15 +29,20 @@ struct Scratch {
   uint16_t* block_hist;  // per-block histogram rows of the fused router (16-bit counts)
 };
 
+// the lookback status words of the layout; the same bytes hold the
+// per-chunk counts of moe_capacity_keep
+size_t status_bytes(const moe_shape* s) {
+  const size_t nb = (size_t)layout_blocks(s->T), bins = (size_t)layout_bins(s->E, s->ep);
+  return align_up(std::max(nb * bins * 8, capacity_scratch_bytes(s->T, s->k, s->E)));
+}
+
 size_t scratch_bytes(const moe_shape* s) {
   const size_t nb = (size_t)layout_blocks(s->T), bins = (size_t)layout_bins(s->E, s->ep);
   const size_t hs = (size_t)layout_hist_stride((int)nb);
-  return align_up(sizeof(Control)) + kTotalsBytes + align_up(nb * bins * 8) +
-         align_up(hs * bins * 2);
+  return align_up(sizeof(Control)) + kTotalsBytes + status_bytes(s) + align_up(hs * bins * 2);
 }
 
 Scratch carve_scratch(const moe_shape* s, void* ws) {
-  const size_t nb = (size_t)layout_blocks(s->T), bins = (size_t)layout_bins(s->E, s->ep);
   uint8_t* p = static_cast<uint8_t*>(ws);
   Scratch sc;
   sc.ctl = reinterpret_cast<Control*>(p);
@@ -45,7 +50,7 @@ Scratch carve_scratch(const moe_shape* s, void* ws) {
   sc.totals = reinterpret_cast<int32_t*>(p);
   p += kTotalsBytes;
   sc.status = reinterpret_cast<uint64_t*>(p);
-  p += align_up(nb * bins * 8);
+  p += status_bytes(s);
   sc.block_hist = reinterpret_cast<uint16_t*>(p);
   return sc;
 }
@@ -714,8 +719,15 @@ moe_status moe_capacity_keep(const moe_shape* s, const int32_t* topk_idx, const 
   // entries with an out-of-range expert are written by no block: they read 0
   if (cudaMemsetAsync(keep, 0, R * 4, st) != cudaSuccess) return MOE_ERR_CUDA;
   if (kept_gate && cudaMemsetAsync(kept_gate, 0, R * 4, st) != cudaSuccess) return MOE_ERR_CUDA;
-  return cuda_status(launch_capacity_keep(topk_idx, s->T, s->k, s->E, cap, topk_gate, keep,
-                                          kept_gate, carve_scratch(s, ws).ctl, st));
+  // the per-chunk counts borrow the layout's lookback words, which must be
+  // zero again before the next layout on this workspace
+  const Scratch sc = carve_scratch(s, ws);
+  if ((r = cuda_status(launch_capacity_keep(topk_idx, s->T, s->k, s->E, cap, topk_gate, keep,
+                                            kept_gate, reinterpret_cast<int32_t*>(sc.status),
+                                            sc.ctl, st))) != MOE_OK)
+    return r;
+  return cuda_status(
+      cudaMemsetAsync(sc.status, 0, capacity_scratch_bytes(s->T, s->k, s->E), st));
 }
 
 moe_status moe_coselection_counts(const moe_shape* s, const int32_t* topk_idx, uint64_t* counts,
@@ -747,11 +759,11 @@ moe_status moe_ep_pack(const moe_shape* s, const void* x, const int32_t* topk_id
   if (s->ep < 2) return MOE_ERR_INVALID_ARG;
   if (send_rows < 0) return MOE_ERR_INVALID_ARG;
   if (s->T == 0 || send_rows == 0) return MOE_OK;
-  if (!x || !topk_idx || !layout || !layout->send_token || !layout->rank_offsets || !send_x ||
+  if (!x || !topk_idx || !layout || !layout->slot_send_row || !layout->rank_offsets || !send_x ||
       !send_idx || !send_gate)
     return MOE_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(send_x, 16) || !aligned(topk_idx, 4) ||
-      !aligned(layout->send_token, 4) || !aligned(layout->rank_offsets, 4) ||
+      !aligned(layout->slot_send_row, 4) || !aligned(layout->rank_offsets, 4) ||
       !aligned(send_idx, 4) || !aligned(send_gate, 4) || (topk_gate && !aligned(topk_gate, 4)))
     return MOE_ERR_ALIGNMENT;
   RankMap map;
@@ -763,7 +775,7 @@ moe_status moe_ep_pack(const moe_shape* s, const void* x, const int32_t* topk_id
     m.local[e] = (uint8_t)next[map.r[e]]++;
   }
   return cuda_status(launch_ep_pack(s->dtype, x, s->T, s->d, s->k, topk_idx, topk_gate,
-                                    layout->send_token, layout->rank_offsets, s->ep, m, s->E,
+                                    layout->slot_send_row, layout->rank_offsets, s->ep, m, s->E,
                                     send_x, send_idx, send_gate, send_rows, nullptr,
                                     (cudaStream_t)stream));
 }
@@ -793,9 +805,9 @@ moe_status moe_ep_dispatch_peer(const moe_shape* s, const void* x, const int32_t
     cap += d.rows;
   }
   if (s->T == 0 || cap == 0) return MOE_OK;
-  if (!x || !topk_idx || !layout || !layout->send_token || !layout->rank_offsets)
+  if (!x || !topk_idx || !layout || !layout->slot_send_row || !layout->rank_offsets)
     return MOE_ERR_INVALID_ARG;
-  if (!aligned(x, 16) || !aligned(topk_idx, 4) || !aligned(layout->send_token, 4) ||
+  if (!aligned(x, 16) || !aligned(topk_idx, 4) || !aligned(layout->slot_send_row, 4) ||
       !aligned(layout->rank_offsets, 4) || (topk_gate && !aligned(topk_gate, 4)))
     return MOE_ERR_ALIGNMENT;
   RankMap map;
@@ -807,7 +819,7 @@ moe_status moe_ep_dispatch_peer(const moe_shape* s, const void* x, const int32_t
     m.local[e] = (uint8_t)next[map.r[e]]++;
   }
   return cuda_status(launch_ep_pack(s->dtype, x, s->T, s->d, s->k, topk_idx, topk_gate,
-                                    layout->send_token, layout->rank_offsets, s->ep, m, s->E,
+                                    layout->slot_send_row, layout->rank_offsets, s->ep, m, s->E,
                                     nullptr, nullptr, nullptr, cap, &dd, (cudaStream_t)stream));
 }
 

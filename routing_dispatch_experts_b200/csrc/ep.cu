@@ -26,57 +26,111 @@ namespace {
 
 constexpr int kPackWarps = 8;
 
-// one warp per send row s: destination r from rank_offsets (binary search in
-// shared memory), token t = send_token[s].  Row s lands at row s of the send
-// buffers, or, with `dests`, at row dests.d[r].row0 + s - rank_offsets[r] of
-// rank r's receive buffers (the pack and the all-to-all in one pass: plain
-// stores, to another GPU's memory through its peer mapping); rows past
-// dests.d[r].rows are not stored.
+// The distinct send rows of token t, one per destination rank: lane j < k
+// holds slot j's send row; the returned mask has bit j set for the first
+// slot of each distinct, in-range row (the same in every lane).
+__device__ __forceinline__ unsigned distinct_slots(const int32_t* __restrict__ slot_send_row,
+                                                   int64_t t, int k, int64_t total, int lane,
+                                                   int64_t* row_out) {
+  int64_t s = -1;
+  if (lane < k) s = __ldg(slot_send_row + t * k + lane);
+  const bool ok = lane < k && s >= 0 && s < total;
+  const unsigned m = __match_any_sync(0xffffffffu, ok ? (unsigned long long)s
+                                                      : (unsigned long long)(-1 - lane));
+  *row_out = s;
+  return __ballot_sync(0xffffffffu, ok && (__ffs(m) - 1) == lane);
+}
+
+// One warp per token t: its distinct send rows (the distinct values of
+// slot_send_row[t, :]); x[t] is read once, 32 x kPackU vectors at a time,
+// and stored into each of them.  Send row s goes to the rank r with
+// rank_offsets[r] <= s < rank_offsets[r+1] (binary search in shared
+// memory).  It lands at row s of the send buffers (rows s >= cap are not
+// stored) or, with `dests`, at row dests.d[r].row0 + s - rank_offsets[r]
+// of rank r's receive buffers (the pack and the all-to-all in one pass:
+// plain stores, to another GPU's memory through its peer mapping), rows
+// past dests.d[r].rows not stored.
+constexpr int kPackU = 4;
 __global__ void __launch_bounds__(32 * kPackWarps)
     ep_pack_kernel(const uint4* __restrict__ x, int64_t T, int V, int k,
                    const int32_t* __restrict__ idx, const float* __restrict__ gate,
-                   const int32_t* __restrict__ send_token, const int32_t* __restrict__ rank_offsets,
-                   int P, EpMaps maps, int E, int E_loc, uint4* __restrict__ send_x,
-                   int32_t* __restrict__ send_idx, float* __restrict__ send_gate, int64_t cap,
+                   const int32_t* __restrict__ slot_send_row,
+                   const int32_t* __restrict__ rank_offsets, int P, EpMaps maps, int E, int E_loc,
+                   uint4* __restrict__ send_x, int32_t* __restrict__ send_idx,
+                   float* __restrict__ send_gate, int64_t cap,
                    const __grid_constant__ EpDests dests, int use_dests) {
   __shared__ int s_off[257];
   pdl_wait();
   for (int i = threadIdx.x; i <= P; i += blockDim.x) s_off[i] = __ldg(rank_offsets + i);
   __syncthreads();
   const int lane = threadIdx.x & 31;
-  // into send buffers: the first `cap` send rows; into receive buffers: every
-  // send row (the per-destination block bounds apply)
-  const int64_t rows = use_dests ? (int64_t)s_off[P] : min((int64_t)s_off[P], cap);
-  for (int64_t s = (int64_t)blockIdx.x * kPackWarps + (threadIdx.x >> 5); s < rows;
-       s += (int64_t)gridDim.x * kPackWarps) {
-    // last r with s_off[r] <= s
-    int lo = 0, hi = P - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (s_off[mid] <= s) lo = mid; else hi = mid - 1;
-    }
-    const int r = lo;
-    int64_t t = __ldg(send_token + s);
-    if (t < 0 || t >= T) t = 0;
-    const uint4* src = x + t * V;
+  const int64_t total = s_off[P];
+  for (int64_t t = (int64_t)blockIdx.x * kPackWarps + (threadIdx.x >> 5); t < T;
+       t += (int64_t)gridDim.x * kPackWarps) {
+    int64_t s;
+    const unsigned first = distinct_slots(slot_send_row, t, k, total, lane, &s);
+    // lanes holding a distinct row: its rank, its row in the destination
+    // buffers and their base pointers
+    int r = 0;
+    int64_t row = -1;
     uint4* dx = send_x;
     int32_t* di = send_idx;
     float* dg = send_gate;
-    int64_t row = s;
-    if (use_dests) {
-      if (s - s_off[r] >= dests.d[r].rows) continue;  // warp-uniform
-      dx = static_cast<uint4*>(dests.d[r].recv_x);
-      di = dests.d[r].recv_idx;
-      dg = dests.d[r].recv_gate;
-      row = dests.d[r].row0 + (s - s_off[r]);
+    if ((first >> lane) & 1u) {
+      int lo = 0, hi = P - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_off[mid] <= s) lo = mid; else hi = mid - 1;
+      }
+      r = lo;
+      if (use_dests) {
+        const int64_t rel = s - s_off[r];
+        if (rel < dests.d[r].rows) row = dests.d[r].row0 + rel;
+        dx = static_cast<uint4*>(dests.d[r].recv_x);
+        di = dests.d[r].recv_idx;
+        dg = dests.d[r].recv_gate;
+      } else if (s < cap) {
+        row = s;
+      }
     }
-    uint4* dst = dx + row * V;
-    for (int v = lane; v < V; v += 32) dst[v] = __ldg(src + v);
-    if (lane < k) {
-      const int e = __ldg(idx + t * k + lane);
-      const bool here = e >= 0 && e < E && maps.rank[e] == r;
-      di[row * k + lane] = here ? (int)maps.local[e] : E_loc;
-      dg[row * k + lane] = gate ? __ldg(gate + t * k + lane) : 1.f;
+    const unsigned dm = __ballot_sync(0xffffffffu, row >= 0);
+    if (dm == 0) continue;  // warp-uniform
+    // the k local expert ids and gates of every stored row
+    const int e = lane < k ? __ldg(idx + t * k + lane) : -1;
+    const float g = lane < k ? (gate ? __ldg(gate + t * k + lane) : 1.f) : 0.f;
+    for (unsigned b = dm; b; b &= b - 1) {
+      const int d = __ffs(b) - 1;
+      const int rd = __shfl_sync(0xffffffffu, r, d);
+      const int64_t rowd = __shfl_sync(0xffffffffu, row, d);
+      int32_t* dix = reinterpret_cast<int32_t*>(
+          __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(di), d));
+      float* dgx = reinterpret_cast<float*>(
+          __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(dg), d));
+      if (lane < k) {
+        const bool here = e >= 0 && e < E && maps.rank[e] == rd;
+        dix[rowd * k + lane] = here ? (int)maps.local[e] : E_loc;
+        dgx[rowd * k + lane] = g;
+      }
+    }
+    // this lane's destination row starts (lane d holds distinct row d's)
+    uint4* dst_row = row >= 0 ? dx + row * V : nullptr;
+    const uint4* src = x + t * V;
+    for (int v0 = 0; v0 < V; v0 += 32 * kPackU) {
+      uint4 q[kPackU];
+#pragma unroll
+      for (int u = 0; u < kPackU; ++u) {
+        const int v = v0 + lane + 32 * u;
+        if (v < V) q[u] = __ldg(src + v);
+      }
+      for (unsigned b = dm; b; b &= b - 1) {
+        uint4* dst = reinterpret_cast<uint4*>(__shfl_sync(
+            0xffffffffu, reinterpret_cast<unsigned long long>(dst_row), __ffs(b) - 1));
+#pragma unroll
+        for (int u = 0; u < kPackU; ++u) {
+          const int v = v0 + lane + 32 * u;
+          if (v < V) dst[v] = q[u];
+        }
+      }
     }
   }
 }
@@ -158,31 +212,55 @@ __global__ void __launch_bounds__(256)
 
 // y[t] = sum, over the distinct send rows of token t in slot order (each
 // destination rank's row counted once), of y_back[row], in fp32, rounded
-// once.  One thread per 16-byte vector of an output row.
+// once.  One warp per token: the distinct rows found once (distinct_slots),
+// then each lane sums kHomeU of the row's vectors, four rows' loads in
+// flight before they are added (in slot order).
+constexpr int kHomeWarps = 8, kHomeU = 4;
 template <typename T>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(32 * kHomeWarps)
     ep_home_combine_kernel(const uint4* __restrict__ y_back, const int32_t* __restrict__ slot_send_row,
                            uint4* __restrict__ y, int64_t Tn, int V, int k, int64_t rows) {
   pdl_wait();
-  const int64_t n = Tn * V;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t t = i / V;
-    const int v = (int)(i - t * V);
-    float a[Acc<T>::N];
+  const int lane = threadIdx.x & 31;
+  for (int64_t t = (int64_t)blockIdx.x * kHomeWarps + (threadIdx.x >> 5); t < Tn;
+       t += (int64_t)gridDim.x * kHomeWarps) {
+    int64_t s;
+    const unsigned dm = distinct_slots(slot_send_row, t, k, rows, lane, &s);
+    for (int v0 = 0; v0 < V; v0 += 32 * kHomeU) {
+      float a[kHomeU][Acc<T>::N];
 #pragma unroll
-    for (int q = 0; q < Acc<T>::N; ++q) a[q] = 0.f;
-    int seen[16];
-    for (int j = 0; j < k; ++j) {
-      int row = __ldg(slot_send_row + t * k + j);
-      bool dup = false;
-      for (int q = 0; q < j; ++q) dup |= seen[q] == row;
-      seen[j] = row;
-      if (dup) continue;
-      if (row < 0 || row >= rows) row = 0;
-      Acc<T>::add(a, __ldg(y_back + (int64_t)row * V + v), 1.f);
+      for (int u = 0; u < kHomeU; ++u)
+#pragma unroll
+        for (int q = 0; q < Acc<T>::N; ++q) a[u][q] = 0.f;
+      unsigned b = dm;
+      while (b) {  // warp-uniform
+        uint4 q[4][kHomeU];
+        int n = 0;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          const int d = b ? __ffs(b) - 1 : 0;
+          const int64_t row = __shfl_sync(0xffffffffu, s, d);
+          const bool use = b != 0;
+          b &= b - 1;
+          n += use;
+#pragma unroll
+          for (int u = 0; u < kHomeU; ++u) {
+            const int v = v0 + lane + 32 * u;
+            q[w][u] = use && v < V ? __ldg(y_back + row * V + v) : make_uint4(0, 0, 0, 0);
+          }
+        }
+#pragma unroll
+        for (int w = 0; w < 4; ++w)
+          if (w < n)
+#pragma unroll
+            for (int u = 0; u < kHomeU; ++u) Acc<T>::add(a[u], q[w][u], 1.f);
+      }
+#pragma unroll
+      for (int u = 0; u < kHomeU; ++u) {
+        const int v = v0 + lane + 32 * u;
+        if (v < V) y[t * V + v] = Acc<T>::pack(a[u]);
+      }
     }
-    y[i] = Acc<T>::pack(a);
   }
 }
 
@@ -228,17 +306,17 @@ __global__ void ep_signal_wait_kernel(const __grid_constant__ EpFlags fl, int me
 }  // namespace
 
 cudaError_t launch_ep_pack(int dtype, const void* x, int64_t T, int d, int k, const int32_t* idx,
-                           const float* gate, const int32_t* send_token,
+                           const float* gate, const int32_t* slot_send_row,
                            const int32_t* rank_offsets, int P, const EpMaps& maps, int E,
                            void* send_x, int32_t* send_idx, float* send_gate, int64_t cap,
                            const EpDests* dests, cudaStream_t s) {
   if (T == 0 || cap == 0) return cudaSuccess;
   const int V = d * (dtype == MOE_BF16 ? 2 : 4) / 16;
-  const int grid = std::max(1, grid_for(cap, kPackWarps));
+  const int grid = std::max(1, grid_for(T, kPackWarps));
   EpDests dd{};
   if (dests) dd = *dests;
   return launch_pdl(ep_pack_kernel, dim3(grid), dim3(32 * kPackWarps), 0, s,
-                    static_cast<const uint4*>(x), T, V, k, idx, gate, send_token, rank_offsets, P,
+                    static_cast<const uint4*>(x), T, V, k, idx, gate, slot_send_row, rank_offsets, P,
                     maps, E, E / P, static_cast<uint4*>(send_x), send_idx, send_gate, cap, dd,
                     dests ? 1 : 0);
 }
@@ -266,12 +344,12 @@ cudaError_t launch_ep_home_combine(int dtype, const void* y_back, const int32_t*
                                    void* y, int64_t T, int d, int k, int64_t rows, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
   const int V = d * (dtype == MOE_BF16 ? 2 : 4) / 16;
-  const int grid = grid_for(T * V, 256);
+  const int grid = std::max(1, grid_for(T, kHomeWarps));
   if (dtype == MOE_BF16)
-    return launch_pdl(ep_home_combine_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s,
-                      static_cast<const uint4*>(y_back), slot_send_row, static_cast<uint4*>(y), T, V,
-                      k, rows);
-  return launch_pdl(ep_home_combine_kernel<float>, dim3(grid), dim3(256), 0, s,
+    return launch_pdl(ep_home_combine_kernel<__nv_bfloat16>, dim3(grid), dim3(32 * kHomeWarps), 0,
+                      s, static_cast<const uint4*>(y_back), slot_send_row, static_cast<uint4*>(y), T,
+                      V, k, rows);
+  return launch_pdl(ep_home_combine_kernel<float>, dim3(grid), dim3(32 * kHomeWarps), 0, s,
                     static_cast<const uint4*>(y_back), slot_send_row, static_cast<uint4*>(y), T, V, k,
                     rows);
 }

@@ -200,9 +200,11 @@ cudaError_t launch_router_stats(const float* logits, const float* sel_bias, int6
 // expert in (choice rank, token) order, else 0; kept_gate[a] = gate[a] (1
 // when gate is NULL) where kept, 0 where dropped (may be NULL).  Entries of
 // out-of-range indices are not written (MOE_ERR_DEVICE_INDEX in ctl).
+// H: capacity_scratch_bytes(T, k, E) of scratch (per-chunk counts).
+size_t capacity_scratch_bytes(int64_t T, int k, int E);
 cudaError_t launch_capacity_keep(const int32_t* idx, int64_t T, int k, int E, int64_t cap,
-                                 const float* gate, int32_t* keep, float* kept_gate, Control* ctl,
-                                 cudaStream_t s);
+                                 const float* gate, int32_t* keep, float* kept_gate, int32_t* H,
+                                 Control* ctl, cudaStream_t s);
 
 // ---- placement.cu
 // W[e * E + e'] = ordered slot pairs (a != b) of a token with experts
@@ -244,7 +246,7 @@ struct EpReturns {
 };
 // dests NULL: rows into send_x / send_idx / send_gate
 cudaError_t launch_ep_pack(int dtype, const void* x, int64_t T, int d, int k, const int32_t* idx,
-                           const float* gate, const int32_t* send_token,
+                           const float* gate, const int32_t* slot_send_row,
                            const int32_t* rank_offsets, int P, const EpMaps& maps, int E,
                            void* send_x, int32_t* send_idx, float* send_gate, int64_t cap,
                            const EpDests* dests, cudaStream_t s);

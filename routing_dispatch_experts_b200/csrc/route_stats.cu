@@ -123,106 +123,104 @@ __global__ void __launch_bounds__(32 * kStatsWarps)
   if (blockIdx.x == 0 && threadIdx.x == 0) counts[0] = (unsigned long long)T;
 }
 
-// Capacity: one block per expert e.  The expert serves its assignments in
-// priority order -- every token's first choice before any token's second
-// choice (choice rank j ascending), tokens in order within a rank -- and
-// keeps the first `cap`.  Pass 1 counts e's assignments in each choice
-// column; pass 2 walks the tokens in chunks and ranks, for each column j,
-// the chunk's assignments to e with a block-wide prefix count.  The routing
-// is read token-major (coalesced) and staged in shared memory per chunk.
-constexpr int kCapThreads = 256;
+// Capacity: every expert serves its assignments in priority order -- every
+// token's first choice before any token's second choice (choice rank j
+// ascending), tokens in order within a rank -- and keeps the first `cap`.
+// The position of assignment (t, j) to expert e in e's queue is
+//   (assignments to e in the columns before j)
+//   + (tokens before t whose column j holds e),
+// a stable counting sort of each choice column.  Tokens are split into
+// chunks of kCapTok; capacity_hist_kernel counts each chunk's assignments
+// per (column, expert), capacity_rank_kernel turns the counts into each
+// chunk's base per (column, expert) and ranks the chunk's tokens within it
+// (warp match, then per-warp counts scanned in warp order).
+constexpr int kCapTok = 1024;  // tokens per chunk = threads per block
 
-__device__ __forceinline__ int block_excl_scan(int flag, int* warp_sums, int* total) {
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  const unsigned bal = __ballot_sync(0xffffffffu, flag);
-  const int pre = __popc(bal & ((1u << lane) - 1u));
-  if (lane == 0) warp_sums[w] = __popc(bal);
-  __syncthreads();
-  int base = 0, tot = 0;
-#pragma unroll
-  for (int q = 0; q < kCapThreads / 32; ++q) {
-    const int v = warp_sums[q];
-    base += q < w ? v : 0;
-    tot += v;
-  }
-  __syncthreads();  // warp_sums is reused by the next call
-  *total = tot;
-  return base + pre;
-}
-
-__global__ void __launch_bounds__(kCapThreads)
-    capacity_keep_kernel(const int32_t* __restrict__ idx, int64_t T, int k, int E, int64_t cap,
-                         const float* __restrict__ gate, int32_t* __restrict__ keep,
-                         float* __restrict__ kept_gate, Control* ctl) {
-  __shared__ int s_idx[kCapThreads * 16];
-  __shared__ int warp_sums[kCapThreads / 32];
-  __shared__ int col_total[16];
-  const int e = blockIdx.x;
+__global__ void __launch_bounds__(kCapTok)
+    capacity_hist_kernel(const int32_t* __restrict__ idx, int64_t T, int k, int E, int nbc,
+                         int32_t* __restrict__ H, Control* ctl) {
+  __shared__ int hist[16 * 256];
   pdl_wait();
-  // pass 1: assignments to e in each choice column (and, in block 0, the
-  // range check of every index)
-  int cnt[16];
-#pragma unroll
-  for (int j = 0; j < 16; ++j) cnt[j] = 0;
+  for (int i = threadIdx.x; i < k * E; i += kCapTok) hist[i] = 0;
+  __syncthreads();
+  const int64_t t = (int64_t)blockIdx.x * kCapTok + threadIdx.x;
   bool bad = false;
-  for (int64_t t = threadIdx.x; t < T; t += kCapThreads) {
-#pragma unroll
-    for (int j = 0; j < 16; ++j)
-      if (j < k) {
-        const int v = __ldg(idx + t * k + j);
-        cnt[j] += v == e;
-        bad |= v < 0 || v >= E;
-      }
-  }
-  if (e == 0) {  // block-uniform: the whole block takes part in the vote
-    if (__syncthreads_or(bad) && threadIdx.x == 0) record_error(ctl, MOE_ERR_DEVICE_INDEX, 0x900u);
-  }
-  if (threadIdx.x < 16) col_total[threadIdx.x] = 0;
-  __syncthreads();
-#pragma unroll
-  for (int j = 0; j < 16; ++j)
-    if (j < k) {
-      int c = cnt[j];
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(0xffffffffu, c, off);
-      if ((threadIdx.x & 31) == 0 && c) atomicAdd(&col_total[j], c);
+  if (t < T)
+    for (int j = 0; j < k; ++j) {
+      const int e = __ldg(idx + t * k + j);
+      if (e < 0 || e >= E) bad = true;
+      else atomicAdd(&hist[j * E + e], 1);
     }
-  __syncthreads();
-  // kept so far in column j before the current chunk: the columns before j
-  // in full, then column j up to the chunk
-  int64_t before[16];
-  {
-    int64_t acc = 0;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      before[j] = acc;
-      if (j < k) acc += col_total[j];
-    }
-  }
-  // pass 2
-  for (int64_t t0 = 0; t0 < T; t0 += kCapThreads) {
-    const int n = (int)(T - t0 < kCapThreads ? T - t0 : kCapThreads);
-    for (int i = threadIdx.x; i < n * k; i += kCapThreads) s_idx[i] = __ldg(idx + t0 * k + i);
-    __syncthreads();
-    const int r = threadIdx.x;  // token t0 + r
-#pragma unroll
-    for (int j = 0; j < 16; ++j)
-      if (j < k) {
-        const bool mine = r < n && s_idx[r * k + j] == e;
-        int tot;
-        const int pre = block_excl_scan(mine, warp_sums, &tot);
-        if (mine) {
-          const int64_t a = (t0 + r) * k + j;
-          const bool kept = before[j] + pre < cap;
-          keep[a] = kept ? 1 : 0;
-          if (kept_gate) kept_gate[a] = kept ? (gate ? gate[a] : 1.f) : 0.f;
-        }
-        before[j] += tot;
-      }
-    __syncthreads();  // s_idx is refilled next chunk
+  if (__syncthreads_or(bad) && threadIdx.x == 0) record_error(ctl, MOE_ERR_DEVICE_INDEX, 0x900u);
+  // H[j][chunk][e]
+  for (int i = threadIdx.x; i < k * E; i += kCapTok) {
+    const int j = i / E, e = i - j * E;
+    H[((int64_t)j * nbc + blockIdx.x) * E + e] = hist[i];
   }
 }
 
+__global__ void __launch_bounds__(kCapTok)
+    capacity_rank_kernel(const int32_t* __restrict__ idx, int64_t T, int k, int E, int nbc,
+                         const int32_t* __restrict__ H, int64_t cap,
+                         const float* __restrict__ gate, int32_t* __restrict__ keep,
+                         float* __restrict__ kept_gate) {
+  extern __shared__ int cap_smem[];
+  int* base = cap_smem;           // [k][E]: queue position of the chunk's first entry
+  int* wc = cap_smem + k * E;     // [32][E] (first [k][E]: column totals)
+  pdl_wait();
+  const int b = blockIdx.x;
+  for (int i = threadIdx.x; i < k * E; i += kCapTok) {
+    const int j = i / E, e = i - j * E;
+    const int32_t* h = H + (int64_t)j * nbc * E + e;
+    int pre = 0, tot = 0;
+    for (int c = 0; c < nbc; ++c) {
+      const int v = __ldg(h + (int64_t)c * E);
+      pre += c < b ? v : 0;
+      tot += v;
+    }
+    base[i] = pre;
+    wc[i] = tot;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += kCapTok) {
+    int acc = 0;
+    for (int j = 0; j < k; ++j) {
+      base[j * E + e] += acc;
+      acc += wc[j * E + e];
+    }
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int64_t t = (int64_t)b * kCapTok + threadIdx.x;
+  for (int j = 0; j < k; ++j) {
+    for (int i = threadIdx.x; i < 32 * E; i += kCapTok) wc[i] = 0;
+    __syncthreads();
+    int e = -1;
+    if (t < T) e = __ldg(idx + t * k + j);
+    const bool valid = e >= 0 && e < E;
+    // lanes holding the same expert; invalid entries match nobody
+    const unsigned m = __match_any_sync(0xffffffffu, valid ? e : E + lane);
+    const int rank = __popc(m & ((1u << lane) - 1u));
+    if (valid && rank == 0) wc[w * E + e] = __popc(m);
+    __syncthreads();
+    for (int q = threadIdx.x; q < E; q += kCapTok) {  // exclusive scan over warps
+      int acc = 0;
+      for (int ww = 0; ww < 32; ++ww) {
+        const int v = wc[ww * E + q];
+        wc[ww * E + q] = acc;
+        acc += v;
+      }
+    }
+    __syncthreads();
+    if (valid) {
+      const int64_t a = t * k + j;
+      const bool kept = (int64_t)base[j * E + e] + wc[w * E + e] + rank < cap;
+      keep[a] = kept ? 1 : 0;
+      if (kept_gate) kept_gate[a] = kept ? (gate ? gate[a] : 1.f) : 0.f;
+    }
+    __syncthreads();  // wc is cleared for the next column
+  }
+}
 }  // namespace
 
 cudaError_t launch_router_stats(const float* logits, const float* sel_bias, int64_t T, int E,
@@ -250,12 +248,22 @@ cudaError_t launch_router_stats(const float* logits, const float* sel_bias, int6
   }
 }
 
+size_t capacity_scratch_bytes(int64_t T, int k, int E) {
+  return (size_t)k * (size_t)((T + kCapTok - 1) / kCapTok) * (size_t)E * 4;
+}
+
 cudaError_t launch_capacity_keep(const int32_t* idx, int64_t T, int k, int E, int64_t cap,
-                                 const float* gate, int32_t* keep, float* kept_gate, Control* ctl,
-                                 cudaStream_t s) {
+                                 const float* gate, int32_t* keep, float* kept_gate, int32_t* H,
+                                 Control* ctl, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
-  return launch_pdl(capacity_keep_kernel, dim3((unsigned)E), dim3(kCapThreads), 0, s, idx, T, k, E,
-                    cap, gate, keep, kept_gate, ctl);
+  const int nbc = (int)((T + kCapTok - 1) / kCapTok);
+  cudaError_t e = launch_pdl(capacity_hist_kernel, dim3((unsigned)nbc), dim3(kCapTok), 0, s, idx,
+                             T, k, E, nbc, H, ctl);
+  if (e != cudaSuccess) return e;
+  const size_t smem = (size_t)(k + 32) * E * 4;
+  if ((e = set_smem_limit((const void*)capacity_rank_kernel, smem)) != cudaSuccess) return e;
+  return launch_pdl(capacity_rank_kernel, dim3((unsigned)nbc), dim3(kCapTok), smem, s, idx, T, k,
+                    E, nbc, (const int32_t*)H, cap, gate, keep, kept_gate);
 }
 
 }  // namespace moe

@@ -97,11 +97,11 @@ def test_forward_matches_oracle(cfg, T, ep, placement):
     _check_layout(buf, c.w.E, ep, rmap)
 
 
-def test_forward_two_router_tiles_per_cta():
+def test_forward_more_router_tiles_than_sms():
     """The fine-grained workload at 19205 tokens (151 router tiles, more than
-    the SMs): the router's per-tile histograms come from CTAs holding two
-    tiles (the last one a single tile); the whole layout is bit-exact against
-    the oracle's layout of the GPU's routing, and the output matches."""
+    the SMs, so some SMs run two router CTAs): the whole layout built from
+    the router's per-tile histograms is bit-exact against the oracle's
+    layout of the GPU's routing, and the output matches."""
     c = Case(2, T=19205)
     y, buf, shape = _run(c, ep=8)
     _check_layout(buf, c.w.E, 8, None)

@@ -122,12 +122,11 @@ def test_bf16_router_logit_layouts_and_ragged_tiles(T, d, E, k):
                                      (20000, 256, 128, 8), (19205, 128, 64, 16),
                                      (19205, 64, 256, 6), (19205, 64, 192, 2), (19205, 128, 192, 4),
                                      (19205, 64, 224, 8)])
-def test_bf16_router_two_tiles_per_cta(T, d, E, k):
-    """More 128-token tiles than SMs (151 or 157 tiles): each CTA routes two
-    tiles that share every W_r block of its ring (the last CTA one when the
-    count is odd), or one tile where two tiles' staged logits do not fit in
-    shared memory (E >= 192).  Same checks as above for every way the logits
-    leave the SM and for k up to 16."""
+def test_bf16_router_more_tiles_than_sms(T, d, E, k):
+    """More 128-token tiles than SMs (151 or 157 tiles: two CTAs on some
+    SMs, with the ring and the staged logits of each in half the shared
+    memory), up to E = 256 experts.  Same checks as above for every way the
+    logits leave the SM and for k up to 16."""
     x, wr, shape, packed = _bf16_router_case(T, d, E, k, seed=T + 3 * E)
     ws = moe.workspace(shape)
     logits, idx, gate = moe.route(shape, x.cuda(), packed, None, ws)

@@ -174,7 +174,10 @@ def test_router_stats_of_the_forward_routing_with_injected_near_ties():
 
 
 @pytest.mark.parametrize("T,E,k,cf", [(1000, 16, 4, 1.0), (2000, 64, 2, 1.25), (513, 128, 8, 2.0),
-                                      (300, 64, 16, 0.5), (40, 8, 2, 0.1)])
+                                      (300, 64, 16, 0.5), (40, 8, 2, 0.1),
+                                      # several 1024-token chunks, ragged last chunk
+                                      (5000, 128, 8, 1.0), (20001, 64, 4, 1.1),
+                                      (3073, 256, 16, 0.75)])
 def test_capacity_keep_bit_exact(T, E, k, cf):
     # skewed routing so that popular experts overflow their capacity
     g = torch.Generator().manual_seed(T + k)
@@ -194,6 +197,24 @@ def test_capacity_keep_bit_exact(T, E, k, cf):
     # NULL gates: unit gates where kept
     _, kept1, _ = moe.capacity_keep(shape, idx.cuda(), None, cf, ws)
     assert torch.equal(kept1.cpu(), torch.from_numpy(ref).float())
+
+
+def test_layout_after_capacity_on_the_same_workspace():
+    """moe_capacity_keep borrows the layout's lookback words for its
+    per-chunk counts and zeroes them again: a dispatch layout on the same
+    workspace afterwards equals one on a fresh workspace."""
+    T, E, k = 9000, 64, 4
+    g = torch.Generator().manual_seed(7)
+    idx = torch.stack([torch.randperm(E, generator=g)[:k] for _ in range(T)]).int().cuda()
+    shape = moe.Shape(T=T, d=64, E=E, k=k, f=64, ep=8)
+    ws = moe.workspace(shape)
+    moe.capacity_keep(shape, idx, None, 1.0, ws)
+    lay = moe.dispatch_layout(shape, idx, ws)
+    assert moe.get_device_status(ws) == moe.MOE_OK
+    ref = moe.dispatch_layout(shape, idx, moe.workspace(shape))
+    for name in ("expert_counts", "expert_offsets", "row_token", "slot_row", "rank_counts",
+                 "rank_offsets", "send_token", "slot_send_row"):
+        assert torch.equal(lay[name], ref[name]), name
 
 
 def test_capacity_forward_matches_oracle():
