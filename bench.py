@@ -550,7 +550,8 @@ def run_reference(args, rank, world):
 
 # ------------------------------------------------- one kernel, for profilers
 KERNELS = ("route", "topk", "layout", "permute", "permute_by_token", "grouped",
-           "grouped_gather", "combine", "forward", "stats", "capacity", "coselection", "ep_pack",
+           "grouped_gather", "combine", "forward", "forward_combine_in_down", "stats", "capacity",
+           "coselection", "ep_pack",
            "ep_dispatch_peer", "ep_home")
 
 
@@ -567,6 +568,9 @@ def run_kernel(args):
       grouped_gather   moe_grouped_swiglu_gather
       combine          moe_combine
       forward          moe_forward
+      forward_combine_in_down
+                       moe_debug_forward_options with the combine summed in
+                       the down GEMM's epilogue (the opt-in path)
       stats            moe_router_stats (margin, near-tie count)
       capacity         moe_capacity_keep (capacity factor 1.25)
       coselection      moe_coselection_counts (W[e,e'])
@@ -592,7 +596,8 @@ def run_kernel(args):
     E = args.experts or w.E
     ep = min(w.eps[0], E)
     dev = torch.device("cuda", 0)
-    needs_experts = args.kernel in ("grouped", "grouped_gather", "forward")
+    needs_experts = args.kernel in ("grouped", "grouped_gather", "forward",
+                                    "forward_combine_in_down")
     f = w.f if needs_experts else 64
     shape = moe.Shape(T=T, d=w.d, E=E, k=w.k, f=f, ep=ep, dtype=w.torch_dtype)
     wc = dataclasses.replace(w, E=E) if E != w.E else w
@@ -607,7 +612,7 @@ def run_kernel(args):
 
     packed = moe.pack_weights(shape, W.make_router(wc, args.seed).to(dev), stand_in(E, w.d, f),
                               stand_in(E, w.d, f), stand_in(E, f, w.d))
-    ws = moe.workspace(shape, forward=args.kernel == "forward", device=dev)
+    ws = moe.workspace(shape, forward=args.kernel.startswith("forward"), device=dev)
     logits, idx, gate = moe.route(shape, x, packed, bias, ws)
     lay = moe.dispatch_layout(shape, idx, ws)
     torch.cuda.synchronize()
@@ -684,6 +689,10 @@ def run_kernel(args):
         elif k == "capacity":
             r = L.moe_capacity_keep(ctypes.byref(sc), P(idx), P(gate), 1.25, P(idx2), P(gate2),
                                     None, P(ws), ws.numel(), st)
+        elif k == "forward_combine_in_down":
+            r = L.moe_debug_forward_options(ctypes.byref(sc), P(x), P(packed), P(bias), rmap,
+                                            P(out), None, P(ws), ws.numel(),
+                                            moe.FWD_COMBINE_IN_DOWN, st)
         else:
             r = L.moe_forward(ctypes.byref(sc), P(x), P(packed), P(bias), rmap, P(out), None,
                               P(ws), ws.numel(), st)

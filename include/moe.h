@@ -780,6 +780,26 @@ MOE_API moe_status moe_debug_grouped_swiglu_engine(const moe_shape* shape, const
                                                    moe_stream_t stream);
 
 /*
+ * Test and measurement hook: moe_forward with options.
+ *   MOE_FWD_COMBINE_IN_DOWN  the combine summed in the down GEMM's epilogue
+ *     where that GEMM runs on CTA pairs (bf16, d % 256 == 0, f >= 1536;
+ *     ignored elsewhere): after a tile's rows are stored, a per-(token,
+ *     64-column block) arrival counter is incremented, and the last of a
+ *     token's k arrivals sums the token's k rows of y_perm in slot order
+ *     (fp32, gate-weighted, rounded once: the combine kernel's arithmetic,
+ *     so y is bit-identical).  Measured slower than the separate combine on
+ *     the large workload, so moe_forward does not use it.
+ * Other bits: MOE_ERR_INVALID_ARG.  Arguments otherwise as moe_forward.
+ */
+#define MOE_FWD_COMBINE_IN_DOWN 1
+MOE_API moe_status moe_debug_forward_options(const moe_shape* shape, const void* x,
+                                             const void* packed, const float* bias,
+                                             const int32_t* expert_rank_host, void* y,
+                                             const moe_forward_buffers* buffers, void* ws,
+                                             size_t ws_bytes, int32_t options,
+                                             moe_stream_t stream);
+
+/*
  * moe_dispatch_layout for callers that cannot allocate device memory.
  * The source pages have no counterpart of this call; it exists for callers
  * that may not call cudaMalloc or any other allocator where they call this

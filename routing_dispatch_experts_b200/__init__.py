@@ -100,7 +100,8 @@ SYMBOLS = ("moe_status_string", "moe_scratch_size", "moe_forward_workspace_size"
            "moe_ep_expert_forward", "moe_ep_home_combine", "moe_ep_dispatch_peer",
            "moe_ep_expert_forward_peer", "moe_ep_signal_wait", "moe_debug_ep_signal_wait",
            "moe_get_device_status", "moe_debug_dispatch_layout_stall",
-           "moe_debug_grouped_swiglu_engine", "moe_dispatch_layout_static")
+           "moe_debug_grouped_swiglu_engine", "moe_debug_forward_options",
+           "moe_dispatch_layout_static")
 FORWARD_STAGES = ("route", "layout", "permute", "gate_up", "down", "combine")
 
 
@@ -171,6 +172,8 @@ def lib() -> ctypes.CDLL:
             "moe_dispatch_layout_static": ([S, P, P, ctypes.POINTER(moe_layout), P, P], ctypes.c_int),
             "moe_debug_grouped_swiglu_engine": ([S, P, P, P, P, P, P, P, ctypes.c_size_t,
                                                  ctypes.c_int32, P], ctypes.c_int),
+            "moe_debug_forward_options": ([S, P, P, P, P, P, ctypes.POINTER(moe_forward_buffers),
+                                           P, ctypes.c_size_t, ctypes.c_int32, P], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -652,6 +655,25 @@ def forward(shape: Shape, x, packed, bias, ws, expert_rank=None, y=None,
                              _host_map(shape, expert_rank), _p(y),
                              ctypes.byref(b) if b is not None else None, _p(ws), ws.numel(),
                              _stream(stream)), "moe_forward")
+    return y
+
+
+FWD_COMBINE_IN_DOWN = 1  # moe_debug_forward_options: combine in the down GEMM's epilogue
+
+
+def forward_options(shape: Shape, x, packed, bias, ws, options: int, expert_rank=None, y=None,
+                    buffers: Optional[ForwardBuffers] = None, stream=None):
+    """moe_debug_forward_options: moe_forward with the given option bits."""
+    _forward_args(shape, x, packed, bias, y, buffers)
+    if y is None:
+        y = torch.empty((shape.T, shape.d), dtype=shape.dtype, device=x.device)
+    s = shape.c
+    b = buffers.c if buffers is not None else None
+    _check(lib().moe_debug_forward_options(ctypes.byref(s), _p(x), _p(packed), _p(bias),
+                                           _host_map(shape, expert_rank), _p(y),
+                                           ctypes.byref(b) if b is not None else None, _p(ws),
+                                           ws.numel(), int(options), _stream(stream)),
+           "moe_debug_forward_options")
     return y
 
 

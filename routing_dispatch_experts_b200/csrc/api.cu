@@ -89,7 +89,12 @@ struct FwdBufs {
   void* x_perm;
   void* h;
   void* y_perm;
+  uint32_t* arrive;
 };
+
+// arrival counters of the combine fused into the down GEMM: one per token
+// and 64-column block of d (enough for any N tile width)
+size_t arrive_count(const moe_shape* s) { return (size_t)s->T * (size_t)((s->d + 63) / 64); }
 
 size_t forward_bytes(const moe_shape* s) {
   const size_t R = (size_t)s->T * s->k, es = esize(s->dtype);
@@ -102,6 +107,7 @@ size_t forward_bytes(const moe_shape* s) {
   n += 2 * align_up(R * 4);                     // send_token, slot_send_row
   n += align_up(sizeof(moe_stats));
   n += align_up(R * s->d * es) + align_up(R * s->f * es) + align_up(R * s->d * es);
+  n += align_up(arrive_count(s) * 4);           // fused-combine arrival counters
   return n;
 }
 
@@ -129,6 +135,7 @@ FwdBufs carve_forward(const moe_shape* s, void* ws, const moe_forward_buffers* b
   f.x_perm = take(R * s->d * es);
   f.h = take(R * s->f * es);
   f.y_perm = take(R * s->d * es);
+  f.arrive = static_cast<uint32_t*>(take(arrive_count(s) * 4));
   if (b) {
     if (b->logits) f.logits = b->logits;
     if (b->topk_idx) f.idx = b->topk_idx;
@@ -226,6 +233,16 @@ bool pair_chosen(int epi, const GemmArgs& a) {
   return epi == kEpiBF16 && a.gather == nullptr && a.K >= 24 * 64;
 }
 
+// The combine can be summed in the down GEMM's epilogue when the library
+// runs that GEMM on CTA pairs with 256-column tiles (bf16).
+bool combine_fusable(const moe_shape* s) {
+  if (s->dtype != MOE_BF16 || s->d % 256 != 0 || s->f <= 512) return false;
+  GemmArgs a{};
+  a.K = s->f;
+  a.n_per_group = s->d;
+  return pair_chosen(kEpiBF16, a) && gemm_pair_supported(kEpiBF16, 256, a);
+}
+
 cudaError_t launch_gemm(int epi, int bn, const GemmArgs& a, int engine, cudaStream_t st) {
   bool pair = false;
   switch (engine) {
@@ -239,10 +256,19 @@ cudaError_t launch_gemm(int epi, int bn, const GemmArgs& a, int engine, cudaStre
   return launch_gemm_tc(epi, bn, a, st);
 }
 
+// The combine fused into the down GEMM (CTA pairs only; see GemmArgs).
+struct FusedCombine {
+  void* y = nullptr;
+  const int32_t* row_token = nullptr;
+  const int32_t* slot_row = nullptr;
+  const float* gate = nullptr;
+  uint32_t* arrive = nullptr;
+};
+
 moe_status do_grouped_part(int part, const moe_shape* s, const void* a_rows,
                            const int32_t* gather, const int32_t* offsets, const Packed* pk,
                            void* h, void* y_perm, Control* ctl, cudaStream_t st,
-                           int engine = kEngineAuto) {
+                           int engine = kEngineAuto, const FusedCombine* fc = nullptr) {
   const int64_t R = s->T * (int64_t)s->k;
   if (s->dtype == MOE_F32)
     return cuda_status(launch_grouped_f32_part(part, static_cast<const float*>(a_rows), offsets,
@@ -277,6 +303,15 @@ moe_status do_grouped_part(int part, const moe_shape* s, const void* a_rows,
   a.ld_out = s->d;
   // short K (f <= 512): 128-column tiles, so two CTAs fit per SM
   const int bn = (s->d % 256 == 0 && s->f > 512) ? 256 : (s->d % 128 == 0 ? 128 : 64);
+  if (fc) {
+    a.y = fc->y;
+    a.row_token = fc->row_token;
+    a.slot_row = fc->slot_row;
+    a.gate = fc->gate;
+    a.k = s->k;
+    a.T = s->T;
+    a.arrive = fc->arrive;
+  }
   return cuda_status(launch_gemm(kEpiBF16, bn, a, engine, st));
 }
 
@@ -317,7 +352,8 @@ moe_status forward_impl(const moe_shape* s, const void* x, const void* packed, c
                         const int32_t* expert_rank_host, void* y, const moe_forward_buffers* buffers,
                         void* ws, size_t ws_bytes, cudaStream_t st, cudaEvent_t* ev,
                         bool routed = false, const int32_t* r_idx = nullptr,
-                        const float* r_gate = nullptr, const float* sel_bias = nullptr) {
+                        const float* r_gate = nullptr, const float* sel_bias = nullptr,
+                        int options = 0) {
   moe_status r = check_shape(s);
   if (r != MOE_OK) return r;
   if (!ws) return MOE_ERR_INVALID_ARG;
@@ -441,14 +477,29 @@ moe_status forward_impl(const moe_shape* s, const void* x, const void* packed, c
                              sc.ctl, st)) != MOE_OK)
       return r;
   }
+  // on request, the combine in the down GEMM's epilogue where that GEMM
+  // runs on pairs (measured slower than the separate combine kernel on the
+  // large workload, so not the default)
+  const bool fuse_combine = (options & MOE_FWD_COMBINE_IN_DOWN) && !fused && combine_fusable(s);
   if (!fused) {
     if ((r = mark(4)) != MOE_OK) return r;
+    FusedCombine fc;
+    if (fuse_combine) {
+      fc.y = y;
+      fc.row_token = f.lay.row_token;
+      fc.slot_row = f.lay.slot_row;
+      fc.gate = routed ? r_gate : f.gate;
+      fc.arrive = f.arrive;
+      if ((r = cuda_status(cudaMemsetAsync(f.arrive, 0, arrive_count(s) * 4, st))) != MOE_OK)
+        return r;
+    }
     if ((r = do_grouped_part(1, s, nullptr, nullptr, f.lay.expert_offsets, &pk, f.h, f.y_perm,
-                             sc.ctl, st)) != MOE_OK)
+                             sc.ctl, st, kEngineAuto, fuse_combine ? &fc : nullptr)) != MOE_OK)
       return r;
   }
   if ((r = mark(5)) != MOE_OK) return r;
-  if ((r = cuda_status(launch_combine(s->dtype, f.y_perm, f.lay.slot_row, routed ? r_gate : f.gate,
+  if (!fuse_combine &&
+      (r = cuda_status(launch_combine(s->dtype, f.y_perm, f.lay.slot_row, routed ? r_gate : f.gate,
                                       y, s->T, s->d, s->k, st))) != MOE_OK)
     return r;
   return mark(6);
@@ -1056,6 +1107,15 @@ moe_status moe_forward(const moe_shape* s, const void* x, const void* packed, co
                        void* ws, size_t ws_bytes, moe_stream_t stream) {
   return forward_impl(s, x, packed, bias, expert_rank_host, y, buffers, ws, ws_bytes,
                       (cudaStream_t)stream, nullptr);
+}
+
+moe_status moe_debug_forward_options(const moe_shape* s, const void* x, const void* packed,
+                                     const float* bias, const int32_t* expert_rank_host, void* y,
+                                     const moe_forward_buffers* buffers, void* ws, size_t ws_bytes,
+                                     int32_t options, moe_stream_t stream) {
+  if (options & ~MOE_FWD_COMBINE_IN_DOWN) return MOE_ERR_INVALID_ARG;
+  return forward_impl(s, x, packed, bias, expert_rank_host, y, buffers, ws, ws_bytes,
+                      (cudaStream_t)stream, nullptr, false, nullptr, nullptr, nullptr, options);
 }
 
 moe_status moe_forward_selection_bias(const moe_shape* s, const void* x, const void* packed,

@@ -54,6 +54,14 @@ struct Params {
   void* out;
   int64_t ld_out;
   Control* ctl;
+  // combine fused into the down GEMM's epilogue (see GemmArgs)
+  void* y;
+  const int32_t* row_token;
+  const int32_t* slot_row;
+  const float* gate;
+  int k;
+  int64_t T;
+  uint32_t* arrive;
 };
 
 template <int BN, int EPI>
@@ -385,6 +393,54 @@ __global__ void __launch_bounds__(kThreads, 1)
             *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) +
                                       ((int64_t)my_row0 + r) * p.ld_out + ti.nt * OC + ch * 8) = v;
         }
+        if constexpr (EPI == kEpiBF16 && CPR == 32) {
+          if (p.y) {
+            // The combine: this warp wrote rows q*32 + h*16 .. +15 of the
+            // tile (whole OC-column segments).  One arrival per row on its
+            // token's counter for this N tile, after the stores are visible
+            // device-wide; the k-th arrival sums the token's k row segments
+            // in slot order (their writers fenced before arriving).
+            __threadfence();
+            __syncwarp();  // every lane's stores fenced before any lane arrives
+            const int r = q * 32 + h * 16 + (lane & 15);
+            bool last = false;
+            int tok = 0;
+            if (lane < 16 && r < my_rows) {
+              tok = __ldg(p.row_token + my_row0 + r);
+              tok = (tok >= 0 && tok < p.T) ? tok : 0;
+              const unsigned prev = atomicAdd(p.arrive + (int64_t)tok * n_tiles + ti.nt, 1u);
+              last = prev == (unsigned)(p.k - 1);
+            }
+            unsigned todo = __ballot_sync(0xffffffffu, last);
+            if (todo) __threadfence();
+            while (todo) {
+              const int src = __ffs(todo) - 1;
+              todo &= todo - 1;
+              const int64_t t = __shfl_sync(0xffffffffu, tok, src);
+              float acc[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+              const int64_t col = (int64_t)ti.nt * OC + lane * 8;  // 32 lanes x 8 columns
+              for (int j = 0; j < p.k; ++j) {
+                int64_t row = __ldg(p.slot_row + t * p.k + j);
+                if (row < 0 || row >= p.rows) row = 0;
+                const float g = p.gate ? __ldg(p.gate + t * p.k + j) : 1.f;
+                // written by other CTAs of this grid: read through L2
+                const uint4 v = __ldcg(reinterpret_cast<const uint4*>(
+                    static_cast<const __nv_bfloat16*>(p.out) + row * p.ld_out + col));
+                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  acc[2 * i] = fmaf(g, bf16_lo(w[i]), acc[2 * i]);
+                  acc[2 * i + 1] = fmaf(g, bf16_hi(w[i]), acc[2 * i + 1]);
+                }
+              }
+              *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.y) + t * p.ld_out + col) =
+                  make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                             pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+            }
+          }
+        }
       }
     }
   }
@@ -423,6 +479,13 @@ cudaError_t run(const GemmArgs& a, cudaStream_t s) {
   p.out = a.out;
   p.ld_out = a.ld_out;
   p.ctl = a.ctl;
+  p.y = a.y;
+  p.row_token = a.row_token;
+  p.slot_row = a.slot_row;
+  p.gate = a.gate;
+  p.k = a.k;
+  p.T = a.T;
+  p.arrive = a.arrive;
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;

@@ -129,6 +129,18 @@ struct GemmArgs {
   // then has src_rows rows -- the permute fused into the operand load
   const int32_t* gather = nullptr;
   int64_t src_rows = 0;
+  // combine fused into the epilogue (down GEMM on CTA pairs only): with y
+  // set, the last of a token's k rows to be written for an N tile sums the
+  // token's rows y[t] = sum_j gate[t,j] out[slot_row[t*k+j]] for that tile's
+  // columns (fp32 in ascending j, one rounding: the combine kernel's
+  // arithmetic).  arrive: T x (n_per_group / BN) counters, zero on entry.
+  void* y = nullptr;
+  const int32_t* row_token = nullptr;
+  const int32_t* slot_row = nullptr;
+  const float* gate = nullptr;
+  int k = 0;
+  int64_t T = 0;
+  uint32_t* arrive = nullptr;
 };
 cudaError_t launch_gemm_tc(int epi, int bn, const GemmArgs& a, cudaStream_t s);
 // ---- gemm_pair.cu: the same GEMM on CTA pairs (256-row tiles, tcgen05

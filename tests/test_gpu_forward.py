@@ -97,6 +97,28 @@ def test_forward_matches_oracle(cfg, T, ep, placement):
     _check_layout(buf, c.w.E, ep, rmap)
 
 
+def test_fused_combine_equals_the_combine_kernel():
+    """The combine summed in the down GEMM's epilogue (CTA pairs; an opt-in
+    path of the forward, measured slower than the separate combine kernel
+    on the large workload): its y equals the combine kernel run on the same
+    y_perm, slot rows and gates bit for bit (same fp32 sums in slot order),
+    on two calls in a row (the arrival counters start from zero each call),
+    and equals the default forward's y."""
+    c = Case(5, T=2051)
+    shape = c.shape_ep(16)
+    ws = moe.workspace(shape, forward=True)
+    y0 = moe.forward(shape, c.dx, c.packed, c.dbias, ws)
+    moe.check_device_status(ws)
+    for _ in range(2):
+        buf = moe.ForwardBuffers(shape)
+        y = moe.forward_options(shape, c.dx, c.packed, c.dbias, ws, moe.FWD_COMBINE_IN_DOWN,
+                                buffers=buf)
+        moe.check_device_status(ws)
+        y2 = moe.combine(shape, buf.y_perm, buf.layout["slot_row"], buf.topk_gate)
+        assert torch.equal(y, y2)
+        assert torch.equal(y, y0)
+
+
 def test_forward_more_router_tiles_than_sms():
     """The fine-grained workload at 19205 tokens (151 router tiles, more than
     the SMs, so some SMs run two router CTAs): the whole layout built from
