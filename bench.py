@@ -112,6 +112,10 @@ def work(w: W.Workload, T: int):
         # y_perm read, gates / slot rows read, y written
         "combine": dict(bytes=R * w.d * b + T * w.d * b + 2 * R * 4, flops=0),
     }
+    if w.dtype == "bf16" and T * w.d * b <= (96 << 20):
+        # the gate/up GEMM (or fused FFN) gathers the rows of x itself: no
+        # permute kernel runs, and its bytes are the GEMM's row reads
+        out["permute"] = dict(bytes=0, flops=0)
     if fused_ffn(w):
         # one kernel for the whole expert FFN, timed as the gate/up stage:
         # rows of x read, W_g / W_u / W_d read, y_perm written (h stays on chip)
