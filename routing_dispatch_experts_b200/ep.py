@@ -244,34 +244,41 @@ def forward_peer_emulated(ranks: Sequence[EPRank], xs: Sequence[torch.Tensor]):
 class PeerEPRank(EPRank):
     """One rank of the expert-parallel layer over peer memory (one process
     per GPU, the ranks' GPUs peer-connected): the receive rows, the return
-    rows and the rendezvous flags of every rank live in one symmetric-memory
-    allocation per rank (torch.distributed._symmetric_memory), sized for at
-    most `max_tokens` tokens per rank; every forward takes two rendezvous
-    epochs (after the dispatch stores, after the return stores), which also
-    keep the next forward's stores out of buffers still being read."""
+    rows and the rendezvous flags of every rank live in one buffer per rank,
+    by default a symmetric-memory allocation (torch.distributed.
+    _symmetric_memory) sized for at most `max_tokens` tokens per rank;
+    every forward takes two rendezvous epochs (after the dispatch stores,
+    after the return stores), which also keep the next forward's stores out
+    of buffers still being read.
+
+    `buffers` (a list of every rank's byte buffer, as peer_buffer_bytes
+    sizes them, all addressable from this process) replaces the
+    symmetric-memory allocation: the phases (plan, dispatch, experts,
+    finish) can then be driven for P ranks in one process on one device,
+    in phase order with no rendezvous."""
 
     def __init__(self, shape: Shape, rank: int, expert_rank, packed_router, packed_local,
-                 group=None, max_tokens=None, bias=None):
+                 group=None, max_tokens=None, bias=None, buffers=None):
         super().__init__(shape, rank, expert_rank, packed_router, packed_local, bias)
-        import torch.distributed as dist
-        import torch.distributed._symmetric_memory as symm
-        self.ex = TorchExchange(group)
-        P, d, k = shape.ep, shape.d, shape.k
-        Tm = shape.T if max_tokens is None else int(max_tokens)
-        self.cap_recv = P * Tm            # rows from every source, at most one per token
-        self.cap_send = Tm * min(k, P)    # send rows of this rank's tokens
-        es = torch.tensor([], dtype=shape.dtype).element_size()
-        parts = [("flags", 8 * P), ("recv_x", es * d * self.cap_recv),
-                 ("recv_idx", 4 * k * self.cap_recv), ("recv_gate", 4 * k * self.cap_recv),
-                 ("y_back", es * d * self.cap_send)]
-        self.off, n = {}, 0
-        for name, b in parts:
-            self.off[name] = n
-            n += (b + 255) // 256 * 256
-        self.buf = symm.empty(n, dtype=torch.uint8, device=packed_router.device)
-        self.buf.zero_()
-        self.hdl = symm.rendezvous(self.buf, group if group is not None else dist.group.WORLD)
-        self.views = [self._views(self.hdl.get_buffer(q, (n,), torch.uint8)) for q in range(P)]
+        P = shape.ep
+        self.max_tokens = shape.T if max_tokens is None else int(max_tokens)
+        self.off, n = _peer_layout(shape, self.max_tokens)
+        self.cap_recv = P * self.max_tokens      # rows from every source, one per token at most
+        self.cap_send = self.max_tokens * min(shape.k, P)  # send rows of this rank's tokens
+        if buffers is None:
+            import torch.distributed as dist
+            import torch.distributed._symmetric_memory as symm
+            self.ex = TorchExchange(group)
+            self.buf = symm.empty(n, dtype=torch.uint8, device=packed_router.device)
+            self.buf.zero_()
+            self.hdl = symm.rendezvous(self.buf, group if group is not None else dist.group.WORLD)
+            bufs = [self.hdl.get_buffer(q, (n,), torch.uint8) for q in range(P)]
+        else:
+            if len(buffers) != P or any(b.numel() < n for b in buffers):
+                raise ValueError(f"buffers: expected {P} byte buffers of >= {n} bytes")
+            self.ex = None
+            bufs = list(buffers)
+        self.views = [self._views(b) for b in bufs]
         self.epoch = 0
 
     def _views(self, b):
@@ -293,30 +300,81 @@ class PeerEPRank(EPRank):
         self.epoch += 1
         ep_signal_wait([v["flags"] for v in self.views], self.rank, self.epoch, self.ws)
 
-    def forward(self, x, ex=None):
-        """The whole forward of this rank (every rank calls it with its own
-        tokens); raises if a rendezvous timed out."""
-        P = self.shape.ep
-        plan = self.plan(x)
-        counts = self.ex.counts(plan.layout["rank_counts"])
+    # phase 2 (after plan and the count exchange): this rank's send rows
+    # stored straight into every rank's receive rows
+    def dispatch(self, x, plan: Plan, counts: List[List[int]]):
         plan.counts = counts
-        dests, rets = peer_blocks(counts, self.rank)
+        dests, _ = peer_blocks(counts, self.rank)
         V = self.views
         ep_dispatch_peer(self.shape, x, plan.idx, plan.gate, plan.layout,
                          [(V[r]["recv_x"], V[r]["recv_idx"], V[r]["recv_gate"]) + dests[r]
-                          for r in range(P)], expert_rank=self.expert_rank)
-        self._rendezvous()
+                          for r in range(self.shape.ep)], expert_rank=self.expert_rank)
+
+    # phase 3: this rank's experts over its receive rows, the return rows
+    # stored straight into their sources' return rows
+    def experts_peer(self, plan: Plan):
+        _, rets = peer_blocks(plan.counts, self.rank)
         n_recv = sum(rows for _, rows in rets)
-        me = V[self.rank]
+        me, V = self.views[self.rank], self.views
         rs = dataclasses.replace(self.shape, T=n_recv)
-        ws = ep_expert_workspace(rs, device=x.device)
+        ws = ep_expert_workspace(rs, device=me["recv_x"].device)
         ep_expert_forward_peer(rs, me["recv_x"][:n_recv], me["recv_idx"][:n_recv],
                                me["recv_gate"][:n_recv], self.packed_local,
-                               [(V[q]["y_back"],) + rets[q] for q in range(P)], ws)
+                               [(V[q]["y_back"],) + rets[q] for q in range(self.shape.ep)], ws)
+
+    # phase 4: this rank's outputs from its return rows
+    def finish_peer(self, plan: Plan):
+        n_send = sum(plan.counts[self.rank])
+        return self.finish(plan, self.views[self.rank]["y_back"][:n_send])
+
+    def forward(self, x, ex=None):
+        """The whole forward of this rank (every rank calls it with its own
+        tokens, one process per GPU); raises if a rendezvous timed out."""
+        if self.ex is None:
+            raise RuntimeError("forward needs the symmetric-memory buffers of a process group; "
+                               "with caller buffers drive the phases in order")
+        plan = self.plan(x)
+        counts = self.ex.counts(plan.layout["rank_counts"])
+        self.dispatch(x, plan, counts)
+        self._rendezvous()
+        self.experts_peer(plan)
         self._rendezvous()
         check_device_status(self.ws)
-        n_send = sum(counts[self.rank])
-        return self.finish(plan, me["y_back"][:n_send]), counts
+        return self.finish_peer(plan), counts
+
+
+def _peer_layout(shape: Shape, max_tokens: int):
+    """Byte offsets of the parts of one rank's peer buffer, and its size."""
+    P, d, k = shape.ep, shape.d, shape.k
+    cap_recv, cap_send = P * max_tokens, max_tokens * min(k, P)
+    es = torch.tensor([], dtype=shape.dtype).element_size()
+    parts = [("flags", 8 * P), ("recv_x", es * d * cap_recv), ("recv_idx", 4 * k * cap_recv),
+             ("recv_gate", 4 * k * cap_recv), ("y_back", es * d * cap_send)]
+    off, n = {}, 0
+    for name, b in parts:
+        off[name] = n
+        n += (b + 255) // 256 * 256
+    return off, n
+
+
+def peer_buffer_bytes(shape: Shape, max_tokens: int) -> int:
+    """Bytes of one rank's peer buffer (receive rows, return rows, flags)."""
+    return _peer_layout(shape, max_tokens)[1]
+
+
+def forward_peer_ranks_emulated(ranks: Sequence[PeerEPRank], xs: Sequence[torch.Tensor]):
+    """PeerEPRank's phases for P ranks in one process (caller buffers on one
+    device), in phase order: plans, count matrix, every rank's dispatch,
+    every rank's experts, every rank's finish.  Returns (per-rank outputs,
+    count matrix)."""
+    P = len(ranks)
+    plans = [r.plan(x) for r, x in zip(ranks, xs)]
+    counts = LocalExchange(P).counts([p.layout["rank_counts"] for p in plans])
+    for r, x, p in zip(ranks, xs, plans):
+        r.dispatch(x, p, counts)
+    for r, p in zip(ranks, plans):
+        r.experts_peer(p)
+    return [r.finish_peer(p) for r, p in zip(ranks, plans)], counts
 
 
 def local_experts(expert_rank: Sequence[int], rank: int) -> List[int]:

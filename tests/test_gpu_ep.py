@@ -194,3 +194,28 @@ def test_signal_wait_gives_up_on_a_flag_nothing_sets():
     flags[0][1] = 2
     moe.ep_signal_wait(flags, 0, 2, ws)
     assert moe.get_device_status(ws) == moe.MOE_OK
+
+
+@pytest.mark.parametrize("cfg,T,P,placement", [(3, 4096, 8, "contiguous"), (1, 1024, 4, "contiguous"),
+                                               (2, 2048, 8, "permutation")])
+def test_peer_rank_phases_equal_the_collective_exchange(cfg, T, P, placement):
+    """PeerEPRank's own buffer layout and phases (dispatch, experts, finish)
+    for P ranks on one GPU with caller buffers, driven in phase order (no
+    rendezvous: nothing waits on another kernel): every rank's output
+    bit-identical to the collective path; the buffers sized for more tokens
+    than the ranks hold, and reused for a second forward."""
+    *_, ranks, xs, shape = _setup(cfg, T, P, placement)
+    ys, counts = EP.forward_emulated(ranks, xs)
+    n = EP.peer_buffer_bytes(shape, shape.T + 3)
+    bufs = [torch.full((n,), 0xA5, dtype=torch.uint8, device="cuda") for _ in range(P)]
+    peers = [EP.PeerEPRank(shape, r, rk.expert_rank, rk.packed_router, rk.packed_local,
+                           max_tokens=shape.T + 3, bias=rk.bias, buffers=bufs)
+             for r, rk in enumerate(ranks)]
+    for _ in range(2):
+        yp, counts_p = EP.forward_peer_ranks_emulated(peers, xs)
+        torch.cuda.synchronize()
+        assert counts_p == counts
+        for r in range(P):
+            assert torch.equal(yp[r], ys[r]), r
+    with pytest.raises(RuntimeError):
+        peers[0].forward(xs[0])
