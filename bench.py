@@ -335,6 +335,27 @@ def run_ours(args, rank, world, local):
     # the deduplicated send plan of the measured batch ('Expert Coupling',
     # Table I: GPUs per token, rows removed by deduplication)
     dstats = moe.stats_dict(buf.layout["stats"])
+    # rows on the wire of the measured batch under each EP degree the
+    # workload names: one row per assignment (B), deduplicated under the
+    # contiguous placement (D) and under the correlated placement fitted on
+    # a calibration batch (D+P) ('Expert Coupling', Fig. 7; Table III's
+    # co-selection counts and the greedy fit, both on the GPU)
+    placement_rows = {}
+    if shape.ep > 1 and not args.profile:
+        cal_T = min(T, 4096)
+        cshape = dataclasses.replace(shape, T=cal_T)
+        cws = moe.workspace(cshape, device=dev)
+        cal = W.make_x(w, args.seed, cal_T, stream="calib").to(dev)
+        _, cidx, _ = moe.route(cshape, cal, packed, dbias, cws)
+        co = moe.coselection_counts(cshape, cidx, cws)
+        for P_ in w.eps:
+            s_ = dataclasses.replace(shape, ep=P_)
+            ws_ = moe.workspace(s_, device=dev)
+            for name, m_ in (("D_contiguous", W.contiguous_placement(w.E, P_)),
+                             ("D+P_correlated", moe.fit_placement(w.E, P_, co))):
+                lay_ = moe.dispatch_layout(s_, buf.topk_idx, ws_, expert_rank=m_)
+                placement_rows[f"ep{P_}_{name}"] = moe.stats_dict(lay_["stats"])["rows_sent"]
+                moe.check_device_status(ws_)
     if args.profile:
         return {"profile": True, "ms_per_step": ms, "stage_ms": calls}
 
@@ -454,7 +475,10 @@ def run_ours(args, rank, world, local):
             "gpus_per_token": dstats["rows_sent"] / T,
             "tokens_on_one_rank": dstats["tokens_single_rank"],
             "home_rank_assignment_frac": dstats["home_rank_rows"] / R,
-            "computed_by": "moe_forward's dispatch layout (device statistics)"}
+            "computed_by": "moe_forward's dispatch layout (device statistics)",
+            "rows_sent_by_placement": dict(B_per_assignment=R, **placement_rows),
+            "placement_fit": "greedy correlated fit of co-selection counts of a 4096-token "
+                             "calibration batch (moe_coselection_counts, moe_fit_placement)"}
     result["routing"] = {"near_tie_tokens": rstats["near_tie_tokens"],
                          "near_tie_share": rstats["near_tie_tokens"] / max(T, 1),
                          "near_tie_threshold": 1e-5,
