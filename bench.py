@@ -578,7 +578,8 @@ def run_reference(args, rank, world):
 
 # ------------------------------------------------- one kernel, for profilers
 KERNELS = ("route", "topk", "layout", "permute", "permute_by_token", "grouped",
-           "grouped_gather", "combine", "forward", "forward_combine_in_down", "stats", "capacity",
+           "grouped_gather", "combine", "forward", "forward_routed", "forward_combine_in_down",
+           "stats", "capacity",
            "coselection", "ep_pack",
            "ep_dispatch_peer", "ep_home")
 
@@ -596,6 +597,9 @@ def run_kernel(args):
       grouped_gather   moe_grouped_swiglu_gather
       combine          moe_combine
       forward          moe_forward
+      forward_routed   moe_forward_routed on the router's own routing (a
+                       recorded routing table replayed: layout, experts and
+                       combine, no router)
       forward_combine_in_down
                        moe_debug_forward_options with the combine summed in
                        the down GEMM's epilogue (the opt-in path)
@@ -624,7 +628,7 @@ def run_kernel(args):
     E = args.experts or w.E
     ep = min(w.eps[0], E)
     dev = torch.device("cuda", 0)
-    needs_experts = args.kernel in ("grouped", "grouped_gather", "forward",
+    needs_experts = args.kernel in ("grouped", "grouped_gather", "forward", "forward_routed",
                                     "forward_combine_in_down")
     f = w.f if needs_experts else 64
     shape = moe.Shape(T=T, d=w.d, E=E, k=w.k, f=f, ep=ep, dtype=w.torch_dtype)
@@ -717,6 +721,9 @@ def run_kernel(args):
         elif k == "capacity":
             r = L.moe_capacity_keep(ctypes.byref(sc), P(idx), P(gate), 1.25, P(idx2), P(gate2),
                                     None, P(ws), ws.numel(), st)
+        elif k == "forward_routed":
+            r = L.moe_forward_routed(ctypes.byref(sc), P(x), P(packed), P(idx), P(gate), rmap,
+                                     P(out), None, P(ws), ws.numel(), st)
         elif k == "forward_combine_in_down":
             r = L.moe_debug_forward_options(ctypes.byref(sc), P(x), P(packed), P(bias), rmap,
                                             P(out), None, P(ws), ws.numel(),
