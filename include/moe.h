@@ -44,8 +44,9 @@
  *    bit-identical outputs (no floating-point atomics anywhere).
  *  - Calls on different streams with different workspaces may run
  *    concurrently.  The library's only global state is the scratch of
- *    moe_dispatch_layout_static (see there) and a per-device record of the
- *    kernels' shared-memory limits, kept under a lock.
+ *    moe_dispatch_layout_static (see there), a per-device record of the
+ *    kernels' shared-memory limits and the CTA-pair GEMM's count of resident
+ *    clusters (the last device queried), kept under locks.
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H

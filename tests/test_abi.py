@@ -302,3 +302,12 @@ def test_peer_entry_points_reject_bad_arguments(L):
     assert L.moe_debug_ep_signal_wait(flags, 0, 2, 1, 256, 0, None) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_debug_ep_signal_wait(flags, 0, 2, 1, 256, 2_000_000_000,
                                       None) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_forward_options_reject_unknown_bits(L):
+    """moe_debug_forward_options: only MOE_FWD_COMBINE_IN_DOWN is defined;
+    any other bit is an invalid argument, before any check of the rest."""
+    s = moe.Shape(T=64, d=128, E=8, k=2, f=128).c
+    for bad in (2, 4, 1 << 30, -1):
+        assert L.moe_debug_forward_options(ctypes.byref(s), None, None, None, None, None, None,
+                                           None, 0, bad, None) == moe.MOE_ERR_INVALID_ARG
