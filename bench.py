@@ -581,7 +581,7 @@ KERNELS = ("route", "topk", "layout", "permute", "permute_by_token", "grouped",
            "grouped_gather", "combine", "forward", "forward_routed", "forward_combine_in_down",
            "stats", "capacity",
            "coselection", "ep_pack",
-           "ep_dispatch_peer", "ep_home")
+           "ep_dispatch_peer", "ep_expert", "ep_home", "ep_signal")
 
 
 def run_kernel(args):
@@ -611,7 +611,11 @@ def run_kernel(args):
       ep_dispatch_peer moe_ep_dispatch_peer (the same rows stored into one
                        receive buffer per destination rank, here all on this
                        GPU: the pack's stores where NVLink would carry them)
+      ep_expert        moe_ep_expert_forward of rank 0 on the send rows this
+                       batch sends it (layout over its experts, expert FFN,
+                       partial combine)
       ep_home          moe_ep_home_combine (one returned row per send row)
+      ep_signal        moe_ep_signal_wait of a single rank (its own flag)
 
     Routing comes from the workload's own router on its own x; expert
     weights are seeded N(0, 1/d) stand-ins drawn on the device (values do
@@ -629,7 +633,7 @@ def run_kernel(args):
     ep = min(w.eps[0], E)
     dev = torch.device("cuda", 0)
     needs_experts = args.kernel in ("grouped", "grouped_gather", "forward", "forward_routed",
-                                    "forward_combine_in_down")
+                                    "forward_combine_in_down", "ep_expert")
     f = w.f if needs_experts else 64
     shape = moe.Shape(T=T, d=w.d, E=E, k=w.k, f=f, ep=ep, dtype=w.torch_dtype)
     wc = dataclasses.replace(w, E=E) if E != w.E else w
@@ -662,7 +666,7 @@ def run_kernel(args):
     counts = torch.zeros(5, dtype=torch.int64, device=dev)
     cosel = torch.empty((E, E), dtype=torch.int64, device=dev)
     send_rows = int(lay["rank_offsets"][-1]) if ep > 1 else 0
-    if args.kernel in ("ep_pack", "ep_home", "ep_dispatch_peer"):
+    if args.kernel in ("ep_pack", "ep_home", "ep_dispatch_peer", "ep_expert"):
         send = moe.ep_pack(shape, x, idx, gate, lay, send_rows) if ep > 1 else None
         y_back = send[0] if send is not None else None
     if args.kernel == "ep_dispatch_peer":
@@ -674,6 +678,23 @@ def run_kernel(args):
                  torch.empty((n, w.k), dtype=torch.float32, device=dev)) for n in rc]
         dests = (moe.moe_ep_peer_dest * ep)(*[moe.moe_ep_peer_dest(P(a), P(b), P(c), 0, n)
                                               for (a, b, c), n in zip(recv, rc)])
+    if args.kernel == "ep_expert":
+        if ep < 2:
+            raise SystemExit("ep_expert needs a workload with EP >= 2")
+        n0 = int(lay["rank_offsets"][1])
+        rshape = dataclasses.replace(shape, T=n0)
+        rsc = rshape.c
+        El = E // ep
+        lshape = moe.Shape(T=n0, d=w.d, E=El, k=min(w.k, El), f=f, dtype=w.torch_dtype)
+        packed_local = moe.pack_weights(lshape, None, stand_in(El, w.d, f), stand_in(El, w.d, f),
+                                        stand_in(El, f, w.d))
+        rws = moe.ep_expert_workspace(rshape, device=dev)
+        y_ret = torch.empty((n0, w.d), dtype=w.torch_dtype, device=dev)
+        recv = (send[0][:n0], send[1][:n0].contiguous(), send[2][:n0].contiguous())
+    if args.kernel == "ep_signal":
+        flags1 = torch.zeros(1, dtype=torch.int64, device=dev)
+        fl_arr = (ctypes.c_void_p * 1)(P(flags1))
+        epoch = [0]
     clay = moe._c_layout(moe._layout_tensors(shape, dev))
     clay_ep = moe._c_layout(lay)
     rmap = None
@@ -715,6 +736,12 @@ def run_kernel(args):
         elif k == "ep_dispatch_peer":
             r = L.moe_ep_dispatch_peer(ctypes.byref(sc), P(x), P(idx), P(gate), None,
                                        ctypes.byref(clay_ep), dests, st)
+        elif k == "ep_expert":
+            r = L.moe_ep_expert_forward(ctypes.byref(rsc), P(recv[0]), P(recv[1]), P(recv[2]),
+                                        P(packed_local), P(y_ret), P(rws), rws.numel(), st)
+        elif k == "ep_signal":
+            epoch[0] += 1
+            r = L.moe_ep_signal_wait(fl_arr, 0, 1, epoch[0], P(ws), st)
         elif k == "ep_home":
             r = L.moe_ep_home_combine(ctypes.byref(sc), P(y_back), P(lay["slot_send_row"]),
                                       send_rows, P(out), st)

@@ -170,23 +170,30 @@ struct Acc<float> {
 
 // y_ret[i] = sum over slots j (ascending) of received row i whose expert is
 // held here (local id < E_loc) of gate[i,j] * y_perm[slot_row[i*k + j]], in
-// fp32, rounded once.  One thread per 16-byte vector of an output row.
+// fp32, rounded once.  One warp per received row: lane j < k reads slot j,
+// the local slots form a mask, then each lane sums kPartU of the row's
+// vectors, four slots' loads in flight before they are added in slot order.
 // With `rets`, received row t (from source rank s: rets.base[s] <= t <
 // rets.base[s+1]) is stored at row rets.d[s].row0 + t - rets.base[s] of that
 // source's return buffer instead of row t of y_ret.
+constexpr int kPartWarps = 8, kPartU = 4;
 template <typename T>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(32 * kPartWarps)
     ep_partial_combine_kernel(const uint4* __restrict__ y_perm, const int32_t* __restrict__ slot_row,
                               const int32_t* __restrict__ recv_idx, const float* __restrict__ recv_gate,
                               int E_loc, uint4* __restrict__ y_ret, int64_t Tr, int V, int k,
                               const __grid_constant__ EpReturns rets, int use_rets) {
   pdl_wait();
-  const int64_t n = Tr * V;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t t = i / V;
-    const int v = (int)(i - t * V);
-    uint4* out = y_ret + i;
+  const int lane = threadIdx.x & 31;
+  for (int64_t t = (int64_t)blockIdx.x * kPartWarps + (threadIdx.x >> 5); t < Tr;
+       t += (int64_t)gridDim.x * kPartWarps) {
+    const int e = lane < k ? __ldg(recv_idx + t * k + lane) : -1;
+    const bool loc = lane < k && e >= 0 && e < E_loc;  // else held by another rank
+    int64_t row = loc ? __ldg(slot_row + t * k + lane) : 0;
+    if (row < 0 || row >= Tr * k) row = 0;
+    const float g = loc ? __ldg(recv_gate + t * k + lane) : 0.f;
+    const unsigned lm = __ballot_sync(0xffffffffu, loc);
+    uint4* out = y_ret + t * V;
     if (use_rets) {
       // the source rank of received row t: last s with base[s] <= t
       int lo = 0, hi = rets.P - 1;
@@ -194,19 +201,45 @@ __global__ void __launch_bounds__(256)
         const int mid = (lo + hi + 1) >> 1;
         if (rets.base[mid] <= t) lo = mid; else hi = mid - 1;
       }
-      out = static_cast<uint4*>(rets.d[lo].y_back) + (rets.d[lo].row0 + (t - rets.base[lo])) * V + v;
+      out = static_cast<uint4*>(rets.d[lo].y_back) + (rets.d[lo].row0 + (t - rets.base[lo])) * V;
     }
-    float a[Acc<T>::N];
+    for (int v0 = 0; v0 < V; v0 += 32 * kPartU) {
+      float a[kPartU][Acc<T>::N];
 #pragma unroll
-    for (int q = 0; q < Acc<T>::N; ++q) a[q] = 0.f;
-    for (int j = 0; j < k; ++j) {
-      const int e = __ldg(recv_idx + t * k + j);
-      if (e < 0 || e >= E_loc) continue;  // held by another rank
-      int64_t row = __ldg(slot_row + t * k + j);
-      if (row < 0 || row >= Tr * k) row = 0;
-      Acc<T>::add(a, __ldg(y_perm + row * V + v), __ldg(recv_gate + t * k + j));
+      for (int u = 0; u < kPartU; ++u)
+#pragma unroll
+        for (int q = 0; q < Acc<T>::N; ++q) a[u][q] = 0.f;
+      unsigned b = lm;
+      while (b) {  // warp-uniform
+        uint4 q[4][kPartU];
+        float gw[4];
+        int n = 0;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          const int d = b ? __ffs(b) - 1 : 0;
+          const int64_t rd = __shfl_sync(0xffffffffu, row, d);
+          gw[w] = __shfl_sync(0xffffffffu, g, d);
+          const bool use = b != 0;
+          b &= b - 1;
+          n += use;
+#pragma unroll
+          for (int u = 0; u < kPartU; ++u) {
+            const int v = v0 + lane + 32 * u;
+            q[w][u] = use && v < V ? __ldg(y_perm + rd * V + v) : make_uint4(0, 0, 0, 0);
+          }
+        }
+#pragma unroll
+        for (int w = 0; w < 4; ++w)
+          if (w < n)
+#pragma unroll
+            for (int u = 0; u < kPartU; ++u) Acc<T>::add(a[u], q[w][u], gw[w]);
+      }
+#pragma unroll
+      for (int u = 0; u < kPartU; ++u) {
+        const int v = v0 + lane + 32 * u;
+        if (v < V) out[v] = Acc<T>::pack(a[u]);
+      }
     }
-    *out = Acc<T>::pack(a);
   }
 }
 
@@ -327,15 +360,15 @@ cudaError_t launch_ep_partial_combine(int dtype, const void* y_perm, const int32
                                       cudaStream_t s) {
   if (Tr == 0) return cudaSuccess;
   const int V = d * (dtype == MOE_BF16 ? 2 : 4) / 16;
-  const int grid = grid_for(Tr * V, 256);
+  const int grid = std::max(1, grid_for(Tr, kPartWarps));
   EpReturns rr{};
   if (rets) rr = *rets;
   const int use = rets ? 1 : 0;
   if (dtype == MOE_BF16)
-    return launch_pdl(ep_partial_combine_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s,
-                      static_cast<const uint4*>(y_perm), slot_row, recv_idx, recv_gate, E_loc,
+    return launch_pdl(ep_partial_combine_kernel<__nv_bfloat16>, dim3(grid), dim3(32 * kPartWarps),
+                      0, s, static_cast<const uint4*>(y_perm), slot_row, recv_idx, recv_gate, E_loc,
                       static_cast<uint4*>(y_ret), Tr, V, k, rr, use);
-  return launch_pdl(ep_partial_combine_kernel<float>, dim3(grid), dim3(256), 0, s,
+  return launch_pdl(ep_partial_combine_kernel<float>, dim3(grid), dim3(32 * kPartWarps), 0, s,
                     static_cast<const uint4*>(y_perm), slot_row, recv_idx, recv_gate, E_loc,
                     static_cast<uint4*>(y_ret), Tr, V, k, rr, use);
 }
