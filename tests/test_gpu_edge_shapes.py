@@ -32,8 +32,8 @@ def _inputs(T, d, E, f, dtype, seed):
     (1, 256, 8, 2, 64, "bf16", 1),        # one token
     (3, 128, 4, 2, 128, "bf16", 2),       # fewer tokens than experts, EP 2
     (5, 64, 4, 4, 64, "f32", 1),          # k = E: every expert for every token
-    (64, 8192, 8, 2, 128, "bf16", 4),     # widest bf16 rows (16 KB), fused-FFN f
-    (96, 8192, 8, 2, 1536, "bf16", 1),    # widest bf16 rows, separate GEMMs
+    (64, 8192, 8, 2, 128, "bf16", 4),     # widest bf16 rows (16 KB), short down GEMM
+    (96, 8192, 8, 2, 1536, "bf16", 1),    # widest bf16 rows, down GEMM on CTA pairs
     (40, 4096, 8, 2, 64, "f32", 1),       # widest fp32 rows (16 KB)
     (129, 2048, 16, 16, 192, "bf16", 8),  # top-16, ragged tiles
 ])
