@@ -1,7 +1,8 @@
 """The whole layer (moe_forward) at the edges of its shape range, against
 the oracle: no tokens, one token, a handful of tokens over a few experts,
 the widest rows the boundary accepts (d = 8192 in bf16 and d = 4096 in
-fp32: 16 KB rows), top-16, and f at the fused-FFN boundary.  Routing is
+fp32: 16 KB rows), k = E, and top-16 with f = 192 (64-column gate/up
+blocks).  Routing is
 compared as expert sets (a token whose oracle margin is below 1e-5 may
 differ); outputs within 2e-2 * max|y| (bf16) or 1e-5 (fp32)."""
 import math
