@@ -216,6 +216,76 @@ def config_of(w: W.Workload, world: int) -> dict:
             "parallelism": f"replicas x{world} (tokens sharded, no exchange)"}
 
 
+def exchange_splits(idx, rank_map, P: int, dedup: bool):
+    """Rows one rank sends each of the P ranks for its routing idx [T, k]
+    under an expert -> rank map: one row per assignment (dedup False, the
+    per-expert dispatch B of 'Expert Coupling', Fig. 7) or one row per
+    (token, destination rank) (dedup True, D)."""
+    import numpy as np
+    owner = np.asarray(rank_map, dtype=np.int64)[np.asarray(idx, dtype=np.int64)]
+    if not dedup:
+        return np.bincount(owner.ravel(), minlength=P)[:P].astype(np.int64)
+    hit = np.zeros((owner.shape[0], P), dtype=bool)
+    np.put_along_axis(hit, owner, True, axis=1)
+    return hit.sum(0).astype(np.int64)
+
+
+def time_exchange(send_splits, rank: int, world: int, row_elems: int, dtype, dev, reps: int = 5):
+    """The all-to-all of one dispatch plan across the ranks (row payloads
+    only): every rank's send splits are all-gathered, then the rows move
+    with dist.all_to_all_single; median of `reps` timed calls (CUDA events
+    on the GPU), the slowest rank's.  Returns (ms, rows this rank puts on
+    the wire, i.e. to other ranks)."""
+    import statistics as st
+    import torch.distributed as dist
+    mine = torch.tensor([int(v) for v in send_splits], dtype=torch.int64, device=dev)
+    allc = torch.empty(world * world, dtype=torch.int64, device=dev)
+    dist.all_gather_into_tensor(allc, mine)
+    C = allc.view(world, world).cpu().tolist()
+    send = [int(C[rank][r]) for r in range(world)]
+    recv = [int(C[q][rank]) for q in range(world)]
+    inp = torch.empty((sum(send), row_elems), dtype=dtype, device=dev)
+    out = torch.empty((sum(recv), row_elems), dtype=dtype, device=dev)
+    cuda = dev.type == "cuda"
+    for _ in range(2):
+        dist.all_to_all_single(out, inp, output_split_sizes=recv, input_split_sizes=send)
+    times = []
+    for _ in range(reps):
+        dist.barrier()
+        if cuda:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize(dev)
+            e0.record()
+            dist.all_to_all_single(out, inp, output_split_sizes=recv, input_split_sizes=send)
+            e1.record()
+            torch.cuda.synchronize(dev)
+            times.append(e0.elapsed_time(e1))
+        else:
+            t0 = time.perf_counter()
+            dist.all_to_all_single(out, inp, output_split_sizes=recv, input_split_sizes=send)
+            times.append((time.perf_counter() - t0) * 1e3)
+    ms = max_over_ranks(st.median(times), world)
+    return ms, sum(send) - send[rank]
+
+
+def ep_exchange(idx, contiguous_map, correlated_map, rank: int, world: int, d: int, dtype, dev):
+    """Fig. 7 of 'Expert Coupling' on the ranks of this job (P = world):
+    the dispatch all-to-all of every rank's measured batch one row per
+    assignment (B), deduplicated under contiguous placement (D) and under
+    the correlated placement (D+P)."""
+    out = {"ranks": world, "row_bytes": d * torch.tensor([], dtype=dtype).element_size(),
+           "tokens_per_rank": int(idx.shape[0])}
+    for name, m, dedup in (("B", contiguous_map, False), ("D", contiguous_map, True),
+                           ("D+P", correlated_map, True)):
+        ms, wire = time_exchange(exchange_splits(idx, m, world, dedup), rank, world, d, dtype, dev)
+        wire_max = int(max_over_ranks(float(wire), world))
+        out[name] = {"ms": round(ms, 4), "wire_rows_max_rank": wire_max,
+                     "wire_GB_s_max_rank": round(wire_max * out["row_bytes"] / (ms * 1e-3) / 1e9, 1)}
+    out["timing"] = ("dist.all_to_all_single of the row payloads (NCCL), CUDA events, median of 5, "
+                     "slowest rank; not part of the timed step")
+    return out
+
+
 def replica_seed(base: int, rank: int) -> int:
     """Every replica draws its own tokens (the layer shards by tokens)."""
     return base + rank
@@ -479,6 +549,19 @@ def run_ours(args, rank, world, local):
             "rows_sent_by_placement": dict(B_per_assignment=R, **placement_rows),
             "placement_fit": "greedy correlated fit of co-selection counts of a 4096-token "
                              "calibration batch (moe_coselection_counts, moe_fit_placement)"}
+    if world > 1 and w.E % world == 0:
+        # the exchange the dedup send plan is for, on this job's ranks: the
+        # same calibration batch and router on every rank give the same
+        # correlated placement everywhere
+        cal_T = min(T, 4096)
+        cshape = moe.Shape(T=cal_T, d=w.d, E=w.E, k=w.k, f=w.f, ep=world, dtype=w.torch_dtype)
+        cws = moe.workspace(cshape, device=dev)
+        cal = W.make_x(w, args.seed, cal_T, stream="calib").to(dev)
+        _, cidx, _ = moe.route(cshape, cal, packed, dbias, cws)
+        fit = moe.fit_placement(w.E, world, moe.coselection_counts(cshape, cidx, cws))
+        result["ep_exchange"] = ep_exchange(buf.topk_idx.cpu().numpy(),
+                                            W.contiguous_placement(w.E, world), fit, rank, world,
+                                            w.d, w.torch_dtype, dev)
     result["routing"] = {"near_tie_tokens": rstats["near_tie_tokens"],
                          "near_tie_share": rstats["near_tie_tokens"] / max(T, 1),
                          "near_tie_threshold": 1e-5,
