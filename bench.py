@@ -81,6 +81,9 @@ def peaks():
 # holds the summary); None where no capture of the current kernel exists
 NCU_TRAFFIC = {
     (2, "gate_up"): 14_992_128 + 89_088,  # ffn_fused_kernel<64, 256, gather>
+    # gemm_tc_kernel<256, SwiGLU, gather>: a quarter-size capture (4096 of
+    # 16384 tokens, 16 of 64 experts, same rows per expert) scaled by 4
+    (3, "gate_up"): 4 * (157_184_256 + 13_365_504),
     # gemm_tc_kernel<256, SwiGLU> (one CTA per tile, the forward's gate/up
     # engine on this workload): a quarter-size capture (32 of 128 experts,
     # same rows per expert) scaled by 4
