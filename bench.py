@@ -84,6 +84,10 @@ NCU_TRAFFIC = {
     # gemm_tc_kernel<256, SwiGLU, gather>: a quarter-size capture (4096 of
     # 16384 tokens, 16 of 64 experts, same rows per expert) scaled by 4
     (3, "gate_up"): 4 * (157_184_256 + 13_365_504),
+    # the same kernel on the top-6 workload's quarter case, scaled by 4
+    (4, "gate_up"): 4 * (164_507_136 + 36_571_648),
+    # grouped_f32_kernel<SwiGLU> at the tiny workload's full size
+    (1, "gate_up"): 16_829_440,
     # gemm_tc_kernel<256, SwiGLU> (one CTA per tile, the forward's gate/up
     # engine on this workload): a quarter-size capture (32 of 128 experts,
     # same rows per expert) scaled by 4
