@@ -783,7 +783,7 @@ MOE_API moe_status moe_debug_grouped_swiglu_engine(const moe_shape* shape, const
 /*
  * Test and measurement hook: moe_forward with options.
  *   MOE_FWD_COMBINE_IN_DOWN  the combine summed in the down GEMM's epilogue
- *     where that GEMM runs on CTA pairs (bf16, d % 256 == 0, f >= 1536;
+ *     where that GEMM runs on CTA pairs (bf16, d % 256 == 0, f >= 1024;
  *     ignored elsewhere): after a tile's rows are stored, a per-(token,
  *     64-column block) arrival counter is incremented, and the last of a
  *     token's k arrivals sums the token's k rows of y_perm in slot order

@@ -221,16 +221,16 @@ enum Engine {
   kEnginePairGateUp = 4  // CTA pairs for the gate/up GEMM only
 };
 
-// The library's choice, from full-size measurements on B200 (one flushed
-// call of both GEMMs): CTA pairs pay for the down GEMM with a long K loop
-// (the large workload's f = 1536: -10% per clock; its staged epilogue leaves
-// the one-CTA ring three stages deep), not for the gate/up GEMM (more DRAM
-// re-reads of its operands: 9.06 vs 7.0 GB per large-workload launch) nor
-// for the top-2 workload's GEMMs; the pair's TMA gather4 row gather issues
-// 32 row loads per stage and measured twice as slow as the one-CTA cp.async
-// gather.
+// The library's choice, from full-size measurements on B200 (flushed
+// forwards): CTA pairs pay for the down GEMM once its K loop has 16 or more
+// k-blocks (f = 1536: -10% per clock, its staged epilogue leaving the
+// one-CTA ring three stages deep; f = 1024: the top-2 and top-6 forwards 1-2%
+// faster), not for the gate/up GEMM (more DRAM re-reads of its operands:
+// 9.06 vs 7.0 GB per large-workload launch); the pair's TMA gather4 row
+// gather issues 32 row loads per stage and measured twice as slow as the
+// one-CTA cp.async gather.
 bool pair_chosen(int epi, const GemmArgs& a) {
-  return epi == kEpiBF16 && a.gather == nullptr && a.K >= 24 * 64;
+  return epi == kEpiBF16 && a.gather == nullptr && a.K >= 16 * 64;
 }
 
 // The combine can be summed in the down GEMM's epilogue when the library

@@ -97,15 +97,16 @@ def test_forward_matches_oracle(cfg, T, ep, placement):
     _check_layout(buf, c.w.E, ep, rmap)
 
 
-def test_fused_combine_equals_the_combine_kernel():
+@pytest.mark.parametrize("cfg,T,ep", [(5, 2051, 16), (3, 1030, 8)])
+def test_fused_combine_equals_the_combine_kernel(cfg, T, ep):
     """The combine summed in the down GEMM's epilogue (CTA pairs; an opt-in
     path of the forward, measured slower than the separate combine kernel
     on the large workload): its y equals the combine kernel run on the same
     y_perm, slot rows and gates bit for bit (same fp32 sums in slot order),
     on two calls in a row (the arrival counters start from zero each call),
     and equals the default forward's y."""
-    c = Case(5, T=2051)
-    shape = c.shape_ep(16)
+    c = Case(cfg, T=T)
+    shape = c.shape_ep(ep)
     ws = moe.workspace(shape, forward=True)
     y0 = moe.forward(shape, c.dx, c.packed, c.dbias, ws)
     moe.check_device_status(ws)
