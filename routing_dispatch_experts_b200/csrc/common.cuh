@@ -219,6 +219,14 @@ __device__ __forceinline__ void bulk_store(void* gdst, const void* smem_src, uin
                : "memory");
 }
 
+// 32-byte global store (eight 32-bit words; sm_100).  The address must be
+// 32-byte aligned.
+__device__ __forceinline__ void st_global_v8(void* p, const uint32_t* v) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(v[0]),
+               "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
+}
+
 // order this thread's generic-proxy shared-memory writes before later
 // async-proxy (bulk copy / tensor core) reads of them
 __device__ __forceinline__ void fence_proxy_async_shared() {
