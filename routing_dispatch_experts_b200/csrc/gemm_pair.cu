@@ -254,7 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int brow = ti.g * p.n_per_group + ti.nt * BN + (int)rank * (BN / 2);
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
           const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
-          if (!mbar_wait_bounded_cluster(&empty[s], ph ^ 1, &abort_flag)) {
+          if (!mbar_wait_bounded_cluster(&empty[s], ph ^ 1, &abort_flag, true)) {
             ok = false;
             break;
           }
@@ -277,7 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int tile = cluster; tile < total && ok; tile += nclusters, ++tc) {
         const uint32_t b = tc & 1, tph = (tc >> 1) & 1;
-        if (!mbar_wait_bounded_cluster(&tempty[b], tph ^ 1, &abort_flag)) {
+        if (!mbar_wait_bounded_cluster(&tempty[b], tph ^ 1, &abort_flag, true)) {
           ok = false;
           break;
         }
@@ -285,7 +285,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t d_tmem = tmem_base + b * BN;
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
           const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
-          if (!mbar_wait_bounded_cluster(&full[s], ph, &abort_flag)) {
+          // producer and MMA thread sleep in their waits (mbar_try_wait_sleep)
+          if (!mbar_wait_bounded_cluster(&full[s], ph, &abort_flag, true)) {
             ok = false;
             break;
           }

@@ -296,7 +296,7 @@ __global__ void __launch_bounds__(threads_for<GATHER>(), (ctas_per_sm<BN, STAGED
         const int brow = ti.g * p.n_per_group + ti.nt * BN;
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
           const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
-          if (!mbar_wait_bounded(&empty[s], ph ^ 1, &abort_flag)) {
+          if (!mbar_wait_bounded(&empty[s], ph ^ 1, &abort_flag, true)) {
             ok = false;
             break;
           }
@@ -320,7 +320,7 @@ __global__ void __launch_bounds__(threads_for<GATHER>(), (ctas_per_sm<BN, STAGED
       bool ok = true;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++tc) {
         const uint32_t b = tc & 1, tph = (tc >> 1) & 1;
-        if (!mbar_wait_bounded(&tempty[b], tph ^ 1, &abort_flag)) {
+        if (!mbar_wait_bounded(&tempty[b], tph ^ 1, &abort_flag, !GATHER)) {
           ok = false;
           break;
         }
@@ -328,7 +328,9 @@ __global__ void __launch_bounds__(threads_for<GATHER>(), (ctas_per_sm<BN, STAGED
         const uint32_t d_tmem = tmem_base + b * ACC_STRIDE;
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
           const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
-          if (!mbar_wait_bounded(&full[s], ph, &abort_flag)) {
+          // the TMA-fed loop's waits sleep (mbar_try_wait_sleep); the gather
+          // path's measured no faster that way
+          if (!mbar_wait_bounded(&full[s], ph, &abort_flag, !GATHER)) {
             ok = false;
             break;
           }
