@@ -83,15 +83,15 @@ NCU_TRAFFIC = {
     (2, "gate_up"): 14_992_128 + 89_088,  # ffn_fused_kernel<64, 256, gather>
     # gemm_tc_kernel<256, SwiGLU, gather>: a quarter-size capture (4096 of
     # 16384 tokens, 16 of 64 experts, same rows per expert) scaled by 4
-    (3, "gate_up"): 4 * (157_184_256 + 13_365_504),
+    (3, "gate_up"): 4 * (157_726_720 + 12_316_928),
     # the same kernel on the top-6 workload's quarter case, scaled by 4
-    (4, "gate_up"): 4 * (164_507_136 + 36_571_648),
+    (4, "gate_up"): 4 * (166_735_872 + 37_897_216),
     # grouped_f32_kernel<SwiGLU> at the tiny workload's full size
     (1, "gate_up"): 16_829_440,
     # gemm_tc_kernel<256, SwiGLU> (one CTA per tile, the forward's gate/up
     # engine on this workload): a quarter-size capture (32 of 128 experts,
     # same rows per expert) scaled by 4
-    (5, "gate_up"): 4 * (1_551_803_136 + 197_091_072),
+    (5, "gate_up"): 4 * (1_424_801_792 + 197_288_192),
 }
 
 
