@@ -53,6 +53,8 @@ struct Params {
   int G, K, n_per_group;
   void* out;
   int64_t ld_out;
+  // 1: `out` and the row pitch are 32-byte aligned (32-byte epilogue stores)
+  int out_v8;
   Control* ctl;
   // combine fused into the down GEMM's epilogue (see GemmArgs)
   void* y;
@@ -370,7 +372,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         uint4* o = reinterpret_cast<uint4*>(STAGED ? static_cast<void*>(stg + c * 2)
                                                    : static_cast<void*>(out + c));
-        if (STAGED || valid) {
+        if (!STAGED && valid && p.out_v8) {
+          // whole 32-byte sectors (as in the one-CTA engine)
+          st_global_v8(o, pk);
+          st_global_v8(o + 2, pk + 8);
+        } else if (STAGED || valid) {
 #pragma unroll
           for (int v = 0; v < 4; ++v) o[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
         }
@@ -479,6 +485,7 @@ cudaError_t run(const GemmArgs& a, cudaStream_t s) {
   p.n_per_group = a.n_per_group;
   p.out = a.out;
   p.ld_out = a.ld_out;
+  p.out_v8 = (reinterpret_cast<uintptr_t>(a.out) % 32 == 0) && ((a.ld_out * 2) % 32 == 0);
   p.ctl = a.ctl;
   p.y = a.y;
   p.row_token = a.row_token;
@@ -541,8 +548,12 @@ bool gemm_pair_supported(int epi, int bn, const GemmArgs& a) {
 cudaError_t launch_gemm_pair(int epi, int bn, const GemmArgs& a, cudaStream_t s) {
   if (a.rows == 0) return cudaSuccess;
   if (!gemm_pair_supported(epi, bn, a)) return cudaErrorInvalidValue;
-  // short K loops stage the epilogue (as in gemm_tc.cu)
-  const bool st = a.K / BK <= (epi == kEpiBF16 ? 24 : 8);
+  // The bf16 (down) epilogue is staged only for the combine summed in it
+  // (which needs whole staged rows): with 32-byte stores, the unstaged
+  // epilogue's six ring stages beat the staged one's four on B200 (top-2 /
+  // top-6 forwards 2.6-3% faster, large 1-2%).  A short gate/up K loop
+  // stages, as in gemm_tc.cu.
+  const bool st = epi == kEpiBF16 ? a.y != nullptr : a.K / BK <= 8;
   const bool g = a.gather != nullptr;
   if (epi == kEpiSwiGLU)
     return g ? (st ? run<256, kEpiSwiGLU, true, true>(a, s) : run<256, kEpiSwiGLU, false, true>(a, s))
