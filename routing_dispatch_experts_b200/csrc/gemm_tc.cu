@@ -320,7 +320,7 @@ __global__ void __launch_bounds__(threads_for<GATHER>(), (ctas_per_sm<BN, STAGED
       bool ok = true;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++tc) {
         const uint32_t b = tc & 1, tph = (tc >> 1) & 1;
-        if (!mbar_wait_bounded(&tempty[b], tph ^ 1, &abort_flag, !GATHER)) {
+        if (!mbar_wait_bounded(&tempty[b], tph ^ 1, &abort_flag, true)) {
           ok = false;
           break;
         }
@@ -328,9 +328,9 @@ __global__ void __launch_bounds__(threads_for<GATHER>(), (ctas_per_sm<BN, STAGED
         const uint32_t d_tmem = tmem_base + b * ACC_STRIDE;
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
           const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
-          // the TMA-fed loop's waits sleep (mbar_try_wait_sleep); the gather
-          // path's measured no faster that way
-          if (!mbar_wait_bounded(&full[s], ph, &abort_flag, !GATHER)) {
+          // the MMA thread and the TMA producer sleep in their waits
+          // (mbar_try_wait_sleep); the gather warps spin, which measured faster
+          if (!mbar_wait_bounded(&full[s], ph, &abort_flag, true)) {
             ok = false;
             break;
           }
