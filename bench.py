@@ -83,9 +83,9 @@ NCU_TRAFFIC = {
     (2, "gate_up"): 14_992_128 + 89_088,  # ffn_fused_kernel<64, 256, gather>
     # gemm_tc_kernel<256, SwiGLU, gather>: a quarter-size capture (4096 of
     # 16384 tokens, 16 of 64 experts, same rows per expert) scaled by 4
-    (3, "gate_up"): 4 * (157_726_720 + 12_316_928),
+    (3, "gate_up"): 4 * (157_522_688 + 11_830_272),
     # the same kernel on the top-6 workload's quarter case, scaled by 4
-    (4, "gate_up"): 4 * (166_735_872 + 37_897_216),
+    (4, "gate_up"): 4 * (165_850_880 + 37_479_168),
     # grouped_f32_kernel<SwiGLU> at the tiny workload's full size
     (1, "gate_up"): 16_829_440,
     # gemm_tc_kernel<256, SwiGLU> (one CTA per tile, the forward's gate/up
