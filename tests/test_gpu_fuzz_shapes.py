@@ -1,7 +1,8 @@
 """The whole layer (moe_forward) on seeded random shapes across the
 boundary's range, against the oracle: T from 1 to 3000, d and f multiples
 of 64 (the fused expert FFN where its shapes apply, the separate GEMMs
-with 64- and 128-column gate/up blocks elsewhere), E from 2 to 96 (not only
+with 64- and 128-column gate/up blocks elsewhere, f = 1024 / 1536 for the
+down GEMM on CTA pairs), E from 2 to 96 (not only
 multiples of 16), k up to min(E, 16), every divisor of E as the EP degree
 under contiguous or permuted placement, bf16 and fp32.  Checks: the
 dispatch layout bit-exact against the oracle's layout of the GPU's
@@ -37,9 +38,34 @@ def _shape(seed):
     return T, d, E, k, f, ep, dt, rmap
 
 
+def _shape_long_f(seed):
+    """Expert widths of 1024 and 1536 on rows that are multiples of 256: the
+    down GEMM runs on CTA pairs with ragged groups (bf16), the fp32 path on
+    the CUDA cores."""
+    g = np.random.default_rng(seed)
+    dt = "f32" if g.random() < 0.2 else "bf16"
+    E = int(g.choice([2, 5, 8, 12, 24]))
+    k = int(g.integers(1, min(E, 3) + 1))
+    d = int(g.choice([256, 512]))
+    f = int(g.choice([1024, 1536]))
+    T = int(g.choice([1, 7, 129, 300]))
+    divs = [p for p in range(1, E + 1) if E % p == 0]
+    ep = int(g.choice(divs))
+    return T, d, E, k, f, ep, dt, None
+
+
 @pytest.mark.parametrize("seed", range(64))
 def test_forward_random_shape(seed):
-    T, d, E, k, f, ep, dt, rmap = _shape(1000 + seed)
+    _run(seed, _shape(1000 + seed))
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_forward_random_shape_long_f(seed):
+    _run(seed, _shape_long_f(2000 + seed))
+
+
+def _run(seed, shape_args):
+    T, d, E, k, f, ep, dt, rmap = shape_args
     dtype = torch.bfloat16 if dt == "bf16" else torch.float32
     g = torch.Generator().manual_seed(seed)
     x = torch.randn((T, d), generator=g).to(dtype)
