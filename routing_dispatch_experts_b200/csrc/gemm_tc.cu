@@ -557,10 +557,14 @@ cudaError_t run(const GemmArgs& a, cudaStream_t s) {
 cudaError_t launch_gemm_tc(int epi, int bn, const GemmArgs& a, cudaStream_t s) {
   if (a.rows == 0) return cudaSuccess;
   const bool g = a.gather != nullptr;
-  // short K loops: stage the epilogue through shared memory (see above);
-  // measured on B200: a win up to 24 k-blocks for the down GEMM (d-wide
-  // rows), a loss for the 32-block gate/up GEMM
-  const bool st = a.K / BK <= (epi == kEpiBF16 ? 24 : 8);
+  // short K loops: stage the epilogue through shared memory (see above).
+  // Measured on B200: with 16-byte row stores a win up to 24 k-blocks for
+  // the down GEMM (d-wide rows) and up to 8 for gate/up; with the 32-byte
+  // stores (32-byte aligned outputs) the unstaged epilogue wins from 6
+  // k-blocks up (forwards 1-4% faster with f = 384-1536, 2-7% with d = 384
+  // and 512), staging only pays below (0.6-1.4% at f = 128 and 256)
+  const bool v8 = (reinterpret_cast<uintptr_t>(a.out) % 32 == 0) && ((a.ld_out * 2) % 32 == 0);
+  const bool st = a.K / BK <= (v8 ? 4 : (epi == kEpiBF16 ? 24 : 8));
 #define MOE_GEMM_CASE(EPI, BN)                                                         \
   if (epi == EPI && bn == BN)                                                          \
     return g ? (st ? run<BN, EPI, true, true>(a, s) : run<BN, EPI, true, false>(a, s)) \
